@@ -1,0 +1,174 @@
+/*
+ * sherry.h -- C ABI of the B200 (sm_100a) library for Sherry 3:4-sparse
+ * ternary (1.25-bit) weights: quantise+pack, packed linear, unpack.
+ *
+ * The method (page "Sherry: Hardware-Efficient 1.25-Bit Ternary Quantization
+ * via Fine-grained Sparsification", digest paragraphs on the 3:4 rule, on
+ * greedy Sparse-AbsMean and on inference; page "Sherry, Tequila and Fairies in
+ * Python", section 1.1 Sherry Quantization):
+ *   - in every block of 4 consecutive weights along K exactly one weight is 0
+ *     (the smallest |w|) and the other three are +-1 (their signs);
+ *   - the scale alpha of a domain (a group of `group` weights along K, a row,
+ *     or the whole tensor) is the mean |w| of the kept weights;
+ *   - each block is stored in 5 bits, 1 sign bit + 4 lookup bits (32 states);
+ *   - the layer computes Y = X (T alpha)^T.
+ *
+ * Readings fixed by this library where the pages are silent:
+ *   - the lowest index is zeroed when several |w| tie for the minimum;
+ *   - sign(w) = +1 for w >= 0, -0.0 included;
+ *   - nibble = 4*z + 2*d1 + d2 (z = zero position; p0 < p1 < p2 the kept
+ *     positions; d1 = [s(p1) != s(p0)], d2 = [s(p2) != s(p0)]); sign bit
+ *     G = [s(p0) < 0];
+ *   - alpha = S / D in fp32 with S the adjacent-pairwise fp32 sum of the kept
+ *     |w| over the domain in K order (the domain padded with +0.0 to a power of
+ *     two; the zeroed weight contributes +0.0), D = fp32(L*3/4) for a domain of
+ *     L weights (D = 1 for an empty tensor), one IEEE division, no flush to zero;
+ *   - no bias term.
+ *
+ * PACKED LAYOUT (device memory, row-major planes, little-endian):
+ *   idx    uint32 [N][K/32]  nibble of block j (weights 4j..4j+3 of the word's
+ *                            32) at bits 4j..4j+3
+ *   sgn    uint8  [N][K/32]  bit j = G of block j
+ *   scales float  [num]      per-group [N][K/group], per-channel [N], per-tensor [1]
+ *   => 1.25 bit/weight for idx+sgn, plus 32 bits per scale domain.
+ *
+ * CONVENTIONS
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise; the
+ *     caller allocates (and owns) every buffer.  `stream` is a cudaStream_t
+ *     (NULL = legacy default stream).  Calls are asynchronous on `stream`.
+ *   - Arguments are validated on the host before any launch; on an error
+ *     nothing is launched and nothing is written.
+ *   - Inputs must be finite; non-finite weights or activations give
+ *     unspecified (but memory-safe) results.
+ *   - Shapes: N >= 0, M >= 0 (0 = nothing to do), 32 <= K <= SHERRY_MAX_K,
+ *     K % 32 == 0; per-group needs group > 0, group % 32 == 0, K % group == 0.
+ *   - Alignment: W, X, Y, W_out, scales and sgn 4-byte aligned, idx 16-byte
+ *     aligned (else SHERRY_ERR_ALIGN).
+ *   - Results are deterministic: the same call on the same inputs gives the
+ *     same bits (no float atomics; every reduction has a fixed order).
+ */
+#ifndef SHERRY_H
+#define SHERRY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define SHERRY_OK 0
+#define SHERRY_ERR_NULL 1          /* a required pointer is NULL */
+#define SHERRY_ERR_SHAPE 2         /* bad N, K or M */
+#define SHERRY_ERR_GRANULARITY 3   /* unknown granularity */
+#define SHERRY_ERR_GROUP 4         /* bad group size for per-group */
+#define SHERRY_ERR_DTYPE 5         /* unknown element type */
+#define SHERRY_ERR_ALIGN 6         /* misaligned pointer */
+#define SHERRY_ERR_WORKSPACE 7     /* workspace missing or too small */
+#define SHERRY_ERR_CUDA 8          /* a CUDA call or launch failed (see sherry_last_cuda_error) */
+#define SHERRY_ERR_TIMEOUT 9       /* a bounded device wait gave up */
+#define SHERRY_ERR_UNSUPPORTED 10  /* valid request this build cannot run (e.g. no sm_100 device) */
+
+/* granularity of alpha */
+#define SHERRY_PER_TENSOR 0
+#define SHERRY_PER_CHANNEL 1
+#define SHERRY_PER_GROUP 2
+
+/* element types */
+#define SHERRY_F32 0
+#define SHERRY_BF16 1
+
+/* operations, for sherry_workspace_bytes */
+#define SHERRY_OP_QUANTIZE_PACK 0
+#define SHERRY_OP_LINEAR 1
+#define SHERRY_OP_UNPACK 2
+
+#define SHERRY_MAX_K 262144
+
+/* ---- sizes ------------------------------------------------------------- */
+
+/* bytes of the idx plane, N*K/8 (0 on invalid shape) */
+size_t sherry_idx_bytes(int64_t N, int64_t K);
+/* bytes of the sgn plane, N*K/32 (0 on invalid shape) */
+size_t sherry_sgn_bytes(int64_t N, int64_t K);
+/* number of fp32 scales: N*K/group, N or 1 (-1 on invalid arguments) */
+int64_t sherry_num_scales(int64_t N, int64_t K, int granularity, int group);
+/* device workspace an operation needs (0 = none); pass at least this many
+ * bytes.  The linear's workspace must be zero-filled before its first use and
+ * is left zero-filled by every call that returns SHERRY_OK; calls that share a
+ * workspace must not overlap on the device. */
+size_t sherry_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int granularity, int group);
+
+/* ---- quantise + pack ----------------------------------------------------
+ * Greedy Sparse-AbsMean ("Sherry: ... Fine-grained Sparsification", digest
+ * paragraph on the 3:4 rule and quantisation; "Sherry, Tequila and Fairies in
+ * Python" section 1.1, the N:M quantiser with n=3, m=4 and its granularities).
+ *   W        [N][K] row-major, fp32 or bf16 (w_dtype); read only
+ *   idx,sgn  packed planes (layout above); fully overwritten
+ *   scales   sherry_num_scales(...) floats; fully overwritten
+ *   workspace  sherry_workspace_bytes(SHERRY_OP_QUANTIZE_PACK, 0, N, K, g, group)
+ *            bytes (per-tensor only; NULL/0 otherwise)
+ * Output is bit-identical to the definition above. */
+int sherry_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
+                         uint32_t* idx, uint8_t* sgn, float* scales,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- packed linear -------------------------------------------------------
+ * Y[m][n] = sum_k X[m][k] * t[n][k] * alpha(n,k)  ("Sherry: ..." digest: Y = X T alpha;
+ * inference builds lookup tables from the activations, accumulates, then applies
+ * the scale; "Sherry, Tequila and Fairies in Python" section 1.1: F.linear(x, w)).
+ *   X        bf16 [M][K] row-major (uint16 storage); read only
+ *   idx,sgn,scales  packed weight of shape [N][K] with (granularity, group)
+ *   Y        [M][N] row-major, fp32 or bf16 (y_dtype, round to nearest even);
+ *            fully overwritten
+ *   workspace  sherry_workspace_bytes(SHERRY_OP_LINEAR, M, N, K, g, group) bytes
+ * fp32 accumulation; alpha applied once per group (or row).  M <= 16 runs the
+ * lookup-table decode kernel, larger M the tensor-core (tcgen05) kernel. */
+int sherry_linear(const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                  const uint32_t* idx, const uint8_t* sgn, const float* scales,
+                  int granularity, int group,
+                  void* Y, int y_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* One independent linear of a batch (all pointers device pointers). */
+typedef struct sherry_linear_desc {
+    const uint16_t* X;      /* bf16 [M][K] */
+    const uint32_t* idx;
+    const uint8_t* sgn;
+    const float* scales;
+    void* Y;                /* [M][N], y_dtype of the batch call */
+    int64_t N, K;
+    int32_t granularity, group;
+} sherry_linear_desc;
+
+#define SHERRY_MAX_BATCH 256
+
+/* ---- batched packed linear ----------------------------------------------
+ * `count` independent linears with the same M (1 <= M <= 16) in one launch,
+ * e.g. the projections of a decoder layer stack for one token.  Each desc is
+ * computed exactly as by sherry_linear (bit-identical Y).  `descs` is a HOST
+ * array, read during the call only.  count <= SHERRY_MAX_BATCH.
+ *   workspace  sherry_linear_batched_workspace_bytes(descs, count, M) bytes. */
+int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M, int y_dtype,
+                          void* workspace, size_t workspace_bytes, void* stream);
+size_t sherry_linear_batched_workspace_bytes(const sherry_linear_desc* descs, int count, int64_t M);
+
+/* ---- unpack ----------------------------------------------------------------
+ * Dense bf16 W_out[n][k] = round_to_nearest_even(t[n][k] * alpha(n,k)); the
+ * inverse of the 5-bit code (32 states, "Sherry: ..." digest) times the scale.
+ *   W_out    bf16 [N][K] (uint16 storage); fully overwritten */
+int sherry_unpack(const uint32_t* idx, const uint8_t* sgn, const float* scales,
+                  int64_t N, int64_t K, int granularity, int group,
+                  uint16_t* W_out, void* stream);
+
+/* ---- diagnostics ----------------------------------------------------------- */
+const char* sherry_status_string(int status);
+/* cudaError_t value behind the last SHERRY_ERR_CUDA returned on this thread */
+int sherry_last_cuda_error(void);
+/* library version, e.g. 0x000100 = 0.1.0 */
+int sherry_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SHERRY_H */

@@ -1,0 +1,170 @@
+"""Sherry 3:4-sparse ternary (1.25-bit) weights on B200: quantise+pack, packed
+linear and unpack, every step in the CUDA library ``libsherry.so``.
+
+This module only marshals arguments: torch supplies device memory and the
+current stream, and each call goes straight to one C-ABI entry point
+(include/sherry.h).  There is no CPU or PyTorch fallback: if the library is
+missing or the tensors are not on a CUDA device, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+from . import _abi
+from ._abi import (BF16, F32, PER_CHANNEL, PER_GROUP, PER_TENSOR, SherryError,  # noqa: F401
+                   check, lib)
+
+GRANULARITY = {"per_tensor": PER_TENSOR, "per_channel": PER_CHANNEL, "per_group": PER_GROUP}
+
+
+def _gran(g) -> int:
+    if isinstance(g, str):
+        if g not in GRANULARITY:
+            raise ValueError(f"unsupported granularity {g!r}")
+        return GRANULARITY[g]
+    return int(g)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device=None) -> int:
+    import torch
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device (no CPU fallback)")
+
+
+@dataclass
+class PackedWeight:
+    """Packed planes of one [N,K] weight: idx uint32 [N,K/32] (stored as int32),
+    sgn uint8 [N,K/32], scales float32, plus the scale granularity."""
+    idx: "object"
+    sgn: "object"
+    scales: "object"
+    N: int
+    K: int
+    granularity: int
+    group: int
+
+    def nbytes(self) -> int:
+        return self.idx.numel() * 4 + self.sgn.numel() + self.scales.numel() * 4
+
+
+_ws_cache: dict = {}
+
+
+def workspace(nbytes: int, device, kind: str = "linear") -> "object":
+    """A device scratch buffer of at least ``nbytes``, cached per (device, kind).
+    ``kind="linear"`` buffers are zero-filled when allocated and used by the
+    linear calls only: their split-K ticket counters must start at zero, and
+    every successful call leaves them at zero.  Other kinds hold scratch that
+    the next call overwrites."""
+    import torch
+    if nbytes <= 0:
+        return None
+    key = (str(device), kind)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.zeros(max(nbytes, 1 << 16), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def quantize_pack(W, granularity="per_group", group: int = 128, out: PackedWeight | None = None) -> PackedWeight:
+    """Greedy Sparse-AbsMean 3:4 quantise + 5-bit pack of W [N,K] (fp32 or bf16)."""
+    import torch
+    _require_cuda(W)
+    if W.dim() != 2:
+        raise ValueError("expects a 2D weight")
+    W = W.contiguous()
+    N, K = W.shape
+    g = _gran(granularity)
+    L = lib()
+    ns = L.sherry_num_scales(N, K, g, group)
+    if ns < 0:
+        raise SherryError(_abi.ERR_SHAPE if K % 32 or K < 32 else _abi.ERR_GROUP, "quantize_pack")
+    dt = {torch.float32: F32, torch.bfloat16: BF16}.get(W.dtype)
+    if dt is None:
+        raise SherryError(_abi.ERR_DTYPE, "quantize_pack")
+    if out is None:
+        dev = W.device
+        out = PackedWeight(torch.empty((N, K // 32), dtype=torch.int32, device=dev),
+                           torch.empty((N, K // 32), dtype=torch.uint8, device=dev),
+                           torch.empty((max(ns, 1),), dtype=torch.float32, device=dev), N, K, g, group)
+    wsb = L.sherry_workspace_bytes(_abi.OP_QUANTIZE_PACK, 0, N, K, g, group)
+    ws = workspace(wsb, W.device, "quantize")
+    check(L.sherry_quantize_pack(_ptr(W), dt, N, K, g, group, _ptr(out.idx), _ptr(out.sgn), _ptr(out.scales),
+                                 _ptr(ws), wsb, _stream(W.device)), "quantize_pack")
+    return out
+
+
+def linear(X, P: PackedWeight, out_dtype=None, out=None):
+    """Y [M,N] = X [M,K] (bf16) times the packed weight transposed; fp32 or bf16 Y."""
+    import torch
+    _require_cuda(X)
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise ValueError("X must be a 2D bf16 tensor")
+    X = X.contiguous()
+    M, K = X.shape
+    if K != P.K:
+        raise ValueError("inner dimensions differ")
+    out_dtype = out_dtype or torch.float32
+    yd = {torch.float32: F32, torch.bfloat16: BF16}[out_dtype]
+    if out is None:
+        out = torch.empty((M, P.N), dtype=out_dtype, device=X.device)
+    L = lib()
+    wsb = L.sherry_workspace_bytes(_abi.OP_LINEAR, M, P.N, K, P.granularity, P.group)
+    ws = workspace(wsb, X.device)
+    check(L.sherry_linear(_ptr(X), M, P.N, K, _ptr(P.idx), _ptr(P.sgn), _ptr(P.scales), P.granularity, P.group,
+                          _ptr(out), yd, _ptr(ws), wsb, _stream(X.device)), "linear")
+    return out
+
+
+def make_batch(pairs, outs) -> "ctypes.Array":
+    """Descriptor array for :func:`linear_batched` from (X, PackedWeight) pairs."""
+    arr = (_abi.LinearDesc * len(pairs))()
+    for i, ((X, P), Y) in enumerate(zip(pairs, outs)):
+        arr[i] = _abi.LinearDesc(_ptr(X), _ptr(P.idx), _ptr(P.sgn), _ptr(P.scales), _ptr(Y), P.N, P.K,
+                                 P.granularity, P.group)
+    return arr
+
+
+def linear_batched(pairs, out_dtype=None, outs=None, descs=None):
+    """Independent linears with the same M (<= 16) in one launch."""
+    import torch
+    out_dtype = out_dtype or torch.float32
+    yd = {torch.float32: F32, torch.bfloat16: BF16}[out_dtype]
+    if not pairs:
+        return []
+    M = pairs[0][0].shape[0]
+    for X, P in pairs:
+        _require_cuda(X)
+        if X.dtype != torch.bfloat16 or X.shape[0] != M or X.shape[1] != P.K or not X.is_contiguous():
+            raise ValueError("each X must be contiguous bf16 [M,K] with the same M")
+    if outs is None:
+        outs = [torch.empty((M, P.N), dtype=out_dtype, device=X.device) for X, P in pairs]
+    if descs is None:
+        descs = make_batch(pairs, outs)
+    L = lib()
+    wsb = L.sherry_linear_batched_workspace_bytes(descs, len(pairs), M)
+    ws = workspace(wsb, pairs[0][0].device)
+    check(L.sherry_linear_batched(descs, len(pairs), M, yd, _ptr(ws), wsb, _stream(pairs[0][0].device)),
+          "linear_batched")
+    return outs
+
+
+def unpack(P: PackedWeight, out=None):
+    """Dense bf16 [N,K] = RNE(t * alpha)."""
+    import torch
+    if out is None:
+        out = torch.empty((P.N, P.K), dtype=torch.bfloat16, device=P.idx.device)
+    check(lib().sherry_unpack(_ptr(P.idx), _ptr(P.sgn), _ptr(P.scales), P.N, P.K, P.granularity, P.group,
+                              _ptr(out), _stream(P.idx.device)), "unpack")
+    return out

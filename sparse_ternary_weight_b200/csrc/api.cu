@@ -1,0 +1,199 @@
+// api.cu -- the library's C ABI (declared in include/sherry.h): argument checks
+// on the host, then the launches.  Nothing here allocates device memory.
+#include "common.cuh"
+
+#include <mutex>
+#include <vector>
+
+namespace sherry {
+
+static thread_local int g_last_cuda_error = 0;
+void set_cuda_error(cudaError_t e) { g_last_cuda_error = (int)e; }
+
+// number of SMs of the current device (cached per device)
+static int device_sms() {
+    static std::mutex mu;
+    static std::vector<int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    std::lock_guard<std::mutex> lk(mu);
+    if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+    if (cache[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        cache[dev] = v;
+    }
+    return cache[dev];
+}
+
+static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static int check_shape(int64_t N, int64_t K) {
+    if (N < 0 || K < 32 || K > SHERRY_MAX_K || (K % 32) != 0) return SHERRY_ERR_SHAPE;
+    if (N > (int64_t)0x7fffffff) return SHERRY_ERR_SHAPE;
+    return SHERRY_OK;
+}
+
+static int check_gran(int64_t K, int granularity, int group) {
+    if (granularity == SHERRY_PER_TENSOR || granularity == SHERRY_PER_CHANNEL) return SHERRY_OK;
+    if (granularity != SHERRY_PER_GROUP) return SHERRY_ERR_GRANULARITY;
+    if (group <= 0 || (group % 32) != 0 || (K % group) != 0) return SHERRY_ERR_GROUP;
+    return SHERRY_OK;
+}
+
+static int check_planes(const uint32_t* idx, const uint8_t* sgn, const float* scales, int64_t N) {
+    if (N > 0 && (!idx || !sgn || !scales)) return SHERRY_ERR_NULL;
+    if (!aligned(idx, 16) || !aligned(sgn, 16) || !aligned(scales, 16)) return SHERRY_ERR_ALIGN;
+    return SHERRY_OK;
+}
+
+}  // namespace sherry
+
+using namespace sherry;
+
+extern "C" {
+
+int sherry_version(void) { return 0x000100; }
+
+int sherry_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* sherry_status_string(int status) {
+    switch (status) {
+        case SHERRY_OK: return "ok";
+        case SHERRY_ERR_NULL: return "a required pointer is NULL";
+        case SHERRY_ERR_SHAPE: return "bad shape (need N >= 0, M >= 0, 32 <= K <= SHERRY_MAX_K, K % 32 == 0)";
+        case SHERRY_ERR_GRANULARITY: return "unknown granularity";
+        case SHERRY_ERR_GROUP: return "bad group size (need group > 0, group % 32 == 0, K % group == 0)";
+        case SHERRY_ERR_DTYPE: return "unknown element type";
+        case SHERRY_ERR_ALIGN: return "misaligned pointer (16-byte alignment required)";
+        case SHERRY_ERR_WORKSPACE: return "workspace missing or too small";
+        case SHERRY_ERR_CUDA: return "CUDA error (see sherry_last_cuda_error)";
+        case SHERRY_ERR_TIMEOUT: return "a bounded device wait gave up";
+        case SHERRY_ERR_UNSUPPORTED: return "unsupported on this device or build";
+        default: return "unknown status";
+    }
+}
+
+size_t sherry_idx_bytes(int64_t N, int64_t K) {
+    if (check_shape(N, K)) return 0;
+    return (size_t)(N * (K / 32)) * 4;
+}
+
+size_t sherry_sgn_bytes(int64_t N, int64_t K) {
+    if (check_shape(N, K)) return 0;
+    return (size_t)(N * (K / 32));
+}
+
+int64_t sherry_num_scales(int64_t N, int64_t K, int granularity, int group) {
+    if (check_shape(N, K) || check_gran(K, granularity, group)) return -1;
+    if (granularity == SHERRY_PER_TENSOR) return 1;
+    if (granularity == SHERRY_PER_CHANNEL) return N;
+    return N * (K / group);
+}
+
+size_t sherry_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int granularity, int group) {
+    if (check_shape(N, K) || check_gran(K, granularity, group)) return 0;
+    if (op == SHERRY_OP_QUANTIZE_PACK) return quantize_workspace_bytes(N, K, granularity);
+    if (op == SHERRY_OP_LINEAR) {
+        if (M <= 0 || N == 0) return 0;
+        ProbShape s{N, K, granularity, group};
+        return lut_workspace_bytes(&s, 1, M, device_sms());
+    }
+    return 0;
+}
+
+int sherry_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
+                         uint32_t* idx, uint8_t* sgn, float* scales, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    int st = check_shape(N, K);
+    if (st) return st;
+    if ((st = check_gran(K, granularity, group))) return st;
+    if (w_dtype != SHERRY_F32 && w_dtype != SHERRY_BF16) return SHERRY_ERR_DTYPE;
+    if (!scales || (N > 0 && (!W || !idx || !sgn))) return SHERRY_ERR_NULL;
+    if (!aligned(W, 16) || !aligned(idx, 16) || !aligned(sgn, 16) || !aligned(scales, 16)) return SHERRY_ERR_ALIGN;
+    const size_t need = quantize_workspace_bytes(N, K, granularity);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SHERRY_ERR_WORKSPACE;
+    if (need > 0 && !aligned(workspace, 16)) return SHERRY_ERR_ALIGN;
+    return quantize_pack_launch(W, w_dtype, N, K, granularity, group, idx, sgn, scales, workspace,
+                                static_cast<cudaStream_t>(stream));
+}
+
+int sherry_unpack(const uint32_t* idx, const uint8_t* sgn, const float* scales, int64_t N, int64_t K,
+                  int granularity, int group, uint16_t* W_out, void* stream) {
+    int st = check_shape(N, K);
+    if (st) return st;
+    if ((st = check_gran(K, granularity, group))) return st;
+    if ((st = check_planes(idx, sgn, scales, N))) return st;
+    if (N > 0 && !W_out) return SHERRY_ERR_NULL;
+    if (!aligned(W_out, 16)) return SHERRY_ERR_ALIGN;
+    return unpack_launch(idx, sgn, scales, N, K, granularity, group, W_out, static_cast<cudaStream_t>(stream),
+                         device_sms());
+}
+
+static int check_linear_desc(const sherry_linear_desc& d, int64_t M) {
+    int st = check_shape(d.N, d.K);
+    if (st) return st;
+    if ((st = check_gran(d.K, d.granularity, d.group))) return st;
+    if ((st = check_planes(d.idx, d.sgn, d.scales, d.N))) return st;
+    if (M > 0 && d.N > 0 && (!d.X || !d.Y)) return SHERRY_ERR_NULL;
+    if (!aligned(d.X, 16) || !aligned(d.Y, 16)) return SHERRY_ERR_ALIGN;
+    return SHERRY_OK;
+}
+
+int sherry_linear(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* idx, const uint8_t* sgn,
+                  const float* scales, int granularity, int group, void* Y, int y_dtype, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    if (M < 0 || M > (int64_t)0x7fffffff) return SHERRY_ERR_SHAPE;
+    sherry_linear_desc d{X, idx, sgn, scales, Y, N, K, granularity, group};
+    int st = check_linear_desc(d, M);
+    if (st) return st;
+    if (y_dtype != SHERRY_F32 && y_dtype != SHERRY_BF16) return SHERRY_ERR_DTYPE;
+    if (M == 0 || N == 0) return SHERRY_OK;
+    ProbShape s{N, K, granularity, group};
+    const int sms = device_sms();
+    const size_t need = lut_workspace_bytes(&s, 1, M, sms);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SHERRY_ERR_WORKSPACE;
+    if (need > 0 && !aligned(workspace, 256)) return SHERRY_ERR_ALIGN;
+    return lut_linear_launch(&s, &d, 1, M, y_dtype == SHERRY_BF16, workspace, sms,
+                             static_cast<cudaStream_t>(stream));
+}
+
+static int batch_shapes(const sherry_linear_desc* descs, int count, int64_t M, std::vector<ProbShape>& shapes,
+                        std::vector<sherry_linear_desc>& kept) {
+    if (!descs && count > 0) return SHERRY_ERR_NULL;
+    if (count < 0 || count > SHERRY_MAX_BATCH) return SHERRY_ERR_SHAPE;
+    if (M < 0 || M > 16) return SHERRY_ERR_SHAPE;
+    for (int i = 0; i < count; ++i) {
+        int st = check_linear_desc(descs[i], M);
+        if (st) return st;
+        if (descs[i].N == 0) continue;
+        shapes.push_back(ProbShape{descs[i].N, descs[i].K, descs[i].granularity, descs[i].group});
+        kept.push_back(descs[i]);
+    }
+    return SHERRY_OK;
+}
+
+size_t sherry_linear_batched_workspace_bytes(const sherry_linear_desc* descs, int count, int64_t M) {
+    std::vector<ProbShape> shapes;
+    std::vector<sherry_linear_desc> kept;
+    if (batch_shapes(descs, count, M, shapes, kept) || shapes.empty() || M == 0) return 0;
+    return lut_workspace_bytes(shapes.data(), (int)shapes.size(), M, device_sms());
+}
+
+int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M, int y_dtype, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+    std::vector<ProbShape> shapes;
+    std::vector<sherry_linear_desc> kept;
+    int st = batch_shapes(descs, count, M, shapes, kept);
+    if (st) return st;
+    if (y_dtype != SHERRY_F32 && y_dtype != SHERRY_BF16) return SHERRY_ERR_DTYPE;
+    if (shapes.empty() || M == 0) return SHERRY_OK;
+    const int sms = device_sms();
+    const size_t need = lut_workspace_bytes(shapes.data(), (int)shapes.size(), M, sms);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SHERRY_ERR_WORKSPACE;
+    if (need > 0 && !aligned(workspace, 256)) return SHERRY_ERR_ALIGN;
+    return lut_linear_launch(shapes.data(), kept.data(), (int)shapes.size(), M, y_dtype == SHERRY_BF16, workspace,
+                             sms, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,109 @@
+// common.cuh -- internal helpers shared by the library's CUDA sources.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sherry.h"
+
+namespace sherry {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// last CUDA error seen by an entry point on this host thread
+void set_cuda_error(cudaError_t e);
+
+#define SHERRY_CUDA_CHECK(expr)                              \
+    do {                                                     \
+        cudaError_t _e = (expr);                             \
+        if (_e != cudaSuccess) {                             \
+            ::sherry::set_cuda_error(_e);                    \
+            return SHERRY_ERR_CUDA;                          \
+        }                                                    \
+    } while (0)
+
+#define SHERRY_LAUNCH_CHECK() SHERRY_CUDA_CHECK(cudaGetLastError())
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__host__ __device__ __forceinline__ int64_t pow2_ceil64(int64_t x) {
+    int64_t p = 1;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+__host__ __device__ __forceinline__ int ilog2_exact(int64_t x) {  // -1 if not a power of two
+    if (x <= 0 || (x & (x - 1))) return -1;
+    int s = 0;
+    while ((int64_t(1) << s) < x) ++s;
+    return s;
+}
+
+// Canonical pairwise sum of v[0..n) (adjacent pairs, padded with +0.0 to a
+// power of two), evaluated sequentially with a stack of completed subtrees.
+// Every value here is >= 0, so adding a padding zero is exact and the padded
+// tree equals the right fold of the stack.
+__device__ __forceinline__ float tree_sum_seq(const float* v, int n) {
+    float st[32];
+    int lv[32];
+    int top = 0;
+    for (int i = 0; i < n; ++i) {
+        float x = v[i];
+        int l = 0;
+        while (top > 0 && lv[top - 1] == l) {
+            x = st[top - 1] + x;
+            --top;
+            ++l;
+        }
+        st[top] = x;
+        lv[top] = l;
+        ++top;
+    }
+    if (top == 0) return 0.0f;
+    float r = st[top - 1];
+    for (int t = top - 2; t >= 0; --t) r = st[t] + r;
+    return r;
+}
+
+// Canonical pairwise sum of v[0..n) by one full warp; the result is returned in
+// every lane.  Each lane reduces an aligned power-of-two segment sequentially,
+// then the xor butterfly (offsets 1, 2, 4, ...) combines adjacent segments,
+// which is exactly the upper levels of the same tree.
+__device__ __forceinline__ float warp_tree_sum(const float* v, int n) {
+    const int lane = threadIdx.x & 31;
+    int64_t P = pow2_ceil64(n > 0 ? n : 1);
+    float x;
+    int span;  // number of lanes that carry tree nodes
+    if (P <= 32) {
+        x = (lane < n) ? v[lane] : 0.0f;
+        span = (int)P;
+    } else {
+        int seg = (int)(P / 32);
+        int lo = lane * seg;
+        int cnt = n - lo;
+        cnt = cnt < 0 ? 0 : (cnt > seg ? seg : cnt);
+        x = tree_sum_seq(v + lo, cnt);
+        span = 32;
+    }
+    for (int off = 1; off < span; off <<= 1) x = x + __shfl_xor_sync(kFull, x, off);
+    return __shfl_sync(kFull, x, 0);
+}
+
+struct ProbShape {
+    int64_t N, K;
+    int granularity, group;
+};
+
+// launchers (quantize.cu, unpack.cu, gemv.cu)
+size_t quantize_workspace_bytes(int64_t N, int64_t K, int granularity);
+int quantize_pack_launch(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
+                         uint32_t* idx, uint8_t* sgn, float* scales, void* workspace, cudaStream_t stream);
+int unpack_launch(const uint32_t* idx, const uint8_t* sgn, const float* scales, int64_t N, int64_t K,
+                  int granularity, int group, uint16_t* out, cudaStream_t stream, int num_sms);
+size_t lut_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms);
+int lut_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M,
+                      int y_bf16, void* workspace, int sms, cudaStream_t stream);
+
+}  // namespace sherry

@@ -1,0 +1,49 @@
+"""Helpers for the GPU parity tests: run the CUDA path and the oracle on the same
+seeded inputs and compare (packed bytes/scales bit for bit, Y within bounds)."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from sparse_ternary_weight_b200 import synth
+
+GRAN = {"tensor": oracle.PER_TENSOR, "channel": oracle.PER_CHANNEL, "group": oracle.PER_GROUP}
+
+
+def to_dev(a, dtype=None):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.view(dtype)
+    return t.cuda()
+
+
+def packed_to_host(P):
+    idx = P.idx.cpu().numpy().view(np.uint32)
+    sgn = P.sgn.cpu().numpy()
+    sc = P.scales.cpu().numpy()[: max(1, P.scales.numel())]
+    return idx, sgn, sc
+
+
+def gate(y, y_ref):
+    """max|y - y_ref| / max|y_ref| (the method's parity metric)."""
+    d = np.abs(np.asarray(y, np.float64) - y_ref).max()
+    m = np.abs(y_ref).max()
+    return d / m if m > 0 else d
+
+
+def elementwise_bound(Xf, Wq):
+    """fp32 accumulation bound per output: 2^-16 * sum_k |x_k| |w_k|."""
+    return 2.0 ** -16 * (np.abs(Xf).astype(np.float64) @ np.abs(Wq).astype(np.float64).T) + 1e-30
+
+
+def check_linear(y, y_ref, Xb, Wq, y_is_bf16=False):
+    g = gate(y, y_ref)
+    if y_is_bf16:
+        assert g <= 1e-3 + 2.0 ** -8, g
+        return g
+    assert g <= 1e-3, g
+    bound = elementwise_bound(synth.bf16_bits_to_f32(Xb), Wq)
+    err = np.abs(np.asarray(y, np.float64) - y_ref)
+    assert np.all(err <= bound), (err / bound).max()
+    return g

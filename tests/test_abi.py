@@ -1,0 +1,152 @@
+"""The C-ABI library loads and exports every symbol include/sherry.h declares;
+host-side argument checks return their documented status without launching
+anything (these run without a GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from sparse_ternary_weight_b200 import _abi
+from sparse_ternary_weight_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(sherry_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _abi.lib()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("sherry_quantize_pack", "sherry_linear", "sherry_unpack", "sherry_linear_batched",
+                     "sherry_num_scales", "sherry_workspace_bytes", "sherry_status_string"):
+        assert required in names
+
+
+def test_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.SO_PATH], capture_output=True, text=True, check=True)
+    exported = {line.split()[-1] for line in out.stdout.splitlines() if line.strip()}
+    missing = declared_functions() - exported
+    assert not missing, missing
+    for name in declared_functions():
+        assert hasattr(L, name)
+    # the binding declares exactly the header's functions
+    assert set(_abi.SIGNATURES) == declared_functions()
+
+
+def test_size_queries(L):
+    assert L.sherry_idx_bytes(3072, 3072) == 3072 * 3072 // 8
+    assert L.sherry_sgn_bytes(3072, 3072) == 3072 * 3072 // 32
+    # 1.25 bit / weight for the two planes
+    assert (L.sherry_idx_bytes(64, 256) + L.sherry_sgn_bytes(64, 256)) * 8 == 64 * 256 * 1.25
+    assert L.sherry_num_scales(64, 256, _abi.PER_GROUP, 128) == 128
+    assert L.sherry_num_scales(64, 256, _abi.PER_CHANNEL, 0) == 64
+    assert L.sherry_num_scales(64, 256, _abi.PER_TENSOR, 0) == 1
+    assert L.sherry_num_scales(64, 256, _abi.PER_GROUP, 96) == -1
+    assert L.sherry_num_scales(64, 48, _abi.PER_CHANNEL, 0) == -1
+    assert L.sherry_idx_bytes(64, 48) == 0
+    assert L.sherry_workspace_bytes(_abi.OP_QUANTIZE_PACK, 0, 64, 256, _abi.PER_GROUP, 128) == 0
+    assert L.sherry_workspace_bytes(_abi.OP_QUANTIZE_PACK, 0, 64, 256, _abi.PER_TENSOR, 0) > 0
+    assert L.sherry_version() > 0
+    for s in range(11):
+        assert L.sherry_status_string(s)
+
+
+FAKE = 0x10000  # aligned, never dereferenced: every call below fails validation first
+
+
+def test_quantize_pack_validation(L):
+    q = L.sherry_quantize_pack
+    args = lambda **kw: [kw.get("W", FAKE), kw.get("dt", _abi.F32), kw.get("N", 4), kw.get("K", 64),
+                         kw.get("g", _abi.PER_GROUP), kw.get("group", 32), kw.get("idx", FAKE),
+                         kw.get("sgn", FAKE), kw.get("sc", FAKE), None, 0, None]
+    assert q(*args(K=48)) == _abi.ERR_SHAPE
+    assert q(*args(K=0)) == _abi.ERR_SHAPE
+    assert q(*args(K=_abi.MAX_K + 32)) == _abi.ERR_SHAPE
+    assert q(*args(N=-1)) == _abi.ERR_SHAPE
+    assert q(*args(group=0)) == _abi.ERR_GROUP
+    assert q(*args(group=16)) == _abi.ERR_GROUP
+    assert q(*args(group=128)) == _abi.ERR_GROUP
+    assert q(*args(g=3)) == _abi.ERR_GRANULARITY
+    assert q(*args(dt=9)) == _abi.ERR_DTYPE
+    assert q(*args(W=None)) == _abi.ERR_NULL
+    assert q(*args(sc=None)) == _abi.ERR_NULL
+    assert q(*args(W=FAKE + 4)) == _abi.ERR_ALIGN
+    assert q(*args(idx=FAKE + 8)) == _abi.ERR_ALIGN
+    # per-tensor needs a workspace
+    assert q(*args(g=_abi.PER_TENSOR)) == _abi.ERR_WORKSPACE
+    # empty per-group / per-channel tensors are a no-op
+    assert q(*args(N=0, W=None, idx=None, sgn=None)) == _abi.OK
+
+
+def test_linear_validation(L):
+    f = L.sherry_linear
+    args = lambda **kw: [kw.get("X", FAKE), kw.get("M", 1), kw.get("N", 8), kw.get("K", 64), kw.get("idx", FAKE),
+                         kw.get("sgn", FAKE), kw.get("sc", FAKE), kw.get("g", _abi.PER_GROUP),
+                         kw.get("group", 32), kw.get("Y", FAKE), kw.get("yd", _abi.F32), None, 0, None]
+    assert f(*args(M=-1)) == _abi.ERR_SHAPE
+    assert f(*args(K=40)) == _abi.ERR_SHAPE
+    assert f(*args(group=48)) == _abi.ERR_GROUP
+    assert f(*args(g=9)) == _abi.ERR_GRANULARITY
+    assert f(*args(yd=4)) == _abi.ERR_DTYPE
+    assert f(*args(X=None)) == _abi.ERR_NULL
+    assert f(*args(idx=None)) == _abi.ERR_NULL
+    assert f(*args(Y=FAKE + 2)) == _abi.ERR_ALIGN
+    assert f(*args(X=FAKE + 8)) == _abi.ERR_ALIGN
+    # nothing to do
+    assert f(*args(M=0)) == _abi.OK
+    assert f(*args(N=0, idx=None, sgn=None, sc=None)) == _abi.OK
+
+
+def test_batched_validation(L):
+    d = (_abi.LinearDesc * 2)()
+    for i in range(2):
+        d[i] = _abi.LinearDesc(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, _abi.PER_GROUP, 32)
+    assert L.sherry_linear_batched(d, 2, 17, _abi.F32, None, 0, None) == _abi.ERR_SHAPE   # M > 16
+    assert L.sherry_linear_batched(d, _abi.MAX_BATCH + 1, 1, _abi.F32, None, 0, None) == _abi.ERR_SHAPE
+    d[1].K = 40
+    assert L.sherry_linear_batched(d, 2, 1, _abi.F32, None, 0, None) == _abi.ERR_SHAPE
+    d[1].K = 64
+    d[1].Y = FAKE + 4
+    assert L.sherry_linear_batched(d, 2, 1, _abi.F32, None, 0, None) == _abi.ERR_ALIGN
+    assert L.sherry_linear_batched(d, 0, 1, _abi.F32, None, 0, None) == _abi.OK
+    assert L.sherry_linear_batched(d, 2, 0, _abi.F32, None, 0, None) == _abi.ERR_ALIGN
+
+
+def test_unpack_validation(L):
+    u = L.sherry_unpack
+    assert u(FAKE, FAKE, FAKE, 4, 50, _abi.PER_CHANNEL, 0, FAKE, None) == _abi.ERR_SHAPE
+    assert u(None, FAKE, FAKE, 4, 64, _abi.PER_CHANNEL, 0, FAKE, None) == _abi.ERR_NULL
+    assert u(FAKE, FAKE, FAKE, 4, 64, _abi.PER_CHANNEL, 0, None, None) == _abi.ERR_NULL
+    assert u(FAKE, FAKE, FAKE, 4, 64, _abi.PER_CHANNEL, 0, FAKE + 2, None) == _abi.ERR_ALIGN
+    assert u(None, None, None, 0, 64, _abi.PER_CHANNEL, 0, None, None) == _abi.OK
+
+
+def test_product_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_abi, "_lib", None)
+    monkeypatch.setattr(_abi, "SO_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        _abi.lib()
+
+
+def test_product_rejects_cpu_tensors():
+    import torch
+    import sparse_ternary_weight_b200 as sw
+    with pytest.raises(ValueError, match="CUDA"):
+        sw.quantize_pack(torch.zeros(4, 64))

@@ -1,0 +1,222 @@
+"""CUDA path vs the CPU oracle on the same seeded inputs (needs a B200).
+
+Packed idx/sgn planes and scales must be bit-exact; unpacked bf16 weights must
+be bit-exact; Y must satisfy max|y - y_ref| / max|y_ref| <= 1e-3 against the
+fp64 oracle and, for fp32 Y, every element must lie within 2^-16 * sum|x||w|
+of it (the fp32 accumulation bound, far tighter than the gate)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+from sparse_ternary_weight_b200 import synth
+from tests.gpu_common import GRAN, check_linear, packed_to_host, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sw():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_ternary_weight_b200.build import build
+    build()
+    import sparse_ternary_weight_b200 as sw
+    return sw
+
+
+def _weights(kind, N, K, seed):
+    if kind == "normal":
+        return synth.weights_normal(N, K, seed, outlier_frac=0.01)
+    if kind == "t4":
+        return synth.weights_student_t(N, K, seed)
+    if kind == "ties":   # coarse grid: many ties and exact zeros, signed zeros
+        W = np.round(synth.weights_normal(N, K, seed) * 64) / np.float32(64)
+        W[:, ::7] = -0.0
+        return W.astype(np.float32)
+    raise ValueError(kind)
+
+
+QP_CASES = [
+    # (N, K, gran, group, kind)
+    (64, 256, "group", 128, "normal"),
+    (1, 32, "group", 32, "normal"),
+    (3, 96, "group", 96, "ties"),
+    (7, 160, "group", 32, "t4"),
+    (33, 384, "group", 128, "ties"),
+    (33, 384, "group", 64, "t4"),
+    (5, 3072, "group", 128, "t4"),
+    (17, 8192, "group", 256, "normal"),
+    (9, 3072, "group", 3072, "t4"),
+    (2, 65536, "group", 128, "t4"),
+    (64, 256, "channel", 0, "normal"),
+    (3, 96, "channel", 0, "ties"),
+    (5, 3072, "channel", 0, "t4"),
+    (11, 8192, "channel", 0, "ties"),
+    (64, 256, "tensor", 0, "normal"),
+    (7, 96, "tensor", 0, "ties"),
+    (129, 3072, "tensor", 0, "t4"),
+    (300, 160, "tensor", 0, "t4"),
+]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", QP_CASES, ids=lambda c: f"{c[0]}x{c[1]}-{c[2]}{c[3]}-{c[4]}")
+def test_quantize_pack_bit_exact(sw, orc, case, dtype):
+    import torch
+    N, K, gname, group, kind = case
+    W = _weights(kind, N, K, seed=N * 7 + K)
+    gran = GRAN[gname]
+    if dtype == "bf16":
+        Wb = synth.f32_to_bf16_bits(W)
+        Wd = to_dev(Wb.view(np.int16)).view(torch.bfloat16)
+        ref = orc.quantize_pack(Wb, gran, group)
+    else:
+        Wd = to_dev(W)
+        ref = orc.quantize_pack(W, gran, group)
+    P = sw.quantize_pack(Wd, gran, group)
+    got = packed_to_host(P)
+    for g, r, name in zip(got, ref, ("idx", "sgn", "scales")):
+        assert np.array_equal(g.reshape(-1).view(np.uint8), r.reshape(-1).view(np.uint8)), name
+
+
+def test_quantize_pack_empty_and_degenerate(sw, orc):
+    import torch
+    # N = 0: per-tensor scale = 0 / max(0, 1) = 0
+    W = torch.zeros((0, 64), dtype=torch.float32, device="cuda")
+    P = sw.quantize_pack(W, "per_tensor")
+    assert P.scales.cpu().tolist() == [0.0]
+    P = sw.quantize_pack(W, "per_group", 32)
+    assert P.idx.numel() == 0
+    # all-zero weights: every scale 0, every block zeroes position 0, kept signs +
+    W = torch.zeros((4, 64), dtype=torch.float32, device="cuda")
+    P = sw.quantize_pack(W, "per_channel")
+    idx, sgn, sc = packed_to_host(P)
+    assert np.all(idx == 0) and np.all(sgn == 0) and np.all(sc == 0)
+    # all weights -0.0: same code as +0.0
+    Wn = torch.full((4, 64), -0.0, dtype=torch.float32, device="cuda")
+    idx2, sgn2, _ = packed_to_host(sw.quantize_pack(Wn, "per_channel"))
+    assert np.array_equal(idx, idx2) and np.array_equal(sgn, sgn2)
+
+
+@pytest.mark.parametrize("case", [(64, 256, "group", 128), (33, 384, "group", 96), (5, 3072, "channel", 0),
+                                  (129, 160, "tensor", 0), (16, 8192, "group", 32)],
+                         ids=lambda c: f"{c[0]}x{c[1]}-{c[2]}{c[3]}")
+def test_unpack_bit_exact(sw, orc, case):
+    N, K, gname, group = case
+    gran = GRAN[gname]
+    W = _weights("t4", N, K, seed=31 + N)
+    P = sw.quantize_pack(to_dev(W), gran, group)
+    idx, sgn, sc = packed_to_host(P)
+    ref = orc.unpack_bf16(idx, sgn, sc, N, K, gran, group)
+    got = sw.unpack(P).cpu().view(__import__("torch").int16).numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+
+
+LIN_CASES = [
+    # (M, N, K, gran, group)
+    (1, 64, 256, "group", 128),     # the tiny single-linear workload
+    (1, 1, 32, "group", 32),
+    (1, 100, 96, "group", 96),      # K % 128 != 0 path
+    (1, 257, 384, "group", 64),
+    (1, 300, 3072, "group", 128),
+    (1, 1024, 3072, "group", 128),
+    (1, 3072, 8192, "group", 128),
+    (1, 70, 8192, "channel", 0),
+    (1, 513, 160, "tensor", 0),
+    (1, 200, 1024, "group", 256),
+    (1, 64, 2048, "group", 32),
+    (2, 129, 512, "group", 128),
+    (3, 64, 3072, "channel", 0),
+    (4, 500, 1024, "group", 128),
+    (5, 33, 256, "tensor", 0),
+    (8, 1024, 3072, "group", 128),
+    (16, 512, 2048, "group", 128),
+    (16, 77, 96, "group", 32),
+    (17, 256, 1024, "group", 128),
+    (33, 130, 512, "channel", 0),
+]
+
+
+@pytest.mark.parametrize("ydt", ["f32", "bf16"])
+@pytest.mark.parametrize("case", LIN_CASES, ids=lambda c: f"M{c[0]}-{c[1]}x{c[2]}-{c[3]}{c[4]}")
+def test_linear_vs_oracle(sw, orc, case, ydt):
+    import torch
+    M, N, K, gname, group = case
+    gran = GRAN[gname]
+    W = _weights("t4", N, K, seed=1000 + N + K)
+    Xb = synth.activations_bf16(M, K, seed=2000 + M + K)
+    P = sw.quantize_pack(to_dev(W), gran, group)
+    idx, sgn, sc = packed_to_host(P)
+    y_ref = orc.linear(Xb, idx, sgn, sc, N, K, gran, group)
+    Wq = orc.unpack_f32(idx, sgn, sc, N, K, gran, group)
+    X = to_dev(Xb.view(np.int16)).view(torch.bfloat16)
+    y32 = sw.linear(X, P, torch.float32)
+    check_linear(y32.cpu().numpy(), y_ref, Xb, Wq)
+    if ydt == "bf16":
+        yb = sw.linear(X, P, torch.bfloat16)
+        check_linear(yb.float().cpu().numpy(), y_ref, Xb, Wq, y_is_bf16=True)
+        # bf16 Y is the round-to-nearest-even of the fp32 accumulator
+        assert torch.equal(yb, y32.to(torch.bfloat16))
+    # deterministic
+    assert torch.equal(sw.linear(X, P, torch.float32), y32)
+
+
+def test_linear_hand_worked_row(sw):
+    """The hand-worked 32-weight row (tests/golden/hand_worked.json): y = 15.25."""
+    import json
+    import os
+    import torch
+    hw = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_worked.json")))["row"]
+    W = torch.tensor([hw["w"]], dtype=torch.float32, device="cuda")
+    for g, grp in (("per_channel", 0), ("per_group", 32), ("per_tensor", 0)):
+        P = sw.quantize_pack(W, g, grp)
+        assert P.idx.cpu().numpy().view(np.uint32)[0, 0] == int(hw["idx_word"], 16)
+        assert P.sgn.cpu().tolist() == [[int(hw["sgn_byte"], 16)]]
+        assert P.scales.cpu().tolist() == [hw["alpha"]]
+        X = torch.ones((1, 32), dtype=torch.bfloat16, device="cuda")
+        assert sw.linear(X, P).item() == hw["y_all_ones"]
+        assert sw.unpack(P).float().cpu().numpy().tolist() == [[t * hw["alpha"] for t in hw["t"]]]
+
+
+def test_linear_batched_matches_oracle(sw, orc):
+    import torch
+    shapes = [(1024, 3072, "group", 128), (300, 3072, "channel", 0), (64, 96, "group", 32),
+              (513, 8192, "group", 128), (77, 160, "tensor", 0), (2048, 2048, "group", 64)]
+    for M in (1, 2, 4, 7, 16):
+        pairs, refs = [], []
+        for i, (N, K, gname, group) in enumerate(shapes):
+            gran = GRAN[gname]
+            W = _weights("normal", N, K, seed=3000 + i)
+            Xb = synth.activations_bf16(M, K, seed=4000 + i + 10 * M)
+            P = sw.quantize_pack(to_dev(W), gran, group)
+            idx, sgn, sc = packed_to_host(P)
+            refs.append((orc.linear(Xb, idx, sgn, sc, N, K, gran, group),
+                         orc.unpack_f32(idx, sgn, sc, N, K, gran, group), Xb))
+            pairs.append((to_dev(Xb.view(np.int16)).view(torch.bfloat16), P))
+        outs = sw.linear_batched(pairs, torch.float32)
+        for y, (y_ref, Wq, Xb) in zip(outs, refs):
+            check_linear(y.cpu().numpy(), y_ref, Xb, Wq)
+        outs2 = sw.linear_batched(pairs, torch.float32)
+        assert all(torch.equal(a, b) for a, b in zip(outs, outs2))
+
+
+def test_split_k_tickets_left_zero(sw):
+    """A split-K call leaves its ticket counters at zero, so back-to-back calls
+    on one workspace stay correct."""
+    import torch
+    W = torch.randn(64, 8192, device="cuda") * 0.02
+    P = sw.quantize_pack(W)
+    X = torch.randn(1, 8192, device="cuda").to(torch.bfloat16)
+    from sparse_ternary_weight_b200 import _abi
+    L = _abi.lib()
+    wsb = L.sherry_workspace_bytes(_abi.OP_LINEAR, 1, 64, 8192, _abi.PER_GROUP, 128)
+    assert wsb > 0   # this shape splits K across CTAs
+    ys = [sw.linear(X, P) for _ in range(5)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(ys[0], y) for y in ys[1:])
+    ws = sw._ws_cache[(str(X.device), "linear")]
+    cnt_bytes = 256  # ticket region is the first (rounded) block of the workspace
+    assert int(ws[:cnt_bytes].view(torch.int32).abs().sum()) == 0
