@@ -47,6 +47,27 @@ static int check_planes(const uint32_t* idx, const uint8_t* sgn, const float* sc
     return SHERRY_OK;
 }
 
+// the decode path a set of linears takes: the streaming one-token kernel when
+// every problem qualifies, else the general lookup-table kernel
+static bool use_stream(const ProbShape* shapes, int count, int64_t M) {
+    if (M != 1 || count == 0) return false;
+    for (int i = 0; i < count; ++i)
+        if (!stream_eligible(shapes[i], M)) return false;
+    return true;
+}
+
+static size_t linear_ws_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
+    if (use_stream(shapes, count, M)) return stream_workspace_bytes(shapes, count, sms);
+    return lut_workspace_bytes(shapes, count, M, sms);
+}
+
+static int linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
+                         void* workspace, int sms, cudaStream_t stream) {
+    if (use_stream(shapes, count, M))
+        return stream_linear_launch(shapes, descs, count, y_bf16, workspace, sms, stream);
+    return lut_linear_launch(shapes, descs, count, M, y_bf16, workspace, sms, stream);
+}
+
 }  // namespace sherry
 
 using namespace sherry;
@@ -97,7 +118,7 @@ size_t sherry_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int granu
     if (op == SHERRY_OP_LINEAR) {
         if (M <= 0 || N == 0) return 0;
         ProbShape s{N, K, granularity, group};
-        return lut_workspace_bytes(&s, 1, M, device_sms());
+        return linear_ws_bytes(&s, 1, M, device_sms());
     }
     return 0;
 }
@@ -151,11 +172,10 @@ int sherry_linear(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint
     if (M == 0 || N == 0) return SHERRY_OK;
     ProbShape s{N, K, granularity, group};
     const int sms = device_sms();
-    const size_t need = lut_workspace_bytes(&s, 1, M, sms);
+    const size_t need = linear_ws_bytes(&s, 1, M, sms);
     if (need > 0 && (!workspace || workspace_bytes < need)) return SHERRY_ERR_WORKSPACE;
     if (need > 0 && !aligned(workspace, 256)) return SHERRY_ERR_ALIGN;
-    return lut_linear_launch(&s, &d, 1, M, y_dtype == SHERRY_BF16, workspace, sms,
-                             static_cast<cudaStream_t>(stream));
+    return linear_launch(&s, &d, 1, M, y_dtype == SHERRY_BF16, workspace, sms, static_cast<cudaStream_t>(stream));
 }
 
 static int batch_shapes(const sherry_linear_desc* descs, int count, int64_t M, std::vector<ProbShape>& shapes,
@@ -177,7 +197,7 @@ size_t sherry_linear_batched_workspace_bytes(const sherry_linear_desc* descs, in
     std::vector<ProbShape> shapes;
     std::vector<sherry_linear_desc> kept;
     if (batch_shapes(descs, count, M, shapes, kept) || shapes.empty() || M == 0) return 0;
-    return lut_workspace_bytes(shapes.data(), (int)shapes.size(), M, device_sms());
+    return linear_ws_bytes(shapes.data(), (int)shapes.size(), M, device_sms());
 }
 
 int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M, int y_dtype, void* workspace,
@@ -189,11 +209,11 @@ int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M,
     if (y_dtype != SHERRY_F32 && y_dtype != SHERRY_BF16) return SHERRY_ERR_DTYPE;
     if (shapes.empty() || M == 0) return SHERRY_OK;
     const int sms = device_sms();
-    const size_t need = lut_workspace_bytes(shapes.data(), (int)shapes.size(), M, sms);
+    const size_t need = linear_ws_bytes(shapes.data(), (int)shapes.size(), M, sms);
     if (need > 0 && (!workspace || workspace_bytes < need)) return SHERRY_ERR_WORKSPACE;
     if (need > 0 && !aligned(workspace, 256)) return SHERRY_ERR_ALIGN;
-    return lut_linear_launch(shapes.data(), kept.data(), (int)shapes.size(), M, y_dtype == SHERRY_BF16, workspace,
-                             sms, static_cast<cudaStream_t>(stream));
+    return linear_launch(shapes.data(), kept.data(), (int)shapes.size(), M, y_dtype == SHERRY_BF16, workspace, sms,
+                         static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

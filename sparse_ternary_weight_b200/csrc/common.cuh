@@ -105,5 +105,10 @@ int unpack_launch(const uint32_t* idx, const uint8_t* sgn, const float* scales, 
 size_t lut_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms);
 int lut_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M,
                       int y_bf16, void* workspace, int sms, cudaStream_t stream);
+// one-token streaming kernel (gemv_stream.cu)
+bool stream_eligible(const ProbShape& s, int64_t M);
+size_t stream_workspace_bytes(const ProbShape* shapes, int count, int sms);
+int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int y_bf16,
+                         void* workspace, int sms, cudaStream_t stream);
 
 }  // namespace sherry

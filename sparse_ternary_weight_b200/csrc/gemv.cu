@@ -23,6 +23,7 @@
 // the workspace, and the last CTA to arrive (an atomic ticket, no waiting) adds
 // the partials in split order and writes Y, so results are deterministic.
 #include "common.cuh"
+#include "lut.cuh"
 
 #include <cuda_bf16.h>
 
@@ -33,7 +34,6 @@
 namespace sherry {
 
 constexpr int kLThreads = 256;
-constexpr int kTab = 144;                    // bytes per 32-entry table (128 + 16 pad)
 constexpr int kLutTables = 256;              // tables per CTA (= threads)
 constexpr int kLutBytes = kLutTables * kTab; // 36864
 constexpr int kLutSmem = kLutBytes + 256;    // + alignment slack
@@ -70,68 +70,6 @@ struct LinParams {
     int total_tiles;
     LinProb p[MAXP];
 };
-
-__device__ __forceinline__ float lds_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ void sts_v4(uint32_t addr, float a, float b, float c, float d) {
-    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d));
-}
-
-__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
-
-// Build the 32-entry table of one block of 4 activations at `tab` (shared address).
-__device__ __forceinline__ void build_table(uint32_t tab, uint2 xb) {
-    const float x0 = bf16lo(xb.x), x1 = bf16hi(xb.x), x2 = bf16lo(xb.y), x3 = bf16hi(xb.y);
-    float e[16];
-#pragma unroll
-    for (int z = 0; z < 4; ++z) {
-        const float a = z == 0 ? x1 : x0;
-        const float b = z <= 1 ? x2 : x1;
-        const float c = z == 3 ? x2 : x3;
-        const float s = a + b, d = a - b;
-        e[4 * z + 0] = s + c;
-        e[4 * z + 1] = s - c;
-        e[4 * z + 2] = d + c;
-        e[4 * z + 3] = d - c;
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) sts_v4(tab + 16 * q, e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-        sts_v4(tab + 64 + 16 * q, -e[4 * q], -e[4 * q + 1], -e[4 * q + 2], -e[4 * q + 3]);
-}
-
-// Even/odd byte-vectors of one packed word: byte i of `ev` is 4*code of block 2i,
-// byte i of `od` is 4*code of block 2i+1 (code = nibble + 16*G).
-__device__ __forceinline__ void spread_word(uint32_t w, uint32_t s, uint32_t& ev, uint32_t& od) {
-    ev = ((w << 2) & 0x3c3c3c3cu) | (((s & 0x55u) * 0x01041040u) & 0x40404040u);
-    od = ((w >> 2) & 0x3c3c3c3cu) | (((s & 0xaau) * 0x00820820u) & 0x40404040u);
-}
-
-// Sum of the 8 lookups of one word for MT tokens; tables of block j of this
-// word sit at base + (boff + j)*kTab, token m at + m*tstride.
-template <int MT>
-__device__ __forceinline__ void word_lookups(uint32_t w, uint32_t s, uint32_t base, int boff, int tstride,
-                                             float (&ws)[MT]) {
-    uint32_t ev, od;
-    spread_word(w, s, ev, od);
-    float v[MT][8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint32_t src = (j & 1) ? od : ev;
-        const uint32_t a = __byte_perm(src, base, (uint32_t)(j >> 1) | 0x7650u);
-#pragma unroll
-        for (int m = 0; m < MT; ++m) v[m][j] = lds_f32(a + (uint32_t)((boff + j) * kTab + m * tstride));
-    }
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-        ws[m] = ((v[m][0] + v[m][1]) + (v[m][2] + v[m][3])) + ((v[m][4] + v[m][5]) + (v[m][6] + v[m][7]));
-}
 
 template <int MT, int WR, int MAXP>
 __global__ void __launch_bounds__(kLThreads, 2) k_lut_linear(const __grid_constant__ LinParams<MAXP> P) {

@@ -1,0 +1,395 @@
+// gemv_stream.cu -- packed 3:4 ternary linear, one token (M = 1), HBM-streaming
+// version of the lookup-table decode (the method's inference scheme: tables
+// built from the activations, looked up by the packed weights, accumulated,
+// then scaled; "Sherry: Hardware-Efficient 1.25-Bit Ternary Quantization via
+// Fine-grained Sparsification", digest paragraph on inference; Y = X T alpha).
+//
+// Work unit: 256 output rows x 1024 weights (32 packed words) of one linear.
+// All units of a launch (one or many independent linears) are split into equal
+// contiguous ranges, one per CTA (stream-K): every CTA streams the same number
+// of bytes.  A row block whose units straddle two CTAs is finished by the CTA
+// that arrives last at its ticket, adding the partial sums in unit order, so Y
+// is deterministic.
+//
+// Per unit the CTA copies the packed planes with 16-byte cp.async (each 8
+// threads read one full 128-byte row segment, so global reads are coalesced)
+// into an XOR-swizzled shared layout that the row-per-lane reads hit without
+// bank conflicts; three stages are in flight.  The 32-entry tables of the
+// unit's 256 blocks of activations are double buffered and built one unit
+// ahead.  A lane owns one row: per packed word it spreads the 8 nibbles and
+// sign bits into two byte-vectors of table offsets (see lut.cuh) and does 8
+// lookups; alpha is applied once per 128-weight group (or once per row).
+#include "common.cuh"
+#include "lut.cuh"
+
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+namespace sherry {
+
+constexpr int kSThreads = 256;
+constexpr int kSRows = 256;                        // rows per unit, one per thread
+constexpr int kSWords = 32;                        // packed words per unit
+constexpr int kSStages = 3;
+constexpr int kSIdx = kSRows * kSWords * 4;        // 32 KB
+constexpr int kSSgn = kSRows * kSWords;            // 8 KB
+constexpr int kSSc = kSRows * 32;                  // 8 KB (at most 8 fp32 scales per row)
+constexpr int kSStage = kSIdx + kSSgn + kSSc;      // 48 KB
+constexpr int kSLut = 256 * kTab;                  // 36 KB, one table per block of the unit
+constexpr int kSSmem = kSStages * kSStage + 2 * kSLut + 1024;
+
+enum SMode { kSRow = 0, kSG128 = 1, kSG256 = 2 };
+
+struct SProb {
+    const uint16_t* X;
+    const uint32_t* idx;
+    const uint8_t* sgn;
+    const float* scales;
+    void* Y;
+    int N, words, spr;  // spr: scales per row (per-group)
+    int mode, per_tensor;
+    int n_rb, n_sub;    // row blocks, sub-slices (units) per row block
+    int unit_begin, tile_begin;
+};
+
+template <int MAXP>
+struct SParams {
+    int count, y_bf16, total_units, upc;
+    float* part;  // [grid][2][kSRows] split-tile partials
+    int* ticket;  // [total tiles]
+    SProb p[MAXP];
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+
+struct UnitPos {
+    int p, rb, sub;  // problem, row block, sub-slice
+};
+
+// issue the cp.async copies of one unit into `stage`
+template <int MAXP>
+__device__ __forceinline__ void issue_unit(const SParams<MAXP>& P, const UnitPos& u, uint32_t stage) {
+    const SProb& pr = P.p[u.p];
+    const int t = threadIdx.x;
+    const int row0 = u.rb * kSRows;
+    const int w0 = u.sub * kSWords;
+    // idx: 256 rows x 8 chunks of 16 B; chunk c of row r lands at chunk c ^ (r & 7)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int q = t + kSThreads * i;
+        const int r = q >> 3, c = q & 7;
+        const int row = row0 + r, word = w0 + 4 * c;
+        const bool ok = row < pr.N && word < pr.words;
+        const uint32_t* src = ok ? pr.idx + (int64_t)row * pr.words + word : pr.idx;
+        cp_async16(stage + r * 128 + ((c ^ (r & 7)) << 4), src, ok);
+    }
+    // sgn: 256 rows x 2 chunks; chunk h of row r lands at h ^ ((r >> 2) & 1)
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int q = t + kSThreads * i;
+        const int r = q >> 1, h = q & 1;
+        const int row = row0 + r, off = w0 + 16 * h;
+        const bool ok = row < pr.N && off < pr.words;
+        const uint8_t* src = ok ? pr.sgn + (int64_t)row * pr.words + off : pr.sgn;
+        cp_async16(stage + kSIdx + r * 32 + ((h ^ ((r >> 2) & 1)) << 4), src, ok);
+    }
+    if (pr.mode == kSG128) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int q = t + kSThreads * i;
+            const int r = q >> 1, h = q & 1;
+            const int row = row0 + r, off = w0 / 4 + 4 * h;
+            const bool ok = row < pr.N && off < pr.spr;
+            const float* src = ok ? pr.scales + (int64_t)row * pr.spr + off : pr.scales;
+            cp_async16(stage + kSIdx + kSSgn + r * 32 + ((h ^ ((r >> 2) & 1)) << 4), src, ok);
+        }
+    } else if (pr.mode == kSG256) {
+        const int r = t;
+        const int row = row0 + r, off = w0 / 8;
+        const bool ok = row < pr.N && off < pr.spr;
+        const float* src = ok ? pr.scales + (int64_t)row * pr.spr + off : pr.scales;
+        cp_async16(stage + kSIdx + kSSgn + r * 32 + (((r >> 2) & 1) << 4), src, ok);
+    }
+}
+
+template <int MAXP>
+__device__ __forceinline__ UnitPos locate(const SParams<MAXP>& P, int u) {
+    int p = 0;
+    while (p + 1 < P.count && P.p[p + 1].unit_begin <= u) ++p;
+    const int local = u - P.p[p].unit_begin;
+    return UnitPos{p, local / P.p[p].n_sub, local % P.p[p].n_sub};
+}
+
+__device__ __forceinline__ void advance(const SProb* probs, UnitPos& u) {
+    if (++u.sub == probs[u.p].n_sub) {
+        u.sub = 0;
+        if (++u.rb == probs[u.p].n_rb) {
+            u.rb = 0;
+            ++u.p;
+        }
+    }
+}
+
+template <int MAXP>
+__global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_constant__ SParams<MAXP> P) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ int s_last;
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    const uint32_t stages = base;
+    const uint32_t luts = base + kSStages * kSStage;
+
+    const int t = threadIdx.x;
+    const int u_begin = blockIdx.x * P.upc;
+    const int u_end = min(P.total_units, u_begin + P.upc);
+    if (u_begin >= u_end) return;
+
+    // prologue: units u_begin .. u_begin + kSStages - 2 in flight
+    UnitPos pre = locate(P, u_begin);
+    for (int i = 0; i < kSStages - 1; ++i) {
+        if (u_begin + i < u_end) {
+            issue_unit(P, pre, stages + i * kSStage);
+            advance(P.p, pre);
+        }
+        cp_async_commit();
+    }
+    UnitPos cur = locate(P, u_begin);
+    // tables of the first unit
+    {
+        const SProb& pr = P.p[cur.p];
+        const int b = cur.sub * kSWords * 8 + t;
+        if (b < pr.words * 8) build_table(luts + t * kTab, __ldg(reinterpret_cast<const uint2*>(pr.X) + b));
+    }
+    // first unit of the current tile covered by this CTA?
+    const int tile_start_unit0 = P.p[cur.p].unit_begin + cur.rb * P.p[cur.p].n_sub;
+    bool tile_from_start = (tile_start_unit0 == u_begin);
+
+    const int r = t;  // row within the unit
+    float acc = 0.0f;
+
+    for (int u = u_begin; u < u_end; ++u) {
+        const int k = u - u_begin;
+        cp_async_wait<kSStages - 2>();
+        __syncthreads();
+        // refill the stage freed by the previous unit
+        if (u + kSStages - 1 < u_end) issue_unit(P, pre, stages + ((k + kSStages - 1) % kSStages) * kSStage);
+        cp_async_commit();
+        if (u + kSStages - 1 < u_end) advance(P.p, pre);
+
+        // activations of the next unit's tables (latency hidden by this unit)
+        UnitPos nxt = cur;
+        advance(P.p, nxt);
+        uint2 xn = make_uint2(0u, 0u);
+        bool xn_ok = false;
+        if (u + 1 < u_end) {
+            const SProb& pn = P.p[nxt.p];
+            const int b = nxt.sub * kSWords * 8 + t;
+            xn_ok = b < pn.words * 8;
+            if (xn_ok) xn = __ldg(reinterpret_cast<const uint2*>(pn.X) + b);
+        }
+
+        const SProb& pr = P.p[cur.p];
+        const uint32_t st = stages + (k % kSStages) * kSStage;
+        const uint32_t lut = luts + (k & 1) * kSLut;
+        const int nsteps = min(8, (pr.words - cur.sub * kSWords) >> 2);
+        const uint32_t sgn_row = st + kSIdx + r * 32;
+        const uint32_t sw2 = ((r >> 2) & 1) << 4;
+        const uint4 sg0 = lds128(sgn_row + sw2);
+        const uint4 sg1 = lds128(sgn_row + (16u ^ sw2));
+        uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
+        if (pr.mode != kSRow) {
+            a0 = lds128(st + kSIdx + kSSgn + r * 32 + sw2);
+            if (pr.mode == kSG128) a1 = lds128(st + kSIdx + kSSgn + r * 32 + (16u ^ sw2));
+        }
+        const uint32_t idx_row = st + r * 128;
+        const uint32_t sw8 = (uint32_t)(r & 7);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            if (c < nsteps) {
+                const uint4 wq = lds128(idx_row + ((c ^ sw8) << 4));
+                const uint4& sgv = c < 4 ? sg0 : sg1;
+                const uint32_t sq = (c & 3) == 0 ? sgv.x : (c & 3) == 1 ? sgv.y : (c & 3) == 2 ? sgv.z : sgv.w;
+                const uint32_t tb = lut + (uint32_t)(c * 32 * kTab);
+                float ws[4][1];
+                word_lookups<1>(wq.x, sq & 0xffu, tb, 0, 0, ws[0]);
+                word_lookups<1>(wq.y, (sq >> 8) & 0xffu, tb, 8, 0, ws[1]);
+                word_lookups<1>(wq.z, (sq >> 16) & 0xffu, tb, 16, 0, ws[2]);
+                word_lookups<1>(wq.w, sq >> 24, tb, 24, 0, ws[3]);
+                const float s4 = (ws[0][0] + ws[1][0]) + (ws[2][0] + ws[3][0]);
+                if (pr.mode == kSRow) {
+                    acc += s4;
+                } else {
+                    uint32_t ab;
+                    if (pr.mode == kSG128) {
+                        const uint4& av = c < 4 ? a0 : a1;
+                        ab = (c & 3) == 0 ? av.x : (c & 3) == 1 ? av.y : (c & 3) == 2 ? av.z : av.w;
+                    } else {
+                        ab = (c >> 1) == 0 ? a0.x : (c >> 1) == 1 ? a0.y : (c >> 1) == 2 ? a0.z : a0.w;
+                    }
+                    acc = fmaf(__uint_as_float(ab), s4, acc);
+                }
+            }
+        }
+
+        // tile (row block) finished by this unit, or this CTA's range ends inside it
+        const bool tile_end = (cur.sub == pr.n_sub - 1);
+        if (tile_end || u == u_end - 1) {
+            const int n = cur.rb * kSRows + r;
+            const bool row_ok = n < pr.N;
+            float v = acc;
+            if (pr.mode == kSRow && row_ok) v *= __ldg(pr.scales + (pr.per_tensor ? 0 : n));
+            if (tile_from_start && tile_end) {
+                if (row_ok) {
+                    if (P.y_bf16)
+                        reinterpret_cast<__nv_bfloat16*>(pr.Y)[n] = __float2bfloat16_rn(v);
+                    else
+                        reinterpret_cast<float*>(pr.Y)[n] = v;
+                }
+            } else {
+                // split tile: partial into this CTA's slot, then the ticket
+                const int tile = pr.tile_begin + cur.rb;
+                const int tile_u0 = pr.unit_begin + cur.rb * pr.n_sub;
+                const int c_a = tile_u0 / P.upc;
+                const int c_b = (tile_u0 + pr.n_sub - 1) / P.upc;
+                const int slot = (u_begin >= tile_u0) ? 0 : 1;
+                __stcg(P.part + ((int64_t)blockIdx.x * 2 + slot) * kSRows + r, v);
+                __threadfence();
+                __syncthreads();
+                if (t == 0) s_last = (atomicAdd(P.ticket + tile, 1) == c_b - c_a);
+                __syncthreads();
+                if (s_last) {
+                    __threadfence();
+                    float sum = 0.0f;
+                    for (int c = c_a; c <= c_b; ++c) {
+                        const int sl = (c * P.upc >= tile_u0) ? 0 : 1;
+                        const float pv = __ldcg(P.part + ((int64_t)c * 2 + sl) * kSRows + r);
+                        sum = (c == c_a) ? pv : sum + pv;
+                    }
+                    if (row_ok) {
+                        if (P.y_bf16)
+                            reinterpret_cast<__nv_bfloat16*>(pr.Y)[n] = __float2bfloat16_rn(sum);
+                        else
+                            reinterpret_cast<float*>(pr.Y)[n] = sum;
+                    }
+                    if (t == 0) P.ticket[tile] = 0;  // leave the ticket zeroed
+                }
+            }
+            acc = 0.0f;
+            tile_from_start = true;  // every later tile of this range starts inside it
+        }
+
+        // tables of the next unit into the other buffer (its last reader was unit u-1)
+        if (u + 1 < u_end && xn_ok) build_table(luts + ((k + 1) & 1) * kSLut + t * kTab, xn);
+        cur = nxt;
+    }
+    cp_async_wait<0>();
+}
+
+// ---- host side -------------------------------------------------------------------
+
+bool stream_eligible(const ProbShape& s, int64_t M) {
+    if (M != 1 || s.N == 0) return false;
+    if (s.K % 512 != 0) return false;
+    if (s.granularity == SHERRY_PER_TENSOR || s.granularity == SHERRY_PER_CHANNEL) return true;
+    if (s.granularity != SHERRY_PER_GROUP) return false;
+    if (s.group == 128) return true;                        // K/128 % 4 == 0 since K % 512 == 0
+    if (s.group == 256) return (s.K / 256) % 4 == 0;        // 16-byte aligned scale rows
+    return false;
+}
+
+struct SPlan {
+    std::vector<SProb> probs;
+    int total_units = 0, total_tiles = 0, grid = 0, upc = 0;
+    size_t ws_bytes = 0, part_off = 0;
+};
+
+static int stream_ctas(int sms) { return sms; }  // one CTA per SM (the stages fill shared memory)
+
+static SPlan make_splan(const ProbShape* shapes, int count, int sms) {
+    SPlan pl;
+    int ub = 0, tb = 0;
+    for (int i = 0; i < count; ++i) {
+        const ProbShape& s = shapes[i];
+        SProb p{};
+        p.N = (int)s.N;
+        p.words = (int)(s.K / 32);
+        p.spr = s.granularity == SHERRY_PER_GROUP ? (int)(s.K / s.group) : 0;
+        p.mode = s.granularity != SHERRY_PER_GROUP ? kSRow : (s.group == 128 ? kSG128 : kSG256);
+        p.per_tensor = s.granularity == SHERRY_PER_TENSOR;
+        p.n_rb = (int)((s.N + kSRows - 1) / kSRows);
+        p.n_sub = (p.words + kSWords - 1) / kSWords;
+        p.unit_begin = ub;
+        p.tile_begin = tb;
+        ub += p.n_rb * p.n_sub;
+        tb += p.n_rb;
+        pl.probs.push_back(p);
+    }
+    pl.total_units = ub;
+    pl.total_tiles = tb;
+    const int g = std::max(1, std::min(stream_ctas(sms), ub));
+    pl.upc = (ub + g - 1) / g;
+    pl.grid = (ub + pl.upc - 1) / pl.upc;
+    const size_t ticket_bytes = ((size_t)tb * sizeof(int) + 255) / 256 * 256;
+    pl.part_off = ticket_bytes;
+    pl.ws_bytes = ticket_bytes + (size_t)pl.grid * 2 * kSRows * sizeof(float);
+    return pl;
+}
+
+size_t stream_workspace_bytes(const ProbShape* shapes, int count, int sms) {
+    return make_splan(shapes, count, sms).ws_bytes;
+}
+
+template <int MAXP>
+static int stream_launch_t(SPlan& pl, int y_bf16, void* workspace, cudaStream_t stream) {
+    static SParams<MAXP> P;
+    static std::mutex mu;
+    static bool attr = false;
+    std::lock_guard<std::mutex> lk(mu);
+    P.count = (int)pl.probs.size();
+    P.y_bf16 = y_bf16;
+    P.total_units = pl.total_units;
+    P.upc = pl.upc;
+    P.ticket = static_cast<int*>(workspace);
+    P.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.part_off);
+    for (int i = 0; i < P.count; ++i) P.p[i] = pl.probs[i];
+    if (!attr) {
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_lut_stream<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSSmem));
+        attr = true;
+    }
+    k_lut_stream<MAXP><<<pl.grid, kSThreads, kSSmem, stream>>>(P);
+    SHERRY_LAUNCH_CHECK();
+    return SHERRY_OK;
+}
+
+int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int y_bf16,
+                         void* workspace, int sms, cudaStream_t stream) {
+    SPlan pl = make_splan(shapes, count, sms);
+    for (int i = 0; i < count; ++i) {
+        SProb& p = pl.probs[i];
+        p.X = descs[i].X;
+        p.idx = descs[i].idx;
+        p.sgn = descs[i].sgn;
+        p.scales = descs[i].scales;
+        p.Y = descs[i].Y;
+    }
+    if (pl.total_units == 0) return SHERRY_OK;
+    if (count <= 1) return stream_launch_t<1>(pl, y_bf16, workspace, stream);
+    if (count <= 16) return stream_launch_t<16>(pl, y_bf16, workspace, stream);
+    return stream_launch_t<SHERRY_MAX_BATCH>(pl, y_bf16, workspace, stream);
+}
+
+}  // namespace sherry

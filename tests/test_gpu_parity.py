@@ -220,3 +220,34 @@ def test_split_k_tickets_left_zero(sw):
     ws = sw._ws_cache[(str(X.device), "linear")]
     cnt_bytes = 256  # ticket region is the first (rounded) block of the workspace
     assert int(ws[:cnt_bytes].view(torch.int32).abs().sum()) == 0
+
+
+STREAM_SHAPES = [(1024, 3072, "group", 128), (300, 3072, "channel", 0), (3072, 8192, "group", 128),
+                 (77, 1024, "group", 256), (513, 2048, "tensor", 0), (8192, 3072, "group", 128),
+                 (1, 512, "group", 128), (257, 3072, "group", 256)]
+
+
+def test_stream_batch_many_problems_vs_oracle(sw, orc):
+    """One-token batch of many eligible linears (the streaming kernel: units split
+    evenly over CTAs, tiles straddling two CTAs finished through the ticket)."""
+    import torch
+    pairs, refs = [], []
+    for i in range(24):
+        N, K, gname, group = STREAM_SHAPES[i % len(STREAM_SHAPES)]
+        gran = GRAN[gname]
+        W = _weights("t4" if i % 2 else "normal", N, K, seed=5000 + i)
+        Xb = synth.activations_bf16(1, K, seed=6000 + i)
+        P = sw.quantize_pack(to_dev(W), gran, group)
+        idx, sgn, sc = packed_to_host(P)
+        refs.append((orc.linear(Xb, idx, sgn, sc, N, K, gran, group), orc.unpack_f32(idx, sgn, sc, N, K, gran, group),
+                     Xb))
+        pairs.append((to_dev(Xb.view(np.int16)).view(torch.bfloat16), P))
+    for ydt in (torch.float32, torch.bfloat16):
+        outs = sw.linear_batched(pairs, ydt)
+        for y, (y_ref, Wq, Xb) in zip(outs, refs):
+            check_linear(y.float().cpu().numpy(), y_ref, Xb, Wq, y_is_bf16=(ydt == torch.bfloat16))
+        again = sw.linear_batched(pairs, ydt)
+        assert all(torch.equal(a, b) for a, b in zip(outs, again))
+    # single calls agree with the oracle as well
+    for (X, P), (y_ref, Wq, Xb) in zip(pairs[:8], refs[:8]):
+        check_linear(sw.linear(X, P).cpu().numpy(), y_ref, Xb, Wq)
