@@ -95,9 +95,11 @@ size_t sherry_sgn_bytes(int64_t N, int64_t K);
 /* number of fp32 scales: N*K/group, N or 1 (-1 on invalid arguments) */
 int64_t sherry_num_scales(int64_t N, int64_t K, int granularity, int group);
 /* device workspace an operation needs (0 = none); pass at least this many
- * bytes.  The linear's workspace must be zero-filled before its first use and
- * is left zero-filled by every call that returns SHERRY_OK; calls that share a
- * workspace must not overlap on the device. */
+ * bytes.  A linear workspace starts with a 256 KiB region of split-K tickets
+ * that must be zero before its first use; every call that returns SHERRY_OK
+ * leaves that region zero (what follows it is scratch).  One workspace may be
+ * shared by linear calls (single or batched) that do not overlap on the device;
+ * do not share it with the quantise+pack scratch. */
 size_t sherry_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int granularity, int group);
 
 /* ---- quantise + pack ----------------------------------------------------

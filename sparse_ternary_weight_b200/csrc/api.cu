@@ -51,9 +51,12 @@ static int check_planes(const uint32_t* idx, const uint8_t* sgn, const float* sc
 // every problem qualifies, else the general lookup-table kernel
 static bool use_stream(const ProbShape* shapes, int count, int64_t M) {
     if (M != 1 || count == 0) return false;
-    for (int i = 0; i < count; ++i)
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) {
         if (!stream_eligible(shapes[i], M)) return false;
-    return true;
+        tiles += (shapes[i].N + 255) / 256;
+    }
+    return tiles <= kMaxTickets;
 }
 
 static size_t linear_ws_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {

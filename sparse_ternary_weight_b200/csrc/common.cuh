@@ -91,6 +91,13 @@ __device__ __forceinline__ float warp_tree_sum(const float* v, int n) {
     return __shfl_sync(kFull, x, 0);
 }
 
+// Linear workspaces start with a fixed region of split-K tickets, shared by
+// every decode kernel: tickets must be zero before a call and each call leaves
+// them zero; partial sums always live after this region, so calls that take
+// different kernels can share one workspace.
+constexpr size_t kTicketBytes = 256 * 1024;
+constexpr int kMaxTickets = (int)(kTicketBytes / sizeof(int));
+
 struct ProbShape {
     int64_t N, K;
     int granularity, group;

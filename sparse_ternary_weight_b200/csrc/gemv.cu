@@ -338,7 +338,7 @@ static Plan make_plan(const ProbShape* shapes, int count, int64_t M, int sms) {
         pl.probs.push_back(p);
     }
     pl.total_tiles = tb;
-    const size_t cnt_bytes = ((cnt_ints * sizeof(int) + 255) / 256) * 256;
+    const size_t cnt_bytes = kTicketBytes;
     pl.ws_bytes = cnt_ints ? cnt_bytes + part_floats * sizeof(float) : 0;
     // assign workspace slices
     size_t ci = 0, pf = 0;

@@ -303,6 +303,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
 
 bool stream_eligible(const ProbShape& s, int64_t M) {
     if (M != 1 || s.N == 0) return false;
+    if ((s.N + kSRows - 1) / kSRows > kMaxTickets) return false;
     if (s.K % 512 != 0) return false;
     if (s.granularity == SHERRY_PER_TENSOR || s.granularity == SHERRY_PER_CHANNEL) return true;
     if (s.granularity != SHERRY_PER_GROUP) return false;
@@ -343,9 +344,8 @@ static SPlan make_splan(const ProbShape* shapes, int count, int sms) {
     const int g = std::max(1, std::min(stream_ctas(sms), ub));
     pl.upc = (ub + g - 1) / g;
     pl.grid = (ub + pl.upc - 1) / pl.upc;
-    const size_t ticket_bytes = ((size_t)tb * sizeof(int) + 255) / 256 * 256;
-    pl.part_off = ticket_bytes;
-    pl.ws_bytes = ticket_bytes + (size_t)pl.grid * 2 * kSRows * sizeof(float);
+    pl.part_off = kTicketBytes;
+    pl.ws_bytes = kTicketBytes + (size_t)pl.grid * 2 * kSRows * sizeof(float);
     return pl;
 }
 
