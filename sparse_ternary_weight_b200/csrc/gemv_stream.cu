@@ -30,8 +30,8 @@
 
 namespace sherry {
 
-constexpr int kSThreads = 256;
-constexpr int kSRows = 256;                        // rows per unit, one per thread
+constexpr int kSThreads = 512;                     // 16 warps: 8 row-warps x 2 K-halves
+constexpr int kSRows = 256;                        // rows per unit, one per lane of a row-warp
 constexpr int kSWords = 32;                        // packed words per unit
 constexpr int kSStages = 3;
 constexpr int kSIdx = kSRows * kSWords * 4;        // 32 KB
@@ -88,9 +88,10 @@ __device__ __forceinline__ void issue_unit(const SParams<MAXP>& P, const UnitPos
     const int t = threadIdx.x;
     const int row0 = u.rb * kSRows;
     const int w0 = u.sub * kSWords;
-    // idx: 256 rows x 8 chunks of 16 B; chunk c of row r lands at chunk c ^ (r & 7)
+    // idx: 256 rows x 8 chunks of 16 B (8 consecutive threads read one 128-byte
+    // row segment); chunk c of row r lands at chunk c ^ (r & 7)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 4; ++i) {
         const int q = t + kSThreads * i;
         const int r = q >> 3, c = q & 7;
         const int row = row0 + r, word = w0 + 4 * c;
@@ -99,26 +100,20 @@ __device__ __forceinline__ void issue_unit(const SParams<MAXP>& P, const UnitPos
         cp_async16(stage + r * 128 + ((c ^ (r & 7)) << 4), src, ok);
     }
     // sgn: 256 rows x 2 chunks; chunk h of row r lands at h ^ ((r >> 2) & 1)
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int q = t + kSThreads * i;
-        const int r = q >> 1, h = q & 1;
+    {
+        const int r = t >> 1, h = t & 1;
         const int row = row0 + r, off = w0 + 16 * h;
         const bool ok = row < pr.N && off < pr.words;
         const uint8_t* src = ok ? pr.sgn + (int64_t)row * pr.words + off : pr.sgn;
         cp_async16(stage + kSIdx + r * 32 + ((h ^ ((r >> 2) & 1)) << 4), src, ok);
     }
     if (pr.mode == kSG128) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int q = t + kSThreads * i;
-            const int r = q >> 1, h = q & 1;
-            const int row = row0 + r, off = w0 / 4 + 4 * h;
-            const bool ok = row < pr.N && off < pr.spr;
-            const float* src = ok ? pr.scales + (int64_t)row * pr.spr + off : pr.scales;
-            cp_async16(stage + kSIdx + kSSgn + r * 32 + ((h ^ ((r >> 2) & 1)) << 4), src, ok);
-        }
-    } else if (pr.mode == kSG256) {
+        const int r = t >> 1, h = t & 1;
+        const int row = row0 + r, off = w0 / 4 + 4 * h;
+        const bool ok = row < pr.N && off < pr.spr;
+        const float* src = ok ? pr.scales + (int64_t)row * pr.spr + off : pr.scales;
+        cp_async16(stage + kSIdx + kSSgn + r * 32 + ((h ^ ((r >> 2) & 1)) << 4), src, ok);
+    } else if (pr.mode == kSG256 && t < kSRows) {
         const int r = t;
         const int row = row0 + r, off = w0 / 8;
         const bool ok = row < pr.N && off < pr.spr;
@@ -145,15 +140,81 @@ __device__ __forceinline__ void advance(const SProb* probs, UnitPos& u) {
     }
 }
 
+// Half of the 32-entry table of one block of 4 activations: the entries with
+// zero position z in {2h, 2h+1} and their negations.
+__device__ __forceinline__ void build_half_table(uint32_t tab, uint2 xb, int h) {
+    const float x0 = bf16lo(xb.x), x1 = bf16hi(xb.x), x2 = bf16lo(xb.y), x3 = bf16hi(xb.y);
+    // z = 2h: kept (h ? x0,x1,x3 : x1,x2,x3); z = 2h+1: kept (h ? x0,x1,x2 : x0,x2,x3)
+    const float a0 = h ? x0 : x1, b0 = h ? x1 : x2, c0 = x3;
+    const float a1 = x0, b1 = h ? x1 : x2, c1 = h ? x2 : x3;
+    const float s0 = a0 + b0, d0 = a0 - b0, s1 = a1 + b1, d1 = a1 - b1;
+    const float e0 = s0 + c0, e1 = s0 - c0, e2 = d0 + c0, e3 = d0 - c0;
+    const float e4 = s1 + c1, e5 = s1 - c1, e6 = d1 + c1, e7 = d1 - c1;
+    const uint32_t o = tab + 32 * h;
+    sts_v4(o, e0, e1, e2, e3);
+    sts_v4(o + 16, e4, e5, e6, e7);
+    sts_v4(o + 64, -e0, -e1, -e2, -e3);
+    sts_v4(o + 80, -e4, -e5, -e6, -e7);
+}
+
+// Lookups of one row over steps [4*kh, 4*kh + nst) of a unit (4 words each).
+template <int MODE>
+__device__ __forceinline__ float unit_rows(uint32_t st, uint32_t lut, int r, int kh, int nst) {
+    const uint32_t sw2 = ((r >> 2) & 1) << 4;
+    const uint4 sg = lds128(st + kSIdx + r * 32 + ((uint32_t)(kh << 4) ^ sw2));
+    uint4 av = make_uint4(0u, 0u, 0u, 0u);
+    if (MODE == kSG128) av = lds128(st + kSIdx + kSSgn + r * 32 + ((uint32_t)(kh << 4) ^ sw2));
+    if (MODE == kSG256) av = lds128(st + kSIdx + kSSgn + r * 32 + sw2);
+    const uint32_t idx_row = st + r * 128;
+    const uint32_t sw8 = (uint32_t)(r & 7);
+    float acc = 0.0f;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        if (cc < nst) {
+            const int c = 4 * kh + cc;
+            const uint4 wq = lds128(idx_row + (((uint32_t)c ^ sw8) << 4));
+            const uint32_t sq = cc == 0 ? sg.x : cc == 1 ? sg.y : cc == 2 ? sg.z : sg.w;
+            const uint32_t tb = lut + (uint32_t)(c * 32 * kTab);
+            float p0, p1, q0, q1, r0, r1, u0, u1;
+            word_pair_sum<0>(wq.x, sq & 0xffu, tb, p0, p1);
+            word_pair_sum<8>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
+            word_pair_sum<16>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
+            word_pair_sum<24>(wq.w, sq >> 24, tb, u0, u1);
+            add2(p0, p1, p0, p1, q0, q1);
+            add2(r0, r1, r0, r1, u0, u1);
+            add2(p0, p1, p0, p1, r0, r1);
+            const float s4 = p0 + p1;
+            if (MODE == kSRow) {
+                acc += s4;
+            } else {
+                uint32_t ab;
+                if (MODE == kSG128)
+                    ab = cc == 0 ? av.x : cc == 1 ? av.y : cc == 2 ? av.z : av.w;
+                else {
+                    const int gi = c >> 1;
+                    ab = gi == 0 ? av.x : gi == 1 ? av.y : gi == 2 ? av.z : av.w;
+                }
+                acc = fmaf(__uint_as_float(ab), s4, acc);
+            }
+        }
+    }
+    return acc;
+}
+
 template <int MAXP>
 __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_constant__ SParams<MAXP> P) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int s_last;
+    __shared__ float s_half[kSRows];
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t stages = base;
     const uint32_t luts = base + kSStages * kSStage;
 
     const int t = threadIdx.x;
+    const int lane = t & 31, warp = t >> 5;
+    const int r = (warp & 7) * 32 + lane;  // row within the unit
+    const int kh = warp >> 3;              // K half of the unit: steps 4kh .. 4kh+3
+    const int tb_idx = t & 255, tb_half = t >> 8;  // table-building role
     const int u_begin = blockIdx.x * P.upc;
     const int u_end = min(P.total_units, u_begin + P.upc);
     if (u_begin >= u_end) return;
@@ -168,24 +229,19 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         cp_async_commit();
     }
     UnitPos cur = locate(P, u_begin);
-    // tables of the first unit
     {
         const SProb& pr = P.p[cur.p];
-        const int b = cur.sub * kSWords * 8 + t;
-        if (b < pr.words * 8) build_table(luts + t * kTab, __ldg(reinterpret_cast<const uint2*>(pr.X) + b));
+        const int b = cur.sub * kSWords * 8 + tb_idx;
+        if (b < pr.words * 8)
+            build_half_table(luts + tb_idx * kTab, __ldg(reinterpret_cast<const uint2*>(pr.X) + b), tb_half);
     }
-    // first unit of the current tile covered by this CTA?
-    const int tile_start_unit0 = P.p[cur.p].unit_begin + cur.rb * P.p[cur.p].n_sub;
-    bool tile_from_start = (tile_start_unit0 == u_begin);
-
-    const int r = t;  // row within the unit
+    bool tile_from_start = (P.p[cur.p].unit_begin + cur.rb * P.p[cur.p].n_sub == u_begin);
     float acc = 0.0f;
 
     for (int u = u_begin; u < u_end; ++u) {
         const int k = u - u_begin;
         cp_async_wait<kSStages - 2>();
         __syncthreads();
-        // refill the stage freed by the previous unit
         if (u + kSStages - 1 < u_end) issue_unit(P, pre, stages + ((k + kSStages - 1) % kSStages) * kSStage);
         cp_async_commit();
         if (u + kSStages - 1 < u_end) advance(P.p, pre);
@@ -197,7 +253,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         bool xn_ok = false;
         if (u + 1 < u_end) {
             const SProb& pn = P.p[nxt.p];
-            const int b = nxt.sub * kSWords * 8 + t;
+            const int b = nxt.sub * kSWords * 8 + tb_idx;
             xn_ok = b < pn.words * 8;
             if (xn_ok) xn = __ldg(reinterpret_cast<const uint2*>(pn.X) + b);
         }
@@ -205,55 +261,27 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         const SProb& pr = P.p[cur.p];
         const uint32_t st = stages + (k % kSStages) * kSStage;
         const uint32_t lut = luts + (k & 1) * kSLut;
-        const int nsteps = min(8, (pr.words - cur.sub * kSWords) >> 2);
-        const uint32_t sgn_row = st + kSIdx + r * 32;
-        const uint32_t sw2 = ((r >> 2) & 1) << 4;
-        const uint4 sg0 = lds128(sgn_row + sw2);
-        const uint4 sg1 = lds128(sgn_row + (16u ^ sw2));
-        uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
-        if (pr.mode != kSRow) {
-            a0 = lds128(st + kSIdx + kSSgn + r * 32 + sw2);
-            if (pr.mode == kSG128) a1 = lds128(st + kSIdx + kSSgn + r * 32 + (16u ^ sw2));
-        }
-        const uint32_t idx_row = st + r * 128;
-        const uint32_t sw8 = (uint32_t)(r & 7);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            if (c < nsteps) {
-                const uint4 wq = lds128(idx_row + ((c ^ sw8) << 4));
-                const uint4& sgv = c < 4 ? sg0 : sg1;
-                const uint32_t sq = (c & 3) == 0 ? sgv.x : (c & 3) == 1 ? sgv.y : (c & 3) == 2 ? sgv.z : sgv.w;
-                const uint32_t tb = lut + (uint32_t)(c * 32 * kTab);
-                float ws[4][1];
-                word_lookups<1>(wq.x, sq & 0xffu, tb, 0, 0, ws[0]);
-                word_lookups<1>(wq.y, (sq >> 8) & 0xffu, tb, 8, 0, ws[1]);
-                word_lookups<1>(wq.z, (sq >> 16) & 0xffu, tb, 16, 0, ws[2]);
-                word_lookups<1>(wq.w, sq >> 24, tb, 24, 0, ws[3]);
-                const float s4 = (ws[0][0] + ws[1][0]) + (ws[2][0] + ws[3][0]);
-                if (pr.mode == kSRow) {
-                    acc += s4;
-                } else {
-                    uint32_t ab;
-                    if (pr.mode == kSG128) {
-                        const uint4& av = c < 4 ? a0 : a1;
-                        ab = (c & 3) == 0 ? av.x : (c & 3) == 1 ? av.y : (c & 3) == 2 ? av.z : av.w;
-                    } else {
-                        ab = (c >> 1) == 0 ? a0.x : (c >> 1) == 1 ? a0.y : (c >> 1) == 2 ? a0.z : a0.w;
-                    }
-                    acc = fmaf(__uint_as_float(ab), s4, acc);
-                }
-            }
+        const int nst = min(4, ((pr.words - cur.sub * kSWords) >> 2) - 4 * kh);
+        if (nst > 0) {
+            if (pr.mode == kSRow)
+                acc += unit_rows<kSRow>(st, lut, r, kh, nst);
+            else if (pr.mode == kSG128)
+                acc += unit_rows<kSG128>(st, lut, r, kh, nst);
+            else
+                acc += unit_rows<kSG256>(st, lut, r, kh, nst);
         }
 
-        // tile (row block) finished by this unit, or this CTA's range ends inside it
         const bool tile_end = (cur.sub == pr.n_sub - 1);
         if (tile_end || u == u_end - 1) {
+            // the two K halves of each row, in a fixed order
+            if (kh == 1) s_half[r] = acc;
+            __syncthreads();
             const int n = cur.rb * kSRows + r;
             const bool row_ok = n < pr.N;
-            float v = acc;
+            float v = acc + s_half[r];
             if (pr.mode == kSRow && row_ok) v *= __ldg(pr.scales + (pr.per_tensor ? 0 : n));
             if (tile_from_start && tile_end) {
-                if (row_ok) {
+                if (kh == 0 && row_ok) {
                     if (P.y_bf16)
                         reinterpret_cast<__nv_bfloat16*>(pr.Y)[n] = __float2bfloat16_rn(v);
                     else
@@ -266,12 +294,12 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                 const int c_a = tile_u0 / P.upc;
                 const int c_b = (tile_u0 + pr.n_sub - 1) / P.upc;
                 const int slot = (u_begin >= tile_u0) ? 0 : 1;
-                __stcg(P.part + ((int64_t)blockIdx.x * 2 + slot) * kSRows + r, v);
+                if (kh == 0) __stcg(P.part + ((int64_t)blockIdx.x * 2 + slot) * kSRows + r, v);
                 __threadfence();
                 __syncthreads();
                 if (t == 0) s_last = (atomicAdd(P.ticket + tile, 1) == c_b - c_a);
                 __syncthreads();
-                if (s_last) {
+                if (s_last && kh == 0) {
                     __threadfence();
                     float sum = 0.0f;
                     for (int c = c_a; c <= c_b; ++c) {
@@ -293,7 +321,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         }
 
         // tables of the next unit into the other buffer (its last reader was unit u-1)
-        if (u + 1 < u_end && xn_ok) build_table(luts + ((k + 1) & 1) * kSLut + t * kTab, xn);
+        if (u + 1 < u_end && xn_ok) build_half_table(luts + ((k + 1) & 1) * kSLut + tb_idx * kTab, xn, tb_half);
         cur = nxt;
     }
     cp_async_wait<0>();
