@@ -167,6 +167,11 @@ int sherry_unpack(const uint32_t* idx, const uint8_t* sgn, const float* scales,
 const char* sherry_status_string(int status);
 /* cudaError_t value behind the last SHERRY_ERR_CUDA returned on this thread */
 int sherry_last_cuda_error(void);
+/* Synchronises `stream`, then returns SHERRY_ERR_TIMEOUT if a bounded device
+ * wait of a tensor-core kernel gave up since the previous query (its outputs are
+ * then invalid), else SHERRY_OK; clears the flag.  SHERRY_ERR_CUDA if the
+ * synchronisation fails. */
+int sherry_device_status(void* stream);
 /* library version, e.g. 0x000100 = 0.1.0 */
 int sherry_version(void);
 

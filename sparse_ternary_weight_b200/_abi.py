@@ -38,6 +38,7 @@ SIGNATURES = {
     "sherry_unpack": (i32, [vp, vp, vp, i64, i64, i32, i32, vp, vp]),
     "sherry_status_string": (ctypes.c_char_p, [i32]),
     "sherry_last_cuda_error": (i32, []),
+    "sherry_device_status": (i32, [vp]),
     "sherry_version": (i32, []),
 }
 

@@ -60,12 +60,14 @@ static bool use_stream(const ProbShape* shapes, int count, int64_t M) {
 }
 
 static size_t linear_ws_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
+    if (count == 1 && prefill_eligible(shapes[0], M)) return 0;
     if (use_stream(shapes, count, M)) return stream_workspace_bytes(shapes, count, sms);
     return lut_workspace_bytes(shapes, count, M, sms);
 }
 
 static int linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream) {
+    if (count == 1 && prefill_eligible(shapes[0], M)) return prefill_launch(shapes[0], descs[0], M, y_bf16, stream);
     if (use_stream(shapes, count, M))
         return stream_linear_launch(shapes, descs, count, y_bf16, workspace, sms, stream);
     return lut_linear_launch(shapes, descs, count, M, y_bf16, workspace, sms, stream);
@@ -80,6 +82,8 @@ extern "C" {
 int sherry_version(void) { return 0x000100; }
 
 int sherry_last_cuda_error(void) { return g_last_cuda_error; }
+
+int sherry_device_status(void* stream) { return device_status_take(static_cast<cudaStream_t>(stream)); }
 
 const char* sherry_status_string(int status) {
     switch (status) {

@@ -4,7 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/sherry.h"
+#include "sherry.h"
 
 namespace sherry {
 
@@ -112,6 +112,10 @@ int unpack_launch(const uint32_t* idx, const uint8_t* sgn, const float* scales, 
 size_t lut_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms);
 int lut_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M,
                       int y_bf16, void* workspace, int sms, cudaStream_t stream);
+// tensor-core prefill kernel (prefill.cu)
+bool prefill_eligible(const ProbShape& s, int64_t M);
+int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, int y_bf16, cudaStream_t stream);
+int device_status_take(cudaStream_t stream);
 // one-token streaming kernel (gemv_stream.cu)
 bool stream_eligible(const ProbShape& s, int64_t M);
 size_t stream_workspace_bytes(const ProbShape* shapes, int count, int sms);

@@ -39,7 +39,8 @@ constexpr int kSSgn = kSRows * kSWords;            // 8 KB
 constexpr int kSSc = kSRows * 32;                  // 8 KB (at most 8 fp32 scales per row)
 constexpr int kSStage = kSIdx + kSSgn + kSSc;      // 48 KB
 constexpr int kSLut = 256 * kTab;                  // 36 KB, one table per block of the unit
-constexpr int kSSmem = kSStages * kSStage + 2 * kSLut + 1024;
+constexpr int kSSmem = kSStages * kSStage + 2 * kSLut + 256;
+static_assert(kSStage % 256 == 0 && kSLut % 256 == 0, "table bases must stay multiples of 256");
 
 enum SMode { kSRow = 0, kSG128 = 1, kSG256 = 2 };
 
@@ -71,10 +72,30 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+extern __shared__ __align__(16) unsigned char g_smem[];
+
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
     return v;
+}
+
+// 8 lookups of one packed word (tables of blocks BOFF..BOFF+7 at shared address
+// `base`, a multiple of 256) -> even-position and odd-position partial sums
+template <int BOFF>
+__device__ __forceinline__ void word_sums(uint32_t w, uint32_t s, uint32_t base, float& p0, float& p1) {
+    uint32_t ev, od;
+    spread_word(w, s, ev, od);
+    const float v0 = lds_imm<(BOFF + 0) * kTab>(__byte_perm(ev, base, 0x7650u));
+    const float v1 = lds_imm<(BOFF + 1) * kTab>(__byte_perm(od, base, 0x7650u));
+    const float v2 = lds_imm<(BOFF + 2) * kTab>(__byte_perm(ev, base, 0x7651u));
+    const float v3 = lds_imm<(BOFF + 3) * kTab>(__byte_perm(od, base, 0x7651u));
+    const float v4 = lds_imm<(BOFF + 4) * kTab>(__byte_perm(ev, base, 0x7652u));
+    const float v5 = lds_imm<(BOFF + 5) * kTab>(__byte_perm(od, base, 0x7652u));
+    const float v6 = lds_imm<(BOFF + 6) * kTab>(__byte_perm(ev, base, 0x7653u));
+    const float v7 = lds_imm<(BOFF + 7) * kTab>(__byte_perm(od, base, 0x7653u));
+    p0 = (v0 + v2) + (v4 + v6);
+    p1 = (v1 + v3) + (v5 + v7);
 }
 
 struct UnitPos {
@@ -88,37 +109,37 @@ __device__ __forceinline__ void issue_unit(const SParams<MAXP>& P, const UnitPos
     const int t = threadIdx.x;
     const int row0 = u.rb * kSRows;
     const int w0 = u.sub * kSWords;
-    // idx: 256 rows x 8 chunks of 16 B (8 consecutive threads read one 128-byte
-    // row segment); chunk c of row r lands at chunk c ^ (r & 7)
+    const int words = pr.words, N = pr.N;
+    {
+        const int r0 = t >> 3, c = t & 7;
+        const int word = w0 + 4 * c;
+        const bool wok = word < words;
+        const uint32_t* src = pr.idx + (int64_t)(row0 + r0) * words + word;
+        const int64_t stepw = (int64_t)64 * words;
+        uint32_t dst = stage + r0 * 128 + ((c ^ (r0 & 7)) << 4);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int q = t + kSThreads * i;
-        const int r = q >> 3, c = q & 7;
-        const int row = row0 + r, word = w0 + 4 * c;
-        const bool ok = row < pr.N && word < pr.words;
-        const uint32_t* src = ok ? pr.idx + (int64_t)row * pr.words + word : pr.idx;
-        cp_async16(stage + r * 128 + ((c ^ (r & 7)) << 4), src, ok);
+        for (int i = 0; i < 4; ++i) {
+            const bool ok = wok && (row0 + r0 + 64 * i) < N;
+            cp_async16(dst + i * 64 * 128, ok ? src + i * stepw : pr.idx, ok);
+        }
     }
-    // sgn: 256 rows x 2 chunks; chunk h of row r lands at h ^ ((r >> 2) & 1)
     {
         const int r = t >> 1, h = t & 1;
         const int row = row0 + r, off = w0 + 16 * h;
-        const bool ok = row < pr.N && off < pr.words;
-        const uint8_t* src = ok ? pr.sgn + (int64_t)row * pr.words + off : pr.sgn;
-        cp_async16(stage + kSIdx + r * 32 + ((h ^ ((r >> 2) & 1)) << 4), src, ok);
+        const bool ok = row < N && off < words;
+        cp_async16(stage + kSIdx + r * 32 + ((h ^ ((r >> 2) & 1)) << 4), ok ? pr.sgn + (int64_t)row * words + off : pr.sgn, ok);
+        if (pr.mode == kSG128) {
+            const int offs = w0 / 4 + 4 * h;
+            const bool oks = row < N && offs < pr.spr;
+            cp_async16(stage + kSIdx + kSSgn + r * 32 + ((h ^ ((r >> 2) & 1)) << 4),
+                       oks ? pr.scales + (int64_t)row * pr.spr + offs : pr.scales, oks);
+        }
     }
-    if (pr.mode == kSG128) {
-        const int r = t >> 1, h = t & 1;
-        const int row = row0 + r, off = w0 / 4 + 4 * h;
-        const bool ok = row < pr.N && off < pr.spr;
-        const float* src = ok ? pr.scales + (int64_t)row * pr.spr + off : pr.scales;
-        cp_async16(stage + kSIdx + kSSgn + r * 32 + ((h ^ ((r >> 2) & 1)) << 4), src, ok);
-    } else if (pr.mode == kSG256 && t < kSRows) {
+    if (pr.mode == kSG256 && t < kSRows) {
         const int r = t;
         const int row = row0 + r, off = w0 / 8;
-        const bool ok = row < pr.N && off < pr.spr;
-        const float* src = ok ? pr.scales + (int64_t)row * pr.spr + off : pr.scales;
-        cp_async16(stage + kSIdx + kSSgn + r * 32 + (((r >> 2) & 1) << 4), src, ok);
+        const bool ok = row < N && off < pr.spr;
+        cp_async16(stage + kSIdx + kSSgn + r * 32 + (((r >> 2) & 1) << 4), ok ? pr.scales + (int64_t)row * pr.spr + off : pr.scales, ok);
     }
 }
 
@@ -157,8 +178,9 @@ __device__ __forceinline__ void build_half_table(uint32_t tab, uint2 xb, int h) 
     sts_v4(o + 80, -e4, -e5, -e6, -e7);
 }
 
-// Lookups of one row over steps [4*kh, 4*kh + nst) of a unit (4 words each).
-template <int MODE>
+// Lookups of one row over steps [4*kh, 4*kh + nst) of a unit (4 words each);
+// `st` and `lut` are byte offsets into the dynamic shared buffer.
+template <int MODE, bool FULL>
 __device__ __forceinline__ float unit_rows(uint32_t st, uint32_t lut, int r, int kh, int nst) {
     const uint32_t sw2 = ((r >> 2) & 1) << 4;
     const uint4 sg = lds128(st + kSIdx + r * 32 + ((uint32_t)(kh << 4) ^ sw2));
@@ -170,20 +192,17 @@ __device__ __forceinline__ float unit_rows(uint32_t st, uint32_t lut, int r, int
     float acc = 0.0f;
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-        if (cc < nst) {
+        if (FULL || cc < nst) {
             const int c = 4 * kh + cc;
             const uint4 wq = lds128(idx_row + (((uint32_t)c ^ sw8) << 4));
             const uint32_t sq = cc == 0 ? sg.x : cc == 1 ? sg.y : cc == 2 ? sg.z : sg.w;
             const uint32_t tb = lut + (uint32_t)(c * 32 * kTab);
             float p0, p1, q0, q1, r0, r1, u0, u1;
-            word_pair_sum<0>(wq.x, sq & 0xffu, tb, p0, p1);
-            word_pair_sum<8>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
-            word_pair_sum<16>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
-            word_pair_sum<24>(wq.w, sq >> 24, tb, u0, u1);
-            add2(p0, p1, p0, p1, q0, q1);
-            add2(r0, r1, r0, r1, u0, u1);
-            add2(p0, p1, p0, p1, r0, r1);
-            const float s4 = p0 + p1;
+            word_sums<0>(wq.x, sq & 0xffu, tb, p0, p1);
+            word_sums<8>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
+            word_sums<16>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
+            word_sums<24>(wq.w, sq >> 24, tb, u0, u1);
+            const float s4 = ((p0 + q0) + (r0 + u0)) + ((p1 + q1) + (r1 + u1));
             if (MODE == kSRow) {
                 acc += s4;
             } else {
@@ -201,14 +220,20 @@ __device__ __forceinline__ float unit_rows(uint32_t st, uint32_t lut, int r, int
     return acc;
 }
 
+template <int MODE>
+__device__ __forceinline__ float unit_rows_any(uint32_t st, uint32_t lut, int r, int kh, int nst) {
+    return nst == 4 ? unit_rows<MODE, true>(st, lut, r, kh, 4) : unit_rows<MODE, false>(st, lut, r, kh, nst);
+}
+
 template <int MAXP>
 __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_constant__ SParams<MAXP> P) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int s_last;
     __shared__ float s_half[kSRows];
-    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    const uint32_t stages = base;
-    const uint32_t luts = base + kSStages * kSStage;
+    // Shared addresses: the buffer is rounded up to 256 bytes, so every table
+    // base is a multiple of 256 (a lookup's address replaces its low byte); the
+    // XOR swizzles need only 16-byte alignment, since writer and reader apply them.
+    const uint32_t stages = (smem_u32(g_smem) + 255u) & ~255u;
+    const uint32_t luts = stages + kSStages * kSStage;
 
     const int t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5;
@@ -242,7 +267,8 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         const int k = u - u_begin;
         cp_async_wait<kSStages - 2>();
         __syncthreads();
-        if (u + kSStages - 1 < u_end) issue_unit(P, pre, stages + ((k + kSStages - 1) % kSStages) * kSStage);
+        if (u + kSStages - 1 < u_end)
+            issue_unit(P, pre, stages + ((k + kSStages - 1) % kSStages) * kSStage);
         cp_async_commit();
         if (u + kSStages - 1 < u_end) advance(P.p, pre);
 
@@ -264,11 +290,11 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         const int nst = min(4, ((pr.words - cur.sub * kSWords) >> 2) - 4 * kh);
         if (nst > 0) {
             if (pr.mode == kSRow)
-                acc += unit_rows<kSRow>(st, lut, r, kh, nst);
+                acc += unit_rows_any<kSRow>(st, lut, r, kh, nst);
             else if (pr.mode == kSG128)
-                acc += unit_rows<kSG128>(st, lut, r, kh, nst);
+                acc += unit_rows_any<kSG128>(st, lut, r, kh, nst);
             else
-                acc += unit_rows<kSG256>(st, lut, r, kh, nst);
+                acc += unit_rows_any<kSG256>(st, lut, r, kh, nst);
         }
 
         const bool tile_end = (cur.sub == pr.n_sub - 1);

@@ -1,0 +1,402 @@
+// prefill.cu -- packed 3:4 ternary linear for many tokens on the 5th-generation
+// tensor cores (tcgen05 + TMEM), Y = X (T alpha)^T ("Sherry: Hardware-Efficient
+// 1.25-Bit Ternary Quantization via Fine-grained Sparsification", digest: Y = X
+// T alpha; "Sherry, Tequila and Fairies in Python" section 1.1: F.linear).
+//
+// With many tokens the layer is a dense contraction, so the packed weights are
+// expanded to bf16 {-1, 0, +1} tiles in shared memory and multiplied on the
+// tensor cores; alpha cannot be folded into the bf16 tile without losing
+// precision, so each K-group is accumulated separately in TMEM and promoted
+// into fp32 registers with alpha (per-row scales: once at the end).
+//
+// CTA tile: 128 weight rows (MMA M, TMEM lanes) x 128 tokens (MMA N, TMEM
+// columns); K in steps of 64 (one 128-byte swizzle atom of bf16).
+//   warps 0-3  epilogue: wait for a finished group accumulator, tcgen05.ld it,
+//              acc[token] += alpha(row, group) * D; write Y (row per thread)
+//   warps 4-7  decode: expand the packed words of one row per thread into the
+//              SWIZZLE_128B K-major A stage (bf16 +-1/0)
+//   warp 8     TMA: X tiles [128 tokens x 64 K] into the B stage (no multicast)
+//   warp 9     TMEM allocation; one elected thread issues tcgen05.mma
+// Every mbarrier wait is bounded; on timeout the CTA sets a device status flag
+// and drains instead of hanging.
+#include "common.cuh"
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+namespace sherry {
+
+constexpr int kPThreads = 320;
+constexpr int kPBM = 128;     // weight rows per tile
+constexpr int kPBN = 128;     // tokens per tile
+constexpr int kPBK = 64;      // K per stage
+constexpr int kPStages = 4;
+constexpr int kPStageA = kPBM * kPBK * 2;  // 16 KB
+constexpr int kPStageB = kPBN * kPBK * 2;  // 16 KB
+constexpr int kPSmem = kPStages * (kPStageA + kPStageB) + 1024 + 256;
+constexpr int kPTmemCols = 256;            // two 128-column accumulators
+constexpr long long kPWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+
+__device__ int g_device_status = 0;
+
+struct PParams {
+    const uint32_t* idx;
+    const uint8_t* sgn;
+    const float* scales;
+    void* Y;
+    int M, N, K, words;
+    int y_bf16;
+    int row_scale, per_tensor, spr;
+    int group_steps;  // K-steps per scale group (per-row: all of K)
+};
+
+// ---- PTX wrappers -------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// bounded wait: false if it gave up (or another thread of the CTA did)
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kPWaitCycles) {
+            *abort_flag = 1;
+            atomicExch(&g_device_status, SHERRY_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(map), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// K-major, 128-byte swizzled operand: 8-row atoms of 1024 bytes
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3fff);        // start address
+    d |= (uint64_t)1 << 16;                       // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;             // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                       // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;                       // SWIZZLE_128B
+    return d;
+}
+
+// bf16 x bf16 -> fp32, both K-major, M = 128, N = 128
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kPBN >> 3) << 17) |
+                            ((uint32_t)(kPBM >> 4) << 24);
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+#define SHERRY_TMEM_LD32(taddr, v)                                                                               \
+    asm volatile(                                                                                                \
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17," \
+        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                                       \
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),        \
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),  \
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),             \
+          "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),             \
+          "=r"(v[30]), "=r"(v[31])                                                                               \
+        : "r"(taddr))
+
+// bf16 {+1, 0, -1} of the 4 weights of a block: two packed halves
+__device__ __forceinline__ uint2 decode_block_bf16(uint32_t nib, uint32_t g) {
+    const uint32_t z = nib >> 2;
+    const uint32_t d1 = (nib >> 1) & 1u, d2 = nib & 1u;
+    const uint32_t k3 = g | ((g ^ d1) << 1) | ((g ^ d2) << 2);
+    const uint32_t negs = (k3 & ((1u << z) - 1u)) | ((k3 >> z) << (z + 1));
+    uint32_t h[4];
+#pragma unroll
+    for (uint32_t i = 0; i < 4; ++i) h[i] = (i == z) ? 0u : (0x3f80u | (((negs >> i) & 1u) << 15));
+    return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+}
+
+__global__ void __launch_bounds__(kPThreads, 1)
+k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PParams P) {
+    extern __shared__ __align__(1024) unsigned char psmem[];
+    __shared__ uint64_t bars[3 * kPStages + 4];
+    __shared__ uint32_t tmem_base_s;
+    __shared__ volatile int abort_s;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t base = (smem_u32(psmem) + 1023u) & ~1023u;
+    const uint32_t stA = base;                          // kPStages x 16 KB
+    const uint32_t stB = base + kPStages * kPStageA;    // kPStages x 16 KB
+    const uint32_t bar0 = smem_u32(&bars[0]);
+    auto full_a = [&](int s) { return bar0 + 8u * s; };
+    auto full_b = [&](int s) { return bar0 + 8u * (kPStages + s); };
+    auto empty = [&](int s) { return bar0 + 8u * (2 * kPStages + s); };
+    auto acc_full = [&](int b) { return bar0 + 8u * (3 * kPStages + b); };
+    auto acc_empty = [&](int b) { return bar0 + 8u * (3 * kPStages + 2 + b); };
+
+    const int n0 = blockIdx.x * kPBM;   // weight rows
+    const int m0 = blockIdx.y * kPBN;   // tokens
+    const int nk = P.K / kPBK;
+    const int gs = P.group_steps;
+    const int ngroups = nk / gs;
+
+    if (threadIdx.x == 0) {
+        abort_s = 0;
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(full_a(s), 128);
+            mbar_init(full_b(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(acc_full(b), 1);
+            mbar_init(acc_empty(b), 128);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
+                     "r"(kPTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+
+    if (warp < 4) {
+        // ---------------- epilogue: row n = n0 + 32*warp + lane ----------------
+        const int n = n0 + warp * 32 + lane;
+        const bool row_ok = n < P.N;
+        float acc[kPBN];
+#pragma unroll
+        for (int j = 0; j < kPBN; ++j) acc[j] = 0.0f;
+        bool ok = true;
+        for (int g = 0; g < ngroups && ok; ++g) {
+            const int b = g & 1;
+            ok = mbar_wait(acc_full(b), (uint32_t)((g >> 1) & 1), &abort_s);
+            if (!ok) break;
+            tc_fence_after();
+            float a = 1.0f;
+            if (!P.row_scale && row_ok) a = __ldg(P.scales + (int64_t)n * P.spr + g);  // group g = K-steps [g*gs, (g+1)*gs)
+            const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * kPBN);
+#pragma unroll
+            for (int c = 0; c < kPBN / 32; ++c) {
+                uint32_t v[32];
+                SHERRY_TMEM_LD32(t_row + c * 32, v);
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(a, __uint_as_float(v[j]), acc[c * 32 + j]);
+            }
+            tc_fence_before();
+            mbar_arrive(acc_empty(b));
+        }
+        if (ok && row_ok) {
+            float a = 1.0f;
+            if (P.row_scale) a = __ldg(P.scales + (P.per_tensor ? 0 : n));
+#pragma unroll
+            for (int j = 0; j < kPBN; ++j) {
+                const int m = m0 + j;
+                if (m < P.M) {
+                    const float y = acc[j] * a;
+                    if (P.y_bf16)
+                        reinterpret_cast<__nv_bfloat16*>(P.Y)[(int64_t)m * P.N + n] = __float2bfloat16_rn(y);
+                    else
+                        reinterpret_cast<float*>(P.Y)[(int64_t)m * P.N + n] = y;
+                }
+            }
+        }
+    } else if (warp < 8) {
+        // ---------------- decode: row i of the tile per thread ----------------
+        const int i = threadIdx.x - 128;
+        const int n = n0 + i;
+        const bool row_ok = n < P.N;
+        const uint32_t* idxr = P.idx + (int64_t)(row_ok ? n : 0) * P.words;
+        const uint8_t* sgnr = P.sgn + (int64_t)(row_ok ? n : 0) * P.words;
+        const uint32_t rowoff = (uint32_t)((i >> 3) * 1024 + (i & 7) * 128);
+        const uint32_t sw = (uint32_t)(i & 7);
+        uint2 wn = make_uint2(0u, 0u);
+        uint32_t sn = 0u;
+        if (row_ok && nk > 0) {
+            wn = __ldg(reinterpret_cast<const uint2*>(idxr));
+            sn = __ldg(reinterpret_cast<const uint16_t*>(sgnr));
+        }
+        for (int ks = 0; ks < nk; ++ks) {
+            const int s = ks % kPStages;
+            const uint2 w = wn;
+            const uint32_t sb = sn;
+            if (ks + 1 < nk && row_ok) {  // next step's words, loaded one step ahead
+                wn = __ldg(reinterpret_cast<const uint2*>(idxr + 2 * (ks + 1)));
+                sn = __ldg(reinterpret_cast<const uint16_t*>(sgnr + 2 * (ks + 1)));
+            }
+            if (!mbar_wait(empty(s), (uint32_t)(((ks / kPStages) & 1) ^ 1), &abort_s)) break;
+            const uint32_t dst = stA + s * kPStageA + rowoff;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {  // chunk c: blocks 2c, 2c+1 of this 64-weight step
+                const uint32_t word = c < 4 ? w.x : w.y;
+                const int b0 = 2 * (c & 3);
+                const uint2 lo = decode_block_bf16((word >> (4 * b0)) & 15u, (sb >> (2 * c)) & 1u);
+                const uint2 hi = decode_block_bf16((word >> (4 * b0 + 4)) & 15u, (sb >> (2 * c + 1)) & 1u);
+                const uint32_t o = dst + (((uint32_t)c ^ sw) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(o), "r"(row_ok ? lo.x : 0u),
+                             "r"(row_ok ? lo.y : 0u), "r"(row_ok ? hi.x : 0u), "r"(row_ok ? hi.y : 0u)
+                             : "memory");
+            }
+            fence_proxy_async();
+            mbar_arrive(full_a(s));
+        }
+    } else if (warp == 8) {
+        // ---------------- TMA producer for X ----------------
+        if (lane == 0) {
+            for (int ks = 0; ks < nk; ++ks) {
+                const int s = ks % kPStages;
+                if (!mbar_wait(empty(s), (uint32_t)(((ks / kPStages) & 1) ^ 1), &abort_s)) break;
+                mbar_expect_tx(full_b(s), kPStageB);
+                tma_load_2d(stB + s * kPStageB, &xmap, ks * kPBK, m0, full_b(s));
+            }
+        }
+    } else {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            for (int ks = 0; ks < nk; ++ks) {
+                const int s = ks % kPStages;
+                const int g = ks / gs;
+                const int b = g & 1;
+                const bool first = (ks % gs) == 0;
+                if (first && !mbar_wait(acc_empty(b), (uint32_t)(((g >> 1) & 1) ^ 1), &abort_s)) break;
+                if (!mbar_wait(full_a(s), (uint32_t)((ks / kPStages) & 1), &abort_s)) break;
+                if (!mbar_wait(full_b(s), (uint32_t)((ks / kPStages) & 1), &abort_s)) break;
+                tc_fence_after();
+                const uint64_t da = smem_desc(stA + s * kPStageA);
+                const uint64_t db = smem_desc(stB + s * kPStageB);
+#pragma unroll
+                for (int kk = 0; kk < kPBK / 16; ++kk)  // K = 16 per MMA: +32 bytes in the swizzled row
+                    mma_bf16(tmem + (uint32_t)(b * kPBN), da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk),
+                             (first && kk == 0) ? 0u : 1u);
+                mma_commit(empty(s));
+                if ((ks % gs) == gs - 1) mma_commit(acc_full(b));
+            }
+        }
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPTmemCols));
+    }
+}
+
+// ---- host side -------------------------------------------------------------------
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiled encode_fn() {
+    static EncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    });
+    return fn;
+}
+
+bool prefill_eligible(const ProbShape& s, int64_t M) {
+    if (M < 17 || s.N == 0) return false;
+    if (s.K % kPBK != 0) return false;
+    if (s.granularity == SHERRY_PER_GROUP && s.group % kPBK != 0) return false;
+    if (M > (int64_t)0x7fffffff / 2) return false;
+    return true;
+}
+
+int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, int y_bf16, cudaStream_t stream) {
+    EncodeTiled enc = encode_fn();
+    if (!enc) return SHERRY_ERR_UNSUPPORTED;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {(cuuint64_t)s.K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)s.K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kPBK, (cuuint32_t)kPBN};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(d.X), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return SHERRY_ERR_UNSUPPORTED;
+    PParams P{};
+    P.idx = d.idx;
+    P.sgn = d.sgn;
+    P.scales = d.scales;
+    P.Y = d.Y;
+    P.M = (int)M;
+    P.N = (int)s.N;
+    P.K = (int)s.K;
+    P.words = (int)(s.K / 32);
+    P.y_bf16 = y_bf16;
+    P.row_scale = s.granularity != SHERRY_PER_GROUP;
+    P.per_tensor = s.granularity == SHERRY_PER_TENSOR;
+    P.spr = s.granularity == SHERRY_PER_GROUP ? (int)(s.K / s.group) : 1;
+    P.group_steps = s.granularity == SHERRY_PER_GROUP ? s.group / kPBK : (int)(s.K / kPBK);
+    static bool attr = false;
+    static std::mutex mu;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!attr) {
+            SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
+            attr = true;
+        }
+    }
+    dim3 grid((unsigned)((s.N + kPBM - 1) / kPBM), (unsigned)((M + kPBN - 1) / kPBN));
+    k_prefill<<<grid, kPThreads, kPSmem, stream>>>(map, P);
+    SHERRY_LAUNCH_CHECK();
+    return SHERRY_OK;
+}
+
+int device_status_take(cudaStream_t stream) {
+    SHERRY_CUDA_CHECK(cudaStreamSynchronize(stream));
+    int v = 0;
+    SHERRY_CUDA_CHECK(cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)));
+    if (v) {
+        const int zero = 0;
+        SHERRY_CUDA_CHECK(cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)));
+    }
+    return v;
+}
+
+}  // namespace sherry

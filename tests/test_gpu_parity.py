@@ -251,3 +251,37 @@ def test_stream_batch_many_problems_vs_oracle(sw, orc):
     # single calls agree with the oracle as well
     for (X, P), (y_ref, Wq, Xb) in zip(pairs[:8], refs[:8]):
         check_linear(sw.linear(X, P).cpu().numpy(), y_ref, Xb, Wq)
+
+
+PREFILL_CASES = [
+    # (M, N, K, gran, group): M >= 17 runs the tcgen05 kernel
+    (17, 128, 64, "tensor", 0),
+    (128, 128, 128, "group", 128),
+    (129, 200, 256, "group", 64),
+    (300, 384, 3072, "group", 128),
+    (513, 129, 1024, "group", 256),
+    (64, 256, 2048, "channel", 0),
+    (40, 1000, 512, "group", 512),
+]
+
+
+@pytest.mark.parametrize("case", PREFILL_CASES, ids=lambda c: f"M{c[0]}-{c[1]}x{c[2]}-{c[3]}{c[4]}")
+def test_prefill_tensor_core_vs_oracle(sw, orc, case):
+    import torch
+    from sparse_ternary_weight_b200 import _abi
+    M, N, K, gname, group = case
+    gran = GRAN[gname]
+    W = _weights("t4", N, K, seed=7000 + N + K)
+    Xb = synth.activations_bf16(M, K, seed=8000 + M + K)
+    P = sw.quantize_pack(to_dev(W), gran, group)
+    idx, sgn, sc = packed_to_host(P)
+    y_ref = orc.linear(Xb, idx, sgn, sc, N, K, gran, group)
+    Wq = orc.unpack_f32(idx, sgn, sc, N, K, gran, group)
+    X = to_dev(Xb.view(np.int16)).view(torch.bfloat16)
+    y32 = sw.linear(X, P, torch.float32)
+    yb = sw.linear(X, P, torch.bfloat16)
+    assert _abi.lib().sherry_device_status(None) == 0
+    check_linear(y32.cpu().numpy(), y_ref, Xb, Wq)
+    check_linear(yb.float().cpu().numpy(), y_ref, Xb, Wq, y_is_bf16=True)
+    assert torch.equal(yb, y32.to(torch.bfloat16))
+    assert torch.equal(sw.linear(X, P, torch.float32), y32)
