@@ -155,6 +155,26 @@ int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M,
                           void* workspace, size_t workspace_bytes, void* stream);
 size_t sherry_linear_batched_workspace_bytes(const sherry_linear_desc* descs, int count, int64_t M);
 
+/* ---- packed linear without a workspace -------------------------------------
+ * No counterpart on the pages: this is a service for callers that cannot
+ * allocate device memory (a host framework that plans all memory ahead and
+ * hands a kernel only its inputs and outputs, a plugin interface without a
+ * scratch argument, a latency-critical path that must not enter the
+ * allocator).  Same arguments and result as sherry_linear, minus the
+ * workspace.  Its scratch is a fixed device array of
+ * SHERRY_NOALLOC_SCRATCH_BYTES inside the library, held by every GPU that loads
+ * the library until the process exits; a call that would need more returns
+ * SHERRY_ERR_WORKSPACE.  The first call on a device looks up the array's device
+ * address (make that first call before any stream capture).  Every call zeroes
+ * the array's ticket region on `stream` before its kernel and otherwise reuses
+ * what the previous call left; all calls share the one array, so calls that
+ * overlap on the GPU (other streams, other host threads) race -- keep them
+ * ordered.  Nothing is allocated or freed. */
+#define SHERRY_NOALLOC_SCRATCH_BYTES ((size_t)1 << 20)
+int sherry_linear_noalloc(const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                          const uint32_t* idx, const uint8_t* sgn, const float* scales,
+                          int granularity, int group, void* Y, int y_dtype, void* stream);
+
 /* ---- unpack ----------------------------------------------------------------
  * Dense bf16 W_out[n][k] = round_to_nearest_even(t[n][k] * alpha(n,k)); the
  * inverse of the 5-bit code (32 states, "Sherry: ..." digest) times the scale.

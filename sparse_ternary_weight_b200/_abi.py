@@ -16,6 +16,7 @@ F32, BF16 = 0, 1
 OP_QUANTIZE_PACK, OP_LINEAR, OP_UNPACK = 0, 1, 2
 MAX_K = 262144
 MAX_BATCH = 256
+NOALLOC_SCRATCH_BYTES = 1 << 20
 
 vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 
@@ -36,6 +37,7 @@ SIGNATURES = {
     "sherry_linear_batched": (i32, [ctypes.POINTER(LinearDesc), i32, i64, i32, vp, sz, vp]),
     "sherry_linear_batched_workspace_bytes": (sz, [ctypes.POINTER(LinearDesc), i32, i64]),
     "sherry_unpack": (i32, [vp, vp, vp, i64, i64, i32, i32, vp, vp]),
+    "sherry_linear_noalloc": (i32, [vp, i64, i64, i64, vp, vp, vp, i32, i32, vp, i32, vp]),
     "sherry_status_string": (ctypes.c_char_p, [i32]),
     "sherry_last_cuda_error": (i32, []),
     "sherry_device_status": (i32, [vp]),
