@@ -52,6 +52,22 @@ def stack_shapes(stack=STACK):
     return [(l, p, shp[p]) for l in range(layers) for p in synth.PROJ]
 
 
+def profiled_traffic(name):
+    """dram read+write bytes per launch recorded in a profiles/ summary (a line
+    `dram_bytes_per_launch: N` written from an ncu capture of the same kernel
+    build), or None when absent."""
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        if line.strip().startswith("dram_bytes_per_launch:"):
+            try:
+                return int(line.split(":", 1)[1].strip())
+            except ValueError:
+                return None
+    return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -260,14 +276,9 @@ def run_ours(args):
     # oracle check; the oracle check at full size lives in the test-suite)
     roof = {"bound": "hbm", "achieved": round(gbs_rank, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(gbs_rank / pk["hbm_gbs"], 4), "traffic": None,
-            "kernel": "k_lut_linear<1,8,256>", "peak_source": pk["source"],
+            "kernel": "k_lut_stream", "peak_source": pk["source"],
             "algorithmic_bytes_per_launch": step_bytes}
-    prof = os.path.join(ROOT, "profiles", "lut_linear_3b_decode_m1_traffic.json")
-    if os.path.exists(prof):
-        try:
-            roof["traffic"] = json.load(open(prof)).get("dram_bytes_per_launch")
-        except Exception:
-            pass
+    roof["traffic"] = profiled_traffic("lut_stream_3b_decode_m1.md")
 
     # ---------------- e2e: host buffers through the C ABI ----------------
     Ksum = sum(K for _, K in shapes)
@@ -374,6 +385,9 @@ def extra_rows(args, pairs, outs, shapes, ws, dev, pk):
                             "frac_hbm": round(b1 / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
     del p1, o1
 
+    # prefill on the tensor cores: the 3B stack (196 linears, one launch each, CUDA graph)
+    rows["prefill_3b"] = prefill_rows(args, pairs, ws, dev, pk, steps=max(2, args.steps // 10), warm=3)
+
     # quantize + pack of the full 3B weight set (fp32 in HBM), three granularities
     qp = {}
     cfg, layers, shp = synth.STACKS[STACK]
@@ -407,6 +421,45 @@ def extra_rows(args, pairs, outs, shapes, ws, dev, pk):
     del Ws
     torch.cuda.empty_cache()
     return rows
+
+
+def prefill_rows(args, pairs, ws, dev, pk, steps, warm):
+    """Dense-equivalent and nonzero TFLOP/s of the tensor-core prefill over the
+    3B stack at M = 512, 2048, 4096, for group-128 and per-channel scales."""
+    import torch
+    import sparse_ternary_weight_b200 as sw
+    from sparse_ternary_weight_b200 import synth
+    stream = torch.cuda.current_stream()
+    out = {}
+    packs = {"group128": [P for _, P in pairs]}
+    # per-channel copy of the same weights (device draws, same seeds)
+    chan = []
+    for (l, p, _) in stack_shapes():
+        W = synth.torch_stack_weight(STACK, l, p, device=dev)
+        chan.append(sw.quantize_pack(W, "per_channel"))
+        del W
+    packs["channel"] = chan
+    for M in (512, 2048, 4096):
+        # one activation block per distinct K (contents do not change the timing)
+        Xk = {K: synth.torch_activations_bf16(M, K, 900000 + K, device=dev) for K in {P.K for P in chan}}
+        Yn = {N: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for N in {P.N for P in chan}}
+        flops = sum(2.0 * M * P.N * P.K for P in chan)
+        for name, plist in packs.items():
+            def step():
+                for P in plist:
+                    sw.linear(Xk[P.K], P, torch.bfloat16, out=Yn[P.N])
+            g = graph_of(step)
+            ms = time_region(g.replay, steps, warm, ws, stream) / steps
+            tf = flops / (ms * 1e-3) / 1e12
+            out[f"M{M}_{name}"] = {"ms": round(ms, 3), "TFLOP/s_dense_equiv": round(ws * tf, 1),
+                                   "TFLOP/s_nonzero": round(ws * tf * 0.75, 1),
+                                   "frac_bf16_sustained": round(tf / pk["bf16_tflops_sustained"], 4),
+                                   "launches": len(plist)}
+            del g
+        del Xk, Yn
+    del chan, packs
+    torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------------------------------------
