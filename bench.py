@@ -547,6 +547,25 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def profile_prefill(args):
+    import torch
+    from sparse_ternary_weight_b200.build import build
+    build()
+    import sparse_ternary_weight_b200 as sw
+    from sparse_ternary_weight_b200 import synth
+    N, K, M = (int(v) for v in args.profile_prefill.split(","))
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(N + K)
+    P = sw.quantize_pack(torch.randn((N, K), generator=g, device=dev) * 0.02, "per_group", 128)
+    X = synth.torch_activations_bf16(M, K, 1, device=dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ms = time_region(lambda: sw.linear(X, P, torch.bfloat16, out=Y), args.steps, args.warmup, 1,
+                     torch.cuda.current_stream()) / args.steps
+    print(json.dumps({"prefill": f"{N}x{K} M={M}", "ms": round(ms, 4),
+                      "TFLOP/s_dense_equiv": round(2 * M * N * K / (ms * 1e-3) / 1e12, 1)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -558,7 +577,13 @@ def main():
     ap.add_argument("--cpu-layers", type=int, default=1)
     ap.add_argument("--layers", type=int, default=28, help="layers of the 3B stack (28 = the full workload; "
                     "fewer only for profiling captures)")
+    ap.add_argument("--profile-prefill", default=None, metavar="N,K,M",
+                    help="only run one tensor-core prefill linear (N x K weight, M tokens) warmup+steps times, "
+                         "print its time, and exit (for profiler captures)")
     args = ap.parse_args()
+    if args.profile_prefill:
+        profile_prefill(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -4,18 +4,21 @@
 // T alpha; "Sherry, Tequila and Fairies in Python" section 1.1: F.linear).
 //
 // With many tokens the layer is a dense contraction, so the packed weights are
-// expanded to bf16 {-1, 0, +1} tiles in shared memory and multiplied on the
-// tensor cores; alpha cannot be folded into the bf16 tile without losing
-// precision, so each K-group is accumulated separately in TMEM and promoted
-// into fp32 registers with alpha (per-row scales: once at the end).
+// expanded to bf16 {-1, 0, +1} and multiplied on the tensor cores; alpha cannot
+// be folded into the bf16 weights without losing precision, so each K-group is
+// accumulated separately in TMEM and promoted into fp32 registers with alpha
+// (per-row scales: once at the end).
 //
-// CTA tile: 128 weight rows (MMA M, TMEM lanes) x 128 tokens (MMA N, TMEM
-// columns); K in steps of 64 (one 128-byte swizzle atom of bf16).
+// CTA tile: 128 weight rows (MMA M, TMEM lanes) x 128 tokens (MMA N), K in
+// steps of 64.  The expanded weights (MMA operand A) never touch shared memory:
+// decode threads own one TMEM lane (= weight row) each and write their row's
+// 64 bf16 of a step into TMEM with tcgen05.st; only the X tiles (operand B)
+// come through shared memory, by TMA (no multicast).
 //   warps 0-3  epilogue: wait for a finished group accumulator, tcgen05.ld it,
 //              acc[token] += alpha(row, group) * D; write Y (row per thread)
-//   warps 4-7  decode: expand the packed words of one row per thread into the
-//              SWIZZLE_128B K-major A stage (bf16 +-1/0)
-//   warp 8     TMA: X tiles [128 tokens x 64 K] into the B stage (no multicast)
+//   warps 4-7  decode: per block one table lookup (32 bf16x4 patterns indexed by
+//              nibble + 16*sign) -> tcgen05.st into the A stage of their lanes
+//   warp 8     TMA: X tiles [128 tokens x 64 K], SWIZZLE_128B
 //   warp 9     TMEM allocation; one elected thread issues tcgen05.mma
 // Every mbarrier wait is bounded; on timeout the CTA sets a device status flag
 // and drains instead of hanging.
@@ -33,10 +36,12 @@ constexpr int kPBM = 128;     // weight rows per tile
 constexpr int kPBN = 128;     // tokens per tile
 constexpr int kPBK = 64;      // K per stage
 constexpr int kPStages = 4;
-constexpr int kPStageA = kPBM * kPBK * 2;  // 16 KB
-constexpr int kPStageB = kPBN * kPBK * 2;  // 16 KB
-constexpr int kPSmem = kPStages * (kPStageA + kPStageB) + 1024 + 256;
-constexpr int kPTmemCols = 256;            // two 128-column accumulators
+constexpr int kPStageB = kPBN * kPBK * 2;  // 16 KB of X per stage
+constexpr int kPTable = 256;               // 32 x 8-byte weight patterns
+constexpr int kPSmem = kPStages * kPStageB + kPTable + 1024;
+constexpr int kPTmemCols = 512;            // 2 x 128 accumulator columns + 4 x 32 A columns
+constexpr int kPAcol = 256;                // first TMEM column of the A stages
+constexpr int kPAcols = kPBK / 2;          // 32 columns (64 bf16) per A stage
 constexpr long long kPWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
 
 __device__ int g_device_status = 0;
@@ -115,12 +120,29 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kPBN >> 3) << 17) |
                             ((uint32_t)(kPBM >> 4) << 24);
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+// D (TMEM) += A (TMEM, lane = row, 2 bf16 per column) x B (shared, descriptor)
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(kIdesc), "r"(accumulate)
         : "memory");
+}
+
+#define SHERRY_TMEM_ST32(taddr, v)                                                                               \
+    asm volatile(                                                                                                \
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16," \
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),                        \
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),      \
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),          \
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),         \
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])                      \
+        : "memory")
+
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
@@ -158,8 +180,8 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t base = (smem_u32(psmem) + 1023u) & ~1023u;
-    const uint32_t stA = base;                          // kPStages x 16 KB
-    const uint32_t stB = base + kPStages * kPStageA;    // kPStages x 16 KB
+    const uint32_t stB = base;                             // kPStages x 16 KB, 1024-aligned
+    const uint32_t table = base + kPStages * kPStageB;     // 256-aligned
     const uint32_t bar0 = smem_u32(&bars[0]);
     auto full_a = [&](int s) { return bar0 + 8u * s; };
     auto full_b = [&](int s) { return bar0 + 8u * (kPStages + s); };
@@ -167,8 +189,10 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
     auto acc_full = [&](int b) { return bar0 + 8u * (3 * kPStages + b); };
     auto acc_empty = [&](int b) { return bar0 + 8u * (3 * kPStages + 2 + b); };
 
-    const int n0 = blockIdx.x * kPBM;   // weight rows
-    const int m0 = blockIdx.y * kPBN;   // tokens
+    // persistent: tile t = (weight-row tile t % ntn, token tile t / ntn), strided by the grid;
+    // stage and accumulator phases run on across tiles
+    const int ntn = (P.N + kPBM - 1) / kPBM;
+    const int ntiles = ntn * ((P.M + kPBN - 1) / kPBN);
     const int nk = P.K / kPBK;
     const int gs = P.group_steps;
     const int ngroups = nk / gs;
@@ -186,6 +210,11 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
         }
         fence_mbar_init();
     }
+    if (threadIdx.x < 32) {
+        // bf16 patterns of the 32 block codes: entry = nibble + 16 * sign bit
+        const uint2 e = decode_block_bf16((uint32_t)threadIdx.x & 15u, (uint32_t)threadIdx.x >> 4);
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(table + 8u * threadIdx.x), "r"(e.x), "r"(e.y) : "memory");
+    }
     if (warp == 9) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
                      "r"(kPTmemCols));
@@ -197,116 +226,148 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
     const uint32_t tmem = tmem_base_s;
 
     if (warp < 4) {
-        // ---------------- epilogue: row n = n0 + 32*warp + lane ----------------
-        const int n = n0 + warp * 32 + lane;
-        const bool row_ok = n < P.N;
-        float acc[kPBN];
-#pragma unroll
-        for (int j = 0; j < kPBN; ++j) acc[j] = 0.0f;
+        // ---------------- epilogue: row n = n0 + 32*warp + lane of each tile ----------------
         bool ok = true;
-        for (int g = 0; g < ngroups && ok; ++g) {
-            const int b = g & 1;
-            ok = mbar_wait(acc_full(b), (uint32_t)((g >> 1) & 1), &abort_s);
-            if (!ok) break;
-            tc_fence_after();
-            float a = 1.0f;
-            if (!P.row_scale && row_ok) a = __ldg(P.scales + (int64_t)n * P.spr + g);  // group g = K-steps [g*gs, (g+1)*gs)
-            const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * kPBN);
+        int gc = 0;  // groups consumed so far (all tiles)
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const int n = (t % ntn) * kPBM + warp * 32 + lane;
+            const int m0 = (t / ntn) * kPBN;
+            const bool row_ok = n < P.N;
+            float acc[kPBN];
 #pragma unroll
-            for (int c = 0; c < kPBN / 32; ++c) {
-                uint32_t v[32];
-                SHERRY_TMEM_LD32(t_row + c * 32, v);
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            for (int j = 0; j < kPBN; ++j) acc[j] = 0.0f;
+            for (int g = 0; g < ngroups; ++g, ++gc) {
+                const int b = gc & 1;
+                ok = mbar_wait(acc_full(b), (uint32_t)((gc >> 1) & 1), &abort_s);
+                if (!ok) break;
+                tc_fence_after();
+                float a = 1.0f;
+                if (!P.row_scale && row_ok) a = __ldg(P.scales + (int64_t)n * P.spr + g);  // group g: K-steps [g*gs, (g+1)*gs)
+                const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * kPBN);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(a, __uint_as_float(v[j]), acc[c * 32 + j]);
+                for (int c = 0; c < kPBN / 32; ++c) {
+                    uint32_t v[32];
+                    SHERRY_TMEM_LD32(t_row + c * 32, v);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(a, __uint_as_float(v[j]), acc[c * 32 + j]);
+                }
+                tc_fence_before();
+                mbar_arrive(acc_empty(b));
             }
-            tc_fence_before();
-            mbar_arrive(acc_empty(b));
-        }
-        if (ok && row_ok) {
-            float a = 1.0f;
-            if (P.row_scale) a = __ldg(P.scales + (P.per_tensor ? 0 : n));
+            if (ok && row_ok) {
+                float a = 1.0f;
+                if (P.row_scale) a = __ldg(P.scales + (P.per_tensor ? 0 : n));
 #pragma unroll
-            for (int j = 0; j < kPBN; ++j) {
-                const int m = m0 + j;
-                if (m < P.M) {
-                    const float y = acc[j] * a;
-                    if (P.y_bf16)
-                        reinterpret_cast<__nv_bfloat16*>(P.Y)[(int64_t)m * P.N + n] = __float2bfloat16_rn(y);
-                    else
-                        reinterpret_cast<float*>(P.Y)[(int64_t)m * P.N + n] = y;
+                for (int j = 0; j < kPBN; ++j) {
+                    const int m = m0 + j;
+                    if (m < P.M) {
+                        const float y = acc[j] * a;
+                        if (P.y_bf16)
+                            reinterpret_cast<__nv_bfloat16*>(P.Y)[(int64_t)m * P.N + n] = __float2bfloat16_rn(y);
+                        else
+                            reinterpret_cast<float*>(P.Y)[(int64_t)m * P.N + n] = y;
+                    }
                 }
             }
         }
     } else if (warp < 8) {
-        // ---------------- decode: row i of the tile per thread ----------------
-        const int i = threadIdx.x - 128;
-        const int n = n0 + i;
-        const bool row_ok = n < P.N;
-        const uint32_t* idxr = P.idx + (int64_t)(row_ok ? n : 0) * P.words;
-        const uint8_t* sgnr = P.sgn + (int64_t)(row_ok ? n : 0) * P.words;
-        const uint32_t rowoff = (uint32_t)((i >> 3) * 1024 + (i & 7) * 128);
-        const uint32_t sw = (uint32_t)(i & 7);
-        uint2 wn = make_uint2(0u, 0u);
-        uint32_t sn = 0u;
-        if (row_ok && nk > 0) {
-            wn = __ldg(reinterpret_cast<const uint2*>(idxr));
-            sn = __ldg(reinterpret_cast<const uint16_t*>(sgnr));
-        }
-        for (int ks = 0; ks < nk; ++ks) {
-            const int s = ks % kPStages;
-            const uint2 w = wn;
-            const uint32_t sb = sn;
-            if (ks + 1 < nk && row_ok) {  // next step's words, loaded one step ahead
-                wn = __ldg(reinterpret_cast<const uint2*>(idxr + 2 * (ks + 1)));
-                sn = __ldg(reinterpret_cast<const uint16_t*>(sgnr + 2 * (ks + 1)));
+        // ---------------- decode: TMEM lane (= tile row) i per thread ----------------
+        const int q = warp - 4;                 // lane quarter of this warp
+        const int i = q * 32 + lane;
+        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kPAcol;
+        int kc = 0;  // K-steps produced so far (all tiles)
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const int n = (t % ntn) * kPBM + i;
+            const bool row_ok = n < P.N;
+            const uint32_t* idxr = P.idx + (int64_t)(row_ok ? n : 0) * P.words;
+            const uint8_t* sgnr = P.sgn + (int64_t)(row_ok ? n : 0) * P.words;
+            uint2 wn = make_uint2(0u, 0u);
+            uint32_t sn = 0u;
+            if (row_ok) {
+                wn = __ldg(reinterpret_cast<const uint2*>(idxr));
+                sn = __ldg(reinterpret_cast<const uint16_t*>(sgnr));
             }
-            if (!mbar_wait(empty(s), (uint32_t)(((ks / kPStages) & 1) ^ 1), &abort_s)) break;
-            const uint32_t dst = stA + s * kPStageA + rowoff;
+            for (int ks = 0; ks < nk; ++ks, ++kc) {
+                const int s = kc % kPStages;
+                const uint2 w = wn;
+                const uint32_t sb = sn;
+                if (ks + 1 < nk && row_ok) {  // next step's words, loaded one step ahead
+                    wn = __ldg(reinterpret_cast<const uint2*>(idxr + 2 * (ks + 1)));
+                    sn = __ldg(reinterpret_cast<const uint16_t*>(sgnr + 2 * (ks + 1)));
+                }
+                // table offsets (8 * (nibble + 16 G)) of the even / odd blocks of each word
+                uint32_t v[32];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {  // chunk c: blocks 2c, 2c+1 of this 64-weight step
-                const uint32_t word = c < 4 ? w.x : w.y;
-                const int b0 = 2 * (c & 3);
-                const uint2 lo = decode_block_bf16((word >> (4 * b0)) & 15u, (sb >> (2 * c)) & 1u);
-                const uint2 hi = decode_block_bf16((word >> (4 * b0 + 4)) & 15u, (sb >> (2 * c + 1)) & 1u);
-                const uint32_t o = dst + (((uint32_t)c ^ sw) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(o), "r"(row_ok ? lo.x : 0u),
-                             "r"(row_ok ? lo.y : 0u), "r"(row_ok ? hi.x : 0u), "r"(row_ok ? hi.y : 0u)
-                             : "memory");
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t wd = h ? w.y : w.x;
+                    const uint32_t sg = (sb >> (8 * h)) & 0xffu;
+                    const uint32_t ev = ((wd << 3) & 0x78787878u) | (((sg & 0x55u) * 0x02082080u) & 0x80808080u);
+                    const uint32_t od = ((wd >> 1) & 0x78787878u) | (((sg & 0xaau) * 0x01041040u) & 0x80808080u);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t src = (j & 1) ? od : ev;
+                        const uint2 e = lds64(__byte_perm(src, table, (uint32_t)(j >> 1) | 0x7650u));
+                        v[16 * h + 2 * j] = row_ok ? e.x : 0u;
+                        v[16 * h + 2 * j + 1] = row_ok ? e.y : 0u;
+                    }
+                }
+                if (!mbar_wait(empty(s), (uint32_t)(((kc / kPStages) & 1) ^ 1), &abort_s)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                SHERRY_TMEM_ST32(t_lane + (uint32_t)(s * kPAcols), v);
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                mbar_arrive(full_a(s));
             }
-            fence_proxy_async();
-            mbar_arrive(full_a(s));
         }
     } else if (warp == 8) {
         // ---------------- TMA producer for X ----------------
         if (lane == 0) {
-            for (int ks = 0; ks < nk; ++ks) {
-                const int s = ks % kPStages;
-                if (!mbar_wait(empty(s), (uint32_t)(((ks / kPStages) & 1) ^ 1), &abort_s)) break;
-                mbar_expect_tx(full_b(s), kPStageB);
-                tma_load_2d(stB + s * kPStageB, &xmap, ks * kPBK, m0, full_b(s));
+            int kc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                const int m0 = (t / ntn) * kPBN;
+                for (int ks = 0; ks < nk; ++ks, ++kc) {
+                    const int s = kc % kPStages;
+                    if (!mbar_wait(empty(s), (uint32_t)(((kc / kPStages) & 1) ^ 1), &abort_s)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(full_b(s), kPStageB);
+                    tma_load_2d(stB + s * kPStageB, &xmap, ks * kPBK, m0, full_b(s));
+                }
             }
         }
     } else {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            for (int ks = 0; ks < nk; ++ks) {
-                const int s = ks % kPStages;
-                const int g = ks / gs;
-                const int b = g & 1;
-                const bool first = (ks % gs) == 0;
-                if (first && !mbar_wait(acc_empty(b), (uint32_t)(((g >> 1) & 1) ^ 1), &abort_s)) break;
-                if (!mbar_wait(full_a(s), (uint32_t)((ks / kPStages) & 1), &abort_s)) break;
-                if (!mbar_wait(full_b(s), (uint32_t)((ks / kPStages) & 1), &abort_s)) break;
-                tc_fence_after();
-                const uint64_t da = smem_desc(stA + s * kPStageA);
-                const uint64_t db = smem_desc(stB + s * kPStageB);
+            int kc = 0, gc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                for (int ks = 0; ks < nk; ++ks, ++kc) {
+                    const int s = kc % kPStages;
+                    const int b = gc & 1;
+                    const bool first = (ks % gs) == 0;
+                    if (first && !mbar_wait(acc_empty(b), (uint32_t)(((gc >> 1) & 1) ^ 1), &abort_s)) { ok = false; break; }
+                    if (!mbar_wait(full_a(s), (uint32_t)((kc / kPStages) & 1), &abort_s)) { ok = false; break; }
+                    if (!mbar_wait(full_b(s), (uint32_t)((kc / kPStages) & 1), &abort_s)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t db = smem_desc(stB + s * kPStageB);
+                    const uint32_t ta = tmem + (uint32_t)(kPAcol + s * kPAcols);
 #pragma unroll
-                for (int kk = 0; kk < kPBK / 16; ++kk)  // K = 16 per MMA: +32 bytes in the swizzled row
-                    mma_bf16(tmem + (uint32_t)(b * kPBN), da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk),
-                             (first && kk == 0) ? 0u : 1u);
-                mma_commit(empty(s));
-                if ((ks % gs) == gs - 1) mma_commit(acc_full(b));
+                    for (int kk = 0; kk < kPBK / 16; ++kk)  // K = 16 per MMA: 8 A columns, +32 bytes in the B row
+                        mma_bf16_ts(tmem + (uint32_t)(b * kPBN), ta + (uint32_t)(8 * kk), db + (uint64_t)(2 * kk),
+                                    (first && kk == 0) ? 0u : 1u);
+                    mma_commit(empty(s));
+                    if ((ks % gs) == gs - 1) {
+                        mma_commit(acc_full(b));
+                        ++gc;
+                    }
+                }
             }
         }
         __syncwarp();
@@ -382,7 +443,14 @@ int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, i
             attr = true;
         }
     }
-    dim3 grid((unsigned)((s.N + kPBM - 1) / kPBM), (unsigned)((M + kPBN - 1) / kPBN));
+    const int64_t tiles = ((s.N + kPBM - 1) / kPBM) * ((M + kPBN - 1) / kPBN);
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        SHERRY_CUDA_CHECK(cudaGetDevice(&dev));
+        SHERRY_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    }
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
     k_prefill<<<grid, kPThreads, kPSmem, stream>>>(map, P);
     SHERRY_LAUNCH_CHECK();
     return SHERRY_OK;
