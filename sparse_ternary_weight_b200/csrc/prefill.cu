@@ -37,7 +37,8 @@ constexpr int kPBN = 128;     // tokens per tile
 constexpr int kPBK = 64;      // K per stage
 constexpr int kPStages = 4;
 constexpr int kPStageB = kPBN * kPBK * 2;  // 16 KB of X per stage
-constexpr int kPTable = 256;               // 32 x 8-byte weight patterns
+constexpr int kPTable = 256;               // 32 weight patterns: low words (128 B), then high words
+constexpr int kPPrefetch = 4;              // K-steps of packed words in flight per decode thread
 constexpr int kPSmem = kPStages * kPStageB + kPTable + 1024;
 constexpr int kPTmemCols = 512;            // 2 x 128 accumulator columns + 4 x 32 A columns
 constexpr int kPAcol = 256;                // first TMEM column of the A stages
@@ -211,9 +212,12 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
         fence_mbar_init();
     }
     if (threadIdx.x < 32) {
-        // bf16 patterns of the 32 block codes: entry = nibble + 16 * sign bit
+        // bf16 patterns of the 32 block codes (entry = nibble + 16 * sign bit): the
+        // low halves (weights 0, 1) and the high halves (weights 2, 3) in separate
+        // 128-byte tables, so that a warp's lookups never conflict on a bank
         const uint2 e = decode_block_bf16((uint32_t)threadIdx.x & 15u, (uint32_t)threadIdx.x >> 4);
-        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(table + 8u * threadIdx.x), "r"(e.x), "r"(e.y) : "memory");
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 4u * threadIdx.x), "r"(e.x) : "memory");
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 128u + 4u * threadIdx.x), "r"(e.y) : "memory");
     }
     if (warp == 9) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
@@ -283,45 +287,60 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
             const bool row_ok = n < P.N;
             const uint32_t* idxr = P.idx + (int64_t)(row_ok ? n : 0) * P.words;
             const uint8_t* sgnr = P.sgn + (int64_t)(row_ok ? n : 0) * P.words;
-            uint2 wn = make_uint2(0u, 0u);
-            uint32_t sn = 0u;
-            if (row_ok) {
-                wn = __ldg(reinterpret_cast<const uint2*>(idxr));
-                sn = __ldg(reinterpret_cast<const uint16_t*>(sgnr));
+            // ring of the next kPPrefetch steps' packed words (2 idx words + 2 sign bytes each)
+            uint2 rw[kPPrefetch];
+            uint32_t rs[kPPrefetch];
+#pragma unroll
+            for (int u = 0; u < kPPrefetch; ++u) {
+                rw[u] = make_uint2(0u, 0u);
+                rs[u] = 0u;
+                if (row_ok && u < nk) {
+                    rw[u] = __ldg(reinterpret_cast<const uint2*>(idxr + 2 * u));
+                    rs[u] = __ldg(reinterpret_cast<const uint16_t*>(sgnr + 2 * u));
+                }
             }
-            for (int ks = 0; ks < nk; ++ks, ++kc) {
-                const int s = kc % kPStages;
-                const uint2 w = wn;
-                const uint32_t sb = sn;
-                if (ks + 1 < nk && row_ok) {  // next step's words, loaded one step ahead
-                    wn = __ldg(reinterpret_cast<const uint2*>(idxr + 2 * (ks + 1)));
-                    sn = __ldg(reinterpret_cast<const uint16_t*>(sgnr + 2 * (ks + 1)));
-                }
-                // table offsets (8 * (nibble + 16 G)) of the even / odd blocks of each word
-                uint32_t v[32];
+            for (int ks0 = 0; ks0 < nk && ok; ks0 += kPPrefetch) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t wd = h ? w.y : w.x;
-                    const uint32_t sg = (sb >> (8 * h)) & 0xffu;
-                    const uint32_t ev = ((wd << 3) & 0x78787878u) | (((sg & 0x55u) * 0x02082080u) & 0x80808080u);
-                    const uint32_t od = ((wd >> 1) & 0x78787878u) | (((sg & 0xaau) * 0x01041040u) & 0x80808080u);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint32_t src = (j & 1) ? od : ev;
-                        const uint2 e = lds64(__byte_perm(src, table, (uint32_t)(j >> 1) | 0x7650u));
-                        v[16 * h + 2 * j] = row_ok ? e.x : 0u;
-                        v[16 * h + 2 * j + 1] = row_ok ? e.y : 0u;
+                for (int u = 0; u < kPPrefetch; ++u) {
+                    const int ks = ks0 + u;
+                    if (ks >= nk) break;
+                    const int s = kc % kPStages;
+                    const uint2 w = rw[u];
+                    const uint32_t sb = rs[u];
+                    if (ks + kPPrefetch < nk && row_ok) {
+                        rw[u] = __ldg(reinterpret_cast<const uint2*>(idxr + 2 * (ks + kPPrefetch)));
+                        rs[u] = __ldg(reinterpret_cast<const uint16_t*>(sgnr + 2 * (ks + kPPrefetch)));
                     }
+                    // table offsets (4 * (nibble + 16 G)) of the even / odd blocks of each word
+                    uint32_t v[32];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t wd = h ? w.y : w.x;
+                        const uint32_t sg = (sb >> (8 * h)) & 0xffu;
+                        const uint32_t ev = ((wd << 2) & 0x3c3c3c3cu) | (((sg & 0x55u) * 0x01041040u) & 0x40404040u);
+                        const uint32_t od = ((wd >> 2) & 0x3c3c3c3cu) | (((sg & 0xaau) * 0x00820820u) & 0x40404040u);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const uint32_t src = (j & 1) ? od : ev;
+                            const uint32_t a = __byte_perm(src, table, (uint32_t)(j >> 1) | 0x7650u);
+                            uint32_t lo, hi;
+                            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo) : "r"(a));
+                            asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(hi) : "r"(a));
+                            v[16 * h + 2 * j] = row_ok ? lo : 0u;
+                            v[16 * h + 2 * j + 1] = row_ok ? hi : 0u;
+                        }
+                    }
+                    if (!mbar_wait(empty(s), (uint32_t)(((kc / kPStages) & 1) ^ 1), &abort_s)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    SHERRY_TMEM_ST32(t_lane + (uint32_t)(s * kPAcols), v);
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    tc_fence_before();
+                    mbar_arrive(full_a(s));
+                    ++kc;
                 }
-                if (!mbar_wait(empty(s), (uint32_t)(((kc / kPStages) & 1) ^ 1), &abort_s)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                SHERRY_TMEM_ST32(t_lane + (uint32_t)(s * kPAcols), v);
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                tc_fence_before();
-                mbar_arrive(full_a(s));
             }
         }
     } else if (warp == 8) {
