@@ -14,12 +14,13 @@
 // decode threads own one TMEM lane (= weight row) each and write their row's
 // 64 bf16 of a step into TMEM with tcgen05.st; only the X tiles (operand B)
 // come through shared memory, by TMA (no multicast).
-//   warps 0-3  epilogue: wait for a finished group accumulator, tcgen05.ld it,
-//              acc[token] += alpha(row, group) * D; write Y (row per thread)
-//   warps 4-7  decode: per block one table lookup (32 bf16x4 patterns indexed by
+//   warps 0-7  epilogue: wait for one of three finished group accumulators,
+//              tcgen05.ld its 64-token half, acc[token] += alpha(row, group) * D,
+//              write Y (row per thread)
+//   warps 8-11 decode: per block one table lookup (32 bf16x4 patterns indexed by
 //              nibble + 16*sign) -> tcgen05.st into the A stage of their lanes
-//   warp 8     TMA: X tiles [128 tokens x 64 K], SWIZZLE_128B
-//   warp 9     TMEM allocation; one elected thread issues tcgen05.mma
+//   warp 12    TMA: X tiles [128 tokens x 64 K], SWIZZLE_128B
+//   warp 13    TMEM allocation; one elected thread issues tcgen05.mma
 // Every mbarrier wait is bounded; on timeout the CTA sets a device status flag
 // and drains instead of hanging.
 #include "common.cuh"
@@ -31,7 +32,7 @@
 
 namespace sherry {
 
-constexpr int kPThreads = 320;
+constexpr int kPThreads = 448;   // 8 epilogue + 4 decode + TMA + MMA warps
 constexpr int kPBM = 128;     // weight rows per tile
 constexpr int kPBN = 128;     // tokens per tile
 constexpr int kPBK = 64;      // K per stage
@@ -40,8 +41,9 @@ constexpr int kPStageB = kPBN * kPBK * 2;  // 16 KB of X per stage
 constexpr int kPTable = 256;               // 32 weight patterns: low words (128 B), then high words
 constexpr int kPPrefetch = 4;              // K-steps of packed words in flight per decode thread
 constexpr int kPSmem = kPStages * kPStageB + kPTable + 1024;
-constexpr int kPTmemCols = 512;            // 2 x 128 accumulator columns + 4 x 32 A columns
-constexpr int kPAcol = 256;                // first TMEM column of the A stages
+constexpr int kPAcc = 3;                   // group accumulators in flight
+constexpr int kPTmemCols = 512;            // 3 x 128 accumulator columns + 4 x 32 A columns
+constexpr int kPAcol = kPAcc * kPBN;       // first TMEM column of the A stages (384)
 constexpr int kPAcols = kPBK / 2;          // 32 columns (64 bf16) per A stage
 constexpr long long kPWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
 
@@ -175,7 +177,7 @@ __device__ __forceinline__ uint2 decode_block_bf16(uint32_t nib, uint32_t g) {
 __global__ void __launch_bounds__(kPThreads, 1)
 k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PParams P) {
     extern __shared__ __align__(1024) unsigned char psmem[];
-    __shared__ uint64_t bars[3 * kPStages + 4];
+    __shared__ uint64_t bars[3 * kPStages + 2 * kPAcc];
     __shared__ uint32_t tmem_base_s;
     __shared__ volatile int abort_s;
 
@@ -188,7 +190,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
     auto full_b = [&](int s) { return bar0 + 8u * (kPStages + s); };
     auto empty = [&](int s) { return bar0 + 8u * (2 * kPStages + s); };
     auto acc_full = [&](int b) { return bar0 + 8u * (3 * kPStages + b); };
-    auto acc_empty = [&](int b) { return bar0 + 8u * (3 * kPStages + 2 + b); };
+    auto acc_empty = [&](int b) { return bar0 + 8u * (3 * kPStages + kPAcc + b); };
 
     // persistent: tile t = (weight-row tile t % ntn, token tile t / ntn), strided by the grid;
     // stage and accumulator phases run on across tiles
@@ -205,9 +207,9 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
             mbar_init(full_b(s), 1);
             mbar_init(empty(s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kPAcc; ++b) {
             mbar_init(acc_full(b), 1);
-            mbar_init(acc_empty(b), 128);
+            mbar_init(acc_empty(b), 256);
         }
         fence_mbar_init();
     }
@@ -219,7 +221,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 4u * threadIdx.x), "r"(e.x) : "memory");
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 128u + 4u * threadIdx.x), "r"(e.y) : "memory");
     }
-    if (warp == 9) {
+    if (warp == 13) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
                      "r"(kPTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -229,41 +231,45 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;
 
-    if (warp < 4) {
-        // ---------------- epilogue: row n = n0 + 32*warp + lane of each tile ----------------
+    if (warp < 8) {
+        // ---------------- epilogue: row n = tile row 32*(warp%4) + lane, tokens
+        // [64*(warp/4), 64*(warp/4) + 64) of each tile ----------------
+        const int q = warp & 3, half = warp >> 2;
+        constexpr int kCols = kPBN / 2;
         bool ok = true;
         int gc = 0;  // groups consumed so far (all tiles)
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const int n = (t % ntn) * kPBM + warp * 32 + lane;
-            const int m0 = (t / ntn) * kPBN;
+            const int n = (t % ntn) * kPBM + q * 32 + lane;
+            const int m0 = (t / ntn) * kPBN + half * kCols;
             const bool row_ok = n < P.N;
-            float acc[kPBN];
+            float acc[kCols];
 #pragma unroll
-            for (int j = 0; j < kPBN; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < kCols; ++j) acc[j] = 0.0f;
             for (int g = 0; g < ngroups; ++g, ++gc) {
-                const int b = gc & 1;
-                ok = mbar_wait(acc_full(b), (uint32_t)((gc >> 1) & 1), &abort_s);
+                const int b = gc % kPAcc;
+                ok = mbar_wait(acc_full(b), (uint32_t)((gc / kPAcc) & 1), &abort_s);
                 if (!ok) break;
                 tc_fence_after();
                 float a = 1.0f;
                 if (!P.row_scale && row_ok) a = __ldg(P.scales + (int64_t)n * P.spr + g);  // group g: K-steps [g*gs, (g+1)*gs)
-                const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * kPBN);
-#pragma unroll
-                for (int c = 0; c < kPBN / 32; ++c) {
-                    uint32_t v[32];
-                    SHERRY_TMEM_LD32(t_row + c * 32, v);
-                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(a, __uint_as_float(v[j]), acc[c * 32 + j]);
-                }
+                const uint32_t t_row = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kPBN + half * kCols);
+                uint32_t v0[32], v1[32];
+                SHERRY_TMEM_LD32(t_row, v0);
+                SHERRY_TMEM_LD32(t_row + 32, v1);
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
                 tc_fence_before();
                 mbar_arrive(acc_empty(b));
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    acc[j] = fmaf(a, __uint_as_float(v0[j]), acc[j]);
+                    acc[32 + j] = fmaf(a, __uint_as_float(v1[j]), acc[32 + j]);
+                }
             }
             if (ok && row_ok) {
                 float a = 1.0f;
                 if (P.row_scale) a = __ldg(P.scales + (P.per_tensor ? 0 : n));
 #pragma unroll
-                for (int j = 0; j < kPBN; ++j) {
+                for (int j = 0; j < kCols; ++j) {
                     const int m = m0 + j;
                     if (m < P.M) {
                         const float y = acc[j] * a;
@@ -275,9 +281,9 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
                 }
             }
         }
-    } else if (warp < 8) {
+    } else if (warp < 12) {
         // ---------------- decode: TMEM lane (= tile row) i per thread ----------------
-        const int q = warp - 4;                 // lane quarter of this warp
+        const int q = warp - 8;                 // lane quarter of this warp (warp % 4)
         const int i = q * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kPAcol;
         int kc = 0;  // K-steps produced so far (all tiles)
@@ -343,7 +349,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
                 }
             }
         }
-    } else if (warp == 8) {
+    } else if (warp == 12) {
         // ---------------- TMA producer for X ----------------
         if (lane == 0) {
             int kc = 0;
@@ -369,9 +375,9 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 for (int ks = 0; ks < nk; ++ks, ++kc) {
                     const int s = kc % kPStages;
-                    const int b = gc & 1;
+                    const int b = gc % kPAcc;
                     const bool first = (ks % gs) == 0;
-                    if (first && !mbar_wait(acc_empty(b), (uint32_t)(((gc >> 1) & 1) ^ 1), &abort_s)) { ok = false; break; }
+                    if (first && !mbar_wait(acc_empty(b), (uint32_t)(((gc / kPAcc) & 1) ^ 1), &abort_s)) { ok = false; break; }
                     if (!mbar_wait(full_a(s), (uint32_t)((kc / kPStages) & 1), &abort_s)) { ok = false; break; }
                     if (!mbar_wait(full_b(s), (uint32_t)((kc / kPStages) & 1), &abort_s)) { ok = false; break; }
                     tc_fence_after();
@@ -394,7 +400,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == 13) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPTmemCols));
     }
