@@ -466,9 +466,10 @@ def prefill_rows(args, pairs, ws, dev, pk, steps, warm):
 # CPU oracle (the reference arm of this build)
 
 
-def cpu_baseline(layers, steps=1):
+def cpu_baseline(layers, min_seconds=10.0):
     """Oracle linear (fp64 accumulation, OpenMP over rows) on the first `layers`
-    layers of the 3B stack at M = 1: returns the same metric on the host."""
+    layers of the 3B stack at M = 1, repeated until at least `min_seconds` of
+    CPU work: returns the same metric on the host."""
     import oracle
     from sparse_ternary_weight_b200 import synth
     orc = oracle.oracle(omp=True)
@@ -483,17 +484,18 @@ def cpu_baseline(layers, steps=1):
             work.append((X, idx, sgn, sc, N, K))
             del W
     shapes = [(N, K) for (_, _, _, _, N, K) in work]
-    b = stack_bytes(shapes, 1)
-    times = []
-    for _ in range(steps):
-        t0 = time.perf_counter()
+    b1 = stack_bytes(shapes, 1)
+    reps, t = 0, 0.0
+    t0 = time.perf_counter()
+    while t < min_seconds:
         for (X, idx, sgn, sc, N, K) in work:
             orc.linear(X, idx, sgn, sc, N, K, oracle.PER_GROUP, 128)
-        times.append(time.perf_counter() - t0)
-    t = min(times) if steps > 1 else times[0]
+        reps += 1
+        t = time.perf_counter() - t0
+    b = b1 * reps
     return {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": orc.threads(), "kind": "oracle",
-            "sample": f"first {layers} layer(s) of the 3B stack ({len(work)} linears, M=1, group 128): "
-                      f"{b} algorithmic bytes in {t:.3f} s; C oracle, fp64 accumulation, OpenMP over rows",
+            "sample": f"first {layers} layer(s) of the 3B stack ({len(work)} linears, M=1, group 128) x {reps} "
+                      f"passes: {b} algorithmic bytes in {t:.2f} s; C oracle, fp64 accumulation, OpenMP over rows",
             "tok_per_s_equiv": round(b / t / stack_bytes([s for (_, _, s) in stack_shapes()], 1), 4)}
 
 
@@ -566,6 +568,25 @@ def profile_prefill(args):
                       "TFLOP/s_dense_equiv": round(2 * M * N * K / (ms * 1e-3) / 1e12, 1)}), flush=True)
 
 
+def profile_quantize(args):
+    import torch
+    from sparse_ternary_weight_b200.build import build
+    build()
+    import sparse_ternary_weight_b200 as sw
+    n, k, gran = args.profile_quantize.split(",")
+    N, K = int(n), int(k)
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(N + K)
+    W = torch.randn((N, K), generator=g, device=dev) * 0.02
+    out = sw.quantize_pack(W, gran, 128)
+    ms = time_region(lambda: sw.quantize_pack(W, gran, 128, out=out), args.steps, args.warmup, 1,
+                     torch.cuda.current_stream()) / args.steps
+    b = 4 * N * K + out.nbytes()
+    print(json.dumps({"quantize_pack": f"{N}x{K} {gran}", "ms": round(ms, 4),
+                      "GB/s": round(b / (ms * 1e-3) / 1e9, 1), "bytes": b}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -577,12 +598,18 @@ def main():
     ap.add_argument("--cpu-layers", type=int, default=1)
     ap.add_argument("--layers", type=int, default=28, help="layers of the 3B stack (28 = the full workload; "
                     "fewer only for profiling captures)")
+    ap.add_argument("--profile-quantize", default=None, metavar="N,K,GRAN",
+                    help="only quantize+pack one fp32 N x K weight (GRAN per_group|per_channel|per_tensor) "
+                         "warmup+steps times, print its time, and exit (for profiler captures)")
     ap.add_argument("--profile-prefill", default=None, metavar="N,K,M",
                     help="only run one tensor-core prefill linear (N x K weight, M tokens) warmup+steps times, "
                          "print its time, and exit (for profiler captures)")
     args = ap.parse_args()
     if args.profile_prefill:
         profile_prefill(args)
+        return
+    if args.profile_quantize:
+        profile_quantize(args)
         return
     if args.warmup < 3:
         args.warmup = 3
