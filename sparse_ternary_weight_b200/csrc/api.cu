@@ -59,7 +59,15 @@ static bool use_stream(const ProbShape* shapes, int count, int64_t M) {
     return tiles <= kMaxTickets;
 }
 
+static bool use_skinny(const ProbShape* shapes, int count, int64_t M) {
+    if (M < 2 || M > 32 || count == 0) return false;
+    for (int i = 0; i < count; ++i)
+        if (!skinny_eligible(shapes[i], M)) return false;
+    return true;
+}
+
 static size_t linear_ws_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
+    if (use_skinny(shapes, count, M)) return 0;
     if (count == 1 && prefill_eligible(shapes[0], M)) return 0;
     if (use_stream(shapes, count, M)) return stream_workspace_bytes(shapes, count, sms);
     return lut_workspace_bytes(shapes, count, M, sms);
@@ -67,6 +75,7 @@ static size_t linear_ws_bytes(const ProbShape* shapes, int count, int64_t M, int
 
 static int linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream) {
+    if (use_skinny(shapes, count, M)) return skinny_linear_launch(shapes, descs, count, M, y_bf16, sms, stream);
     if (count == 1 && prefill_eligible(shapes[0], M)) return prefill_launch(shapes[0], descs[0], M, y_bf16, stream);
     if (use_stream(shapes, count, M))
         return stream_linear_launch(shapes, descs, count, y_bf16, workspace, sms, stream);

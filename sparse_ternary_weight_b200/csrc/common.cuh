@@ -116,6 +116,11 @@ int lut_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, 
 bool prefill_eligible(const ProbShape& s, int64_t M);
 int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, int y_bf16, cudaStream_t stream);
 int device_status_take(cudaStream_t stream);
+// few-token tensor-core kernel (gemv_tc.cu)
+bool skinny_eligible(const ProbShape& s, int64_t M);
+int skinny_status_take();  // SHERRY_ERR_TIMEOUT if a bounded wait gave up since the last call
+int skinny_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
+                         int sms, cudaStream_t stream);
 // one-token streaming kernel (gemv_stream.cu)
 bool stream_eligible(const ProbShape& s, int64_t M);
 size_t stream_workspace_bytes(const ProbShape* shapes, int count, int sms);

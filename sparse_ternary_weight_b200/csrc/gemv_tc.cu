@@ -1,0 +1,519 @@
+// gemv_tc.cu -- packed 3:4 ternary linear for a few tokens (2 <= M <= 32) on the
+// tensor cores, Y = X (T alpha)^T ("Sherry: Hardware-Efficient 1.25-Bit Ternary
+// Quantization via Fine-grained Sparsification", digest: Y = X T alpha).
+//
+// With a handful of tokens the lookup-table decode does one table lookup per
+// block and token; here every weight is expanded once to bf16 {-1, 0, +1} (one
+// pattern-table lookup per block, whatever M is) and multiplied on the tensor
+// cores with all tokens at once (MMA N = 16 or 32 token columns).  Like the
+// one-token kernel it streams the packed planes from HBM once, for any number
+// of independent linears in one launch.
+//
+// Work unit: one linear's 128 weight rows x all of K.  Units are dealt to one
+// persistent CTA per SM round-robin.  Per CTA (10 warps):
+//   warps 0-3  epilogue (TMEM lane quarter = warp % 4): promote each scale
+//              group's accumulator with alpha in fp32 registers, write Y
+//   warps 4-7  decode: one TMEM lane (= weight row) per thread, per 64-weight
+//              step 16 pattern lookups -> tcgen05.st (operand A in TMEM)
+//   warp 8     producer: 16-byte cp.async of each K-chunk (256 weights): the
+//              packed words and sign bytes of the 128 rows, and the X chunk laid
+//              out as the MMA's SWIZZLE_128B K-major B operand; completion is
+//              signalled on an mbarrier (cp.async.mbarrier.arrive)
+//   warp 9     TMEM allocation; one elected thread issues tcgen05.mma
+//              (A from TMEM, B from shared memory)
+// Every mbarrier wait is bounded.
+#include "common.cuh"
+#include "lut.cuh"
+
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+namespace sherry {
+
+constexpr int kTThreads = 320;            // 10 warps
+constexpr int kTRows = 128;               // weight rows per unit (MMA M, TMEM lanes)
+constexpr int kTStepK = 64;               // K per MMA step (one 128-byte swizzle atom of bf16)
+constexpr int kTChunkSteps = 4;           // steps per staged chunk (256 weights)
+constexpr int kTChunkK = kTStepK * kTChunkSteps;
+constexpr int kTChunks = 4;               // staged chunks in flight
+constexpr int kTAStages = 4;              // A stages in TMEM
+constexpr int kTAcc = 3;                  // group accumulators
+constexpr int kTIdxBytes = kTRows * kTChunkSteps * 8;    // 4 KB: 8 words per row
+constexpr int kTSgnBytes = kTRows * kTChunkSteps * 2;    // 1 KB: 8 sign bytes per row
+constexpr long long kTWaitCycles = 4000000000LL;
+
+struct TProb {
+    const uint16_t* X;
+    const uint32_t* idx;
+    const uint8_t* sgn;
+    const float* scales;
+    void* Y;
+    int N, K, words;
+    int row_scale, per_tensor, spr, group_steps;
+    int unit_begin, n_rt;
+};
+
+template <int MAXP>
+struct TParams {
+    int count, M, y_bf16, total_units;
+    TProb p[MAXP];
+};
+
+// bounded-wait timeouts of this file's kernel (read and cleared by sherry_device_status)
+__device__ int g_skinny_status = 0;
+
+namespace {
+
+__device__ __forceinline__ void t_mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void t_mbar_arrive(uint32_t bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool t_mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool t_mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (t_mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (t_mbar_try(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kTWaitCycles) {
+            *abort_flag = 1;
+            atomicExch(&g_skinny_status, SHERRY_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void t_cp16(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void t_cp8(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(valid ? 8 : 0)
+                 : "memory");
+}
+// the mbarrier receives one arrival when all of this thread's prior cp.async complete
+__device__ __forceinline__ void t_cp_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void t_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void t_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ uint64_t t_smem_desc(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3fff);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+template <int BN>
+struct TIdesc {
+    static constexpr uint32_t v =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kTRows >> 4) << 24);
+};
+
+__device__ __forceinline__ void t_mma(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void t_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+}  // namespace
+
+#define SHERRY_T_ST32(taddr, v)                                                                                  \
+    asm volatile(                                                                                                \
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16," \
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),                        \
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),      \
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),          \
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),         \
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])                      \
+        : "memory")
+
+#define SHERRY_T_LD16(taddr, v)                                                                          \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+                 "%15}, [%16];"                                                                          \
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),    \
+                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), \
+                   "=r"(v[14]), "=r"(v[15])                                                               \
+                 : "r"(taddr))
+
+// unit u -> (problem, row tile)
+template <int MAXP>
+__device__ __forceinline__ void t_locate(const TParams<MAXP>& P, int u, int& p, int& rt) {
+    p = 0;
+    while (p + 1 < P.count && P.p[p + 1].unit_begin <= u) ++p;
+    rt = u - P.p[p].unit_begin;
+}
+
+template <int BN, int MAXP>
+__global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__ TParams<MAXP> P) {
+    constexpr int kXStep = BN * 128;                 // X bytes per 64-K step (BN rows x 128 B)
+    constexpr int kXBytes = kXStep * kTChunkSteps;   // per chunk
+    constexpr uint32_t kIdesc = TIdesc<BN>::v;
+    constexpr int kAccStride = 32;                   // TMEM columns per accumulator (>= BN, 32-aligned)
+    constexpr int kAcol = 128;                       // first A column in TMEM (A stages: 128..255)
+    static_assert(BN <= kAccStride && kTAcc * kAccStride <= kAcol && kAcol + 32 * kTAStages <= 256, "TMEM plan");
+    extern __shared__ __align__(1024) unsigned char tsm[];
+    __shared__ uint64_t bars[2 * kTChunks + 2 * kTAStages + 2 * kTAcc];
+    __shared__ uint32_t tmem_s;
+    __shared__ volatile int abort_s;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t base = (smem_u32(tsm) + 1023u) & ~1023u;  // X stages first (1024-aligned)
+    auto xst = [&](int c) { return base + (uint32_t)(c * kXBytes); };
+    const uint32_t pbase = base + (uint32_t)(kTChunks * kXBytes);
+    auto ist = [&](int c) { return pbase + (uint32_t)(c * (kTIdxBytes + kTSgnBytes)); };
+    const uint32_t table = pbase + (uint32_t)(kTChunks * (kTIdxBytes + kTSgnBytes));  // 256-aligned
+    const uint32_t bar0 = smem_u32(&bars[0]);
+    auto full_c = [&](int c) { return bar0 + 8u * c; };
+    auto empty_c = [&](int c) { return bar0 + 8u * (kTChunks + c); };
+    auto full_a = [&](int s) { return bar0 + 8u * (2 * kTChunks + s); };
+    auto empty_a = [&](int s) { return bar0 + 8u * (2 * kTChunks + kTAStages + s); };
+    auto acc_full = [&](int b) { return bar0 + 8u * (2 * kTChunks + 2 * kTAStages + b); };
+    auto acc_empty = [&](int b) { return bar0 + 8u * (2 * kTChunks + 2 * kTAStages + kTAcc + b); };
+
+    if (threadIdx.x == 0) {
+        abort_s = 0;
+        for (int c = 0; c < kTChunks; ++c) {
+            t_mbar_init(full_c(c), 32);         // the producer warp's cp.async arrivals
+            t_mbar_init(empty_c(c), 1 + 128);   // the MMA commit (X read) + the decode threads (words read)
+        }
+        for (int s = 0; s < kTAStages; ++s) {
+            t_mbar_init(full_a(s), 128);
+            t_mbar_init(empty_a(s), 1);
+        }
+        for (int b = 0; b < kTAcc; ++b) {
+            t_mbar_init(acc_full(b), 1);
+            t_mbar_init(acc_empty(b), 128);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (threadIdx.x < 32) {
+        const uint32_t e = threadIdx.x;
+        const uint2 pat = decode_block_bf16(e & 15u, e >> 4);
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 4u * e), "r"(pat.x) : "memory");
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 128u + 4u * e), "r"(pat.y) : "memory");
+    }
+    if (warp == 9) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_s)),
+                     "r"(256));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    t_fence_before();
+    __syncthreads();
+    t_fence_after();
+    const uint32_t tmem = tmem_s;
+    const int M = P.M;
+
+    if (warp == 8) {
+        // ---------------- producer ----------------
+        int cc = 0;  // chunks produced (all units)
+        bool ok = true;
+        for (int u = blockIdx.x; u < P.total_units && ok; u += gridDim.x) {
+            int p, rt;
+            t_locate(P, u, p, rt);
+            const TProb& pr = P.p[p];
+            const int row0 = rt * kTRows;
+            const int nchunks = pr.K / kTChunkK;
+            for (int ch = 0; ch < nchunks; ++ch, ++cc) {
+                const int c = cc % kTChunks;
+                if (!t_mbar_wait(empty_c(c), (uint32_t)(((cc / kTChunks) & 1) ^ 1), &abort_s)) {
+                    ok = false;
+                    break;
+                }
+                const int w0 = ch * kTChunkSteps * 2;  // first packed word of the chunk
+                // packed words: 128 rows x 32 B (two 16-B halves), half h of row r at h ^ ((r >> 2) & 1)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int q = lane + 32 * i;
+                    const int r = q >> 1, h = q & 1;
+                    const int row = row0 + r;
+                    const bool v = row < pr.N;
+                    t_cp16(ist(c) + r * 32 + ((h ^ ((r >> 2) & 1)) << 4),
+                           v ? (const void*)(pr.idx + (int64_t)row * pr.words + w0 + 4 * h) : (const void*)pr.idx,
+                           v);
+                }
+                // sign bytes: 128 rows x 8 B
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = lane + 32 * i;
+                    const int row = row0 + r;
+                    const bool v = row < pr.N;
+                    t_cp8(ist(c) + kTIdxBytes + r * 8,
+                          v ? (const void*)(pr.sgn + (int64_t)row * pr.words + w0) : (const void*)pr.sgn, v);
+                }
+                // X chunk: 4 steps x BN token rows x 8 chunks of 16 B, SWIZZLE_128B K-major
+#pragma unroll
+                for (int i = 0; i < (kTChunkSteps * BN * 8) / 32; ++i) {
+                    const int q = lane + 32 * i;
+                    const int s = q / (BN * 8);
+                    const int r = (q / 8) % BN, cq = q % 8;
+                    const bool v = r < M;
+                    const int kk = ch * kTChunkK + s * kTStepK + cq * 8;
+                    t_cp16(xst(c) + s * kXStep + (r >> 3) * 1024 + (r & 7) * 128 + ((cq ^ (r & 7)) << 4),
+                           v ? (const void*)(pr.X + (int64_t)r * pr.K + kk) : (const void*)pr.X, v);
+                }
+                t_cp_arrive(full_c(c));
+            }
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp >= 4 && warp < 8) {
+        // ---------------- decode: TMEM lane (= unit row) per thread ----------------
+        const int q = warp - 4, i = q * 32 + lane;
+        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kAcol;
+        int cc = 0, kc = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < P.total_units && ok; u += gridDim.x) {
+            int p, rt;
+            t_locate(P, u, p, rt);
+            const TProb& pr = P.p[p];
+            const bool row_ok = rt * kTRows + i < pr.N;
+            const int nchunks = pr.K / kTChunkK;
+            for (int ch = 0; ch < nchunks && ok; ++ch, ++cc) {
+                const int c = cc % kTChunks;
+                if (!t_mbar_wait(full_c(c), (uint32_t)((cc / kTChunks) & 1), &abort_s)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sw = ((uint32_t)(i >> 2) & 1u) << 4;
+                uint4 wlo, whi;
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(wlo.x), "=r"(wlo.y), "=r"(wlo.z), "=r"(wlo.w)
+                             : "r"(ist(c) + i * 32 + sw));
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(whi.x), "=r"(whi.y), "=r"(whi.z), "=r"(whi.w)
+                             : "r"(ist(c) + i * 32 + (16u ^ sw)));
+                uint2 sgv;
+                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(sgv.x), "=r"(sgv.y) : "r"(ist(c) + kTIdxBytes + i * 8));
+                t_mbar_arrive(empty_c(c));  // this thread has its words
+                const uint32_t words[8] = {wlo.x, wlo.y, wlo.z, wlo.w, whi.x, whi.y, whi.z, whi.w};
+#pragma unroll
+                for (int st = 0; st < kTChunkSteps; ++st, ++kc) {
+                    const int s = kc % kTAStages;
+                    uint32_t v[32];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t wd = words[2 * st + h];
+                        const uint32_t sg = ((st < 2 ? sgv.x : sgv.y) >> (16 * (st & 1) + 8 * h)) & 0xffu;
+                        const uint32_t ev = ((wd << 2) & 0x3c3c3c3cu) | (((sg & 0x55u) * 0x01041040u) & 0x40404040u);
+                        const uint32_t od = ((wd >> 2) & 0x3c3c3c3cu) | (((sg & 0xaau) * 0x00820820u) & 0x40404040u);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const uint32_t a = __byte_perm((j & 1) ? od : ev, table, (uint32_t)(j >> 1) | 0x7650u);
+                            uint32_t lo, hi;
+                            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo) : "r"(a));
+                            asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(hi) : "r"(a));
+                            v[16 * h + 2 * j] = row_ok ? lo : 0u;
+                            v[16 * h + 2 * j + 1] = row_ok ? hi : 0u;
+                        }
+                    }
+                    if (!t_mbar_wait(empty_a(s), (uint32_t)(((kc / kTAStages) & 1) ^ 1), &abort_s)) {
+                        ok = false;
+                        break;
+                    }
+                    t_fence_after();
+                    SHERRY_T_ST32(t_lane + (uint32_t)(s * 32), v);
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    t_fence_before();
+                    t_mbar_arrive(full_a(s));
+                }
+            }
+        }
+    } else if (warp == 9) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            int cc = 0, kc = 0, gc = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < P.total_units && ok; u += gridDim.x) {
+                int p, rt;
+                t_locate(P, u, p, rt);
+                const TProb& pr = P.p[p];
+                const int nk = pr.K / kTStepK, gs = pr.group_steps;
+                for (int ks = 0; ks < nk; ++ks, ++kc) {
+                    const int c = cc % kTChunks, st = ks % kTChunkSteps;
+                    const int s = kc % kTAStages;
+                    const int b = gc % kTAcc;
+                    const bool first = (ks % gs) == 0;
+                    if (first && !t_mbar_wait(acc_empty(b), (uint32_t)(((gc / kTAcc) & 1) ^ 1), &abort_s)) { ok = false; break; }
+                    if (st == 0 && !t_mbar_wait(full_c(c), (uint32_t)((cc / kTChunks) & 1), &abort_s)) { ok = false; break; }
+                    if (!t_mbar_wait(full_a(s), (uint32_t)((kc / kTAStages) & 1), &abort_s)) { ok = false; break; }
+                    t_fence_after();
+                    const uint64_t db = t_smem_desc(xst(c) + st * kXStep);
+                    const uint32_t ta = tmem + (uint32_t)(kAcol + s * 32);
+#pragma unroll
+                    for (int kk = 0; kk < kTStepK / 16; ++kk)
+                        t_mma(tmem + (uint32_t)(b * kAccStride), ta + (uint32_t)(8 * kk), db + (uint64_t)(2 * kk), kIdesc,
+                              (first && kk == 0) ? 0u : 1u);
+                    t_commit(empty_a(s));
+                    if (st == kTChunkSteps - 1) {
+                        t_commit(empty_c(c));
+                        ++cc;
+                    }
+                    if ((ks % gs) == gs - 1) {
+                        t_commit(acc_full(b));
+                        ++gc;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        // ---------------- epilogue: unit row 32*warp + lane per thread ----------------
+        int gc = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < P.total_units && ok; u += gridDim.x) {
+            int p, rt;
+            t_locate(P, u, p, rt);
+            const TProb& pr = P.p[p];
+            const int n = rt * kTRows + warp * 32 + lane;
+            const bool row_ok = n < pr.N;
+            const int ngroups = (pr.K / kTStepK) / pr.group_steps;
+            float acc[BN];
+#pragma unroll
+            for (int j = 0; j < BN; ++j) acc[j] = 0.0f;
+            for (int g = 0; g < ngroups; ++g, ++gc) {
+                const int b = gc % kTAcc;
+                ok = t_mbar_wait(acc_full(b), (uint32_t)((gc / kTAcc) & 1), &abort_s);
+                if (!ok) break;
+                t_fence_after();
+                const float a = (!pr.row_scale && row_ok) ? __ldg(pr.scales + (int64_t)n * pr.spr + g) : 1.0f;
+                const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * kAccStride);
+                uint32_t v[BN];
+#pragma unroll
+                for (int c = 0; c < BN / 16; ++c) SHERRY_T_LD16(t_row + 16 * c, (v + 16 * c));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                t_fence_before();
+                t_mbar_arrive(acc_empty(b));
+#pragma unroll
+                for (int j = 0; j < BN; ++j) acc[j] = fmaf(a, __uint_as_float(v[j]), acc[j]);
+            }
+            if (ok && row_ok) {
+                const float a = pr.row_scale ? __ldg(pr.scales + (pr.per_tensor ? 0 : n)) : 1.0f;
+#pragma unroll
+                for (int j = 0; j < BN; ++j) {
+                    if (j < M) {
+                        const float y = acc[j] * a;
+                        if (P.y_bf16)
+                            reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)j * pr.N + n] = __float2bfloat16_rn(y);
+                        else
+                            reinterpret_cast<float*>(pr.Y)[(int64_t)j * pr.N + n] = y;
+                    }
+                }
+            }
+        }
+    }
+
+    t_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        t_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+    }
+}
+
+}  // namespace sherry
+
+// ---- host side -------------------------------------------------------------------
+
+namespace sherry {
+
+bool skinny_eligible(const ProbShape& s, int64_t M) {
+    if (M < 2 || M > 32 || s.N == 0) return false;
+    if (s.K % kTChunkK != 0) return false;
+    if (s.granularity == SHERRY_PER_GROUP && s.group % kTStepK != 0) return false;
+    return true;
+}
+
+template <int BN>
+static constexpr int skinny_smem() {
+    return kTChunks * (BN * 128 * kTChunkSteps + kTIdxBytes + kTSgnBytes) + 256 + 1024;
+}
+
+template <int BN, int MAXP>
+static int skinny_launch_t(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M,
+                           int y_bf16, int sms, cudaStream_t stream) {
+    static TParams<MAXP> P;
+    static std::mutex mu;
+    static bool attr = false;
+    std::lock_guard<std::mutex> lk(mu);
+    P.count = count;
+    P.M = (int)M;
+    P.y_bf16 = y_bf16;
+    int ub = 0;
+    for (int i = 0; i < count; ++i) {
+        const ProbShape& s = shapes[i];
+        TProb& p = P.p[i];
+        p.X = descs[i].X;
+        p.idx = descs[i].idx;
+        p.sgn = descs[i].sgn;
+        p.scales = descs[i].scales;
+        p.Y = descs[i].Y;
+        p.N = (int)s.N;
+        p.K = (int)s.K;
+        p.words = (int)(s.K / 32);
+        p.row_scale = s.granularity != SHERRY_PER_GROUP;
+        p.per_tensor = s.granularity == SHERRY_PER_TENSOR;
+        p.spr = s.granularity == SHERRY_PER_GROUP ? (int)(s.K / s.group) : 1;
+        p.group_steps = s.granularity == SHERRY_PER_GROUP ? s.group / kTStepK : (int)(s.K / kTStepK);
+        p.n_rt = (int)((s.N + kTRows - 1) / kTRows);
+        p.unit_begin = ub;
+        ub += p.n_rt;
+    }
+    P.total_units = ub;
+    if (ub == 0) return SHERRY_OK;
+    constexpr int smem = skinny_smem<BN>();
+    if (!attr) {
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_skinny<BN, MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+        attr = true;
+    }
+    const int grid = ub < sms ? ub : sms;
+    k_skinny<BN, MAXP><<<grid, kTThreads, smem, stream>>>(P);
+    SHERRY_LAUNCH_CHECK();
+    return SHERRY_OK;
+}
+
+template <int BN>
+static int skinny_launch_n(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M,
+                           int y_bf16, int sms, cudaStream_t stream) {
+    if (count <= 1) return skinny_launch_t<BN, 1>(shapes, descs, count, M, y_bf16, sms, stream);
+    if (count <= 16) return skinny_launch_t<BN, 16>(shapes, descs, count, M, y_bf16, sms, stream);
+    return skinny_launch_t<BN, SHERRY_MAX_BATCH>(shapes, descs, count, M, y_bf16, sms, stream);
+}
+
+int skinny_status_take() {
+    int v = 0;
+    SHERRY_CUDA_CHECK(cudaMemcpyFromSymbol(&v, g_skinny_status, sizeof(int)));
+    if (v) {
+        const int zero = 0;
+        SHERRY_CUDA_CHECK(cudaMemcpyToSymbol(g_skinny_status, &zero, sizeof(int)));
+    }
+    return v;
+}
+
+int skinny_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
+                         int sms, cudaStream_t stream) {
+    if (M <= 16) return skinny_launch_n<16>(shapes, descs, count, M, y_bf16, sms, stream);
+    return skinny_launch_n<32>(shapes, descs, count, M, y_bf16, sms, stream);
+}
+
+}  // namespace sherry

@@ -116,4 +116,16 @@ __device__ __forceinline__ void word_pair_sum(uint32_t w, uint32_t s, uint32_t b
     add2(p0, p1, a0, a1, b0, b1);
 }
 
+// bf16 {+1, 0, -1} of the 4 weights of a block: two packed halves
+__device__ __forceinline__ uint2 decode_block_bf16(uint32_t nib, uint32_t g) {
+    const uint32_t z = nib >> 2;
+    const uint32_t d1 = (nib >> 1) & 1u, d2 = nib & 1u;
+    const uint32_t k3 = g | ((g ^ d1) << 1) | ((g ^ d2) << 2);
+    const uint32_t negs = (k3 & ((1u << z) - 1u)) | ((k3 >> z) << (z + 1));
+    uint32_t h[4];
+#pragma unroll
+    for (uint32_t i = 0; i < 4; ++i) h[i] = (i == z) ? 0u : (0x3f80u | (((negs >> i) & 1u) << 15));
+    return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+}
+
 }  // namespace sherry

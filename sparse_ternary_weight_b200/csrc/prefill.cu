@@ -24,6 +24,7 @@
 // Every mbarrier wait is bounded; on timeout the CTA sets a device status flag
 // and drains instead of hanging.
 #include "common.cuh"
+#include "lut.cuh"
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -161,18 +162,6 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
           "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),             \
           "=r"(v[30]), "=r"(v[31])                                                                               \
         : "r"(taddr))
-
-// bf16 {+1, 0, -1} of the 4 weights of a block: two packed halves
-__device__ __forceinline__ uint2 decode_block_bf16(uint32_t nib, uint32_t g) {
-    const uint32_t z = nib >> 2;
-    const uint32_t d1 = (nib >> 1) & 1u, d2 = nib & 1u;
-    const uint32_t k3 = g | ((g ^ d1) << 1) | ((g ^ d2) << 2);
-    const uint32_t negs = (k3 & ((1u << z) - 1u)) | ((k3 >> z) << (z + 1));
-    uint32_t h[4];
-#pragma unroll
-    for (uint32_t i = 0; i < 4; ++i) h[i] = (i == z) ? 0u : (0x3f80u | (((negs >> i) & 1u) << 15));
-    return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
-}
 
 __global__ void __launch_bounds__(kPThreads, 1)
 k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PParams P) {
@@ -489,7 +478,8 @@ int device_status_take(cudaStream_t stream) {
         const int zero = 0;
         SHERRY_CUDA_CHECK(cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)));
     }
-    return v;
+    const int w = skinny_status_take();
+    return v ? v : w;
 }
 
 }  // namespace sherry

@@ -285,3 +285,59 @@ def test_prefill_tensor_core_vs_oracle(sw, orc, case):
     check_linear(yb.float().cpu().numpy(), y_ref, Xb, Wq, y_is_bf16=True)
     assert torch.equal(yb, y32.to(torch.bfloat16))
     assert torch.equal(sw.linear(X, P, torch.float32), y32)
+
+
+SKINNY_CASES = [
+    # (M, N, K, gran, group): 2 <= M <= 32 runs the few-token tensor-core kernel
+    (2, 128, 256, "group", 128),
+    (3, 300, 1024, "channel", 0),
+    (4, 1024, 3072, "group", 128),
+    (8, 77, 512, "tensor", 0),
+    (16, 2048, 2048, "group", 64),
+    (17, 200, 768, "group", 256),
+    (24, 129, 3072, "group", 128),
+    (32, 512, 8192, "channel", 0),
+]
+
+
+@pytest.mark.parametrize("case", SKINNY_CASES, ids=lambda c: f"M{c[0]}-{c[1]}x{c[2]}-{c[3]}{c[4]}")
+def test_skinny_tensor_core_vs_oracle(sw, orc, case):
+    import torch
+    from sparse_ternary_weight_b200 import _abi
+    M, N, K, gname, group = case
+    gran = GRAN[gname]
+    W = _weights("normal", N, K, seed=9000 + N + K)
+    Xb = synth.activations_bf16(M, K, seed=9500 + M + K)
+    P = sw.quantize_pack(to_dev(W), gran, group)
+    idx, sgn, sc = packed_to_host(P)
+    y_ref = orc.linear(Xb, idx, sgn, sc, N, K, gran, group)
+    Wq = orc.unpack_f32(idx, sgn, sc, N, K, gran, group)
+    X = to_dev(Xb.view(np.int16)).view(torch.bfloat16)
+    y32 = sw.linear(X, P, torch.float32)
+    yb = sw.linear(X, P, torch.bfloat16)
+    assert _abi.lib().sherry_device_status(None) == 0
+    check_linear(y32.cpu().numpy(), y_ref, Xb, Wq)
+    check_linear(yb.float().cpu().numpy(), y_ref, Xb, Wq, y_is_bf16=True)
+    assert torch.equal(yb, y32.to(torch.bfloat16))
+
+
+def test_skinny_batch_vs_oracle(sw, orc):
+    """Several linears with 2..16 tokens in one launch of the few-token kernel."""
+    import torch
+    from sparse_ternary_weight_b200 import _abi
+    shapes = [(1024, 3072, "group", 128), (300, 3072, "channel", 0), (3072, 8192, "group", 128),
+              (77, 1024, "group", 256), (513, 2048, "tensor", 0)]
+    for M in (2, 5, 16):
+        pairs, refs = [], []
+        for i, (N, K, gname, group) in enumerate(shapes):
+            gran = GRAN[gname]
+            W = _weights("t4", N, K, seed=9900 + i)
+            Xb = synth.activations_bf16(M, K, seed=9950 + i + 10 * M)
+            P = sw.quantize_pack(to_dev(W), gran, group)
+            idx, sgn, sc = packed_to_host(P)
+            refs.append((orc.linear(Xb, idx, sgn, sc, N, K, gran, group), orc.unpack_f32(idx, sgn, sc, N, K, gran, group), Xb))
+            pairs.append((to_dev(Xb.view(np.int16)).view(torch.bfloat16), P))
+        outs = sw.linear_batched(pairs, torch.float32)
+        assert _abi.lib().sherry_device_status(None) == 0
+        for y, (y_ref, Wq, Xb) in zip(outs, refs):
+            check_linear(y.cpu().numpy(), y_ref, Xb, Wq)
