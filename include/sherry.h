@@ -125,8 +125,11 @@ int sherry_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K, int g
  *   Y        [M][N] row-major, fp32 or bf16 (y_dtype, round to nearest even);
  *            fully overwritten
  *   workspace  sherry_workspace_bytes(SHERRY_OP_LINEAR, M, N, K, g, group) bytes
- * fp32 accumulation; alpha applied once per group (or row).  M <= 16 runs the
- * lookup-table decode kernel, larger M the tensor-core (tcgen05) kernel. */
+ * fp32 accumulation; alpha applied once per group (or row).  Kernels:
+ * M == 1 a lookup-table decode kernel; 5 <= M <= 32 with K % 256 == 0 and
+ * (per-group) group % 64 == 0 a tensor-core (tcgen05) kernel for few tokens;
+ * M >= 17 with K % 64 == 0 and group % 64 == 0 the tcgen05 prefill kernel;
+ * anything else the general lookup-table kernel (any M). */
 int sherry_linear(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                   const uint32_t* idx, const uint8_t* sgn, const float* scales,
                   int granularity, int group,
@@ -146,9 +149,14 @@ typedef struct sherry_linear_desc {
 #define SHERRY_MAX_BATCH 256
 
 /* ---- batched packed linear ----------------------------------------------
- * `count` independent linears with the same M (1 <= M <= 16) in one launch,
- * e.g. the projections of a decoder layer stack for one token.  Each desc is
- * computed exactly as by sherry_linear (bit-identical Y).  `descs` is a HOST
+ * `count` independent linears with the same M in one call, e.g. the
+ * projections of a decoder layer stack for one token.  Each desc is computed
+ * as by sherry_linear, by the kernel that sherry_linear would pick for it: the
+ * problems that share a kernel share one launch of it (each prefill problem,
+ * M >= 17, gets a launch of its own).  Y agrees with sherry_linear's within the
+ * fp32 summation-order bound; the one-token kernel splits K where the batch as
+ * a whole balances best, so it is not bit-identical to a single call.  A call
+ * repeated with the same arguments gives bit-identical Y.  `descs` is a HOST
  * array, read during the call only.  count <= SHERRY_MAX_BATCH.
  *   workspace  sherry_linear_batched_workspace_bytes(descs, count, M) bytes. */
 int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M, int y_dtype,

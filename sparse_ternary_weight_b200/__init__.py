@@ -137,7 +137,7 @@ def make_batch(pairs, outs) -> "ctypes.Array":
 
 
 def linear_batched(pairs, out_dtype=None, outs=None, descs=None):
-    """Independent linears with the same M (<= 16) in one launch."""
+    """Independent linears with the same M in one call (one launch per kernel used)."""
     import torch
     out_dtype = out_dtype or torch.float32
     yd = {torch.float32: F32, torch.bfloat16: BF16}[out_dtype]

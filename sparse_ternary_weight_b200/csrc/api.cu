@@ -59,27 +59,56 @@ static bool use_stream(const ProbShape* shapes, int count, int64_t M) {
     return tiles <= kMaxTickets;
 }
 
-static bool use_skinny(const ProbShape* shapes, int count, int64_t M) {
-    if (M < 2 || M > 32 || count == 0) return false;
-    for (int i = 0; i < count; ++i)
-        if (!skinny_eligible(shapes[i], M)) return false;
-    return true;
+// Which kernel computes each problem of a call.  2 <= M <= 32 problems that fit
+// the few-token tensor-core kernel share one launch of it; of the rest, each
+// problem with M >= 17 that fits the prefill kernel gets a launch of its own;
+// what remains shares one launch of the one-token streaming kernel (M == 1,
+// every remaining problem eligible) or of the general lookup-table kernel.
+struct Routes {
+    std::vector<ProbShape> skinny_s, rest_s;
+    std::vector<sherry_linear_desc> skinny_d, rest_d;
+    std::vector<int> prefill;  // indices into the call's problems
+};
+
+static void route(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, Routes& r) {
+    for (int i = 0; i < count; ++i) {
+        if (skinny_eligible(shapes[i], M)) {
+            r.skinny_s.push_back(shapes[i]);
+            if (descs) r.skinny_d.push_back(descs[i]);
+        } else if (prefill_eligible(shapes[i], M)) {
+            r.prefill.push_back(i);
+        } else {
+            r.rest_s.push_back(shapes[i]);
+            if (descs) r.rest_d.push_back(descs[i]);
+        }
+    }
 }
 
 static size_t linear_ws_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
-    if (use_skinny(shapes, count, M)) return 0;
-    if (count == 1 && prefill_eligible(shapes[0], M)) return 0;
-    if (use_stream(shapes, count, M)) return stream_workspace_bytes(shapes, count, sms);
-    return lut_workspace_bytes(shapes, count, M, sms);
+    Routes r;
+    route(shapes, nullptr, count, M, r);
+    const int n = (int)r.rest_s.size();
+    if (n == 0) return 0;
+    if (use_stream(r.rest_s.data(), n, M)) return stream_workspace_bytes(r.rest_s.data(), n, sms);
+    return lut_workspace_bytes(r.rest_s.data(), n, M, sms);
 }
 
 static int linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream) {
-    if (use_skinny(shapes, count, M)) return skinny_linear_launch(shapes, descs, count, M, y_bf16, sms, stream);
-    if (count == 1 && prefill_eligible(shapes[0], M)) return prefill_launch(shapes[0], descs[0], M, y_bf16, stream);
-    if (use_stream(shapes, count, M))
-        return stream_linear_launch(shapes, descs, count, y_bf16, workspace, sms, stream);
-    return lut_linear_launch(shapes, descs, count, M, y_bf16, workspace, sms, stream);
+    Routes r;
+    route(shapes, descs, count, M, r);
+    int st = SHERRY_OK;
+    if (!r.skinny_s.empty() &&
+        (st = skinny_linear_launch(r.skinny_s.data(), r.skinny_d.data(), (int)r.skinny_s.size(), M, y_bf16, sms,
+                                   stream)))
+        return st;
+    for (int i : r.prefill)
+        if ((st = prefill_launch(shapes[i], descs[i], M, y_bf16, stream))) return st;
+    const int n = (int)r.rest_s.size();
+    if (n == 0) return SHERRY_OK;
+    if (use_stream(r.rest_s.data(), n, M))
+        return stream_linear_launch(r.rest_s.data(), r.rest_d.data(), n, y_bf16, workspace, sms, stream);
+    return lut_linear_launch(r.rest_s.data(), r.rest_d.data(), n, M, y_bf16, workspace, sms, stream);
 }
 
 }  // namespace sherry
@@ -198,7 +227,7 @@ static int batch_shapes(const sherry_linear_desc* descs, int count, int64_t M, s
                         std::vector<sherry_linear_desc>& kept) {
     if (!descs && count > 0) return SHERRY_ERR_NULL;
     if (count < 0 || count > SHERRY_MAX_BATCH) return SHERRY_ERR_SHAPE;
-    if (M < 0 || M > 16) return SHERRY_ERR_SHAPE;
+    if (M < 0 || M > (int64_t)0x7fffffff) return SHERRY_ERR_SHAPE;
     for (int i = 0; i < count; ++i) {
         int st = check_linear_desc(descs[i], M);
         if (st) return st;

@@ -89,8 +89,8 @@ __global__ void __launch_bounds__(kLThreads, 2) k_lut_linear(const __grid_consta
     const int wr = warp % WR;
     const int kw = warp / WR;
 
+    int pi = 0;  // problem cursor: tiles are visited in increasing order
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x) {
-        int pi = 0;
         while (pi + 1 < P.count && P.p[pi + 1].tile_begin <= t) ++pi;
         const LinProb& pr = P.p[pi];
         int local = t - pr.tile_begin;

@@ -10,17 +10,21 @@
 // of independent linears in one launch.
 //
 // Work unit: one linear's 128 weight rows x all of K.  Units are dealt to one
-// persistent CTA per SM round-robin.  Per CTA (10 warps):
-//   warps 0-3  epilogue (TMEM lane quarter = warp % 4): promote each scale
-//              group's accumulator with alpha in fp32 registers, write Y
-//   warps 4-7  decode: one TMEM lane (= weight row) per thread, per 64-weight
-//              step 16 pattern lookups -> tcgen05.st (operand A in TMEM)
-//   warp 8     producer: 16-byte cp.async of each K-chunk (256 weights): the
-//              packed words and sign bytes of the 128 rows, and the X chunk laid
-//              out as the MMA's SWIZZLE_128B K-major B operand; completion is
-//              signalled on an mbarrier (cp.async.mbarrier.arrive)
-//   warp 9     TMEM allocation; one elected thread issues tcgen05.mma
-//              (A from TMEM, B from shared memory)
+// persistent CTA per SM round-robin; K advances in chunks of 256 weights (four
+// 64-weight MMA steps).  Per CTA (22 warps):
+//   warps 0-3    epilogue (TMEM lane quarter = warp % 4): promote each scale
+//                group's accumulator with alpha in fp32 registers, write Y
+//   warps 4-19   decode, four groups of four warps: group g expands step g of
+//                every chunk, one TMEM lane (= weight row) per thread, 16
+//                pattern lookups per thread -> tcgen05.st (operand A in TMEM).
+//                Four groups keep four independent decode chains in flight.
+//   warp 20      producer: cp.async of each chunk -- the packed words (stored
+//                step-major so a group's reads are conflict-free), the sign
+//                bytes, and the X chunk laid out as the MMA's SWIZZLE_128B
+//                K-major B operand (rows >= M are zeroed once, never copied);
+//                completion is signalled on an mbarrier (cp.async.mbarrier.arrive)
+//   warp 21      TMEM allocation; one elected thread issues tcgen05.mma
+//                (A from TMEM, B from shared memory)
 // Every mbarrier wait is bounded.
 #include "common.cuh"
 #include "lut.cuh"
@@ -33,17 +37,28 @@
 
 namespace sherry {
 
-constexpr int kTThreads = 320;            // 10 warps
+constexpr int kTDecGroups = 4;                      // decode groups (one per step of a chunk)
+constexpr int kTThreads = 32 * (4 + 4 * kTDecGroups + 2);  // 22 warps
+constexpr int kTProdWarp = 4 + 4 * kTDecGroups;     // 20
+constexpr int kTMmaWarp = kTProdWarp + 1;           // 21
 constexpr int kTRows = 128;               // weight rows per unit (MMA M, TMEM lanes)
 constexpr int kTStepK = 64;               // K per MMA step (one 128-byte swizzle atom of bf16)
 constexpr int kTChunkSteps = 4;           // steps per staged chunk (256 weights)
 constexpr int kTChunkK = kTStepK * kTChunkSteps;
-constexpr int kTChunks = 4;               // staged chunks in flight
-constexpr int kTAStages = 4;              // A stages in TMEM
-constexpr int kTAcc = 3;                  // group accumulators
-constexpr int kTIdxBytes = kTRows * kTChunkSteps * 8;    // 4 KB: 8 words per row
-constexpr int kTSgnBytes = kTRows * kTChunkSteps * 2;    // 1 KB: 8 sign bytes per row
+constexpr int kTChunks = 6;               // staged chunks in flight
+constexpr int kTAStages = 2 * kTChunkSteps;  // A stages in TMEM: two per decode group
+constexpr int kTAcc = 4;                  // group accumulators
+constexpr int kTAccCols = 32;             // TMEM columns per accumulator (>= BN)
+constexpr int kTAcol = kTAcc * kTAccCols; // first A column (A stage s at kTAcol + 32 s)
+constexpr int kTTmemCols = 512;
+constexpr int kTIdxBytes = kTRows * kTChunkSteps * 8;    // 4 KB: [step][row] 8 bytes (2 words)
+constexpr int kTSgnBytes = kTRows * kTChunkSteps * 2;    // 1 KB: [row] 8 sign bytes
 constexpr long long kTWaitCycles = 4000000000LL;
+// below this many tokens the lookup-table kernels are faster (measured on the
+// 3B decode stack)
+constexpr int kSkinnyMinM = 5;
+static_assert(kTDecGroups == kTChunkSteps, "one decode group per chunk step");
+static_assert(kTAcol + 32 * kTAStages <= kTTmemCols, "TMEM plan");
 
 struct TProb {
     const uint16_t* X;
@@ -157,10 +172,10 @@ __device__ __forceinline__ void t_commit(uint32_t bar) {
                    "=r"(v[14]), "=r"(v[15])                                                               \
                  : "r"(taddr))
 
-// unit u -> (problem, row tile)
+// unit u -> (problem, row tile).  A CTA visits its units in increasing order, so
+// the problem index only moves forward: `p` is the caller's cursor (start at 0).
 template <int MAXP>
 __device__ __forceinline__ void t_locate(const TParams<MAXP>& P, int u, int& p, int& rt) {
-    p = 0;
     while (p + 1 < P.count && P.p[p + 1].unit_begin <= u) ++p;
     rt = u - P.p[p].unit_begin;
 }
@@ -170,9 +185,7 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
     constexpr int kXStep = BN * 128;                 // X bytes per 64-K step (BN rows x 128 B)
     constexpr int kXBytes = kXStep * kTChunkSteps;   // per chunk
     constexpr uint32_t kIdesc = TIdesc<BN>::v;
-    constexpr int kAccStride = 32;                   // TMEM columns per accumulator (>= BN, 32-aligned)
-    constexpr int kAcol = 128;                       // first A column in TMEM (A stages: 128..255)
-    static_assert(BN <= kAccStride && kTAcc * kAccStride <= kAcol && kAcol + 32 * kTAStages <= 256, "TMEM plan");
+    static_assert(BN <= kTAccCols, "accumulator width");
     extern __shared__ __align__(1024) unsigned char tsm[];
     __shared__ uint64_t bars[2 * kTChunks + 2 * kTAStages + 2 * kTAcc];
     __shared__ uint32_t tmem_s;
@@ -191,12 +204,13 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
     auto empty_a = [&](int s) { return bar0 + 8u * (2 * kTChunks + kTAStages + s); };
     auto acc_full = [&](int b) { return bar0 + 8u * (2 * kTChunks + 2 * kTAStages + b); };
     auto acc_empty = [&](int b) { return bar0 + 8u * (2 * kTChunks + 2 * kTAStages + kTAcc + b); };
+    const int M = P.M;
 
     if (threadIdx.x == 0) {
         abort_s = 0;
         for (int c = 0; c < kTChunks; ++c) {
-            t_mbar_init(full_c(c), 32);         // the producer warp's cp.async arrivals
-            t_mbar_init(empty_c(c), 1 + 128);   // the MMA commit (X read) + the decode threads (words read)
+            t_mbar_init(full_c(c), 32);                       // the producer warp's cp.async arrivals
+            t_mbar_init(empty_c(c), 1 + 128 * kTDecGroups);   // the MMA commit (X read) + every decode thread
         }
         for (int s = 0; s < kTAStages; ++s) {
             t_mbar_init(full_a(s), 128);
@@ -214,27 +228,40 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 4u * e), "r"(pat.x) : "memory");
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 128u + 4u * e), "r"(pat.y) : "memory");
     }
-    if (warp == 9) {
+    // token rows M..BN-1 of every X stage stay zero for the whole launch
+    for (int q = threadIdx.x; q < kTChunks * kTChunkSteps * (BN - M) * 8; q += kTThreads) {
+        const int cq = q & 7, rr = q >> 3;
+        const int r = M + rr % (BN - M), cs = rr / (BN - M);
+        const uint32_t a = xst(cs / kTChunkSteps) + (uint32_t)((cs % kTChunkSteps) * kXStep + (r >> 3) * 1024 +
+                                                               (r & 7) * 128 + (cq << 4));
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (warp == kTMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_s)),
-                     "r"(256));
+                     "r"(kTTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     t_fence_before();
     __syncthreads();
     t_fence_after();
     const uint32_t tmem = tmem_s;
-    const int M = P.M;
 
-    if (warp == 8) {
+    if (warp == kTProdWarp) {
         // ---------------- producer ----------------
         int cc = 0;  // chunks produced (all units)
+        int p = 0;   // problem cursor
         bool ok = true;
         for (int u = blockIdx.x; u < P.total_units && ok; u += gridDim.x) {
-            int p, rt;
+            int rt;
             t_locate(P, u, p, rt);
-            const TProb& pr = P.p[p];
+            const TProb& pr_ = P.p[p];
+            const uint16_t* const pr_X = pr_.X;
+            const uint32_t* const pr_idx = pr_.idx;
+            const uint8_t* const pr_sgn = pr_.sgn;
+            const int pr_N = pr_.N, pr_K = pr_.K, pr_words = pr_.words;
             const int row0 = rt * kTRows;
-            const int nchunks = pr.K / kTChunkK;
+            const int nchunks = pr_K / kTChunkK;
             for (int ch = 0; ch < nchunks; ++ch, ++cc) {
                 const int c = cc % kTChunks;
                 if (!t_mbar_wait(empty_c(c), (uint32_t)(((cc / kTChunks) & 1) ^ 1), &abort_s)) {
@@ -242,128 +269,112 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
                     break;
                 }
                 const int w0 = ch * kTChunkSteps * 2;  // first packed word of the chunk
-                // packed words: 128 rows x 32 B (two 16-B halves), half h of row r at h ^ ((r >> 2) & 1)
+                // packed words: 128 rows x 4 steps x 8 B, stored [step][row]
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     const int q = lane + 32 * i;
-                    const int r = q >> 1, h = q & 1;
+                    const int r = q >> 2, g = q & 3;
                     const int row = row0 + r;
-                    const bool v = row < pr.N;
-                    t_cp16(ist(c) + r * 32 + ((h ^ ((r >> 2) & 1)) << 4),
-                           v ? (const void*)(pr.idx + (int64_t)row * pr.words + w0 + 4 * h) : (const void*)pr.idx,
-                           v);
+                    const bool v = row < pr_N;
+                    t_cp8(ist(c) + g * (kTRows * 8) + r * 8,
+                          v ? (const void*)(pr_idx + (int64_t)row * pr_words + w0 + 2 * g) : (const void*)pr_idx, v);
                 }
                 // sign bytes: 128 rows x 8 B
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int r = lane + 32 * i;
                     const int row = row0 + r;
-                    const bool v = row < pr.N;
+                    const bool v = row < pr_N;
                     t_cp8(ist(c) + kTIdxBytes + r * 8,
-                          v ? (const void*)(pr.sgn + (int64_t)row * pr.words + w0) : (const void*)pr.sgn, v);
+                          v ? (const void*)(pr_sgn + (int64_t)row * pr_words + w0) : (const void*)pr_sgn, v);
                 }
-                // X chunk: 4 steps x BN token rows x 8 chunks of 16 B, SWIZZLE_128B K-major
-#pragma unroll
-                for (int i = 0; i < (kTChunkSteps * BN * 8) / 32; ++i) {
-                    const int q = lane + 32 * i;
-                    const int s = q / (BN * 8);
-                    const int r = (q / 8) % BN, cq = q % 8;
-                    const bool v = r < M;
-                    const int kk = ch * kTChunkK + s * kTStepK + cq * 8;
-                    t_cp16(xst(c) + s * kXStep + (r >> 3) * 1024 + (r & 7) * 128 + ((cq ^ (r & 7)) << 4),
-                           v ? (const void*)(pr.X + (int64_t)r * pr.K + kk) : (const void*)pr.X, v);
+                // X chunk, token rows < M: 4 steps x 8 pieces of 16 B per row, SWIZZLE_128B K-major
+                for (int r = 0; r < M; ++r) {
+                    const int st = lane >> 3, cq = lane & 7;
+                    const int kk = ch * kTChunkK + st * kTStepK + cq * 8;
+                    t_cp16(xst(c) + st * kXStep + (r >> 3) * 1024 + (r & 7) * 128 + ((cq ^ (r & 7)) << 4),
+                           pr_X + (int64_t)r * pr_K + kk, true);
                 }
                 t_cp_arrive(full_c(c));
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp >= 4 && warp < 8) {
-        // ---------------- decode: TMEM lane (= unit row) per thread ----------------
-        const int q = warp - 4, i = q * 32 + lane;
-        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kAcol;
-        int cc = 0, kc = 0;
+    } else if (warp >= 4 && warp < kTProdWarp) {
+        // ---------------- decode: group g expands step g of every chunk ----------------
+        const int g = (warp - 4) >> 2, q = warp & 3, i = q * 32 + lane;
+        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kTAcol;
+        int cc = 0, p = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < P.total_units && ok; u += gridDim.x) {
-            int p, rt;
+            int rt;
             t_locate(P, u, p, rt);
-            const TProb& pr = P.p[p];
-            const bool row_ok = rt * kTRows + i < pr.N;
-            const int nchunks = pr.K / kTChunkK;
-            for (int ch = 0; ch < nchunks && ok; ++ch, ++cc) {
+            const int nchunks = P.p[p].K / kTChunkK;
+            for (int ch = 0; ch < nchunks; ++ch, ++cc) {
                 const int c = cc % kTChunks;
                 if (!t_mbar_wait(full_c(c), (uint32_t)((cc / kTChunks) & 1), &abort_s)) {
                     ok = false;
                     break;
                 }
-                const uint32_t sw = ((uint32_t)(i >> 2) & 1u) << 4;
-                uint4 wlo, whi;
-                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(wlo.x), "=r"(wlo.y), "=r"(wlo.z), "=r"(wlo.w)
-                             : "r"(ist(c) + i * 32 + sw));
-                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(whi.x), "=r"(whi.y), "=r"(whi.z), "=r"(whi.w)
-                             : "r"(ist(c) + i * 32 + (16u ^ sw)));
-                uint2 sgv;
-                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(sgv.x), "=r"(sgv.y) : "r"(ist(c) + kTIdxBytes + i * 8));
+                uint32_t w_lo, w_hi, sg;
+                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                             : "=r"(w_lo), "=r"(w_hi)
+                             : "r"(ist(c) + g * (kTRows * 8) + i * 8));
+                asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sg) : "r"(ist(c) + kTIdxBytes + i * 8 + 2 * g));
                 t_mbar_arrive(empty_c(c));  // this thread has its words
-                const uint32_t words[8] = {wlo.x, wlo.y, wlo.z, wlo.w, whi.x, whi.y, whi.z, whi.w};
+                uint32_t v[32];
 #pragma unroll
-                for (int st = 0; st < kTChunkSteps; ++st, ++kc) {
-                    const int s = kc % kTAStages;
-                    uint32_t v[32];
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t wd = h ? w_hi : w_lo;
+                    const uint32_t sb = (sg >> (8 * h)) & 0xffu;
+                    const uint32_t ev = ((wd << 2) & 0x3c3c3c3cu) | (((sb & 0x55u) * 0x01041040u) & 0x40404040u);
+                    const uint32_t od = ((wd >> 2) & 0x3c3c3c3cu) | (((sb & 0xaau) * 0x00820820u) & 0x40404040u);
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t wd = words[2 * st + h];
-                        const uint32_t sg = ((st < 2 ? sgv.x : sgv.y) >> (16 * (st & 1) + 8 * h)) & 0xffu;
-                        const uint32_t ev = ((wd << 2) & 0x3c3c3c3cu) | (((sg & 0x55u) * 0x01041040u) & 0x40404040u);
-                        const uint32_t od = ((wd >> 2) & 0x3c3c3c3cu) | (((sg & 0xaau) * 0x00820820u) & 0x40404040u);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const uint32_t a = __byte_perm((j & 1) ? od : ev, table, (uint32_t)(j >> 1) | 0x7650u);
-                            uint32_t lo, hi;
-                            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo) : "r"(a));
-                            asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(hi) : "r"(a));
-                            v[16 * h + 2 * j] = row_ok ? lo : 0u;
-                            v[16 * h + 2 * j + 1] = row_ok ? hi : 0u;
-                        }
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t a = __byte_perm((j & 1) ? od : ev, table, (uint32_t)(j >> 1) | 0x7650u);
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v[16 * h + 2 * j]) : "r"(a));
+                        asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(v[16 * h + 2 * j + 1]) : "r"(a));
                     }
-                    if (!t_mbar_wait(empty_a(s), (uint32_t)(((kc / kTAStages) & 1) ^ 1), &abort_s)) {
-                        ok = false;
-                        break;
-                    }
-                    t_fence_after();
-                    SHERRY_T_ST32(t_lane + (uint32_t)(s * 32), v);
-                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                    t_fence_before();
-                    t_mbar_arrive(full_a(s));
                 }
+                const int s = 2 * g + (cc & 1);
+                if (!t_mbar_wait(empty_a(s), (uint32_t)(((cc >> 1) & 1) ^ 1), &abort_s)) {
+                    ok = false;
+                    break;
+                }
+                t_fence_after();
+                SHERRY_T_ST32(t_lane + (uint32_t)(s * 32), v);
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                t_fence_before();
+                t_mbar_arrive(full_a(s));
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == kTMmaWarp) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            int cc = 0, kc = 0, gc = 0;
+            int cc = 0, kc = 0, gc = 0, p = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < P.total_units && ok; u += gridDim.x) {
-                int p, rt;
+                int rt;
                 t_locate(P, u, p, rt);
-                const TProb& pr = P.p[p];
-                const int nk = pr.K / kTStepK, gs = pr.group_steps;
+                const int nk = P.p[p].K / kTStepK, gs = P.p[p].group_steps;
                 for (int ks = 0; ks < nk; ++ks, ++kc) {
                     const int c = cc % kTChunks, st = ks % kTChunkSteps;
-                    const int s = kc % kTAStages;
+                    const int s = 2 * st + (cc & 1);
                     const int b = gc % kTAcc;
                     const bool first = (ks % gs) == 0;
                     if (first && !t_mbar_wait(acc_empty(b), (uint32_t)(((gc / kTAcc) & 1) ^ 1), &abort_s)) { ok = false; break; }
-                    if (st == 0 && !t_mbar_wait(full_c(c), (uint32_t)((cc / kTChunks) & 1), &abort_s)) { ok = false; break; }
-                    if (!t_mbar_wait(full_a(s), (uint32_t)((kc / kTAStages) & 1), &abort_s)) { ok = false; break; }
+                    if (st == 0) {
+                        if (!t_mbar_wait(full_c(c), (uint32_t)((cc / kTChunks) & 1), &abort_s)) { ok = false; break; }
+                        // X arrived through cp.async (generic proxy); the MMA reads it through the async proxy
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    }
+                    if (!t_mbar_wait(full_a(s), (uint32_t)((cc >> 1) & 1), &abort_s)) { ok = false; break; }
                     t_fence_after();
                     const uint64_t db = t_smem_desc(xst(c) + st * kXStep);
-                    const uint32_t ta = tmem + (uint32_t)(kAcol + s * 32);
+                    const uint32_t ta = tmem + (uint32_t)(kTAcol + s * 32);
 #pragma unroll
                     for (int kk = 0; kk < kTStepK / 16; ++kk)
-                        t_mma(tmem + (uint32_t)(b * kAccStride), ta + (uint32_t)(8 * kk), db + (uint64_t)(2 * kk), kIdesc,
-                              (first && kk == 0) ? 0u : 1u);
+                        t_mma(tmem + (uint32_t)(b * kTAccCols), ta + (uint32_t)(8 * kk), db + (uint64_t)(2 * kk),
+                              kIdesc, (first && kk == 0) ? 0u : 1u);
                     t_commit(empty_a(s));
                     if (st == kTChunkSteps - 1) {
                         t_commit(empty_c(c));
@@ -377,27 +388,38 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
             }
         }
         __syncwarp();
-    } else if (warp < 4) {
+    } else {
         // ---------------- epilogue: unit row 32*warp + lane per thread ----------------
-        int gc = 0;
+        int gc = 0, p = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < P.total_units && ok; u += gridDim.x) {
-            int p, rt;
+            int rt;
             t_locate(P, u, p, rt);
-            const TProb& pr = P.p[p];
+            const TProb& pr_ = P.p[p];
+            const float* const pr_scales = pr_.scales;
+            void* const pr_Y = pr_.Y;
+            const int pr_N = pr_.N, pr_spr = pr_.spr;
+            const int row_scale = pr_.row_scale, per_tensor = pr_.per_tensor;
             const int n = rt * kTRows + warp * 32 + lane;
-            const bool row_ok = n < pr.N;
-            const int ngroups = (pr.K / kTStepK) / pr.group_steps;
+            const bool row_ok = n < pr_N;
+            const int ngroups = (pr_.K / kTStepK) / pr_.group_steps;
+            const float* srow = pr_scales + (int64_t)(row_ok ? n : 0) * pr_spr;
+            // group scales are loaded two groups ahead of their use
+            const bool gsc = !row_scale && row_ok;
+            float a_next = gsc ? __ldg(srow) : 1.0f;
+            float a_next2 = (gsc && ngroups > 1) ? __ldg(srow + 1) : 1.0f;
             float acc[BN];
 #pragma unroll
             for (int j = 0; j < BN; ++j) acc[j] = 0.0f;
-            for (int g = 0; g < ngroups; ++g, ++gc) {
+            for (int gi = 0; gi < ngroups; ++gi, ++gc) {
+                const float a = a_next;
+                a_next = a_next2;
+                a_next2 = (gsc && gi + 2 < ngroups) ? __ldg(srow + gi + 2) : 1.0f;
                 const int b = gc % kTAcc;
                 ok = t_mbar_wait(acc_full(b), (uint32_t)((gc / kTAcc) & 1), &abort_s);
                 if (!ok) break;
                 t_fence_after();
-                const float a = (!pr.row_scale && row_ok) ? __ldg(pr.scales + (int64_t)n * pr.spr + g) : 1.0f;
-                const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * kAccStride);
+                const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * kTAccCols);
                 uint32_t v[BN];
 #pragma unroll
                 for (int c = 0; c < BN / 16; ++c) SHERRY_T_LD16(t_row + 16 * c, (v + 16 * c));
@@ -408,15 +430,15 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
                 for (int j = 0; j < BN; ++j) acc[j] = fmaf(a, __uint_as_float(v[j]), acc[j]);
             }
             if (ok && row_ok) {
-                const float a = pr.row_scale ? __ldg(pr.scales + (pr.per_tensor ? 0 : n)) : 1.0f;
+                const float a = row_scale ? __ldg(pr_scales + (per_tensor ? 0 : n)) : 1.0f;
 #pragma unroll
                 for (int j = 0; j < BN; ++j) {
                     if (j < M) {
                         const float y = acc[j] * a;
                         if (P.y_bf16)
-                            reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)j * pr.N + n] = __float2bfloat16_rn(y);
+                            reinterpret_cast<__nv_bfloat16*>(pr_Y)[(int64_t)j * pr_N + n] = __float2bfloat16_rn(y);
                         else
-                            reinterpret_cast<float*>(pr.Y)[(int64_t)j * pr.N + n] = y;
+                            reinterpret_cast<float*>(pr_Y)[(int64_t)j * pr_N + n] = y;
                     }
                 }
             }
@@ -425,9 +447,9 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
 
     t_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kTMmaWarp) {
         t_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTTmemCols));
     }
 }
 
@@ -438,7 +460,7 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
 namespace sherry {
 
 bool skinny_eligible(const ProbShape& s, int64_t M) {
-    if (M < 2 || M > 32 || s.N == 0) return false;
+    if (M < kSkinnyMinM || M > 32 || s.N == 0) return false;
     if (s.K % kTChunkK != 0) return false;
     if (s.granularity == SHERRY_PER_GROUP && s.group % kTStepK != 0) return false;
     return true;
@@ -446,7 +468,7 @@ bool skinny_eligible(const ProbShape& s, int64_t M) {
 
 template <int BN>
 static constexpr int skinny_smem() {
-    return kTChunks * (BN * 128 * kTChunkSteps + kTIdxBytes + kTSgnBytes) + 256 + 1024;
+    return kTChunks * (BN * 128 * kTChunkSteps + kTIdxBytes + kTSgnBytes) + 256 + 1024;  // + table + alignment
 }
 
 template <int BN, int MAXP>

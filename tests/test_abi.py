@@ -118,7 +118,7 @@ def test_batched_validation(L):
     d = (_abi.LinearDesc * 2)()
     for i in range(2):
         d[i] = _abi.LinearDesc(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, _abi.PER_GROUP, 32)
-    assert L.sherry_linear_batched(d, 2, 17, _abi.F32, None, 0, None) == _abi.ERR_SHAPE   # M > 16
+    assert L.sherry_linear_batched(d, 2, -1, _abi.F32, None, 0, None) == _abi.ERR_SHAPE
     assert L.sherry_linear_batched(d, _abi.MAX_BATCH + 1, 1, _abi.F32, None, 0, None) == _abi.ERR_SHAPE
     d[1].K = 40
     assert L.sherry_linear_batched(d, 2, 1, _abi.F32, None, 0, None) == _abi.ERR_SHAPE

@@ -288,10 +288,10 @@ def test_prefill_tensor_core_vs_oracle(sw, orc, case):
 
 
 SKINNY_CASES = [
-    # (M, N, K, gran, group): 2 <= M <= 32 runs the few-token tensor-core kernel
-    (2, 128, 256, "group", 128),
-    (3, 300, 1024, "channel", 0),
-    (4, 1024, 3072, "group", 128),
+    # (M, N, K, gran, group): 5 <= M <= 32 runs the few-token tensor-core kernel
+    (5, 128, 256, "group", 128),
+    (6, 300, 1024, "channel", 0),
+    (7, 1024, 3072, "group", 128),
     (8, 77, 512, "tensor", 0),
     (16, 2048, 2048, "group", 64),
     (17, 200, 768, "group", 256),
@@ -322,12 +322,12 @@ def test_skinny_tensor_core_vs_oracle(sw, orc, case):
 
 
 def test_skinny_batch_vs_oracle(sw, orc):
-    """Several linears with 2..16 tokens in one launch of the few-token kernel."""
+    """Several linears with 5..16 tokens in one launch of the few-token kernel."""
     import torch
     from sparse_ternary_weight_b200 import _abi
     shapes = [(1024, 3072, "group", 128), (300, 3072, "channel", 0), (3072, 8192, "group", 128),
               (77, 1024, "group", 256), (513, 2048, "tensor", 0)]
-    for M in (2, 5, 16):
+    for M in (5, 9, 16):
         pairs, refs = [], []
         for i, (N, K, gname, group) in enumerate(shapes):
             gran = GRAN[gname]
@@ -341,3 +341,35 @@ def test_skinny_batch_vs_oracle(sw, orc):
         assert _abi.lib().sherry_device_status(None) == 0
         for y, (y_ref, Wq, Xb) in zip(outs, refs):
             check_linear(y.cpu().numpy(), y_ref, Xb, Wq)
+
+
+SKINNY_MIN_M = 5   # fewest tokens routed to the few-token tensor-core kernel
+MIXED_SHAPES = [(1024, 3072, "group", 128), (300, 768, "channel", 0), (200, 96, "group", 32),
+                (129, 3072, "group", 128), (96, 320, "group", 64), (513, 1024, "tensor", 0)]
+
+
+@pytest.mark.parametrize("M", [1, 2, 9, 20, 33, 300])
+def test_batched_mixed_routes_vs_oracle(sw, orc, M):
+    """A batch whose problems take different kernels (few-token tensor-core
+    kernel, one prefill launch each, lookup-table kernel) agrees with the oracle;
+    problems on the tensor-core kernels equal their single calls bit for bit."""
+    import torch
+    pairs, refs = [], []
+    for i, (N, K, gname, group) in enumerate(MIXED_SHAPES):
+        gran = GRAN[gname]
+        W = _weights("t4", N, K, seed=12000 + i)
+        Xb = synth.activations_bf16(M, K, seed=12500 + i + 7 * M)
+        P = sw.quantize_pack(to_dev(W), gran, group)
+        idx, sgn, sc = packed_to_host(P)
+        refs.append((orc.linear(Xb, idx, sgn, sc, N, K, gran, group), orc.unpack_f32(idx, sgn, sc, N, K, gran, group), Xb))
+        pairs.append((to_dev(Xb.view(np.int16)).view(torch.bfloat16), P))
+    outs = sw.linear_batched(pairs, torch.float32)
+    from sparse_ternary_weight_b200 import _abi
+    assert _abi.lib().sherry_device_status(None) == 0
+    for y, (y_ref, Wq, Xb) in zip(outs, refs):
+        check_linear(y.cpu().numpy(), y_ref, Xb, Wq)
+    for (X, P), y, (N, K, gname, group) in zip(pairs, outs, MIXED_SHAPES):
+        tc = (SKINNY_MIN_M <= M <= 32 and K % 256 == 0 and (gname != "group" or group % 64 == 0)) or \
+             (M >= 17 and K % 64 == 0 and (gname != "group" or group % 64 == 0))
+        if tc:
+            assert torch.equal(sw.linear(X, P), y)
