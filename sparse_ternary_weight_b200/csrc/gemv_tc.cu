@@ -11,20 +11,22 @@
 //
 // Work unit: one linear's 128 weight rows x all of K.  Units are dealt to one
 // persistent CTA per SM round-robin; K advances in chunks of 256 weights (four
-// 64-weight MMA steps).  Per CTA (22 warps):
+// 64-weight MMA steps).  Per CTA (25 warps):
 //   warps 0-3    epilogue (TMEM lane quarter = warp % 4): promote each scale
 //                group's accumulator with alpha in fp32 registers, write Y
 //   warps 4-19   decode, four groups of four warps: group g expands step g of
 //                every chunk, one TMEM lane (= weight row) per thread, 16
 //                pattern lookups per thread -> tcgen05.st (operand A in TMEM).
 //                Four groups keep four independent decode chains in flight.
-//   warp 20      producer: cp.async of each chunk -- the packed words (stored
+//   warps 20-22  producers: cp.async of each chunk -- the packed words (stored
 //                step-major so a group's reads are conflict-free), the sign
 //                bytes, and the X chunk laid out as the MMA's SWIZZLE_128B
 //                K-major B operand (rows >= M are zeroed once, never copied);
 //                completion is signalled on an mbarrier (cp.async.mbarrier.arrive)
-//   warp 21      TMEM allocation; one elected thread issues tcgen05.mma
-//                (A from TMEM, B from shared memory)
+//   warps 23-24  TMEM allocation (warp 23); one thread of each issues the
+//                tcgen05.mma sub-steps kk = me, me + 2 of every step (A from TMEM,
+//                B from shared memory) into its own column slice of the
+//                accumulator; the epilogue adds the two slices
 // Every mbarrier wait is bounded.
 #include "common.cuh"
 #include "lut.cuh"
@@ -38,19 +40,19 @@
 namespace sherry {
 
 constexpr int kTDecGroups = 4;                      // decode groups (one per step of a chunk)
-constexpr int kTThreads = 32 * (4 + 4 * kTDecGroups + 2);  // 22 warps
-constexpr int kTProdWarp = 4 + 4 * kTDecGroups;     // 20
-constexpr int kTMmaWarp = kTProdWarp + 1;           // 21
+constexpr int kTProdWarps = 2;                      // producer warps
+constexpr int kTMmaWarps = 2;                       // MMA-issuing warps (one thread each)
+constexpr int kTThreads = 32 * (4 + 4 * kTDecGroups + kTProdWarps + kTMmaWarps);  // 25 warps
+constexpr int kTProdWarp = 4 + 4 * kTDecGroups;     // first producer warp (20)
+constexpr int kTMmaWarp = kTProdWarp + kTProdWarps; // first MMA warp (23)
 constexpr int kTRows = 128;               // weight rows per unit (MMA M, TMEM lanes)
 constexpr int kTStepK = 64;               // K per MMA step (one 128-byte swizzle atom of bf16)
 constexpr int kTChunkSteps = 4;           // steps per staged chunk (256 weights)
 constexpr int kTChunkK = kTStepK * kTChunkSteps;
 constexpr int kTChunks = 6;               // staged chunks in flight
-constexpr int kTAStages = 2 * kTChunkSteps;  // A stages in TMEM: two per decode group
-constexpr int kTAcc = 4;                  // group accumulators
-constexpr int kTAccCols = 32;             // TMEM columns per accumulator (>= BN)
-constexpr int kTAcol = kTAcc * kTAccCols; // first A column (A stage s at kTAcol + 32 s)
-constexpr int kTTmemCols = 512;
+constexpr int kTAcc = 4;                  // group accumulators, each split in kTMmaWarps column slices
+constexpr int kTTmemCols = 512;           // accumulators first, then the A stages
+constexpr int kTAParMax = 3;              // A buffers per decode group, at most
 constexpr int kTIdxBytes = kTRows * kTChunkSteps * 8;    // 4 KB: [step][row] 8 bytes (2 words)
 constexpr int kTSgnBytes = kTRows * kTChunkSteps * 2;    // 1 KB: [row] 8 sign bytes
 constexpr long long kTWaitCycles = 4000000000LL;
@@ -58,7 +60,7 @@ constexpr long long kTWaitCycles = 4000000000LL;
 // 3B decode stack)
 constexpr int kSkinnyMinM = 5;
 static_assert(kTDecGroups == kTChunkSteps, "one decode group per chunk step");
-static_assert(kTAcol + 32 * kTAStages <= kTTmemCols, "TMEM plan");
+static_assert(kTAParMax < kTChunks, "an A buffer's release is still tracked by its chunk slot");
 
 struct TProb {
     const uint16_t* X;
@@ -185,9 +187,15 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
     constexpr int kXStep = BN * 128;                 // X bytes per 64-K step (BN rows x 128 B)
     constexpr int kXBytes = kXStep * kTChunkSteps;   // per chunk
     constexpr uint32_t kIdesc = TIdesc<BN>::v;
-    static_assert(BN <= kTAccCols, "accumulator width");
+    constexpr int kAccCols = kTMmaWarps * BN;        // TMEM columns per accumulator
+    constexpr int kAcolT = kTAcc * kAccCols;         // first A column
+    // A buffers per decode group: as many as TMEM holds (3 for 16 token columns, 2 for 32);
+    // A stage (group g, buffer h) at column kAcolT + 32 (kAPar g + h)
+    constexpr int kAPar0 = (kTTmemCols - kAcolT) / (32 * kTDecGroups);
+    constexpr int kAPar = kAPar0 < kTAParMax ? kAPar0 : kTAParMax;
+    static_assert(BN % 16 == 0 && kAPar >= 2, "TMEM plan");
     extern __shared__ __align__(1024) unsigned char tsm[];
-    __shared__ uint64_t bars[2 * kTChunks + 2 * kTAStages + 2 * kTAcc];
+    __shared__ uint64_t bars[2 * kTChunks + kTAParMax + 2 * kTAcc];
     __shared__ uint32_t tmem_s;
     __shared__ volatile int abort_s;
 
@@ -200,24 +208,21 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
     const uint32_t bar0 = smem_u32(&bars[0]);
     auto full_c = [&](int c) { return bar0 + 8u * c; };
     auto empty_c = [&](int c) { return bar0 + 8u * (kTChunks + c); };
-    auto full_a = [&](int s) { return bar0 + 8u * (2 * kTChunks + s); };
-    auto empty_a = [&](int s) { return bar0 + 8u * (2 * kTChunks + kTAStages + s); };
-    auto acc_full = [&](int b) { return bar0 + 8u * (2 * kTChunks + 2 * kTAStages + b); };
-    auto acc_empty = [&](int b) { return bar0 + 8u * (2 * kTChunks + 2 * kTAStages + kTAcc + b); };
+    auto full_a = [&](int h) { return bar0 + 8u * (2 * kTChunks + h); };  // A buffer h of every group written
+    auto acc_full = [&](int b) { return bar0 + 8u * (2 * kTChunks + kTAParMax + b); };
+    auto acc_empty = [&](int b) { return bar0 + 8u * (2 * kTChunks + kTAParMax + kTAcc + b); };
     const int M = P.M;
 
     if (threadIdx.x == 0) {
         abort_s = 0;
         for (int c = 0; c < kTChunks; ++c) {
-            t_mbar_init(full_c(c), 32);                       // the producer warp's cp.async arrivals
-            t_mbar_init(empty_c(c), 1 + 128 * kTDecGroups);   // the MMA commit (X read) + every decode thread
+            t_mbar_init(full_c(c), 32 * kTProdWarps);         // the producer warps' cp.async arrivals
+            // the MMA commit (X and the chunk's A stages read) + every decode thread (words read)
+            t_mbar_init(empty_c(c), kTMmaWarps + 128 * kTDecGroups);
         }
-        for (int s = 0; s < kTAStages; ++s) {
-            t_mbar_init(full_a(s), 128);
-            t_mbar_init(empty_a(s), 1);
-        }
+        for (int h = 0; h < kAPar; ++h) t_mbar_init(full_a(h), 128 * kTDecGroups);
         for (int b = 0; b < kTAcc; ++b) {
-            t_mbar_init(acc_full(b), 1);
+            t_mbar_init(acc_full(b), kTMmaWarps);
             t_mbar_init(acc_empty(b), 128);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -247,8 +252,9 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
     t_fence_after();
     const uint32_t tmem = tmem_s;
 
-    if (warp == kTProdWarp) {
-        // ---------------- producer ----------------
+    if (warp >= kTProdWarp && warp < kTProdWarp + kTProdWarps) {
+        // ---------------- producers: copy job j of a chunk goes to warp j % kTProdWarps ----------------
+        const int pw = warp - kTProdWarp;
         int cc = 0;  // chunks produced (all units)
         int p = 0;   // problem cursor
         bool ok = true;
@@ -271,7 +277,7 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
                 const int w0 = ch * kTChunkSteps * 2;  // first packed word of the chunk
                 // packed words: 128 rows x 4 steps x 8 B, stored [step][row]
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = pw; i < 16; i += kTProdWarps) {
                     const int q = lane + 32 * i;
                     const int r = q >> 2, g = q & 3;
                     const int row = row0 + r;
@@ -281,7 +287,7 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
                 }
                 // sign bytes: 128 rows x 8 B
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = pw; i < 4; i += kTProdWarps) {
                     const int r = lane + 32 * i;
                     const int row = row0 + r;
                     const bool v = row < pr_N;
@@ -289,7 +295,7 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
                           v ? (const void*)(pr_sgn + (int64_t)row * pr_words + w0) : (const void*)pr_sgn, v);
                 }
                 // X chunk, token rows < M: 4 steps x 8 pieces of 16 B per row, SWIZZLE_128B K-major
-                for (int r = 0; r < M; ++r) {
+                for (int r = pw; r < M; r += kTProdWarps) {
                     const int st = lane >> 3, cq = lane & 7;
                     const int kk = ch * kTChunkK + st * kTStepK + cq * 8;
                     t_cp16(xst(c) + st * kXStep + (r >> 3) * 1024 + (r & 7) * 128 + ((cq ^ (r & 7)) << 4),
@@ -302,7 +308,7 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
     } else if (warp >= 4 && warp < kTProdWarp) {
         // ---------------- decode: group g expands step g of every chunk ----------------
         const int g = (warp - 4) >> 2, q = warp & 3, i = q * 32 + lane;
-        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kTAcol;
+        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kAcolT;
         int cc = 0, p = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < P.total_units && ok; u += gridDim.x) {
@@ -335,57 +341,75 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
                         asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(v[16 * h + 2 * j + 1]) : "r"(a));
                     }
                 }
-                const int s = 2 * g + (cc & 1);
-                if (!t_mbar_wait(empty_a(s), (uint32_t)(((cc >> 1) & 1) ^ 1), &abort_s)) {
-                    ok = false;
-                    break;
+                // stage (g, cc % kAPar) was last read by the MMAs of chunk cc - kAPar, whose
+                // completion the MMA threads commit to that chunk's slot barrier
+                const int h = cc % kAPar;
+                const int s = kAPar * g + h;
+                if (cc >= kAPar) {
+                    const int c2 = (cc - kAPar) % kTChunks;
+                    if (!t_mbar_wait(empty_c(c2), (uint32_t)(((cc - kAPar) / kTChunks) & 1), &abort_s)) {
+                        ok = false;
+                        break;
+                    }
                 }
                 t_fence_after();
                 SHERRY_T_ST32(t_lane + (uint32_t)(s * 32), v);
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                 t_fence_before();
-                t_mbar_arrive(full_a(s));
+                t_mbar_arrive(full_a(h));
             }
         }
-    } else if (warp == kTMmaWarp) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp >= kTMmaWarp) {
+        // ---------------- MMA issuers: warp kTMmaWarp + me issues sub-steps kk of every step
+        // with kk % kTMmaWarps == me into its own column slice of the accumulator ----------------
+        const int me = warp - kTMmaWarp;
+        // One wait per chunk (all four A stages written; the decode threads had
+        // waited for the chunk's X, so it has landed too), 16 MMAs, one commit
+        // per chunk; group bookkeeping by counters only.
         if (lane == 0) {
-            int cc = 0, kc = 0, gc = 0, p = 0;
+            int cc = 0, c = 0, p = 0;
+            uint32_t cph = 0;           // phase parity of slot c
+            int b = 0;                  // accumulator
+            uint32_t bph = 0;           // phase parity of accumulator b's use
             bool ok = true;
             for (int u = blockIdx.x; u < P.total_units && ok; u += gridDim.x) {
                 int rt;
                 t_locate(P, u, p, rt);
-                const int nk = P.p[p].K / kTStepK, gs = P.p[p].group_steps;
-                for (int ks = 0; ks < nk; ++ks, ++kc) {
-                    const int c = cc % kTChunks, st = ks % kTChunkSteps;
-                    const int s = 2 * st + (cc & 1);
-                    const int b = gc % kTAcc;
-                    const bool first = (ks % gs) == 0;
-                    if (first && !t_mbar_wait(acc_empty(b), (uint32_t)(((gc / kTAcc) & 1) ^ 1), &abort_s)) { ok = false; break; }
-                    if (st == 0) {
-                        if (!t_mbar_wait(full_c(c), (uint32_t)((cc / kTChunks) & 1), &abort_s)) { ok = false; break; }
-                        // X arrived through cp.async (generic proxy); the MMA reads it through the async proxy
-                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    }
-                    if (!t_mbar_wait(full_a(s), (uint32_t)((cc >> 1) & 1), &abort_s)) { ok = false; break; }
+                const int nchunks = P.p[p].K / kTChunkK, gs = P.p[p].group_steps;
+                int gstep = 0;          // steps done in the current group
+                for (int ch = 0; ch < nchunks; ++ch, ++cc) {
+                    const int h = cc % kAPar;
+                    if (!t_mbar_wait(full_a(h), (uint32_t)((cc / kAPar) & 1), &abort_s)) { ok = false; break; }
+                    // X arrived through cp.async (generic proxy); the MMA reads it through the async proxy
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     t_fence_after();
-                    const uint64_t db = t_smem_desc(xst(c) + st * kXStep);
-                    const uint32_t ta = tmem + (uint32_t)(kTAcol + s * 32);
+                    const uint64_t db0 = t_smem_desc(xst(c));
+                    const uint32_t ta0 = tmem + (uint32_t)(kAcolT + h * 32);
 #pragma unroll
-                    for (int kk = 0; kk < kTStepK / 16; ++kk)
-                        t_mma(tmem + (uint32_t)(b * kTAccCols), ta + (uint32_t)(8 * kk), db + (uint64_t)(2 * kk),
-                              kIdesc, (first && kk == 0) ? 0u : 1u);
-                    t_commit(empty_a(s));
-                    if (st == kTChunkSteps - 1) {
-                        t_commit(empty_c(c));
-                        ++cc;
+                    for (int st = 0; st < kTChunkSteps; ++st) {
+                        if (gstep == 0) {
+                            if (!t_mbar_wait(acc_empty(b), bph ^ 1u, &abort_s)) { ok = false; break; }
+                            t_fence_after();
+                        }
+                        const uint32_t td = tmem + (uint32_t)(b * kAccCols + me * BN);
+                        const uint32_t ta = ta0 + (uint32_t)(st * kAPar * 32);
+                        const uint64_t db = db0 + (uint64_t)((st * kXStep) >> 4);
+#pragma unroll
+                        for (int kk = me; kk < kTStepK / 16; kk += kTMmaWarps)
+                            t_mma(td, ta + (uint32_t)(8 * kk), db + (uint64_t)(2 * kk), kIdesc,
+                                  (gstep == 0 && kk == me) ? 0u : 1u);
+                        if (++gstep == gs) {
+                            t_commit(acc_full(b));
+                            gstep = 0;
+                            if (++b == kTAcc) { b = 0; bph ^= 1u; }
+                        }
                     }
-                    if ((ks % gs) == gs - 1) {
-                        t_commit(acc_full(b));
-                        ++gc;
-                    }
+                    if (!ok) break;
+                    t_commit(empty_c(c));
+                    if (++c == kTChunks) { c = 0; cph ^= 1u; }
                 }
             }
+            (void)cph;
         }
         __syncwarp();
     } else {
@@ -419,15 +443,24 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
                 ok = t_mbar_wait(acc_full(b), (uint32_t)((gc / kTAcc) & 1), &abort_s);
                 if (!ok) break;
                 t_fence_after();
-                const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * kTAccCols);
-                uint32_t v[BN];
+                const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * kAccCols);
+                // 16 token columns at a time: the slices' partial sums, added in a fixed order
 #pragma unroll
-                for (int c = 0; c < BN / 16; ++c) SHERRY_T_LD16(t_row + 16 * c, (v + 16 * c));
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                for (int c = 0; c < BN / 16; ++c) {
+                    uint32_t v[16 * kTMmaWarps];
+#pragma unroll
+                    for (int m = 0; m < kTMmaWarps; ++m) SHERRY_T_LD16(t_row + m * BN + 16 * c, (v + 16 * m));
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        float g = __uint_as_float(v[j]);
+#pragma unroll
+                        for (int m = 1; m < kTMmaWarps; ++m) g += __uint_as_float(v[16 * m + j]);
+                        acc[16 * c + j] = fmaf(a, g, acc[16 * c + j]);
+                    }
+                }
                 t_fence_before();
                 t_mbar_arrive(acc_empty(b));
-#pragma unroll
-                for (int j = 0; j < BN; ++j) acc[j] = fmaf(a, __uint_as_float(v[j]), acc[j]);
             }
             if (ok && row_ok) {
                 const float a = row_scale ? __ldg(pr_scales + (per_tensor ? 0 : n)) : 1.0f;
