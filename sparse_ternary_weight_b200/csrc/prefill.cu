@@ -9,20 +9,23 @@
 // accumulated separately in TMEM and promoted into fp32 registers with alpha
 // (per-row scales: once at the end).
 //
-// CTA tile: 128 weight rows (MMA M, TMEM lanes) x 128 tokens (MMA N), K in
-// steps of 64.  The expanded weights (MMA operand A) never touch shared memory:
-// decode threads own one TMEM lane (= weight row) each and write their row's
-// 64 bf16 of a step into TMEM with tcgen05.st; only the X tiles (operand B)
-// come through shared memory, by TMA (no multicast).
-//   warps 0-7  epilogue: wait for one of three finished group accumulators,
-//              tcgen05.ld its 64-token half, acc[token] += alpha(row, group) * D,
-//              write Y (row per thread)
-//   warps 8-11 decode: per block one table lookup (32 bf16x4 patterns indexed by
-//              nibble + 16*sign) -> tcgen05.st into the A stage of their lanes
-//   warp 12    TMA: X tiles [128 tokens x 64 K], SWIZZLE_128B
-//   warp 13    TMEM allocation; one elected thread issues tcgen05.mma
-// Every mbarrier wait is bounded; on timeout the CTA sets a device status flag
-// and drains instead of hanging.
+// CTA tile: 128 weight rows (MMA M, TMEM lanes) x 128 tokens (MMA N); K runs in
+// chunks of 256 (four 64-wide MMA steps).  The expanded weights (MMA operand A)
+// never touch shared memory: decode threads own one TMEM lane (= weight row)
+// each and write their row's 64 bf16 of a step into TMEM with tcgen05.st; only
+// the X tiles (operand B) come through shared memory, by TMA (no multicast).
+// Synchronisation is per chunk: the MMA thread waits once for the chunk's four A
+// stages and once for its X, issues the 16 MMAs, and commits once; that commit
+// frees both the X slot and the chunk's A buffer.
+//   warps 0-7    epilogue: wait for one of two finished group accumulators,
+//                tcgen05.ld its 64-token half, acc[token] += alpha(row, group) * D,
+//                write Y (row per thread)
+//   warps 8-15   decode, two groups of four warps: group g expands steps 2g and
+//                2g + 1 of every chunk, one pattern-table lookup per block of 4
+//                weights; packed words come straight from global memory through
+//                a per-thread prefetch ring
+//   warp 16      TMA: the chunk's four X tiles [128 tokens x 64 K], SWIZZLE_128B
+//   warp 17      TMEM allocation; one elected thread issues tcgen05.mma
 #include "common.cuh"
 #include "lut.cuh"
 
@@ -33,20 +36,27 @@
 
 namespace sherry {
 
-constexpr int kPThreads = 448;   // 8 epilogue + 4 decode + TMA + MMA warps
+constexpr int kPDecGroups = 2;   // decode groups (two MMA steps of every chunk each)
+constexpr int kPThreads = 32 * (8 + 4 * kPDecGroups + 2);  // 18 warps
+constexpr int kPTmaWarp = 8 + 4 * kPDecGroups;   // 16
+constexpr int kPMmaWarp = kPTmaWarp + 1;         // 17
 constexpr int kPBM = 128;     // weight rows per tile
 constexpr int kPBN = 128;     // tokens per tile
-constexpr int kPBK = 64;      // K per stage
-constexpr int kPStages = 4;
-constexpr int kPStageB = kPBN * kPBK * 2;  // 16 KB of X per stage
-constexpr int kPTable = 256;               // 32 weight patterns: low words (128 B), then high words
-constexpr int kPPrefetch = 4;              // K-steps of packed words in flight per decode thread
-constexpr int kPSmem = kPStages * kPStageB + kPTable + 1024;
-constexpr int kPAcc = 3;                   // group accumulators in flight
-constexpr int kPTmemCols = 512;            // 3 x 128 accumulator columns + 4 x 32 A columns
-constexpr int kPAcol = kPAcc * kPBN;       // first TMEM column of the A stages (384)
-constexpr int kPAcols = kPBK / 2;          // 32 columns (64 bf16) per A stage
+constexpr int kPBK = 64;      // K per MMA step
+constexpr int kPChunkSteps = 4;                  // steps per chunk
+constexpr int kPStepB = kPBN * kPBK * 2;         // 16 KB of X per step
+constexpr int kPChunkB = kPChunkSteps * kPStepB; // 64 KB of X per chunk
+constexpr int kPXSlots = 3;                      // X chunks in flight
+constexpr int kPTable = 256;                     // 32 weight patterns: low words (128 B), then high words
+constexpr int kPRing = 2;                        // chunks of packed words in flight per decode thread
+constexpr int kPSmem = kPXSlots * kPChunkB + kPTable + 1024;
+constexpr int kPAcc = 2;                         // group accumulators in flight
+constexpr int kPTmemCols = 512;                  // 2 x 128 accumulator columns + 2 x 4 x 32 A columns
+constexpr int kPAcol = kPAcc * kPBN;             // first TMEM column of the A stages (256)
+constexpr int kPAcols = kPBK / 2;                // 32 columns (64 bf16) per A stage
 constexpr long long kPWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+static_assert(kPAcol + 2 * kPChunkSteps * kPAcols <= kPTmemCols, "TMEM plan");
+static_assert(kPXSlots >= 3, "the decode's A-buffer wait reads the slot barrier of chunk cc - 2");
 
 __device__ int g_device_status = 0;
 
@@ -152,6 +162,14 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+#define SHERRY_TMEM_LD16(taddr, v)                                                                       \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+                 "%15}, [%16];"                                                                          \
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),    \
+                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), \
+                   "=r"(v[14]), "=r"(v[15])                                                               \
+                 : "r"(taddr))
+
 #define SHERRY_TMEM_LD32(taddr, v)                                                                               \
     asm volatile(                                                                                                \
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17," \
@@ -166,36 +184,37 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 __global__ void __launch_bounds__(kPThreads, 1)
 k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PParams P) {
     extern __shared__ __align__(1024) unsigned char psmem[];
-    __shared__ uint64_t bars[3 * kPStages + 2 * kPAcc];
+    __shared__ uint64_t bars[2 * kPXSlots + 2 + 2 * kPAcc];
     __shared__ uint32_t tmem_base_s;
     __shared__ volatile int abort_s;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t base = (smem_u32(psmem) + 1023u) & ~1023u;
-    const uint32_t stB = base;                             // kPStages x 16 KB, 1024-aligned
-    const uint32_t table = base + kPStages * kPStageB;     // 256-aligned
+    const uint32_t stX = base;                               // kPXSlots x 64 KB, 1024-aligned
+    const uint32_t table = base + kPXSlots * kPChunkB;       // 256-aligned
     const uint32_t bar0 = smem_u32(&bars[0]);
-    auto full_a = [&](int s) { return bar0 + 8u * s; };
-    auto full_b = [&](int s) { return bar0 + 8u * (kPStages + s); };
-    auto empty = [&](int s) { return bar0 + 8u * (2 * kPStages + s); };
-    auto acc_full = [&](int b) { return bar0 + 8u * (3 * kPStages + b); };
-    auto acc_empty = [&](int b) { return bar0 + 8u * (3 * kPStages + kPAcc + b); };
+    auto full_x = [&](int c) { return bar0 + 8u * c; };                    // X chunk in slot c landed
+    auto chunk_empty = [&](int c) { return bar0 + 8u * (kPXSlots + c); };  // MMAs of slot c's chunk done
+    auto full_a = [&](int h) { return bar0 + 8u * (2 * kPXSlots + h); };   // A buffer h written
+    auto acc_full = [&](int b) { return bar0 + 8u * (2 * kPXSlots + 2 + b); };
+    auto acc_empty = [&](int b) { return bar0 + 8u * (2 * kPXSlots + 2 + kPAcc + b); };
 
     // persistent: tile t = (weight-row tile t % ntn, token tile t / ntn), strided by the grid;
-    // stage and accumulator phases run on across tiles
+    // chunk and accumulator phases run on across tiles
     const int ntn = (P.N + kPBM - 1) / kPBM;
     const int ntiles = ntn * ((P.M + kPBN - 1) / kPBN);
     const int nk = P.K / kPBK;
+    const int nchunks = (nk + kPChunkSteps - 1) / kPChunkSteps;  // the last one may hold fewer steps
     const int gs = P.group_steps;
     const int ngroups = nk / gs;
 
     if (threadIdx.x == 0) {
         abort_s = 0;
-        for (int s = 0; s < kPStages; ++s) {
-            mbar_init(full_a(s), 128);
-            mbar_init(full_b(s), 1);
-            mbar_init(empty(s), 1);
+        for (int c = 0; c < kPXSlots; ++c) {
+            mbar_init(full_x(c), 1);
+            mbar_init(chunk_empty(c), 1);
         }
+        for (int h = 0; h < 2; ++h) mbar_init(full_a(h), 128 * kPDecGroups);
         for (int b = 0; b < kPAcc; ++b) {
             mbar_init(acc_full(b), 1);
             mbar_init(acc_empty(b), 256);
@@ -210,7 +229,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 4u * threadIdx.x), "r"(e.x) : "memory");
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 128u + 4u * threadIdx.x), "r"(e.y) : "memory");
     }
-    if (warp == 13) {
+    if (warp == kPMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
                      "r"(kPTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -226,33 +245,40 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
         const int q = warp & 3, half = warp >> 2;
         constexpr int kCols = kPBN / 2;
         bool ok = true;
-        int gc = 0;  // groups consumed so far (all tiles)
+        int b = 0;
+        uint32_t bph = 0;  // phase parity of accumulator b's use
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             const int n = (t % ntn) * kPBM + q * 32 + lane;
             const int m0 = (t / ntn) * kPBN + half * kCols;
             const bool row_ok = n < P.N;
+            const bool gsc = !P.row_scale && row_ok;
+            const float* srow = P.scales + (int64_t)(row_ok ? n : 0) * P.spr;
+            // group scales are loaded two groups ahead of their use
+            float a_next = gsc ? __ldg(srow) : 1.0f;
+            float a_next2 = (gsc && ngroups > 1) ? __ldg(srow + 1) : 1.0f;
             float acc[kCols];
 #pragma unroll
             for (int j = 0; j < kCols; ++j) acc[j] = 0.0f;
-            for (int g = 0; g < ngroups; ++g, ++gc) {
-                const int b = gc % kPAcc;
-                ok = mbar_wait(acc_full(b), (uint32_t)((gc / kPAcc) & 1), &abort_s);
+            for (int g = 0; g < ngroups; ++g) {
+                const float a = a_next;
+                a_next = a_next2;
+                a_next2 = (gsc && g + 2 < ngroups) ? __ldg(srow + g + 2) : 1.0f;
+                ok = mbar_wait(acc_full(b), bph, &abort_s);
                 if (!ok) break;
                 tc_fence_after();
-                float a = 1.0f;
-                if (!P.row_scale && row_ok) a = __ldg(P.scales + (int64_t)n * P.spr + g);  // group g: K-steps [g*gs, (g+1)*gs)
                 const uint32_t t_row = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kPBN + half * kCols);
-                uint32_t v0[32], v1[32];
-                SHERRY_TMEM_LD32(t_row, v0);
-                SHERRY_TMEM_LD32(t_row + 32, v1);
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                // 16 columns at a time keeps the 64 running sums in registers
+#pragma unroll
+                for (int c = 0; c < kCols / 16; ++c) {
+                    uint32_t v[16];
+                    SHERRY_TMEM_LD16(t_row + 16 * c, v);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) acc[16 * c + j] = fmaf(a, __uint_as_float(v[j]), acc[16 * c + j]);
+                }
                 tc_fence_before();
                 mbar_arrive(acc_empty(b));
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    acc[j] = fmaf(a, __uint_as_float(v0[j]), acc[j]);
-                    acc[32 + j] = fmaf(a, __uint_as_float(v1[j]), acc[32 + j]);
-                }
+                if (++b == kPAcc) { b = 0; bph ^= 1u; }
             }
             if (ok && row_ok) {
                 float a = 1.0f;
@@ -270,117 +296,160 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
                 }
             }
         }
-    } else if (warp < 12) {
-        // ---------------- decode: TMEM lane (= tile row) i per thread ----------------
-        const int q = warp - 8;                 // lane quarter of this warp (warp % 4)
+    } else if (warp < kPTmaWarp) {
+        // ---------------- decode: TMEM lane (= tile row) i per thread; group g expands
+        // steps 2g, 2g + 1 of every chunk into A buffer (cc & 1) ----------------
+        const int g = (warp - 8) >> 2, q = warp & 3;
         const int i = q * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kPAcol;
-        int kc = 0;  // K-steps produced so far (all tiles)
+        int cc = 0;  // chunks done so far (all tiles)
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             const int n = (t % ntn) * kPBM + i;
             const bool row_ok = n < P.N;
             const uint32_t* idxr = P.idx + (int64_t)(row_ok ? n : 0) * P.words;
             const uint8_t* sgnr = P.sgn + (int64_t)(row_ok ? n : 0) * P.words;
-            // ring of the next kPPrefetch steps' packed words (2 idx words + 2 sign bytes each)
-            uint2 rw[kPPrefetch];
-            uint32_t rs[kPPrefetch];
+            // ring of the next kPRing chunks' packed words: per step 2 idx words + 2 sign bytes
+            uint2 rw[kPRing][2];
+            uint32_t rs[kPRing][2];
+            auto fetch = [&](int ch, uint2* w, uint32_t* sg) {
 #pragma unroll
-            for (int u = 0; u < kPPrefetch; ++u) {
-                rw[u] = make_uint2(0u, 0u);
-                rs[u] = 0u;
-                if (row_ok && u < nk) {
-                    rw[u] = __ldg(reinterpret_cast<const uint2*>(idxr + 2 * u));
-                    rs[u] = __ldg(reinterpret_cast<const uint16_t*>(sgnr + 2 * u));
+                for (int e = 0; e < 2; ++e) {
+                    const int ks = ch * kPChunkSteps + 2 * g + e;
+                    w[e] = make_uint2(0u, 0u);
+                    sg[e] = 0u;
+                    if (row_ok && ch < nchunks && ks < nk) {
+                        w[e] = __ldg(reinterpret_cast<const uint2*>(idxr + 2 * ks));
+                        sg[e] = __ldg(reinterpret_cast<const uint16_t*>(sgnr + 2 * ks));
+                    }
                 }
-            }
-            for (int ks0 = 0; ks0 < nk && ok; ks0 += kPPrefetch) {
+            };
 #pragma unroll
-                for (int u = 0; u < kPPrefetch; ++u) {
-                    const int ks = ks0 + u;
-                    if (ks >= nk) break;
-                    const int s = kc % kPStages;
-                    const uint2 w = rw[u];
-                    const uint32_t sb = rs[u];
-                    if (ks + kPPrefetch < nk && row_ok) {
-                        rw[u] = __ldg(reinterpret_cast<const uint2*>(idxr + 2 * (ks + kPPrefetch)));
-                        rs[u] = __ldg(reinterpret_cast<const uint16_t*>(sgnr + 2 * (ks + kPPrefetch)));
-                    }
-                    // table offsets (4 * (nibble + 16 G)) of the even / odd blocks of each word
-                    uint32_t v[32];
+            for (int r = 0; r < kPRing; ++r) fetch(r, rw[r], rs[r]);
+            for (int ch0 = 0; ch0 < nchunks && ok; ch0 += kPRing) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t wd = h ? w.y : w.x;
-                        const uint32_t sg = (sb >> (8 * h)) & 0xffu;
-                        const uint32_t ev = ((wd << 2) & 0x3c3c3c3cu) | (((sg & 0x55u) * 0x01041040u) & 0x40404040u);
-                        const uint32_t od = ((wd >> 2) & 0x3c3c3c3cu) | (((sg & 0xaau) * 0x00820820u) & 0x40404040u);
+                for (int r = 0; r < kPRing; ++r) {
+                    const int ch = ch0 + r;
+                    if (ch >= nchunks) break;
+                    uint2 w[2] = {rw[r][0], rw[r][1]};
+                    uint32_t sb[2] = {rs[r][0], rs[r][1]};
+                    fetch(ch + kPRing, rw[r], rs[r]);
+                    const int hbuf = cc & 1;
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const uint32_t src = (j & 1) ? od : ev;
-                            const uint32_t a = __byte_perm(src, table, (uint32_t)(j >> 1) | 0x7650u);
-                            uint32_t lo, hi;
-                            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(lo) : "r"(a));
-                            asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(hi) : "r"(a));
-                            v[16 * h + 2 * j] = row_ok ? lo : 0u;
-                            v[16 * h + 2 * j + 1] = row_ok ? hi : 0u;
+                    for (int e = 0; e < 2; ++e) {
+                        const int st = 2 * g + e;
+                        if (ch * kPChunkSteps + st >= nk) break;
+                        uint32_t v[32];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t wd = h ? w[e].y : w[e].x;
+                            const uint32_t sg = (sb[e] >> (8 * h)) & 0xffu;
+                            const uint32_t ev = ((wd << 2) & 0x3c3c3c3cu) | (((sg & 0x55u) * 0x01041040u) & 0x40404040u);
+                            const uint32_t od = ((wd >> 2) & 0x3c3c3c3cu) | (((sg & 0xaau) * 0x00820820u) & 0x40404040u);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const uint32_t a = __byte_perm((j & 1) ? od : ev, table, (uint32_t)(j >> 1) | 0x7650u);
+                                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v[16 * h + 2 * j]) : "r"(a));
+                                asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(v[16 * h + 2 * j + 1]) : "r"(a));
+                            }
                         }
+                        // A buffer hbuf was last read by the MMAs of chunk cc - 2, whose
+                        // completion the MMA thread commits to that chunk's slot barrier
+                        if (e == 0 && cc >= 2) {
+                            if (!mbar_wait(chunk_empty((cc - 2) % kPXSlots), (uint32_t)(((cc - 2) / kPXSlots) & 1),
+                                           &abort_s)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                        }
+                        SHERRY_TMEM_ST32(t_lane + (uint32_t)((hbuf * kPChunkSteps + st) * kPAcols), v);
                     }
-                    if (!mbar_wait(empty(s), (uint32_t)(((kc / kPStages) & 1) ^ 1), &abort_s)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    SHERRY_TMEM_ST32(t_lane + (uint32_t)(s * kPAcols), v);
+                    if (!ok) break;
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                     tc_fence_before();
-                    mbar_arrive(full_a(s));
-                    ++kc;
+                    mbar_arrive(full_a(hbuf));
+                    ++cc;
                 }
             }
         }
-    } else if (warp == 12) {
+    } else if (warp == kPTmaWarp) {
         // ---------------- TMA producer for X ----------------
         if (lane == 0) {
-            int kc = 0;
+            int c = 0;
+            uint32_t cph = 0;  // phase parity of slot c's use
             bool ok = true;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const int m0 = (t / ntn) * kPBN;
-                for (int ks = 0; ks < nk; ++ks, ++kc) {
-                    const int s = kc % kPStages;
-                    if (!mbar_wait(empty(s), (uint32_t)(((kc / kPStages) & 1) ^ 1), &abort_s)) {
+                for (int ch = 0; ch < nchunks; ++ch) {
+                    if (!mbar_wait(chunk_empty(c), cph ^ 1u, &abort_s)) {
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(full_b(s), kPStageB);
-                    tma_load_2d(stB + s * kPStageB, &xmap, ks * kPBK, m0, full_b(s));
+                    const int steps = min(kPChunkSteps, nk - ch * kPChunkSteps);
+                    mbar_expect_tx(full_x(c), (uint32_t)(steps * kPStepB));
+                    for (int st = 0; st < steps; ++st)
+                        tma_load_2d(stX + c * kPChunkB + st * kPStepB, &xmap, (ch * kPChunkSteps + st) * kPBK, m0,
+                                    full_x(c));
+                    if (++c == kPXSlots) { c = 0; cph ^= 1u; }
                 }
             }
         }
     } else {
         // ---------------- MMA issuer ----------------
+        // A single thread issues every MMA, so its own instruction stream is on the
+        // critical path: full chunks take an unrolled path, group boundaries are a
+        // count-down, and operand addresses are fixed offsets from the chunk base.
         if (lane == 0) {
-            int kc = 0, gc = 0;
+            int cc = 0, c = 0, b = 0;
+            uint32_t cph = 0, bph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                for (int ks = 0; ks < nk; ++ks, ++kc) {
-                    const int s = kc % kPStages;
-                    const int b = gc % kPAcc;
-                    const bool first = (ks % gs) == 0;
-                    if (first && !mbar_wait(acc_empty(b), (uint32_t)(((gc / kPAcc) & 1) ^ 1), &abort_s)) { ok = false; break; }
-                    if (!mbar_wait(full_a(s), (uint32_t)((kc / kPStages) & 1), &abort_s)) { ok = false; break; }
-                    if (!mbar_wait(full_b(s), (uint32_t)((kc / kPStages) & 1), &abort_s)) { ok = false; break; }
+            // one MMA step (K = 64: four K = 16 MMAs) into accumulator b; returns false on a timed-out wait
+            auto step = [&](int& gleft, uint32_t ta, uint64_t db) -> bool {
+                const bool first = gleft == gs;
+                if (first) {
+                    if (!mbar_wait(acc_empty(b), bph ^ 1u, &abort_s)) return false;
                     tc_fence_after();
-                    const uint64_t db = smem_desc(stB + s * kPStageB);
-                    const uint32_t ta = tmem + (uint32_t)(kPAcol + s * kPAcols);
+                }
+                const uint32_t td = tmem + (uint32_t)(b * kPBN);
+                mma_bf16_ts(td, ta, db, first ? 0u : 1u);
 #pragma unroll
-                    for (int kk = 0; kk < kPBK / 16; ++kk)  // K = 16 per MMA: 8 A columns, +32 bytes in the B row
-                        mma_bf16_ts(tmem + (uint32_t)(b * kPBN), ta + (uint32_t)(8 * kk), db + (uint64_t)(2 * kk),
-                                    (first && kk == 0) ? 0u : 1u);
-                    mma_commit(empty(s));
-                    if ((ks % gs) == gs - 1) {
-                        mma_commit(acc_full(b));
-                        ++gc;
+                for (int kk = 1; kk < kPBK / 16; ++kk)  // K = 16 per MMA: 8 A columns, +32 bytes in the B row
+                    mma_bf16_ts(td, ta + (uint32_t)(8 * kk), db + (uint64_t)(2 * kk), 1u);
+                if (--gleft == 0) {
+                    mma_commit(acc_full(b));
+                    gleft = gs;
+                    if (++b == kPAcc) { b = 0; bph ^= 1u; }
+                }
+                return true;
+            };
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                int gleft = gs;  // steps left in the current group
+                for (int ch = 0; ch < nchunks; ++ch, ++cc) {
+                    const int hbuf = cc & 1;
+                    if (!mbar_wait(full_a(hbuf), (uint32_t)((cc >> 1) & 1), &abort_s)) { ok = false; break; }
+                    if (!mbar_wait(full_x(c), cph, &abort_s)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t db0 = smem_desc(stX + c * kPChunkB);
+                    const uint32_t ta0 = tmem + (uint32_t)(kPAcol + hbuf * kPChunkSteps * kPAcols);
+                    const int steps = min(kPChunkSteps, nk - ch * kPChunkSteps);
+                    if (steps == kPChunkSteps) {
+#pragma unroll
+                        for (int st = 0; st < kPChunkSteps; ++st)
+                            if (!step(gleft, ta0 + (uint32_t)(st * kPAcols), db0 + (uint64_t)((st * kPStepB) >> 4))) {
+                                ok = false;
+                                break;
+                            }
+                    } else {
+                        for (int st = 0; st < steps; ++st)
+                            if (!step(gleft, ta0 + (uint32_t)(st * kPAcols), db0 + (uint64_t)((st * kPStepB) >> 4))) {
+                                ok = false;
+                                break;
+                            }
                     }
+                    if (!ok) break;
+                    mma_commit(chunk_empty(c));
+                    if (++c == kPXSlots) { c = 0; cph ^= 1u; }
                 }
             }
         }
@@ -389,7 +458,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 13) {
+    if (warp == kPMmaWarp) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPTmemCols));
     }
