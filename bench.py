@@ -568,6 +568,22 @@ def profile_prefill(args):
                       "TFLOP/s_dense_equiv": round(2 * M * N * K / (ms * 1e-3) / 1e12, 1)}), flush=True)
 
 
+def profile_decode(args):
+    """The batched decode call over the first LAYERS layers of the 3B stack at M tokens
+    (for profiler captures of the few-token and one-token kernels)."""
+    import torch
+    from sparse_ternary_weight_b200.build import build
+    build()
+    M, layers = (int(v) for v in args.profile_decode.split(","))
+    dev = torch.device("cuda", 0)
+    pairs, outs = build_stack(STACK, M, torch.float32, dev, layers)
+    call = batched_caller(pairs, outs, torch.float32)
+    ms = time_region(call, args.steps, args.warmup, 1, torch.cuda.current_stream()) / args.steps
+    b = stack_bytes([(P.N, P.K) for _, P in pairs], M)
+    print(json.dumps({"decode": f"3B stack, {layers} layers, M={M}", "ms": round(ms, 4),
+                      "GB/s": round(b / (ms * 1e-3) / 1e9, 1), "bytes": b}), flush=True)
+
+
 def profile_quantize(args):
     import torch
     from sparse_ternary_weight_b200.build import build
@@ -604,7 +620,13 @@ def main():
     ap.add_argument("--profile-prefill", default=None, metavar="N,K,M",
                     help="only run one tensor-core prefill linear (N x K weight, M tokens) warmup+steps times, "
                          "print its time, and exit (for profiler captures)")
+    ap.add_argument("--profile-decode", default=None, metavar="M,LAYERS",
+                    help="only run the batched decode call over the first LAYERS layers of the 3B stack at M "
+                         "tokens warmup+steps times, print its time, and exit (for profiler captures)")
     args = ap.parse_args()
+    if args.profile_decode:
+        profile_decode(args)
+        return
     if args.profile_prefill:
         profile_prefill(args)
         return

@@ -58,7 +58,7 @@ constexpr int kTSgnBytes = kTRows * kTChunkSteps * 2;    // 1 KB: [row] 8 sign b
 constexpr long long kTWaitCycles = 4000000000LL;
 // below this many tokens the lookup-table kernels are faster (measured on the
 // 3B decode stack)
-constexpr int kSkinnyMinM = 5;
+constexpr int kSkinnyMinM = 3;
 static_assert(kTDecGroups == kTChunkSteps, "one decode group per chunk step");
 static_assert(kTAParMax < kTChunks, "an A buffer's release is still tracked by its chunk slot");
 
