@@ -388,6 +388,21 @@ def extra_rows(args, pairs, outs, shapes, ws, dev, pk):
     # prefill on the tensor cores: the 3B stack (196 linears, one launch each, CUDA graph)
     rows["prefill_3b"] = prefill_rows(args, pairs, ws, dev, pk, steps=max(2, args.steps // 10), warm=3)
 
+    # unpack of the whole 3B stack (group 128) to dense bf16, one launch per linear (CUDA graph)
+    big = max(P.N * P.K for _, P in pairs)
+    wout = torch.empty(big, dtype=torch.bfloat16, device=dev)
+
+    def ustep():
+        for _, P in pairs:
+            sw.unpack(P, out=wout[: P.N * P.K].view(P.N, P.K))
+    gu = graph_of(ustep)
+    ms = time_region(gu.replay, steps, warm, ws, stream) / steps
+    ub = sum(P.nbytes() + 2 * P.N * P.K for _, P in pairs)
+    rows["unpack_3b_full"] = {"GB/s": round(ws * ub / (ms * 1e-3) / 1e9, 1), "ms": round(ms, 4),
+                              "frac_hbm": round(ub / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4), "bytes": ub,
+                              "launches": len(pairs)}
+    del gu, wout
+
     # quantize + pack of the full 3B weight set (fp32 in HBM), three granularities
     qp = {}
     cfg, layers, shp = synth.STACKS[STACK]

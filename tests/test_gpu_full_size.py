@@ -163,7 +163,8 @@ def test_prefill_stack_sampled(sw, orc, gran):
 def test_quantize_full_3b(sw, orc, gran):
     """Quantise + pack of every linear of the 3B set from fp32: sampled rows bit for
     bit (idx and sgn do not depend on the scale); per-tensor weights whole on the
-    first and the last layer (the scale is a mean over the whole tensor)."""
+    first and the last layer (the scale is a mean over the whole tensor).  With
+    group scales also the dense bf16 unpack of every linear, sampled rows bit for bit."""
     import torch
     rng = np.random.default_rng(13)
     cfg, layers, shp = synth.STACKS["3b"]
@@ -190,6 +191,11 @@ def test_quantize_full_3b(sw, orc, gran):
                     assert np.array_equal(P.idx.index_select(0, r).cpu().numpy().view(np.uint32), ref[0]), (l, p)
                     assert np.array_equal(P.sgn.index_select(0, r).cpu().numpy(), ref[1]), (l, p)
                 else:
-                    _check_packed_rows(orc, W_rows, P, rows)
+                    ref = _check_packed_rows(orc, W_rows, P, rows)
+                    if g == oracle.PER_GROUP:
+                        # dense bf16 unpack of the whole linear, sampled rows bit for bit
+                        Wd = sw.unpack(P).index_select(0, torch.from_numpy(rows).cuda())
+                        got = Wd.view(torch.int16).cpu().numpy().view(np.uint16)
+                        assert np.array_equal(got, orc.unpack_bf16(*ref, len(rows), K, g, 128)), (l, p)
             del W, P
     torch.cuda.synchronize()
