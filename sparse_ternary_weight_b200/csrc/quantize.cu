@@ -8,83 +8,99 @@
 // group of `group` weights along K, a row, or the whole tensor, and the
 // denominator is max(L * 3/4, 1) for a domain of L weights.
 //
-// Kernel 1 (one CTA per row, HBM-bound on the read of W): each lane owns one
-// block of 4, finds the zero position and signs in registers, builds its
-// nibble; 8 lanes OR their nibbles into one uint32 word with three xor
-// shuffles, a ballot gives the sign bytes, and the masked |w| are reduced per
-// 32-weight word with the same shuffles (the lower five levels of the
-// canonical pairwise tree).  Word sums sit in shared memory; the scales are
-// then the upper levels of the tree over each domain.
+// Kernel 1 (one CTA per row, HBM-bound on the read of W): each lane owns four
+// blocks of 4 (16 consecutive weights, half a packed word), finds each zero
+// position and the negative-sign bits in registers and takes the 5-bit code
+// (nibble + 16 G) from a 64-entry table indexed by (zero position, sign bits);
+// one xor shuffle with the partner lane completes the word's nibbles, its sign
+// byte and its masked |w| sum (the lower five levels of the canonical pairwise
+// tree, in that order).  Word sums sit in shared memory; the scales are then
+// the upper levels of the tree over each domain.
 // Kernel 2 (per-tensor only): one CTA folds the per-row subtree sums.
 #include "common.cuh"
 
 namespace sherry {
 
 constexpr int kQThreads = 256;
-constexpr int kQUnroll = 4;
+constexpr int kQUnroll = 2;  // warp-steps (16 weights per lane each) in flight
 
-struct BlockCode {
-    uint32_t nib;   // 4z + 2 d1 + d2
-    uint32_t g;     // sign of the first kept weight is negative
-    float mag;      // (m0 + m1) + (m2 + m3), masked magnitudes
-};
+// 5-bit code (nibble 4z + 2 d1 + d2, plus 16 G) of a block whose smallest |w|
+// is at z and whose negative weights are the set bits of `neg` (w < 0; -0.0 is
+// not negative): the kept signs in position order are k0 k1 k2, G = k0,
+// d1 = k1 ^ k0, d2 = k2 ^ k0.
+__device__ __forceinline__ uint32_t code_of(uint32_t z, uint32_t neg) {
+    const uint32_t low = neg & ((1u << z) - 1u);
+    const uint32_t k3 = low | ((neg >> (z + 1)) << z);
+    const uint32_t g = k3 & 1u;
+    const uint32_t d1 = ((k3 >> 1) ^ k3) & 1u;
+    const uint32_t d2 = ((k3 >> 2) ^ k3) & 1u;
+    return 4u * z + 2u * d1 + d2 + 16u * g;
+}
 
-__device__ __forceinline__ BlockCode encode4(float w0, float w1, float w2, float w3) {
-    float a0 = fabsf(w0), a1 = fabsf(w1), a2 = fabsf(w2), a3 = fabsf(w3);
+// one block of 4: code from the table, masked magnitude sum (m0 + m1) + (m2 + m3)
+__device__ __forceinline__ uint32_t encode4(float w0, float w1, float w2, float w3, const uint8_t* ctab,
+                                            float& mag) {
+    const float a0 = fabsf(w0), a1 = fabsf(w1), a2 = fabsf(w2), a3 = fabsf(w3);
     // first index of the minimum |w| (strict < keeps the earlier index on ties)
-    int z = 0;
+    uint32_t z = 0;
     float m = a0;
     if (a1 < m) { z = 1; m = a1; }
     if (a2 < m) { z = 2; m = a2; }
     if (a3 < m) { z = 3; }
-    // negative-sign bits; w >= 0 (and -0.0) count as +1
-    uint32_t neg = (w0 < 0.0f ? 1u : 0u) | (w1 < 0.0f ? 2u : 0u) | (w2 < 0.0f ? 4u : 0u) |
-                   (w3 < 0.0f ? 8u : 0u);
-    // drop bit z: kept signs in position order at bits 0..2
-    uint32_t low = neg & ((1u << z) - 1u);
-    uint32_t k3 = low | ((neg >> (z + 1)) << z);
-    uint32_t g = k3 & 1u;
-    uint32_t d1 = ((k3 >> 1) ^ k3) & 1u;
-    uint32_t d2 = ((k3 >> 2) ^ k3) & 1u;
-    BlockCode c;
-    c.nib = 4u * (uint32_t)z + 2u * d1 + d2;
-    c.g = g;
-    float m0 = z == 0 ? 0.0f : a0;
-    float m1 = z == 1 ? 0.0f : a1;
-    float m2 = z == 2 ? 0.0f : a2;
-    float m3 = z == 3 ? 0.0f : a3;
-    c.mag = (m0 + m1) + (m2 + m3);
-    return c;
+    const uint32_t neg = (w0 < 0.0f ? 1u : 0u) | (w1 < 0.0f ? 2u : 0u) | (w2 < 0.0f ? 4u : 0u) |
+                         (w3 < 0.0f ? 8u : 0u);
+    mag = ((z == 0 ? 0.0f : a0) + (z == 1 ? 0.0f : a1)) + ((z == 2 ? 0.0f : a2) + (z == 3 ? 0.0f : a3));
+    return ctab[(z << 4) | neg];
 }
 
+// 16 consecutive weights (4 blocks) per lane
 template <bool kBF16>
 struct WLoad;
 
 template <>
 struct WLoad<false> {
-    using T = float4;
-    __device__ __forceinline__ static T load(const void* W, int64_t off_blocks) {
-        return __ldcs(reinterpret_cast<const float4*>(W) + off_blocks);
+    struct T { float4 q[4]; };
+    __device__ __forceinline__ static T load(const void* W, int64_t off16) {
+        const float4* p = reinterpret_cast<const float4*>(W) + off16 * 4;
+        T v;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v.q[i] = __ldcs(p + i);
+        return v;
     }
-    __device__ __forceinline__ static void unpack(const T& v, float& a, float& b, float& c, float& d) {
-        a = v.x; b = v.y; c = v.z; d = v.w;
+    __device__ __forceinline__ static void block(const T& v, int j, float& a, float& b, float& c, float& d) {
+        a = v.q[j].x; b = v.q[j].y; c = v.q[j].z; d = v.q[j].w;
     }
-    __device__ __forceinline__ static T zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ static T zero() {
+        T v;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v.q[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        return v;
+    }
 };
 
 template <>
 struct WLoad<true> {
-    using T = uint2;
-    __device__ __forceinline__ static T load(const void* W, int64_t off_blocks) {
-        return __ldcs(reinterpret_cast<const uint2*>(W) + off_blocks);
+    struct T { uint4 q[2]; };
+    __device__ __forceinline__ static T load(const void* W, int64_t off16) {
+        const uint4* p = reinterpret_cast<const uint4*>(W) + off16 * 2;
+        T v;
+        v.q[0] = __ldcs(p);
+        v.q[1] = __ldcs(p + 1);
+        return v;
     }
-    __device__ __forceinline__ static void unpack(const T& v, float& a, float& b, float& c, float& d) {
-        a = __uint_as_float(v.x << 16);
-        b = __uint_as_float(v.x & 0xffff0000u);
-        c = __uint_as_float(v.y << 16);
-        d = __uint_as_float(v.y & 0xffff0000u);
+    __device__ __forceinline__ static void block(const T& v, int j, float& a, float& b, float& c, float& d) {
+        const uint4& u = v.q[j >> 1];
+        const uint32_t x = (j & 1) ? u.z : u.x, y = (j & 1) ? u.w : u.y;
+        a = __uint_as_float(x << 16);
+        b = __uint_as_float(x & 0xffff0000u);
+        c = __uint_as_float(y << 16);
+        d = __uint_as_float(y & 0xffff0000u);
     }
-    __device__ __forceinline__ static T zero() { return make_uint2(0u, 0u); }
+    __device__ __forceinline__ static T zero() {
+        T v;
+        v.q[0] = v.q[1] = make_uint4(0u, 0u, 0u, 0u);
+        return v;
+    }
 };
 
 // granularity of the scale written by kernel 1
@@ -96,45 +112,55 @@ k_quantize_rows(const void* __restrict__ W, int K, uint32_t* __restrict__ idx,
                 uint8_t* __restrict__ sgn, float* __restrict__ out,
                 int gw /* group words (per-group) or chunk words (per-tensor) */, float D) {
     extern __shared__ float wsum[];  // K/32 word sums of masked |w|
+    __shared__ uint8_t ctab[64];     // 5-bit code by (zero position, negative bits)
     using L = WLoad<kBF16>;
     const int64_t n = blockIdx.x;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int words = K >> 5;
-    const int nblk = K >> 2;
-    const int nchunks = (K + 127) >> 7;  // 128 weights = 32 blocks = one warp-step
-    const int64_t row_blk = n * (int64_t)nblk;
+    const int n16 = K >> 4;                  // 16-weight pieces (two per word)
+    const int nsteps = (n16 + 31) >> 5;      // 512 weights = 16 words = one warp-step
+    const int64_t row16 = n * (int64_t)n16;
     const int64_t row_word = n * (int64_t)words;
+    if (threadIdx.x < 64) ctab[threadIdx.x] = (uint8_t)code_of(threadIdx.x >> 4, threadIdx.x & 15u);
+    __syncthreads();
 
-    for (int c0 = warp; c0 < nchunks; c0 += 8 * kQUnroll) {
+    for (int c0 = warp; c0 < nsteps; c0 += 8 * kQUnroll) {
         typename L::T v[kQUnroll];
 #pragma unroll
         for (int u = 0; u < kQUnroll; ++u) {
-            int b = (c0 + 8 * u) * 32 + lane;
-            v[u] = (c0 + 8 * u < nchunks && b < nblk) ? L::load(W, row_blk + b) : L::zero();
+            const int piece = (c0 + 8 * u) * 32 + lane;
+            v[u] = (c0 + 8 * u < nsteps && piece < n16) ? L::load(W, row16 + piece) : L::zero();
         }
 #pragma unroll
         for (int u = 0; u < kQUnroll; ++u) {
             const int c = c0 + 8 * u;
-            if (c >= nchunks) break;  // warp-uniform
-            const int b = c * 32 + lane;
-            float w0, w1, w2, w3;
-            L::unpack(v[u], w0, w1, w2, w3);
-            BlockCode bc = encode4(w0, w1, w2, w3);
-            uint32_t word = bc.nib << (4 * (lane & 7));
+            if (c >= nsteps) continue;  // warp-uniform
+            const int piece = c * 32 + lane;
+            const int half = lane & 1;
+            uint32_t nib = 0, sg = 0;
+            float m4[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float w0, w1, w2, w3;
+                L::block(v[u], j, w0, w1, w2, w3);
+                const uint32_t code = encode4(w0, w1, w2, w3, ctab, m4[j]);
+                nib |= (code & 15u) << (4 * j);
+                sg |= (code >> 4) << j;
+            }
+            // half 0 holds blocks 0..3 of the word, half 1 blocks 4..7
+            uint32_t word = nib << (16 * half);
             word |= __shfl_xor_sync(kFull, word, 1);
-            word |= __shfl_xor_sync(kFull, word, 2);
-            word |= __shfl_xor_sync(kFull, word, 4);
-            const uint32_t bal = __ballot_sync(kFull, bc.g);
-            float s = bc.mag;
-            s = s + __shfl_xor_sync(kFull, s, 1);
-            s = s + __shfl_xor_sync(kFull, s, 2);
-            s = s + __shfl_xor_sync(kFull, s, 4);
-            // whole 8-lane groups are valid or not (K % 32 == 0)
-            if ((lane & 7) == 0 && b < nblk) {
-                const int w = c * 4 + (lane >> 3);
+            uint32_t sb = sg << (4 * half);
+            sb |= __shfl_xor_sync(kFull, sb, 1);
+            float s = (m4[0] + m4[1]) + (m4[2] + m4[3]);
+            const float o = __shfl_xor_sync(kFull, s, 1);
+            s = half ? o + s : s + o;  // ((b0 + b1) + (b2 + b3)) + ((b4 + b5) + (b6 + b7))
+            // both lanes of a word are valid or neither (K % 32 == 0)
+            if (half == 0 && piece < n16) {
+                const int w = piece >> 1;
                 idx[row_word + w] = word;
-                sgn[row_word + w] = (uint8_t)((bal >> lane) & 0xffu);
+                sgn[row_word + w] = (uint8_t)sb;
                 wsum[w] = s;
             }
         }
