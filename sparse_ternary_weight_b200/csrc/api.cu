@@ -59,20 +59,25 @@ static bool use_stream(const ProbShape* shapes, int count, int64_t M) {
     return tiles <= kMaxTickets;
 }
 
-// Which kernel computes each problem of a call.  2 <= M <= 32 problems that fit
-// the few-token tensor-core kernel share one launch of it; of the rest, each
+// Which kernel computes each problem of a call.  2 <= M <= 8 problems with
+// K % 128 == 0 share one launch of the warp-MMA kernel; other problems with up
+// to 32 tokens that fit the tcgen05 few-token kernel share one launch of it; of
+// the rest, each
 // problem with M >= 17 that fits the prefill kernel gets a launch of its own;
 // what remains shares one launch of the one-token streaming kernel (M == 1,
 // every remaining problem eligible) or of the general lookup-table kernel.
 struct Routes {
-    std::vector<ProbShape> skinny_s, rest_s;
-    std::vector<sherry_linear_desc> skinny_d, rest_d;
+    std::vector<ProbShape> hmma_s, skinny_s, rest_s;
+    std::vector<sherry_linear_desc> hmma_d, skinny_d, rest_d;
     std::vector<int> prefill;  // indices into the call's problems
 };
 
 static void route(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, Routes& r) {
     for (int i = 0; i < count; ++i) {
-        if (skinny_eligible(shapes[i], M)) {
+        if (hmma_eligible(shapes[i], M)) {
+            r.hmma_s.push_back(shapes[i]);
+            if (descs) r.hmma_d.push_back(descs[i]);
+        } else if (skinny_eligible(shapes[i], M)) {
             r.skinny_s.push_back(shapes[i]);
             if (descs) r.skinny_d.push_back(descs[i]);
         } else if (prefill_eligible(shapes[i], M)) {
@@ -98,6 +103,9 @@ static int linear_launch(const ProbShape* shapes, const sherry_linear_desc* desc
     Routes r;
     route(shapes, descs, count, M, r);
     int st = SHERRY_OK;
+    if (!r.hmma_s.empty() &&
+        (st = hmma_linear_launch(r.hmma_s.data(), r.hmma_d.data(), (int)r.hmma_s.size(), M, y_bf16, stream)))
+        return st;
     if (!r.skinny_s.empty() &&
         (st = skinny_linear_launch(r.skinny_s.data(), r.skinny_d.data(), (int)r.skinny_s.size(), M, y_bf16, sms,
                                    stream)))

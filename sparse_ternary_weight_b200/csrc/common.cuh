@@ -117,6 +117,9 @@ bool prefill_eligible(const ProbShape& s, int64_t M);
 int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, int y_bf16, cudaStream_t stream);
 int device_status_take(cudaStream_t stream);
 // few-token tensor-core kernel (gemv_tc.cu)
+bool hmma_eligible(const ProbShape& s, int64_t M);
+int hmma_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
+                       cudaStream_t stream);
 bool skinny_eligible(const ProbShape& s, int64_t M);
 int skinny_status_take();  // SHERRY_ERR_TIMEOUT if a bounded wait gave up since the last call
 int skinny_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,

@@ -373,3 +373,39 @@ def test_batched_mixed_routes_vs_oracle(sw, orc, M):
              (M >= 17 and K % 64 == 0 and (gname != "group" or group % 64 == 0))
         if tc:
             assert torch.equal(sw.linear(X, P), y)
+
+
+HMMA_CASES = [
+    # (M, N, K, gran, group): 2 <= M <= 8 with K % 128 == 0 runs the warp-MMA kernel (larger M the
+    # tcgen05 few-token kernel)
+    (2, 64, 128, "group", 32),
+    (2, 129, 384, "channel", 0),
+    (4, 33, 640, "group", 128),
+    (9, 500, 1152, "group", 96),
+    (8, 1000, 8192, "tensor", 0),
+    (7, 17, 2048, "group", 256),
+    (8, 3072, 3072, "group", 128),
+    (12, 1000, 8192, "tensor", 0),
+]
+
+
+@pytest.mark.parametrize("case", HMMA_CASES, ids=lambda c: f"M{c[0]}-{c[1]}x{c[2]}-{c[3]}{c[4]}")
+def test_warp_mma_vs_oracle(sw, orc, case):
+    import torch
+    from sparse_ternary_weight_b200 import _abi
+    M, N, K, gname, group = case
+    gran = GRAN[gname]
+    W = _weights("t4", N, K, seed=13000 + N + K)
+    Xb = synth.activations_bf16(M, K, seed=13500 + M + K)
+    P = sw.quantize_pack(to_dev(W), gran, group)
+    idx, sgn, sc = packed_to_host(P)
+    y_ref = orc.linear(Xb, idx, sgn, sc, N, K, gran, group)
+    Wq = orc.unpack_f32(idx, sgn, sc, N, K, gran, group)
+    X = to_dev(Xb.view(np.int16)).view(torch.bfloat16)
+    y32 = sw.linear(X, P, torch.float32)
+    yb = sw.linear(X, P, torch.bfloat16)
+    assert _abi.lib().sherry_device_status(None) == 0
+    check_linear(y32.cpu().numpy(), y_ref, Xb, Wq)
+    check_linear(yb.float().cpu().numpy(), y_ref, Xb, Wq, y_is_bf16=True)
+    assert torch.equal(yb, y32.to(torch.bfloat16))
+    assert torch.equal(sw.linear(X, P, torch.float32), y32)
