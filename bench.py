@@ -152,14 +152,21 @@ def barrier(ws):
         dist.barrier()
 
 
-def allreduce_max(ws, v):
+def allreduce_max(ws, v, device="cuda"):
+    """max of v over the ranks (every rank gets it); replicas are timed by the slowest one"""
     if ws <= 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(units_per_rank, ms_max, steps, ws):
+    """whole-job throughput of ws independent replicas: all ranks' units over the
+    slowest rank's time (units per second)"""
+    return ws * units_per_rank * steps / (ms_max * 1e-3)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -268,7 +275,7 @@ def run_ours(args):
     clocks = clk.summary()
     ms_step = ms / args.steps
     gbs_rank = step_bytes / (ms_step * 1e-3) / 1e9
-    value = gbs_rank * ws
+    value = replica_throughput(step_bytes, ms, args.steps, ws) / 1e9
     tok_s = ws * M / (ms_step * 1e-3)
 
     # parity spot check of this exact launch configuration (sampled rows vs a
