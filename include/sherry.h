@@ -127,7 +127,7 @@ int sherry_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K, int g
  *   workspace  sherry_workspace_bytes(SHERRY_OP_LINEAR, M, N, K, g, group) bytes
  * fp32 accumulation; alpha applied once per group (or row).  Kernels:
  * M == 1 a lookup-table decode kernel; 2 <= M <= 8 with K % 128 == 0 a
- * warp-level tensor-core (mma.sync) kernel; 3 <= M <= 32 with K % 256 == 0 and
+ * warp-level tensor-core (mma.sync) kernel; 9 <= M <= 32 with K % 256 == 0 and
  * (per-group) group % 64 == 0 a tensor-core (tcgen05) kernel for few tokens;
  * M >= 17 with K % 64 == 0 and group % 64 == 0 the tcgen05 prefill kernel;
  * anything else the general lookup-table kernel (any M). */

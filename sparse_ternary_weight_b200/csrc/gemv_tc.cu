@@ -1,4 +1,4 @@
-// gemv_tc.cu -- packed 3:4 ternary linear for a few tokens (2 <= M <= 32) on the
+// gemv_tc.cu -- packed 3:4 ternary linear for a few tokens (9 <= M <= 32) on the
 // tensor cores, Y = X (T alpha)^T ("Sherry: Hardware-Efficient 1.25-Bit Ternary
 // Quantization via Fine-grained Sparsification", digest: Y = X T alpha).
 //
@@ -56,9 +56,9 @@ constexpr int kTAParMax = 3;              // A buffers per decode group, at most
 constexpr int kTIdxBytes = kTRows * kTChunkSteps * 8;    // 4 KB: [step][row] 8 bytes (2 words)
 constexpr int kTSgnBytes = kTRows * kTChunkSteps * 2;    // 1 KB: [row] 8 sign bytes
 constexpr long long kTWaitCycles = 4000000000LL;
-// below this many tokens the lookup-table kernels are faster (measured on the
-// 3B decode stack)
-constexpr int kSkinnyMinM = 3;
+// below this many tokens the warp-level MMA kernel is faster (measured on the 3B
+// decode stack: M = 8: 0.566 vs 0.620 ms; M = 16: 0.760 vs 0.634 ms)
+constexpr int kSkinnyMinM = 9;
 static_assert(kTDecGroups == kTChunkSteps, "one decode group per chunk step");
 static_assert(kTAParMax < kTChunks, "an A buffer's release is still tracked by its chunk slot");
 

@@ -288,11 +288,11 @@ def test_prefill_tensor_core_vs_oracle(sw, orc, case):
 
 
 SKINNY_CASES = [
-    # (M, N, K, gran, group): 3 <= M <= 32 runs the few-token tensor-core kernel
-    (3, 128, 256, "group", 128),
-    (6, 300, 1024, "channel", 0),
-    (7, 1024, 3072, "group", 128),
-    (8, 77, 512, "tensor", 0),
+    # (M, N, K, gran, group): 9 <= M <= 32 runs the tcgen05 few-token kernel
+    (9, 128, 256, "group", 128),
+    (10, 300, 1024, "channel", 0),
+    (11, 1024, 3072, "group", 128),
+    (12, 77, 512, "tensor", 0),
     (16, 2048, 2048, "group", 64),
     (17, 200, 768, "group", 256),
     (24, 129, 3072, "group", 128),
@@ -322,12 +322,12 @@ def test_skinny_tensor_core_vs_oracle(sw, orc, case):
 
 
 def test_skinny_batch_vs_oracle(sw, orc):
-    """Several linears with 3..16 tokens in one launch of the few-token kernel."""
+    """Several linears with 9..16 tokens in one launch of the tcgen05 few-token kernel."""
     import torch
     from sparse_ternary_weight_b200 import _abi
     shapes = [(1024, 3072, "group", 128), (300, 3072, "channel", 0), (3072, 8192, "group", 128),
               (77, 1024, "group", 256), (513, 2048, "tensor", 0)]
-    for M in (3, 9, 16):
+    for M in (9, 13, 16):
         pairs, refs = [], []
         for i, (N, K, gname, group) in enumerate(shapes):
             gran = GRAN[gname]
@@ -343,7 +343,7 @@ def test_skinny_batch_vs_oracle(sw, orc):
             check_linear(y.cpu().numpy(), y_ref, Xb, Wq)
 
 
-SKINNY_MIN_M = 3   # fewest tokens routed to the few-token tensor-core kernel
+SKINNY_MIN_M = 9   # fewest tokens routed to the tcgen05 few-token kernel
 MIXED_SHAPES = [(1024, 3072, "group", 128), (300, 768, "channel", 0), (200, 96, "group", 32),
                 (129, 3072, "group", 128), (96, 320, "group", 64), (513, 1024, "tensor", 0)]
 
