@@ -537,7 +537,7 @@ def prefill_rows(args, pairs, ws, dev, pk, steps, warm):
 
 
 # ---------------------------------------------------------------------------------------------
-# CPU oracle (the reference arm of this build)
+# CPU oracle: the reference arm (the plain CPU implementation, timed on the host cores)
 
 
 def cpu_baseline(layers, min_seconds=10.0):

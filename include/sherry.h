@@ -68,7 +68,7 @@ extern "C" {
 #define SHERRY_ERR_WORKSPACE 7     /* workspace missing or too small */
 #define SHERRY_ERR_CUDA 8          /* a CUDA call or launch failed (see sherry_last_cuda_error) */
 #define SHERRY_ERR_TIMEOUT 9       /* a bounded device wait gave up */
-#define SHERRY_ERR_UNSUPPORTED 10  /* valid request this build cannot run (e.g. no sm_100 device) */
+#define SHERRY_ERR_UNSUPPORTED 10  /* valid request the library cannot run here (e.g. no sm_100 device) */
 
 /* granularity of alpha */
 #define SHERRY_PER_TENSOR 0
