@@ -192,6 +192,23 @@ int sherry_unpack(const uint32_t* idx, const uint8_t* sgn, const float* scales,
                   int64_t N, int64_t K, int granularity, int group,
                   uint16_t* W_out, void* stream);
 
+/* One weight of a batched unpack (all pointers device pointers). */
+typedef struct sherry_unpack_desc {
+    const uint32_t* idx;
+    const uint8_t* sgn;
+    const float* scales;
+    int64_t N, K;
+    int32_t granularity, group;
+    uint16_t* W_out;        /* bf16 [N][K] */
+} sherry_unpack_desc;
+
+/* ---- batched unpack ---------------------------------------------------------
+ * `count` independent unpacks (count <= SHERRY_MAX_BATCH) in one launch, each
+ * exactly as by sherry_unpack (bit-identical W_out).  `descs` is a HOST array,
+ * read during the call only.  Each desc is validated like the arguments of
+ * sherry_unpack; on an error nothing is launched. */
+int sherry_unpack_batched(const sherry_unpack_desc* descs, int count, void* stream);
+
 /* ---- diagnostics ----------------------------------------------------------- */
 const char* sherry_status_string(int status);
 /* cudaError_t value behind the last SHERRY_ERR_CUDA returned on this thread */

@@ -160,6 +160,22 @@ def linear_batched(pairs, out_dtype=None, outs=None, descs=None):
     return outs
 
 
+def unpack_batched(packs, outs=None):
+    """Dense bf16 of several packed weights in one launch (each as by :func:`unpack`)."""
+    import torch
+    if not packs:
+        return []
+    if outs is None:
+        outs = [torch.empty((P.N, P.K), dtype=torch.bfloat16, device=P.idx.device) for P in packs]
+    arr = (_abi.UnpackDesc * len(packs))()
+    for i, (P, o) in enumerate(zip(packs, outs)):
+        _require_cuda(P.idx, o)
+        arr[i] = _abi.UnpackDesc(_ptr(P.idx), _ptr(P.sgn), _ptr(P.scales), P.N, P.K, P.granularity, P.group,
+                                 _ptr(o))
+    check(lib().sherry_unpack_batched(arr, len(packs), _stream(packs[0].idx.device)), "unpack_batched")
+    return outs
+
+
 def unpack(P: PackedWeight, out=None):
     """Dense bf16 [N,K] = RNE(t * alpha)."""
     import torch

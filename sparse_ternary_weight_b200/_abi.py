@@ -27,6 +27,12 @@ class LinearDesc(ctypes.Structure):
                 ("N", i64), ("K", i64), ("granularity", ctypes.c_int32), ("group", ctypes.c_int32)]
 
 
+class UnpackDesc(ctypes.Structure):
+    """Mirror of ``sherry_unpack_desc``."""
+    _fields_ = [("idx", vp), ("sgn", vp), ("scales", vp), ("N", i64), ("K", i64),
+                ("granularity", ctypes.c_int32), ("group", ctypes.c_int32), ("W_out", vp)]
+
+
 SIGNATURES = {
     "sherry_idx_bytes": (sz, [i64, i64]),
     "sherry_sgn_bytes": (sz, [i64, i64]),
@@ -37,6 +43,7 @@ SIGNATURES = {
     "sherry_linear_batched": (i32, [ctypes.POINTER(LinearDesc), i32, i64, i32, vp, sz, vp]),
     "sherry_linear_batched_workspace_bytes": (sz, [ctypes.POINTER(LinearDesc), i32, i64]),
     "sherry_unpack": (i32, [vp, vp, vp, i64, i64, i32, i32, vp, vp]),
+    "sherry_unpack_batched": (i32, [ctypes.POINTER(UnpackDesc), i32, vp]),
     "sherry_linear_noalloc": (i32, [vp, i64, i64, i64, vp, vp, vp, i32, i32, vp, i32, vp]),
     "sherry_status_string": (ctypes.c_char_p, [i32]),
     "sherry_last_cuda_error": (i32, []),

@@ -192,16 +192,33 @@ int sherry_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K, int g
                                 static_cast<cudaStream_t>(stream));
 }
 
+static int check_unpack_desc(const sherry_unpack_desc& d) {
+    int st = check_shape(d.N, d.K);
+    if (st) return st;
+    if ((st = check_gran(d.K, d.granularity, d.group))) return st;
+    if ((st = check_planes(d.idx, d.sgn, d.scales, d.N))) return st;
+    if (d.N > 0 && !d.W_out) return SHERRY_ERR_NULL;
+    if (!aligned(d.W_out, 16)) return SHERRY_ERR_ALIGN;
+    return SHERRY_OK;
+}
+
 int sherry_unpack(const uint32_t* idx, const uint8_t* sgn, const float* scales, int64_t N, int64_t K,
                   int granularity, int group, uint16_t* W_out, void* stream) {
-    int st = check_shape(N, K);
+    const sherry_unpack_desc d{idx, sgn, scales, N, K, granularity, group, W_out};
+    const int st = check_unpack_desc(d);
     if (st) return st;
-    if ((st = check_gran(K, granularity, group))) return st;
-    if ((st = check_planes(idx, sgn, scales, N))) return st;
-    if (N > 0 && !W_out) return SHERRY_ERR_NULL;
-    if (!aligned(W_out, 16)) return SHERRY_ERR_ALIGN;
-    return unpack_launch(idx, sgn, scales, N, K, granularity, group, W_out, static_cast<cudaStream_t>(stream),
-                         device_sms());
+    return unpack_launch(&d, 1, static_cast<cudaStream_t>(stream), device_sms());
+}
+
+int sherry_unpack_batched(const sherry_unpack_desc* descs, int count, void* stream) {
+    if (!descs && count > 0) return SHERRY_ERR_NULL;
+    if (count < 0 || count > SHERRY_MAX_BATCH) return SHERRY_ERR_SHAPE;
+    for (int i = 0; i < count; ++i) {
+        const int st = check_unpack_desc(descs[i]);
+        if (st) return st;
+    }
+    if (count == 0) return SHERRY_OK;
+    return unpack_launch(descs, count, static_cast<cudaStream_t>(stream), device_sms());
 }
 
 static int check_linear_desc(const sherry_linear_desc& d, int64_t M) {

@@ -107,8 +107,7 @@ struct ProbShape {
 size_t quantize_workspace_bytes(int64_t N, int64_t K, int granularity);
 int quantize_pack_launch(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
                          uint32_t* idx, uint8_t* sgn, float* scales, void* workspace, cudaStream_t stream);
-int unpack_launch(const uint32_t* idx, const uint8_t* sgn, const float* scales, int64_t N, int64_t K,
-                  int granularity, int group, uint16_t* out, cudaStream_t stream, int num_sms);
+int unpack_launch(const sherry_unpack_desc* descs, int count, cudaStream_t stream, int num_sms);
 size_t lut_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms);
 int lut_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M,
                       int y_bf16, void* workspace, int sms, cudaStream_t stream);

@@ -150,3 +150,23 @@ def test_product_rejects_cpu_tensors():
     import sparse_ternary_weight_b200 as sw
     with pytest.raises(ValueError, match="CUDA"):
         sw.quantize_pack(torch.zeros(4, 64))
+
+
+def test_unpack_batched_validation(L):
+    d = (_abi.UnpackDesc * 2)()
+    for i in range(2):
+        d[i] = _abi.UnpackDesc(FAKE, FAKE, FAKE, 8, 64, _abi.PER_GROUP, 32, FAKE)
+    assert L.sherry_unpack_batched(None, 1, None) == _abi.ERR_NULL
+    assert L.sherry_unpack_batched(d, -1, None) == _abi.ERR_SHAPE
+    assert L.sherry_unpack_batched(d, _abi.MAX_BATCH + 1, None) == _abi.ERR_SHAPE
+    assert L.sherry_unpack_batched(d, 0, None) == _abi.OK
+    d[1].K = 40
+    assert L.sherry_unpack_batched(d, 2, None) == _abi.ERR_SHAPE
+    d[1].K = 64
+    d[1].group = 48
+    assert L.sherry_unpack_batched(d, 2, None) == _abi.ERR_GROUP
+    d[1].group = 32
+    d[1].W_out = None
+    assert L.sherry_unpack_batched(d, 2, None) == _abi.ERR_NULL
+    d[1].W_out = FAKE + 8
+    assert L.sherry_unpack_batched(d, 2, None) == _abi.ERR_ALIGN

@@ -409,3 +409,24 @@ def test_warp_mma_vs_oracle(sw, orc, case):
     check_linear(yb.float().cpu().numpy(), y_ref, Xb, Wq, y_is_bf16=True)
     assert torch.equal(yb, y32.to(torch.bfloat16))
     assert torch.equal(sw.linear(X, P, torch.float32), y32)
+
+
+def test_unpack_batched_matches_single_and_oracle(sw, orc):
+    """Several weights of different shapes and granularities in one unpack launch:
+    bit-identical to the single calls and to the oracle."""
+    import torch
+    shapes = [(64, 256, "group", 128), (3, 96, "channel", 0), (33, 384, "group", 64), (7, 160, "tensor", 0),
+              (300, 3072, "group", 128), (1, 32, "group", 32)]
+    packs, refs = [], []
+    for i, (N, K, gname, group) in enumerate(shapes):
+        gran = GRAN[gname]
+        W = _weights("ties" if i % 2 else "t4", N, K, seed=14000 + i)
+        P = sw.quantize_pack(to_dev(W), gran, group)
+        packs.append(P)
+        idx, sgn, sc = packed_to_host(P)
+        refs.append(orc.unpack_bf16(idx, sgn, sc, N, K, gran, group))
+    outs = sw.unpack_batched(packs)
+    for P, o, ref in zip(packs, outs, refs):
+        got = o.view(torch.int16).cpu().numpy().view(np.uint16)
+        assert np.array_equal(got, ref)
+        assert torch.equal(o, sw.unpack(P))
