@@ -430,3 +430,34 @@ def test_unpack_batched_matches_single_and_oracle(sw, orc):
         got = o.view(torch.int16).cpu().numpy().view(np.uint16)
         assert np.array_equal(got, ref)
         assert torch.equal(o, sw.unpack(P))
+
+
+MAXK_CASES = [
+    # (M, N, gran, group) at K = SHERRY_MAX_K: one case per linear kernel route
+    (1, 5, "group", 128),   # one-token streaming kernel
+    (1, 3, "group", 32),    # general lookup-table kernel
+    (4, 5, "group", 128),   # warp-MMA kernel
+    (16, 3, "channel", 0),  # tcgen05 few-token kernel
+    (64, 3, "group", 256),  # tcgen05 prefill kernel
+]
+
+
+@pytest.mark.parametrize("case", MAXK_CASES, ids=lambda c: f"M{c[0]}-N{c[1]}-{c[2]}{c[3]}")
+def test_linear_at_max_k(sw, orc, case):
+    import torch
+    from sparse_ternary_weight_b200 import _abi
+    M, N, gname, group = case
+    K = _abi.MAX_K
+    gran = GRAN[gname]
+    W = _weights("t4", N, K, seed=15000 + M + N)
+    Xb = synth.activations_bf16(M, K, seed=15500 + M)
+    P = sw.quantize_pack(to_dev(W), gran, group)
+    ref = orc.quantize_pack(W, gran, group)
+    got = packed_to_host(P)
+    assert np.array_equal(got[0], ref[0]) and np.array_equal(got[1], ref[1])
+    assert np.array_equal(got[2].view(np.uint32), ref[2].view(np.uint32))
+    y_ref = orc.linear(Xb, *ref, N, K, gran, group)
+    X = to_dev(Xb.view(np.int16)).view(torch.bfloat16)
+    y = sw.linear(X, P, torch.float32)
+    assert _abi.lib().sherry_device_status(None) == 0
+    check_linear(y.cpu().numpy(), y_ref, Xb, orc.unpack_f32(*ref, N, K, gran, group))
