@@ -17,15 +17,16 @@
 // Synchronisation is per chunk: the MMA thread waits once for the chunk's four A
 // stages and once for its X, issues the 16 MMAs, and commits once; that commit
 // frees both the X slot and the chunk's A buffer.
-//   warps 0-7    epilogue: wait for one of two finished group accumulators,
-//                tcgen05.ld its 64-token half, acc[token] += alpha(row, group) * D,
-//                write Y (row per thread)
-//   warps 8-15   decode, two groups of four warps: group g expands steps 2g and
+//   warps 0..E-1 epilogue (E = 16 for group scales and K <= 4096, else 8): wait for one of two
+//                finished group accumulators, tcgen05.ld its share of the tokens
+//                (128 / (E / 4) each), acc[token] += alpha(row, group) * D, write
+//                Y (row per thread)
+//   next 8 warps decode, two groups of four warps: group g expands steps 2g and
 //                2g + 1 of every chunk, one pattern-table lookup per block of 4
 //                weights; packed words come straight from global memory through
 //                a per-thread prefetch ring
-//   warp 16      TMA: the chunk's four X tiles [128 tokens x 64 K], SWIZZLE_128B
-//   warp 17      TMEM allocation; one elected thread issues tcgen05.mma
+//   next warp    TMA: the chunk's four X tiles [128 tokens x 64 K], SWIZZLE_128B
+//   last warp    TMEM allocation; one elected thread issues tcgen05.mma
 #include "common.cuh"
 #include "lut.cuh"
 
@@ -37,9 +38,14 @@
 namespace sherry {
 
 constexpr int kPDecGroups = 2;   // decode groups (two MMA steps of every chunk each)
-constexpr int kPThreads = 32 * (8 + 4 * kPDecGroups + 2);  // 18 warps
-constexpr int kPTmaWarp = 8 + 4 * kPDecGroups;   // 16
-constexpr int kPMmaWarp = kPTmaWarp + 1;         // 17
+// epilogue warps EPI (8 or 16; a template parameter of the kernel), then the decode
+// warps, the TMA warp and the MMA warp
+template <int EPI>
+struct PRoles {
+    static constexpr int kThreads = 32 * (EPI + 4 * kPDecGroups + 2);
+    static constexpr int kTmaWarp = EPI + 4 * kPDecGroups;
+    static constexpr int kMmaWarp = kTmaWarp + 1;
+};
 constexpr int kPBM = 128;     // weight rows per tile
 constexpr int kPBN = 128;     // tokens per tile
 constexpr int kPBK = 64;      // K per MMA step
@@ -181,8 +187,10 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
           "=r"(v[30]), "=r"(v[31])                                                                               \
         : "r"(taddr))
 
-__global__ void __launch_bounds__(kPThreads, 1)
+template <int EPI>
+__global__ void __launch_bounds__(PRoles<EPI>::kThreads, 1)
 k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PParams P) {
+    constexpr int kPTmaWarp = PRoles<EPI>::kTmaWarp, kPMmaWarp = PRoles<EPI>::kMmaWarp;
     extern __shared__ __align__(1024) unsigned char psmem[];
     __shared__ uint64_t bars[2 * kPXSlots + 2 + 2 * kPAcc];
     __shared__ uint32_t tmem_base_s;
@@ -217,7 +225,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
         for (int h = 0; h < 2; ++h) mbar_init(full_a(h), 128 * kPDecGroups);
         for (int b = 0; b < kPAcc; ++b) {
             mbar_init(acc_full(b), 1);
-            mbar_init(acc_empty(b), 256);
+            mbar_init(acc_empty(b), 32 * EPI);
         }
         fence_mbar_init();
     }
@@ -239,11 +247,11 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;
 
-    if (warp < 8) {
+    if (warp < EPI) {
         // ---------------- epilogue: row n = tile row 32*(warp%4) + lane, tokens
         // [64*(warp/4), 64*(warp/4) + 64) of each tile ----------------
         const int q = warp & 3, half = warp >> 2;
-        constexpr int kCols = kPBN / 2;
+        constexpr int kCols = kPBN / (EPI / 4);
         bool ok = true;
         int b = 0;
         uint32_t bph = 0;  // phase parity of accumulator b's use
@@ -299,7 +307,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
     } else if (warp < kPTmaWarp) {
         // ---------------- decode: TMEM lane (= tile row) i per thread; group g expands
         // steps 2g, 2g + 1 of every chunk into A buffer (cc & 1) ----------------
-        const int g = (warp - 8) >> 2, q = warp & 3;
+        const int g = (warp - EPI) >> 2, q = warp & 3;
         const int i = q * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kPAcol;
         int cc = 0;  // chunks done so far (all tiles)
@@ -522,7 +530,8 @@ int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, i
     {
         std::lock_guard<std::mutex> lk(mu);
         if (!attr) {
-            SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
+            SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
+            SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
             attr = true;
         }
     }
@@ -534,7 +543,13 @@ int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, i
         SHERRY_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     }
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    k_prefill<<<grid, kPThreads, kPSmem, stream>>>(map, P);
+    // 16 epilogue warps (32 token columns each) drain a group accumulator faster; measured on the
+    // 3B shapes that pays for group scales up to K = 4096 (+6%) and costs at K = 8192 (-15%) and
+    // for per-row scales (one drain per tile; -1.5% at 2048 and 4096 tokens)
+    if (s.granularity == SHERRY_PER_GROUP && s.K <= 4096)
+        k_prefill<16><<<grid, PRoles<16>::kThreads, kPSmem, stream>>>(map, P);
+    else
+        k_prefill<8><<<grid, PRoles<8>::kThreads, kPSmem, stream>>>(map, P);
     SHERRY_LAUNCH_CHECK();
     return SHERRY_OK;
 }
