@@ -54,7 +54,7 @@ static bool use_stream(const ProbShape* shapes, int count, int64_t M) {
     int64_t tiles = 0;
     for (int i = 0; i < count; ++i) {
         if (!stream_eligible(shapes[i], M)) return false;
-        tiles += (shapes[i].N + 255) / 256;
+        tiles += stream_tiles(shapes[i]);
     }
     return tiles <= kMaxTickets;
 }

@@ -4,21 +4,24 @@
 // then scaled; "Sherry: Hardware-Efficient 1.25-Bit Ternary Quantization via
 // Fine-grained Sparsification", digest paragraph on inference; Y = X T alpha).
 //
-// Work unit: 256 output rows x 1024 weights (32 packed words) of one linear.
+// Work unit: 512 output rows x 512 weights (16 packed words) of one linear.
 // All units of a launch (one or many independent linears) are split into equal
 // contiguous ranges, one per CTA (stream-K): every CTA streams the same number
 // of bytes.  A row block whose units straddle two CTAs is finished by the CTA
-// that arrives last at its ticket, adding the partial sums in unit order, so Y
+// that arrives last at its ticket, adding the partial sums in CTA order, so Y
 // is deterministic.
 //
-// Per unit the CTA copies the packed planes with 16-byte cp.async (each 8
-// threads read one full 128-byte row segment, so global reads are coalesced)
-// into an XOR-swizzled shared layout that the row-per-lane reads hit without
-// bank conflicts; three stages are in flight.  The 32-entry tables of the
-// unit's 256 blocks of activations are double buffered and built one unit
-// ahead.  A lane owns one row: per packed word it spreads the 8 nibbles and
-// sign bits into two byte-vectors of table offsets (see lut.cuh) and does 8
-// lookups; alpha is applied once per 128-weight group (or once per row).
+// Roles (20 warps).  16 consumer warps: each thread owns one row of the unit
+// and only looks up and accumulates (per packed word it spreads the 8 nibbles
+// and sign bits into two byte-vectors of table offsets, see lut.cuh, and does 8
+// lookups; alpha is applied once per 128-weight group, or once per row).  4
+// helper warps, one per SM sub-partition: they copy each unit's packed planes
+// with 16-byte cp.async (8 lanes read one row's 64 contiguous bytes, so global
+// reads are coalesced) into an XOR-swizzled 3-stage ring that the row-per-lane
+// reads hit without bank conflicts, and build the unit's 128 tables of 32
+// entries into one of two buffers.  Stages and table buffers change hands
+// through mbarriers; every wait is bounded, and a timeout sets a device status
+// flag (reported by sherry_device_status) and ends the CTA.
 #include "common.cuh"
 #include "lut.cuh"
 
@@ -30,17 +33,23 @@
 
 namespace sherry {
 
-constexpr int kSThreads = 512;                     // 16 warps: 8 row-warps x 2 K-halves
-constexpr int kSRows = 256;                        // rows per unit, one per lane of a row-warp
-constexpr int kSWords = 32;                        // packed words per unit
+constexpr int kSConsumers = 16;                    // consumer warps: one row per thread
+constexpr int kSHelpers = 4;                       // copy + table warps
+constexpr int kSThreads = 32 * (kSConsumers + kSHelpers);
+constexpr int kSRows = 32 * kSConsumers;           // 512 rows per unit
+constexpr int kSWords = 16;                        // packed words per unit (512 weights)
 constexpr int kSStages = 3;
 constexpr int kSIdx = kSRows * kSWords * 4;        // 32 KB
-constexpr int kSSgn = kSRows * kSWords;            // 8 KB
-constexpr int kSSc = kSRows * 32;                  // 8 KB (at most 8 fp32 scales per row)
+constexpr int kSSgn = kSRows * 16;                 // 8 KB (16 sign bytes per row)
+constexpr int kSSc = kSRows * 16;                  // 8 KB (at most 4 fp32 scales per row)
 constexpr int kSStage = kSIdx + kSSgn + kSSc;      // 48 KB
-constexpr int kSLut = 256 * kTab;                  // 36 KB, one table per block of the unit
-constexpr int kSSmem = kSStages * kSStage + 2 * kSLut + 256;
+constexpr int kSTabs = kSWords * 8;                // 128 tables per unit
+constexpr int kSLut = kSTabs * kTab;               // 18 KB
+constexpr int kSBars = 128;                        // mbarriers
+constexpr int kSSmem = 256 + kSStages * kSStage + 2 * kSLut + kSBars;
 static_assert(kSStage % 256 == 0 && kSLut % 256 == 0, "table bases must stay multiples of 256");
+static_assert(kSTabs == 32 * kSHelpers, "one table per helper thread");
+constexpr long long kSWaitCycles = 4000000000LL;   // ~2 s at the boost clock
 
 enum SMode { kSRow = 0, kSG128 = 1, kSG256 = 2 };
 
@@ -64,19 +73,66 @@ struct SParams {
     SProb p[MAXP];
 };
 
+// bounded-wait timeouts of this file's kernel (read and cleared by sherry_device_status)
+__device__ int g_stream_status = 0;
+
+namespace {
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
                  : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(valid ? 8 : 0)
+                 : "memory");
+}
+// the mbarrier receives one arrival when all of this thread's prior cp.async complete
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// wait for the phase with the given parity to complete; false on timeout or
+// when another thread of the CTA has given up
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kSWaitCycles) {
+            *abort_flag = 1;
+            atomicExch(&g_stream_status, SHERRY_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+}  // namespace
 
 extern __shared__ __align__(16) unsigned char g_smem[];
 
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
     return v;
 }
 
@@ -102,47 +158,6 @@ struct UnitPos {
     int p, rb, sub;  // problem, row block, sub-slice
 };
 
-// issue the cp.async copies of one unit into `stage`
-template <int MAXP>
-__device__ __forceinline__ void issue_unit(const SParams<MAXP>& P, const UnitPos& u, uint32_t stage) {
-    const SProb& pr = P.p[u.p];
-    const int t = threadIdx.x;
-    const int row0 = u.rb * kSRows;
-    const int w0 = u.sub * kSWords;
-    const int words = pr.words, N = pr.N;
-    {
-        const int r0 = t >> 3, c = t & 7;
-        const int word = w0 + 4 * c;
-        const bool wok = word < words;
-        const uint32_t* src = pr.idx + (int64_t)(row0 + r0) * words + word;
-        const int64_t stepw = (int64_t)64 * words;
-        uint32_t dst = stage + r0 * 128 + ((c ^ (r0 & 7)) << 4);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const bool ok = wok && (row0 + r0 + 64 * i) < N;
-            cp_async16(dst + i * 64 * 128, ok ? src + i * stepw : pr.idx, ok);
-        }
-    }
-    {
-        const int r = t >> 1, h = t & 1;
-        const int row = row0 + r, off = w0 + 16 * h;
-        const bool ok = row < N && off < words;
-        cp_async16(stage + kSIdx + r * 32 + ((h ^ ((r >> 2) & 1)) << 4), ok ? pr.sgn + (int64_t)row * words + off : pr.sgn, ok);
-        if (pr.mode == kSG128) {
-            const int offs = w0 / 4 + 4 * h;
-            const bool oks = row < N && offs < pr.spr;
-            cp_async16(stage + kSIdx + kSSgn + r * 32 + ((h ^ ((r >> 2) & 1)) << 4),
-                       oks ? pr.scales + (int64_t)row * pr.spr + offs : pr.scales, oks);
-        }
-    }
-    if (pr.mode == kSG256 && t < kSRows) {
-        const int r = t;
-        const int row = row0 + r, off = w0 / 8;
-        const bool ok = row < N && off < pr.spr;
-        cp_async16(stage + kSIdx + kSSgn + r * 32 + (((r >> 2) & 1) << 4), ok ? pr.scales + (int64_t)row * pr.spr + off : pr.scales, ok);
-    }
-}
-
 template <int MAXP>
 __device__ __forceinline__ UnitPos locate(const SParams<MAXP>& P, int u) {
     int p = 0;
@@ -161,153 +176,183 @@ __device__ __forceinline__ void advance(const SProb* probs, UnitPos& u) {
     }
 }
 
-// Half of the 32-entry table of one block of 4 activations: the entries with
-// zero position z in {2h, 2h+1} and their negations.
-__device__ __forceinline__ void build_half_table(uint32_t tab, uint2 xb, int h) {
-    const float x0 = bf16lo(xb.x), x1 = bf16hi(xb.x), x2 = bf16lo(xb.y), x3 = bf16hi(xb.y);
-    // z = 2h: kept (h ? x0,x1,x3 : x1,x2,x3); z = 2h+1: kept (h ? x0,x1,x2 : x0,x2,x3)
-    const float a0 = h ? x0 : x1, b0 = h ? x1 : x2, c0 = x3;
-    const float a1 = x0, b1 = h ? x1 : x2, c1 = h ? x2 : x3;
-    const float s0 = a0 + b0, d0 = a0 - b0, s1 = a1 + b1, d1 = a1 - b1;
-    const float e0 = s0 + c0, e1 = s0 - c0, e2 = d0 + c0, e3 = d0 - c0;
-    const float e4 = s1 + c1, e5 = s1 - c1, e6 = d1 + c1, e7 = d1 - c1;
-    const uint32_t o = tab + 32 * h;
-    sts_v4(o, e0, e1, e2, e3);
-    sts_v4(o + 16, e4, e5, e6, e7);
-    sts_v4(o + 64, -e0, -e1, -e2, -e3);
-    sts_v4(o + 80, -e4, -e5, -e6, -e7);
+// Helper warp h's share of one unit's copies into `stage`: rows [128h, 128h+128)
+// of the unit.  Packed words: row rl's 64 bytes land as four 16-byte chunks, chunk
+// c at (c ^ ((rl >> 1) & 3)); sign bytes and scales: 16 bytes per row.
+__device__ __forceinline__ void copy_unit(const SProb& pr, const UnitPos& u, uint32_t stage, int h, int lane) {
+    const int row0 = u.rb * kSRows;
+    const int N = pr.N, words = pr.words;
+    {
+        const int c = lane & 3;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+            const int rl = 128 * h + 8 * i + (lane >> 2);
+            const int row = row0 + rl;
+            const bool ok = row < N;
+            const uint32_t* src = pr.idx + (int64_t)row * words + u.sub * kSWords + 4 * c;
+            cp_async16(stage + rl * 64 + ((c ^ ((rl >> 1) & 3)) << 4), ok ? src : pr.idx, ok);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int rl = 128 * h + 32 * i + lane;
+        const int row = row0 + rl;
+        const bool ok = row < N;
+        cp_async16(stage + kSIdx + rl * 16, ok ? pr.sgn + (int64_t)row * words + u.sub * kSWords : pr.sgn, ok);
+        if (pr.mode == kSG128)
+            cp_async16(stage + kSIdx + kSSgn + rl * 16, ok ? pr.scales + (int64_t)row * pr.spr + u.sub * 4 : pr.scales,
+                       ok);
+        else if (pr.mode == kSG256)
+            cp_async8(stage + kSIdx + kSSgn + rl * 16, ok ? pr.scales + (int64_t)row * pr.spr + u.sub * 2 : pr.scales,
+                      ok);
+    }
 }
 
-// Lookups of one row over steps [4*kh, 4*kh + nst) of a unit (4 words each);
-// `st` and `lut` are byte offsets into the dynamic shared buffer.
-template <int MODE, bool FULL>
-__device__ __forceinline__ float unit_rows(uint32_t st, uint32_t lut, int r, int kh, int nst) {
-    const uint32_t sw2 = ((r >> 2) & 1) << 4;
-    const uint4 sg = lds128(st + kSIdx + r * 32 + ((uint32_t)(kh << 4) ^ sw2));
+// Lookups of one row over the 16 words of a unit; `st` and `lut` are shared
+// addresses of the unit's stage and table buffer.
+template <int MODE>
+__device__ __forceinline__ float unit_row(uint32_t st, uint32_t lut, int r) {
+    const uint32_t sw = (uint32_t)((r >> 1) & 3);
+    const uint4 sg = lds128(st + kSIdx + r * 16);
     uint4 av = make_uint4(0u, 0u, 0u, 0u);
-    if (MODE == kSG128) av = lds128(st + kSIdx + kSSgn + r * 32 + ((uint32_t)(kh << 4) ^ sw2));
-    if (MODE == kSG256) av = lds128(st + kSIdx + kSSgn + r * 32 + sw2);
-    const uint32_t idx_row = st + r * 128;
-    const uint32_t sw8 = (uint32_t)(r & 7);
+    if (MODE == kSG128) av = lds128(st + kSIdx + kSSgn + r * 16);
+    if (MODE == kSG256) {
+        const uint2 a2 = lds64(st + kSIdx + kSSgn + r * 16);
+        av = make_uint4(a2.x, a2.y, 0u, 0u);
+    }
+    const uint32_t idx_row = st + r * 64;
     float acc = 0.0f;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-        if (FULL || cc < nst) {
-            const int c = 4 * kh + cc;
-            const uint4 wq = lds128(idx_row + (((uint32_t)c ^ sw8) << 4));
-            const uint32_t sq = cc == 0 ? sg.x : cc == 1 ? sg.y : cc == 2 ? sg.z : sg.w;
-            const uint32_t tb = lut + (uint32_t)(c * 32 * kTab);
-            float p0, p1, q0, q1, r0, r1, u0, u1;
-            word_sums<0>(wq.x, sq & 0xffu, tb, p0, p1);
-            word_sums<8>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
-            word_sums<16>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
-            word_sums<24>(wq.w, sq >> 24, tb, u0, u1);
-            const float s4 = ((p0 + q0) + (r0 + u0)) + ((p1 + q1) + (r1 + u1));
-            if (MODE == kSRow) {
-                acc += s4;
-            } else {
-                uint32_t ab;
-                if (MODE == kSG128)
-                    ab = cc == 0 ? av.x : cc == 1 ? av.y : cc == 2 ? av.z : av.w;
-                else {
-                    const int gi = c >> 1;
-                    ab = gi == 0 ? av.x : gi == 1 ? av.y : gi == 2 ? av.z : av.w;
-                }
-                acc = fmaf(__uint_as_float(ab), s4, acc);
-            }
+    for (int q = 0; q < 4; ++q) {
+        const uint4 wq = lds128(idx_row + (((uint32_t)q ^ sw) << 4));
+        const uint32_t sq = q == 0 ? sg.x : q == 1 ? sg.y : q == 2 ? sg.z : sg.w;
+        const uint32_t tb = lut + (uint32_t)(q * 32 * kTab);  // tables of words 4q..4q+3 (256-aligned)
+        float p0, p1, q0, q1, r0, r1, u0, u1;
+        word_sums<0>(wq.x, sq & 0xffu, tb, p0, p1);
+        word_sums<8>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
+        word_sums<16>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
+        word_sums<24>(wq.w, sq >> 24, tb, u0, u1);
+        const float s4 = ((p0 + q0) + (r0 + u0)) + ((p1 + q1) + (r1 + u1));
+        if (MODE == kSRow) {
+            acc += s4;
+        } else {
+            uint32_t ab;
+            if (MODE == kSG128)
+                ab = q == 0 ? av.x : q == 1 ? av.y : q == 2 ? av.z : av.w;
+            else
+                ab = q < 2 ? av.x : av.y;
+            acc = fmaf(__uint_as_float(ab), s4, acc);
         }
     }
     return acc;
 }
 
-template <int MODE>
-__device__ __forceinline__ float unit_rows_any(uint32_t st, uint32_t lut, int r, int kh, int nst) {
-    return nst == 4 ? unit_rows<MODE, true>(st, lut, r, kh, 4) : unit_rows<MODE, false>(st, lut, r, kh, nst);
-}
-
 template <int MAXP>
 __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_constant__ SParams<MAXP> P) {
     __shared__ int s_last;
-    __shared__ float s_half[kSRows];
+    __shared__ int s_abort;
     // Shared addresses: the buffer is rounded up to 256 bytes, so every table
     // base is a multiple of 256 (a lookup's address replaces its low byte); the
     // XOR swizzles need only 16-byte alignment, since writer and reader apply them.
     const uint32_t stages = (smem_u32(g_smem) + 255u) & ~255u;
     const uint32_t luts = stages + kSStages * kSStage;
+    const uint32_t bars = luts + 2 * kSLut;
+    auto full = [&](int s) { return bars + 8u * (uint32_t)s; };             // planes of a stage landed
+    auto empty = [&](int s) { return bars + 24u + 8u * (uint32_t)s; };      // consumers done with a stage
+    auto tfull = [&](int b) { return bars + 48u + 8u * (uint32_t)b; };      // tables of a buffer built
+    auto tempty = [&](int b) { return bars + 64u + 8u * (uint32_t)b; };     // consumers done with a buffer
+    const uint32_t bar_part = bars + 80u;  // every consumer stored its split-tile partial
+    const uint32_t bar_last = bars + 88u;  // the ticket's verdict is in s_last
 
     const int t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5;
-    const int r = (warp & 7) * 32 + lane;  // row within the unit
-    const int kh = warp >> 3;              // K half of the unit: steps 4kh .. 4kh+3
-    const int tb_idx = t & 255, tb_half = t >> 8;  // table-building role
     const int u_begin = blockIdx.x * P.upc;
     const int u_end = min(P.total_units, u_begin + P.upc);
     if (u_begin >= u_end) return;
-
-    // prologue: units u_begin .. u_begin + kSStages - 2 in flight
-    UnitPos pre = locate(P, u_begin);
-    for (int i = 0; i < kSStages - 1; ++i) {
-        if (u_begin + i < u_end) {
-            issue_unit(P, pre, stages + i * kSStage);
-            advance(P.p, pre);
+    const int nu = u_end - u_begin;
+    if (t == 0) {
+        for (int s = 0; s < kSStages; ++s) {
+            mbar_init(full(s), 32 * kSHelpers);
+            mbar_init(empty(s), kSRows);
         }
-        cp_async_commit();
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull(b), 32 * kSHelpers);
+            mbar_init(tempty(b), kSRows);
+        }
+        mbar_init(bar_part, kSRows);
+        mbar_init(bar_last, 1);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    __syncthreads();
+    volatile int* abort_flag = &s_abort;
+
+    if (warp >= kSConsumers) {
+        // ---- helpers: copies run two units ahead of the consumers, tables one
+        const int h = warp - kSConsumers;
+        const int ht = t - 32 * kSConsumers;  // table (block of 4 activations) of the unit
+        UnitPos cu = locate(P, u_begin);      // next unit to copy
+        UnitPos tu = cu;                      // next unit to build tables for
+        uint2 xb = make_uint2(0u, 0u);
+        {
+            const SProb& pr = P.p[tu.p];
+            xb = __ldg(reinterpret_cast<const uint2*>(pr.X) + tu.sub * kSTabs + ht);
+        }
+        for (int j = 0; j <= nu; ++j) {
+            if (j < nu) {
+                const int s = j % kSStages;
+                if (j >= kSStages && !mbar_wait(empty(s), (uint32_t)(((j / kSStages) & 1) ^ 1), abort_flag)) break;
+                copy_unit(P.p[cu.p], cu, stages + s * kSStage, h, lane);
+                cp_async_arrive(full(s));
+                advance(P.p, cu);
+            }
+            const int tj = j - 1;  // tables of unit j-1 (its planes are in flight)
+            if (tj >= 0) {
+                const int b = tj & 1;
+                if (tj >= 2 && !mbar_wait(tempty(b), (uint32_t)(((tj >> 1) & 1) ^ 1), abort_flag)) break;
+                build_table(luts + b * kSLut + ht * kTab, xb);
+                mbar_arrive(tfull(b));
+                advance(P.p, tu);
+                if (tj + 1 < nu) {
+                    const SProb& pr = P.p[tu.p];
+                    xb = __ldg(reinterpret_cast<const uint2*>(pr.X) + tu.sub * kSTabs + ht);
+                }
+            }
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        return;
+    }
+
+    // ---- consumers: thread t owns row t of every unit
+    const int r = t;
     UnitPos cur = locate(P, u_begin);
-    {
-        const SProb& pr = P.p[cur.p];
-        const int b = cur.sub * kSWords * 8 + tb_idx;
-        if (b < pr.words * 8)
-            build_half_table(luts + tb_idx * kTab, __ldg(reinterpret_cast<const uint2*>(pr.X) + b), tb_half);
-    }
     bool tile_from_start = (P.p[cur.p].unit_begin + cur.rb * P.p[cur.p].n_sub == u_begin);
     float acc = 0.0f;
-
-    for (int u = u_begin; u < u_end; ++u) {
-        const int k = u - u_begin;
-        cp_async_wait<kSStages - 2>();
-        __syncthreads();
-        if (u + kSStages - 1 < u_end)
-            issue_unit(P, pre, stages + ((k + kSStages - 1) % kSStages) * kSStage);
-        cp_async_commit();
-        if (u + kSStages - 1 < u_end) advance(P.p, pre);
-
-        // activations of the next unit's tables (latency hidden by this unit)
-        UnitPos nxt = cur;
-        advance(P.p, nxt);
-        uint2 xn = make_uint2(0u, 0u);
-        bool xn_ok = false;
-        if (u + 1 < u_end) {
-            const SProb& pn = P.p[nxt.p];
-            const int b = nxt.sub * kSWords * 8 + tb_idx;
-            xn_ok = b < pn.words * 8;
-            if (xn_ok) xn = __ldg(reinterpret_cast<const uint2*>(pn.X) + b);
-        }
-
+    int events = 0;  // split tiles handled so far (phase of bar_part / bar_last)
+    for (int k = 0; k < nu; ++k) {
+        const int s = k % kSStages, b = k & 1;
+        if (!mbar_wait(full(s), (uint32_t)((k / kSStages) & 1), abort_flag)) break;
+        if (!mbar_wait(tfull(b), (uint32_t)((k >> 1) & 1), abort_flag)) break;
         const SProb& pr = P.p[cur.p];
-        const uint32_t st = stages + (k % kSStages) * kSStage;
-        const uint32_t lut = luts + (k & 1) * kSLut;
-        const int nst = min(4, ((pr.words - cur.sub * kSWords) >> 2) - 4 * kh);
-        if (nst > 0) {
-            if (pr.mode == kSRow)
-                acc += unit_rows_any<kSRow>(st, lut, r, kh, nst);
-            else if (pr.mode == kSG128)
-                acc += unit_rows_any<kSG128>(st, lut, r, kh, nst);
-            else
-                acc += unit_rows_any<kSG256>(st, lut, r, kh, nst);
-        }
+        const uint32_t st = stages + s * kSStage;
+        const uint32_t lut = luts + b * kSLut;
+        if (pr.mode == kSRow)
+            acc += unit_row<kSRow>(st, lut, r);
+        else if (pr.mode == kSG128)
+            acc += unit_row<kSG128>(st, lut, r);
+        else
+            acc += unit_row<kSG256>(st, lut, r);
+        mbar_arrive(empty(s));
+        mbar_arrive(tempty(b));
 
         const bool tile_end = (cur.sub == pr.n_sub - 1);
-        if (tile_end || u == u_end - 1) {
-            // the two K halves of each row, in a fixed order
-            if (kh == 1) s_half[r] = acc;
-            __syncthreads();
+        if (tile_end || k == nu - 1) {
             const int n = cur.rb * kSRows + r;
             const bool row_ok = n < pr.N;
-            float v = acc + s_half[r];
+            float v = acc;
             if (pr.mode == kSRow && row_ok) v *= __ldg(pr.scales + (pr.per_tensor ? 0 : n));
             if (tile_from_start && tile_end) {
-                if (kh == 0 && row_ok) {
+                if (row_ok) {
                     if (P.y_bf16)
                         reinterpret_cast<__nv_bfloat16*>(pr.Y)[n] = __float2bfloat16_rn(v);
                     else
@@ -320,12 +365,18 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                 const int c_a = tile_u0 / P.upc;
                 const int c_b = (tile_u0 + pr.n_sub - 1) / P.upc;
                 const int slot = (u_begin >= tile_u0) ? 0 : 1;
-                if (kh == 0) __stcg(P.part + ((int64_t)blockIdx.x * 2 + slot) * kSRows + r, v);
+                __stcg(P.part + ((int64_t)blockIdx.x * 2 + slot) * kSRows + r, v);
                 __threadfence();
-                __syncthreads();
-                if (t == 0) s_last = (atomicAdd(P.ticket + tile, 1) == c_b - c_a);
-                __syncthreads();
-                if (s_last && kh == 0) {
+                mbar_arrive(bar_part);
+                const uint32_t ph = (uint32_t)(events & 1);
+                ++events;
+                if (r == 0) {
+                    if (!mbar_wait(bar_part, ph, abort_flag)) break;
+                    s_last = (atomicAdd(P.ticket + tile, 1) == c_b - c_a);
+                    mbar_arrive(bar_last);
+                }
+                if (!mbar_wait(bar_last, ph, abort_flag)) break;
+                if (s_last) {
                     __threadfence();
                     float sum = 0.0f;
                     for (int c = c_a; c <= c_b; ++c) {
@@ -339,18 +390,14 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                         else
                             reinterpret_cast<float*>(pr.Y)[n] = sum;
                     }
-                    if (t == 0) P.ticket[tile] = 0;  // leave the ticket zeroed
+                    if (r == 0) P.ticket[tile] = 0;  // leave the ticket zeroed
                 }
             }
             acc = 0.0f;
             tile_from_start = true;  // every later tile of this range starts inside it
         }
-
-        // tables of the next unit into the other buffer (its last reader was unit u-1)
-        if (u + 1 < u_end && xn_ok) build_half_table(luts + ((k + 1) & 1) * kSLut + tb_idx * kTab, xn, tb_half);
-        cur = nxt;
+        advance(P.p, cur);
     }
-    cp_async_wait<0>();
 }
 
 // ---- host side -------------------------------------------------------------------
@@ -361,10 +408,10 @@ bool stream_eligible(const ProbShape& s, int64_t M) {
     if (s.K % 512 != 0) return false;
     if (s.granularity == SHERRY_PER_TENSOR || s.granularity == SHERRY_PER_CHANNEL) return true;
     if (s.granularity != SHERRY_PER_GROUP) return false;
-    if (s.group == 128) return true;                        // K/128 % 4 == 0 since K % 512 == 0
-    if (s.group == 256) return (s.K / 256) % 4 == 0;        // 16-byte aligned scale rows
-    return false;
+    return s.group == 128 || s.group == 256;  // K % 512 == 0: 4 or 2 whole groups per unit
 }
+
+int64_t stream_tiles(const ProbShape& s) { return (s.N + kSRows - 1) / kSRows; }
 
 struct SPlan {
     std::vector<SProb> probs;
@@ -444,6 +491,16 @@ int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* desc
     if (count <= 1) return stream_launch_t<1>(pl, y_bf16, workspace, stream);
     if (count <= 16) return stream_launch_t<16>(pl, y_bf16, workspace, stream);
     return stream_launch_t<SHERRY_MAX_BATCH>(pl, y_bf16, workspace, stream);
+}
+
+int stream_status_take() {
+    int v = 0;
+    SHERRY_CUDA_CHECK(cudaMemcpyFromSymbol(&v, g_stream_status, sizeof(int)));
+    if (v) {
+        const int zero = 0;
+        SHERRY_CUDA_CHECK(cudaMemcpyToSymbol(g_stream_status, &zero, sizeof(int)));
+    }
+    return v;
 }
 
 }  // namespace sherry

@@ -563,7 +563,8 @@ int device_status_take(cudaStream_t stream) {
         SHERRY_CUDA_CHECK(cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)));
     }
     const int w = skinny_status_take();
-    return v ? v : w;
+    const int x = stream_status_take();
+    return v ? v : w ? w : x;
 }
 
 }  // namespace sherry
