@@ -44,9 +44,9 @@ constexpr int kSSgn = kSRows * 16;                 // 8 KB (16 sign bytes per ro
 constexpr int kSSc = kSRows * 16;                  // 8 KB (at most 4 fp32 scales per row)
 constexpr int kSStage = kSIdx + kSSgn + kSSc;      // 48 KB
 constexpr int kSTabs = kSWords * 8;                // 128 tables per unit
-constexpr int kSLut = kSTabs * kTab;               // 18 KB
+constexpr int kSLut = kSTabs * kTab;               // 18 KB, one table buffer per stage
 constexpr int kSBars = 128;                        // mbarriers
-constexpr int kSSmem = 256 + kSStages * kSStage + 2 * kSLut + kSBars;
+constexpr int kSSmem = 256 + kSStages * (kSStage + kSLut) + kSBars;
 static_assert(kSStage % 256 == 0 && kSLut % 256 == 0, "table bases must stay multiples of 256");
 static_assert(kSTabs == 32 * kSHelpers, "one table per helper thread");
 constexpr long long kSWaitCycles = 4000000000LL;   // ~2 s at the boost clock
@@ -136,8 +136,17 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
     return v;
 }
 
+// (x, y) = (a0 + b0, a1 + b1): one packed fp32x2 add
+__device__ __forceinline__ void add_pair(float& x, float& y, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(x), "=f"(y)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // 8 lookups of one packed word (tables of blocks BOFF..BOFF+7 at shared address
 // `base`, a multiple of 256) -> even-position and odd-position partial sums
+// p0 = (v0 + v2) + (v4 + v6), p1 = (v1 + v3) + (v5 + v7), as packed pair adds
 template <int BOFF>
 __device__ __forceinline__ void word_sums(uint32_t w, uint32_t s, uint32_t base, float& p0, float& p1) {
     uint32_t ev, od;
@@ -150,8 +159,10 @@ __device__ __forceinline__ void word_sums(uint32_t w, uint32_t s, uint32_t base,
     const float v5 = lds_imm<(BOFF + 5) * kTab>(__byte_perm(od, base, 0x7652u));
     const float v6 = lds_imm<(BOFF + 6) * kTab>(__byte_perm(ev, base, 0x7653u));
     const float v7 = lds_imm<(BOFF + 7) * kTab>(__byte_perm(od, base, 0x7653u));
-    p0 = (v0 + v2) + (v4 + v6);
-    p1 = (v1 + v3) + (v5 + v7);
+    float a0, a1, b0, b1;
+    add_pair(a0, a1, v0, v1, v2, v3);
+    add_pair(b0, b1, v4, v5, v6, v7);
+    add_pair(p0, p1, a0, a1, b0, b1);
 }
 
 struct UnitPos {
@@ -176,35 +187,57 @@ __device__ __forceinline__ void advance(const SProb* probs, UnitPos& u) {
     }
 }
 
-// Helper warp h's share of one unit's copies into `stage`: rows [128h, 128h+128)
-// of the unit.  Packed words: row rl's 64 bytes land as four 16-byte chunks, chunk
-// c at (c ^ ((rl >> 1) & 3)); sign bytes and scales: 16 bytes per row.
-__device__ __forceinline__ void copy_unit(const SProb& pr, const UnitPos& u, uint32_t stage, int h, int lane) {
-    const int row0 = u.rb * kSRows;
-    const int N = pr.N, words = pr.words;
-    {
-        const int c = lane & 3;
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-            const int rl = 128 * h + 8 * i + (lane >> 2);
-            const int row = row0 + rl;
-            const bool ok = row < N;
-            const uint32_t* src = pr.idx + (int64_t)row * words + u.sub * kSWords + 4 * c;
-            cp_async16(stage + rl * 64 + ((c ^ ((rl >> 1) & 3)) << 4), ok ? src : pr.idx, ok);
-        }
+// Copy geometry of helper lane (h, lane) for one row block: the unit's rows
+// [128h, 128h+128).  Packed words: rows 128h + 8i + lane/4 (i = 0..15), 16-byte
+// chunk lane%4 of the row's 64 bytes, stored at chunk (c ^ ((row >> 1) & 3)) of a
+// 64-byte shared row (that swizzle term is (lane >> 3) & 3 for every i).  Sign
+// bytes and scales: rows 128h + 32i + lane (i = 0..3), 16 bytes each.  Byte
+// offsets from the plane bases; a row past N reads row 0 instead (its results
+// are never stored), so every copy is a full in-bounds 16 bytes.
+struct CopyRows {
+    uint32_t idx[16], sgn[4], sc[4];
+};
+
+__device__ __forceinline__ void copy_rows(const SProb& pr, int rb, int h, int lane, CopyRows& cr) {
+    const int row0 = rb * kSRows;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int row = row0 + 128 * h + 8 * i + (lane >> 2);
+        cr.idx[i] = (uint32_t)((int64_t)(row < pr.N ? row : 0) * pr.words * 4 + 16 * (lane & 3));
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int rl = 128 * h + 32 * i + lane;
-        const int row = row0 + rl;
-        const bool ok = row < N;
-        cp_async16(stage + kSIdx + rl * 16, ok ? pr.sgn + (int64_t)row * words + u.sub * kSWords : pr.sgn, ok);
-        if (pr.mode == kSG128)
-            cp_async16(stage + kSIdx + kSSgn + rl * 16, ok ? pr.scales + (int64_t)row * pr.spr + u.sub * 4 : pr.scales,
-                       ok);
-        else if (pr.mode == kSG256)
-            cp_async8(stage + kSIdx + kSSgn + rl * 16, ok ? pr.scales + (int64_t)row * pr.spr + u.sub * 2 : pr.scales,
-                      ok);
+        const int row = row0 + 128 * h + 32 * i + lane;
+        const int rr = row < pr.N ? row : 0;
+        cr.sgn[i] = (uint32_t)((int64_t)rr * pr.words);
+        cr.sc[i] = (uint32_t)((int64_t)rr * pr.spr * 4);
+    }
+}
+
+__device__ __forceinline__ const void* byte_off(const void* base, uint32_t off) {
+    return static_cast<const char*>(base) + off;
+}
+
+// Helper lane's copies of unit (cr's row block, sub-slice `sub`) into `stage`.
+__device__ __forceinline__ void copy_unit(const SProb& pr, const CopyRows& cr, int sub, uint32_t stage, int h,
+                                          int lane) {
+    const char* bi = reinterpret_cast<const char*>(pr.idx) + sub * (kSWords * 4);
+    const uint32_t di = stage + (uint32_t)(128 * h + (lane >> 2)) * 64u +
+                        ((uint32_t)((lane & 3) ^ ((lane >> 3) & 3)) << 4);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) cp_async16(di + 512u * i, byte_off(bi, cr.idx[i]), true);
+    const char* bs = reinterpret_cast<const char*>(pr.sgn) + sub * kSWords;
+    const uint32_t ds = stage + kSIdx + (uint32_t)(128 * h + lane) * 16u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) cp_async16(ds + 512u * i, byte_off(bs, cr.sgn[i]), true);
+    if (pr.mode == kSG128) {
+        const char* ba = reinterpret_cast<const char*>(pr.scales) + sub * 16;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cp_async16(ds + kSSgn + 512u * i, byte_off(ba, cr.sc[i]), true);
+    } else if (pr.mode == kSG256) {
+        const char* ba = reinterpret_cast<const char*>(pr.scales) + sub * 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cp_async8(ds + kSSgn + 512u * i, byte_off(ba, cr.sc[i]), true);
     }
 }
 
@@ -232,7 +265,11 @@ __device__ __forceinline__ float unit_row(uint32_t st, uint32_t lut, int r) {
         word_sums<8>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
         word_sums<16>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
         word_sums<24>(wq.w, sq >> 24, tb, u0, u1);
-        const float s4 = ((p0 + q0) + (r0 + u0)) + ((p1 + q1) + (r1 + u1));
+        float e0, e1, f0, f1, g0, g1;
+        add_pair(e0, e1, p0, p1, q0, q1);
+        add_pair(f0, f1, r0, r1, u0, u1);
+        add_pair(g0, g1, e0, e1, f0, f1);
+        const float s4 = g0 + g1;  // ((p0 + q0) + (r0 + u0)) + ((p1 + q1) + (r1 + u1))
         if (MODE == kSRow) {
             acc += s4;
         } else {
@@ -255,14 +292,13 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     // base is a multiple of 256 (a lookup's address replaces its low byte); the
     // XOR swizzles need only 16-byte alignment, since writer and reader apply them.
     const uint32_t stages = (smem_u32(g_smem) + 255u) & ~255u;
-    const uint32_t luts = stages + kSStages * kSStage;
-    const uint32_t bars = luts + 2 * kSLut;
-    auto full = [&](int s) { return bars + 8u * (uint32_t)s; };             // planes of a stage landed
-    auto empty = [&](int s) { return bars + 24u + 8u * (uint32_t)s; };      // consumers done with a stage
-    auto tfull = [&](int b) { return bars + 48u + 8u * (uint32_t)b; };      // tables of a buffer built
-    auto tempty = [&](int b) { return bars + 64u + 8u * (uint32_t)b; };     // consumers done with a buffer
-    const uint32_t bar_part = bars + 80u;  // every consumer stored its split-tile partial
-    const uint32_t bar_last = bars + 88u;  // the ticket's verdict is in s_last
+    const uint32_t luts = stages + kSStages * kSStage;  // table buffer s belongs to stage s
+    const uint32_t bars = luts + kSStages * kSLut;
+    // ready(s): the stage's planes landed and its tables are built; empty(s): consumers are done with both
+    auto ready = [&](int s) { return bars + 8u * (uint32_t)s; };
+    auto empty = [&](int s) { return bars + 32u + 8u * (uint32_t)s; };
+    const uint32_t bar_part = bars + 64u;  // every consumer stored its split-tile partial
+    const uint32_t bar_last = bars + 72u;  // the ticket's verdict is in s_last
 
     const int t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5;
@@ -272,12 +308,8 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     const int nu = u_end - u_begin;
     if (t == 0) {
         for (int s = 0; s < kSStages; ++s) {
-            mbar_init(full(s), 32 * kSHelpers);
+            mbar_init(ready(s), 2 * 32 * kSHelpers);  // one cp.async arrival and one table arrival per helper thread
             mbar_init(empty(s), kSRows);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(tfull(b), 32 * kSHelpers);
-            mbar_init(tempty(b), kSRows);
         }
         mbar_init(bar_part, kSRows);
         mbar_init(bar_last, 1);
@@ -288,35 +320,28 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     volatile int* abort_flag = &s_abort;
 
     if (warp >= kSConsumers) {
-        // ---- helpers: copies run two units ahead of the consumers, tables one
+        // ---- helpers: unit j's copies and tables go to stage j % kSStages once the
+        // consumers are done with unit j - kSStages there
         const int h = warp - kSConsumers;
         const int ht = t - 32 * kSConsumers;  // table (block of 4 activations) of the unit
-        UnitPos cu = locate(P, u_begin);      // next unit to copy
-        UnitPos tu = cu;                      // next unit to build tables for
-        uint2 xb = make_uint2(0u, 0u);
-        {
-            const SProb& pr = P.p[tu.p];
-            xb = __ldg(reinterpret_cast<const uint2*>(pr.X) + tu.sub * kSTabs + ht);
-        }
-        for (int j = 0; j <= nu; ++j) {
-            if (j < nu) {
-                const int s = j % kSStages;
-                if (j >= kSStages && !mbar_wait(empty(s), (uint32_t)(((j / kSStages) & 1) ^ 1), abort_flag)) break;
-                copy_unit(P.p[cu.p], cu, stages + s * kSStage, h, lane);
-                cp_async_arrive(full(s));
-                advance(P.p, cu);
-            }
-            const int tj = j - 1;  // tables of unit j-1 (its planes are in flight)
-            if (tj >= 0) {
-                const int b = tj & 1;
-                if (tj >= 2 && !mbar_wait(tempty(b), (uint32_t)(((tj >> 1) & 1) ^ 1), abort_flag)) break;
-                build_table(luts + b * kSLut + ht * kTab, xb);
-                mbar_arrive(tfull(b));
-                advance(P.p, tu);
-                if (tj + 1 < nu) {
-                    const SProb& pr = P.p[tu.p];
-                    xb = __ldg(reinterpret_cast<const uint2*>(pr.X) + tu.sub * kSTabs + ht);
-                }
+        UnitPos cu = locate(P, u_begin);
+        CopyRows cr;
+        copy_rows(P.p[cu.p], cu.rb, h, lane, cr);
+        uint2 xb = __ldg(reinterpret_cast<const uint2*>(P.p[cu.p].X) + cu.sub * kSTabs + ht);
+        for (int j = 0; j < nu; ++j) {
+            const int s = j % kSStages;
+            if (j >= kSStages && !mbar_wait(empty(s), (uint32_t)(((j / kSStages) & 1) ^ 1), abort_flag)) break;
+            const SProb& pr = P.p[cu.p];
+            copy_unit(pr, cr, cu.sub, stages + s * kSStage, h, lane);
+            cp_async_arrive(ready(s));
+            build_table(luts + s * kSLut + ht * kTab, xb);
+            mbar_arrive(ready(s));
+            const int p0 = cu.p, rb0 = cu.rb;
+            advance(P.p, cu);
+            if (j + 1 < nu) {
+                const SProb& pn = P.p[cu.p];
+                if (cu.p != p0 || cu.rb != rb0) copy_rows(pn, cu.rb, h, lane, cr);
+                xb = __ldg(reinterpret_cast<const uint2*>(pn.X) + cu.sub * kSTabs + ht);
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
@@ -330,12 +355,11 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     float acc = 0.0f;
     int events = 0;  // split tiles handled so far (phase of bar_part / bar_last)
     for (int k = 0; k < nu; ++k) {
-        const int s = k % kSStages, b = k & 1;
-        if (!mbar_wait(full(s), (uint32_t)((k / kSStages) & 1), abort_flag)) break;
-        if (!mbar_wait(tfull(b), (uint32_t)((k >> 1) & 1), abort_flag)) break;
+        const int s = k % kSStages;
+        if (!mbar_wait(ready(s), (uint32_t)((k / kSStages) & 1), abort_flag)) break;
         const SProb& pr = P.p[cur.p];
         const uint32_t st = stages + s * kSStage;
-        const uint32_t lut = luts + b * kSLut;
+        const uint32_t lut = luts + s * kSLut;
         if (pr.mode == kSRow)
             acc += unit_row<kSRow>(st, lut, r);
         else if (pr.mode == kSG128)
@@ -343,7 +367,6 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         else
             acc += unit_row<kSG256>(st, lut, r);
         mbar_arrive(empty(s));
-        mbar_arrive(tempty(b));
 
         const bool tile_end = (cur.sub == pr.n_sub - 1);
         if (tile_end || k == nu - 1) {
@@ -406,6 +429,7 @@ bool stream_eligible(const ProbShape& s, int64_t M) {
     if (M != 1 || s.N == 0) return false;
     if ((s.N + kSRows - 1) / kSRows > kMaxTickets) return false;
     if (s.K % 512 != 0) return false;
+    if (s.N * (s.K / 8) >= (int64_t(1) << 32) - 64) return false;  // 32-bit byte offsets into the planes
     if (s.granularity == SHERRY_PER_TENSOR || s.granularity == SHERRY_PER_CHANNEL) return true;
     if (s.granularity != SHERRY_PER_GROUP) return false;
     return s.group == 128 || s.group == 256;  // K % 512 == 0: 4 or 2 whole groups per unit
