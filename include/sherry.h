@@ -126,7 +126,8 @@ int sherry_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K, int g
  *            fully overwritten
  *   workspace  sherry_workspace_bytes(SHERRY_OP_LINEAR, M, N, K, g, group) bytes
  * fp32 accumulation; alpha applied once per group (or row).  Kernels:
- * M == 1 a lookup-table decode kernel; 2 <= M <= 8 with K % 128 == 0 a
+ * M == 1 with K % 512 == 0 (group 128 or 256, per-channel or per-tensor) a
+ * warp-specialised lookup-table decode kernel; 2 <= M <= 8 with K % 128 == 0 a
  * warp-level tensor-core (mma.sync) kernel; 9 <= M <= 32 with K % 256 == 0 and
  * (per-group) group % 64 == 0 a tensor-core (tcgen05) kernel for few tokens;
  * M >= 17 with K % 64 == 0 and group % 64 == 0 the tcgen05 prefill kernel;
@@ -214,9 +215,9 @@ const char* sherry_status_string(int status);
 /* cudaError_t value behind the last SHERRY_ERR_CUDA returned on this thread */
 int sherry_last_cuda_error(void);
 /* Synchronises `stream`, then returns SHERRY_ERR_TIMEOUT if a bounded device
- * wait of a tensor-core kernel gave up since the previous query (its outputs are
- * then invalid), else SHERRY_OK; clears the flag.  SHERRY_ERR_CUDA if the
- * synchronisation fails. */
+ * wait of a tensor-core kernel or of the one-token decode kernel gave up since
+ * the previous query (its outputs are then invalid), else SHERRY_OK; clears the
+ * flag.  SHERRY_ERR_CUDA if the synchronisation fails. */
 int sherry_device_status(void* stream);
 /* library version, e.g. 0x000100 = 0.1.0 */
 int sherry_version(void);

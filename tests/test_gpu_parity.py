@@ -127,6 +127,7 @@ LIN_CASES = [
     (1, 70, 8192, "channel", 0),
     (1, 513, 160, "tensor", 0),
     (1, 200, 1024, "group", 256),
+    (1, 130, 512, "group", 256),    # one-token kernel, one 512-weight unit, two groups of 256
     (1, 64, 2048, "group", 32),
     (2, 129, 512, "group", 128),
     (3, 64, 3072, "channel", 0),
@@ -224,7 +225,7 @@ def test_split_k_tickets_left_zero(sw):
 
 STREAM_SHAPES = [(1024, 3072, "group", 128), (300, 3072, "channel", 0), (3072, 8192, "group", 128),
                  (77, 1024, "group", 256), (513, 2048, "tensor", 0), (8192, 3072, "group", 128),
-                 (1, 512, "group", 128), (257, 3072, "group", 256)]
+                 (1, 512, "group", 128), (257, 3072, "group", 256), (96, 1536, "group", 256)]
 
 
 def test_stream_batch_many_problems_vs_oracle(sw, orc):
