@@ -136,14 +136,6 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
     return v;
 }
 
-// (x, y) = (a0 + b0, a1 + b1): one packed fp32x2 add
-__device__ __forceinline__ void add_pair(float& x, float& y, float a0, float a1, float b0, float b1) {
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(x), "=f"(y)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
 // 8 lookups of one packed word (tables of blocks BOFF..BOFF+7 at shared address
 // `base`, a multiple of 256) -> even-position and odd-position partial sums
 // p0 = (v0 + v2) + (v4 + v6), p1 = (v1 + v3) + (v5 + v7), as packed pair adds
@@ -160,9 +152,9 @@ __device__ __forceinline__ void word_sums(uint32_t w, uint32_t s, uint32_t base,
     const float v6 = lds_imm<(BOFF + 6) * kTab>(__byte_perm(ev, base, 0x7653u));
     const float v7 = lds_imm<(BOFF + 7) * kTab>(__byte_perm(od, base, 0x7653u));
     float a0, a1, b0, b1;
-    add_pair(a0, a1, v0, v1, v2, v3);
-    add_pair(b0, b1, v4, v5, v6, v7);
-    add_pair(p0, p1, a0, a1, b0, b1);
+    add2(a0, a1, v0, v1, v2, v3);
+    add2(b0, b1, v4, v5, v6, v7);
+    add2(p0, p1, a0, a1, b0, b1);
 }
 
 struct UnitPos {
@@ -266,9 +258,9 @@ __device__ __forceinline__ float unit_row(uint32_t st, uint32_t lut, int r) {
         word_sums<16>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
         word_sums<24>(wq.w, sq >> 24, tb, u0, u1);
         float e0, e1, f0, f1, g0, g1;
-        add_pair(e0, e1, p0, p1, q0, q1);
-        add_pair(f0, f1, r0, r1, u0, u1);
-        add_pair(g0, g1, e0, e1, f0, f1);
+        add2(e0, e1, p0, p1, q0, q1);
+        add2(f0, f1, r0, r1, u0, u1);
+        add2(g0, g1, e0, e1, f0, f1);
         const float s4 = g0 + g1;  // ((p0 + q0) + (r0 + u0)) + ((p1 + q1) + (r1 + u1))
         if (MODE == kSRow) {
             acc += s4;

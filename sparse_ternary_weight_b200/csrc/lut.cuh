@@ -95,27 +95,6 @@ __device__ __forceinline__ void add2(float& x, float& y, float a0, float a1, flo
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// 8 lookups of one packed word against the tables of blocks BOFF..BOFF+7 at
-// `base` (a multiple of 256 bytes); returns the lookups as two partial sums
-// (even-position and odd-position pairs), using packed fp32x2 adds.
-template <int BOFF>
-__device__ __forceinline__ void word_pair_sum(uint32_t w, uint32_t s, uint32_t base, float& p0, float& p1) {
-    uint32_t ev, od;
-    spread_word(w, s, ev, od);
-    const float v0 = lds_imm<(BOFF + 0) * kTab>(__byte_perm(ev, base, 0x7650u));
-    const float v1 = lds_imm<(BOFF + 1) * kTab>(__byte_perm(od, base, 0x7650u));
-    const float v2 = lds_imm<(BOFF + 2) * kTab>(__byte_perm(ev, base, 0x7651u));
-    const float v3 = lds_imm<(BOFF + 3) * kTab>(__byte_perm(od, base, 0x7651u));
-    const float v4 = lds_imm<(BOFF + 4) * kTab>(__byte_perm(ev, base, 0x7652u));
-    const float v5 = lds_imm<(BOFF + 5) * kTab>(__byte_perm(od, base, 0x7652u));
-    const float v6 = lds_imm<(BOFF + 6) * kTab>(__byte_perm(ev, base, 0x7653u));
-    const float v7 = lds_imm<(BOFF + 7) * kTab>(__byte_perm(od, base, 0x7653u));
-    float a0, a1, b0, b1;
-    add2(a0, a1, v0, v1, v2, v3);
-    add2(b0, b1, v4, v5, v6, v7);
-    add2(p0, p1, a0, a1, b0, b1);
-}
-
 // bf16 {+1, 0, -1} of the 4 weights of a block: two packed halves
 __device__ __forceinline__ uint2 decode_block_bf16(uint32_t nib, uint32_t g) {
     const uint32_t z = nib >> 2;
