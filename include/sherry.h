@@ -126,9 +126,9 @@ int sherry_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K, int g
  *            fully overwritten
  *   workspace  sherry_workspace_bytes(SHERRY_OP_LINEAR, M, N, K, g, group) bytes
  * fp32 accumulation; alpha applied once per group (or row).  Kernels:
- * M == 1 with K % 512 == 0 (group 128 or 256, per-channel or per-tensor) a
- * warp-specialised lookup-table decode kernel; 2 <= M <= 8 with K % 128 == 0 a
- * warp-level tensor-core (mma.sync) kernel; 9 <= M <= 32 with K % 256 == 0 and
+ * M <= 2 with K % 512 == 0 (group 128 or 256, per-channel or per-tensor) a
+ * warp-specialised lookup-table decode kernel; other 2 <= M <= 8 with
+ * K % 128 == 0 a warp-level tensor-core (mma.sync) kernel; 9 <= M <= 32 with K % 256 == 0 and
  * (per-group) group % 64 == 0 a tensor-core (tcgen05) kernel for few tokens;
  * M >= 17 with K % 64 == 0 and group % 64 == 0 the tcgen05 prefill kernel;
  * anything else the general lookup-table kernel (any M). */
@@ -153,11 +153,13 @@ typedef struct sherry_linear_desc {
 /* ---- batched packed linear ----------------------------------------------
  * `count` independent linears with the same M in one call, e.g. the
  * projections of a decoder layer stack for one token.  Each desc is computed
- * as by sherry_linear, by the kernel that sherry_linear would pick for it: the
- * problems that share a kernel share one launch of it (each prefill problem,
- * M >= 17, gets a launch of its own).  Y agrees with sherry_linear's within the
- * fp32 summation-order bound; the one-token kernel splits K where the batch as
- * a whole balances best, so it is not bit-identical to a single call.  A call
+ * as by sherry_linear, by the kernel that sherry_linear would pick for it
+ * (except that the streaming kernel's problems go to the others when the whole
+ * batch has more row blocks than its tickets): the problems that share a kernel
+ * share one launch of it (each prefill problem, M >= 17, gets a launch of its
+ * own).  Y agrees with sherry_linear's within the fp32 summation-order bound;
+ * the streaming kernel (one or two tokens) splits K where the batch as a whole
+ * balances best, so it is not bit-identical to a single call.  A call
  * repeated with the same arguments gives bit-identical Y.  `descs` is a HOST
  * array, read during the call only.  count <= SHERRY_MAX_BATCH.
  *   workspace  sherry_linear_batched_workspace_bytes(descs, count, M) bytes. */
@@ -180,7 +182,7 @@ size_t sherry_linear_batched_workspace_bytes(const sherry_linear_desc* descs, in
  * what the previous call left; all calls share the one array, so calls that
  * overlap on the GPU (other streams, other host threads) race -- keep them
  * ordered.  Nothing is allocated or freed. */
-#define SHERRY_NOALLOC_SCRATCH_BYTES ((size_t)1 << 20)
+#define SHERRY_NOALLOC_SCRATCH_BYTES ((size_t)2 << 20)  /* enough for every kernel on up to 224 SMs */
 int sherry_linear_noalloc(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                           const uint32_t* idx, const uint8_t* sgn, const float* scales,
                           int granularity, int group, void* Y, int y_dtype, void* stream);
@@ -215,7 +217,7 @@ const char* sherry_status_string(int status);
 /* cudaError_t value behind the last SHERRY_ERR_CUDA returned on this thread */
 int sherry_last_cuda_error(void);
 /* Synchronises `stream`, then returns SHERRY_ERR_TIMEOUT if a bounded device
- * wait of a tensor-core kernel or of the one-token decode kernel gave up since
+ * wait of a tensor-core kernel or of the streaming decode kernel gave up since
  * the previous query (its outputs are then invalid), else SHERRY_OK; clears the
  * flag.  SHERRY_ERR_CUDA if the synchronisation fails. */
 int sherry_device_status(void* stream);

@@ -2,6 +2,7 @@
 // on the host, then the launches.  Nothing here allocates device memory.
 #include "common.cuh"
 
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
@@ -47,34 +48,29 @@ static int check_planes(const uint32_t* idx, const uint8_t* sgn, const float* sc
     return SHERRY_OK;
 }
 
-// the decode path a set of linears takes: the streaming one-token kernel when
-// every problem qualifies, else the general lookup-table kernel
-static bool use_stream(const ProbShape* shapes, int count, int64_t M) {
-    if (M != 1 || count == 0) return false;
-    int64_t tiles = 0;
-    for (int i = 0; i < count; ++i) {
-        if (!stream_eligible(shapes[i], M)) return false;
-        tiles += stream_tiles(shapes[i]);
-    }
-    return tiles <= kMaxTickets;
-}
-
-// Which kernel computes each problem of a call.  2 <= M <= 8 problems with
-// K % 128 == 0 share one launch of the warp-MMA kernel; other problems with up
-// to 32 tokens that fit the tcgen05 few-token kernel share one launch of it; of
-// the rest, each
-// problem with M >= 17 that fits the prefill kernel gets a launch of its own;
-// what remains shares one launch of the one-token streaming kernel (M == 1,
-// every remaining problem eligible) or of the general lookup-table kernel.
+// Which kernel computes each problem of a call.  Problems with one or two tokens
+// that fit the streaming lookup-table kernel share one launch of it (unless their
+// row blocks would outnumber its tickets); 2 <= M <= 8 problems with K % 128 == 0
+// share one launch of the warp-MMA kernel; other problems with up to 32 tokens
+// that fit the tcgen05 few-token kernel share one launch of it; each problem with
+// M >= 17 that fits the prefill kernel gets a launch of its own; what remains
+// shares one launch of the general lookup-table kernel.
 struct Routes {
-    std::vector<ProbShape> hmma_s, skinny_s, rest_s;
-    std::vector<sherry_linear_desc> hmma_d, skinny_d, rest_d;
+    std::vector<ProbShape> stream_s, hmma_s, skinny_s, rest_s;
+    std::vector<sherry_linear_desc> stream_d, hmma_d, skinny_d, rest_d;
     std::vector<int> prefill;  // indices into the call's problems
 };
 
 static void route(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, Routes& r) {
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i)
+        if (stream_eligible(shapes[i], M)) tiles += stream_tiles(shapes[i]);
+    const bool stream_ok = tiles > 0 && tiles <= kMaxTickets;
     for (int i = 0; i < count; ++i) {
-        if (hmma_eligible(shapes[i], M)) {
+        if (stream_ok && stream_eligible(shapes[i], M)) {
+            r.stream_s.push_back(shapes[i]);
+            if (descs) r.stream_d.push_back(descs[i]);
+        } else if (hmma_eligible(shapes[i], M)) {
             r.hmma_s.push_back(shapes[i]);
             if (descs) r.hmma_d.push_back(descs[i]);
         } else if (skinny_eligible(shapes[i], M)) {
@@ -89,13 +85,15 @@ static void route(const ProbShape* shapes, const sherry_linear_desc* descs, int 
     }
 }
 
+// The streaming and general lookup-table launches of a call run one after the
+// other on its stream and share the workspace (tickets first, both leave them zero).
 static size_t linear_ws_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
     Routes r;
     route(shapes, nullptr, count, M, r);
-    const int n = (int)r.rest_s.size();
-    if (n == 0) return 0;
-    if (use_stream(r.rest_s.data(), n, M)) return stream_workspace_bytes(r.rest_s.data(), n, sms);
-    return lut_workspace_bytes(r.rest_s.data(), n, M, sms);
+    size_t ws = 0;
+    if (!r.stream_s.empty()) ws = stream_workspace_bytes(r.stream_s.data(), (int)r.stream_s.size(), M, sms);
+    if (!r.rest_s.empty()) ws = std::max(ws, lut_workspace_bytes(r.rest_s.data(), (int)r.rest_s.size(), M, sms));
+    return ws;
 }
 
 static int linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
@@ -112,11 +110,12 @@ static int linear_launch(const ProbShape* shapes, const sherry_linear_desc* desc
         return st;
     for (int i : r.prefill)
         if ((st = prefill_launch(shapes[i], descs[i], M, y_bf16, stream))) return st;
-    const int n = (int)r.rest_s.size();
-    if (n == 0) return SHERRY_OK;
-    if (use_stream(r.rest_s.data(), n, M))
-        return stream_linear_launch(r.rest_s.data(), r.rest_d.data(), n, y_bf16, workspace, sms, stream);
-    return lut_linear_launch(r.rest_s.data(), r.rest_d.data(), n, M, y_bf16, workspace, sms, stream);
+    if (!r.stream_s.empty() &&
+        (st = stream_linear_launch(r.stream_s.data(), r.stream_d.data(), (int)r.stream_s.size(), M, y_bf16, workspace,
+                                   sms, stream)))
+        return st;
+    if (r.rest_s.empty()) return SHERRY_OK;
+    return lut_linear_launch(r.rest_s.data(), r.rest_d.data(), (int)r.rest_s.size(), M, y_bf16, workspace, sms, stream);
 }
 
 }  // namespace sherry

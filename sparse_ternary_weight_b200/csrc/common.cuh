@@ -123,12 +123,12 @@ bool skinny_eligible(const ProbShape& s, int64_t M);
 int skinny_status_take();  // SHERRY_ERR_TIMEOUT if a bounded wait gave up since the last call
 int skinny_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          int sms, cudaStream_t stream);
-// one-token streaming kernel (gemv_stream.cu)
+// one- and two-token streaming kernel (gemv_stream.cu)
 bool stream_eligible(const ProbShape& s, int64_t M);
 int64_t stream_tiles(const ProbShape& s);  // row blocks (tickets) of one problem
 int stream_status_take();                   // SHERRY_ERR_TIMEOUT if a bounded wait gave up since the last call
-size_t stream_workspace_bytes(const ProbShape* shapes, int count, int sms);
-int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int y_bf16,
+size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms);
+int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream);
 
 }  // namespace sherry

@@ -1,8 +1,9 @@
-// gemv_stream.cu -- packed 3:4 ternary linear, one token (M = 1), HBM-streaming
-// version of the lookup-table decode (the method's inference scheme: tables
-// built from the activations, looked up by the packed weights, accumulated,
-// then scaled; "Sherry: Hardware-Efficient 1.25-Bit Ternary Quantization via
-// Fine-grained Sparsification", digest paragraph on inference; Y = X T alpha).
+// gemv_stream.cu -- packed 3:4 ternary linear for one or two tokens (M <= 2),
+// HBM-streaming version of the lookup-table decode (the method's inference
+// scheme: tables built from the activations, looked up by the packed weights,
+// accumulated, then scaled; "Sherry: Hardware-Efficient 1.25-Bit Ternary
+// Quantization via Fine-grained Sparsification", digest paragraph on inference;
+// Y = X T alpha).
 //
 // Work unit: 512 output rows x 512 weights (16 packed words) of one linear.
 // All units of a launch (one or many independent linears) are split into equal
@@ -14,14 +15,15 @@
 // Roles (20 warps).  16 consumer warps: each thread owns one row of the unit
 // and only looks up and accumulates (per packed word it spreads the 8 nibbles
 // and sign bits into two byte-vectors of table offsets, see lut.cuh, and does 8
-// lookups; alpha is applied once per 128-weight group, or once per row).  4
-// helper warps, one per SM sub-partition: they copy each unit's packed planes
-// with 16-byte cp.async (8 lanes read one row's 64 contiguous bytes, so global
-// reads are coalesced) into an XOR-swizzled 3-stage ring that the row-per-lane
-// reads hit without bank conflicts, and build the unit's 128 tables of 32
-// entries into one of two buffers.  Stages and table buffers change hands
-// through mbarriers; every wait is bounded, and a timeout sets a device status
-// flag (reported by sherry_device_status) and ends the CTA.
+// lookups per token at the same offsets; alpha is applied once per 128-weight
+// group, or once per row).  4 helper warps, one per SM sub-partition: they copy
+// each unit's packed planes with 16-byte cp.async (4 lanes read one row's 64
+// contiguous bytes, so global reads are coalesced) into an XOR-swizzled ring of
+// stages (three for one token, two for two) that the row-per-lane reads hit
+// without bank conflicts, and build the unit's 128 tables of 32 entries per
+// token into the stage's table buffer.  Stages change hands through mbarriers;
+// every wait is bounded, and a timeout sets a device status flag (reported by
+// sherry_device_status) and ends the CTA.
 #include "common.cuh"
 #include "lut.cuh"
 
@@ -38,16 +40,23 @@ constexpr int kSHelpers = 4;                       // copy + table warps
 constexpr int kSThreads = 32 * (kSConsumers + kSHelpers);
 constexpr int kSRows = 32 * kSConsumers;           // 512 rows per unit
 constexpr int kSWords = 16;                        // packed words per unit (512 weights)
-constexpr int kSStages = 3;
 constexpr int kSIdx = kSRows * kSWords * 4;        // 32 KB
 constexpr int kSSgn = kSRows * 16;                 // 8 KB (16 sign bytes per row)
 constexpr int kSSc = kSRows * 16;                  // 8 KB (at most 4 fp32 scales per row)
 constexpr int kSStage = kSIdx + kSSgn + kSSc;      // 48 KB
 constexpr int kSTabs = kSWords * 8;                // 128 tables per unit
-constexpr int kSLut = kSTabs * kTab;               // 18 KB, one table buffer per stage
+constexpr int kSLut = kSTabs * kTab;               // 18 KB: one token's tables of a unit
 constexpr int kSBars = 128;                        // mbarriers
-constexpr int kSSmem = 256 + kSStages * (kSStage + kSLut) + kSBars;
 static_assert(kSStage % 256 == 0 && kSLut % 256 == 0, "table bases must stay multiples of 256");
+
+// Ring depth and shared bytes for MT tokens (tables are token-major within a stage).
+template <int MT>
+struct SCfg {
+    static constexpr int kStages = MT == 1 ? 3 : 2;
+    static constexpr int kLutStage = MT * kSLut;
+    static constexpr int kSmem = 256 + kStages * (kSStage + kLutStage) + kSBars;
+};
+static_assert(SCfg<1>::kSmem <= 232448 && SCfg<2>::kSmem <= 232448, "shared memory per CTA");
 static_assert(kSTabs == 32 * kSHelpers, "one table per helper thread");
 constexpr long long kSWaitCycles = 4000000000LL;   // ~2 s at the boost clock
 
@@ -68,7 +77,7 @@ struct SProb {
 template <int MAXP>
 struct SParams {
     int count, y_bf16, total_units, upc;
-    float* part;  // [grid][2][kSRows] split-tile partials
+    float* part;  // [grid][2][MT][kSRows] split-tile partials
     int* ticket;  // [total tiles]
     SProb p[MAXP];
 };
@@ -136,25 +145,41 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
     return v;
 }
 
-// 8 lookups of one packed word (tables of blocks BOFF..BOFF+7 at shared address
-// `base`, a multiple of 256) -> even-position and odd-position partial sums
-// p0 = (v0 + v2) + (v4 + v6), p1 = (v1 + v3) + (v5 + v7), as packed pair adds
-template <int BOFF>
-__device__ __forceinline__ void word_sums(uint32_t w, uint32_t s, uint32_t base, float& p0, float& p1) {
-    uint32_t ev, od;
-    spread_word(w, s, ev, od);
-    const float v0 = lds_imm<(BOFF + 0) * kTab>(__byte_perm(ev, base, 0x7650u));
-    const float v1 = lds_imm<(BOFF + 1) * kTab>(__byte_perm(od, base, 0x7650u));
-    const float v2 = lds_imm<(BOFF + 2) * kTab>(__byte_perm(ev, base, 0x7651u));
-    const float v3 = lds_imm<(BOFF + 3) * kTab>(__byte_perm(od, base, 0x7651u));
-    const float v4 = lds_imm<(BOFF + 4) * kTab>(__byte_perm(ev, base, 0x7652u));
-    const float v5 = lds_imm<(BOFF + 5) * kTab>(__byte_perm(od, base, 0x7652u));
-    const float v6 = lds_imm<(BOFF + 6) * kTab>(__byte_perm(ev, base, 0x7653u));
-    const float v7 = lds_imm<(BOFF + 7) * kTab>(__byte_perm(od, base, 0x7653u));
+// 8 lookups of one packed word for token TOK: the tables of blocks BOFF..BOFF+7
+// sit at shared offsets (BOFF + j) * kTab + TOK * kSLut from the addresses in a[],
+// whose low byte is the block's table offset -> even-position and odd-position
+// partial sums p0 = (v0 + v2) + (v4 + v6), p1 = (v1 + v3) + (v5 + v7), as
+// packed pair adds
+template <int BOFF, int TOK>
+__device__ __forceinline__ void token_sums(const uint32_t (&a)[8], float& p0, float& p1) {
+    constexpr int T = TOK * kSLut;
+    const float v0 = lds_imm<(BOFF + 0) * kTab + T>(a[0]);
+    const float v1 = lds_imm<(BOFF + 1) * kTab + T>(a[1]);
+    const float v2 = lds_imm<(BOFF + 2) * kTab + T>(a[2]);
+    const float v3 = lds_imm<(BOFF + 3) * kTab + T>(a[3]);
+    const float v4 = lds_imm<(BOFF + 4) * kTab + T>(a[4]);
+    const float v5 = lds_imm<(BOFF + 5) * kTab + T>(a[5]);
+    const float v6 = lds_imm<(BOFF + 6) * kTab + T>(a[6]);
+    const float v7 = lds_imm<(BOFF + 7) * kTab + T>(a[7]);
     float a0, a1, b0, b1;
     add2(a0, a1, v0, v1, v2, v3);
     add2(b0, b1, v4, v5, v6, v7);
     add2(p0, p1, a0, a1, b0, b1);
+}
+
+// One packed word (nibbles w, sign byte s; its 8 tables at `base`, a multiple of
+// 256, plus BOFF * kTab): the 8 table addresses are formed once and looked up for
+// each of the MT tokens.
+template <int BOFF, int MT>
+__device__ __forceinline__ void word_sums(uint32_t w, uint32_t s, uint32_t base, float (&p0)[MT], float (&p1)[MT]) {
+    uint32_t ev, od;
+    spread_word(w, s, ev, od);
+    const uint32_t a[8] = {__byte_perm(ev, base, 0x7650u), __byte_perm(od, base, 0x7650u),
+                           __byte_perm(ev, base, 0x7651u), __byte_perm(od, base, 0x7651u),
+                           __byte_perm(ev, base, 0x7652u), __byte_perm(od, base, 0x7652u),
+                           __byte_perm(ev, base, 0x7653u), __byte_perm(od, base, 0x7653u)};
+    token_sums<BOFF, 0>(a, p0[0], p1[0]);
+    if constexpr (MT > 1) token_sums<BOFF, 1>(a, p0[1], p1[1]);
 }
 
 struct UnitPos {
@@ -233,10 +258,10 @@ __device__ __forceinline__ void copy_unit(const SProb& pr, const CopyRows& cr, i
     }
 }
 
-// Lookups of one row over the 16 words of a unit; `st` and `lut` are shared
-// addresses of the unit's stage and table buffer.
-template <int MODE>
-__device__ __forceinline__ float unit_row(uint32_t st, uint32_t lut, int r) {
+// Lookups of one row over the 16 words of a unit for MT tokens, into u[]; `st`
+// and `lut` are shared addresses of the unit's stage and of token 0's tables.
+template <int MODE, int MT>
+__device__ __forceinline__ void unit_row(uint32_t st, uint32_t lut, int r, float (&u)[MT]) {
     const uint32_t sw = (uint32_t)((r >> 1) & 3);
     const uint4 sg = lds128(st + kSIdx + r * 16);
     uint4 av = make_uint4(0u, 0u, 0u, 0u);
@@ -246,46 +271,48 @@ __device__ __forceinline__ float unit_row(uint32_t st, uint32_t lut, int r) {
         av = make_uint4(a2.x, a2.y, 0u, 0u);
     }
     const uint32_t idx_row = st + r * 64;
-    float acc = 0.0f;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) u[m] = 0.0f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const uint4 wq = lds128(idx_row + (((uint32_t)q ^ sw) << 4));
         const uint32_t sq = q == 0 ? sg.x : q == 1 ? sg.y : q == 2 ? sg.z : sg.w;
         const uint32_t tb = lut + (uint32_t)(q * 32 * kTab);  // tables of words 4q..4q+3 (256-aligned)
-        float p0, p1, q0, q1, r0, r1, u0, u1;
-        word_sums<0>(wq.x, sq & 0xffu, tb, p0, p1);
-        word_sums<8>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
-        word_sums<16>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
-        word_sums<24>(wq.w, sq >> 24, tb, u0, u1);
-        float e0, e1, f0, f1, g0, g1;
-        add2(e0, e1, p0, p1, q0, q1);
-        add2(f0, f1, r0, r1, u0, u1);
-        add2(g0, g1, e0, e1, f0, f1);
-        const float s4 = g0 + g1;  // ((p0 + q0) + (r0 + u0)) + ((p1 + q1) + (r1 + u1))
-        if (MODE == kSRow) {
-            acc += s4;
-        } else {
-            uint32_t ab;
-            if (MODE == kSG128)
-                ab = q == 0 ? av.x : q == 1 ? av.y : q == 2 ? av.z : av.w;
+        float p0[MT], p1[MT], q0[MT], q1[MT], r0[MT], r1[MT], u0[MT], u1[MT];
+        word_sums<0, MT>(wq.x, sq & 0xffu, tb, p0, p1);
+        word_sums<8, MT>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
+        word_sums<16, MT>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
+        word_sums<24, MT>(wq.w, sq >> 24, tb, u0, u1);
+        uint32_t ab = 0u;
+        if (MODE == kSG128) ab = q == 0 ? av.x : q == 1 ? av.y : q == 2 ? av.z : av.w;
+        if (MODE == kSG256) ab = q < 2 ? av.x : av.y;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            float e0, e1, f0, f1, g0, g1;
+            add2(e0, e1, p0[m], p1[m], q0[m], q1[m]);
+            add2(f0, f1, r0[m], r1[m], u0[m], u1[m]);
+            add2(g0, g1, e0, e1, f0, f1);
+            const float s4 = g0 + g1;  // ((p0 + q0) + (r0 + u0)) + ((p1 + q1) + (r1 + u1))
+            if (MODE == kSRow)
+                u[m] += s4;
             else
-                ab = q < 2 ? av.x : av.y;
-            acc = fmaf(__uint_as_float(ab), s4, acc);
+                u[m] = fmaf(__uint_as_float(ab), s4, u[m]);
         }
     }
-    return acc;
 }
 
-template <int MAXP>
+template <int MAXP, int MT>
 __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_constant__ SParams<MAXP> P) {
+    using C = SCfg<MT>;
+    constexpr int S = C::kStages;
     __shared__ int s_last;
     __shared__ int s_abort;
     // Shared addresses: the buffer is rounded up to 256 bytes, so every table
     // base is a multiple of 256 (a lookup's address replaces its low byte); the
     // XOR swizzles need only 16-byte alignment, since writer and reader apply them.
     const uint32_t stages = (smem_u32(g_smem) + 255u) & ~255u;
-    const uint32_t luts = stages + kSStages * kSStage;  // table buffer s belongs to stage s
-    const uint32_t bars = luts + kSStages * kSLut;
+    const uint32_t luts = stages + S * kSStage;  // table buffer s (MT tokens' tables) belongs to stage s
+    const uint32_t bars = luts + S * C::kLutStage;
     // ready(s): the stage's planes landed and its tables are built; empty(s): consumers are done with both
     auto ready = [&](int s) { return bars + 8u * (uint32_t)s; };
     auto empty = [&](int s) { return bars + 32u + 8u * (uint32_t)s; };
@@ -299,7 +326,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     if (u_begin >= u_end) return;
     const int nu = u_end - u_begin;
     if (t == 0) {
-        for (int s = 0; s < kSStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(ready(s), 2 * 32 * kSHelpers);  // one cp.async arrival and one table arrival per helper thread
             mbar_init(empty(s), kSRows);
         }
@@ -312,28 +339,37 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     volatile int* abort_flag = &s_abort;
 
     if (warp >= kSConsumers) {
-        // ---- helpers: unit j's copies and tables go to stage j % kSStages once the
-        // consumers are done with unit j - kSStages there
+        // ---- helpers: unit j's copies and tables go to stage j % S once the
+        // consumers are done with unit j - S there
         const int h = warp - kSConsumers;
         const int ht = t - 32 * kSConsumers;  // table (block of 4 activations) of the unit
         UnitPos cu = locate(P, u_begin);
         CopyRows cr;
         copy_rows(P.p[cu.p], cu.rb, h, lane, cr);
-        uint2 xb = __ldg(reinterpret_cast<const uint2*>(P.p[cu.p].X) + cu.sub * kSTabs + ht);
+        // activations: token m's row of X starts K bf16 (words * 8 groups of 4) after token m-1's
+        uint2 xb[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+            xb[m] = __ldg(reinterpret_cast<const uint2*>(P.p[cu.p].X) + (int64_t)m * P.p[cu.p].words * 8 +
+                          cu.sub * kSTabs + ht);
         for (int j = 0; j < nu; ++j) {
-            const int s = j % kSStages;
-            if (j >= kSStages && !mbar_wait(empty(s), (uint32_t)(((j / kSStages) & 1) ^ 1), abort_flag)) break;
+            const int s = j % S;
+            if (j >= S && !mbar_wait(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag)) break;
             const SProb& pr = P.p[cu.p];
             copy_unit(pr, cr, cu.sub, stages + s * kSStage, h, lane);
             cp_async_arrive(ready(s));
-            build_table(luts + s * kSLut + ht * kTab, xb);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) build_table(luts + s * C::kLutStage + m * kSLut + ht * kTab, xb[m]);
             mbar_arrive(ready(s));
             const int p0 = cu.p, rb0 = cu.rb;
             advance(P.p, cu);
             if (j + 1 < nu) {
                 const SProb& pn = P.p[cu.p];
                 if (cu.p != p0 || cu.rb != rb0) copy_rows(pn, cu.rb, h, lane, cr);
-                xb = __ldg(reinterpret_cast<const uint2*>(pn.X) + cu.sub * kSTabs + ht);
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+                    xb[m] = __ldg(reinterpret_cast<const uint2*>(pn.X) + (int64_t)m * pn.words * 8 + cu.sub * kSTabs +
+                                  ht);
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
@@ -344,43 +380,55 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     const int r = t;
     UnitPos cur = locate(P, u_begin);
     bool tile_from_start = (P.p[cur.p].unit_begin + cur.rb * P.p[cur.p].n_sub == u_begin);
-    float acc = 0.0f;
+    float acc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
     int events = 0;  // split tiles handled so far (phase of bar_part / bar_last)
     for (int k = 0; k < nu; ++k) {
-        const int s = k % kSStages;
-        if (!mbar_wait(ready(s), (uint32_t)((k / kSStages) & 1), abort_flag)) break;
+        const int s = k % S;
+        if (!mbar_wait(ready(s), (uint32_t)((k / S) & 1), abort_flag)) break;
         const SProb& pr = P.p[cur.p];
         const uint32_t st = stages + s * kSStage;
-        const uint32_t lut = luts + s * kSLut;
+        const uint32_t lut = luts + s * C::kLutStage;
+        float u[MT];
         if (pr.mode == kSRow)
-            acc += unit_row<kSRow>(st, lut, r);
+            unit_row<kSRow, MT>(st, lut, r, u);
         else if (pr.mode == kSG128)
-            acc += unit_row<kSG128>(st, lut, r);
+            unit_row<kSG128, MT>(st, lut, r, u);
         else
-            acc += unit_row<kSG256>(st, lut, r);
+            unit_row<kSG256, MT>(st, lut, r, u);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[m] += u[m];
         mbar_arrive(empty(s));
 
         const bool tile_end = (cur.sub == pr.n_sub - 1);
         if (tile_end || k == nu - 1) {
             const int n = cur.rb * kSRows + r;
             const bool row_ok = n < pr.N;
-            float v = acc;
-            if (pr.mode == kSRow && row_ok) v *= __ldg(pr.scales + (pr.per_tensor ? 0 : n));
+            float v[MT];
+            const float rs = (pr.mode == kSRow && row_ok) ? __ldg(pr.scales + (pr.per_tensor ? 0 : n)) : 1.0f;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) v[m] = pr.mode == kSRow ? acc[m] * rs : acc[m];
             if (tile_from_start && tile_end) {
                 if (row_ok) {
-                    if (P.y_bf16)
-                        reinterpret_cast<__nv_bfloat16*>(pr.Y)[n] = __float2bfloat16_rn(v);
-                    else
-                        reinterpret_cast<float*>(pr.Y)[n] = v;
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        if (P.y_bf16)
+                            reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)m * pr.N + n] = __float2bfloat16_rn(v[m]);
+                        else
+                            reinterpret_cast<float*>(pr.Y)[(int64_t)m * pr.N + n] = v[m];
+                    }
                 }
             } else {
-                // split tile: partial into this CTA's slot, then the ticket
+                // split tile: partials into this CTA's slot, then the ticket
                 const int tile = pr.tile_begin + cur.rb;
                 const int tile_u0 = pr.unit_begin + cur.rb * pr.n_sub;
                 const int c_a = tile_u0 / P.upc;
                 const int c_b = (tile_u0 + pr.n_sub - 1) / P.upc;
                 const int slot = (u_begin >= tile_u0) ? 0 : 1;
-                __stcg(P.part + ((int64_t)blockIdx.x * 2 + slot) * kSRows + r, v);
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+                    __stcg(P.part + (((int64_t)blockIdx.x * 2 + slot) * MT + m) * kSRows + r, v[m]);
                 __threadfence();
                 mbar_arrive(bar_part);
                 const uint32_t ph = (uint32_t)(events & 1);
@@ -393,22 +441,26 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                 if (!mbar_wait(bar_last, ph, abort_flag)) break;
                 if (s_last) {
                     __threadfence();
-                    float sum = 0.0f;
-                    for (int c = c_a; c <= c_b; ++c) {
-                        const int sl = (c * P.upc >= tile_u0) ? 0 : 1;
-                        const float pv = __ldcg(P.part + ((int64_t)c * 2 + sl) * kSRows + r);
-                        sum = (c == c_a) ? pv : sum + pv;
-                    }
-                    if (row_ok) {
-                        if (P.y_bf16)
-                            reinterpret_cast<__nv_bfloat16*>(pr.Y)[n] = __float2bfloat16_rn(sum);
-                        else
-                            reinterpret_cast<float*>(pr.Y)[n] = sum;
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        float sum = 0.0f;
+                        for (int c = c_a; c <= c_b; ++c) {
+                            const int sl = (c * P.upc >= tile_u0) ? 0 : 1;
+                            const float pv = __ldcg(P.part + (((int64_t)c * 2 + sl) * MT + m) * kSRows + r);
+                            sum = (c == c_a) ? pv : sum + pv;
+                        }
+                        if (row_ok) {
+                            if (P.y_bf16)
+                                reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)m * pr.N + n] = __float2bfloat16_rn(sum);
+                            else
+                                reinterpret_cast<float*>(pr.Y)[(int64_t)m * pr.N + n] = sum;
+                        }
                     }
                     if (r == 0) P.ticket[tile] = 0;  // leave the ticket zeroed
                 }
             }
-            acc = 0.0f;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
             tile_from_start = true;  // every later tile of this range starts inside it
         }
         advance(P.p, cur);
@@ -418,7 +470,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
 // ---- host side -------------------------------------------------------------------
 
 bool stream_eligible(const ProbShape& s, int64_t M) {
-    if (M != 1 || s.N == 0) return false;
+    if ((M != 1 && M != 2) || s.N == 0) return false;
     if ((s.N + kSRows - 1) / kSRows > kMaxTickets) return false;
     if (s.K % 512 != 0) return false;
     if (s.N * (s.K / 8) >= (int64_t(1) << 32) - 64) return false;  // 32-bit byte offsets into the planes
@@ -437,7 +489,7 @@ struct SPlan {
 
 static int stream_ctas(int sms) { return sms; }  // one CTA per SM (the stages fill shared memory)
 
-static SPlan make_splan(const ProbShape* shapes, int count, int sms) {
+static SPlan make_splan(const ProbShape* shapes, int count, int64_t M, int sms) {
     SPlan pl;
     int ub = 0, tb = 0;
     for (int i = 0; i < count; ++i) {
@@ -462,15 +514,15 @@ static SPlan make_splan(const ProbShape* shapes, int count, int sms) {
     pl.upc = (ub + g - 1) / g;
     pl.grid = (ub + pl.upc - 1) / pl.upc;
     pl.part_off = kTicketBytes;
-    pl.ws_bytes = kTicketBytes + (size_t)pl.grid * 2 * kSRows * sizeof(float);
+    pl.ws_bytes = kTicketBytes + (size_t)pl.grid * 2 * (size_t)M * kSRows * sizeof(float);
     return pl;
 }
 
-size_t stream_workspace_bytes(const ProbShape* shapes, int count, int sms) {
-    return make_splan(shapes, count, sms).ws_bytes;
+size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
+    return make_splan(shapes, count, M, sms).ws_bytes;
 }
 
-template <int MAXP>
+template <int MAXP, int MT>
 static int stream_launch_t(SPlan& pl, int y_bf16, void* workspace, cudaStream_t stream) {
     static SParams<MAXP> P;
     static std::mutex mu;
@@ -484,17 +536,26 @@ static int stream_launch_t(SPlan& pl, int y_bf16, void* workspace, cudaStream_t 
     P.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.part_off);
     for (int i = 0; i < P.count; ++i) P.p[i] = pl.probs[i];
     if (!attr) {
-        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_lut_stream<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSSmem));
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_lut_stream<MAXP, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               SCfg<MT>::kSmem));
         attr = true;
     }
-    k_lut_stream<MAXP><<<pl.grid, kSThreads, kSSmem, stream>>>(P);
+    k_lut_stream<MAXP, MT><<<pl.grid, kSThreads, SCfg<MT>::kSmem, stream>>>(P);
     SHERRY_LAUNCH_CHECK();
     return SHERRY_OK;
 }
 
-int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int y_bf16,
+template <int MT>
+static int stream_launch_mt(SPlan& pl, int count, int y_bf16, void* workspace, cudaStream_t stream) {
+    if (count <= 1) return stream_launch_t<1, MT>(pl, y_bf16, workspace, stream);
+    if (count <= 16) return stream_launch_t<16, MT>(pl, y_bf16, workspace, stream);
+    return stream_launch_t<SHERRY_MAX_BATCH, MT>(pl, y_bf16, workspace, stream);
+}
+
+int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream) {
-    SPlan pl = make_splan(shapes, count, sms);
+    if (M != 1 && M != 2) return SHERRY_ERR_UNSUPPORTED;
+    SPlan pl = make_splan(shapes, count, M, sms);
     for (int i = 0; i < count; ++i) {
         SProb& p = pl.probs[i];
         p.X = descs[i].X;
@@ -504,9 +565,8 @@ int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* desc
         p.Y = descs[i].Y;
     }
     if (pl.total_units == 0) return SHERRY_OK;
-    if (count <= 1) return stream_launch_t<1>(pl, y_bf16, workspace, stream);
-    if (count <= 16) return stream_launch_t<16>(pl, y_bf16, workspace, stream);
-    return stream_launch_t<SHERRY_MAX_BATCH>(pl, y_bf16, workspace, stream);
+    return M == 1 ? stream_launch_mt<1>(pl, count, y_bf16, workspace, stream)
+                  : stream_launch_mt<2>(pl, count, y_bf16, workspace, stream);
 }
 
 int stream_status_take() {

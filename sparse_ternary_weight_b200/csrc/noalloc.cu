@@ -20,7 +20,7 @@
 
 namespace sherry {
 
-constexpr size_t kNoallocBytes = SHERRY_NOALLOC_SCRATCH_BYTES;  // 256 KiB of tickets + partial sums
+constexpr size_t kNoallocBytes = SHERRY_NOALLOC_SCRATCH_BYTES;  // 256 KiB of tickets, then partial sums
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocBytes];
 
 // Device address of the array for the current device, looked up once per device

@@ -170,3 +170,18 @@ def test_unpack_batched_validation(L):
     assert L.sherry_unpack_batched(d, 2, None) == _abi.ERR_NULL
     d[1].W_out = FAKE + 8
     assert L.sherry_unpack_batched(d, 2, None) == _abi.ERR_ALIGN
+
+
+def test_header_constants_match_binding():
+    """Every numeric #define of include/sherry.h equals its mirror in the ctypes binding."""
+    import os
+    import re
+    text = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "sherry.h")).read()
+    defines = {}
+    for name, expr in re.findall(r"^#define SHERRY_(\w+)\s+([^/\n]+)", text, flags=re.M):
+        expr = expr.strip().replace("(size_t)", "")
+        if re.fullmatch(r"[\d\s()<]+", expr):
+            defines[name] = eval(expr)  # integers and shifts only
+    assert {"OK", "MAX_K", "MAX_BATCH", "NOALLOC_SCRATCH_BYTES", "PER_GROUP", "BF16", "OP_UNPACK"} <= set(defines)
+    for name, value in defines.items():
+        assert getattr(_abi, name) == value, name

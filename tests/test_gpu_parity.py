@@ -129,7 +129,11 @@ LIN_CASES = [
     (1, 200, 1024, "group", 256),
     (1, 130, 512, "group", 256),    # one-token kernel, one 512-weight unit, two groups of 256
     (1, 64, 2048, "group", 32),
-    (2, 129, 512, "group", 128),
+    (2, 129, 512, "group", 128),    # two tokens: streaming kernel from here on
+    (2, 300, 3072, "group", 128),
+    (2, 513, 1024, "channel", 0),
+    (2, 77, 1536, "group", 256),
+    (2, 1000, 8192, "tensor", 0),
     (3, 64, 3072, "channel", 0),
     (4, 500, 1024, "group", 128),
     (5, 33, 256, "tensor", 0),
@@ -228,16 +232,18 @@ STREAM_SHAPES = [(1024, 3072, "group", 128), (300, 3072, "channel", 0), (3072, 8
                  (1, 512, "group", 128), (257, 3072, "group", 256), (96, 1536, "group", 256)]
 
 
-def test_stream_batch_many_problems_vs_oracle(sw, orc):
-    """One-token batch of many eligible linears (the streaming kernel: units split
-    evenly over CTAs, tiles straddling two CTAs finished through the ticket)."""
+@pytest.mark.parametrize("M", [1, 2])
+def test_stream_batch_many_problems_vs_oracle(sw, orc, M):
+    """One- and two-token batches of many eligible linears (the streaming kernel:
+    units split evenly over CTAs, tiles straddling two CTAs finished through the
+    ticket)."""
     import torch
     pairs, refs = [], []
     for i in range(24):
         N, K, gname, group = STREAM_SHAPES[i % len(STREAM_SHAPES)]
         gran = GRAN[gname]
         W = _weights("t4" if i % 2 else "normal", N, K, seed=5000 + i)
-        Xb = synth.activations_bf16(1, K, seed=6000 + i)
+        Xb = synth.activations_bf16(M, K, seed=6000 + i + 100 * M)
         P = sw.quantize_pack(to_dev(W), gran, group)
         idx, sgn, sc = packed_to_host(P)
         refs.append((orc.linear(Xb, idx, sgn, sc, N, K, gran, group), orc.unpack_f32(idx, sgn, sc, N, K, gran, group),
@@ -436,6 +442,7 @@ def test_unpack_batched_matches_single_and_oracle(sw, orc):
 MAXK_CASES = [
     # (M, N, gran, group) at K = SHERRY_MAX_K: one case per linear kernel route
     (1, 5, "group", 128),   # one-token streaming kernel
+    (2, 5, "group", 128),   # two-token streaming kernel
     (1, 3, "group", 32),    # general lookup-table kernel
     (4, 5, "group", 128),   # warp-MMA kernel
     (16, 3, "channel", 0),  # tcgen05 few-token kernel

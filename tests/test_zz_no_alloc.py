@@ -13,11 +13,12 @@ from sparse_ternary_weight_b200 import _abi
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    # (M, N, K, granularity, group): the one-token streaming kernel with tiles
-    # split over CTAs, the same over a wide linear, the general kernel with
-    # split K, and the tensor-core kernel (which needs no scratch)
+    # (M, N, K, granularity, group): the streaming kernel (one and two tokens)
+    # with tiles split over CTAs, the same over a wide linear, the general kernel
+    # with split K, and the tensor-core kernel (which needs no scratch)
     (1, 64, 8192, _abi.PER_GROUP, 128),
     (1, 3072, 3072, _abi.PER_GROUP, 128),
+    (2, 3072, 3072, _abi.PER_GROUP, 128),
     (3, 300, 3072, _abi.PER_CHANNEL, 0),
     (16, 64, 2048, _abi.PER_GROUP, 32),
     (40, 200, 1024, _abi.PER_GROUP, 128),
