@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     auto ready = [&](int s) { return bars + 8u * (uint32_t)s; };
     auto empty = [&](int s) { return bars + 32u + 8u * (uint32_t)s; };
     const uint32_t bar_part = bars + 64u;  // every consumer stored its split-tile partial
-    const uint32_t bar_last = bars + 72u;  // the ticket's verdict is in s_last
+    const uint32_t bar_last = bars + 72u;  // the ticket's outcome is in s_last
 
     const int t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5;
