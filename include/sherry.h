@@ -182,7 +182,8 @@ size_t sherry_linear_batched_workspace_bytes(const sherry_linear_desc* descs, in
  * what the previous call left; all calls share the one array, so calls that
  * overlap on the GPU (other streams, other host threads) race -- keep them
  * ordered.  Nothing is allocated or freed. */
-#define SHERRY_NOALLOC_SCRATCH_BYTES ((size_t)2 << 20)  /* enough for every kernel on up to 224 SMs */
+#define SHERRY_NOALLOC_SCRATCH_BYTES ((size_t)2 << 20)  /* one problem's largest plan on up to 224 SMs
+                                                           (checked at compile time for each plan) */
 int sherry_linear_noalloc(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                           const uint32_t* idx, const uint8_t* sgn, const float* scales,
                           int granularity, int group, void* Y, int y_dtype, void* stream);
@@ -219,8 +220,20 @@ int sherry_last_cuda_error(void);
 /* Synchronises `stream`, then returns SHERRY_ERR_TIMEOUT if a bounded device
  * wait of a tensor-core kernel or of the streaming decode kernel gave up since
  * the previous query (its outputs are then invalid), else SHERRY_OK; clears the
- * flag.  SHERRY_ERR_CUDA if the synchronisation fails. */
+ * flag.  SHERRY_ERR_CUDA if the synchronisation fails.  After SHERRY_ERR_TIMEOUT
+ * the split-K tickets of the linear workspace used by the failed call may be
+ * left nonzero: zero its first 256 KiB (or take a fresh zeroed workspace)
+ * before the next linear call with it. */
 int sherry_device_status(void* stream);
+/* Budget, in SM clock cycles, of every bounded wait of the streaming decode
+ * kernel (one or two tokens), for launches made after this call; cycles <= 0
+ * restores the default (4e9, about 2 s at the boost clock).  Returns the previous
+ * budget.  Meant for exercising the failure path: with a budget of a few cycles
+ * the waits give up, the call's outputs are invalid, and sherry_device_status
+ * reports SHERRY_ERR_TIMEOUT.  That kernel holds no tensor memory and issues
+ * only cp.async copies, which it completes before exiting, so the context stays
+ * usable.  The tensor-core kernels keep the default budget. */
+int64_t sherry_set_wait_budget(int64_t cycles);
 /* library version, e.g. 0x000100 = 0.1.0 */
 int sherry_version(void);
 

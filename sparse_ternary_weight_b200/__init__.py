@@ -77,6 +77,20 @@ def workspace(nbytes: int, device, kind: str = "linear") -> "object":
     return buf
 
 
+def device_status(device=None) -> int:
+    """Synchronise the current stream of ``device`` and return the library's
+    device status (0, or ERR_TIMEOUT when a bounded wait of a kernel gave up
+    since the last query).  After a timeout the cached linear workspace of that
+    device may hold nonzero split-K tickets, so it is dropped here and the next
+    linear call gets a fresh zeroed one."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = lib().sherry_device_status(_stream(dev))
+    if st:
+        _ws_cache.pop((str(dev), "linear"), None)
+    return st
+
+
 def quantize_pack(W, granularity="per_group", group: int = 128, out: PackedWeight | None = None) -> PackedWeight:
     """Greedy Sparse-AbsMean 3:4 quantise + 5-bit pack of W [N,K] (fp32 or bf16)."""
     import torch

@@ -130,6 +130,8 @@ int sherry_last_cuda_error(void) { return g_last_cuda_error; }
 
 int sherry_device_status(void* stream) { return device_status_take(static_cast<cudaStream_t>(stream)); }
 
+int64_t sherry_set_wait_budget(int64_t cycles) { return (int64_t)stream_set_wait_cycles((long long)cycles); }
+
 const char* sherry_status_string(int status) {
     switch (status) {
         case SHERRY_OK: return "ok";

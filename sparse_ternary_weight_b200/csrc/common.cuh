@@ -4,6 +4,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <vector>
+
 #include "sherry.h"
 
 namespace sherry {
@@ -23,6 +26,33 @@ void set_cuda_error(cudaError_t e);
     } while (0)
 
 #define SHERRY_LAUNCH_CHECK() SHERRY_CUDA_CHECK(cudaGetLastError())
+
+// One value per device, computed on first use with that device current.  Kernel
+// attributes (the opt-in to more than 48 KB of dynamic shared memory), occupancies
+// and device properties belong to a device: a process-wide flag would skip them
+// on the second GPU a process uses.
+struct PerDevice {
+    std::mutex mu;
+    std::vector<int> val;  // 0 = not computed yet
+};
+
+// *out = pd's value for the current device; `init(int& v)` computes it the first
+// time (returns a status; v must be nonzero on success).
+template <class F>
+inline int per_device(PerDevice& pd, int* out, F&& init) {
+    int dev = 0;
+    SHERRY_CUDA_CHECK(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lk(pd.mu);
+    if ((int)pd.val.size() <= dev) pd.val.resize(dev + 1, 0);
+    if (pd.val[dev] == 0) {
+        int v = 0;
+        const int st = init(v);
+        if (st) return st;
+        pd.val[dev] = v;
+    }
+    *out = pd.val[dev];
+    return SHERRY_OK;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -127,6 +157,7 @@ int skinny_linear_launch(const ProbShape* shapes, const sherry_linear_desc* desc
 bool stream_eligible(const ProbShape& s, int64_t M);
 int64_t stream_tiles(const ProbShape& s);  // row blocks (tickets) of one problem
 int stream_status_take();                   // SHERRY_ERR_TIMEOUT if a bounded wait gave up since the last call
+long long stream_set_wait_cycles(long long cycles);  // returns the previous budget; <= 0 restores the default
 size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms);
 int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream);

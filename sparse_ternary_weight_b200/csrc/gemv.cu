@@ -262,6 +262,13 @@ struct DevInfo {
 
 static int tokens_per_pass(int64_t M) { return M <= 1 ? 1 : (M <= 2 ? 2 : 4); }
 
+// make_plan splits K only with 64-row tiles (WR = 2: 256-row tiles already give
+// at least the target of 2 CTAs per SM), and then gives one problem fewer than
+// twice the target tiles of at most 4 tokens: the no-workspace entry point's
+// fixed scratch holds that on up to 224 SMs.
+static_assert(kTicketBytes + (size_t)2 * (2 * 224) * 4 * 64 * sizeof(float) <= SHERRY_NOALLOC_SCRATCH_BYTES,
+              "no-workspace scratch too small for the general lookup-table plan");
+
 struct Plan {
     int MT, WR;
     std::vector<LinProb> probs;
@@ -368,12 +375,15 @@ static int launch_plan_t(const Plan& pl, int64_t M, int y_bf16, int sms, cudaStr
     P.total_tiles = pl.total_tiles;
     for (int i = 0; i < P.count; ++i) P.p[i] = pl.probs[i];
     auto kern = k_lut_linear<MT, WR, MAXP>;
-    static int occ = -1;
-    if (occ < 0) {
+    static PerDevice occ_dev;
+    int occ = 0;
+    const int st = per_device(occ_dev, &occ, [&](int& v) {
         SHERRY_CUDA_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem));
-        SHERRY_CUDA_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kLThreads, kLutSmem));
-        if (occ < 1) occ = 1;
-    }
+        SHERRY_CUDA_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kern, kLThreads, kLutSmem));
+        if (v < 1) v = 1;
+        return SHERRY_OK;
+    });
+    if (st) return st;
     const int grid = std::min(pl.total_tiles, occ * sms);
     kern<<<grid, kLThreads, kLutSmem, stream>>>(P);
     SHERRY_LAUNCH_CHECK();

@@ -30,6 +30,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -58,7 +59,11 @@ struct SCfg {
 };
 static_assert(SCfg<1>::kSmem <= 232448 && SCfg<2>::kSmem <= 232448, "shared memory per CTA");
 static_assert(kSTabs == 32 * kSHelpers, "one table per helper thread");
-constexpr long long kSWaitCycles = 4000000000LL;   // ~2 s at the boost clock
+constexpr long long kSWaitCycles = 4000000000LL;   // default wait budget, ~2 s at the boost clock
+// The no-workspace entry point's fixed scratch holds this kernel's largest plan
+// (two tokens, one CTA per SM, two partial slots per CTA) on up to 224 SMs.
+static_assert(kTicketBytes + (size_t)224 * 2 * 2 * kSRows * sizeof(float) <= SHERRY_NOALLOC_SCRATCH_BYTES,
+              "no-workspace scratch too small for the streaming plan");
 
 enum SMode { kSRow = 0, kSG128 = 1, kSG256 = 2 };
 
@@ -76,6 +81,7 @@ struct SProb {
 
 template <int MAXP>
 struct SParams {
+    long long wait_cycles;  // budget of every bounded wait, in SM clock cycles
     int count, y_bf16, total_units, upc;
     float* part;  // [grid][2][MT][kSRows] split-tile partials
     int* ticket;  // [total tiles]
@@ -114,15 +120,15 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// wait for the phase with the given parity to complete; false on timeout or
-// when another thread of the CTA has given up
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// wait for the phase with the given parity to complete; false on timeout (after
+// `budget` cycles) or when another thread of the CTA has given up
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, long long budget) {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kSWaitCycles) {
+        if (clock64() - t0 > budget) {
             *abort_flag = 1;
             atomicExch(&g_stream_status, SHERRY_ERR_TIMEOUT);
             return false;
@@ -354,7 +360,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                           cu.sub * kSTabs + ht);
         for (int j = 0; j < nu; ++j) {
             const int s = j % S;
-            if (j >= S && !mbar_wait(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag)) break;
+            if (j >= S && !mbar_wait(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag, P.wait_cycles)) break;
             const SProb& pr = P.p[cu.p];
             copy_unit(pr, cr, cu.sub, stages + s * kSStage, h, lane);
             cp_async_arrive(ready(s));
@@ -386,7 +392,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     int events = 0;  // split tiles handled so far (phase of bar_part / bar_last)
     for (int k = 0; k < nu; ++k) {
         const int s = k % S;
-        if (!mbar_wait(ready(s), (uint32_t)((k / S) & 1), abort_flag)) break;
+        if (!mbar_wait(ready(s), (uint32_t)((k / S) & 1), abort_flag, P.wait_cycles)) break;
         const SProb& pr = P.p[cur.p];
         const uint32_t st = stages + s * kSStage;
         const uint32_t lut = luts + s * C::kLutStage;
@@ -434,11 +440,11 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                 const uint32_t ph = (uint32_t)(events & 1);
                 ++events;
                 if (r == 0) {
-                    if (!mbar_wait(bar_part, ph, abort_flag)) break;
+                    if (!mbar_wait(bar_part, ph, abort_flag, P.wait_cycles)) break;
                     s_last = (atomicAdd(P.ticket + tile, 1) == c_b - c_a);
                     mbar_arrive(bar_last);
                 }
-                if (!mbar_wait(bar_last, ph, abort_flag)) break;
+                if (!mbar_wait(bar_last, ph, abort_flag, P.wait_cycles)) break;
                 if (s_last) {
                     __threadfence();
 #pragma unroll
@@ -480,6 +486,13 @@ bool stream_eligible(const ProbShape& s, int64_t M) {
 }
 
 int64_t stream_tiles(const ProbShape& s) { return (s.N + kSRows - 1) / kSRows; }
+
+// wait budget of the launches (sherry_set_wait_budget)
+static std::atomic<long long> g_stream_wait{kSWaitCycles};
+
+long long stream_set_wait_cycles(long long cycles) {
+    return g_stream_wait.exchange(cycles > 0 ? cycles : kSWaitCycles);
+}
 
 struct SPlan {
     std::vector<SProb> probs;
@@ -526,8 +539,9 @@ template <int MAXP, int MT>
 static int stream_launch_t(SPlan& pl, int y_bf16, void* workspace, cudaStream_t stream) {
     static SParams<MAXP> P;
     static std::mutex mu;
-    static bool attr = false;
+    static PerDevice attr;
     std::lock_guard<std::mutex> lk(mu);
+    P.wait_cycles = g_stream_wait.load();
     P.count = (int)pl.probs.size();
     P.y_bf16 = y_bf16;
     P.total_units = pl.total_units;
@@ -535,11 +549,14 @@ static int stream_launch_t(SPlan& pl, int y_bf16, void* workspace, cudaStream_t 
     P.ticket = static_cast<int*>(workspace);
     P.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.part_off);
     for (int i = 0; i < P.count; ++i) P.p[i] = pl.probs[i];
-    if (!attr) {
+    int done = 0;
+    const int st = per_device(attr, &done, [](int& v) {
         SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_lut_stream<MAXP, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                SCfg<MT>::kSmem));
-        attr = true;
-    }
+        v = 1;
+        return SHERRY_OK;
+    });
+    if (st) return st;
     k_lut_stream<MAXP, MT><<<pl.grid, kSThreads, SCfg<MT>::kSmem, stream>>>(P);
     SHERRY_LAUNCH_CHECK();
     return SHERRY_OK;

@@ -112,6 +112,17 @@ __device__ __forceinline__ bool t_mbar_wait(uint32_t bar, uint32_t parity, volat
         }
     }
 }
+// Bounded wait used on the way out (normal finish or abort): it ignores the
+// abort flag so that the MMAs this CTA committed complete before TMEM is freed.
+__device__ __forceinline__ void t_mbar_drain(uint32_t bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!t_mbar_try(bar, parity)) {
+        if (clock64() - t0 > kTWaitCycles) {
+            atomicExch(&g_skinny_status, SHERRY_ERR_TIMEOUT);
+            return;
+        }
+    }
+}
 __device__ __forceinline__ void t_cp16(uint32_t dst, const void* src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
                  : "memory");
@@ -195,7 +206,7 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
     constexpr int kAPar = kAPar0 < kTAParMax ? kAPar0 : kTAParMax;
     static_assert(BN % 16 == 0 && kAPar >= 2, "TMEM plan");
     extern __shared__ __align__(1024) unsigned char tsm[];
-    __shared__ uint64_t bars[2 * kTChunks + kTAParMax + 2 * kTAcc];
+    __shared__ uint64_t bars[2 * kTChunks + kTAParMax + 2 * kTAcc + 1];
     __shared__ uint32_t tmem_s;
     __shared__ volatile int abort_s;
 
@@ -211,6 +222,7 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
     auto full_a = [&](int h) { return bar0 + 8u * (2 * kTChunks + h); };  // A buffer h of every group written
     auto acc_full = [&](int b) { return bar0 + 8u * (2 * kTChunks + kTAParMax + b); };
     auto acc_empty = [&](int b) { return bar0 + 8u * (2 * kTChunks + kTAParMax + kTAcc + b); };
+    const uint32_t drain = bar0 + 8u * (2 * kTChunks + kTAParMax + 2 * kTAcc);  // MMA threads' last commits
     const int M = P.M;
 
     if (threadIdx.x == 0) {
@@ -225,6 +237,7 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
             t_mbar_init(acc_full(b), kTMmaWarps);
             t_mbar_init(acc_empty(b), 128);
         }
+        t_mbar_init(drain, kTMmaWarps);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (threadIdx.x < 32) {
@@ -410,6 +423,10 @@ __global__ void __launch_bounds__(kTThreads, 1) k_skinny(const __grid_constant__
                 }
             }
             (void)cph;
+            // the MMAs of both issuers complete before TMEM is freed (after an abort
+            // no epilogue has waited for them)
+            t_commit(drain);
+            t_mbar_drain(drain, 0u);
         }
         __syncwarp();
     } else {
@@ -509,7 +526,7 @@ static int skinny_launch_t(const ProbShape* shapes, const sherry_linear_desc* de
                            int y_bf16, int sms, cudaStream_t stream) {
     static TParams<MAXP> P;
     static std::mutex mu;
-    static bool attr = false;
+    static PerDevice attr;
     std::lock_guard<std::mutex> lk(mu);
     P.count = count;
     P.M = (int)M;
@@ -537,10 +554,13 @@ static int skinny_launch_t(const ProbShape* shapes, const sherry_linear_desc* de
     P.total_units = ub;
     if (ub == 0) return SHERRY_OK;
     constexpr int smem = skinny_smem<BN>();
-    if (!attr) {
+    int done = 0;
+    const int st = per_device(attr, &done, [](int& v) {
         SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_skinny<BN, MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-        attr = true;
-    }
+        v = 1;
+        return SHERRY_OK;
+    });
+    if (st) return st;
     const int grid = ub < sms ? ub : sms;
     k_skinny<BN, MAXP><<<grid, kTThreads, smem, stream>>>(P);
     SHERRY_LAUNCH_CHECK();

@@ -112,6 +112,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         }
     }
 }
+// Bounded wait used on the way out of the kernel, after a normal finish or an
+// abort: it ignores the abort flag, so that the CTA's own asynchronous work (its
+// committed MMAs, its TMA loads in flight) lands before TMEM is freed and the
+// CTA's shared memory is released.  On timeout it records the error and returns.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try(bar, parity)) {
+        if (clock64() - t0 > kPWaitCycles) {
+            atomicExch(&g_device_status, SHERRY_ERR_TIMEOUT);
+            return;
+        }
+    }
+}
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -192,7 +205,7 @@ __global__ void __launch_bounds__(PRoles<EPI>::kThreads, 1)
 k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PParams P) {
     constexpr int kPTmaWarp = PRoles<EPI>::kTmaWarp, kPMmaWarp = PRoles<EPI>::kMmaWarp;
     extern __shared__ __align__(1024) unsigned char psmem[];
-    __shared__ uint64_t bars[2 * kPXSlots + 2 + 2 * kPAcc];
+    __shared__ uint64_t bars[2 * kPXSlots + 2 + 2 * kPAcc + 1];
     __shared__ uint32_t tmem_base_s;
     __shared__ volatile int abort_s;
 
@@ -206,6 +219,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
     auto full_a = [&](int h) { return bar0 + 8u * (2 * kPXSlots + h); };   // A buffer h written
     auto acc_full = [&](int b) { return bar0 + 8u * (2 * kPXSlots + 2 + b); };
     auto acc_empty = [&](int b) { return bar0 + 8u * (2 * kPXSlots + 2 + kPAcc + b); };
+    const uint32_t drain = bar0 + 8u * (2 * kPXSlots + 2 + 2 * kPAcc);  // the MMA thread's last commit
 
     // persistent: tile t = (weight-row tile t % ntn, token tile t / ntn), strided by the grid;
     // chunk and accumulator phases run on across tiles
@@ -227,6 +241,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
             mbar_init(acc_full(b), 1);
             mbar_init(acc_empty(b), 32 * EPI);
         }
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
     if (threadIdx.x < 32) {
@@ -386,6 +401,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
         if (lane == 0) {
             int c = 0;
             uint32_t cph = 0;  // phase parity of slot c's use
+            int issued[kPXSlots] = {};  // chunks loaded into each slot (phases of full_x)
             bool ok = true;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const int m0 = (t / ntn) * kPBN;
@@ -399,9 +415,14 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
                     for (int st = 0; st < steps; ++st)
                         tma_load_2d(stX + c * kPChunkB + st * kPStepB, &xmap, (ch * kPChunkSteps + st) * kPBK, m0,
                                     full_x(c));
+                    ++issued[c];
                     if (++c == kPXSlots) { c = 0; cph ^= 1u; }
                 }
             }
+            // every load issued must land before the CTA's shared memory goes away
+            // (after an abort the MMA thread may not have waited for the last ones)
+            for (int s = 0; s < kPXSlots; ++s)
+                if (issued[s] > 0) mbar_drain(full_x(s), (uint32_t)((issued[s] - 1) & 1));
         }
     } else {
         // ---------------- MMA issuer ----------------
@@ -460,6 +481,10 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
                     if (++c == kPXSlots) { c = 0; cph ^= 1u; }
                 }
             }
+            // all MMAs this thread issued complete before TMEM is freed (after an abort
+            // no epilogue has waited for them)
+            mma_commit(drain);
+            mbar_drain(drain, 0u);
         }
         __syncwarp();
     }
@@ -525,23 +550,20 @@ int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, i
     P.per_tensor = s.granularity == SHERRY_PER_TENSOR;
     P.spr = s.granularity == SHERRY_PER_GROUP ? (int)(s.K / s.group) : 1;
     P.group_steps = s.granularity == SHERRY_PER_GROUP ? s.group / kPBK : (int)(s.K / kPBK);
-    static bool attr = false;
-    static std::mutex mu;
-    {
-        std::lock_guard<std::mutex> lk(mu);
-        if (!attr) {
-            SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
-            SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
-            attr = true;
-        }
-    }
-    const int64_t tiles = ((s.N + kPBM - 1) / kPBM) * ((M + kPBN - 1) / kPBN);
-    static int sms = 0;
-    if (sms == 0) {
+    // per device: the shared-memory opt-in of both instantiations, and the SM count
+    static PerDevice dev_sms;
+    int sms = 0;
+    const int st = per_device(dev_sms, &sms, [](int& v) {
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
         int dev = 0;
         SHERRY_CUDA_CHECK(cudaGetDevice(&dev));
-        SHERRY_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-    }
+        SHERRY_CUDA_CHECK(cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev));
+        if (v < 1) v = 1;
+        return SHERRY_OK;
+    });
+    if (st) return st;
+    const int64_t tiles = ((s.N + kPBM - 1) / kPBM) * ((M + kPBN - 1) / kPBN);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
     // 16 epilogue warps (32 token columns each) drain a group accumulator faster; measured on the
     // 3B shapes that pays for group scales up to K = 4096 (+6%) and costs at K = 8192 (-15%) and
