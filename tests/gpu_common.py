@@ -47,3 +47,25 @@ def check_linear(y, y_ref, Xb, Wq, y_is_bf16=False):
     err = np.abs(np.asarray(y, np.float64) - y_ref)
     assert np.all(err <= bound), (err / bound).max()
     return g
+
+
+CANARY_BYTE = 0xA5
+CANARY_PAD = 256   # guard bytes before and after an output (keeps the view 256-byte aligned)
+
+
+def canaried(shape, dtype):
+    """A device output buffer guarded by CANARY_PAD bytes of a fixed pattern on
+    each side: returns (whole allocation, the output view of `shape`)."""
+    import torch
+    n = int(np.prod(shape)) if len(shape) else 1
+    item = torch.empty((), dtype=dtype).element_size()
+    pad = CANARY_PAD // item
+    full = torch.empty(n + 2 * pad, dtype=dtype, device="cuda")
+    full.view(torch.uint8).fill_(CANARY_BYTE)
+    return full, full[pad:pad + n].view(*shape)
+
+
+def canaries_intact(full) -> bool:
+    """True if no byte of either guard region of a `canaried` buffer changed."""
+    b = full.view(__import__("torch").uint8)
+    return bool((b[:CANARY_PAD] == CANARY_BYTE).all()) and bool((b[-CANARY_PAD:] == CANARY_BYTE).all())
