@@ -549,13 +549,31 @@ def prefill_rows(args, pairs, ws, dev, pk, steps, warm):
 # CPU oracle: the reference arm (the plain CPU implementation, timed on the host cores)
 
 
-def cpu_baseline(layers, min_seconds=10.0):
-    """Oracle linear (fp64 accumulation, OpenMP over rows) on the first `layers`
-    layers of the 3B stack at M = 1, repeated until at least `min_seconds` of
-    CPU work: returns the same metric on the host."""
+def cpu_model():
+    """the host CPU's model name from /proc/cpuinfo (None if unreadable)"""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def cpu_baseline(layers, min_seconds=8.0, one_core_seconds=4.0, prefill_tokens=4):
+    """The oracle (C, fp64 accumulation) on the host cores, three legs:
+    * all cores (OpenMP over rows): the linear on the first `layers` layers of the
+      3B stack at M = 1, repeated until at least `min_seconds` -> the same metric
+      as the headline (GB/s of algorithmic bytes);
+    * one core (the plain single-threaded build) on the same linears, at least
+      `one_core_seconds`;
+    * prefill (config 4): the same linears at `prefill_tokens` token rows, all
+      cores; the time per token is extrapolated to M = 512, 2048, 4096 over the
+      whole stack and labelled as such."""
     import oracle
     from sparse_ternary_weight_b200 import synth
     orc = oracle.oracle(omp=True)
+    one = oracle.oracle(omp=False)
     cfg, _, shp = synth.STACKS[STACK]
     work = []
     for l in range(layers):
@@ -568,18 +586,51 @@ def cpu_baseline(layers, min_seconds=10.0):
             del W
     shapes = [(N, K) for (_, _, _, _, N, K) in work]
     b1 = stack_bytes(shapes, 1)
-    reps, t = 0, 0.0
-    t0 = time.perf_counter()
-    while t < min_seconds:
-        for (X, idx, sgn, sc, N, K) in work:
+    full_shapes = [s for (_, _, s) in stack_shapes()]
+
+    def timed(o, limit):
+        reps, t, t0 = 0, 0.0, time.perf_counter()
+        while t < limit:
+            for (X, idx, sgn, sc, N, K) in work:
+                o.linear(X, idx, sgn, sc, N, K, oracle.PER_GROUP, 128)
+            reps += 1
+            t = time.perf_counter() - t0
+        return reps, t
+
+    reps, t = timed(orc, min_seconds)
+    reps1, t1 = timed(one, one_core_seconds)
+    # prefill leg, all cores: the oracle's time per linear is a decode pass over the
+    # weights plus one multiply-add pass per token row, so it is measured at two
+    # token counts and fitted as a + b * tokens before extrapolating
+    def prefill_time(T):
+        Xp = [synth.activations_bf16(T, K, 700000 + K) for (_, _, _, _, _, K) in work]
+        t0 = time.perf_counter()
+        for (_, idx, sgn, sc, N, K), X in zip(work, Xp):
             orc.linear(X, idx, sgn, sc, N, K, oracle.PER_GROUP, 128)
-        reps += 1
-        t = time.perf_counter() - t0
-    b = b1 * reps
-    return {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": orc.threads(), "kind": "oracle",
+        return time.perf_counter() - t0
+    T0, T1 = 2, 2 + 2 * prefill_tokens
+    ta, tb = prefill_time(T0), prefill_time(T1)
+    per_tok = max((tb - ta) / (T1 - T0), 1e-9)
+    fixed = max(ta - T0 * per_tok, 0.0)
+    w_sample = sum(N * K for (N, K) in shapes)
+    w_full = sum(N * K for (N, K) in full_shapes)
+    prefill = {}
+    for M in (512, 2048, 4096):
+        sec = (fixed + M * per_tok) * w_full / w_sample
+        prefill[f"M{M}"] = {"seconds_per_step_extrapolated": round(sec, 1),
+                            "TFLOP/s_dense_equiv_extrapolated": round(2.0 * M * w_full / sec / 1e12, 6)}
+    prefill["sample"] = (f"the first {layers} layer(s) ({len(work)} linears, group 128) at {T0} and {T1} token rows, "
+                         f"{ta:.2f} s and {tb:.2f} s on all cores; fitted as decode {fixed:.3f} s + {per_tok:.4f} s "
+                         "per token and scaled by weights to the whole 28-layer stack (extrapolated)")
+    return {"value": round(b1 * reps / t / 1e9, 4), "unit": "GB/s", "cores": orc.threads(), "kind": "oracle",
+            "cpu_model": cpu_model(),
             "sample": f"first {layers} layer(s) of the 3B stack ({len(work)} linears, M=1, group 128) x {reps} "
-                      f"passes: {b} algorithmic bytes in {t:.2f} s; C oracle, fp64 accumulation, OpenMP over rows",
-            "tok_per_s_equiv": round(b / t / stack_bytes([s for (_, _, s) in stack_shapes()], 1), 4)}
+                      f"passes: {b1 * reps} algorithmic bytes in {t:.2f} s; C oracle, fp64 accumulation, OpenMP "
+                      "over rows",
+            "tok_per_s_equiv": round(b1 * reps / t / stack_bytes(full_shapes, 1), 4),
+            "one_core": {"value": round(b1 * reps1 / t1 / 1e9, 4), "unit": "GB/s", "cores": one.threads(),
+                         "sample": f"the same linears x {reps1} passes in {t1:.2f} s, single-threaded build"},
+            "prefill_extrapolated": prefill}
 
 
 def run_reference(args):
@@ -695,6 +746,7 @@ def main():
     ap.add_argument("--quick", action="store_true", help="headline only, skip the other rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-layers", type=int, default=1)
+    ap.add_argument("--cpu-only", action="store_true", help="only run the CPU oracle baseline and print it")
     ap.add_argument("--layers", type=int, default=28, help="layers of the 3B stack (28 = the full workload; "
                     "fewer only for profiling captures)")
     ap.add_argument("--profile-quantize", default=None, metavar="N,K,GRAN",
@@ -715,6 +767,9 @@ def main():
         return
     if args.profile_quantize:
         profile_quantize(args)
+        return
+    if args.cpu_only:
+        print(json.dumps(cpu_baseline(max(1, args.cpu_layers))), flush=True)
         return
     if args.warmup < 3:
         args.warmup = 3
