@@ -68,6 +68,8 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
         f.restype = i32
     L.sherry_ref_linear.argtypes = [vp, i64, vp, i64, vp, vp, vp, i64, i64, i32, i32, vp]
     L.sherry_ref_linear.restype = i32
+    L.sherry_ref_fake_quant.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp]
+    L.sherry_ref_fake_quant.restype = i32
     L.sherry_ref_threads.argtypes = []
     L.sherry_ref_threads.restype = i32
     return L
@@ -147,6 +149,19 @@ class Oracle:
         if st:
             raise ValueError(f"oracle linear status {st}")
         return Y
+
+    def fake_quant(self, W, gran=PER_GROUP, group=128, w_dtype=None):
+        """The quantiser's forward output: (Wq float32 [N,K], Wq as bf16 bits [N,K])."""
+        W = np.ascontiguousarray(W)
+        if w_dtype is None:
+            w_dtype = BF16 if W.dtype == np.uint16 else F32
+        N, K = W.shape
+        Wq = np.empty((N, K), np.float32)
+        Wb = np.empty((N, K), np.uint16)
+        st = self.L.sherry_ref_fake_quant(_p(W), w_dtype, N, K, gran, group, _p(Wq), _p(Wb))
+        if st:
+            raise ValueError(f"oracle fake_quant status {st}")
+        return Wq, Wb
 
     def threads(self) -> int:
         return int(self.L.sherry_ref_threads())

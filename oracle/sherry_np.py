@@ -127,3 +127,13 @@ def scale_map(N: int, K: int, scales: np.ndarray, gran: int, group: int) -> np.n
     if gran == PER_CHANNEL:
         return np.repeat(scales.reshape(N, 1), K, axis=1).astype(np.float32)
     return np.repeat(scales.reshape(N, K // group), group, axis=1).astype(np.float32)
+
+
+def fake_quant(W: np.ndarray, gran: int = PER_GROUP, group: int = 128) -> np.ndarray:
+    """The quantiser's forward output in the pages' order: sign of the masked
+    weight (kept weights +-1, the zeroed one 0) times the scale of its domain,
+    float32 [N,K] (the zeroed positions are +0.0)."""
+    t, scales, _ = quantize(W, gran, group)
+    N, K = t.shape
+    out = t.astype(np.float32) * scale_map(N, K, scales, gran, group)
+    return np.where(t == 0, np.float32(0.0), out).astype(np.float32)

@@ -202,6 +202,65 @@ int sherry_ref_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K,
     return SHERRY_REF_OK;
 }
 
+/* ---- forward output of the quantiser: mask the smallest |w| of every block,
+ * keep the signs (w >= 0 -> +1), scale = PairSum(masked |w| over the domain)
+ * / max(L * 3/4, 1), output sign * mask * scale.  No packing is involved. ---- */
+int sherry_ref_fake_quant(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
+                          float* Wq, uint16_t* Wb) {
+    int st = check_shape(N, K);
+    if (st) return st;
+    st = check_gran(K, granularity, group);
+    if (st) return st;
+    if (w_dtype != SHERRY_REF_F32 && w_dtype != SHERRY_REF_BF16) return SHERRY_REF_ERR_DTYPE;
+    if (N > 0 && (!W || !Wq)) return SHERRY_REF_ERR_NULL;
+
+    float* mag = (float*)malloc((size_t)(N * K > 0 ? N * K : 1) * sizeof(float));
+    int8_t* sgn = (int8_t*)malloc((size_t)(N * K > 0 ? N * K : 1));
+    if (!mag || !sgn) abort();
+    /* mask and signs, block by block */
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t b = 0; b < K / 4; ++b) {
+            float wv[4];
+            for (int i = 0; i < 4; ++i) {
+                int64_t off = n * K + 4 * b + i;
+                wv[i] = (w_dtype == SHERRY_REF_F32) ? ((const float*)W)[off]
+                                                    : bf16_bits_to_f32(((const uint16_t*)W)[off]);
+            }
+            unsigned nib, g;
+            encode_block(wv, &nib, &g, &mag[n * K + 4 * b]);
+            int z = (int)(nib >> 2);
+            for (int i = 0; i < 4; ++i)
+                sgn[n * K + 4 * b + i] = (int8_t)((i == z) ? 0 : ((wv[i] >= 0.0f) ? 1 : -1));
+        }
+    }
+    /* one scale per domain, then sign * scale */
+    if (granularity == SHERRY_REF_PER_TENSOR) {
+        const int64_t L = N * K;
+        const double kept = 3.0 * (double)L / 4.0; /* D = max(L * 3/4, 1) */
+        float a = sherry_ref_pairsum(mag, L) / (float)(kept < 1.0 ? 1.0 : kept);
+        for (int64_t i = 0; i < N * K; ++i) Wq[i] = (float)sgn[i] * a;
+    } else {
+        const int64_t L = (granularity == SHERRY_REF_PER_CHANNEL) ? K : group;
+        const float D = (float)((double)L / 4.0 * 3.0);
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t j = 0; j < K / L; ++j) {
+                float a = sherry_ref_pairsum(&mag[n * K + j * L], L) / D;
+                for (int64_t k = j * L; k < j * L + L; ++k) Wq[n * K + k] = (float)sgn[n * K + k] * a;
+            }
+    }
+    if (Wb)
+        for (int64_t i = 0; i < N * K; ++i) Wb[i] = f32_to_bf16_rne(Wq[i]);
+    free(mag);
+    free(sgn);
+    return SHERRY_REF_OK;
+}
+
 /* ternary value of weight (n, k) decoded from the planes */
 static int ternary_at(const uint32_t* idx, const uint8_t* sgn, int64_t n, int64_t k, int64_t K) {
     int64_t words = K / 32;

@@ -82,6 +82,15 @@ int sherry_ref_linear(const uint16_t* X, int64_t M, const int64_t* rows, int64_t
                       const uint32_t* idx, const uint8_t* sgn, const float* scales,
                       int64_t N, int64_t K, int granularity, int group, double* Y);
 
+/* The quantiser's forward output ("Sherry, Tequila and Fairies in Python",
+ * section 1.1, SherryNMQuant.forward): the masked weight's signs times the
+ * scale of their domain, computed directly from W (block argmin -> mask, signs,
+ * pairwise sums of the kept |w|, one division) without packing.  Wq fp32
+ * [N][K] (zeroed positions +0.0); Wb (optional, may be NULL) receives
+ * round-to-nearest-even bf16 bits of Wq. */
+int sherry_ref_fake_quant(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
+                          float* Wq, uint16_t* Wb);
+
 /* number of threads the build uses (1 unless built with OpenMP) */
 int sherry_ref_threads(void);
 

@@ -380,6 +380,58 @@ def pin_topk_reading(orc: oracle.Oracle):
         assert np.all(np.abs(Wq - deq) <= bound * np.abs(deq) + 1e-30), gran
 
 
-ALL_PINS = [pin_topk_reading, pin_code_bijection, pin_argmin_bruteforce, pin_hand_worked, pin_sparsity,
+# ---------------------------------------------------------------- forward output (fake quantisation)
+
+def pin_fake_quant(orc: oracle.Oracle):
+    """The quantiser's forward output W_q ("Sherry, Tequila and Fairies in
+    Python" section 1.1: sign of the masked weight times the domain's scale):
+    * the pages' torch formulation on continuous inputs: same zero pattern and
+      signs, values within the summation-order bound;
+    * |w| = 2^e everywhere: W_q = t * 2^e exactly, t from a stable sort by |w|;
+    * exactly one +0.0 per block; kept entries carry sign(w) and one magnitude
+      per scale domain;
+    * the bf16 output is torch's round-to-nearest-even cast of the fp32 one;
+    * the C oracle equals the NumPy restatement and the pack -> unpack
+      round trip, bit for bit."""
+    import torch
+    N, K = 24, 384
+    W = synth.weights_student_t(N, K, seed=801)
+    w = torch.from_numpy(W)
+    blocks = w.reshape(N, K // 4, 4)
+    top3 = torch.topk(blocks.abs(), 3, dim=-1).indices
+    kept = torch.zeros(blocks.shape, dtype=torch.bool).scatter_(-1, top3, True)
+    sparse = torch.where(kept, blocks, torch.zeros(())).reshape(N, K)
+    t_ref = expected_ternary(W)
+    for gran, group, view in ((oracle.PER_GROUP, 128, (N, K // 128, 128)), (oracle.PER_GROUP, 32, (N, K // 32, 32)),
+                              (oracle.PER_CHANNEL, 0, (N, K)), (oracle.PER_TENSOR, 0, (1, N * K))):
+        Wq, Wb = orc.fake_quant(W, gran, group if group else 128)
+        x = sparse.reshape(view)
+        L = x.shape[-1]
+        deq = (torch.sign(x) * (x.abs().sum(-1, keepdim=True) / max(L * 3.0 / 4.0, 1.0))).reshape(N, K).numpy()
+        assert np.array_equal(Wq == 0, deq == 0) and np.array_equal(np.sign(Wq), np.sign(deq))
+        bound = (math.ceil(math.log2(L)) + 2) * 2.0 ** -24
+        assert np.all(np.abs(Wq - deq) <= bound * np.abs(deq) + 1e-30), (gran, group)
+        # one +0.0 per block, kept signs, one magnitude per domain
+        assert np.array_equal(Wq.view(np.uint32) == 0, t_ref == 0)
+        assert np.array_equal(np.sign(Wq).astype(np.int8), t_ref)
+        mags = np.abs(Wq).reshape(view)
+        dom_max = mags.max(axis=-1, keepdims=True)
+        assert np.all((mags == 0) | (mags == dom_max)), (gran, group)
+        ref_b = torch.from_numpy(Wq).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(Wb, ref_b)
+        g = group if group else 128
+        assert np.array_equal(Wq.view(np.uint32), sherry_np.fake_quant(W, gran, g).view(np.uint32))
+        idx, sgn, sc = orc.quantize_pack(W, gran, g)
+        assert np.array_equal(Wq.view(np.uint32), orc.unpack_f32(idx, sgn, sc, N, K, gran, g).view(np.uint32))
+    # powers of two: exact, with ties resolved to the lowest index
+    rng = synth.rng(802)
+    e = rng.integers(-10, 4, size=(N, K // 128))
+    signs = np.where(rng.random((N, K)) < 0.5, -1.0, 1.0).astype(np.float32)
+    W2 = (signs * np.repeat(np.exp2(e), 128, axis=1)).astype(np.float32)
+    Wq, _ = orc.fake_quant(W2, oracle.PER_GROUP, 128)
+    assert np.array_equal(Wq, expected_ternary(W2).astype(np.float32) * np.repeat(np.exp2(e), 128, axis=1))
+
+
+ALL_PINS = [pin_fake_quant, pin_topk_reading, pin_code_bijection, pin_argmin_bruteforce, pin_hand_worked, pin_sparsity,
             pin_scale_power_of_two, pin_scale_closed_form, pin_c_vs_numpy, pin_bf16_input,
             pin_unpack_bf16, pin_linear, pin_errors, pin_pairsum_tree]

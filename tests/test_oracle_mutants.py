@@ -37,6 +37,12 @@ MUTANTS = {
                                 "sgn[n * words + b / 8] |= (uint8_t)(g << (7 - b % 8));"),
     "pad_with_one": ("buf[i] = (i < L) ? v[i] : 0.0f;", "buf[i] = (i < L) ? v[i] : 1.0f;"),
     "group_error_not_checked": ("(group % 32) != 0 || ", ""),
+    "fake_quant_zero_keeps_sign": ("sgn[n * K + 4 * b + i] = (int8_t)((i == z) ? 0 : ((wv[i] >= 0.0f) ? 1 : -1));",
+                                   "sgn[n * K + 4 * b + i] = (int8_t)((wv[i] >= 0.0f) ? 1 : -1);"),
+    "fake_quant_scale_from_next_domain": ("for (int64_t k = j * L; k < j * L + L; ++k) Wq[n * K + k] = (float)sgn[n * K + k] * a;",
+                                          "for (int64_t k = j * L; k < j * L + L; ++k) Wq[n * K + (k + L) % K] = (float)sgn[n * K + (k + L) % K] * a;"),
+    "fake_quant_bf16_truncated": ("if (Wb)\n        for (int64_t i = 0; i < N * K; ++i) Wb[i] = f32_to_bf16_rne(Wq[i]);",
+                                  "if (Wb)\n        for (int64_t i = 0; i < N * K; ++i) Wb[i] = (uint16_t)(f32_to_bf16_rne(Wq[i]) & 0xFFFEu);"),
 }
 
 
