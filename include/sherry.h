@@ -116,6 +116,45 @@ int sherry_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K, int g
                          uint32_t* idx, uint8_t* sgn, float* scales,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- fake quantisation (the quantiser's forward output, for QAT) -----------
+ * "Sherry, Tequila and Fairies in Python", section 1.1 (SherryNMQuant.forward
+ * and SherryLinear): W_q = sign(w) * mask * alpha, i.e. t[n][k] * alpha(n,k),
+ * written together with the packed planes and scales of sherry_quantize_pack
+ * (same arguments, same workspace, bit-identical planes and scales).
+ *   Wq       [N][K] fp32 (wq_dtype SHERRY_F32: t * alpha exactly) or bf16
+ *            (SHERRY_BF16: round to nearest even of t * alpha); fully overwritten
+ * Group and row scales: one pass over W (the row's Wq is written from its packed
+ * words once its scales are known).  Per-tensor: the scale needs the whole
+ * tensor, so Wq is written by a second pass over the packed planes.
+ * The straight-through estimator's backward is the identity (the gradient with
+ * respect to W_q is the gradient with respect to W): it needs no kernel. */
+int sherry_fake_quant(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
+                      void* Wq, int wq_dtype, uint32_t* idx, uint8_t* sgn, float* scales,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* One weight of a batched quantise + pack (all pointers device pointers). */
+typedef struct sherry_quantize_desc {
+    const void* W;          /* [N][K], w_dtype */
+    uint32_t* idx;
+    uint8_t* sgn;
+    float* scales;
+    void* Wq;               /* optional fake-quantised output [N][K] in wq_dtype (NULL: none) */
+    int64_t N, K;
+    int32_t w_dtype, granularity, group, wq_dtype;
+} sherry_quantize_desc;
+
+/* ---- batched quantise + pack ----------------------------------------------
+ * `count` independent weights (count <= SHERRY_MAX_BATCH; any mix of element
+ * types and granularities) in one launch of the quantise kernel, plus one launch
+ * that finalises every per-tensor scale (and, for per-tensor weights with Wq, one
+ * pass that writes Wq).  Each desc's outputs are bit-identical to the single
+ * call's.  `descs` is a HOST array read during the call only.
+ *   workspace  sherry_quantize_pack_batched_workspace_bytes(descs, count) bytes
+ *            (per-tensor weights only; 256-byte aligned) */
+int sherry_quantize_pack_batched(const sherry_quantize_desc* descs, int count,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+size_t sherry_quantize_pack_batched_workspace_bytes(const sherry_quantize_desc* descs, int count);
+
 /* ---- packed linear -------------------------------------------------------
  * Y[m][n] = sum_k X[m][k] * t[n][k] * alpha(n,k)  ("Sherry: ..." digest: Y = X T alpha;
  * inference builds lookup tables from the activations, accumulates, then applies

@@ -108,15 +108,113 @@ def quantize_pack(W, granularity="per_group", group: int = 128, out: PackedWeigh
     if dt is None:
         raise SherryError(_abi.ERR_DTYPE, "quantize_pack")
     if out is None:
-        dev = W.device
-        out = PackedWeight(torch.empty((N, K // 32), dtype=torch.int32, device=dev),
-                           torch.empty((N, K // 32), dtype=torch.uint8, device=dev),
-                           torch.empty((max(ns, 1),), dtype=torch.float32, device=dev), N, K, g, group)
+        out = _new_packed(N, K, g, group, ns, W.device)
     wsb = L.sherry_workspace_bytes(_abi.OP_QUANTIZE_PACK, 0, N, K, g, group)
     ws = workspace(wsb, W.device, "quantize")
     check(L.sherry_quantize_pack(_ptr(W), dt, N, K, g, group, _ptr(out.idx), _ptr(out.sgn), _ptr(out.scales),
                                  _ptr(ws), wsb, _stream(W.device)), "quantize_pack")
     return out
+
+
+def _new_packed(N, K, g, group, ns, dev) -> PackedWeight:
+    import torch
+    return PackedWeight(torch.empty((N, K // 32), dtype=torch.int32, device=dev),
+                        torch.empty((N, K // 32), dtype=torch.uint8, device=dev),
+                        torch.empty((max(ns, 1),), dtype=torch.float32, device=dev), N, K, g, group)
+
+
+def fake_quant(W, granularity="per_group", group: int = 128, out_dtype=None, out=None,
+               packed: PackedWeight | None = None):
+    """The quantiser's forward output W_q = t * alpha [N,K] (fp32 or bf16, default
+    W's dtype) in one pass over W, plus the packed weight.  Returns (W_q, packed)."""
+    import torch
+    _require_cuda(W)
+    if W.dim() != 2:
+        raise ValueError("expects a 2D weight")
+    W = W.contiguous()
+    N, K = W.shape
+    g = _gran(granularity)
+    L = lib()
+    ns = L.sherry_num_scales(N, K, g, group)
+    if ns < 0:
+        raise SherryError(_abi.ERR_SHAPE if K % 32 or K < 32 else _abi.ERR_GROUP, "fake_quant")
+    dt = {torch.float32: F32, torch.bfloat16: BF16}.get(W.dtype)
+    if dt is None:
+        raise SherryError(_abi.ERR_DTYPE, "fake_quant")
+    out_dtype = out_dtype or W.dtype
+    qd = {torch.float32: F32, torch.bfloat16: BF16}[out_dtype]
+    if out is None:
+        out = torch.empty((N, K), dtype=out_dtype, device=W.device)
+    if packed is None:
+        packed = _new_packed(N, K, g, group, ns, W.device)
+    wsb = L.sherry_workspace_bytes(_abi.OP_QUANTIZE_PACK, 0, N, K, g, group)
+    ws = workspace(wsb, W.device, "quantize")
+    check(L.sherry_fake_quant(_ptr(W), dt, N, K, g, group, _ptr(out), qd, _ptr(packed.idx), _ptr(packed.sgn),
+                              _ptr(packed.scales), _ptr(ws), wsb, _stream(W.device)), "fake_quant")
+    return out, packed
+
+
+def _ste_function():
+    import torch
+
+    class SherryFakeQuant(torch.autograd.Function):
+        """Fake quantisation with the straight-through estimator: the forward is
+        :func:`fake_quant` (one kernel), the backward passes the incoming gradient
+        to W unchanged ("Sherry, Tequila and Fairies in Python", section 1.1:
+        SherryNMQuant.backward returns grad_output) -- no kernel and no copy."""
+
+        @staticmethod
+        def forward(ctx, W, granularity, group):
+            return fake_quant(W, granularity, group)[0]
+
+        @staticmethod
+        def backward(ctx, grad):
+            return grad, None, None
+
+    return SherryFakeQuant
+
+
+_STE = None
+
+
+def fake_quant_ste(W, granularity="per_group", group: int = 128):
+    """Differentiable fake quantisation for QAT: W_q from the CUDA kernel, identity gradient."""
+    global _STE
+    if _STE is None:
+        _STE = _ste_function()
+    return _STE.apply(W, granularity, group)
+
+
+def quantize_pack_batched(weights, granularity="per_group", group: int = 128, outs=None, wq_outs=None):
+    """Quantise + pack several weights in one launch (plus one scale-finalise launch
+    when any scale is per-tensor).  ``weights`` is a list of 2D fp32/bf16 tensors;
+    ``wq_outs`` (optional) a list of fake-quantised outputs (or None entries)."""
+    import torch
+    if not weights:
+        return []
+    g = _gran(granularity)
+    L = lib()
+    dev = weights[0].device
+    arr = (_abi.QuantizeDesc * len(weights))()
+    packs = []
+    for i, W in enumerate(weights):
+        _require_cuda(W)
+        if W.dim() != 2 or not W.is_contiguous():
+            raise ValueError("each weight must be a contiguous 2D tensor")
+        N, K = W.shape
+        ns = L.sherry_num_scales(N, K, g, group)
+        if ns < 0:
+            raise SherryError(_abi.ERR_SHAPE if K % 32 or K < 32 else _abi.ERR_GROUP, "quantize_pack_batched")
+        P = outs[i] if outs is not None else _new_packed(N, K, g, group, ns, W.device)
+        packs.append(P)
+        wq = wq_outs[i] if wq_outs is not None else None
+        arr[i] = _abi.QuantizeDesc(_ptr(W), _ptr(P.idx), _ptr(P.sgn), _ptr(P.scales), _ptr(wq), N, K,
+                                   {torch.float32: F32, torch.bfloat16: BF16}[W.dtype], g, group,
+                                   BF16 if (wq is not None and wq.dtype == torch.bfloat16) else F32)
+    wsb = L.sherry_quantize_pack_batched_workspace_bytes(arr, len(weights))
+    ws = workspace(wsb, dev, "quantize")
+    check(L.sherry_quantize_pack_batched(arr, len(weights), _ptr(ws), wsb, _stream(dev)), "quantize_pack_batched")
+    return packs
 
 
 def linear(X, P: PackedWeight, out_dtype=None, out=None):

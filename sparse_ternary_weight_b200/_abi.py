@@ -27,6 +27,13 @@ class LinearDesc(ctypes.Structure):
                 ("N", i64), ("K", i64), ("granularity", ctypes.c_int32), ("group", ctypes.c_int32)]
 
 
+class QuantizeDesc(ctypes.Structure):
+    """Mirror of ``sherry_quantize_desc``."""
+    _fields_ = [("W", vp), ("idx", vp), ("sgn", vp), ("scales", vp), ("Wq", vp), ("N", i64), ("K", i64),
+                ("w_dtype", ctypes.c_int32), ("granularity", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("wq_dtype", ctypes.c_int32)]
+
+
 class UnpackDesc(ctypes.Structure):
     """Mirror of ``sherry_unpack_desc``."""
     _fields_ = [("idx", vp), ("sgn", vp), ("scales", vp), ("N", i64), ("K", i64),
@@ -39,6 +46,9 @@ SIGNATURES = {
     "sherry_num_scales": (i64, [i64, i64, i32, i32]),
     "sherry_workspace_bytes": (sz, [i32, i64, i64, i64, i32, i32]),
     "sherry_quantize_pack": (i32, [vp, i32, i64, i64, i32, i32, vp, vp, vp, vp, sz, vp]),
+    "sherry_fake_quant": (i32, [vp, i32, i64, i64, i32, i32, vp, i32, vp, vp, vp, vp, sz, vp]),
+    "sherry_quantize_pack_batched": (i32, [ctypes.POINTER(QuantizeDesc), i32, vp, sz, vp]),
+    "sherry_quantize_pack_batched_workspace_bytes": (sz, [ctypes.POINTER(QuantizeDesc), i32]),
     "sherry_linear": (i32, [vp, i64, i64, i64, vp, vp, vp, i32, i32, vp, i32, vp, sz, vp]),
     "sherry_linear_batched": (i32, [ctypes.POINTER(LinearDesc), i32, i64, i32, vp, sz, vp]),
     "sherry_linear_batched_workspace_bytes": (sz, [ctypes.POINTER(LinearDesc), i32, i64]),

@@ -177,20 +177,68 @@ size_t sherry_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int granu
     return 0;
 }
 
+static int check_quantize_desc(const sherry_quantize_desc& d) {
+    int st = check_shape(d.N, d.K);
+    if (st) return st;
+    if ((st = check_gran(d.K, d.granularity, d.group))) return st;
+    if (d.w_dtype != SHERRY_F32 && d.w_dtype != SHERRY_BF16) return SHERRY_ERR_DTYPE;
+    if (d.Wq && d.wq_dtype != SHERRY_F32 && d.wq_dtype != SHERRY_BF16) return SHERRY_ERR_DTYPE;
+    if (!d.scales || (d.N > 0 && (!d.W || !d.idx || !d.sgn))) return SHERRY_ERR_NULL;
+    if (!aligned(d.W, 16) || !aligned(d.idx, 16) || !aligned(d.sgn, 16) || !aligned(d.scales, 16) ||
+        !aligned(d.Wq, 16))
+        return SHERRY_ERR_ALIGN;
+    return SHERRY_OK;
+}
+
+static QuantizeJob job_of(const sherry_quantize_desc& d) {
+    return QuantizeJob{d.W, d.w_dtype, d.N, d.K, d.granularity, d.group, d.idx, d.sgn, d.scales, d.Wq, d.wq_dtype};
+}
+
+static int quantize_call(const sherry_quantize_desc* descs, int count, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    if (!descs && count > 0) return SHERRY_ERR_NULL;
+    if (count < 0 || count > SHERRY_MAX_BATCH) return SHERRY_ERR_SHAPE;
+    std::vector<QuantizeJob> jobs;
+    for (int i = 0; i < count; ++i) {
+        const int st = check_quantize_desc(descs[i]);
+        if (st) return st;
+        jobs.push_back(job_of(descs[i]));
+    }
+    const size_t need = quantize_batch_workspace_bytes(jobs.data(), count);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SHERRY_ERR_WORKSPACE;
+    if (need > 0 && !aligned(workspace, 256)) return SHERRY_ERR_ALIGN;
+    if (count == 0) return SHERRY_OK;
+    return quantize_jobs_launch(jobs.data(), count, workspace, device_sms(), static_cast<cudaStream_t>(stream));
+}
+
 int sherry_quantize_pack(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
                          uint32_t* idx, uint8_t* sgn, float* scales, void* workspace, size_t workspace_bytes,
                          void* stream) {
-    int st = check_shape(N, K);
-    if (st) return st;
-    if ((st = check_gran(K, granularity, group))) return st;
-    if (w_dtype != SHERRY_F32 && w_dtype != SHERRY_BF16) return SHERRY_ERR_DTYPE;
-    if (!scales || (N > 0 && (!W || !idx || !sgn))) return SHERRY_ERR_NULL;
-    if (!aligned(W, 16) || !aligned(idx, 16) || !aligned(sgn, 16) || !aligned(scales, 16)) return SHERRY_ERR_ALIGN;
-    const size_t need = quantize_workspace_bytes(N, K, granularity);
-    if (need > 0 && (!workspace || workspace_bytes < need)) return SHERRY_ERR_WORKSPACE;
-    if (need > 0 && !aligned(workspace, 16)) return SHERRY_ERR_ALIGN;
-    return quantize_pack_launch(W, w_dtype, N, K, granularity, group, idx, sgn, scales, workspace,
-                                static_cast<cudaStream_t>(stream));
+    const sherry_quantize_desc d{W, idx, sgn, scales, nullptr, N, K, w_dtype, granularity, group, SHERRY_F32};
+    return quantize_call(&d, 1, workspace, workspace_bytes, stream);
+}
+
+int sherry_fake_quant(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group, void* Wq,
+                      int wq_dtype, uint32_t* idx, uint8_t* sgn, float* scales, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+    if (N > 0 && !Wq) return SHERRY_ERR_NULL;
+    const sherry_quantize_desc d{W, idx, sgn, scales, Wq, N, K, w_dtype, granularity, group, wq_dtype};
+    return quantize_call(&d, 1, workspace, workspace_bytes, stream);
+}
+
+int sherry_quantize_pack_batched(const sherry_quantize_desc* descs, int count, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    return quantize_call(descs, count, workspace, workspace_bytes, stream);
+}
+
+size_t sherry_quantize_pack_batched_workspace_bytes(const sherry_quantize_desc* descs, int count) {
+    if (!descs || count <= 0 || count > SHERRY_MAX_BATCH) return 0;
+    std::vector<QuantizeJob> jobs;
+    for (int i = 0; i < count; ++i) {
+        if (check_quantize_desc(descs[i])) return 0;
+        jobs.push_back(job_of(descs[i]));
+    }
+    return quantize_batch_workspace_bytes(jobs.data(), count);
 }
 
 static int check_unpack_desc(const sherry_unpack_desc& d) {

@@ -133,11 +133,27 @@ struct ProbShape {
     int granularity, group;
 };
 
+// One weight to quantise and pack (quantize.cu); Wq, if not null, also receives
+// the fake-quantised weights t * alpha in wq_dtype.
+struct QuantizeJob {
+    const void* W;
+    int w_dtype;
+    int64_t N, K;
+    int granularity, group;
+    uint32_t* idx;
+    uint8_t* sgn;
+    float* scales;
+    void* Wq;
+    int wq_dtype;
+};
+
 // launchers (quantize.cu, unpack.cu, gemv.cu)
 size_t quantize_workspace_bytes(int64_t N, int64_t K, int granularity);
-int quantize_pack_launch(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
-                         uint32_t* idx, uint8_t* sgn, float* scales, void* workspace, cudaStream_t stream);
+size_t quantize_batch_workspace_bytes(const QuantizeJob* jobs, int count);
+int quantize_jobs_launch(const QuantizeJob* jobs, int count, void* workspace, int sms, cudaStream_t stream);
 int unpack_launch(const sherry_unpack_desc* descs, int count, cudaStream_t stream, int num_sms);
+// f32[i] != 0: problem i's W_out is fp32 t * alpha instead of bf16
+int unpack_launch_ex(const sherry_unpack_desc* descs, const int* f32, int count, cudaStream_t stream, int num_sms);
 size_t lut_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms);
 int lut_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M,
                       int y_bf16, void* workspace, int sms, cudaStream_t stream);

@@ -1,4 +1,5 @@
-// unpack.cu -- packed planes -> dense bf16 W[n][k] = RNE(t[n][k] * alpha).
+// unpack.cu -- packed planes -> dense bf16 W[n][k] = RNE(t[n][k] * alpha), or
+// fp32 t[n][k] * alpha (the quantiser's forward output for per-tensor scales).
 //
 // The inverse of the 32-state block code ("Sherry: Hardware-Efficient 1.25-Bit
 // Ternary Quantization via Fine-grained Sparsification", digest paragraph on the
@@ -39,7 +40,8 @@ struct UProb {
     const uint32_t* idx;
     const uint8_t* sgn;
     const float* scales;
-    uint16_t* out;
+    void* out;            // bf16 [N][K], or fp32 [N][K] when f32
+    int f32;
     int64_t words_total;  // N * K / 32
     int64_t seg_begin;    // first 8-word segment of this problem in the launch
     int words, granularity, gwords;
@@ -58,7 +60,19 @@ struct UParams {
 template <int MAXP>
 __global__ void __launch_bounds__(256) k_unpack(const __grid_constant__ UParams<MAXP> P) {
     __shared__ uint32_t sel[32];
-    if (threadIdx.x < 32) sel[threadIdx.x] = block_selector(threadIdx.x & 15u, threadIdx.x >> 4);
+    __shared__ float4 tpat[32];  // ternary values of each block code (fp32 output)
+    if (threadIdx.x < 32) {
+        const uint32_t s4 = block_selector(threadIdx.x & 15u, threadIdx.x >> 4);
+        sel[threadIdx.x] = s4;
+        // the selector's (lo, hi) picks: (3, 3) = 0, (0, 1) = +1, (0, 2) = -1
+        float t[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t hi = (s4 >> (8 * i + 4)) & 0xfu;
+            t[i] = hi == 3u ? 0.0f : (hi == 2u ? -1.0f : 1.0f);
+        }
+        tpat[threadIdx.x] = make_float4(t[0], t[1], t[2], t[3]);
+    }
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const int q = lane & 3;
@@ -100,7 +114,16 @@ __global__ void __launch_bounds__(256) k_unpack(const __grid_constant__ UParams<
         }
 #pragma unroll
         for (int j = 0; j < kUSeg; ++j) {
-            if (off[j] >= 0) {
+            if (off[j] >= 0 && pp[j]->f32) {
+                const float a = __uint_as_float(R[j]);
+                const uint32_t byte = (code[j] >> (8 * q)) & 0xffu;
+                const uint32_t sb = sbits[j] >> (2 * q);
+                const float4 t0 = tpat[(byte & 15u) | ((sb & 1u) << 4)];
+                const float4 t1 = tpat[(byte >> 4) | ((sb & 2u) << 3)];
+                float4* o = reinterpret_cast<float4*>(static_cast<float*>(pp[j]->out) + off[j]);
+                __stcs(o, make_float4(t0.x * a, t0.y * a, t0.z * a, t0.w * a));
+                __stcs(o + 1, make_float4(t1.x * a, t1.y * a, t1.z * a, t1.w * a));
+            } else if (off[j] >= 0) {
                 const uint32_t pos = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(R[j])));
                 const uint32_t r4 = pos | (((pos >> 8) | 0x80u) << 16);  // RNE is symmetric in the sign
                 const uint32_t byte = (code[j] >> (8 * q)) & 0xffu;
@@ -112,14 +135,15 @@ __global__ void __launch_bounds__(256) k_unpack(const __grid_constant__ UParams<
                 o.y = __byte_perm(r4, r4, s0 >> 16);
                 o.z = __byte_perm(r4, r4, s1 & 0xffffu);
                 o.w = __byte_perm(r4, r4, s1 >> 16);
-                __stcs(reinterpret_cast<uint4*>(pp[j]->out + off[j]), o);
+                __stcs(reinterpret_cast<uint4*>(static_cast<uint16_t*>(pp[j]->out) + off[j]), o);
             }
         }
     }
 }
 
 template <int MAXP>
-static int unpack_launch_t(const sherry_unpack_desc* d, int count, cudaStream_t stream, int num_sms) {
+static int unpack_launch_t(const sherry_unpack_desc* d, const int* f32, int count, cudaStream_t stream,
+                           int num_sms) {
     static UParams<MAXP> P;
     static std::mutex mu;
     std::lock_guard<std::mutex> lk(mu);
@@ -133,6 +157,7 @@ static int unpack_launch_t(const sherry_unpack_desc* d, int count, cudaStream_t 
         p.sgn = d[i].sgn;
         p.scales = d[i].scales;
         p.out = d[i].W_out;
+        p.f32 = f32 ? f32[i] : 0;
         p.words_total = total;
         p.seg_begin = segs;
         p.words = (int)(d[i].K / 32);
@@ -151,10 +176,14 @@ static int unpack_launch_t(const sherry_unpack_desc* d, int count, cudaStream_t 
     return SHERRY_OK;
 }
 
+int unpack_launch_ex(const sherry_unpack_desc* descs, const int* f32, int count, cudaStream_t stream, int num_sms) {
+    if (count <= 1) return unpack_launch_t<1>(descs, f32, count, stream, num_sms);
+    if (count <= 16) return unpack_launch_t<16>(descs, f32, count, stream, num_sms);
+    return unpack_launch_t<SHERRY_MAX_BATCH>(descs, f32, count, stream, num_sms);
+}
+
 int unpack_launch(const sherry_unpack_desc* descs, int count, cudaStream_t stream, int num_sms) {
-    if (count <= 1) return unpack_launch_t<1>(descs, count, stream, num_sms);
-    if (count <= 16) return unpack_launch_t<16>(descs, count, stream, num_sms);
-    return unpack_launch_t<SHERRY_MAX_BATCH>(descs, count, stream, num_sms);
+    return unpack_launch_ex(descs, nullptr, count, stream, num_sms);
 }
 
 }  // namespace sherry

@@ -185,3 +185,40 @@ def test_header_constants_match_binding():
     assert {"OK", "MAX_K", "MAX_BATCH", "NOALLOC_SCRATCH_BYTES", "PER_GROUP", "BF16", "OP_UNPACK"} <= set(defines)
     for name, value in defines.items():
         assert getattr(_abi, name) == value, name
+
+
+def test_fake_quant_and_batched_quantize_validation(L):
+    fq = L.sherry_fake_quant
+    args = lambda **kw: [kw.get("W", FAKE), kw.get("dt", _abi.F32), kw.get("N", 4), kw.get("K", 64),
+                         kw.get("g", _abi.PER_GROUP), kw.get("group", 32), kw.get("Wq", FAKE),
+                         kw.get("qdt", _abi.F32), kw.get("idx", FAKE), kw.get("sgn", FAKE), kw.get("sc", FAKE),
+                         kw.get("ws", None), kw.get("wsb", 0), None]
+    assert fq(*args(K=48)) == _abi.ERR_SHAPE
+    assert fq(*args(g=7)) == _abi.ERR_GRANULARITY
+    assert fq(*args(group=48)) == _abi.ERR_GROUP
+    assert fq(*args(dt=3)) == _abi.ERR_DTYPE
+    assert fq(*args(qdt=3)) == _abi.ERR_DTYPE
+    assert fq(*args(Wq=None)) == _abi.ERR_NULL
+    assert fq(*args(idx=None)) == _abi.ERR_NULL
+    assert fq(*args(Wq=FAKE + 4)) == _abi.ERR_ALIGN
+    assert fq(*args(g=_abi.PER_TENSOR, group=0)) == _abi.ERR_WORKSPACE  # per-tensor needs its partial sums
+    # batched: every desc is validated before anything runs
+    D = _abi.QuantizeDesc
+    good = D(FAKE, FAKE, FAKE, FAKE, None, 4, 64, _abi.F32, _abi.PER_GROUP, 32, _abi.F32)
+    bad = D(FAKE, FAKE, FAKE, FAKE, None, 4, 48, _abi.F32, _abi.PER_GROUP, 32, _abi.F32)
+    arr = (D * 2)(good, bad)
+    assert L.sherry_quantize_pack_batched(arr, 2, None, 0, None) == _abi.ERR_SHAPE
+    assert L.sherry_quantize_pack_batched(arr, -1, None, 0, None) == _abi.ERR_SHAPE
+    assert L.sherry_quantize_pack_batched(None, 1, None, 0, None) == _abi.ERR_NULL
+    assert L.sherry_quantize_pack_batched_workspace_bytes(arr, 2) == 0
+    t = D(FAKE, FAKE, FAKE, FAKE, None, 4, 3072, _abi.F32, _abi.PER_TENSOR, 0, _abi.F32)
+    arr2 = (D * 2)(good, t)
+    # per-tensor: one partial sum per 1024-weight subtree of each row, 256-byte aligned
+    assert L.sherry_quantize_pack_batched_workspace_bytes(arr2, 2) == 256
+    assert L.sherry_quantize_pack_batched(arr2, 2, None, 0, None) == _abi.ERR_WORKSPACE
+
+
+def test_wait_budget_setter(L):
+    prev = L.sherry_set_wait_budget(1000)
+    assert L.sherry_set_wait_budget(0) == 1000
+    assert L.sherry_set_wait_budget(prev) > 1000  # the default (about 2 s of clock cycles)
