@@ -444,6 +444,10 @@ def extra_rows(args, pairs, outs, shapes, ws, dev, pk):
                             "frac_hbm": round(b1 / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
     del p1, o1
 
+    # decode through the layer chain: q/k/v -> o -> gate/up -> down per layer, each step
+    # reading the previous step's bf16 output on the device (one cooperative launch per token)
+    rows["decode_3b_dependent"] = dependent_rows(args, ws, dev, pk, steps=steps, warm=warm)
+
     # prefill on the tensor cores: the 3B stack (196 linears, one launch each, CUDA graph)
     rows["prefill_3b"] = prefill_rows(args, pairs, ws, dev, pk, steps=max(2, args.steps // 10), warm=3)
 
@@ -471,39 +475,139 @@ def extra_rows(args, pairs, outs, shapes, ws, dev, pk):
                               "launches": 1, "call": "sherry_unpack_batched, 196 weights"}
     del gu, wall, uouts
 
-    # quantize + pack of the full 3B weight set (fp32 in HBM), three granularities
+    # quantize + pack of the full 3B weight set (fp32 in HBM), three granularities: one
+    # batched call (one quantise launch, plus one scale-finalise launch for per-tensor)
     qp = {}
     cfg, layers, shp = synth.STACKS[STACK]
     Ws = [synth.torch_stack_weight(STACK, l, p, device=dev) for (l, p, _) in stack_shapes()]
     tot_w = sum(W.numel() for W in Ws)
     L = _abi.lib()
-    for gname, g, grp in (("group128", _abi.PER_GROUP, 128), ("channel", _abi.PER_CHANNEL, 0),
-                          ("tensor", _abi.PER_TENSOR, 0)):
-        outsP = [sw.quantize_pack(W, g, grp) for W in Ws]
-        wsb = max(L.sherry_workspace_bytes(_abi.OP_QUANTIZE_PACK, 0, W.shape[0], W.shape[1], g, grp) for W in Ws)
+
+    def qdescs(packs, g, grp, wq=None):
+        arr = (_abi.QuantizeDesc * len(Ws))()
+        for i, (W, P) in enumerate(zip(Ws, packs)):
+            q = None if wq is None else wq[i]
+            arr[i] = _abi.QuantizeDesc(W.data_ptr(), P.idx.data_ptr(), P.sgn.data_ptr(), P.scales.data_ptr(),
+                                       None if q is None else q.data_ptr(), W.shape[0], W.shape[1], _abi.F32, g, grp,
+                                       _abi.BF16 if (q is not None and q.dtype == torch.bfloat16) else _abi.F32)
+        return arr
+
+    for gname, g, grp in (("group128", _abi.PER_GROUP, 128), ("channel", _abi.PER_CHANNEL, 128),
+                          ("tensor", _abi.PER_TENSOR, 128)):
+        outsP = sw.quantize_pack_batched(Ws, g, grp)
+        arr = qdescs(outsP, g, grp)
+        wsb = L.sherry_quantize_pack_batched_workspace_bytes(arr, len(Ws))
         wbuf = sw.workspace(wsb, dev, "quantize")
         wptr = wbuf.data_ptr() if wbuf is not None else None
-        argsl = [(W.data_ptr(), W.shape[0], W.shape[1], P.idx.data_ptr(), P.sgn.data_ptr(), P.scales.data_ptr())
-                 for W, P in zip(Ws, outsP)]
-        s_ptr = stream.cuda_stream
 
         def qstep():
-            for (w, N, K, i, sgn, sc) in argsl:
-                st = L.sherry_quantize_pack(w, _abi.F32, N, K, g, grp, i, sgn, sc, wptr, wsb,
-                                            torch.cuda.current_stream().cuda_stream)
-                if st:
-                    raise _abi.SherryError(st, "quantize_pack")
+            st = L.sherry_quantize_pack_batched(arr, len(Ws), wptr, wsb, torch.cuda.current_stream().cuda_stream)
+            if st:
+                raise _abi.SherryError(st, "quantize_pack_batched")
         gq = graph_of(qstep)
         ms = time_region(gq.replay, steps, warm, ws, stream) / steps
         b = sum(4 * W.numel() for W in Ws) + sum(P.nbytes() for P in outsP)
         qp[gname] = {"GB/s": round(ws * b / (ms * 1e-3) / 1e9, 1), "ms": round(ms, 4),
                      "frac_hbm": round(b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4), "weights": tot_w,
-                     "bytes": b, "launches": len(Ws) * (2 if g == _abi.PER_TENSOR else 1)}
+                     "bytes": b, "launches": 2 if g == _abi.PER_TENSOR else 1,
+                     "call": f"sherry_quantize_pack_batched, {len(Ws)} weights"}
         del gq, outsP
+
+    # fake quantisation (the quantiser's forward output t * alpha, for QAT) of the full set,
+    # group 128, with the packed planes: fp32 in, bf16 and fp32 W_q out
+    fq = {}
+    for oname, odt in (("bf16_out", torch.bfloat16), ("fp32_out", torch.float32)):
+        packs = sw.quantize_pack_batched(Ws, _abi.PER_GROUP, 128)
+        wq = [torch.empty_like(W, dtype=odt) for W in Ws]
+        arr = qdescs(packs, _abi.PER_GROUP, 128, wq)
+
+        def fstep():
+            st = L.sherry_quantize_pack_batched(arr, len(Ws), None, 0, torch.cuda.current_stream().cuda_stream)
+            if st:
+                raise _abi.SherryError(st, "fake_quant batched")
+        gq = graph_of(fstep)
+        ms = time_region(gq.replay, steps, warm, ws, stream) / steps
+        b = sum(4 * W.numel() + W.numel() * wq[0].element_size() for W in Ws) + sum(P.nbytes() for P in packs)
+        fq[oname] = {"GB/s": round(ws * b / (ms * 1e-3) / 1e9, 1), "ms": round(ms, 4),
+                     "frac_hbm": round(b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4), "bytes": b, "launches": 1,
+                     "call": f"sherry_quantize_pack_batched with W_q outputs, {len(Ws)} weights"}
+        del gq, packs, wq
+    rows["fake_quant_3b_full"] = fq
     rows["quantize_pack_3b_full"] = qp
     del Ws
     torch.cuda.empty_cache()
     return rows
+
+
+def chain_stack(M, dev, layers=None, stack=STACK):
+    """The decode stack as a chain of dependent steps for M tokens: per layer the fused
+    q/k/v weight, o, the fused gate/up weight and down (group 128), four phases, bf16
+    activations.  The o projection reads the first M*K values of the q/k/v output and
+    the down projection the first M*K values of the gate/up output (stand-ins for
+    attention and the gated activation, which are outside the packed linear); the next
+    layer's q/k/v read the down output.  Returns (phases, fused shapes)."""
+    import torch
+    import sparse_ternary_weight_b200 as sw
+    from sparse_ternary_weight_b200 import synth
+    cfg, all_layers, shp = synth.STACKS[stack]
+    layers = all_layers if layers is None else min(layers, all_layers)
+    d, f = shp["o"][0], shp["down"][1]
+    X0 = synth.torch_activations_bf16(M, d, synth.act_seed(cfg, 0, "q"), device=dev)
+    phases, shapes, x = [], [], X0
+    for l in range(layers):
+        W = {p: synth.torch_stack_weight(stack, l, p, device=dev) for p in synth.PROJ}
+        qkv = sw.quantize_pack_fused([W["q"], W["k"], W["v"]], "per_group", 128)
+        o = sw.quantize_pack(W["o"], "per_group", 128)
+        gu = sw.quantize_pack_fused([W["gate"], W["up"]], "per_group", 128)
+        dn = sw.quantize_pack(W["down"], "per_group", 128)
+        del W
+        ys = [torch.empty((M, P.N), dtype=torch.bfloat16, device=dev) for P in (qkv, o, gu, dn)]
+        phases += [[(x, qkv, ys[0])], [(ys[0].view(-1)[: M * d].view(M, d), o, ys[1])],
+                   [(ys[1], gu, ys[2])], [(ys[2].view(-1)[: M * f].view(M, f), dn, ys[3])]]
+        shapes += [(P.N, P.K) for P in (qkv, o, gu, dn)]
+        x = ys[3]
+    torch.cuda.synchronize()
+    return phases, shapes
+
+
+def dependent_rows(args, ws, dev, pk, steps, warm):
+    """GB/s and tok/s of the chained decode (one token, and two tokens) over the 3B stack."""
+    import torch
+    import sparse_ternary_weight_b200 as sw
+    from sparse_ternary_weight_b200 import _abi
+    stream = torch.cuda.current_stream()
+    out = {}
+    for M in (1, 2):
+        phases, shapes = chain_stack(M, dev)
+        flat = [t for ph in phases for t in ph]
+        descs = sw.make_batch([(X, P) for X, P, _ in flat], [Y for _, _, Y in flat])
+        sw.linear_chain(phases, torch.bfloat16, descs=descs)  # allocates the workspace
+        L = _abi.lib()
+        import ctypes
+        begin = [0]
+        for ph in phases:
+            begin.append(begin[-1] + len(ph))
+        pb = (ctypes.c_int * len(begin))(*begin)
+        wsb = L.sherry_linear_chain_workspace_bytes(descs, len(flat), pb, len(phases), M)
+        wbuf = sw.workspace(wsb, dev)
+        wptr = wbuf.data_ptr() if wbuf is not None else None
+
+        def call():
+            st = L.sherry_linear_chain(descs, len(flat), pb, len(phases), M, _abi.BF16, wptr, wsb,
+                                       torch.cuda.current_stream().cuda_stream)
+            if st:
+                raise _abi.SherryError(st, "linear_chain")
+        ms = time_region(call, steps, warm, ws, stream) / steps
+        b = stack_bytes(shapes, M, y_bytes=2)
+        assert sw.device_status(dev) == 0
+        out[f"M{M}"] = {"GB/s": round(ws * b / (ms * 1e-3) / 1e9, 1), "tok_per_s": round(ws * M / (ms * 1e-3), 1),
+                        "ms_per_step": round(ms, 4), "frac_hbm": round(b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                        "bytes": b, "phases": len(phases), "launches": 1,
+                        "call": "sherry_linear_chain: 28 layers x (fused q/k/v, o, fused gate/up, down), "
+                                "each phase reading the previous one's bf16 output"}
+        del phases, flat, descs
+        torch.cuda.empty_cache()
+    return out
 
 
 def prefill_rows(args, pairs, ws, dev, pk, steps, warm):
@@ -718,6 +822,23 @@ def profile_decode(args):
                       "GB/s": round(b / (ms * 1e-3) / 1e9, 1), "bytes": b}), flush=True)
 
 
+def profile_chain(args):
+    """The chained decode over the first LAYERS layers of the 3B stack at M tokens
+    (for profiler captures of the chained kernel)."""
+    import torch
+    from sparse_ternary_weight_b200.build import build
+    build()
+    import sparse_ternary_weight_b200 as sw
+    M, layers = (int(v) for v in args.profile_chain.split(","))
+    dev = torch.device("cuda", 0)
+    phases, shapes = chain_stack(M, dev, layers)
+    ms = time_region(lambda: sw.linear_chain(phases, torch.bfloat16), args.steps, args.warmup, 1,
+                     torch.cuda.current_stream()) / args.steps
+    b = stack_bytes(shapes, M, y_bytes=2)
+    print(json.dumps({"chain": f"3B stack, {layers} layers, M={M}", "ms": round(ms, 4),
+                      "GB/s": round(b / (ms * 1e-3) / 1e9, 1), "bytes": b}), flush=True)
+
+
 def profile_quantize(args):
     import torch
     from sparse_ternary_weight_b200.build import build
@@ -758,7 +879,13 @@ def main():
     ap.add_argument("--profile-decode", default=None, metavar="M,LAYERS",
                     help="only run the batched decode call over the first LAYERS layers of the 3B stack at M "
                          "tokens warmup+steps times, print its time, and exit (for profiler captures)")
+    ap.add_argument("--profile-chain", default=None, metavar="M,LAYERS",
+                    help="only run the chained decode over the first LAYERS layers of the 3B stack at M tokens "
+                         "warmup+steps times, print its time, and exit (for profiler captures)")
     args = ap.parse_args()
+    if args.profile_chain:
+        profile_chain(args)
+        return
     if args.profile_decode:
         profile_decode(args)
         return

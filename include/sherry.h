@@ -206,6 +206,31 @@ int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M,
                           void* workspace, size_t workspace_bytes, void* stream);
 size_t sherry_linear_batched_workspace_bytes(const sherry_linear_desc* descs, int count, int64_t M);
 
+/* ---- chained linears (dependent phases) -----------------------------------
+ * `count` linears with the same M (e.g. one decode token through a layer
+ * stack) grouped into n_phases phases: phase p holds descs[phase_begin[p] ..
+ * phase_begin[p+1]) (phase_begin: HOST array of n_phases + 1 indices,
+ * phase_begin[0] = 0, non-decreasing, phase_begin[n_phases] = count).  The
+ * linears of a phase are independent; every linear of phase p+1 starts after
+ * every linear of phase p has written Y, so a later phase may read an earlier
+ * phase's Y as its X (bf16 Y, y_dtype SHERRY_BF16, read in place).  Each Y is
+ * computed as by sherry_linear (fp32 accumulation, alpha once per group), within
+ * the fp32 summation-order bound of it.
+ *   One and two tokens with every K % 256 == 0 and group 128 or 256 (or row
+ *   scales): one cooperative launch (one CTA per SM, all resident) in which a
+ *   grid-wide bounded barrier separates the phases and the packed weights of the
+ *   next phase stream in while it resolves ("Sherry: ..." digest: inference
+ *   streams the packed weights through lookup tables; the pages' layer is
+ *   F.linear).  Otherwise: one sherry_linear_batched-style launch set per phase,
+ *   ordered by the stream.
+ *   workspace  sherry_linear_chain_workspace_bytes(...) bytes; the same ticket
+ *            contract as a linear workspace (first 256 KiB zero before the first
+ *            use; every successful call leaves it zero). */
+int sherry_linear_chain(const sherry_linear_desc* descs, int count, const int* phase_begin, int n_phases,
+                        int64_t M, int y_dtype, void* workspace, size_t workspace_bytes, void* stream);
+size_t sherry_linear_chain_workspace_bytes(const sherry_linear_desc* descs, int count, const int* phase_begin,
+                                           int n_phases, int64_t M);
+
 /* ---- packed linear without a workspace -------------------------------------
  * No counterpart on the pages: this is a service for callers that cannot
  * allocate device memory (a host framework that plans all memory ahead and

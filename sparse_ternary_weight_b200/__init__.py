@@ -272,6 +272,69 @@ def linear_batched(pairs, out_dtype=None, outs=None, descs=None):
     return outs
 
 
+def linear_chain(phases, out_dtype=None, descs=None):
+    """Chained linears: ``phases`` is a list of phases, each a list of (X, P, Y)
+    triples (X bf16 [M,K], Y [M,N] preallocated).  Every linear of a phase starts
+    after every linear of the previous phase has written its Y, so an X may be
+    (a view of) an earlier phase's Y.  Returns the list of Y per phase."""
+    import torch
+    out_dtype = out_dtype or torch.float32
+    yd = {torch.float32: F32, torch.bfloat16: BF16}[out_dtype]
+    flat = [t for ph in phases for t in ph]
+    if not flat:
+        return []
+    M = flat[0][0].shape[0]
+    for X, P, Y in flat:
+        _require_cuda(X, Y)
+        if X.dtype != torch.bfloat16 or X.shape != (M, P.K) or not X.is_contiguous():
+            raise ValueError("each X must be contiguous bf16 [M,K] with the same M")
+        if Y.dtype != out_dtype or Y.shape != (M, P.N) or not Y.is_contiguous():
+            raise ValueError("each Y must be contiguous [M,N] of out_dtype")
+    if descs is None:
+        descs = make_batch([(X, P) for X, P, _ in flat], [Y for _, _, Y in flat])
+    begin = [0]
+    for ph in phases:
+        begin.append(begin[-1] + len(ph))
+    pb = (ctypes.c_int * len(begin))(*begin)
+    L = lib()
+    wsb = L.sherry_linear_chain_workspace_bytes(descs, len(flat), pb, len(phases), M)
+    ws = workspace(wsb, flat[0][0].device)
+    check(L.sherry_linear_chain(descs, len(flat), pb, len(phases), M, yd, _ptr(ws), wsb, _stream(flat[0][0].device)),
+          "linear_chain")
+    return [[Y for _, _, Y in ph] for ph in phases]
+
+
+def quantize_pack_fused(weights, granularity="per_group", group: int = 128) -> PackedWeight:
+    """One packed weight whose rows are the rows of ``weights`` in order (e.g. the
+    q, k and v projections, or gate and up, of a decoder layer), so that one
+    linear call computes all of them.  The planes and the group or row scales of
+    each part are exactly those of packing it alone (they depend on its own rows
+    only); per-tensor scales are per part and cannot share one packed weight."""
+    import torch
+    g = _gran(granularity)
+    if g == PER_TENSOR:
+        raise ValueError("per-tensor scales are one per weight: pack the parts separately")
+    K = weights[0].shape[1]
+    if any(W.dim() != 2 or W.shape[1] != K for W in weights):
+        raise ValueError("every part must be 2D with the same K")
+    N = sum(W.shape[0] for W in weights)
+    L = lib()
+    ns = L.sherry_num_scales(N, K, g, group)
+    if ns < 0:
+        raise SherryError(_abi.ERR_SHAPE if K % 32 or K < 32 else _abi.ERR_GROUP, "quantize_pack_fused")
+    fused = _new_packed(N, K, g, group, ns, weights[0].device)
+    spr = ns // N  # scales per row
+    r0 = 0
+    parts = []
+    for W in weights:
+        n = W.shape[0]
+        parts.append(PackedWeight(fused.idx[r0:r0 + n], fused.sgn[r0:r0 + n], fused.scales[r0 * spr:(r0 + n) * spr],
+                                  n, K, g, group))
+        r0 += n
+    quantize_pack_batched([W.contiguous() for W in weights], g, group, outs=parts)
+    return fused
+
+
 def unpack_batched(packs, outs=None):
     """Dense bf16 of several packed weights in one launch (each as by :func:`unpack`)."""
     import torch

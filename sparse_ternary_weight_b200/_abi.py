@@ -52,6 +52,10 @@ SIGNATURES = {
     "sherry_linear": (i32, [vp, i64, i64, i64, vp, vp, vp, i32, i32, vp, i32, vp, sz, vp]),
     "sherry_linear_batched": (i32, [ctypes.POINTER(LinearDesc), i32, i64, i32, vp, sz, vp]),
     "sherry_linear_batched_workspace_bytes": (sz, [ctypes.POINTER(LinearDesc), i32, i64]),
+    "sherry_linear_chain": (i32, [ctypes.POINTER(LinearDesc), i32, ctypes.POINTER(ctypes.c_int), i32, i64, i32, vp,
+                                  sz, vp]),
+    "sherry_linear_chain_workspace_bytes": (sz, [ctypes.POINTER(LinearDesc), i32, ctypes.POINTER(ctypes.c_int), i32,
+                                                 i64]),
     "sherry_unpack": (i32, [vp, vp, vp, i64, i64, i32, i32, vp, vp]),
     "sherry_unpack_batched": (i32, [ctypes.POINTER(UnpackDesc), i32, vp]),
     "sherry_linear_noalloc": (i32, [vp, i64, i64, i64, vp, vp, vp, i32, i32, vp, i32, vp]),

@@ -335,4 +335,78 @@ int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M,
                          static_cast<cudaStream_t>(stream));
 }
 
+// A chain without its empty linears: problems, descriptors and phase bounds.
+struct Chain {
+    std::vector<ProbShape> shapes;
+    std::vector<sherry_linear_desc> descs;
+    std::vector<int> begin;  // n_phases + 1 problem indices
+};
+
+static int chain_of(const sherry_linear_desc* descs, int count, const int* phase_begin, int n_phases, int64_t M,
+                    Chain& c) {
+    if ((!descs && count > 0) || !phase_begin) return SHERRY_ERR_NULL;
+    if (count < 0 || count > SHERRY_MAX_BATCH || n_phases < 1 || n_phases > SHERRY_MAX_BATCH) return SHERRY_ERR_SHAPE;
+    if (M < 0 || M > (int64_t)0x7fffffff) return SHERRY_ERR_SHAPE;
+    if (phase_begin[0] != 0 || phase_begin[n_phases] != count) return SHERRY_ERR_SHAPE;
+    for (int ph = 0; ph < n_phases; ++ph)
+        if (phase_begin[ph + 1] < phase_begin[ph]) return SHERRY_ERR_SHAPE;
+    for (int ph = 0; ph < n_phases; ++ph) {
+        c.begin.push_back((int)c.shapes.size());
+        for (int i = phase_begin[ph]; i < phase_begin[ph + 1]; ++i) {
+            const int st = check_linear_desc(descs[i], M);
+            if (st) return st;
+            if (descs[i].N == 0) continue;
+            c.shapes.push_back(ProbShape{descs[i].N, descs[i].K, descs[i].granularity, descs[i].group});
+            c.descs.push_back(descs[i]);
+        }
+    }
+    c.begin.push_back((int)c.shapes.size());
+    return SHERRY_OK;
+}
+
+static size_t chain_ws(const Chain& c, int64_t M, int sms) {
+    const int n = (int)c.begin.size() - 1;
+    if (c.shapes.empty() || M == 0) return 0;
+    if (chain_launch_ok(c.shapes.data(), (int)c.shapes.size(), n, M))
+        return chain_workspace_bytes(c.shapes.data(), (int)c.shapes.size(), c.begin.data(), n, M, sms);
+    size_t ws = 0;
+    for (int ph = 0; ph < n; ++ph)
+        if (c.begin[ph + 1] > c.begin[ph])
+            ws = std::max(ws, linear_ws_bytes(c.shapes.data() + c.begin[ph], c.begin[ph + 1] - c.begin[ph], M, sms));
+    return ws;
+}
+
+size_t sherry_linear_chain_workspace_bytes(const sherry_linear_desc* descs, int count, const int* phase_begin,
+                                           int n_phases, int64_t M) {
+    Chain c;
+    if (chain_of(descs, count, phase_begin, n_phases, M, c)) return 0;
+    return chain_ws(c, M, device_sms());
+}
+
+int sherry_linear_chain(const sherry_linear_desc* descs, int count, const int* phase_begin, int n_phases, int64_t M,
+                        int y_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    Chain c;
+    int st = chain_of(descs, count, phase_begin, n_phases, M, c);
+    if (st) return st;
+    if (y_dtype != SHERRY_F32 && y_dtype != SHERRY_BF16) return SHERRY_ERR_DTYPE;
+    if (c.shapes.empty() || M == 0) return SHERRY_OK;
+    const int sms = device_sms();
+    const size_t need = chain_ws(c, M, sms);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SHERRY_ERR_WORKSPACE;
+    if (need > 0 && !aligned(workspace, 256)) return SHERRY_ERR_ALIGN;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int n = (int)c.begin.size() - 1;
+    if (chain_launch_ok(c.shapes.data(), (int)c.shapes.size(), n, M))
+        return chain_linear_launch(c.shapes.data(), c.descs.data(), (int)c.shapes.size(), c.begin.data(), n, M,
+                                   y_dtype == SHERRY_BF16, workspace, sms, s);
+    // otherwise one batched launch set per phase, ordered by the stream
+    for (int ph = 0; ph < n; ++ph) {
+        const int b = c.begin[ph], e = c.begin[ph + 1];
+        if (e > b && (st = linear_launch(c.shapes.data() + b, c.descs.data() + b, e - b, M, y_dtype == SHERRY_BF16,
+                                         workspace, sms, s)))
+            return st;
+    }
+    return SHERRY_OK;
+}
+
 }  // extern "C"

@@ -177,5 +177,12 @@ long long stream_set_wait_cycles(long long cycles);  // returns the previous bud
 size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms);
 int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream);
+// chained phases on the streaming kernel (cooperative launch, one CTA per SM)
+bool chain_eligible(const ProbShape& s, int64_t M);
+bool chain_launch_ok(const ProbShape* shapes, int count, int n_phases, int64_t M);
+size_t chain_workspace_bytes(const ProbShape* shapes, int count, const int* phase_begin, int n_phases, int64_t M,
+                             int sms);
+int chain_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, const int* phase_begin,
+                        int n_phases, int64_t M, int y_bf16, void* workspace, int sms, cudaStream_t stream);
 
 }  // namespace sherry

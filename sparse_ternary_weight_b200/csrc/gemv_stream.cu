@@ -5,25 +5,35 @@
 // Quantization via Fine-grained Sparsification", digest paragraph on inference;
 // Y = X T alpha).
 //
-// Work unit: 512 output rows x 512 weights (16 packed words) of one linear.
-// All units of a launch (one or many independent linears) are split into equal
+// Work unit: 512 output rows x 32 W weights (W packed words) of one linear, W =
+// 16 for independent linears (one batched launch per decode step) and W = 8 for
+// chained phases, whose layers are small enough that finer units balance better.
+// All units of a phase (one or many independent linears) are split into equal
 // contiguous ranges, one per CTA (stream-K): every CTA streams the same number
-// of bytes.  A row block whose units straddle two CTAs is finished by the CTA
-// that arrives last at its ticket, adding the partial sums in CTA order, so Y
-// is deterministic.
+// of bytes.  A row block whose units straddle CTAs is finished by the CTA that
+// arrives last at its ticket, adding the partial sums in CTA order, so Y is
+// deterministic.
+//
+// Phases (chained linears, e.g. the q/k/v -> o -> gate/up -> down projections
+// of a decoder layer stack for one token): a later phase may read an earlier
+// phase's Y as its X.  The launch is cooperative (one CTA per SM, all resident);
+// after its last unit of a phase a CTA adds one arrival to the phase's counter,
+// and before building the first tables of a phase a CTA waits (bounded) until
+// every CTA has arrived at the previous phase.  Packed weights do not depend on
+// X, so the copies of the next units run ahead of that wait and stream from HBM
+// while the barrier resolves.
 //
 // Roles (20 warps).  16 consumer warps: each thread owns one row of the unit
 // and only looks up and accumulates (per packed word it spreads the 8 nibbles
 // and sign bits into two byte-vectors of table offsets, see lut.cuh, and does 8
 // lookups per token at the same offsets; alpha is applied once per 128-weight
 // group, or once per row).  4 helper warps, one per SM sub-partition: they copy
-// each unit's packed planes with 16-byte cp.async (4 lanes read one row's 64
-// contiguous bytes, so global reads are coalesced) into an XOR-swizzled ring of
-// stages (three for one token, two for two) that the row-per-lane reads hit
-// without bank conflicts, and build the unit's 128 tables of 32 entries per
-// token into the stage's table buffer.  Stages change hands through mbarriers;
-// every wait is bounded, and a timeout sets a device status flag (reported by
-// sherry_device_status) and ends the CTA.
+// each unit's packed planes with cp.async (W/4 lanes read one row's 4W
+// contiguous bytes) into an XOR-swizzled ring of stages that the row-per-lane
+// reads hit without bank conflicts, and build the unit's 8W tables of 32
+// entries per token into the stage's table buffer.  Stages change hands through
+// mbarriers; every wait is bounded, and a timeout sets a device status flag
+// (reported by sherry_device_status) and ends the CTA.
 #include "common.cuh"
 #include "lut.cuh"
 
@@ -40,25 +50,43 @@ constexpr int kSConsumers = 16;                    // consumer warps: one row pe
 constexpr int kSHelpers = 4;                       // copy + table warps
 constexpr int kSThreads = 32 * (kSConsumers + kSHelpers);
 constexpr int kSRows = 32 * kSConsumers;           // 512 rows per unit
-constexpr int kSWords = 16;                        // packed words per unit (512 weights)
-constexpr int kSIdx = kSRows * kSWords * 4;        // 32 KB
-constexpr int kSSgn = kSRows * 16;                 // 8 KB (16 sign bytes per row)
-constexpr int kSSc = kSRows * 16;                  // 8 KB (at most 4 fp32 scales per row)
-constexpr int kSStage = kSIdx + kSSgn + kSSc;      // 48 KB
-constexpr int kSTabs = kSWords * 8;                // 128 tables per unit
-constexpr int kSLut = kSTabs * kTab;               // 18 KB: one token's tables of a unit
 constexpr int kSBars = 128;                        // mbarriers
-static_assert(kSStage % 256 == 0 && kSLut % 256 == 0, "table bases must stay multiples of 256");
+constexpr int kSHelperThreads = 32 * kSHelpers;
+// chained launches keep their phase counters at the end of the ticket region
+constexpr int kChainCtrs = 512;                    // up to 511 phases + the exit counter
+constexpr int kSMaxPhases = kChainCtrs - 1;
 
-// Ring depth and shared bytes for MT tokens (tables are token-major within a stage).
-template <int MT>
-struct SCfg {
-    static constexpr int kStages = MT == 1 ? 3 : 2;
-    static constexpr int kLutStage = MT * kSLut;
-    static constexpr int kSmem = 256 + kStages * (kSStage + kLutStage) + kSBars;
+// Geometry of a unit of W packed words.
+template <int W>
+struct SGeo {
+    static constexpr int kIdx = kSRows * W * 4;    // packed words of a stage
+    static constexpr int kSgn = kSRows * W;        // sign bytes (W per row)
+    static constexpr int kSc = kSRows * W;         // scales (at most W/4 floats per row)
+    static constexpr int kStage = kIdx + kSgn + kSc;
+    static constexpr int kTabs = W * 8;            // tables per unit (one per block of 4 activations)
+    static constexpr int kLut = kTabs * kTab;      // one token's tables of a unit
+    static constexpr int kRowB = 4 * W;            // packed-word bytes of one row
+    static constexpr int kLanesPerRow = W / 4;     // 16-byte chunks per row
+    static constexpr int kRowsPerCopy = 32 / kLanesPerRow;
+    static constexpr int kSwz = 128 / kRowB;       // rows per 128-byte cycle of the banks
+    static_assert(W == 16 || W == 8, "unit widths");
+    static_assert(kStage % 256 == 0 && kLut % 256 == 0, "table bases must stay multiples of 256");
+    static_assert(kTabs <= kSHelperThreads, "one table per helper thread");
 };
-static_assert(SCfg<1>::kSmem <= 232448 && SCfg<2>::kSmem <= 232448, "shared memory per CTA");
-static_assert(kSTabs == 32 * kSHelpers, "one table per helper thread");
+
+// Ring depth, copy lookahead and shared bytes for MT tokens and W-word units
+// (tables are token-major within a stage).  The lookahead L lets the copies run
+// L units ahead of the table builds (used across phase barriers).
+template <int MT, int W>
+struct SCfg {
+    using G = SGeo<W>;
+    static constexpr int kStages = W == 16 ? (MT == 1 ? 3 : 2) : (MT == 1 ? 6 : 5);
+    static constexpr int kAhead = W == 16 ? 0 : kStages - 2;
+    static constexpr int kLutStage = MT * G::kLut;
+    static constexpr int kSmem = 256 + kStages * (G::kStage + kLutStage) + kSBars;
+    static_assert(kSmem <= 232448, "shared memory per CTA");
+    static_assert(kStages <= 6, "barrier slots");
+};
 constexpr long long kSWaitCycles = 4000000000LL;   // default wait budget, ~2 s at the boost clock
 // The no-workspace entry point's fixed scratch holds this kernel's largest plan
 // (two tokens, one CTA per SM, two partial slots per CTA) on up to 224 SMs.
@@ -82,9 +110,12 @@ struct SProb {
 template <int MAXP>
 struct SParams {
     long long wait_cycles;  // budget of every bounded wait, in SM clock cycles
-    int count, y_bf16, total_units, upc;
-    float* part;  // [grid][2][MT][kSRows] split-tile partials
-    int* ticket;  // [total tiles]
+    int count, y_bf16, n_phases;
+    float* part;            // [grid][2][MT][kSRows] split-tile partials
+    int* ticket;            // [total tiles]
+    int* phase_cnt;         // chained launches: [n_phases] arrivals + exit counter; else null
+    int ph_unit[MAXP + 1];  // first unit of each phase; ph_unit[n_phases] = all units
+    int ph_upc[MAXP];       // units per CTA of each phase
     SProb p[MAXP];
 };
 
@@ -93,13 +124,14 @@ __device__ int g_stream_status = 0;
 
 namespace {
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(valid ? 8 : 0)
-                 : "memory");
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 // the mbarrier receives one arrival when all of this thread's prior cp.async complete
 __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
@@ -135,6 +167,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         }
     }
 }
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// wait until *cnt >= target (every CTA arrived at a phase); false on timeout or abort
+__device__ __forceinline__ bool grid_wait(const int* cnt, int target, volatile int* abort_flag, long long budget) {
+    if (ld_acquire(cnt) >= target) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (ld_acquire(cnt) >= target) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > budget) {
+            *abort_flag = 1;
+            atomicExch(&g_stream_status, SHERRY_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
 
 }  // namespace
 
@@ -150,15 +201,20 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
     return v;
 }
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
 
 // 8 lookups of one packed word for token TOK: the tables of blocks BOFF..BOFF+7
-// sit at shared offsets (BOFF + j) * kTab + TOK * kSLut from the addresses in a[],
+// sit at shared offsets (BOFF + j) * kTab + TOK * LUT from the addresses in a[],
 // whose low byte is the block's table offset -> even-position and odd-position
 // partial sums p0 = (v0 + v2) + (v4 + v6), p1 = (v1 + v3) + (v5 + v7), as
 // packed pair adds
-template <int BOFF, int TOK>
+template <int BOFF, int TOK, int LUT>
 __device__ __forceinline__ void token_sums(const uint32_t (&a)[8], float& p0, float& p1) {
-    constexpr int T = TOK * kSLut;
+    constexpr int T = TOK * LUT;
     const float v0 = lds_imm<(BOFF + 0) * kTab + T>(a[0]);
     const float v1 = lds_imm<(BOFF + 1) * kTab + T>(a[1]);
     const float v2 = lds_imm<(BOFF + 2) * kTab + T>(a[2]);
@@ -176,7 +232,7 @@ __device__ __forceinline__ void token_sums(const uint32_t (&a)[8], float& p0, fl
 // One packed word (nibbles w, sign byte s; its 8 tables at `base`, a multiple of
 // 256, plus BOFF * kTab): the 8 table addresses are formed once and looked up for
 // each of the MT tokens.
-template <int BOFF, int MT>
+template <int BOFF, int MT, int LUT>
 __device__ __forceinline__ void word_sums(uint32_t w, uint32_t s, uint32_t base, float (&p0)[MT], float (&p1)[MT]) {
     uint32_t ev, od;
     spread_word(w, s, ev, od);
@@ -184,8 +240,8 @@ __device__ __forceinline__ void word_sums(uint32_t w, uint32_t s, uint32_t base,
                            __byte_perm(ev, base, 0x7651u), __byte_perm(od, base, 0x7651u),
                            __byte_perm(ev, base, 0x7652u), __byte_perm(od, base, 0x7652u),
                            __byte_perm(ev, base, 0x7653u), __byte_perm(od, base, 0x7653u)};
-    token_sums<BOFF, 0>(a, p0[0], p1[0]);
-    if constexpr (MT > 1) token_sums<BOFF, 1>(a, p0[1], p1[1]);
+    token_sums<BOFF, 0, LUT>(a, p0[0], p1[0]);
+    if constexpr (MT > 1) token_sums<BOFF, 1, LUT>(a, p0[1], p1[1]);
 }
 
 struct UnitPos {
@@ -210,23 +266,59 @@ __device__ __forceinline__ void advance(const SProb* probs, UnitPos& u) {
     }
 }
 
-// Copy geometry of helper lane (h, lane) for one row block: the unit's rows
-// [128h, 128h+128).  Packed words: rows 128h + 8i + lane/4 (i = 0..15), 16-byte
-// chunk lane%4 of the row's 64 bytes, stored at chunk (c ^ ((row >> 1) & 3)) of a
-// 64-byte shared row (that swizzle term is (lane >> 3) & 3 for every i).  Sign
-// bytes and scales: rows 128h + 32i + lane (i = 0..3), 16 bytes each.  Byte
-// offsets from the plane bases; a row past N reads row 0 instead (its results
-// are never stored), so every copy is a full in-bounds 16 bytes.
-struct CopyRows {
-    uint32_t idx[16], sgn[4], sc[4];
+// This CTA's unit range [b, e) of phase ph.
+template <int MAXP>
+__device__ __forceinline__ void phase_range(const SParams<MAXP>& P, int ph, int& b, int& e) {
+    b = P.ph_unit[ph] + (int)blockIdx.x * P.ph_upc[ph];
+    e = min(P.ph_unit[ph + 1], b + P.ph_upc[ph]);
+}
+
+// The CTA's units in order over all phases (empty phase ranges skipped).
+template <int MAXP>
+struct UnitCursor {
+    int ph, u, e;
+    UnitPos pos;
+    __device__ __forceinline__ void seek(const SParams<MAXP>& P, int from_ph) {
+        for (ph = from_ph; ph < P.n_phases; ++ph) {
+            int b;
+            phase_range(P, ph, b, e);
+            if (b < e) {
+                u = b;
+                pos = locate(P, u);
+                return;
+            }
+        }
+        u = e = 0;
+    }
+    __device__ __forceinline__ void next(const SParams<MAXP>& P) {
+        if (++u < e)
+            advance(P.p, pos);
+        else
+            seek(P, ph + 1);
+    }
 };
 
-__device__ __forceinline__ void copy_rows(const SProb& pr, int rb, int h, int lane, CopyRows& cr) {
+// Copy geometry of helper lane (h, lane) for one row block: the unit's rows
+// [128h, 128h+128).  Packed words: rows 128h + R*i + lane/C (C = W/4 lanes per
+// row, R = 32/C rows per copy), 16-byte chunk lane%C of the row's 4W bytes,
+// stored at chunk (c ^ ((row / S) % C)) of the row in shared memory, S = 128/4W
+// rows per bank cycle (that swizzle term only depends on the lane).  Sign bytes
+// and scales: rows 128h + 32i + lane (i = 0..3).  Byte offsets from the plane
+// bases; a row past N reads row 0 instead (its results are never stored), so
+// every copy is in bounds.
+template <int W>
+struct CopyRows {
+    uint32_t idx[W], sgn[4], sc[4];
+};
+
+template <int W>
+__device__ __forceinline__ void copy_rows(const SProb& pr, int rb, int h, int lane, CopyRows<W>& cr) {
+    using G = SGeo<W>;
     const int row0 = rb * kSRows;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int row = row0 + 128 * h + 8 * i + (lane >> 2);
-        cr.idx[i] = (uint32_t)((int64_t)(row < pr.N ? row : 0) * pr.words * 4 + 16 * (lane & 3));
+    for (int i = 0; i < 128 / G::kRowsPerCopy; ++i) {
+        const int row = row0 + 128 * h + G::kRowsPerCopy * i + lane / G::kLanesPerRow;
+        cr.idx[i] = (uint32_t)((int64_t)(row < pr.N ? row : 0) * pr.words * 4 + 16 * (lane % G::kLanesPerRow));
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -242,56 +334,90 @@ __device__ __forceinline__ const void* byte_off(const void* base, uint32_t off) 
 }
 
 // Helper lane's copies of unit (cr's row block, sub-slice `sub`) into `stage`.
-__device__ __forceinline__ void copy_unit(const SProb& pr, const CopyRows& cr, int sub, uint32_t stage, int h,
+template <int W>
+__device__ __forceinline__ void copy_unit(const SProb& pr, const CopyRows<W>& cr, int sub, uint32_t stage, int h,
                                           int lane) {
-    const char* bi = reinterpret_cast<const char*>(pr.idx) + sub * (kSWords * 4);
-    const uint32_t di = stage + (uint32_t)(128 * h + (lane >> 2)) * 64u +
-                        ((uint32_t)((lane & 3) ^ ((lane >> 3) & 3)) << 4);
+    using G = SGeo<W>;
+    constexpr int C = G::kLanesPerRow;
+    const char* bi = reinterpret_cast<const char*>(pr.idx) + sub * G::kRowB;
+    const uint32_t lrow = (uint32_t)(lane / C);
+    const uint32_t di = stage + (uint32_t)(128 * h + lrow) * G::kRowB +
+                        ((uint32_t)((lane % C) ^ ((lrow / G::kSwz) % C)) << 4);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) cp_async16(di + 512u * i, byte_off(bi, cr.idx[i]), true);
-    const char* bs = reinterpret_cast<const char*>(pr.sgn) + sub * kSWords;
-    const uint32_t ds = stage + kSIdx + (uint32_t)(128 * h + lane) * 16u;
+    for (int i = 0; i < 128 / G::kRowsPerCopy; ++i)
+        cp_async16(di + (uint32_t)(G::kRowsPerCopy * G::kRowB * i), byte_off(bi, cr.idx[i]));
+    const char* bs = reinterpret_cast<const char*>(pr.sgn) + sub * W;
+    const uint32_t ds = stage + G::kIdx + (uint32_t)(128 * h + lane) * W;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) cp_async16(ds + 512u * i, byte_off(bs, cr.sgn[i]), true);
-    if (pr.mode == kSG128) {
-        const char* ba = reinterpret_cast<const char*>(pr.scales) + sub * 16;
+    for (int i = 0; i < 4; ++i) {
+        if (W == 16)
+            cp_async16(ds + 32u * W * i, byte_off(bs, cr.sgn[i]));
+        else
+            cp_async8(ds + 32u * W * i, byte_off(bs, cr.sgn[i]));
+    }
+    const uint32_t dc = ds + G::kSgn;
+    if (pr.mode == kSG128) {  // W/4 scales per row and unit
+        const char* ba = reinterpret_cast<const char*>(pr.scales) + sub * W;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cp_async16(ds + kSSgn + 512u * i, byte_off(ba, cr.sc[i]), true);
-    } else if (pr.mode == kSG256) {
-        const char* ba = reinterpret_cast<const char*>(pr.scales) + sub * 8;
+        for (int i = 0; i < 4; ++i) {
+            if (W == 16)
+                cp_async16(dc + 32u * W * i, byte_off(ba, cr.sc[i]));
+            else
+                cp_async8(dc + 32u * W * i, byte_off(ba, cr.sc[i]));
+        }
+    } else if (pr.mode == kSG256) {  // W/8 scales per row and unit
+        const char* ba = reinterpret_cast<const char*>(pr.scales) + sub * (W / 2);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cp_async8(ds + kSSgn + 512u * i, byte_off(ba, cr.sc[i]), true);
+        for (int i = 0; i < 4; ++i) {
+            if (W == 16)
+                cp_async8(dc + 32u * W * i, byte_off(ba, cr.sc[i]));
+            else
+                cp_async4(dc + 32u * W * i, byte_off(ba, cr.sc[i]));
+        }
     }
 }
 
-// Lookups of one row over the 16 words of a unit for MT tokens, into u[]; `st`
+// Lookups of one row over the W words of a unit for MT tokens, into u[]; `st`
 // and `lut` are shared addresses of the unit's stage and of token 0's tables.
-template <int MODE, int MT>
+template <int MODE, int MT, int W>
 __device__ __forceinline__ void unit_row(uint32_t st, uint32_t lut, int r, float (&u)[MT]) {
-    const uint32_t sw = (uint32_t)((r >> 1) & 3);
-    const uint4 sg = lds128(st + kSIdx + r * 16);
-    uint4 av = make_uint4(0u, 0u, 0u, 0u);
-    if (MODE == kSG128) av = lds128(st + kSIdx + kSSgn + r * 16);
-    if (MODE == kSG256) {
-        const uint2 a2 = lds64(st + kSIdx + kSSgn + r * 16);
-        av = make_uint4(a2.x, a2.y, 0u, 0u);
+    using G = SGeo<W>;
+    constexpr int C = G::kLanesPerRow;
+    const uint32_t sw = (uint32_t)((r / G::kSwz) % C);
+    uint4 sg, av = make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t sgn_a = st + G::kIdx + r * W, sc_a = st + G::kIdx + G::kSgn + r * W;
+    if (W == 16) {
+        sg = lds128(sgn_a);
+        if (MODE == kSG128) av = lds128(sc_a);
+        if (MODE == kSG256) {
+            const uint2 a2 = lds64(sc_a);
+            av = make_uint4(a2.x, a2.y, 0u, 0u);
+        }
+    } else {
+        const uint2 s2 = lds64(sgn_a);
+        sg = make_uint4(s2.x, s2.y, 0u, 0u);
+        if (MODE == kSG128) {
+            const uint2 a2 = lds64(sc_a);
+            av = make_uint4(a2.x, a2.y, 0u, 0u);
+        }
+        if (MODE == kSG256) av.x = lds32(sc_a);
     }
-    const uint32_t idx_row = st + r * 64;
+    const uint32_t idx_row = st + r * G::kRowB;
 #pragma unroll
     for (int m = 0; m < MT; ++m) u[m] = 0.0f;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < C; ++q) {
         const uint4 wq = lds128(idx_row + (((uint32_t)q ^ sw) << 4));
         const uint32_t sq = q == 0 ? sg.x : q == 1 ? sg.y : q == 2 ? sg.z : sg.w;
         const uint32_t tb = lut + (uint32_t)(q * 32 * kTab);  // tables of words 4q..4q+3 (256-aligned)
         float p0[MT], p1[MT], q0[MT], q1[MT], r0[MT], r1[MT], u0[MT], u1[MT];
-        word_sums<0, MT>(wq.x, sq & 0xffu, tb, p0, p1);
-        word_sums<8, MT>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
-        word_sums<16, MT>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
-        word_sums<24, MT>(wq.w, sq >> 24, tb, u0, u1);
+        word_sums<0, MT, G::kLut>(wq.x, sq & 0xffu, tb, p0, p1);
+        word_sums<8, MT, G::kLut>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
+        word_sums<16, MT, G::kLut>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
+        word_sums<24, MT, G::kLut>(wq.w, sq >> 24, tb, u0, u1);
         uint32_t ab = 0u;
         if (MODE == kSG128) ab = q == 0 ? av.x : q == 1 ? av.y : q == 2 ? av.z : av.w;
-        if (MODE == kSG256) ab = q < 2 ? av.x : av.y;
+        if (MODE == kSG256) ab = (W == 16 && q >= 2) ? av.y : av.x;
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             float e0, e1, f0, f1, g0, g1;
@@ -307,183 +433,266 @@ __device__ __forceinline__ void unit_row(uint32_t st, uint32_t lut, int r, float
     }
 }
 
-template <int MAXP, int MT>
+template <int MAXP, int MT, int W>
 __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_constant__ SParams<MAXP> P) {
-    using C = SCfg<MT>;
+    using C = SCfg<MT, W>;
+    using G = SGeo<W>;
     constexpr int S = C::kStages;
+    constexpr int L = C::kAhead;
     __shared__ int s_last;
     __shared__ int s_abort;
     // Shared addresses: the buffer is rounded up to 256 bytes, so every table
     // base is a multiple of 256 (a lookup's address replaces its low byte); the
     // XOR swizzles need only 16-byte alignment, since writer and reader apply them.
     const uint32_t stages = (smem_u32(g_smem) + 255u) & ~255u;
-    const uint32_t luts = stages + S * kSStage;  // table buffer s (MT tokens' tables) belongs to stage s
+    const uint32_t luts = stages + S * G::kStage;  // table buffer s (MT tokens' tables) belongs to stage s
     const uint32_t bars = luts + S * C::kLutStage;
     // ready(s): the stage's planes landed and its tables are built; empty(s): consumers are done with both
     auto ready = [&](int s) { return bars + 8u * (uint32_t)s; };
-    auto empty = [&](int s) { return bars + 32u + 8u * (uint32_t)s; };
-    const uint32_t bar_part = bars + 64u;  // every consumer stored its split-tile partial
-    const uint32_t bar_last = bars + 72u;  // the ticket's outcome is in s_last
+    auto empty = [&](int s) { return bars + 48u + 8u * (uint32_t)s; };
+    const uint32_t bar_part = bars + 96u;    // every consumer stored its split-tile partial
+    const uint32_t bar_last = bars + 104u;   // the ticket's outcome is in s_last
+    const uint32_t bar_phase = bars + 112u;  // every consumer finished the CTA's units of a phase
+    const uint32_t bar_gate = bars + 120u;   // the previous phase is complete on every CTA
 
     const int t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5;
-    const int u_begin = blockIdx.x * P.upc;
-    const int u_end = min(P.total_units, u_begin + P.upc);
-    if (u_begin >= u_end) return;
-    const int nu = u_end - u_begin;
+    const bool chain = P.phase_cnt != nullptr;
     if (t == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(ready(s), 2 * 32 * kSHelpers);  // one cp.async arrival and one table arrival per helper thread
+            mbar_init(ready(s), kSHelperThreads + G::kTabs);  // a cp.async arrival per helper, one per table
             mbar_init(empty(s), kSRows);
         }
         mbar_init(bar_part, kSRows);
         mbar_init(bar_last, 1);
+        mbar_init(bar_phase, kSRows);
+        mbar_init(bar_gate, 1);
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
     volatile int* abort_flag = &s_abort;
+    // units of this CTA over all phases
+    int nu = 0;
+    for (int ph = 0; ph < P.n_phases; ++ph) {
+        int b, e;
+        phase_range(P, ph, b, e);
+        nu += max(0, e - b);
+    }
 
     if (warp >= kSConsumers) {
-        // ---- helpers: unit j's copies and tables go to stage j % S once the
-        // consumers are done with unit j - S there
+        // ---- helpers: unit j's copies go to stage j % S once the consumers are done
+        // with unit j - S there; its tables follow L units later (after the previous
+        // phase completed on every CTA, for a unit that opens a phase)
         const int h = warp - kSConsumers;
         const int ht = t - 32 * kSConsumers;  // table (block of 4 activations) of the unit
-        UnitPos cu = locate(P, u_begin);
-        CopyRows cr;
-        copy_rows(P.p[cu.p], cu.rb, h, lane, cr);
-        // activations: token m's row of X starts K bf16 (words * 8 groups of 4) after token m-1's
-        uint2 xb[MT];
+        UnitCursor<MAXP> cc, tc;              // copy and table cursors
+        cc.seek(P, 0);
+        tc.seek(P, 0);
+        CopyRows<W> cr;
+        int cr_p = -1, cr_rb = -1;
+        int passed = 0;  // phases known complete on every CTA
+        int gates = 0;
+        for (int j = 0; j < nu + L; ++j) {
+            if (j < nu) {
+                const int s = j % S;
+                if (j >= S && !mbar_wait(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag, P.wait_cycles)) break;
+                const SProb& pr = P.p[cc.pos.p];
+                if (cc.pos.p != cr_p || cc.pos.rb != cr_rb) {
+                    copy_rows<W>(pr, cc.pos.rb, h, lane, cr);
+                    cr_p = cc.pos.p;
+                    cr_rb = cc.pos.rb;
+                }
+                copy_unit<W>(pr, cr, cc.pos.sub, stages + s * G::kStage, h, lane);
+                cp_async_arrive(ready(s));
+                cc.next(P);
+            }
+            const int jt = j - L;
+            if (jt >= 0 && jt < nu) {
+                const int s = jt % S;
+                if (chain && tc.ph > passed) {
+                    // the first tables of a phase read the previous phase's Y
+                    if (ht == 0 && grid_wait(P.phase_cnt + tc.ph - 1, (int)gridDim.x, abort_flag, P.wait_cycles))
+                        mbar_arrive(bar_gate);
+                    if (!mbar_wait(bar_gate, (uint32_t)(gates & 1), abort_flag, P.wait_cycles)) break;
+                    ++gates;
+                    __threadfence();
+                    passed = tc.ph;
+                }
+                const SProb& pt = P.p[tc.pos.p];
+                if (ht < G::kTabs) {
+                    // activations: token m's row of X starts K bf16 (words * 8 groups of 4) after token m-1's
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
-            xb[m] = __ldg(reinterpret_cast<const uint2*>(P.p[cu.p].X) + (int64_t)m * P.p[cu.p].words * 8 +
-                          cu.sub * kSTabs + ht);
-        for (int j = 0; j < nu; ++j) {
-            const int s = j % S;
-            if (j >= S && !mbar_wait(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag, P.wait_cycles)) break;
-            const SProb& pr = P.p[cu.p];
-            copy_unit(pr, cr, cu.sub, stages + s * kSStage, h, lane);
-            cp_async_arrive(ready(s));
-#pragma unroll
-            for (int m = 0; m < MT; ++m) build_table(luts + s * C::kLutStage + m * kSLut + ht * kTab, xb[m]);
-            mbar_arrive(ready(s));
-            const int p0 = cu.p, rb0 = cu.rb;
-            advance(P.p, cu);
-            if (j + 1 < nu) {
-                const SProb& pn = P.p[cu.p];
-                if (cu.p != p0 || cu.rb != rb0) copy_rows(pn, cu.rb, h, lane, cr);
-#pragma unroll
-                for (int m = 0; m < MT; ++m)
-                    xb[m] = __ldg(reinterpret_cast<const uint2*>(pn.X) + (int64_t)m * pn.words * 8 + cu.sub * kSTabs +
-                                  ht);
+                    for (int m = 0; m < MT; ++m) {
+                        const uint2 xb = __ldcg(reinterpret_cast<const uint2*>(pt.X) + (int64_t)m * pt.words * 8 +
+                                                tc.pos.sub * G::kTabs + ht);
+                        build_table(luts + s * C::kLutStage + m * G::kLut + ht * kTab, xb);
+                    }
+                    mbar_arrive(ready(s));
+                }
+                tc.next(P);
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-        return;
+    } else {
+        // ---- consumers: thread t owns row t of every unit
+        const int r = t;
+        float acc[MT];
+        int k = 0;       // units consumed so far (all phases): stage k % S
+        int events = 0;  // split tiles handled so far (phase of bar_part / bar_last)
+        int phases = 0;  // phases this CTA's consumers completed with units (phase of bar_phase)
+        bool ok = true;
+        for (int ph = 0; ph < P.n_phases && ok; ++ph) {
+            int u_begin, u_end;
+            phase_range(P, ph, u_begin, u_end);
+            const int pb = P.ph_unit[ph], upc = P.ph_upc[ph];
+            if (u_begin < u_end) {
+                UnitPos cur = locate(P, u_begin);
+                bool tile_from_start = (P.p[cur.p].unit_begin + cur.rb * P.p[cur.p].n_sub == u_begin);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+                for (int uu = u_begin; uu < u_end; ++uu, ++k) {
+                    const int s = k % S;
+                    if (!mbar_wait(ready(s), (uint32_t)((k / S) & 1), abort_flag, P.wait_cycles)) {
+                        ok = false;
+                        break;
+                    }
+                    const SProb& pr = P.p[cur.p];
+                    const uint32_t st = stages + s * G::kStage;
+                    const uint32_t lut = luts + s * C::kLutStage;
+                    float u[MT];
+                    if (pr.mode == kSRow)
+                        unit_row<kSRow, MT, W>(st, lut, r, u);
+                    else if (pr.mode == kSG128)
+                        unit_row<kSG128, MT, W>(st, lut, r, u);
+                    else
+                        unit_row<kSG256, MT, W>(st, lut, r, u);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) acc[m] += u[m];
+                    mbar_arrive(empty(s));
+
+                    const bool tile_end = (cur.sub == pr.n_sub - 1);
+                    if (tile_end || uu == u_end - 1) {
+                        const int n = cur.rb * kSRows + r;
+                        const bool row_ok = n < pr.N;
+                        float v[MT];
+                        const float rs =
+                            (pr.mode == kSRow && row_ok) ? __ldg(pr.scales + (pr.per_tensor ? 0 : n)) : 1.0f;
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) v[m] = pr.mode == kSRow ? acc[m] * rs : acc[m];
+                        if (tile_from_start && tile_end) {
+                            if (row_ok) {
+#pragma unroll
+                                for (int m = 0; m < MT; ++m) {
+                                    if (P.y_bf16)
+                                        reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)m * pr.N + n] =
+                                            __float2bfloat16_rn(v[m]);
+                                    else
+                                        reinterpret_cast<float*>(pr.Y)[(int64_t)m * pr.N + n] = v[m];
+                                }
+                            }
+                        } else {
+                            // split tile: partials into this CTA's slot, then the ticket
+                            const int tile = pr.tile_begin + cur.rb;
+                            const int tile_u0 = pr.unit_begin + cur.rb * pr.n_sub;
+                            const int c_a = (tile_u0 - pb) / upc;
+                            const int c_b = (tile_u0 + pr.n_sub - 1 - pb) / upc;
+                            const int slot = (u_begin >= tile_u0) ? 0 : 1;
+#pragma unroll
+                            for (int m = 0; m < MT; ++m)
+                                __stcg(P.part + (((int64_t)blockIdx.x * 2 + slot) * MT + m) * kSRows + r, v[m]);
+                            __threadfence();
+                            mbar_arrive(bar_part);
+                            const uint32_t ph2 = (uint32_t)(events & 1);
+                            ++events;
+                            if (r == 0) {
+                                if (!mbar_wait(bar_part, ph2, abort_flag, P.wait_cycles)) {
+                                    ok = false;
+                                    break;
+                                }
+                                s_last = (atomicAdd(P.ticket + tile, 1) == c_b - c_a);
+                                mbar_arrive(bar_last);
+                            }
+                            if (!mbar_wait(bar_last, ph2, abort_flag, P.wait_cycles)) {
+                                ok = false;
+                                break;
+                            }
+                            if (s_last) {
+                                __threadfence();
+#pragma unroll
+                                for (int m = 0; m < MT; ++m) {
+                                    float sum = 0.0f;
+                                    for (int c = c_a; c <= c_b; ++c) {
+                                        const int sl = (pb + c * upc >= tile_u0) ? 0 : 1;
+                                        const float pv = __ldcg(P.part + (((int64_t)c * 2 + sl) * MT + m) * kSRows + r);
+                                        sum = (c == c_a) ? pv : sum + pv;
+                                    }
+                                    if (row_ok) {
+                                        if (P.y_bf16)
+                                            reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)m * pr.N + n] =
+                                                __float2bfloat16_rn(sum);
+                                        else
+                                            reinterpret_cast<float*>(pr.Y)[(int64_t)m * pr.N + n] = sum;
+                                    }
+                                }
+                                if (r == 0) P.ticket[tile] = 0;  // leave the ticket zeroed
+                            }
+                        }
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+                        tile_from_start = true;  // every later tile of this range starts inside it
+                    }
+                    advance(P.p, cur);
+                }
+                if (!ok) break;
+                if (chain) {
+                    // every consumer's Y of this phase is written before the CTA's arrival
+                    __threadfence();
+                    mbar_arrive(bar_phase);
+                    if (r == 0) {
+                        if (!mbar_wait(bar_phase, (uint32_t)(phases & 1), abort_flag, P.wait_cycles)) {
+                            ok = false;
+                            break;
+                        }
+                        __threadfence();
+                        atomicAdd(P.phase_cnt + ph, 1);
+                    }
+                    ++phases;
+                }
+            } else if (chain && r == 0) {
+                atomicAdd(P.phase_cnt + ph, 1);  // nothing of this phase here
+            }
+        }
     }
 
-    // ---- consumers: thread t owns row t of every unit
-    const int r = t;
-    UnitPos cur = locate(P, u_begin);
-    bool tile_from_start = (P.p[cur.p].unit_begin + cur.rb * P.p[cur.p].n_sub == u_begin);
-    float acc[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
-    int events = 0;  // split tiles handled so far (phase of bar_part / bar_last)
-    for (int k = 0; k < nu; ++k) {
-        const int s = k % S;
-        if (!mbar_wait(ready(s), (uint32_t)((k / S) & 1), abort_flag, P.wait_cycles)) break;
-        const SProb& pr = P.p[cur.p];
-        const uint32_t st = stages + s * kSStage;
-        const uint32_t lut = luts + s * C::kLutStage;
-        float u[MT];
-        if (pr.mode == kSRow)
-            unit_row<kSRow, MT>(st, lut, r, u);
-        else if (pr.mode == kSG128)
-            unit_row<kSG128, MT>(st, lut, r, u);
-        else
-            unit_row<kSG256, MT>(st, lut, r, u);
-#pragma unroll
-        for (int m = 0; m < MT; ++m) acc[m] += u[m];
-        mbar_arrive(empty(s));
-
-        const bool tile_end = (cur.sub == pr.n_sub - 1);
-        if (tile_end || k == nu - 1) {
-            const int n = cur.rb * kSRows + r;
-            const bool row_ok = n < pr.N;
-            float v[MT];
-            const float rs = (pr.mode == kSRow && row_ok) ? __ldg(pr.scales + (pr.per_tensor ? 0 : n)) : 1.0f;
-#pragma unroll
-            for (int m = 0; m < MT; ++m) v[m] = pr.mode == kSRow ? acc[m] * rs : acc[m];
-            if (tile_from_start && tile_end) {
-                if (row_ok) {
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        if (P.y_bf16)
-                            reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)m * pr.N + n] = __float2bfloat16_rn(v[m]);
-                        else
-                            reinterpret_cast<float*>(pr.Y)[(int64_t)m * pr.N + n] = v[m];
-                    }
-                }
-            } else {
-                // split tile: partials into this CTA's slot, then the ticket
-                const int tile = pr.tile_begin + cur.rb;
-                const int tile_u0 = pr.unit_begin + cur.rb * pr.n_sub;
-                const int c_a = tile_u0 / P.upc;
-                const int c_b = (tile_u0 + pr.n_sub - 1) / P.upc;
-                const int slot = (u_begin >= tile_u0) ? 0 : 1;
-#pragma unroll
-                for (int m = 0; m < MT; ++m)
-                    __stcg(P.part + (((int64_t)blockIdx.x * 2 + slot) * MT + m) * kSRows + r, v[m]);
-                __threadfence();
-                mbar_arrive(bar_part);
-                const uint32_t ph = (uint32_t)(events & 1);
-                ++events;
-                if (r == 0) {
-                    if (!mbar_wait(bar_part, ph, abort_flag, P.wait_cycles)) break;
-                    s_last = (atomicAdd(P.ticket + tile, 1) == c_b - c_a);
-                    mbar_arrive(bar_last);
-                }
-                if (!mbar_wait(bar_last, ph, abort_flag, P.wait_cycles)) break;
-                if (s_last) {
-                    __threadfence();
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        float sum = 0.0f;
-                        for (int c = c_a; c <= c_b; ++c) {
-                            const int sl = (c * P.upc >= tile_u0) ? 0 : 1;
-                            const float pv = __ldcg(P.part + (((int64_t)c * 2 + sl) * MT + m) * kSRows + r);
-                            sum = (c == c_a) ? pv : sum + pv;
-                        }
-                        if (row_ok) {
-                            if (P.y_bf16)
-                                reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)m * pr.N + n] = __float2bfloat16_rn(sum);
-                            else
-                                reinterpret_cast<float*>(pr.Y)[(int64_t)m * pr.N + n] = sum;
-                        }
-                    }
-                    if (r == 0) P.ticket[tile] = 0;  // leave the ticket zeroed
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
-            tile_from_start = true;  // every later tile of this range starts inside it
+    __syncthreads();
+    if (chain && t == 0 && !*abort_flag) {
+        // the last CTA to leave zeroes the phase counters for the next launch
+        __threadfence();
+        if (atomicAdd(P.phase_cnt + P.n_phases, 1) == (int)gridDim.x - 1) {
+            for (int ph = 0; ph <= P.n_phases; ++ph) P.phase_cnt[ph] = 0;
+            __threadfence();
         }
-        advance(P.p, cur);
     }
 }
 
 // ---- host side -------------------------------------------------------------------
 
-bool stream_eligible(const ProbShape& s, int64_t M) {
+// Units of W words: K a multiple of 32 W; group scales of 128 or 256 weights
+// (whole groups per unit), or row scales.
+template <int W>
+static bool stream_eligible_w(const ProbShape& s, int64_t M) {
     if ((M != 1 && M != 2) || s.N == 0) return false;
-    if ((s.N + kSRows - 1) / kSRows > kMaxTickets) return false;
-    if (s.K % 512 != 0) return false;
+    if ((s.N + kSRows - 1) / kSRows > kMaxTickets - kChainCtrs) return false;
+    if (s.K % (32 * W) != 0) return false;
     if (s.N * (s.K / 8) >= (int64_t(1) << 32) - 64) return false;  // 32-bit byte offsets into the planes
     if (s.granularity == SHERRY_PER_TENSOR || s.granularity == SHERRY_PER_CHANNEL) return true;
     if (s.granularity != SHERRY_PER_GROUP) return false;
-    return s.group == 128 || s.group == 256;  // K % 512 == 0: 4 or 2 whole groups per unit
+    return s.group == 128 || s.group == 256;
 }
+
+bool stream_eligible(const ProbShape& s, int64_t M) { return stream_eligible_w<16>(s, M); }
+bool chain_eligible(const ProbShape& s, int64_t M) { return stream_eligible_w<8>(s, M); }
 
 int64_t stream_tiles(const ProbShape& s) { return (s.N + kSRows - 1) / kSRows; }
 
@@ -496,13 +705,16 @@ long long stream_set_wait_cycles(long long cycles) {
 
 struct SPlan {
     std::vector<SProb> probs;
-    int total_units = 0, total_tiles = 0, grid = 0, upc = 0;
+    std::vector<int> ph_unit, ph_upc;
+    int total_units = 0, total_tiles = 0, grid = 0;
     size_t ws_bytes = 0, part_off = 0;
 };
 
-static int stream_ctas(int sms) { return sms; }  // one CTA per SM (the stages fill shared memory)
-
-static SPlan make_splan(const ProbShape* shapes, int count, int64_t M, int sms) {
+// phase_begin: n_phases + 1 problem indices (null: one phase of all problems).
+// Independent problems: one CTA per SM at most (the stages fill shared memory)
+// and no more CTAs than units; chained phases: one CTA per SM (cooperative).
+static SPlan make_splan(const ProbShape* shapes, int count, const int* phase_begin, int n_phases, int64_t M,
+                        int sms, int W) {
     SPlan pl;
     int ub = 0, tb = 0;
     for (int i = 0; i < count; ++i) {
@@ -514,7 +726,7 @@ static SPlan make_splan(const ProbShape* shapes, int count, int64_t M, int sms) 
         p.mode = s.granularity != SHERRY_PER_GROUP ? kSRow : (s.group == 128 ? kSG128 : kSG256);
         p.per_tensor = s.granularity == SHERRY_PER_TENSOR;
         p.n_rb = (int)((s.N + kSRows - 1) / kSRows);
-        p.n_sub = (p.words + kSWords - 1) / kSWords;
+        p.n_sub = (p.words + W - 1) / W;
         p.unit_begin = ub;
         p.tile_begin = tb;
         ub += p.n_rb * p.n_sub;
@@ -523,20 +735,38 @@ static SPlan make_splan(const ProbShape* shapes, int count, int64_t M, int sms) 
     }
     pl.total_units = ub;
     pl.total_tiles = tb;
-    const int g = std::max(1, std::min(stream_ctas(sms), ub));
-    pl.upc = (ub + g - 1) / g;
-    pl.grid = (ub + pl.upc - 1) / pl.upc;
+    if (phase_begin == nullptr) {
+        const int g = std::max(1, std::min(sms, ub));
+        const int upc = std::max(1, (ub + g - 1) / g);
+        pl.ph_unit = {0, ub};
+        pl.ph_upc = {upc};
+        pl.grid = std::max(1, (ub + upc - 1) / upc);
+    } else {
+        pl.grid = std::max(1, sms);
+        for (int ph = 0; ph < n_phases; ++ph) {
+            const int b = phase_begin[ph] < count ? pl.probs[phase_begin[ph]].unit_begin : ub;
+            const int e = phase_begin[ph + 1] < count ? pl.probs[phase_begin[ph + 1]].unit_begin : ub;
+            pl.ph_unit.push_back(b);
+            pl.ph_upc.push_back(std::max(1, (e - b + pl.grid - 1) / pl.grid));
+        }
+        pl.ph_unit.push_back(ub);
+    }
     pl.part_off = kTicketBytes;
     pl.ws_bytes = kTicketBytes + (size_t)pl.grid * 2 * (size_t)M * kSRows * sizeof(float);
     return pl;
 }
 
 size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
-    return make_splan(shapes, count, M, sms).ws_bytes;
+    return make_splan(shapes, count, nullptr, 1, M, sms, 16).ws_bytes;
 }
 
-template <int MAXP, int MT>
-static int stream_launch_t(SPlan& pl, int y_bf16, void* workspace, cudaStream_t stream) {
+size_t chain_workspace_bytes(const ProbShape* shapes, int count, const int* phase_begin, int n_phases, int64_t M,
+                             int sms) {
+    return make_splan(shapes, count, phase_begin, n_phases, M, sms, 8).ws_bytes;
+}
+
+template <int MAXP, int MT, int W>
+static int stream_launch_t(SPlan& pl, int y_bf16, void* workspace, bool chain, cudaStream_t stream) {
     static SParams<MAXP> P;
     static std::mutex mu;
     static PerDevice attr;
@@ -544,35 +774,49 @@ static int stream_launch_t(SPlan& pl, int y_bf16, void* workspace, cudaStream_t 
     P.wait_cycles = g_stream_wait.load();
     P.count = (int)pl.probs.size();
     P.y_bf16 = y_bf16;
-    P.total_units = pl.total_units;
-    P.upc = pl.upc;
+    P.n_phases = (int)pl.ph_upc.size();
     P.ticket = static_cast<int*>(workspace);
     P.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.part_off);
+    P.phase_cnt = chain ? static_cast<int*>(workspace) + (kMaxTickets - kChainCtrs) : nullptr;
     for (int i = 0; i < P.count; ++i) P.p[i] = pl.probs[i];
+    for (int i = 0; i <= P.n_phases; ++i) P.ph_unit[i] = pl.ph_unit[i];
+    for (int i = 0; i < P.n_phases; ++i) P.ph_upc[i] = pl.ph_upc[i];
     int done = 0;
     const int st = per_device(attr, &done, [](int& v) {
-        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_lut_stream<MAXP, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               SCfg<MT>::kSmem));
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_lut_stream<MAXP, MT, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               SCfg<MT, W>::kSmem));
         v = 1;
         return SHERRY_OK;
     });
     if (st) return st;
-    k_lut_stream<MAXP, MT><<<pl.grid, kSThreads, SCfg<MT>::kSmem, stream>>>(P);
+    if (!chain) {
+        k_lut_stream<MAXP, MT, W><<<pl.grid, kSThreads, SCfg<MT, W>::kSmem, stream>>>(P);
+    } else {
+        // every CTA must be resident: the phase barrier waits for all of them
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)pl.grid);
+        cfg.blockDim = dim3(kSThreads);
+        cfg.dynamicSmemBytes = SCfg<MT, W>::kSmem;
+        cfg.stream = stream;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeCooperative;
+        at[0].val.cooperative = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        SHERRY_CUDA_CHECK(cudaLaunchKernelEx(&cfg, k_lut_stream<MAXP, MT, W>, P));
+    }
     SHERRY_LAUNCH_CHECK();
     return SHERRY_OK;
 }
 
-template <int MT>
-static int stream_launch_mt(SPlan& pl, int count, int y_bf16, void* workspace, cudaStream_t stream) {
-    if (count <= 1) return stream_launch_t<1, MT>(pl, y_bf16, workspace, stream);
-    if (count <= 16) return stream_launch_t<16, MT>(pl, y_bf16, workspace, stream);
-    return stream_launch_t<SHERRY_MAX_BATCH, MT>(pl, y_bf16, workspace, stream);
+template <int MT, int W>
+static int stream_launch_mt(SPlan& pl, int slots, int y_bf16, void* workspace, bool chain, cudaStream_t stream) {
+    if (slots <= 1) return stream_launch_t<1, MT, W>(pl, y_bf16, workspace, chain, stream);
+    if (slots <= 16) return stream_launch_t<16, MT, W>(pl, y_bf16, workspace, chain, stream);
+    return stream_launch_t<SHERRY_MAX_BATCH, MT, W>(pl, y_bf16, workspace, chain, stream);
 }
 
-int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
-                         void* workspace, int sms, cudaStream_t stream) {
-    if (M != 1 && M != 2) return SHERRY_ERR_UNSUPPORTED;
-    SPlan pl = make_splan(shapes, count, M, sms);
+static void attach(SPlan& pl, const sherry_linear_desc* descs, int count) {
     for (int i = 0; i < count; ++i) {
         SProb& p = pl.probs[i];
         p.X = descs[i].X;
@@ -581,9 +825,38 @@ int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* desc
         p.scales = descs[i].scales;
         p.Y = descs[i].Y;
     }
+}
+
+int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
+                         void* workspace, int sms, cudaStream_t stream) {
+    if (M != 1 && M != 2) return SHERRY_ERR_UNSUPPORTED;
+    SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, 16);
+    attach(pl, descs, count);
     if (pl.total_units == 0) return SHERRY_OK;
-    return M == 1 ? stream_launch_mt<1>(pl, count, y_bf16, workspace, stream)
-                  : stream_launch_mt<2>(pl, count, y_bf16, workspace, stream);
+    return M == 1 ? stream_launch_mt<1, 16>(pl, count, y_bf16, workspace, false, stream)
+                  : stream_launch_mt<2, 16>(pl, count, y_bf16, workspace, false, stream);
+}
+
+bool chain_launch_ok(const ProbShape* shapes, int count, int n_phases, int64_t M) {
+    if ((M != 1 && M != 2) || n_phases > kSMaxPhases || n_phases > SHERRY_MAX_BATCH || count > SHERRY_MAX_BATCH)
+        return false;
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        if (!chain_eligible(shapes[i], M)) return false;
+        tiles += stream_tiles(shapes[i]);
+    }
+    return tiles <= kMaxTickets - kChainCtrs;
+}
+
+int chain_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, const int* phase_begin,
+                        int n_phases, int64_t M, int y_bf16, void* workspace, int sms, cudaStream_t stream) {
+    if (!chain_launch_ok(shapes, count, n_phases, M)) return SHERRY_ERR_UNSUPPORTED;
+    SPlan pl = make_splan(shapes, count, phase_begin, n_phases, M, sms, 8);
+    attach(pl, descs, count);
+    // the kernel's phase table has one slot per problem slot of its instantiation
+    const int slots = std::max(count, n_phases);
+    return M == 1 ? stream_launch_mt<1, 8>(pl, slots, y_bf16, workspace, true, stream)
+                  : stream_launch_mt<2, 8>(pl, slots, y_bf16, workspace, true, stream);
 }
 
 int stream_status_take() {

@@ -222,3 +222,22 @@ def test_wait_budget_setter(L):
     prev = L.sherry_set_wait_budget(1000)
     assert L.sherry_set_wait_budget(0) == 1000
     assert L.sherry_set_wait_budget(prev) > 1000  # the default (about 2 s of clock cycles)
+
+
+def test_linear_chain_validation(L):
+    D = _abi.LinearDesc
+    good = D(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 256, _abi.PER_GROUP, 128)
+    arr = (D * 2)(good, good)
+    pb = lambda *v: (ctypes.c_int * len(v))(*v)
+    ch = L.sherry_linear_chain
+    assert ch(arr, 2, None, 1, 1, _abi.F32, None, 0, None) == _abi.ERR_NULL
+    assert ch(arr, 2, pb(0, 1), 1, 1, _abi.F32, None, 0, None) == _abi.ERR_SHAPE      # last bound != count
+    assert ch(arr, 2, pb(1, 2), 1, 1, _abi.F32, None, 0, None) == _abi.ERR_SHAPE      # first bound != 0
+    assert ch(arr, 2, pb(0, 2, 1, 2), 3, 1, _abi.F32, None, 0, None) == _abi.ERR_SHAPE  # decreasing
+    assert ch(arr, 2, pb(0, 1, 2), 0, 1, _abi.F32, None, 0, None) == _abi.ERR_SHAPE   # no phase
+    assert ch(arr, 2, pb(0, 1, 2), 2, 1, 7, None, 0, None) == _abi.ERR_DTYPE
+    bad = (D * 2)(good, D(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 48, _abi.PER_GROUP, 128))
+    assert ch(bad, 2, pb(0, 1, 2), 2, 1, _abi.F32, None, 0, None) == _abi.ERR_SHAPE
+    assert L.sherry_linear_chain_workspace_bytes(bad, 2, pb(0, 1, 2), 2, 1) == 0
+    # M = 0: nothing to do
+    assert ch(arr, 2, pb(0, 1, 2), 2, 0, _abi.F32, None, 0, None) == _abi.OK
