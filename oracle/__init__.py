@@ -70,6 +70,10 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.sherry_ref_linear.restype = i32
     L.sherry_ref_fake_quant.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp]
     L.sherry_ref_fake_quant.restype = i32
+    L.sherry_ref_tequila_dead.argtypes = [vp, i32, i64, i64, ctypes.c_float, vp, vp]
+    L.sherry_ref_tequila_dead.restype = i32
+    L.sherry_ref_tequila_term.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, vp]
+    L.sherry_ref_tequila_term.restype = i32
     L.sherry_ref_threads.argtypes = []
     L.sherry_ref_threads.restype = i32
     return L
@@ -162,6 +166,30 @@ class Oracle:
         if st:
             raise ValueError(f"oracle fake_quant status {st}")
         return Wq, Wb
+
+    def tequila_dead(self, W, eps, w_dtype=None):
+        """(D bf16 bits [N, K/4], bias float32 [N]): the zeroed weight of every block times eps."""
+        W = np.ascontiguousarray(W)
+        if w_dtype is None:
+            w_dtype = BF16 if W.dtype == np.uint16 else F32
+        N, K = W.shape
+        D = np.empty((N, K // 4), np.uint16)
+        bias = np.empty(N, np.float32)
+        st = self.L.sherry_ref_tequila_dead(_p(W), w_dtype, N, K, float(eps), _p(D), _p(bias))
+        if st:
+            raise ValueError(f"oracle tequila_dead status {st}")
+        return D, bias
+
+    def tequila_term(self, X_bf16, idx, D, bias, N, K, mode):
+        """The dead-weight term T [M, N] (float64); mode 0: bias, 1: sign(X) D^T."""
+        X = np.ascontiguousarray(X_bf16, np.uint16)
+        M = X.shape[0]
+        T = np.zeros((M, N), np.float64)
+        st = self.L.sherry_ref_tequila_term(_p(X), M, _p(np.ascontiguousarray(idx)), _p(np.ascontiguousarray(D)),
+                                            _p(np.ascontiguousarray(bias, np.float32)), N, K, mode, _p(T))
+        if st:
+            raise ValueError(f"oracle tequila_term status {st}")
+        return T
 
     def threads(self) -> int:
         return int(self.L.sherry_ref_threads())

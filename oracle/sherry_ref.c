@@ -261,6 +261,68 @@ int sherry_ref_fake_quant(const void* W, int w_dtype, int64_t N, int64_t K, int 
     return SHERRY_REF_OK;
 }
 
+/* ---- Tequila-style dead-weight term: the zeroed weight of every block, times
+ * eps, rounded to bf16; its row sums for the "ones" input. ---- */
+int sherry_ref_tequila_dead(const void* W, int w_dtype, int64_t N, int64_t K, float eps, uint16_t* D, float* bias) {
+    int st = check_shape(N, K);
+    if (st) return st;
+    if (w_dtype != SHERRY_REF_F32 && w_dtype != SHERRY_REF_BF16) return SHERRY_REF_ERR_DTYPE;
+    if (N > 0 && (!W || !D)) return SHERRY_REF_ERR_NULL;
+    const int64_t nb = K / 4;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n) {
+        float* dv = (float*)malloc((size_t)nb * sizeof(float));
+        if (!dv) abort();
+        for (int64_t b = 0; b < nb; ++b) {
+            float wv[4], mag[4];
+            for (int i = 0; i < 4; ++i) {
+                int64_t off = n * K + 4 * b + i;
+                wv[i] = (w_dtype == SHERRY_REF_F32) ? ((const float*)W)[off]
+                                                    : bf16_bits_to_f32(((const uint16_t*)W)[off]);
+            }
+            unsigned nib, g;
+            encode_block(wv, &nib, &g, mag);
+            const float dead = eps * wv[nib >> 2];
+            D[n * nb + b] = f32_to_bf16_rne(dead);
+            dv[b] = bf16_bits_to_f32(D[n * nb + b]);
+        }
+        if (bias) bias[n] = sherry_ref_pairsum(dv, nb);
+        free(dv);
+    }
+    return SHERRY_REF_OK;
+}
+
+int sherry_ref_tequila_term(const uint16_t* X, int64_t M, const uint32_t* idx, const uint16_t* D,
+                            const float* bias, int64_t N, int64_t K, int mode, double* T) {
+    int st = check_shape(N, K);
+    if (st) return st;
+    if (M < 0 || (mode != 0 && mode != 1)) return SHERRY_REF_ERR_SHAPE;
+    if (M > 0 && N > 0 && (!T || (mode == 0 && !bias) || (mode == 1 && (!X || !idx || !D))))
+        return SHERRY_REF_ERR_NULL;
+    const int64_t words = K / 32, nb = K / 4;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0;
+            if (mode == 0) {
+                acc = (double)bias[n];
+            } else {
+                for (int64_t b = 0; b < nb; ++b) {
+                    const unsigned z = (idx[n * words + b / 8] >> (4 * (b % 8) + 2)) & 3u;
+                    const float x = bf16_bits_to_f32(X[m * K + 4 * b + z]);
+                    const double sx = (x > 0.0f) ? 1.0 : ((x < 0.0f) ? -1.0 : 0.0);
+                    acc += sx * (double)bf16_bits_to_f32(D[n * nb + b]);
+                }
+            }
+            T[m * N + n] = acc;
+        }
+    return SHERRY_REF_OK;
+}
+
 /* ternary value of weight (n, k) decoded from the planes */
 static int ternary_at(const uint32_t* idx, const uint8_t* sgn, int64_t n, int64_t k, int64_t K) {
     int64_t words = K / 32;

@@ -91,6 +91,23 @@ int sherry_ref_linear(const uint16_t* X, int64_t M, const int64_t* rows, int64_t
 int sherry_ref_fake_quant(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
                           float* Wq, uint16_t* Wb);
 
+/* Tequila-style dead-weight term on Sherry's weights ("Sherry, Tequila and
+ * Fairies in Python", sections 1.2 and 2.1: UltraQuantV2 keeps the weights the
+ * ternary quantiser sets to zero as B = eps * w, and UltraQuantLinear adds
+ * F.linear(ones, B) -- or F.linear(sign(x), B) -- to F.linear(x, A)).  Here the
+ * zeroed weights are Sherry's: the smallest |w| of every block of 4.
+ * D [N][K/4] bf16 bits: round-to-nearest-even of the fp32 product eps * w at the
+ * zeroed position of each block (B cast to the activations' bf16, as the page
+ * does before the linear); bias [N] (optional): the canonical pairwise fp32 sum
+ * of D[n][*] as fp32 values, i.e. F.linear(ones, B). */
+int sherry_ref_tequila_dead(const void* W, int w_dtype, int64_t N, int64_t K, float eps, uint16_t* D, float* bias);
+
+/* The term added to Y [M][N] (fp64): mode 0 (ones): T[m][n] = bias[n]; mode 1
+ * (signs of the activations): T[m][n] = sum_b sign(x[m][4b + z(n, b)]) * D[n][b],
+ * sign(0) = 0 as torch.sign, z the zero position of block b in the idx plane. */
+int sherry_ref_tequila_term(const uint16_t* X, int64_t M, const uint32_t* idx, const uint16_t* D,
+                            const float* bias, int64_t N, int64_t K, int mode, double* T);
+
 /* number of threads the build uses (1 unless built with OpenMP) */
 int sherry_ref_threads(void);
 

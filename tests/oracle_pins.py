@@ -432,6 +432,63 @@ def pin_fake_quant(orc: oracle.Oracle):
     assert np.array_equal(Wq, expected_ternary(W2).astype(np.float32) * np.repeat(np.exp2(e), 128, axis=1))
 
 
-ALL_PINS = [pin_fake_quant, pin_topk_reading, pin_code_bijection, pin_argmin_bruteforce, pin_hand_worked, pin_sparsity,
+# ---------------------------------------------------------------- Tequila-style dead-weight term
+
+def pin_tequila(orc: oracle.Oracle):
+    """The dead-weight term ("Sherry, Tequila and Fairies in Python", sections 1.2,
+    2.1: B = eps * w where the quantiser zeroes w, then F.linear(ones, B) or
+    F.linear(sign(x), B)), with Sherry's zeroed weight (smallest |w| per block):
+    * D = torch's bf16 cast of eps * w at the zero position found by a stable
+      sort (ties to the lowest index);
+    * bias = F.linear(ones, B) and the sign term = F.linear(sign(X), B), both in
+      float64 torch, within the summation-order bound;
+    * one-hot activations pick single D entries; an activation of 0 at the zeroed
+      position contributes nothing (torch.sign(0) = 0);
+    * exact sums for equal powers of two."""
+    import torch
+    N, K, M = 16, 256, 3
+    eps = np.float32(1e-2)
+    W = synth.weights_student_t(N, K, seed=901)
+    D, bias = orc.tequila_dead(W, eps)
+    t = expected_ternary(W)
+    dead = np.where(t == 0, W * eps, np.float32(0)).astype(np.float32)            # B before the cast
+    Bb = torch.from_numpy(dead).to(torch.bfloat16)
+    d_ref = Bb.float().numpy().reshape(N, K // 4, 4).sum(-1)                      # one nonzero per block
+    assert np.array_equal(D, torch.from_numpy(d_ref).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    ones = torch.ones((1, K), dtype=torch.float64)
+    b_ref = torch.nn.functional.linear(ones, Bb.double()).numpy()[0]
+    L = K // 4
+    assert np.all(np.abs(bias - b_ref) <= (math.ceil(math.log2(L)) + 1) * 2.0 ** -24 * Bb.double().abs().sum(1).numpy())
+    idx, sgn, sc = orc.quantize_pack(W, oracle.PER_GROUP, 128)
+    Xb = synth.activations_bf16(M, K, seed=902)
+    Xb[0, ::5] = 0                                                                 # some exact zeros
+    X = torch.from_numpy(synth.bf16_bits_to_f32(Xb)).double()
+    T1 = orc.tequila_term(Xb, idx, D, bias, N, K, 1)
+    ref1 = torch.nn.functional.linear(torch.sign(X), Bb.double()).numpy()
+    assert np.all(np.abs(T1 - ref1) <= 1e-12 * (Bb.double().abs().sum(1).numpy() + 1e-30))
+    T0 = orc.tequila_term(Xb, idx, D, bias, N, K, 0)
+    assert np.array_equal(T0, np.broadcast_to(bias.astype(np.float64), (M, N)))
+    # one-hot activations: k at the zeroed position of row n picks D[n][k/4]
+    for k in (0, 5, 130, 255):
+        Xo = np.zeros((1, K), np.uint16)
+        Xo[0, k] = synth.f32_to_bf16_bits(np.array([-3.0], np.float32))[0]
+        To = orc.tequila_term(Xo, idx, D, bias, N, K, 1)[0]
+        want = np.where(t[:, k] == 0, -synth.bf16_bits_to_f32(D[:, k // 4]).astype(np.float64), 0.0)
+        assert np.array_equal(To, want), k
+    # a zero activation at every zeroed position: no term at all
+    Xz = np.tile(synth.f32_to_bf16_bits(np.ones((1, K), np.float32)), (N, 1))
+    Xz[t == 0] = 0
+    for n in range(N):
+        assert orc.tequila_term(Xz[n:n + 1], idx, D, bias, N, K, 1)[0, n] == 0.0
+    # equal powers of two: D exact and the sums exact
+    W2 = np.where(synth.rng(903).random((4, 128)) < 0.5, -1.0, 1.0).astype(np.float32) * np.float32(2.0 ** -3)
+    D2, b2 = orc.tequila_dead(W2, np.float32(2.0 ** -7))
+    t2 = expected_ternary(W2)
+    z_sign = np.where(np.sign(W2)[t2 == 0] >= 0, 1.0, -1.0).reshape(4, 32)
+    assert np.array_equal(synth.bf16_bits_to_f32(D2), (z_sign * 2.0 ** -10).astype(np.float32))
+    assert np.array_equal(b2, (z_sign.sum(1) * 2.0 ** -10).astype(np.float32))
+
+
+ALL_PINS = [pin_tequila, pin_fake_quant, pin_topk_reading, pin_code_bijection, pin_argmin_bruteforce, pin_hand_worked, pin_sparsity,
             pin_scale_power_of_two, pin_scale_closed_form, pin_c_vs_numpy, pin_bf16_input,
             pin_unpack_bf16, pin_linear, pin_errors, pin_pairsum_tree]

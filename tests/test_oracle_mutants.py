@@ -37,6 +37,11 @@ MUTANTS = {
                                 "sgn[n * words + b / 8] |= (uint8_t)(g << (7 - b % 8));"),
     "pad_with_one": ("buf[i] = (i < L) ? v[i] : 0.0f;", "buf[i] = (i < L) ? v[i] : 1.0f;"),
     "group_error_not_checked": ("(group % 32) != 0 || ", ""),
+    "tequila_dead_from_first_weight": ("const float dead = eps * wv[nib >> 2];", "const float dead = eps * wv[0];"),
+    "tequila_sign_of_zero_positive": ("const double sx = (x > 0.0f) ? 1.0 : ((x < 0.0f) ? -1.0 : 0.0);",
+                                      "const double sx = (x >= 0.0f) ? 1.0 : -1.0;"),
+    "tequila_zero_position_low_bits": ("const unsigned z = (idx[n * words + b / 8] >> (4 * (b % 8) + 2)) & 3u;",
+                                       "const unsigned z = (idx[n * words + b / 8] >> (4 * (b % 8))) & 3u;"),
     "fake_quant_zero_keeps_sign": ("sgn[n * K + 4 * b + i] = (int8_t)((i == z) ? 0 : ((wv[i] >= 0.0f) ? 1 : -1));",
                                    "sgn[n * K + 4 * b + i] = (int8_t)((wv[i] >= 0.0f) ? 1 : -1);"),
     "fake_quant_scale_from_next_domain": ("for (int64_t k = j * L; k < j * L + L; ++k) Wq[n * K + k] = (float)sgn[n * K + k] * a;",
