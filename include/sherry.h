@@ -132,6 +132,37 @@ int sherry_fake_quant(const void* W, int w_dtype, int64_t N, int64_t K, int gran
                       void* Wq, int wq_dtype, uint32_t* idx, uint8_t* sgn, float* scales,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Tequila-style dead-weight term ----------------------------------------
+ * "Sherry, Tequila and Fairies in Python", sections 1.2 and 2.1 (UltraQuantV2,
+ * UltraQuantLinear): the weights a ternary quantiser zeroes are kept as
+ * B = eps * w and add F.linear(ones, B) or F.linear(sign(x), B) to the layer.
+ * Here the zeroed weights are Sherry's (the smallest |w| of every block of 4).
+ * sherry_quantize_pack_tequila quantises and packs as sherry_quantize_pack (same
+ * planes, scales, workspace) and, in the same pass over W, writes
+ *   D      bf16 [N][K/4]: round-to-nearest-even of the fp32 product eps * w at
+ *          the zeroed position of each block (16-byte aligned)
+ *   bias   fp32 [N] (optional, NULL: none): the canonical pairwise fp32 sum of
+ *          the row's D values = F.linear(ones, B)
+ * sherry_linear_tequila computes Y = X (T alpha)^T + term with
+ *   mode SHERRY_TEQUILA_ONES: term[m][n] = bias[n]
+ *   mode SHERRY_TEQUILA_SIGN: term[m][n] = sum_b sign(X[m][4b + z(n,b)]) D[n][b]
+ *        (sign(0) = 0), z the zero position recorded in idx
+ * the linear by its usual kernel into fp32, then one term pass (fp32; Y fp32 or
+ * bf16, round to nearest even of the sum).
+ *   workspace  sherry_linear_tequila_workspace_bytes(M, N, K, g, group, y_dtype) bytes
+ *            (the linear's ticket contract; bf16 Y adds fp32 scratch after it) */
+#define SHERRY_TEQUILA_ONES 0
+#define SHERRY_TEQUILA_SIGN 1
+int sherry_quantize_pack_tequila(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
+                                 float eps, uint32_t* idx, uint8_t* sgn, float* scales, uint16_t* D, float* bias,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+int sherry_linear_tequila(const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                          const uint32_t* idx, const uint8_t* sgn, const float* scales, int granularity, int group,
+                          const uint16_t* D, const float* bias, int mode,
+                          void* Y, int y_dtype, void* workspace, size_t workspace_bytes, void* stream);
+size_t sherry_linear_tequila_workspace_bytes(int64_t M, int64_t N, int64_t K, int granularity, int group,
+                                             int y_dtype);
+
 /* One weight of a batched quantise + pack (all pointers device pointers). */
 typedef struct sherry_quantize_desc {
     const void* W;          /* [N][K], w_dtype */

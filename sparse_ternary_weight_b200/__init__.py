@@ -272,6 +272,58 @@ def linear_batched(pairs, out_dtype=None, outs=None, descs=None):
     return outs
 
 
+def quantize_pack_tequila(W, granularity="per_group", group: int = 128, eps: float = 1e-5):
+    """Quantise + pack as :func:`quantize_pack` and, in the same pass over W, the
+    Tequila-style dead-weight plane D (bf16 [N, K/4]: eps * the zeroed weight of
+    each block) and its row sums (fp32 [N]).  Returns (packed, D, bias)."""
+    import torch
+    _require_cuda(W)
+    if W.dim() != 2:
+        raise ValueError("expects a 2D weight")
+    W = W.contiguous()
+    N, K = W.shape
+    g = _gran(granularity)
+    L = lib()
+    ns = L.sherry_num_scales(N, K, g, group)
+    if ns < 0:
+        raise SherryError(_abi.ERR_SHAPE if K % 32 or K < 32 else _abi.ERR_GROUP, "quantize_pack_tequila")
+    dt = {torch.float32: F32, torch.bfloat16: BF16}.get(W.dtype)
+    if dt is None:
+        raise SherryError(_abi.ERR_DTYPE, "quantize_pack_tequila")
+    P = _new_packed(N, K, g, group, ns, W.device)
+    D = torch.empty((N, K // 4), dtype=torch.bfloat16, device=W.device)
+    bias = torch.empty((N,), dtype=torch.float32, device=W.device)
+    wsb = L.sherry_workspace_bytes(_abi.OP_QUANTIZE_PACK, 0, N, K, g, group)
+    ws = workspace(wsb, W.device, "quantize")
+    check(L.sherry_quantize_pack_tequila(_ptr(W), dt, N, K, g, group, float(eps), _ptr(P.idx), _ptr(P.sgn),
+                                         _ptr(P.scales), _ptr(D), _ptr(bias), _ptr(ws), wsb, _stream(W.device)),
+          "quantize_pack_tequila")
+    return P, D, bias
+
+
+def linear_tequila(X, P: PackedWeight, D, bias, mode="sign", out_dtype=None, out=None):
+    """Y = X (T alpha)^T + the dead-weight term: ``mode="ones"`` adds bias[n],
+    ``mode="sign"`` adds sign(X) D^T."""
+    import torch
+    _require_cuda(X)
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != P.K:
+        raise ValueError("X must be a 2D bf16 tensor [M, K]")
+    X = X.contiguous()
+    M, K = X.shape
+    md = {"ones": _abi.TEQUILA_ONES, "sign": _abi.TEQUILA_SIGN}[mode]
+    out_dtype = out_dtype or torch.float32
+    yd = {torch.float32: F32, torch.bfloat16: BF16}[out_dtype]
+    if out is None:
+        out = torch.empty((M, P.N), dtype=out_dtype, device=X.device)
+    L = lib()
+    wsb = L.sherry_linear_tequila_workspace_bytes(M, P.N, K, P.granularity, P.group, yd)
+    ws = workspace(wsb, X.device)
+    check(L.sherry_linear_tequila(_ptr(X), M, P.N, K, _ptr(P.idx), _ptr(P.sgn), _ptr(P.scales), P.granularity,
+                                  P.group, _ptr(D), _ptr(bias), md, _ptr(out), yd, _ptr(ws), wsb, _stream(X.device)),
+          "linear_tequila")
+    return out
+
+
 def linear_chain(phases, out_dtype=None, descs=None):
     """Chained linears: ``phases`` is a list of phases, each a list of (X, P, Y)
     triples (X bf16 [M,K], Y [M,N] preallocated).  Every linear of a phase starts

@@ -17,6 +17,7 @@ OP_QUANTIZE_PACK, OP_LINEAR, OP_UNPACK = 0, 1, 2
 MAX_K = 262144
 MAX_BATCH = 256
 NOALLOC_SCRATCH_BYTES = 2 << 20
+TEQUILA_ONES, TEQUILA_SIGN = 0, 1
 
 vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 
@@ -49,6 +50,10 @@ SIGNATURES = {
     "sherry_fake_quant": (i32, [vp, i32, i64, i64, i32, i32, vp, i32, vp, vp, vp, vp, sz, vp]),
     "sherry_quantize_pack_batched": (i32, [ctypes.POINTER(QuantizeDesc), i32, vp, sz, vp]),
     "sherry_quantize_pack_batched_workspace_bytes": (sz, [ctypes.POINTER(QuantizeDesc), i32]),
+    "sherry_quantize_pack_tequila": (i32, [vp, i32, i64, i64, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, vp, sz,
+                                           vp]),
+    "sherry_linear_tequila": (i32, [vp, i64, i64, i64, vp, vp, vp, i32, i32, vp, vp, i32, vp, i32, vp, sz, vp]),
+    "sherry_linear_tequila_workspace_bytes": (sz, [i64, i64, i64, i32, i32, i32]),
     "sherry_linear": (i32, [vp, i64, i64, i64, vp, vp, vp, i32, i32, vp, i32, vp, sz, vp]),
     "sherry_linear_batched": (i32, [ctypes.POINTER(LinearDesc), i32, i64, i32, vp, sz, vp]),
     "sherry_linear_batched_workspace_bytes": (sz, [ctypes.POINTER(LinearDesc), i32, i64]),

@@ -17,11 +17,11 @@ CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libsherry.so")
 OBJ = os.path.join(ROOT, "_build")
 
-SOURCES = ["api.cu", "quantize.cu", "unpack.cu", "gemv.cu", "gemv_stream.cu", "gemv_mma.cu", "gemv_tc.cu", "prefill.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quantize.cu", "unpack.cu", "gemv.cu", "gemv_stream.cu", "gemv_mma.cu", "gemv_tc.cu", "prefill.cu", "noalloc.cu", "tequila.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--ftz=false", "--prec-div=true",
           "--prec-sqrt=true", "-I", os.path.join(ROOT, "include")]
-PER_FILE = {"quantize.cu": ["--fmad=false"]}
+PER_FILE = {"quantize.cu": ["--fmad=false"], "tequila.cu": ["--fmad=false"]}
 
 
 def nvcc() -> str:

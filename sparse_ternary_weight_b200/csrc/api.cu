@@ -191,7 +191,8 @@ static int check_quantize_desc(const sherry_quantize_desc& d) {
 }
 
 static QuantizeJob job_of(const sherry_quantize_desc& d) {
-    return QuantizeJob{d.W, d.w_dtype, d.N, d.K, d.granularity, d.group, d.idx, d.sgn, d.scales, d.Wq, d.wq_dtype};
+    return QuantizeJob{d.W, d.w_dtype, d.N, d.K, d.granularity, d.group, d.idx, d.sgn, d.scales, d.Wq, d.wq_dtype,
+                       nullptr, nullptr, 0.0f};
 }
 
 static int quantize_call(const sherry_quantize_desc* descs, int count, void* workspace, size_t workspace_bytes,
@@ -224,6 +225,24 @@ int sherry_fake_quant(const void* W, int w_dtype, int64_t N, int64_t K, int gran
     if (N > 0 && !Wq) return SHERRY_ERR_NULL;
     const sherry_quantize_desc d{W, idx, sgn, scales, Wq, N, K, w_dtype, granularity, group, wq_dtype};
     return quantize_call(&d, 1, workspace, workspace_bytes, stream);
+}
+
+int sherry_quantize_pack_tequila(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,
+                                 float eps, uint32_t* idx, uint8_t* sgn, float* scales, uint16_t* D, float* bias,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    const sherry_quantize_desc d{W, idx, sgn, scales, nullptr, N, K, w_dtype, granularity, group, SHERRY_F32};
+    int st = check_quantize_desc(d);
+    if (st) return st;
+    if (N > 0 && !D) return SHERRY_ERR_NULL;
+    if (!aligned(D, 16) || !aligned(bias, 4)) return SHERRY_ERR_ALIGN;
+    QuantizeJob j = job_of(d);
+    j.D = D;
+    j.bias = bias;
+    j.eps = eps;
+    const size_t need = quantize_batch_workspace_bytes(&j, 1);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SHERRY_ERR_WORKSPACE;
+    if (need > 0 && !aligned(workspace, 256)) return SHERRY_ERR_ALIGN;
+    return quantize_jobs_launch(&j, 1, workspace, device_sms(), static_cast<cudaStream_t>(stream));
 }
 
 int sherry_quantize_pack_batched(const sherry_quantize_desc* descs, int count, void* workspace,
@@ -333,6 +352,48 @@ int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M,
     if (need > 0 && !aligned(workspace, 256)) return SHERRY_ERR_ALIGN;
     return linear_launch(shapes.data(), kept.data(), (int)shapes.size(), M, y_dtype == SHERRY_BF16, workspace, sms,
                          static_cast<cudaStream_t>(stream));
+}
+
+// The Tequila-style linear: the packed linear into fp32 (Y itself, or scratch after
+// the linear's workspace for bf16 Y), then the dead-weight term.
+static size_t tequila_ws(int64_t M, int64_t N, int64_t K, int granularity, int group, int y_dtype, size_t* lin_ws) {
+    ProbShape s{N, K, granularity, group};
+    const size_t lw = linear_ws_bytes(&s, 1, M, device_sms());
+    *lin_ws = (lw + 255) & ~(size_t)255;
+    return *lin_ws + (y_dtype == SHERRY_BF16 ? (size_t)(M * N) * sizeof(float) : 0);
+}
+
+size_t sherry_linear_tequila_workspace_bytes(int64_t M, int64_t N, int64_t K, int granularity, int group,
+                                             int y_dtype) {
+    if (check_shape(N, K) || check_gran(K, granularity, group) || M <= 0 || N == 0) return 0;
+    size_t lw = 0;
+    return tequila_ws(M, N, K, granularity, group, y_dtype, &lw);
+}
+
+int sherry_linear_tequila(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* idx, const uint8_t* sgn,
+                          const float* scales, int granularity, int group, const uint16_t* D, const float* bias,
+                          int mode, void* Y, int y_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    if (M < 0 || M > (int64_t)0x7fffffff) return SHERRY_ERR_SHAPE;
+    sherry_linear_desc d{X, idx, sgn, scales, Y, N, K, granularity, group};
+    int st = check_linear_desc(d, M);
+    if (st) return st;
+    if (y_dtype != SHERRY_F32 && y_dtype != SHERRY_BF16) return SHERRY_ERR_DTYPE;
+    if (mode != SHERRY_TEQUILA_ONES && mode != SHERRY_TEQUILA_SIGN) return SHERRY_ERR_SHAPE;
+    if (M > 0 && N > 0 && ((mode == SHERRY_TEQUILA_ONES && !bias) || (mode == SHERRY_TEQUILA_SIGN && !D)))
+        return SHERRY_ERR_NULL;
+    if (!aligned(D, 16) || !aligned(bias, 4)) return SHERRY_ERR_ALIGN;
+    if (M == 0 || N == 0) return SHERRY_OK;
+    size_t lw = 0;
+    const size_t need = tequila_ws(M, N, K, granularity, group, y_dtype, &lw);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SHERRY_ERR_WORKSPACE;
+    if (need > 0 && !aligned(workspace, 256)) return SHERRY_ERR_ALIGN;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* y32 = y_dtype == SHERRY_BF16 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + lw)
+                                        : static_cast<float*>(Y);
+    ProbShape ps{N, K, granularity, group};
+    d.Y = y32;
+    if ((st = linear_launch(&ps, &d, 1, M, 0, workspace, device_sms(), s))) return st;
+    return tequila_term_launch(X, M, N, K, idx, D, bias, mode, y32, Y, y_dtype == SHERRY_BF16, s);
 }
 
 // A chain without its empty linears: problems, descriptors and phase bounds.

@@ -145,6 +145,9 @@ struct QuantizeJob {
     float* scales;
     void* Wq;
     int wq_dtype;
+    uint16_t* D;   // optional Tequila-style dead-weight plane, bf16 [N][K/4]
+    float* bias;   // optional row sums of D, fp32 [N]
+    float eps;
 };
 
 // launchers (quantize.cu, unpack.cu, gemv.cu)
@@ -177,6 +180,10 @@ long long stream_set_wait_cycles(long long cycles);  // returns the previous bud
 size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms);
 int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream);
+// Tequila-style dead-weight term added to an fp32 linear output (tequila.cu):
+// mode 0 Y = Yin + bias[n], mode 1 Y = Yin + sign(X) D^T
+int tequila_term_launch(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* idx, const uint16_t* D,
+                        const float* bias, int mode, const float* Yin, void* Y, int y_bf16, cudaStream_t stream);
 // chained phases on the streaming kernel (cooperative launch, one CTA per SM)
 bool chain_eligible(const ProbShape& s, int64_t M);
 bool chain_launch_ok(const ProbShape* shapes, int count, int n_phases, int64_t M);

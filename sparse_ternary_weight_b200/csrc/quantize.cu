@@ -128,6 +128,9 @@ struct QProb {
     uint8_t* sgn;
     float* out;      // scales (group, channel) or per-row subtree sums (per-tensor)
     void* Wq;        // fake-quantised weights (group and channel scales only)
+    uint16_t* dead;  // Tequila-style dead-weight plane (or null)
+    float* dead_sum; // its row sums (or null)
+    float eps;
     int64_t row_begin;
     int N, K;
     int w_bf16, mode, gw, wq;  // gw: words per group (group), per subtree (per-tensor)
@@ -143,7 +146,8 @@ struct QParams {
 
 // Packed words, sign bytes and word sums of row n (phase 1).
 template <bool kBF16>
-__device__ __forceinline__ void encode_row(const QProb& pr, int64_t n, const uint8_t* ctab, float* wsum) {
+__device__ __forceinline__ void encode_row(const QProb& pr, int64_t n, const uint8_t* ctab, float* wsum,
+                                           float* dsum) {
     using L = WLoad<kBF16>;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -166,7 +170,8 @@ __device__ __forceinline__ void encode_row(const QProb& pr, int64_t n, const uin
             const int piece = c * 32 + lane;
             const int half = lane & 1;
             uint32_t nib = 0, sg = 0;
-            float m4[4];
+            float m4[4], d4[4];
+            uint32_t dbits[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 float w0, w1, w2, w3;
@@ -174,6 +179,13 @@ __device__ __forceinline__ void encode_row(const QProb& pr, int64_t n, const uin
                 const uint32_t code = encode4(w0, w1, w2, w3, ctab, m4[j]);
                 nib |= (code & 15u) << (4 * j);
                 sg |= (code >> 4) << j;
+                if (pr.dead) {
+                    // the zeroed weight times eps, rounded to bf16 (one fp32 product)
+                    const uint32_t z = (code >> 2) & 3u;
+                    const float wz = z == 0 ? w0 : z == 1 ? w1 : z == 2 ? w2 : w3;
+                    dbits[j] = __bfloat16_as_ushort(__float2bfloat16_rn(pr.eps * wz));
+                    d4[j] = __uint_as_float(dbits[j] << 16);
+                }
             }
             // half 0 holds blocks 0..3 of the word, half 1 blocks 4..7
             uint32_t word = nib << (16 * half);
@@ -190,13 +202,23 @@ __device__ __forceinline__ void encode_row(const QProb& pr, int64_t n, const uin
                 pr.sgn[row_word + w] = (uint8_t)sb;
                 wsum[w] = s;
             }
+            if (pr.dead) {
+                // the lane's 4 dead values (8 bytes), and their word sum in tree order
+                if (piece < n16)
+                    *reinterpret_cast<uint2*>(pr.dead + n * (int64_t)(pr.K >> 2) + 4 * (int64_t)piece) =
+                        make_uint2(dbits[0] | (dbits[1] << 16), dbits[2] | (dbits[3] << 16));
+                float ds = (d4[0] + d4[1]) + (d4[2] + d4[3]);
+                const float od = __shfl_xor_sync(kFull, ds, 1);
+                ds = half ? od + ds : ds + od;
+                if (half == 0 && piece < n16) dsum[piece >> 1] = ds;
+            }
         }
     }
 }
 
 template <int MAXP>
 __global__ void __launch_bounds__(kQThreads) k_quantize(const __grid_constant__ QParams<MAXP> P) {
-    extern __shared__ float qsm[];   // [words] word sums of the row, then its [ngroups] scales
+    extern __shared__ float qsm[];   // [words] word sums, [words] dead-value sums, [ngroups] scales of the row
     __shared__ uint8_t ctab[64];     // 5-bit code by (zero position, negative bits)
     __shared__ float4 tpat[32];      // the block's ternary values by 5-bit code
     if (threadIdx.x < 64) ctab[threadIdx.x] = (uint8_t)code_of(threadIdx.x >> 4, threadIdx.x & 15u);
@@ -220,13 +242,18 @@ __global__ void __launch_bounds__(kQThreads) k_quantize(const __grid_constant__ 
         const int64_t n = r - pr.row_begin;
         const int words = pr.K >> 5;
         float* wsum = qsm;
-        float* srow = qsm + words;
+        float* dsum = qsm + words;            // dead-value word sums (Tequila plane)
+        float* srow = qsm + 2 * words;
         __syncthreads();  // the tables are ready; the previous row is done with the shared buffers
         if (pr.w_bf16)
-            encode_row<true>(pr, n, ctab, wsum);
+            encode_row<true>(pr, n, ctab, wsum, dsum);
         else
-            encode_row<false>(pr, n, ctab, wsum);
+            encode_row<false>(pr, n, ctab, wsum, dsum);
         __syncthreads();
+        if (pr.dead_sum && warp == (kQThreads / 32) - 1) {
+            const float B = warp_tree_sum(dsum, words);
+            if (lane == 0) pr.dead_sum[n] = B;
+        }
 
         if (pr.mode == kQGroup) {
             // one scale per group of gw words: upper tree levels over the word sums
@@ -391,13 +418,13 @@ static int quantize_launch_t(const std::vector<QProb>& probs, int64_t rows, int 
         maxw = std::max(maxw, probs[i].K / 32);
         if (probs[i].mode == kQGroup) maxg = std::max(maxg, probs[i].K / 32 / probs[i].gw);
     }
-    const size_t smem = (size_t)(maxw + maxg) * sizeof(float);
+    const size_t smem = (size_t)(2 * maxw + maxg) * sizeof(float);
     if (smem > 48 * 1024) {
         static PerDevice attr;
         int done = 0;
         const int st = per_device(attr, &done, [](int& v) {
             SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_quantize<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (SHERRY_MAX_K / 32 + SHERRY_MAX_K / 32) * (int)sizeof(float)));
+                                                   3 * (SHERRY_MAX_K / 32) * (int)sizeof(float)));
             v = 1;
             return SHERRY_OK;
         });
@@ -445,6 +472,9 @@ int quantize_jobs_launch(const QuantizeJob* jobs, int count, void* workspace, in
         p.K = (int)j.K;
         p.w_bf16 = j.w_dtype == SHERRY_BF16;
         p.wq = j.Wq == nullptr ? kWqNone : (j.wq_dtype == SHERRY_BF16 ? kWqBF16 : kWqF32);
+        p.dead = j.D;
+        p.dead_sum = j.D ? j.bias : nullptr;
+        p.eps = j.eps;
         if (j.granularity == SHERRY_PER_GROUP) {
             p.mode = kQGroup;
             p.gw = j.group / 32;
