@@ -74,6 +74,10 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.sherry_ref_tequila_dead.restype = i32
     L.sherry_ref_tequila_term.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, vp]
     L.sherry_ref_tequila_term.restype = i32
+    L.sherry_ref_arenas_linear.argtypes = [vp, i64, vp, vp, vp, vp, ctypes.c_float, i64, i64, i32, i32, vp]
+    L.sherry_ref_arenas_linear.restype = i32
+    L.sherry_ref_arenas_lambda.argtypes = [i64, i64, ctypes.c_double]
+    L.sherry_ref_arenas_lambda.restype = ctypes.c_double
     L.sherry_ref_threads.argtypes = []
     L.sherry_ref_threads.restype = i32
     return L
@@ -190,6 +194,21 @@ class Oracle:
         if st:
             raise ValueError(f"oracle tequila_term status {st}")
         return T
+
+    def arenas_linear(self, X_bf16, idx, sgn, scales, Wd_bf16, lam, N, K, gran=PER_GROUP, group=128):
+        """Y (float64) = X (T alpha)^T + lam * X Wd^T (Wd: the latent weight as bf16 bits [N,K])."""
+        X = np.ascontiguousarray(X_bf16, np.uint16)
+        M = X.shape[0]
+        Y = np.zeros((M, N), np.float64)
+        st = self.L.sherry_ref_arenas_linear(_p(X), M, _p(idx), _p(sgn), _p(np.ascontiguousarray(scales, np.float32)),
+                                             _p(np.ascontiguousarray(Wd_bf16, np.uint16)), float(lam), N, K, gran,
+                                             group, _p(Y))
+        if st:
+            raise ValueError(f"oracle arenas_linear status {st}")
+        return Y
+
+    def arenas_lambda(self, step, total, lam0) -> float:
+        return float(self.L.sherry_ref_arenas_lambda(step, total, lam0))
 
     def threads(self) -> int:
         return int(self.L.sherry_ref_threads())

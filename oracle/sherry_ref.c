@@ -323,6 +323,13 @@ int sherry_ref_tequila_term(const uint16_t* X, int64_t M, const uint32_t* idx, c
     return SHERRY_REF_OK;
 }
 
+/* ---- Arenas: the quantised product plus lambda times the latent-weight product ---- */
+double sherry_ref_arenas_lambda(int64_t step, int64_t total, double lambda0) {
+    if (total <= 0) return lambda0;
+    double s = (double)(step < 0 ? 0 : (step > total ? total : step));
+    return lambda0 * 0.5 * (1.0 + cos(3.14159265358979323846 * s / (double)total));
+}
+
 /* ternary value of weight (n, k) decoded from the planes */
 static int ternary_at(const uint32_t* idx, const uint8_t* sgn, int64_t n, int64_t k, int64_t K) {
     int64_t words = K / 32;
@@ -373,6 +380,31 @@ int sherry_ref_unpack_bf16(const uint32_t* idx, const uint8_t* sgn, const float*
                       scales[scale_index(n, k, K, granularity, group)];
             Wb[n * K + k] = f32_to_bf16_rne(v);
         }
+    return SHERRY_REF_OK;
+}
+
+int sherry_ref_arenas_linear(const uint16_t* X, int64_t M, const uint32_t* idx, const uint8_t* sgn,
+                             const float* scales, const uint16_t* Wd, float lambda, int64_t N, int64_t K,
+                             int granularity, int group, double* Y) {
+    int st = check_planes(idx, sgn, scales, N, K, granularity, group);
+    if (st) return st;
+    if (M < 0) return SHERRY_REF_ERR_SHAPE;
+    if (M > 0 && N > 0 && (!X || !Wd || !Y)) return SHERRY_REF_ERR_NULL;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t m = 0; m < M; ++m) {
+            double yt = 0.0, yw = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                const double x = (double)bf16_bits_to_f32(X[m * K + k]);
+                yt += x * (double)((float)ternary_at(idx, sgn, n, k, K) *
+                                   scales[scale_index(n, k, K, granularity, group)]);
+                yw += x * (double)bf16_bits_to_f32(Wd[n * K + k]);
+            }
+            Y[m * N + n] = yt + (double)lambda * yw;
+        }
+    }
     return SHERRY_REF_OK;
 }
 

@@ -108,6 +108,19 @@ int sherry_ref_tequila_dead(const void* W, int w_dtype, int64_t N, int64_t K, fl
 int sherry_ref_tequila_term(const uint16_t* X, int64_t M, const uint32_t* idx, const uint16_t* D,
                             const float* bias, int64_t N, int64_t K, int mode, double* T);
 
+/* Arenas, the annealed residual of Sherry's training ("Sherry: Hardware-Efficient
+ * 1.25-Bit Ternary Quantization via Fine-grained Sparsification", digest
+ * paragraph on Arenas: Y = X T alpha + lambda_t X W, lambda_t decayed to 0 with a
+ * cosine, gone at inference).  Y [n_rows][N] fp64 for all token rows of X (bf16
+ * bits [M][K]); Wd is the latent weight as bf16 bits [N][K]; the two products are
+ * accumulated in fp64 and combined as y = yT + lambda * yW. */
+int sherry_ref_arenas_linear(const uint16_t* X, int64_t M, const uint32_t* idx, const uint8_t* sgn,
+                             const float* scales, const uint16_t* Wd, float lambda, int64_t N, int64_t K,
+                             int granularity, int group, double* Y);
+/* lambda_t = lambda0 * (1 + cos(pi * min(step, total) / total)) / 2 (cosine decay
+ * from lambda0 at step 0 to 0 at step total; lambda0 for total <= 0) */
+double sherry_ref_arenas_lambda(int64_t step, int64_t total, double lambda0);
+
 /* number of threads the build uses (1 unless built with OpenMP) */
 int sherry_ref_threads(void);
 

@@ -489,6 +489,57 @@ def pin_tequila(orc: oracle.Oracle):
     assert np.array_equal(b2, (z_sign.sum(1) * 2.0 ** -10).astype(np.float32))
 
 
-ALL_PINS = [pin_tequila, pin_fake_quant, pin_topk_reading, pin_code_bijection, pin_argmin_bruteforce, pin_hand_worked, pin_sparsity,
+# ---------------------------------------------------------------- Arenas
+
+def pin_arenas(orc: oracle.Oracle):
+    """Arenas ("Sherry: ..." digest: Y = X T alpha + lambda_t X W, lambda_t
+    cosine-decayed to 0):
+    * lambda = 0 gives the plain linear exactly;
+    * one-hot activations give column k of T alpha + lambda W;
+    * a latent weight equal to the dequantised weight gives (1 + lambda) times
+      the plain linear (within fp64 rounding);
+    * float64 torch of X (T alpha + lambda W)^T within fp64 rounding;
+    * the schedule: lambda0 at step 0, 0 at the last step, lambda0/2 half-way,
+      (2 + sqrt 2)/4 lambda0 at a quarter, non-increasing."""
+    import torch
+    N, K, M = 24, 256, 3
+    W = synth.weights_student_t(N, K, seed=1001)
+    Wd = synth.f32_to_bf16_bits(W)
+    for gran, group in ((oracle.PER_GROUP, 128), (oracle.PER_CHANNEL, 128), (oracle.PER_TENSOR, 128)):
+        idx, sgn, sc = orc.quantize_pack(W, gran, group)
+        Xb = synth.activations_bf16(M, K, seed=1002)
+        plain = orc.linear(Xb, idx, sgn, sc, N, K, gran, group)
+        assert np.array_equal(orc.arenas_linear(Xb, idx, sgn, sc, Wd, 0.0, N, K, gran, group), plain)
+        lam = np.float32(0.3)
+        Wq = orc.unpack_f32(idx, sgn, sc, N, K, gran, group).astype(np.float64)
+        Wl = synth.bf16_bits_to_f32(Wd).astype(np.float64)
+        ref = torch.from_numpy(synth.bf16_bits_to_f32(Xb)).double() @ torch.from_numpy(Wq + float(lam) * Wl).t()
+        y = orc.arenas_linear(Xb, idx, sgn, sc, Wd, lam, N, K, gran, group)
+        assert np.allclose(y, ref.numpy(), rtol=1e-12, atol=1e-12)
+        for k in (0, 77, 255):
+            Xo = np.zeros((1, K), np.uint16)
+            Xo[0, k] = synth.f32_to_bf16_bits(np.array([1.0], np.float32))[0]
+            yo = orc.arenas_linear(Xo, idx, sgn, sc, Wd, lam, N, K, gran, group)[0]
+            assert np.array_equal(yo, Wq[:, k] + float(lam) * Wl[:, k]), k
+        # latent weight = the dequantised weight (exact in bf16 for a power-of-two scale)
+    Wp = (np.where(synth.rng(1003).random((N, K)) < 0.5, -1.0, 1.0) * 2.0 ** -5).astype(np.float32)
+    idx, sgn, sc = orc.quantize_pack(Wp, oracle.PER_GROUP, 128)
+    Wq = orc.unpack_f32(idx, sgn, sc, N, K, oracle.PER_GROUP, 128)
+    Xb = synth.activations_bf16(M, K, seed=1004)
+    plain = orc.linear(Xb, idx, sgn, sc, N, K, oracle.PER_GROUP, 128)
+    y = orc.arenas_linear(Xb, idx, sgn, sc, synth.f32_to_bf16_bits(Wq), 0.5, N, K, oracle.PER_GROUP, 128)
+    assert np.allclose(y, 1.5 * plain, rtol=1e-13, atol=1e-13)
+    # the schedule
+    lam0 = 0.8
+    assert orc.arenas_lambda(0, 1000, lam0) == lam0
+    assert orc.arenas_lambda(1000, 1000, lam0) == 0.0 or abs(orc.arenas_lambda(1000, 1000, lam0)) < 1e-16
+    assert abs(orc.arenas_lambda(500, 1000, lam0) - lam0 / 2) < 1e-15
+    assert abs(orc.arenas_lambda(250, 1000, lam0) - lam0 * (2 + math.sqrt(2)) / 4) < 1e-15
+    assert orc.arenas_lambda(2000, 1000, lam0) == orc.arenas_lambda(1000, 1000, lam0)
+    seq = [orc.arenas_lambda(s, 1000, lam0) for s in range(0, 1001, 50)]
+    assert all(a >= b for a, b in zip(seq, seq[1:]))
+
+
+ALL_PINS = [pin_arenas, pin_tequila, pin_fake_quant, pin_topk_reading, pin_code_bijection, pin_argmin_bruteforce, pin_hand_worked, pin_sparsity,
             pin_scale_power_of_two, pin_scale_closed_form, pin_c_vs_numpy, pin_bf16_input,
             pin_unpack_bf16, pin_linear, pin_errors, pin_pairsum_tree]

@@ -37,6 +37,9 @@ MUTANTS = {
                                 "sgn[n * words + b / 8] |= (uint8_t)(g << (7 - b % 8));"),
     "pad_with_one": ("buf[i] = (i < L) ? v[i] : 0.0f;", "buf[i] = (i < L) ? v[i] : 1.0f;"),
     "group_error_not_checked": ("(group % 32) != 0 || ", ""),
+    "arenas_residual_unscaled": ("Y[m * N + n] = yt + (double)lambda * yw;", "Y[m * N + n] = yt + yw;"),
+    "arenas_linear_schedule": ("return lambda0 * 0.5 * (1.0 + cos(3.14159265358979323846 * s / (double)total));",
+                               "return lambda0 * (1.0 - s / (double)total);"),
     "tequila_dead_from_first_weight": ("const float dead = eps * wv[nib >> 2];", "const float dead = eps * wv[0];"),
     "tequila_sign_of_zero_positive": ("const double sx = (x > 0.0f) ? 1.0 : ((x < 0.0f) ? -1.0 : 0.0);",
                                       "const double sx = (x >= 0.0f) ? 1.0 : -1.0;"),
