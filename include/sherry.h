@@ -237,6 +237,22 @@ int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M,
                           void* workspace, size_t workspace_bytes, void* stream);
 size_t sherry_linear_batched_workspace_bytes(const sherry_linear_desc* descs, int count, int64_t M);
 
+/* ---- Arenas training linear ------------------------------------------------
+ * "Sherry: ... Fine-grained Sparsification", digest paragraph on Arenas: during
+ * quantisation-aware training the layer adds an annealed full-precision
+ * residual, Y = X T alpha + lambda_t X W, with lambda_t decayed to 0 by a cosine;
+ * at inference it is gone.  One kernel computes both products on the tensor
+ * cores (the ternary one with alpha promoted per group in fp32, the dense one in
+ * its own fp32 accumulator) and writes Y = ternary + lambda * dense.
+ *   Wd       the latent weight, bf16 [N][K] row-major (16-byte aligned)
+ *   other arguments as sherry_linear (no workspace); needs K % 64 == 0 and, for
+ *   group scales, group % 64 == 0 (else SHERRY_ERR_UNSUPPORTED).
+ * sherry_arenas_lambda: lambda0 * (1 + cos(pi * min(step, total) / total)) / 2. */
+int sherry_arenas_linear(const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                         const uint32_t* idx, const uint8_t* sgn, const float* scales, int granularity, int group,
+                         const uint16_t* Wd, float lambda, void* Y, int y_dtype, void* stream);
+float sherry_arenas_lambda(int64_t step, int64_t total, float lambda0);
+
 /* ---- chained linears (dependent phases) -----------------------------------
  * `count` linears with the same M (e.g. one decode token through a layer
  * stack) grouped into n_phases phases: phase p holds descs[phase_begin[p] ..

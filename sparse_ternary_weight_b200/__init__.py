@@ -324,6 +324,32 @@ def linear_tequila(X, P: PackedWeight, D, bias, mode="sign", out_dtype=None, out
     return out
 
 
+def arenas_lambda(step: int, total: int, lambda0: float) -> float:
+    """Cosine-decayed weight of the Arenas residual: lambda0 (1 + cos(pi t / T)) / 2."""
+    return float(lib().sherry_arenas_lambda(int(step), int(total), float(lambda0)))
+
+
+def arenas_linear(X, P: PackedWeight, Wd, lam: float, out_dtype=None, out=None):
+    """Arenas training linear Y = X (T alpha)^T + lam X Wd^T in one tensor-core
+    kernel (Wd: the latent weight, bf16 [N, K])."""
+    import torch
+    _require_cuda(X, Wd)
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != P.K:
+        raise ValueError("X must be a 2D bf16 tensor [M, K]")
+    if Wd.dtype != torch.bfloat16 or tuple(Wd.shape) != (P.N, P.K):
+        raise ValueError("Wd must be bf16 [N, K]")
+    X = X.contiguous()
+    Wd = Wd.contiguous()
+    M = X.shape[0]
+    out_dtype = out_dtype or torch.float32
+    yd = {torch.float32: F32, torch.bfloat16: BF16}[out_dtype]
+    if out is None:
+        out = torch.empty((M, P.N), dtype=out_dtype, device=X.device)
+    check(lib().sherry_arenas_linear(_ptr(X), M, P.N, P.K, _ptr(P.idx), _ptr(P.sgn), _ptr(P.scales), P.granularity,
+                                     P.group, _ptr(Wd), float(lam), _ptr(out), yd, _stream(X.device)), "arenas_linear")
+    return out
+
+
 def linear_chain(phases, out_dtype=None, descs=None):
     """Chained linears: ``phases`` is a list of phases, each a list of (X, P, Y)
     triples (X bf16 [M,K], Y [M,N] preallocated).  Every linear of a phase starts

@@ -54,6 +54,8 @@ SIGNATURES = {
                                            vp]),
     "sherry_linear_tequila": (i32, [vp, i64, i64, i64, vp, vp, vp, i32, i32, vp, vp, i32, vp, i32, vp, sz, vp]),
     "sherry_linear_tequila_workspace_bytes": (sz, [i64, i64, i64, i32, i32, i32]),
+    "sherry_arenas_linear": (i32, [vp, i64, i64, i64, vp, vp, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp]),
+    "sherry_arenas_lambda": (ctypes.c_float, [i64, i64, ctypes.c_float]),
     "sherry_linear": (i32, [vp, i64, i64, i64, vp, vp, vp, i32, i32, vp, i32, vp, sz, vp]),
     "sherry_linear_batched": (i32, [ctypes.POINTER(LinearDesc), i32, i64, i32, vp, sz, vp]),
     "sherry_linear_batched_workspace_bytes": (sz, [ctypes.POINTER(LinearDesc), i32, i64]),

@@ -3,6 +3,7 @@
 #include "common.cuh"
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <vector>
 
@@ -394,6 +395,28 @@ int sherry_linear_tequila(const uint16_t* X, int64_t M, int64_t N, int64_t K, co
     d.Y = y32;
     if ((st = linear_launch(&ps, &d, 1, M, 0, workspace, device_sms(), s))) return st;
     return tequila_term_launch(X, M, N, K, idx, D, bias, mode, y32, Y, y_dtype == SHERRY_BF16, s);
+}
+
+int sherry_arenas_linear(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* idx, const uint8_t* sgn,
+                         const float* scales, int granularity, int group, const uint16_t* Wd, float lambda, void* Y,
+                         int y_dtype, void* stream) {
+    if (M < 0 || M > (int64_t)0x7fffffff) return SHERRY_ERR_SHAPE;
+    const sherry_linear_desc d{X, idx, sgn, scales, Y, N, K, granularity, group};
+    int st = check_linear_desc(d, M);
+    if (st) return st;
+    if (y_dtype != SHERRY_F32 && y_dtype != SHERRY_BF16) return SHERRY_ERR_DTYPE;
+    if (M > 0 && N > 0 && !Wd) return SHERRY_ERR_NULL;
+    if (!aligned(Wd, 16)) return SHERRY_ERR_ALIGN;
+    if (M == 0 || N == 0) return SHERRY_OK;
+    const ProbShape s{N, K, granularity, group};
+    if (!arenas_eligible(s, M)) return SHERRY_ERR_UNSUPPORTED;
+    return arenas_launch(s, d, M, y_dtype == SHERRY_BF16, Wd, lambda, static_cast<cudaStream_t>(stream));
+}
+
+float sherry_arenas_lambda(int64_t step, int64_t total, float lambda0) {
+    if (total <= 0) return lambda0;
+    const double t = (double)(step < 0 ? 0 : (step > total ? total : step));
+    return (float)((double)lambda0 * 0.5 * (1.0 + cos(3.14159265358979323846 * t / (double)total)));
 }
 
 // A chain without its empty linears: problems, descriptors and phase bounds.

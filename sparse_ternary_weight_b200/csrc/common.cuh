@@ -164,6 +164,10 @@ int lut_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, 
 bool prefill_eligible(const ProbShape& s, int64_t M);
 int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, int y_bf16, cudaStream_t stream);
 int device_status_take(cudaStream_t stream);
+// Arenas training linear on the prefill kernel: Y = X (T alpha)^T + lambda X Wd^T (prefill.cu)
+bool arenas_eligible(const ProbShape& s, int64_t M);
+int arenas_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, int y_bf16, const uint16_t* Wd,
+                  float lambda, cudaStream_t stream);
 // few-token tensor-core kernel (gemv_tc.cu)
 bool hmma_eligible(const ProbShape& s, int64_t M);
 int hmma_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,

@@ -75,6 +75,7 @@ struct PParams {
     int y_bf16;
     int row_scale, per_tensor, spr;
     int group_steps;  // K-steps per scale group (per-row: all of K)
+    float lambda;     // Arenas: weight of the dense product
 };
 
 // ---- PTX wrappers -------------------------------------------------------------
@@ -162,6 +163,15 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
+// D (TMEM) += A (shared, descriptor) x B (shared, descriptor), both K-major
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
 #define SHERRY_TMEM_ST32(taddr, v)                                                                               \
     asm volatile(                                                                                                \
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16," \
@@ -200,12 +210,24 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
           "=r"(v[30]), "=r"(v[31])                                                                               \
         : "r"(taddr))
 
-template <int EPI>
+// Arenas (ARN): the same kernel also accumulates X W^T for a dense bf16 latent
+// weight W in a third TMEM accumulator and writes Y = (the promoted ternary sum)
+// + lambda * that product.  Its W tiles [128 rows x 64 K] come by TMA into the
+// same slots as X: a chunk is then two K-steps of X and two of W (64 KB), and the
+// ternary A stages shrink to 2 x 2 steps so that the dense accumulator fits in
+// TMEM (columns 384..511).
+template <int EPI, bool ARN>
 __global__ void __launch_bounds__(PRoles<EPI>::kThreads, 1)
-k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PParams P) {
+k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
+          const __grid_constant__ PParams P) {
     constexpr int kPTmaWarp = PRoles<EPI>::kTmaWarp, kPMmaWarp = PRoles<EPI>::kMmaWarp;
+    constexpr int CS = ARN ? 2 : kPChunkSteps;      // K-steps per chunk
+    constexpr int SPG = CS / kPDecGroups;           // steps each decode group expands per chunk
+    constexpr int kWOff = CS * kPStepB;             // W tiles after the X tiles of a slot (ARN)
+    constexpr int kDenseCol = kPAcol + 2 * CS * kPAcols;  // dense accumulator (ARN)
+    static_assert(!ARN || (kWOff + CS * kPStepB <= kPChunkB && kDenseCol + kPBN <= kPTmemCols), "Arenas plan");
     extern __shared__ __align__(1024) unsigned char psmem[];
-    __shared__ uint64_t bars[2 * kPXSlots + 2 + 2 * kPAcc + 1];
+    __shared__ uint64_t bars[2 * kPXSlots + 2 + 2 * kPAcc + 3];
     __shared__ uint32_t tmem_base_s;
     __shared__ volatile int abort_s;
 
@@ -214,19 +236,21 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
     const uint32_t stX = base;                               // kPXSlots x 64 KB, 1024-aligned
     const uint32_t table = base + kPXSlots * kPChunkB;       // 256-aligned
     const uint32_t bar0 = smem_u32(&bars[0]);
-    auto full_x = [&](int c) { return bar0 + 8u * c; };                    // X chunk in slot c landed
+    auto full_x = [&](int c) { return bar0 + 8u * c; };                    // X (and W) chunk in slot c landed
     auto chunk_empty = [&](int c) { return bar0 + 8u * (kPXSlots + c); };  // MMAs of slot c's chunk done
     auto full_a = [&](int h) { return bar0 + 8u * (2 * kPXSlots + h); };   // A buffer h written
     auto acc_full = [&](int b) { return bar0 + 8u * (2 * kPXSlots + 2 + b); };
     auto acc_empty = [&](int b) { return bar0 + 8u * (2 * kPXSlots + 2 + kPAcc + b); };
     const uint32_t drain = bar0 + 8u * (2 * kPXSlots + 2 + 2 * kPAcc);  // the MMA thread's last commit
+    const uint32_t dense_full = drain + 8u;    // ARN: a tile's dense product is complete
+    const uint32_t dense_empty = drain + 16u;  // ARN: the epilogue has read it
 
     // persistent: tile t = (weight-row tile t % ntn, token tile t / ntn), strided by the grid;
     // chunk and accumulator phases run on across tiles
     const int ntn = (P.N + kPBM - 1) / kPBM;
     const int ntiles = ntn * ((P.M + kPBN - 1) / kPBN);
     const int nk = P.K / kPBK;
-    const int nchunks = (nk + kPChunkSteps - 1) / kPChunkSteps;  // the last one may hold fewer steps
+    const int nchunks = (nk + CS - 1) / CS;  // the last one may hold fewer steps
     const int gs = P.group_steps;
     const int ngroups = nk / gs;
 
@@ -242,6 +266,8 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
             mbar_init(acc_empty(b), 32 * EPI);
         }
         mbar_init(drain, 1);
+        mbar_init(dense_full, 1);
+        mbar_init(dense_empty, 32 * EPI);
         fence_mbar_init();
     }
     if (threadIdx.x < 32) {
@@ -264,12 +290,13 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
 
     if (warp < EPI) {
         // ---------------- epilogue: row n = tile row 32*(warp%4) + lane, tokens
-        // [64*(warp/4), 64*(warp/4) + 64) of each tile ----------------
+        // [kCols*(warp/4), kCols*(warp/4) + kCols) of each tile ----------------
         const int q = warp & 3, half = warp >> 2;
         constexpr int kCols = kPBN / (EPI / 4);
         bool ok = true;
         int b = 0;
         uint32_t bph = 0;  // phase parity of accumulator b's use
+        uint32_t dph = 0;  // ARN: phase parity of the dense accumulator's use
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             const int n = (t % ntn) * kPBM + q * 32 + lane;
             const int m0 = (t / ntn) * kPBN + half * kCols;
@@ -303,14 +330,35 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
                 mbar_arrive(acc_empty(b));
                 if (++b == kPAcc) { b = 0; bph ^= 1u; }
             }
-            if (ok && row_ok) {
-                float a = 1.0f;
-                if (P.row_scale) a = __ldg(P.scales + (P.per_tensor ? 0 : n));
+            if (!ok) break;
+            float a = 1.0f;
+            if (P.row_scale && row_ok) a = __ldg(P.scales + (P.per_tensor ? 0 : n));
+#pragma unroll
+            for (int j = 0; j < kCols; ++j) acc[j] *= a;
+            if constexpr (ARN) {
+                // Y = the ternary sum + lambda * the dense product
+                ok = mbar_wait(dense_full, dph, &abort_s);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t t_d = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(kDenseCol + half * kCols);
+#pragma unroll
+                for (int c = 0; c < kCols / 16; ++c) {
+                    uint32_t v[16];
+                    SHERRY_TMEM_LD16(t_d + 16 * c, v);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) acc[16 * c + j] = fmaf(P.lambda, __uint_as_float(v[j]), acc[16 * c + j]);
+                }
+                tc_fence_before();
+                mbar_arrive(dense_empty);
+                dph ^= 1u;
+            }
+            if (row_ok) {
 #pragma unroll
                 for (int j = 0; j < kCols; ++j) {
                     const int m = m0 + j;
                     if (m < P.M) {
-                        const float y = acc[j] * a;
+                        const float y = acc[j];
                         if (P.y_bf16)
                             reinterpret_cast<__nv_bfloat16*>(P.Y)[(int64_t)m * P.N + n] = __float2bfloat16_rn(y);
                         else
@@ -321,7 +369,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
         }
     } else if (warp < kPTmaWarp) {
         // ---------------- decode: TMEM lane (= tile row) i per thread; group g expands
-        // steps 2g, 2g + 1 of every chunk into A buffer (cc & 1) ----------------
+        // steps SPG*g .. SPG*g + SPG-1 of every chunk into A buffer (cc & 1) ----------------
         const int g = (warp - EPI) >> 2, q = warp & 3;
         const int i = q * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kPAcol;
@@ -337,8 +385,8 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
             uint32_t rs[kPRing][2];
             auto fetch = [&](int ch, uint2* w, uint32_t* sg) {
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int ks = ch * kPChunkSteps + 2 * g + e;
+                for (int e = 0; e < SPG; ++e) {
+                    const int ks = ch * CS + SPG * g + e;
                     w[e] = make_uint2(0u, 0u);
                     sg[e] = 0u;
                     if (row_ok && ch < nchunks && ks < nk) {
@@ -359,9 +407,9 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
                     fetch(ch + kPRing, rw[r], rs[r]);
                     const int hbuf = cc & 1;
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int st = 2 * g + e;
-                        if (ch * kPChunkSteps + st >= nk) break;
+                    for (int e = 0; e < SPG; ++e) {
+                        const int st = SPG * g + e;
+                        if (ch * CS + st >= nk) break;
                         uint32_t v[32];
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
@@ -386,7 +434,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
                             }
                             tc_fence_after();
                         }
-                        SHERRY_TMEM_ST32(t_lane + (uint32_t)((hbuf * kPChunkSteps + st) * kPAcols), v);
+                        SHERRY_TMEM_ST32(t_lane + (uint32_t)((hbuf * CS + st) * kPAcols), v);
                     }
                     if (!ok) break;
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -397,7 +445,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
             }
         }
     } else if (warp == kPTmaWarp) {
-        // ---------------- TMA producer for X ----------------
+        // ---------------- TMA producer for X (and, ARN, the latent-weight tiles) ----------------
         if (lane == 0) {
             int c = 0;
             uint32_t cph = 0;  // phase parity of slot c's use
@@ -405,16 +453,20 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
             bool ok = true;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const int m0 = (t / ntn) * kPBN;
+                const int n0 = (t % ntn) * kPBM;
                 for (int ch = 0; ch < nchunks; ++ch) {
                     if (!mbar_wait(chunk_empty(c), cph ^ 1u, &abort_s)) {
                         ok = false;
                         break;
                     }
-                    const int steps = min(kPChunkSteps, nk - ch * kPChunkSteps);
-                    mbar_expect_tx(full_x(c), (uint32_t)(steps * kPStepB));
-                    for (int st = 0; st < steps; ++st)
-                        tma_load_2d(stX + c * kPChunkB + st * kPStepB, &xmap, (ch * kPChunkSteps + st) * kPBK, m0,
-                                    full_x(c));
+                    const int steps = min(CS, nk - ch * CS);
+                    mbar_expect_tx(full_x(c), (uint32_t)(steps * kPStepB * (ARN ? 2 : 1)));
+                    for (int st = 0; st < steps; ++st) {
+                        tma_load_2d(stX + c * kPChunkB + st * kPStepB, &xmap, (ch * CS + st) * kPBK, m0, full_x(c));
+                        if constexpr (ARN)
+                            tma_load_2d(stX + c * kPChunkB + kWOff + st * kPStepB, &wmap, (ch * CS + st) * kPBK, n0,
+                                        full_x(c));
+                    }
                     ++issued[c];
                     if (++c == kPXSlots) { c = 0; cph ^= 1u; }
                 }
@@ -432,9 +484,11 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
         if (lane == 0) {
             int cc = 0, c = 0, b = 0;
             uint32_t cph = 0, bph = 0;
+            uint32_t dph = 0;  // ARN: phase parity of the dense accumulator's use
             bool ok = true;
-            // one MMA step (K = 64: four K = 16 MMAs) into accumulator b; returns false on a timed-out wait
-            auto step = [&](int& gleft, uint32_t ta, uint64_t db) -> bool {
+            // one MMA step (K = 64: four K = 16 MMAs) into accumulator b, and (ARN) the
+            // dense step into the dense accumulator; returns false on a timed-out wait
+            auto step = [&](int& gleft, int ks, uint32_t ta, uint64_t db, uint64_t dw) -> bool {
                 const bool first = gleft == gs;
                 if (first) {
                     if (!mbar_wait(acc_empty(b), bph ^ 1u, &abort_s)) return false;
@@ -445,6 +499,21 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
 #pragma unroll
                 for (int kk = 1; kk < kPBK / 16; ++kk)  // K = 16 per MMA: 8 A columns, +32 bytes in the B row
                     mma_bf16_ts(td, ta + (uint32_t)(8 * kk), db + (uint64_t)(2 * kk), 1u);
+                if constexpr (ARN) {
+                    if (ks == 0) {
+                        if (!mbar_wait(dense_empty, dph ^ 1u, &abort_s)) return false;
+                        tc_fence_after();
+                    }
+                    const uint32_t tdd = tmem + (uint32_t)kDenseCol;
+#pragma unroll
+                    for (int kk = 0; kk < kPBK / 16; ++kk)
+                        mma_bf16_ss(tdd, dw + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk),
+                                    (ks == 0 && kk == 0) ? 0u : 1u);
+                    if (ks == nk - 1) {
+                        mma_commit(dense_full);
+                        dph ^= 1u;
+                    }
+                }
                 if (--gleft == 0) {
                     mma_commit(acc_full(b));
                     gleft = gs;
@@ -460,18 +529,21 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PPar
                     if (!mbar_wait(full_x(c), cph, &abort_s)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t db0 = smem_desc(stX + c * kPChunkB);
-                    const uint32_t ta0 = tmem + (uint32_t)(kPAcol + hbuf * kPChunkSteps * kPAcols);
-                    const int steps = min(kPChunkSteps, nk - ch * kPChunkSteps);
-                    if (steps == kPChunkSteps) {
+                    const uint64_t dw0 = smem_desc(stX + c * kPChunkB + kWOff);
+                    const uint32_t ta0 = tmem + (uint32_t)(kPAcol + hbuf * CS * kPAcols);
+                    const int steps = min(CS, nk - ch * CS);
+                    if (steps == CS) {
 #pragma unroll
-                        for (int st = 0; st < kPChunkSteps; ++st)
-                            if (!step(gleft, ta0 + (uint32_t)(st * kPAcols), db0 + (uint64_t)((st * kPStepB) >> 4))) {
+                        for (int st = 0; st < CS; ++st)
+                            if (!step(gleft, ch * CS + st, ta0 + (uint32_t)(st * kPAcols),
+                                      db0 + (uint64_t)((st * kPStepB) >> 4), dw0 + (uint64_t)((st * kPStepB) >> 4))) {
                                 ok = false;
                                 break;
                             }
                     } else {
                         for (int st = 0; st < steps; ++st)
-                            if (!step(gleft, ta0 + (uint32_t)(st * kPAcols), db0 + (uint64_t)((st * kPStepB) >> 4))) {
+                            if (!step(gleft, ch * CS + st, ta0 + (uint32_t)(st * kPAcols),
+                                      db0 + (uint64_t)((st * kPStepB) >> 4), dw0 + (uint64_t)((st * kPStepB) >> 4))) {
                                 ok = false;
                                 break;
                             }
@@ -524,18 +596,27 @@ bool prefill_eligible(const ProbShape& s, int64_t M) {
     return true;
 }
 
-int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, int y_bf16, cudaStream_t stream) {
+static int encode_2d(CUtensorMap* map, const void* base, int64_t inner, int64_t rows, int box_rows) {
     EncodeTiled enc = encode_fn();
     if (!enc) return SHERRY_ERR_UNSUPPORTED;
-    CUtensorMap map;
-    const cuuint64_t dims[2] = {(cuuint64_t)s.K, (cuuint64_t)M};
-    const cuuint64_t strides[1] = {(cuuint64_t)s.K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kPBK, (cuuint32_t)kPBN};
+    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kPBK, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(d.X), dims, strides, box, estr,
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return SHERRY_ERR_UNSUPPORTED;
+    return r == CUDA_SUCCESS ? SHERRY_OK : SHERRY_ERR_UNSUPPORTED;
+}
+
+// Wd: the latent bf16 weight for Arenas (null: the plain linear)
+static int prefill_launch_any(const ProbShape& s, const sherry_linear_desc& d, int64_t M, int y_bf16,
+                              const uint16_t* Wd, float lambda, cudaStream_t stream) {
+    CUtensorMap map, wmap;
+    int st = encode_2d(&map, d.X, s.K, M, kPBN);
+    if (st) return st;
+    if (Wd && (st = encode_2d(&wmap, Wd, s.K, s.N, kPBM))) return st;
+    if (!Wd) wmap = map;  // unused
     PParams P{};
     P.idx = d.idx;
     P.sgn = d.sgn;
@@ -550,12 +631,15 @@ int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, i
     P.per_tensor = s.granularity == SHERRY_PER_TENSOR;
     P.spr = s.granularity == SHERRY_PER_GROUP ? (int)(s.K / s.group) : 1;
     P.group_steps = s.granularity == SHERRY_PER_GROUP ? s.group / kPBK : (int)(s.K / kPBK);
-    // per device: the shared-memory opt-in of both instantiations, and the SM count
+    P.lambda = lambda;
+    // per device: the shared-memory opt-in of every instantiation, and the SM count
     static PerDevice dev_sms;
     int sms = 0;
-    const int st = per_device(dev_sms, &sms, [](int& v) {
-        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
-        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
+    st = per_device(dev_sms, &sms, [](int& v) {
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_prefill<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem));
         int dev = 0;
         SHERRY_CUDA_CHECK(cudaGetDevice(&dev));
         SHERRY_CUDA_CHECK(cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev));
@@ -568,12 +652,35 @@ int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, i
     // 16 epilogue warps (32 token columns each) drain a group accumulator faster; measured on the
     // 3B shapes that pays for group scales up to K = 4096 (+6%) and costs at K = 8192 (-15%) and
     // for per-row scales (one drain per tile; -1.5% at 2048 and 4096 tokens)
-    if (s.granularity == SHERRY_PER_GROUP && s.K <= 4096)
-        k_prefill<16><<<grid, PRoles<16>::kThreads, kPSmem, stream>>>(map, P);
-    else
-        k_prefill<8><<<grid, PRoles<8>::kThreads, kPSmem, stream>>>(map, P);
+    const bool epi16 = s.granularity == SHERRY_PER_GROUP && s.K <= 4096;
+    if (Wd) {
+        if (epi16)
+            k_prefill<16, true><<<grid, PRoles<16>::kThreads, kPSmem, stream>>>(map, wmap, P);
+        else
+            k_prefill<8, true><<<grid, PRoles<8>::kThreads, kPSmem, stream>>>(map, wmap, P);
+    } else {
+        if (epi16)
+            k_prefill<16, false><<<grid, PRoles<16>::kThreads, kPSmem, stream>>>(map, wmap, P);
+        else
+            k_prefill<8, false><<<grid, PRoles<8>::kThreads, kPSmem, stream>>>(map, wmap, P);
+    }
     SHERRY_LAUNCH_CHECK();
     return SHERRY_OK;
+}
+
+int prefill_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, int y_bf16, cudaStream_t stream) {
+    return prefill_launch_any(s, d, M, y_bf16, nullptr, 0.0f, stream);
+}
+
+bool arenas_eligible(const ProbShape& s, int64_t M) {
+    if (M < 1 || s.N == 0 || s.K % kPBK != 0) return false;
+    if (s.granularity == SHERRY_PER_GROUP && s.group % kPBK != 0) return false;
+    return M <= (int64_t)0x7fffffff / 2 && s.N <= (int64_t)0x7fffffff / 2;
+}
+
+int arenas_launch(const ProbShape& s, const sherry_linear_desc& d, int64_t M, int y_bf16, const uint16_t* Wd,
+                  float lambda, cudaStream_t stream) {
+    return prefill_launch_any(s, d, M, y_bf16, Wd, lambda, stream);
 }
 
 int device_status_take(cudaStream_t stream) {
