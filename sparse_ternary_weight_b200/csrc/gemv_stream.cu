@@ -167,6 +167,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         }
     }
 }
+// wait until the shared phase counter reaches `target`; false on timeout or abort
+__device__ __forceinline__ bool gate_wait(const int* gate, int target, volatile int* abort_flag, long long budget) {
+    const volatile int* g = gate;
+    if (*g >= target) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (*g >= target) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > budget) {
+            *abort_flag = 1;
+            atomicExch(&g_stream_status, SHERRY_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
 __device__ __forceinline__ int ld_acquire(const int* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -441,6 +456,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     constexpr int L = C::kAhead;
     __shared__ int s_last;
     __shared__ int s_abort;
+    __shared__ int s_gate;  // phases known complete on every CTA (written by helper thread 0)
     // Shared addresses: the buffer is rounded up to 256 bytes, so every table
     // base is a multiple of 256 (a lookup's address replaces its low byte); the
     // XOR swizzles need only 16-byte alignment, since writer and reader apply them.
@@ -453,7 +469,6 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     const uint32_t bar_part = bars + 96u;    // every consumer stored its split-tile partial
     const uint32_t bar_last = bars + 104u;   // the ticket's outcome is in s_last
     const uint32_t bar_phase = bars + 112u;  // every consumer finished the CTA's units of a phase
-    const uint32_t bar_gate = bars + 120u;   // the previous phase is complete on every CTA
 
     const int t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5;
@@ -466,8 +481,8 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         mbar_init(bar_part, kSRows);
         mbar_init(bar_last, 1);
         mbar_init(bar_phase, kSRows);
-        mbar_init(bar_gate, 1);
         s_abort = 0;
+        s_gate = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -492,7 +507,6 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         CopyRows<W> cr;
         int cr_p = -1, cr_rb = -1;
         int passed = 0;  // phases known complete on every CTA
-        int gates = 0;
         for (int j = 0; j < nu + L; ++j) {
             if (j < nu) {
                 const int s = j % S;
@@ -511,11 +525,14 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
             if (jt >= 0 && jt < nu) {
                 const int s = jt % S;
                 if (chain && tc.ph > passed) {
-                    // the first tables of a phase read the previous phase's Y
-                    if (ht == 0 && grid_wait(P.phase_cnt + tc.ph - 1, (int)gridDim.x, abort_flag, P.wait_cycles))
-                        mbar_arrive(bar_gate);
-                    if (!mbar_wait(bar_gate, (uint32_t)(gates & 1), abort_flag, P.wait_cycles)) break;
-                    ++gates;
+                    // the first tables of a phase read the previous phase's Y: helper thread 0
+                    // waits for every CTA's arrival and publishes the phase in a shared counter
+                    // (a monotonic count, so a helper that looks late still sees it)
+                    if (ht == 0 && grid_wait(P.phase_cnt + tc.ph - 1, (int)gridDim.x, abort_flag, P.wait_cycles)) {
+                        __threadfence();
+                        *reinterpret_cast<volatile int*>(&s_gate) = tc.ph;
+                    }
+                    if (!gate_wait(&s_gate, tc.ph, abort_flag, P.wait_cycles)) break;
                     __threadfence();
                     passed = tc.ph;
                 }

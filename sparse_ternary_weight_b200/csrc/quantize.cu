@@ -380,22 +380,24 @@ __global__ void __launch_bounds__(1024) k_tensor_scale(const __grid_constant__ Q
 
 // ---- host side ---------------------------------------------------------------
 
+static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
 // largest power of two dividing K, i.e. the subtree size that tiles both each
 // row and the flattened tensor
 static int64_t tensor_chunk(int64_t K) { return K & (-K); }
 
-static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
-
+// per-tensor only: the subtree sums of every row, rounded up to 256 bytes (a
+// batched call places each weight's sums at a 256-byte boundary)
 size_t quantize_workspace_bytes(int64_t N, int64_t K, int granularity) {
-    if (granularity != SHERRY_PER_TENSOR) return 0;
-    return (size_t)(N * (K / tensor_chunk(K))) * sizeof(float);
+    if (granularity != SHERRY_PER_TENSOR || N <= 0) return 0;
+    return align256((size_t)(N * (K / tensor_chunk(K))) * sizeof(float));
 }
 
 size_t quantize_batch_workspace_bytes(const QuantizeJob* jobs, int count) {
     size_t b = 0;
     for (int i = 0; i < count; ++i)
         if (jobs[i].granularity == SHERRY_PER_TENSOR && jobs[i].N > 0)
-            b += align256(quantize_workspace_bytes(jobs[i].N, jobs[i].K, SHERRY_PER_TENSOR));
+            b += quantize_workspace_bytes(jobs[i].N, jobs[i].K, SHERRY_PER_TENSOR);
     return b;
 }
 
@@ -491,7 +493,7 @@ int quantize_jobs_launch(const QuantizeJob* jobs, int count, void* workspace, in
             p.wq = kWqNone;
             p.out = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws_off);
             fins.push_back(QFin{p.out, j.N * (j.K / c), denom(j.N * j.K), j.scales});
-            ws_off += align256(quantize_workspace_bytes(j.N, j.K, SHERRY_PER_TENSOR));
+            ws_off += quantize_workspace_bytes(j.N, j.K, SHERRY_PER_TENSOR);
             if (j.Wq) {
                 tensor_wq.push_back(sherry_unpack_desc{j.idx, j.sgn, j.scales, j.N, j.K, j.granularity, j.group,
                                                        static_cast<uint16_t*>(j.Wq)});

@@ -23,3 +23,26 @@ def orc():
 def orc_omp():
     import oracle
     return oracle.oracle(omp=True)
+
+
+@pytest.fixture(autouse=True)
+def _device_status_guard(request):
+    """After every GPU test: no bounded device wait may have timed out during it.
+    The query goes through the binding, which also drops a linear workspace whose
+    split-K tickets a timed-out kernel may have left nonzero, so one failure does
+    not spread to the next test."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import sys as _sys
+    if "sparse_ternary_weight_b200" not in _sys.modules:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import sparse_ternary_weight_b200 as sw
+    from sparse_ternary_weight_b200 import _abi
+    if _abi._lib is None:
+        return
+    st = sw.device_status()
+    assert st == 0, f"a bounded device wait timed out during {request.node.name} (status {st})"
