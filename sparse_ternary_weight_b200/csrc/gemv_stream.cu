@@ -52,6 +52,8 @@ constexpr int kSThreads = 32 * (kSConsumers + kSHelpers);
 constexpr int kSRows = 32 * kSConsumers;           // 512 rows per unit
 constexpr int kSBars = 128;                        // mbarriers
 constexpr int kSHelperThreads = 32 * kSHelpers;
+constexpr int kSHelperRows = kSRows / kSHelpers;   // rows each helper warp copies
+static_assert(kSHelperRows % 32 == 0, "whole rows per helper lane");
 // chained launches keep their phase counters at the end of the ticket region
 constexpr int kChainCtrs = 512;                    // up to 511 phases + the exit counter
 constexpr int kSMaxPhases = kChainCtrs - 1;
@@ -314,16 +316,16 @@ struct UnitCursor {
 };
 
 // Copy geometry of helper lane (h, lane) for one row block: the unit's rows
-// [128h, 128h+128).  Packed words: rows 128h + R*i + lane/C (C = W/4 lanes per
-// row, R = 32/C rows per copy), 16-byte chunk lane%C of the row's 4W bytes,
-// stored at chunk (c ^ ((row / S) % C)) of the row in shared memory, S = 128/4W
-// rows per bank cycle (that swizzle term only depends on the lane).  Sign bytes
-// and scales: rows 128h + 32i + lane (i = 0..3).  Byte offsets from the plane
+// [Hh, Hh+H), H = kSHelperRows.  Packed words: rows Hh + R*i + lane/C (C = W/4
+// lanes per row, R = 32/C rows per copy), 16-byte chunk lane%C of the row's 4W
+// bytes, stored at chunk (c ^ ((row / S) % C)) of the row in shared memory, S =
+// 128/4W rows per bank cycle (that swizzle term only depends on the lane).  Sign
+// bytes and scales: rows Hh + 32i + lane.  Byte offsets from the plane
 // bases; a row past N reads row 0 instead (its results are never stored), so
 // every copy is in bounds.
 template <int W>
 struct CopyRows {
-    uint32_t idx[W], sgn[4], sc[4];
+    uint32_t idx[kSHelperRows / SGeo<W>::kRowsPerCopy], sgn[kSHelperRows / 32], sc[kSHelperRows / 32];
 };
 
 template <int W>
@@ -331,13 +333,13 @@ __device__ __forceinline__ void copy_rows(const SProb& pr, int rb, int h, int la
     using G = SGeo<W>;
     const int row0 = rb * kSRows;
 #pragma unroll
-    for (int i = 0; i < 128 / G::kRowsPerCopy; ++i) {
-        const int row = row0 + 128 * h + G::kRowsPerCopy * i + lane / G::kLanesPerRow;
+    for (int i = 0; i < kSHelperRows / G::kRowsPerCopy; ++i) {
+        const int row = row0 + kSHelperRows * h + G::kRowsPerCopy * i + lane / G::kLanesPerRow;
         cr.idx[i] = (uint32_t)((int64_t)(row < pr.N ? row : 0) * pr.words * 4 + 16 * (lane % G::kLanesPerRow));
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int row = row0 + 128 * h + 32 * i + lane;
+    for (int i = 0; i < kSHelperRows / 32; ++i) {
+        const int row = row0 + kSHelperRows * h + 32 * i + lane;
         const int rr = row < pr.N ? row : 0;
         cr.sgn[i] = (uint32_t)((int64_t)rr * pr.words);
         cr.sc[i] = (uint32_t)((int64_t)rr * pr.spr * 4);
@@ -356,15 +358,15 @@ __device__ __forceinline__ void copy_unit(const SProb& pr, const CopyRows<W>& cr
     constexpr int C = G::kLanesPerRow;
     const char* bi = reinterpret_cast<const char*>(pr.idx) + sub * G::kRowB;
     const uint32_t lrow = (uint32_t)(lane / C);
-    const uint32_t di = stage + (uint32_t)(128 * h + lrow) * G::kRowB +
+    const uint32_t di = stage + (uint32_t)(kSHelperRows * h + lrow) * G::kRowB +
                         ((uint32_t)((lane % C) ^ ((lrow / G::kSwz) % C)) << 4);
 #pragma unroll
-    for (int i = 0; i < 128 / G::kRowsPerCopy; ++i)
+    for (int i = 0; i < kSHelperRows / G::kRowsPerCopy; ++i)
         cp_async16(di + (uint32_t)(G::kRowsPerCopy * G::kRowB * i), byte_off(bi, cr.idx[i]));
     const char* bs = reinterpret_cast<const char*>(pr.sgn) + sub * W;
-    const uint32_t ds = stage + G::kIdx + (uint32_t)(128 * h + lane) * W;
+    const uint32_t ds = stage + G::kIdx + (uint32_t)(kSHelperRows * h + lane) * W;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kSHelperRows / 32; ++i) {
         if (W == 16)
             cp_async16(ds + 32u * W * i, byte_off(bs, cr.sgn[i]));
         else
@@ -374,7 +376,7 @@ __device__ __forceinline__ void copy_unit(const SProb& pr, const CopyRows<W>& cr
     if (pr.mode == kSG128) {  // W/4 scales per row and unit
         const char* ba = reinterpret_cast<const char*>(pr.scales) + sub * W;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kSHelperRows / 32; ++i) {
             if (W == 16)
                 cp_async16(dc + 32u * W * i, byte_off(ba, cr.sc[i]));
             else
@@ -383,7 +385,7 @@ __device__ __forceinline__ void copy_unit(const SProb& pr, const CopyRows<W>& cr
     } else if (pr.mode == kSG256) {  // W/8 scales per row and unit
         const char* ba = reinterpret_cast<const char*>(pr.scales) + sub * (W / 2);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kSHelperRows / 32; ++i) {
             if (W == 16)
                 cp_async8(dc + 32u * W * i, byte_off(ba, cr.sc[i]));
             else
