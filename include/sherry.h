@@ -336,6 +336,11 @@ int sherry_last_cuda_error(void);
  * left nonzero: zero its first 256 KiB (or take a fresh zeroed workspace)
  * before the next linear call with it. */
 int sherry_device_status(void* stream);
+/* How many nonzero statuses sherry_device_status has returned in this process
+ * (a host-side count, no device work).  A caller that caches workspaces
+ * compares it with the value it saw when it last zeroed them: a change means a
+ * wait gave up since, and the cached ticket regions must be zeroed again. */
+int64_t sherry_timeout_count(void);
 /* Budget, in SM clock cycles, of every bounded wait of the streaming decode
  * kernel (one or two tokens), for launches made after this call; cycles <= 0
  * restores the default (4e9, about 2 s at the boost clock).  Returns the previous

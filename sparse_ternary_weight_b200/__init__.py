@@ -58,6 +58,7 @@ class PackedWeight:
 
 
 _ws_cache: dict = {}
+_ws_timeouts = [0]  # the library's timeout count when the cached buffers were last known clean
 
 
 def workspace(nbytes: int, device, kind: str = "linear") -> "object":
@@ -65,10 +66,16 @@ def workspace(nbytes: int, device, kind: str = "linear") -> "object":
     ``kind="linear"`` buffers are zero-filled when allocated and used by the
     linear calls only: their split-K ticket counters must start at zero, and
     every successful call leaves them at zero.  Other kinds hold scratch that
-    the next call overwrites."""
+    the next call overwrites.  Once any bounded device wait has been reported
+    as given up (sherry_device_status, by whichever caller), every cached
+    buffer is dropped: a timed-out kernel may have left tickets nonzero."""
     import torch
     if nbytes <= 0:
         return None
+    seen = lib().sherry_timeout_count()
+    if seen != _ws_timeouts[0]:
+        _ws_cache.clear()
+        _ws_timeouts[0] = seen
     key = (str(device), kind)
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < nbytes:
@@ -80,15 +87,12 @@ def workspace(nbytes: int, device, kind: str = "linear") -> "object":
 def device_status(device=None) -> int:
     """Synchronise the current stream of ``device`` and return the library's
     device status (0, or ERR_TIMEOUT when a bounded wait of a kernel gave up
-    since the last query).  After a timeout the cached linear workspace of that
-    device may hold nonzero split-K tickets, so it is dropped here and the next
-    linear call gets a fresh zeroed one."""
+    since the last query).  After a timeout the cached workspaces may hold
+    nonzero split-K tickets; the next workspace request drops them (the
+    library counts every nonzero status it reports)."""
     import torch
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-    st = lib().sherry_device_status(_stream(dev))
-    if st:
-        _ws_cache.pop((str(dev), "linear"), None)
-    return st
+    return lib().sherry_device_status(_stream(dev))
 
 
 def quantize_pack(W, granularity="per_group", group: int = 128, out: PackedWeight | None = None) -> PackedWeight:

@@ -69,6 +69,7 @@ SIGNATURES = {
     "sherry_status_string": (ctypes.c_char_p, [i32]),
     "sherry_last_cuda_error": (i32, []),
     "sherry_device_status": (i32, [vp]),
+    "sherry_timeout_count": (i64, []),
     "sherry_set_wait_budget": (i64, [i64]),
     "sherry_version": (i32, []),
 }

@@ -3,6 +3,7 @@
 #include "common.cuh"
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <mutex>
 #include <vector>
@@ -129,7 +130,15 @@ int sherry_version(void) { return 0x000100; }
 
 int sherry_last_cuda_error(void) { return g_last_cuda_error; }
 
-int sherry_device_status(void* stream) { return device_status_take(static_cast<cudaStream_t>(stream)); }
+static std::atomic<int64_t> g_timeouts_seen{0};
+
+int sherry_device_status(void* stream) {
+    const int st = device_status_take(static_cast<cudaStream_t>(stream));
+    if (st) g_timeouts_seen.fetch_add(1);
+    return st;
+}
+
+int64_t sherry_timeout_count(void) { return g_timeouts_seen.load(); }
 
 int64_t sherry_set_wait_budget(int64_t cycles) { return (int64_t)stream_set_wait_cycles((long long)cycles); }
 

@@ -527,14 +527,20 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
             if (jt >= 0 && jt < nu) {
                 const int s = jt % S;
                 if (chain && tc.ph > passed) {
-                    // the first tables of a phase read the previous phase's Y: helper thread 0
-                    // waits for every CTA's arrival and publishes the phase in a shared counter
-                    // (a monotonic count, so a helper that looks late still sees it)
-                    if (ht == 0 && grid_wait(P.phase_cnt + tc.ph - 1, (int)gridDim.x, abort_flag, P.wait_cycles)) {
+                    // the first tables of a phase read the previous phase's Y: helper warp 0
+                    // (as a whole warp) waits for every CTA's arrival and publishes the phase
+                    // in a shared counter that the other helper warps poll (a monotonic
+                    // count, so a warp that looks late still sees it)
+                    if (h == 0) {
+                        const bool all = grid_wait(P.phase_cnt + tc.ph - 1, (int)gridDim.x, abort_flag,
+                                                   P.wait_cycles);
+                        __syncwarp();
+                        if (!all) break;
                         __threadfence();
-                        *reinterpret_cast<volatile int*>(&s_gate) = tc.ph;
+                        if (lane == 0) *reinterpret_cast<volatile int*>(&s_gate) = tc.ph;
+                    } else if (!gate_wait(&s_gate, tc.ph, abort_flag, P.wait_cycles)) {
+                        break;
                     }
-                    if (!gate_wait(&s_gate, tc.ph, abort_flag, P.wait_cycles)) break;
                     __threadfence();
                     passed = tc.ph;
                 }
@@ -624,15 +630,15 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                             mbar_arrive(bar_part);
                             const uint32_t ph2 = (uint32_t)(events & 1);
                             ++events;
-                            if (r == 0) {
-                                if (!mbar_wait(bar_part, ph2, abort_flag, P.wait_cycles)) {
-                                    ok = false;
-                                    break;
-                                }
+                            // every consumer waits for all partials (no lane of a warp spins on
+                            // another barrier than its neighbours: divergent spins can starve)
+                            const bool stored = mbar_wait(bar_part, ph2, abort_flag, P.wait_cycles);
+                            if (stored && r == 0) {
                                 s_last = (atomicAdd(P.ticket + tile, 1) == c_b - c_a);
                                 mbar_arrive(bar_last);
                             }
-                            if (!mbar_wait(bar_last, ph2, abort_flag, P.wait_cycles)) {
+                            __syncwarp();
+                            if (!stored || !mbar_wait(bar_last, ph2, abort_flag, P.wait_cycles)) {
                                 ok = false;
                                 break;
                             }
@@ -665,16 +671,21 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                 }
                 if (!ok) break;
                 if (chain) {
-                    // every consumer's Y of this phase is written before the CTA's arrival
+                    // every consumer's Y of this phase is written before the CTA's arrival;
+                    // warp 0 waits for all of them (as a whole warp) and lane 0 arrives
                     __threadfence();
                     mbar_arrive(bar_phase);
-                    if (r == 0) {
-                        if (!mbar_wait(bar_phase, (uint32_t)(phases & 1), abort_flag, P.wait_cycles)) {
+                    if (warp == 0) {
+                        const bool done = mbar_wait(bar_phase, (uint32_t)(phases & 1), abort_flag, P.wait_cycles);
+                        if (done && lane == 0) {
+                            __threadfence();
+                            atomicAdd(P.phase_cnt + ph, 1);
+                        }
+                        __syncwarp();
+                        if (!done) {
                             ok = false;
                             break;
                         }
-                        __threadfence();
-                        atomicAdd(P.phase_cnt + ph, 1);
                     }
                     ++phases;
                 }

@@ -241,3 +241,8 @@ def test_linear_chain_validation(L):
     assert L.sherry_linear_chain_workspace_bytes(bad, 2, pb(0, 1, 2), 2, 1) == 0
     # M = 0: nothing to do
     assert ch(arr, 2, pb(0, 1, 2), 2, 0, _abi.F32, None, 0, None) == _abi.OK
+
+
+def test_timeout_count_starts_at_zero(L):
+    # host-side count of nonzero device statuses; no device work, so it runs without a GPU
+    assert L.sherry_timeout_count() == 0
