@@ -509,6 +509,8 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         CopyRows<W> cr;
         int cr_p = -1, cr_rb = -1;
         int passed = 0;  // phases known complete on every CTA
+        uint2 xn[MT];        // the activations of table cursor's unit, loaded one unit ahead
+        bool have_x = false;
         for (int j = 0; j < nu + L; ++j) {
             if (j < nu) {
                 const int s = j % S;
@@ -544,18 +546,25 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                     __threadfence();
                     passed = tc.ph;
                 }
-                const SProb& pt = P.p[tc.pos.p];
-                if (ht < G::kTabs) {
-                    // activations: token m's row of X starts K bf16 (words * 8 groups of 4) after token m-1's
+                // activations: token m's row of X starts K bf16 (words * 8 groups of 4) after
+                // token m-1's; read through L2 (a chained phase's X is written by this launch)
+                auto load_x = [&](const SProb& px, int sub) {
 #pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        const uint2 xb = __ldcg(reinterpret_cast<const uint2*>(pt.X) + (int64_t)m * pt.words * 8 +
-                                                tc.pos.sub * G::kTabs + ht);
-                        build_table(luts + s * C::kLutStage + m * G::kLut + ht * kTab, xb);
-                    }
+                    for (int m = 0; m < MT; ++m)
+                        xn[m] = __ldcg(reinterpret_cast<const uint2*>(px.X) + (int64_t)m * px.words * 8 +
+                                       sub * G::kTabs + ht);
+                };
+                if (ht < G::kTabs) {
+                    if (!have_x) load_x(P.p[tc.pos.p], tc.pos.sub);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) build_table(luts + s * C::kLutStage + m * G::kLut + ht * kTab, xn[m]);
                     mbar_arrive(ready(s));
                 }
                 tc.next(P);
+                // the next unit's activations are fetched now unless it opens a phase that is
+                // still being written
+                have_x = ht < G::kTabs && jt + 1 < nu && (!chain || tc.ph <= passed);
+                if (have_x) load_x(P.p[tc.pos.p], tc.pos.sub);
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");

@@ -27,10 +27,11 @@ def orc_omp():
 
 @pytest.fixture(autouse=True)
 def _device_status_guard(request):
-    """After every GPU test: no bounded device wait may have timed out during it.
-    The query goes through the binding, which also drops a linear workspace whose
-    split-K tickets a timed-out kernel may have left nonzero, so one failure does
-    not spread to the next test."""
+    """After every GPU test: no bounded device wait may have timed out during it,
+    and every cached linear workspace has its split-K ticket region back at zero
+    (each call that completes must leave it so).  A nonzero status makes the
+    binding drop its cached workspaces; dirty tickets are reported and the
+    buffer dropped, so one failure does not spread to the next test."""
     yield
     if request.node.get_closest_marker("gpu") is None:
         return
@@ -46,3 +47,11 @@ def _device_status_guard(request):
         return
     st = sw.device_status()
     assert st == 0, f"a bounded device wait timed out during {request.node.name} (status {st})"
+    ticket_bytes = 256 * 1024
+    for key, buf in list(sw._ws_cache.items()):
+        if key[1] != "linear":
+            continue
+        dirty = int(buf[:ticket_bytes].view(torch.int32).ne(0).sum())
+        if dirty:
+            sw._ws_cache.pop(key, None)
+        assert dirty == 0, f"{request.node.name} left {dirty} nonzero ticket words in the {key} workspace"
