@@ -150,7 +150,8 @@ int sherry_fake_quant(const void* W, int w_dtype, int64_t N, int64_t K, int gran
  * the linear by its usual kernel into fp32, then one term pass (fp32; Y fp32 or
  * bf16, round to nearest even of the sum).
  *   workspace  sherry_linear_tequila_workspace_bytes(M, N, K, g, group, y_dtype) bytes
- *            (the linear's ticket contract; bf16 Y adds fp32 scratch after it) */
+ *            (the linear's ticket contract: the first 256 KiB zero on entry and left
+ *            zero; bf16 Y adds M*N fp32 scratch after max(the linear's bytes, 256 KiB)) */
 #define SHERRY_TEQUILA_ONES 0
 #define SHERRY_TEQUILA_SIGN 1
 int sherry_quantize_pack_tequila(const void* W, int w_dtype, int64_t N, int64_t K, int granularity, int group,

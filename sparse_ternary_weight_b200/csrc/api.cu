@@ -365,12 +365,17 @@ int sherry_linear_batched(const sherry_linear_desc* descs, int count, int64_t M,
 }
 
 // The Tequila-style linear: the packed linear into fp32 (Y itself, or scratch after
-// the linear's workspace for bf16 Y), then the dead-weight term.
+// the linear's workspace for bf16 Y), then the dead-weight term.  The fp32 scratch
+// never overlaps the ticket region at the front of the workspace, even when the
+// linear itself needs no workspace: other linear calls sharing the buffer rely on
+// that region being zero.
 static size_t tequila_ws(int64_t M, int64_t N, int64_t K, int granularity, int group, int y_dtype, size_t* lin_ws) {
     ProbShape s{N, K, granularity, group};
     const size_t lw = linear_ws_bytes(&s, 1, M, device_sms());
     *lin_ws = (lw + 255) & ~(size_t)255;
-    return *lin_ws + (y_dtype == SHERRY_BF16 ? (size_t)(M * N) * sizeof(float) : 0);
+    if (y_dtype != SHERRY_BF16) return lw;
+    *lin_ws = std::max(*lin_ws, kTicketBytes);
+    return *lin_ws + (size_t)(M * N) * sizeof(float);
 }
 
 size_t sherry_linear_tequila_workspace_bytes(int64_t M, int64_t N, int64_t K, int granularity, int group,

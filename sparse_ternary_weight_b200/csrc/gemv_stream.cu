@@ -265,10 +265,18 @@ struct UnitPos {
     int p, rb, sub;  // problem, row block, sub-slice
 };
 
+// the last problem whose first unit is <= u: a binary search, since a CTA's first
+// lookup sits on its start-up path and a batch holds up to hundreds of problems
 template <int MAXP>
 __device__ __forceinline__ UnitPos locate(const SParams<MAXP>& P, int u) {
-    int p = 0;
-    while (p + 1 < P.count && P.p[p + 1].unit_begin <= u) ++p;
+    int p = 0, hi = P.count - 1;
+    while (p < hi) {
+        const int mid = (p + hi + 1) >> 1;
+        if (P.p[mid].unit_begin <= u)
+            p = mid;
+        else
+            hi = mid - 1;
+    }
     const int local = u - P.p[p].unit_begin;
     return UnitPos{p, local / P.p[p].n_sub, local % P.p[p].n_sub};
 }
@@ -505,7 +513,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         const int ht = t - 32 * kSConsumers;  // table (block of 4 activations) of the unit
         UnitCursor<MAXP> cc, tc;              // copy and table cursors
         cc.seek(P, 0);
-        tc.seek(P, 0);
+        tc = cc;
         CopyRows<W> cr;
         int cr_p = -1, cr_rb = -1;
         int passed = 0;  // phases known complete on every CTA

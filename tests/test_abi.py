@@ -246,3 +246,13 @@ def test_linear_chain_validation(L):
 def test_timeout_count_starts_at_zero(L):
     # host-side count of nonzero device statuses; no device work, so it runs without a GPU
     assert L.sherry_timeout_count() == 0
+
+
+def test_tequila_scratch_stays_out_of_the_ticket_region(L):
+    # M = 300 runs a kernel without split-K tickets, so the linear needs no workspace;
+    # the bf16 path's fp32 scratch still starts after the 256 KiB ticket region
+    M, N, K = 300, 200, 512
+    f32 = L.sherry_linear_tequila_workspace_bytes(M, N, K, _abi.PER_GROUP, 64, _abi.F32)
+    bf16 = L.sherry_linear_tequila_workspace_bytes(M, N, K, _abi.PER_GROUP, 64, _abi.BF16)
+    assert bf16 >= 256 * 1024 + M * N * 4
+    assert bf16 - f32 >= M * N * 4
