@@ -408,7 +408,7 @@ def extra_rows(args, pairs, outs, shapes, ws, dev, pk):
 
     # decode batch sweep on the 3B stack
     sweep = {}
-    for M in (2, 4, 8, 16, 32):
+    for M in (2, 3, 4, 8, 16, 32):
         cfg, layers, shp = synth.STACKS[STACK]
         mp = []
         mo = []

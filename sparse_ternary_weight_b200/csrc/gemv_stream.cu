@@ -1,4 +1,4 @@
-// gemv_stream.cu -- packed 3:4 ternary linear for one or two tokens (M <= 2),
+// gemv_stream.cu -- packed 3:4 ternary linear for one to four tokens (M <= 4),
 // HBM-streaming version of the lookup-table decode (the method's inference
 // scheme: tables built from the activations, looked up by the packed weights,
 // accumulated, then scaled; "Sherry: Hardware-Efficient 1.25-Bit Ternary
@@ -6,8 +6,9 @@
 // Y = X T alpha).
 //
 // Work unit: 512 output rows x 32 W weights (W packed words) of one linear, W =
-// 16 for independent linears (one batched launch per decode step) and W = 8 for
-// chained phases, whose layers are small enough that finer units balance better.
+// 16 for independent linears of one or two tokens (one batched launch per decode
+// step), W = 8 for three or four tokens (whose tables take more shared memory) and
+// for chained phases, whose layers are small enough that finer units balance better.
 // All units of a phase (one or many independent linears) are split into equal
 // contiguous ranges, one per CTA (stream-K): every CTA streams the same number
 // of bytes.  A row block whose units straddle CTAs is finished by the CTA that
@@ -76,23 +77,24 @@ struct SGeo {
     static_assert(kTabs <= kSHelperThreads, "one table per helper thread");
 };
 
-// Ring depth, copy lookahead and shared bytes for MT tokens and W-word units
-// (tables are token-major within a stage).  The lookahead L lets the copies run
-// L units ahead of the table builds (used across phase barriers).
+// Ring depth and shared bytes for MT tokens and W-word units (tables are
+// token-major within a stage): as many stages as fit next to one CTA's
+// registers; three or four tokens take 8-word units (a 16-word stage with their
+// tables leaves room for one stage only).
 template <int MT, int W>
 struct SCfg {
     using G = SGeo<W>;
-    static constexpr int kStages = W == 16 ? (MT == 1 ? 3 : 2) : (MT == 1 ? 6 : 5);
-    static constexpr int kAhead = W == 16 ? 0 : kStages - 2;
+    static constexpr int kStages =
+        W == 16 ? (MT == 1 ? 3 : MT == 2 ? 2 : 1) : (MT == 1 ? 6 : MT == 2 ? 5 : MT == 3 ? 4 : 3);
     static constexpr int kLutStage = MT * G::kLut;
     static constexpr int kSmem = 256 + kStages * (G::kStage + kLutStage) + kSBars;
     static_assert(kSmem <= 232448, "shared memory per CTA");
-    static_assert(kStages <= 6, "barrier slots");
+    static_assert(kStages >= 2 && kStages <= 6, "ring depth / barrier slots");
 };
 constexpr long long kSWaitCycles = 4000000000LL;   // default wait budget, ~2 s at the boost clock
 // The no-workspace entry point's fixed scratch holds this kernel's largest plan
-// (two tokens, one CTA per SM, two partial slots per CTA) on up to 224 SMs.
-static_assert(kTicketBytes + (size_t)224 * 2 * 2 * kSRows * sizeof(float) <= SHERRY_NOALLOC_SCRATCH_BYTES,
+// (four tokens, one CTA per SM, two partial slots per CTA) on up to 224 SMs.
+static_assert(kTicketBytes + (size_t)224 * 2 * 4 * kSRows * sizeof(float) <= SHERRY_NOALLOC_SCRATCH_BYTES,
               "no-workspace scratch too small for the streaming plan");
 
 enum SMode { kSRow = 0, kSG128 = 1, kSG256 = 2 };
@@ -189,21 +191,30 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-// wait until *cnt >= target (every CTA arrived at a phase); false on timeout or abort
-__device__ __forceinline__ bool grid_wait(const int* cnt, int target, volatile int* abort_flag, long long budget) {
-    if (ld_acquire(cnt) >= target) return true;
+// One warp (all lanes, converged) reads *cnt until it reaches target (every CTA
+// arrived at a phase), or once when block is false: 1 = reached, 0 = not yet
+// (non-blocking), -1 = timeout or abort.  Lane 0's reads decide for the warp.
+__device__ __forceinline__ int grid_poll(const int* cnt, int target, volatile int* abort_flag, long long budget,
+                                         bool block, int lane) {
     const long long t0 = clock64();
     while (true) {
-        if (ld_acquire(cnt) >= target) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > budget) {
-            *abort_flag = 1;
-            atomicExch(&g_stream_status, SHERRY_ERR_TIMEOUT);
-            return false;
+        int v = lane == 0 ? ld_acquire(cnt) : 0;
+        v = __shfl_sync(kFull, v, 0);
+        if (v >= target) return 1;
+        if (!block) return 0;
+        int quit = 0;
+        if (lane == 0) {
+            if (*abort_flag) {
+                quit = 1;
+            } else if (clock64() - t0 > budget) {
+                *abort_flag = 1;
+                atomicExch(&g_stream_status, SHERRY_ERR_TIMEOUT);
+                quit = 1;
+            }
         }
+        if (__shfl_sync(kFull, quit, 0)) return -1;
     }
 }
-
 }  // namespace
 
 extern __shared__ __align__(16) unsigned char g_smem[];
@@ -259,6 +270,8 @@ __device__ __forceinline__ void word_sums(uint32_t w, uint32_t s, uint32_t base,
                            __byte_perm(ev, base, 0x7653u), __byte_perm(od, base, 0x7653u)};
     token_sums<BOFF, 0, LUT>(a, p0[0], p1[0]);
     if constexpr (MT > 1) token_sums<BOFF, 1, LUT>(a, p0[1], p1[1]);
+    if constexpr (MT > 2) token_sums<BOFF, 2, LUT>(a, p0[2], p1[2]);
+    if constexpr (MT > 3) token_sums<BOFF, 3, LUT>(a, p0[3], p1[3]);
 }
 
 struct UnitPos {
@@ -463,7 +476,6 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     using C = SCfg<MT, W>;
     using G = SGeo<W>;
     constexpr int S = C::kStages;
-    constexpr int L = C::kAhead;
     __shared__ int s_last;
     __shared__ int s_abort;
     __shared__ int s_gate;  // phases known complete on every CTA (written by helper thread 0)
@@ -507,73 +519,97 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
 
     if (warp >= kSConsumers) {
         // ---- helpers: unit j's copies go to stage j % S once the consumers are done
-        // with unit j - S there; its tables follow L units later (after the previous
-        // phase completed on every CTA, for a unit that opens a phase)
+        // with unit j - S there.  Its tables are built right after, unless the unit opens
+        // a phase whose input (the previous phase's Y) is not complete yet: then the
+        // copies run on and the tables follow once the phase barrier is seen, at the
+        // latest before a stage is reused whose consumers need them.
         const int h = warp - kSConsumers;
         const int ht = t - 32 * kSConsumers;  // table (block of 4 activations) of the unit
+        const bool tab = ht < G::kTabs;
         UnitCursor<MAXP> cc, tc;              // copy and table cursors
         cc.seek(P, 0);
         tc = cc;
         CopyRows<W> cr;
         int cr_p = -1, cr_rb = -1;
-        int passed = 0;  // phases known complete on every CTA
-        uint2 xn[MT];        // the activations of table cursor's unit, loaded one unit ahead
+        int passed = 0;       // phases this thread knows complete on every CTA
+        int jt = 0;           // units whose tables this thread has built
+        bool fail = false;    // a bounded wait gave up
+        uint2 xn[MT];         // the activations of the table cursor's unit, loaded one unit ahead
         bool have_x = false;
-        for (int j = 0; j < nu + L; ++j) {
-            if (j < nu) {
-                const int s = j % S;
-                if (j >= S && !mbar_wait(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag, P.wait_cycles)) break;
-                const SProb& pr = P.p[cc.pos.p];
-                if (cc.pos.p != cr_p || cc.pos.rb != cr_rb) {
-                    copy_rows<W>(pr, cc.pos.rb, h, lane, cr);
-                    cr_p = cc.pos.p;
-                    cr_rb = cc.pos.rb;
-                }
-                copy_unit<W>(pr, cr, cc.pos.sub, stages + s * G::kStage, h, lane);
-                cp_async_arrive(ready(s));
-                cc.next(P);
+        // activations: token m's row of X starts K bf16 (words * 8 groups of 4) after
+        // token m-1's; read through L2 (a chained phase's X is written by this launch)
+        auto load_x = [&](const SProb& px, int sub) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                xn[m] = __ldcg(reinterpret_cast<const uint2*>(px.X) + (int64_t)m * px.words * 8 + sub * G::kTabs + ht);
+        };
+        // build unit jt's tables; with block == false return false instead of waiting for
+        // the phase barrier
+        auto tables = [&](bool block) -> bool {
+            if (!tab) {  // this thread builds no table: only the cursor moves
+                tc.next(P);
+                ++jt;
+                return true;
             }
-            const int jt = j - L;
-            if (jt >= 0 && jt < nu) {
-                const int s = jt % S;
-                if (chain && tc.ph > passed) {
-                    // the first tables of a phase read the previous phase's Y: helper warp 0
-                    // (as a whole warp) waits for every CTA's arrival and publishes the phase
-                    // in a shared counter that the other helper warps poll (a monotonic
-                    // count, so a warp that looks late still sees it)
-                    if (h == 0) {
-                        const bool all = grid_wait(P.phase_cnt + tc.ph - 1, (int)gridDim.x, abort_flag,
-                                                   P.wait_cycles);
-                        __syncwarp();
-                        if (!all) break;
-                        __threadfence();
-                        if (lane == 0) *reinterpret_cast<volatile int*>(&s_gate) = tc.ph;
-                    } else if (!gate_wait(&s_gate, tc.ph, abort_flag, P.wait_cycles)) {
-                        break;
+            if (chain && tc.ph > passed) {
+                // helper warp 0 (as a whole warp) reads the arrivals of every CTA and
+                // publishes the phase in a shared counter that the other helper warps read
+                // (a monotonic count, so a warp that looks late still sees it)
+                if (h == 0) {
+                    const int st = grid_poll(P.phase_cnt + tc.ph - 1, (int)gridDim.x, abort_flag, P.wait_cycles,
+                                             block, lane);
+                    if (st != 1) {
+                        fail = st < 0;
+                        return false;
                     }
                     __threadfence();
-                    passed = tc.ph;
+                    if (lane == 0) *reinterpret_cast<volatile int*>(&s_gate) = tc.ph;
+                } else if (block) {
+                    if (!gate_wait(&s_gate, tc.ph, abort_flag, P.wait_cycles)) {
+                        fail = true;
+                        return false;
+                    }
+                } else if (*reinterpret_cast<volatile int*>(&s_gate) < tc.ph) {
+                    return false;
                 }
-                // activations: token m's row of X starts K bf16 (words * 8 groups of 4) after
-                // token m-1's; read through L2 (a chained phase's X is written by this launch)
-                auto load_x = [&](const SProb& px, int sub) {
-#pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        xn[m] = __ldcg(reinterpret_cast<const uint2*>(px.X) + (int64_t)m * px.words * 8 +
-                                       sub * G::kTabs + ht);
-                };
-                if (ht < G::kTabs) {
-                    if (!have_x) load_x(P.p[tc.pos.p], tc.pos.sub);
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) build_table(luts + s * C::kLutStage + m * G::kLut + ht * kTab, xn[m]);
-                    mbar_arrive(ready(s));
-                }
-                tc.next(P);
-                // the next unit's activations are fetched now unless it opens a phase that is
-                // still being written
-                have_x = ht < G::kTabs && jt + 1 < nu && (!chain || tc.ph <= passed);
-                if (have_x) load_x(P.p[tc.pos.p], tc.pos.sub);
+                __threadfence();
+                passed = tc.ph;
+                have_x = false;
             }
+            const int s = jt % S;
+            if (!have_x) load_x(P.p[tc.pos.p], tc.pos.sub);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) build_table(luts + s * C::kLutStage + m * G::kLut + ht * kTab, xn[m]);
+            mbar_arrive(ready(s));
+            tc.next(P);
+            ++jt;
+            // the next unit's activations are fetched now unless it opens a phase that is
+            // still being written
+            have_x = jt < nu && (!chain || tc.ph <= passed);
+            if (have_x) load_x(P.p[tc.pos.p], tc.pos.sub);
+            return true;
+        };
+        for (int j = 0; j < nu && !fail; ++j) {
+            const int s = j % S;
+            if (j >= S) {
+                // the consumers free stage s after unit j - S, whose tables must exist
+                while (jt <= j - S && tables(true)) {
+                }
+                if (fail || !mbar_wait(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag, P.wait_cycles)) break;
+            }
+            const SProb& pr = P.p[cc.pos.p];
+            if (cc.pos.p != cr_p || cc.pos.rb != cr_rb) {
+                copy_rows<W>(pr, cc.pos.rb, h, lane, cr);
+                cr_p = cc.pos.p;
+                cr_rb = cc.pos.rb;
+            }
+            copy_unit<W>(pr, cr, cc.pos.sub, stages + s * G::kStage, h, lane);
+            cp_async_arrive(ready(s));
+            cc.next(P);
+            while (jt <= j && tables(false)) {
+            }
+        }
+        while (!fail && jt < nu && tables(true)) {
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else {
@@ -729,7 +765,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
 // (whole groups per unit), or row scales.
 template <int W>
 static bool stream_eligible_w(const ProbShape& s, int64_t M) {
-    if ((M != 1 && M != 2) || s.N == 0) return false;
+    if (M < 1 || M > (W == 16 ? 2 : 4) || s.N == 0) return false;
     if ((s.N + kSRows - 1) / kSRows > kMaxTickets - kChainCtrs) return false;
     if (s.K % (32 * W) != 0) return false;
     if (s.N * (s.K / 8) >= (int64_t(1) << 32) - 64) return false;  // 32-bit byte offsets into the planes
@@ -738,7 +774,10 @@ static bool stream_eligible_w(const ProbShape& s, int64_t M) {
     return s.group == 128 || s.group == 256;
 }
 
-bool stream_eligible(const ProbShape& s, int64_t M) { return stream_eligible_w<16>(s, M); }
+// one or two tokens: 16-word units; three or four: 8-word units
+bool stream_eligible(const ProbShape& s, int64_t M) {
+    return M <= 2 ? stream_eligible_w<16>(s, M) : stream_eligible_w<8>(s, M);
+}
 bool chain_eligible(const ProbShape& s, int64_t M) { return stream_eligible_w<8>(s, M); }
 
 int64_t stream_tiles(const ProbShape& s) { return (s.N + kSRows - 1) / kSRows; }
@@ -804,7 +843,7 @@ static SPlan make_splan(const ProbShape* shapes, int count, const int* phase_beg
 }
 
 size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
-    return make_splan(shapes, count, nullptr, 1, M, sms, 16).ws_bytes;
+    return make_splan(shapes, count, nullptr, 1, M, sms, M <= 2 ? 16 : 8).ws_bytes;
 }
 
 size_t chain_workspace_bytes(const ProbShape* shapes, int count, const int* phase_begin, int n_phases, int64_t M,
@@ -876,16 +915,20 @@ static void attach(SPlan& pl, const sherry_linear_desc* descs, int count) {
 
 int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream) {
-    if (M != 1 && M != 2) return SHERRY_ERR_UNSUPPORTED;
-    SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, 16);
+    if (M < 1 || M > 4) return SHERRY_ERR_UNSUPPORTED;
+    SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, M <= 2 ? 16 : 8);
     attach(pl, descs, count);
     if (pl.total_units == 0) return SHERRY_OK;
-    return M == 1 ? stream_launch_mt<1, 16>(pl, count, y_bf16, workspace, false, stream)
-                  : stream_launch_mt<2, 16>(pl, count, y_bf16, workspace, false, stream);
+    switch (M) {
+        case 1: return stream_launch_mt<1, 16>(pl, count, y_bf16, workspace, false, stream);
+        case 2: return stream_launch_mt<2, 16>(pl, count, y_bf16, workspace, false, stream);
+        case 3: return stream_launch_mt<3, 8>(pl, count, y_bf16, workspace, false, stream);
+        default: return stream_launch_mt<4, 8>(pl, count, y_bf16, workspace, false, stream);
+    }
 }
 
 bool chain_launch_ok(const ProbShape* shapes, int count, int n_phases, int64_t M) {
-    if ((M != 1 && M != 2) || n_phases > kSMaxPhases || n_phases > SHERRY_MAX_BATCH || count > SHERRY_MAX_BATCH)
+    if (M < 1 || M > 4 || n_phases > kSMaxPhases || n_phases > SHERRY_MAX_BATCH || count > SHERRY_MAX_BATCH)
         return false;
     int64_t tiles = 0;
     for (int i = 0; i < count; ++i) {
@@ -902,8 +945,12 @@ int chain_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs
     attach(pl, descs, count);
     // the kernel's phase table has one slot per problem slot of its instantiation
     const int slots = std::max(count, n_phases);
-    return M == 1 ? stream_launch_mt<1, 8>(pl, slots, y_bf16, workspace, true, stream)
-                  : stream_launch_mt<2, 8>(pl, slots, y_bf16, workspace, true, stream);
+    switch (M) {
+        case 1: return stream_launch_mt<1, 8>(pl, slots, y_bf16, workspace, true, stream);
+        case 2: return stream_launch_mt<2, 8>(pl, slots, y_bf16, workspace, true, stream);
+        case 3: return stream_launch_mt<3, 8>(pl, slots, y_bf16, workspace, true, stream);
+        default: return stream_launch_mt<4, 8>(pl, slots, y_bf16, workspace, true, stream);
+    }
 }
 
 int stream_status_take() {

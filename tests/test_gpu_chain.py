@@ -92,7 +92,7 @@ def _oracle_chain(orc, packs, X0, M, d, f, gran, group):
     return refs
 
 
-@pytest.mark.parametrize("M", [1, 2])
+@pytest.mark.parametrize("M", [1, 2, 4])
 @pytest.mark.parametrize("gran,group", [("group", 128), ("channel", 128), ("group", 256)])
 def test_chain_vs_oracle_chain(sw, orc_omp, M, gran, group):
     import torch
@@ -139,10 +139,10 @@ def test_chain_single_phase_matches_oracle_fp32(sw, orc):
 
 
 def test_chain_fallback_routes(sw, orc):
-    """Phases the chained kernel does not take (K % 256 != 0, four tokens) run as
+    """Phases the chained kernel does not take (K % 256 != 0, five tokens) run as
     ordered batched launches; results still follow the chain."""
     import torch
-    for M, K1 in ((1, 96), (4, 512)):
+    for M, K1 in ((1, 96), (5, 512)):
         g = oracle.PER_GROUP
         W1 = synth.weights_student_t(K1 * 2, K1, 33000)
         W2 = synth.weights_student_t(300, K1 * 2, 33001)

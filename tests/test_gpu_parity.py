@@ -134,8 +134,11 @@ LIN_CASES = [
     (2, 513, 1024, "channel", 0),
     (2, 77, 1536, "group", 256),
     (2, 1000, 8192, "tensor", 0),
-    (3, 64, 3072, "channel", 0),
+    (3, 64, 3072, "channel", 0),    # three and four tokens: streaming kernel, 8-word units
+    (3, 1000, 2048, "group", 256),
     (4, 500, 1024, "group", 128),
+    (4, 77, 768, "tensor", 0),
+    (4, 100, 96, "group", 32),      # K % 256 != 0: general kernel
     (5, 33, 256, "tensor", 0),
     (8, 1024, 3072, "group", 128),
     (16, 512, 2048, "group", 128),
@@ -232,11 +235,11 @@ STREAM_SHAPES = [(1024, 3072, "group", 128), (300, 3072, "channel", 0), (3072, 8
                  (1, 512, "group", 128), (257, 3072, "group", 256), (96, 1536, "group", 256)]
 
 
-@pytest.mark.parametrize("M", [1, 2])
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
 def test_stream_batch_many_problems_vs_oracle(sw, orc, M):
-    """One- and two-token batches of many eligible linears (the streaming kernel:
-    units split evenly over CTAs, tiles straddling two CTAs finished through the
-    ticket)."""
+    """Batches of one to four tokens over many eligible linears (the streaming
+    kernel: units split evenly over CTAs, tiles straddling CTAs finished through
+    the ticket)."""
     import torch
     pairs, refs = [], []
     for i in range(24):
@@ -443,8 +446,10 @@ MAXK_CASES = [
     # (M, N, gran, group) at K = SHERRY_MAX_K: one case per linear kernel route
     (1, 5, "group", 128),   # one-token streaming kernel
     (2, 5, "group", 128),   # two-token streaming kernel
+    (3, 5, "channel", 0),   # three-token streaming kernel (8-word units)
+    (4, 5, "group", 256),   # four-token streaming kernel
     (1, 3, "group", 32),    # general lookup-table kernel
-    (4, 5, "group", 128),   # warp-MMA kernel
+    (5, 5, "group", 128),   # warp-MMA kernel
     (16, 3, "channel", 0),  # tcgen05 few-token kernel
     (64, 3, "group", 256),  # tcgen05 prefill kernel
 ]
