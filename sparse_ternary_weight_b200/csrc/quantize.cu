@@ -34,9 +34,9 @@
 
 namespace sherry {
 
-constexpr int kQThreads = 256;
+constexpr int kQThreads = 128;
 constexpr int kQUnroll = 2;      // warp-steps (16 weights per lane each) in flight
-constexpr int kQCtasPerSm = 8;   // resident CTAs per SM (256 threads each)
+constexpr int kQCtasPerSm = 16;  // CTAs per SM in the grid (128 threads each; registers allow about 10 resident)
 
 // 5-bit code (nibble 4z + 2 d1 + d2, plus 16 G) of a block whose smallest |w|
 // is at z and whose negative weights are the set bits of `neg` (w < 0; -0.0 is
