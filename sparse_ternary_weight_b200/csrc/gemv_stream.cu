@@ -6,8 +6,8 @@
 // Y = X T alpha).
 //
 // Work unit: 512 output rows x 32 W weights (W packed words) of one linear, W =
-// 16 for independent linears of one or two tokens (one batched launch per decode
-// step), W = 8 for three or four tokens (whose tables take more shared memory) and
+// 16 for independent linears of one to three tokens (one batched launch per decode
+// step), W = 8 for four tokens (whose tables take more shared memory) and
 // for chained phases, whose layers are small enough that finer units balance better.
 // All units of a phase (one or many independent linears) are split into equal
 // contiguous ranges, one per CTA (stream-K): every CTA streams the same number
@@ -54,6 +54,7 @@ constexpr int kSRows = 32 * kSConsumers;           // 512 rows per unit
 constexpr int kSBars = 128;                        // mbarriers
 constexpr int kSHelperThreads = 32 * kSHelpers;
 constexpr int kSHelperRows = kSRows / kSHelpers;   // rows each helper warp copies
+constexpr int kSRed = 8;                           // split-tile partials loaded at a time
 static_assert(kSHelperRows % 32 == 0, "whole rows per helper lane");
 // chained launches keep their phase counters at the end of the ticket region
 constexpr int kChainCtrs = 512;                    // up to 511 phases + the exit counter
@@ -79,13 +80,13 @@ struct SGeo {
 
 // Ring depth and shared bytes for MT tokens and W-word units (tables are
 // token-major within a stage): as many stages as fit next to one CTA's
-// registers; three or four tokens take 8-word units (a 16-word stage with their
-// tables leaves room for one stage only).
+// registers; four tokens take 8-word units (a 16-word stage with their tables
+// leaves room for one stage only).
 template <int MT, int W>
 struct SCfg {
     using G = SGeo<W>;
     static constexpr int kStages =
-        W == 16 ? (MT == 1 ? 3 : MT == 2 ? 2 : 1) : (MT == 1 ? 6 : MT == 2 ? 5 : MT == 3 ? 4 : 3);
+        W == 16 ? (MT == 1 ? 3 : MT <= 3 ? 2 : 1) : (MT == 1 ? 6 : MT == 2 ? 5 : MT == 3 ? 4 : 3);
     static constexpr int kLutStage = MT * G::kLut;
     static constexpr int kSmem = 256 + kStages * (G::kStage + kLutStage) + kSBars;
     static_assert(kSmem <= 232448, "shared memory per CTA");
@@ -185,6 +186,11 @@ __device__ __forceinline__ bool gate_wait(const int* gate, int target, volatile 
             return false;
         }
     }
+}
+// arrival at a phase counter: a release at GPU scope (the Y this CTA wrote, seen by
+// this thread through the CTA's mbarrier, is visible before the count), no reply
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ int ld_acquire(const int* p) {
     int v;
@@ -697,14 +703,32 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                             }
                             if (s_last) {
                                 __threadfence();
+                                // the partials of CTAs c_a..c_b added in CTA order; their loads are
+                                // issued kSRed at a time (a chained phase splits a tile over up to
+                                // 32 CTAs, and one dependent L2 round trip each would dominate it)
+                                float sums[MT];
+#pragma unroll
+                                for (int m = 0; m < MT; ++m) sums[m] = 0.0f;
+                                for (int c0 = c_a; c0 <= c_b; c0 += kSRed) {
+                                    float pv[kSRed][MT];
+#pragma unroll
+                                    for (int i = 0; i < kSRed; ++i) {
+                                        const int c = c0 + i;
+                                        const int sl = (pb + c * upc >= tile_u0) ? 0 : 1;
+#pragma unroll
+                                        for (int m = 0; m < MT; ++m)
+                                            pv[i][m] = c <= c_b ? __ldcg(P.part + (((int64_t)c * 2 + sl) * MT + m) * kSRows + r)
+                                                                : 0.0f;
+                                    }
+#pragma unroll
+                                    for (int i = 0; i < kSRed; ++i)
+#pragma unroll
+                                        for (int m = 0; m < MT; ++m)
+                                            if (c0 + i <= c_b) sums[m] = (c0 + i == c_a) ? pv[i][m] : sums[m] + pv[i][m];
+                                }
 #pragma unroll
                                 for (int m = 0; m < MT; ++m) {
-                                    float sum = 0.0f;
-                                    for (int c = c_a; c <= c_b; ++c) {
-                                        const int sl = (pb + c * upc >= tile_u0) ? 0 : 1;
-                                        const float pv = __ldcg(P.part + (((int64_t)c * 2 + sl) * MT + m) * kSRows + r);
-                                        sum = (c == c_a) ? pv : sum + pv;
-                                    }
+                                    const float sum = sums[m];
                                     if (row_ok) {
                                         if (P.y_bf16)
                                             reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)m * pr.N + n] =
@@ -730,10 +754,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                     mbar_arrive(bar_phase);
                     if (warp == 0) {
                         const bool done = mbar_wait(bar_phase, (uint32_t)(phases & 1), abort_flag, P.wait_cycles);
-                        if (done && lane == 0) {
-                            __threadfence();
-                            atomicAdd(P.phase_cnt + ph, 1);
-                        }
+                        if (done && lane == 0) red_release_add(P.phase_cnt + ph, 1);
                         __syncwarp();
                         if (!done) {
                             ok = false;
@@ -743,7 +764,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                     ++phases;
                 }
             } else if (chain && r == 0) {
-                atomicAdd(P.phase_cnt + ph, 1);  // nothing of this phase here
+                red_release_add(P.phase_cnt + ph, 1);  // nothing of this phase here
             }
         }
     }
@@ -765,7 +786,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
 // (whole groups per unit), or row scales.
 template <int W>
 static bool stream_eligible_w(const ProbShape& s, int64_t M) {
-    if (M < 1 || M > (W == 16 ? 2 : 4) || s.N == 0) return false;
+    if (M < 1 || M > (W == 16 ? 3 : 4) || s.N == 0) return false;
     if ((s.N + kSRows - 1) / kSRows > kMaxTickets - kChainCtrs) return false;
     if (s.K % (32 * W) != 0) return false;
     if (s.N * (s.K / 8) >= (int64_t(1) << 32) - 64) return false;  // 32-bit byte offsets into the planes
@@ -774,9 +795,9 @@ static bool stream_eligible_w(const ProbShape& s, int64_t M) {
     return s.group == 128 || s.group == 256;
 }
 
-// one or two tokens: 16-word units; three or four: 8-word units
+// one to three tokens: 16-word units; four: 8-word units
 bool stream_eligible(const ProbShape& s, int64_t M) {
-    return M <= 2 ? stream_eligible_w<16>(s, M) : stream_eligible_w<8>(s, M);
+    return M <= 3 ? stream_eligible_w<16>(s, M) : stream_eligible_w<8>(s, M);
 }
 bool chain_eligible(const ProbShape& s, int64_t M) { return stream_eligible_w<8>(s, M); }
 
@@ -843,7 +864,7 @@ static SPlan make_splan(const ProbShape* shapes, int count, const int* phase_beg
 }
 
 size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
-    return make_splan(shapes, count, nullptr, 1, M, sms, M <= 2 ? 16 : 8).ws_bytes;
+    return make_splan(shapes, count, nullptr, 1, M, sms, M <= 3 ? 16 : 8).ws_bytes;
 }
 
 size_t chain_workspace_bytes(const ProbShape* shapes, int count, const int* phase_begin, int n_phases, int64_t M,
@@ -916,13 +937,13 @@ static void attach(SPlan& pl, const sherry_linear_desc* descs, int count) {
 int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream) {
     if (M < 1 || M > 4) return SHERRY_ERR_UNSUPPORTED;
-    SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, M <= 2 ? 16 : 8);
+    SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, M <= 3 ? 16 : 8);
     attach(pl, descs, count);
     if (pl.total_units == 0) return SHERRY_OK;
     switch (M) {
         case 1: return stream_launch_mt<1, 16>(pl, count, y_bf16, workspace, false, stream);
         case 2: return stream_launch_mt<2, 16>(pl, count, y_bf16, workspace, false, stream);
-        case 3: return stream_launch_mt<3, 8>(pl, count, y_bf16, workspace, false, stream);
+        case 3: return stream_launch_mt<3, 16>(pl, count, y_bf16, workspace, false, stream);
         default: return stream_launch_mt<4, 8>(pl, count, y_bf16, workspace, false, stream);
     }
 }

@@ -134,7 +134,7 @@ LIN_CASES = [
     (2, 513, 1024, "channel", 0),
     (2, 77, 1536, "group", 256),
     (2, 1000, 8192, "tensor", 0),
-    (3, 64, 3072, "channel", 0),    # three and four tokens: streaming kernel, 8-word units
+    (3, 64, 3072, "channel", 0),    # three and four tokens: streaming kernel (four: 8-word units)
     (3, 1000, 2048, "group", 256),
     (4, 500, 1024, "group", 128),
     (4, 77, 768, "tensor", 0),
@@ -446,8 +446,8 @@ MAXK_CASES = [
     # (M, N, gran, group) at K = SHERRY_MAX_K: one case per linear kernel route
     (1, 5, "group", 128),   # one-token streaming kernel
     (2, 5, "group", 128),   # two-token streaming kernel
-    (3, 5, "channel", 0),   # three-token streaming kernel (8-word units)
-    (4, 5, "group", 256),   # four-token streaming kernel
+    (3, 5, "channel", 0),   # three-token streaming kernel
+    (4, 5, "group", 256),   # four-token streaming kernel (8-word units)
     (1, 3, "group", 32),    # general lookup-table kernel
     (5, 5, "group", 128),   # warp-MMA kernel
     (16, 3, "channel", 0),  # tcgen05 few-token kernel
