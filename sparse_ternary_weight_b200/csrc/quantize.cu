@@ -67,35 +67,18 @@ __device__ __forceinline__ uint32_t encode4(float w0, float w1, float w2, float 
     return ctab[(z << 4) | neg];
 }
 
-__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-    return v;
-}
-
-// 16 consecutive weights (4 blocks) per lane, from global memory or from this
-// thread's own copy of them in the shared-memory row ring
+// 16 consecutive weights (4 blocks) per lane
 template <bool kBF16>
 struct WLoad;
 
 template <>
 struct WLoad<false> {
     struct T { float4 q[4]; };
-    static constexpr int kPiece = 64;  // bytes of 16 weights
     __device__ __forceinline__ static T load(const void* W, int64_t off16) {
         const float4* p = reinterpret_cast<const float4*>(W) + off16 * 4;
         T v;
 #pragma unroll
         for (int i = 0; i < 4; ++i) v.q[i] = __ldcs(p + i);
-        return v;
-    }
-    __device__ __forceinline__ static T load_s(uint32_t a) {
-        T v;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint4 u = lds_v4(a + 16u * i);
-            v.q[i] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
-        }
         return v;
     }
     __device__ __forceinline__ static void block(const T& v, int j, float& a, float& b, float& c, float& d) {
@@ -112,18 +95,11 @@ struct WLoad<false> {
 template <>
 struct WLoad<true> {
     struct T { uint4 q[2]; };
-    static constexpr int kPiece = 32;  // bytes of 16 weights
     __device__ __forceinline__ static T load(const void* W, int64_t off16) {
         const uint4* p = reinterpret_cast<const uint4*>(W) + off16 * 2;
         T v;
         v.q[0] = __ldcs(p);
         v.q[1] = __ldcs(p + 1);
-        return v;
-    }
-    __device__ __forceinline__ static T load_s(uint32_t a) {
-        T v;
-        v.q[0] = lds_v4(a);
-        v.q[1] = lds_v4(a + 16u);
         return v;
     }
     __device__ __forceinline__ static void block(const T& v, int j, float& a, float& b, float& c, float& d) {
@@ -164,53 +140,14 @@ struct QProb {
 template <int MAXP>
 struct QParams {
     int count;
-    int ring_bytes;  // shared-memory row ring per CTA (0: rows are read from global memory directly)
     int64_t total_rows;
     QProb p[MAXP];
 };
 
-constexpr int kQLook = 8;             // rows in the ring at most (cp.async groups in flight)
-constexpr int kQRingBytes = 64 << 10; // ring size when the largest row fits twice
-constexpr int kQRingMaxRow = 32 << 10;
-
-__device__ __forceinline__ void q_cp16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-// wait until at most n (0..kQLook-1) of this thread's cp.async groups are pending
-__device__ __forceinline__ void q_wait_groups(int n) {
-    switch (n) {
-        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
-        case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
-        case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
-        default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
-    }
-}
-// This thread's copies of row n of `pr` into the ring at shared address dst: the
-// same 16-weight pieces encode_row gives this thread, at the same offsets, so a
-// thread only ever reads back its own copies.  One cp.async group per row.
-__device__ __forceinline__ void ring_issue(const QProb& pr, int64_t n, uint32_t dst) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n16 = pr.K >> 4, nsteps = (n16 + 31) >> 5;
-    const int pb = pr.w_bf16 ? 32 : 64;
-    const char* src = static_cast<const char*>(pr.W) + n * (int64_t)n16 * pb;
-    for (int c = warp; c < nsteps; c += kQThreads / 32) {
-        const int piece = c * 32 + lane;
-        if (piece < n16)
-            for (int i = 0; i < pb; i += 16) q_cp16(dst + (uint32_t)(piece * pb + i), src + (int64_t)piece * pb + i);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// Packed words, sign bytes and word sums of row n (phase 1).  W comes from global
-// memory, or (ring != 0) from the row's place in the shared-memory ring, where
-// this thread copied exactly the pieces it reads here.
+// Packed words, sign bytes and word sums of row n (phase 1).
 template <bool kBF16>
 __device__ __forceinline__ void encode_row(const QProb& pr, int64_t n, const uint8_t* ctab, float* wsum,
-                                           float* dsum, uint32_t ring) {
+                                           float* dsum) {
     using L = WLoad<kBF16>;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -224,8 +161,7 @@ __device__ __forceinline__ void encode_row(const QProb& pr, int64_t n, const uin
 #pragma unroll
         for (int u = 0; u < kQUnroll; ++u) {
             const int piece = (c0 + (kQThreads / 32) * u) * 32 + lane;
-            const bool in = c0 + (kQThreads / 32) * u < nsteps && piece < n16;
-            v[u] = !in ? L::zero() : ring ? L::load_s(ring + (uint32_t)(piece * L::kPiece)) : L::load(pr.W, row16 + piece);
+            v[u] = (c0 + (kQThreads / 32) * u < nsteps && piece < n16) ? L::load(pr.W, row16 + piece) : L::zero();
         }
 #pragma unroll
         for (int u = 0; u < kQUnroll; ++u) {
@@ -282,8 +218,7 @@ __device__ __forceinline__ void encode_row(const QProb& pr, int64_t n, const uin
 
 template <int MAXP>
 __global__ void __launch_bounds__(kQThreads) k_quantize(const __grid_constant__ QParams<MAXP> P) {
-    // [ring_bytes] row ring, then [words] word sums, [words] dead-value sums, [ngroups] scales of the row
-    extern __shared__ __align__(16) float qsm_raw[];
+    extern __shared__ float qsm[];   // [words] word sums, [words] dead-value sums, [ngroups] scales of the row
     __shared__ uint8_t ctab[64];     // 5-bit code by (zero position, negative bits)
     __shared__ float4 tpat[32];      // the block's ternary values by 5-bit code
     if (threadIdx.x < 64) ctab[threadIdx.x] = (uint8_t)code_of(threadIdx.x >> 4, threadIdx.x & 15u);
@@ -300,40 +235,6 @@ __global__ void __launch_bounds__(kQThreads) k_quantize(const __grid_constant__ 
     }
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    float* const qsm = qsm_raw + P.ring_bytes / 4;
-    // Row ring: the CTA's next rows are copied ahead (cp.async, one group per row)
-    // while it encodes the current one.  Rows take their own size in a circular
-    // byte buffer (skipping to its start when a row does not fit before the end);
-    // a row's bytes are reused only after every thread has passed the barrier that
-    // follows its encoding.  Every thread keeps the same bookkeeping.
-    const int rb = P.ring_bytes;
-    const uint32_t ring = smem_u32(qsm_raw);
-    int64_t ir = blockIdx.x;  // next row to copy
-    int ipi = 0;              // its problem
-    int ioff = 0, live = 0;   // next free byte; bytes held by copied, unfinished rows (with skips)
-    int issued = 0, done = 0;
-    int q_off[kQLook], q_fp[kQLook];
-    auto issue = [&]() {
-        while (rb && ir < P.total_rows && issued - done < kQLook) {
-            while (ipi + 1 < P.count && P.p[ipi + 1].row_begin <= ir) ++ipi;
-            const QProb& q = P.p[ipi];
-            const int b = q.K * (q.w_bf16 ? 2 : 4);
-            int off = ioff, fp = b;
-            if (off + b > rb) {
-                fp += rb - off;
-                off = 0;
-            }
-            if (live + fp > rb) break;
-            ring_issue(q, ir - q.row_begin, ring + (uint32_t)off);
-            q_off[issued % kQLook] = off;
-            q_fp[issued % kQLook] = fp;
-            ioff = off + b;
-            live += fp;
-            ++issued;
-            ir += gridDim.x;
-        }
-    };
-    issue();
     int pi = 0;  // rows are visited in increasing order per CTA
     for (int64_t r = blockIdx.x; r < P.total_rows; r += gridDim.x) {
         while (pi + 1 < P.count && P.p[pi + 1].row_begin <= r) ++pi;
@@ -344,21 +245,11 @@ __global__ void __launch_bounds__(kQThreads) k_quantize(const __grid_constant__ 
         float* dsum = qsm + words;            // dead-value word sums (Tequila plane)
         float* srow = qsm + 2 * words;
         __syncthreads();  // the tables are ready; the previous row is done with the shared buffers
-        uint32_t src = 0;
-        if (rb) {
-            q_wait_groups(issued - done - 1);  // this row's copies (made by this thread) have landed
-            src = ring + (uint32_t)q_off[done % kQLook];
-        }
         if (pr.w_bf16)
-            encode_row<true>(pr, n, ctab, wsum, dsum, src);
+            encode_row<true>(pr, n, ctab, wsum, dsum);
         else
-            encode_row<false>(pr, n, ctab, wsum, dsum, src);
+            encode_row<false>(pr, n, ctab, wsum, dsum);
         __syncthreads();
-        if (rb) {  // the row's ring bytes are free: copy further rows
-            live -= q_fp[done % kQLook];
-            ++done;
-            issue();
-        }
         if (pr.dead_sum && warp == (kQThreads / 32) - 1) {
             const float B = warp_tree_sum(dsum, words);
             if (lane == 0) pr.dead_sum[n] = B;
@@ -523,30 +414,25 @@ static int quantize_launch_t(const std::vector<QProb>& probs, int64_t rows, int 
     std::lock_guard<std::mutex> lk(mu);
     P.count = (int)probs.size();
     P.total_rows = rows;
-    int maxw = 0, maxg = 1, max_row = 0;
+    int maxw = 0, maxg = 1;
     for (int i = 0; i < P.count; ++i) {
         P.p[i] = probs[i];
         maxw = std::max(maxw, probs[i].K / 32);
         if (probs[i].mode == kQGroup) maxg = std::max(maxg, probs[i].K / 32 / probs[i].gw);
-        max_row = std::max(max_row, probs[i].K * (probs[i].w_bf16 ? 2 : 4));
     }
-    // the row ring when the largest row fits it twice (K <= 8192 fp32, 16384 bf16)
-    P.ring_bytes = max_row <= kQRingMaxRow ? std::max(kQRingBytes, 2 * max_row) : 0;
-    const size_t smem = (size_t)P.ring_bytes + (size_t)(2 * maxw + maxg) * sizeof(float);
+    const size_t smem = (size_t)(2 * maxw + maxg) * sizeof(float);
     if (smem > 48 * 1024) {
         static PerDevice attr;
         int done = 0;
         const int st = per_device(attr, &done, [](int& v) {
             SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_quantize<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   kQRingBytes + 3 * (SHERRY_MAX_K / 32) * (int)sizeof(float)));
+                                                   3 * (SHERRY_MAX_K / 32) * (int)sizeof(float)));
             v = 1;
             return SHERRY_OK;
         });
         if (st) return st;
     }
-    // as many CTAs per SM as shared memory holds (and at most kQCtasPerSm)
-    const int per_sm = std::max(1, std::min(kQCtasPerSm, (int)(227 * 1024 / (smem + 1024))));
-    const int64_t grid = std::min<int64_t>(rows, (int64_t)sms * per_sm);
+    const int64_t grid = std::min<int64_t>(rows, (int64_t)sms * kQCtasPerSm);
     k_quantize<MAXP><<<(unsigned)grid, kQThreads, smem, stream>>>(P);
     SHERRY_LAUNCH_CHECK();
     return SHERRY_OK;
