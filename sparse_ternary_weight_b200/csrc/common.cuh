@@ -97,6 +97,21 @@ __device__ __forceinline__ float tree_sum_seq(const float* v, int n) {
     return r;
 }
 
+// The same canonical sum for n <= 8 (n <= 16), in registers: padding to 8 (16)
+// adds whole zero subtrees, which is exact for values >= 0, so the result equals
+// the tree over the next power of two of n.
+__device__ __forceinline__ float tree_sum8(const float* v, int n) {
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = i < n ? v[i] : 0.0f;
+    return ((x[0] + x[1]) + (x[2] + x[3])) + ((x[4] + x[5]) + (x[6] + x[7]));
+}
+__device__ __forceinline__ float tree_sum16(const float* v, int n) {
+    const float a = tree_sum8(v, n < 8 ? n : 8);
+    const float b = n > 8 ? tree_sum8(v + 8, n - 8) : 0.0f;
+    return a + b;
+}
+
 // Canonical pairwise sum of v[0..n) by one full warp; the result is returned in
 // every lane.  Each lane reduces an aligned power-of-two segment sequentially,
 // then the xor butterfly (offsets 1, 2, 4, ...) combines adjacent segments,
@@ -114,7 +129,7 @@ __device__ __forceinline__ float warp_tree_sum(const float* v, int n) {
         int lo = lane * seg;
         int cnt = n - lo;
         cnt = cnt < 0 ? 0 : (cnt > seg ? seg : cnt);
-        x = tree_sum_seq(v + lo, cnt);
+        x = seg <= 8 ? tree_sum8(v + lo, cnt) : seg <= 16 ? tree_sum16(v + lo, cnt) : tree_sum_seq(v + lo, cnt);
         span = 32;
     }
     for (int off = 1; off < span; off <<= 1) x = x + __shfl_xor_sync(kFull, x, off);

@@ -55,15 +55,17 @@ __host__ __device__ __forceinline__ uint32_t code_of(uint32_t z, uint32_t neg) {
 __device__ __forceinline__ uint32_t encode4(float w0, float w1, float w2, float w3, const uint8_t* ctab,
                                             float& mag) {
     const float a0 = fabsf(w0), a1 = fabsf(w1), a2 = fabsf(w2), a3 = fabsf(w3);
-    // first index of the minimum |w| (strict < keeps the earlier index on ties)
-    uint32_t z = 0;
-    float m = a0;
-    if (a1 < m) { z = 1; m = a1; }
-    if (a2 < m) { z = 2; m = a2; }
-    if (a3 < m) { z = 3; }
+    // first index of the minimum |w|, as a tournament of pairs (strict < keeps the
+    // earlier index on ties, inside a pair and between the pairs)
+    const bool hi = fminf(a2, a3) < fminf(a0, a1);     // the zero falls in the second pair
+    const uint32_t z = hi ? (a3 < a2 ? 3u : 2u) : (a1 < a0 ? 1u : 0u);
     const uint32_t neg = (w0 < 0.0f ? 1u : 0u) | (w1 < 0.0f ? 2u : 0u) | (w2 < 0.0f ? 4u : 0u) |
                          (w3 < 0.0f ? 8u : 0u);
-    mag = ((z == 0 ? 0.0f : a0) + (z == 1 ? 0.0f : a1)) + ((z == 2 ? 0.0f : a2) + (z == 3 ? 0.0f : a3));
+    // masked sum (m0 + m1) + (m2 + m3) with the zeroed weight as +0.0: in the pair
+    // holding the zero, +0.0 + the other |w| is that |w|, i.e. the pair's max
+    const float s01 = hi ? a0 + a1 : fmaxf(a0, a1);
+    const float s23 = hi ? fmaxf(a2, a3) : a2 + a3;
+    mag = s01 + s23;
     return ctab[(z << 4) | neg];
 }
 
@@ -268,6 +270,8 @@ __global__ void __launch_bounds__(kQThreads) k_quantize(const __grid_constant__ 
                     S = v[0];
                 } else if (gw == 2) {
                     S = v[0] + v[1];
+                } else if (gw <= 16) {
+                    S = tree_sum16(v, gw);
                 } else {
                     S = tree_sum_seq(v, gw);
                 }
