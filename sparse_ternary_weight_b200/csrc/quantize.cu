@@ -34,9 +34,9 @@
 
 namespace sherry {
 
-constexpr int kQThreads = 128;
+constexpr int kQThreads = 64;
 constexpr int kQUnroll = 2;      // warp-steps (16 weights per lane each) in flight
-constexpr int kQCtasPerSm = 16;  // CTAs per SM in the grid (128 threads each; registers allow about 10 resident)
+constexpr int kQCtasPerSm = 28;  // CTAs per SM in the grid (two warps each: many rows in flight per SM)
 
 // 5-bit code (nibble 4z + 2 d1 + d2, plus 16 G) of a block whose smallest |w|
 // is at z and whose negative weights are the set bits of `neg` (w < 0; -0.0 is
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(kQThreads) k_quantize(const __grid_constant__ 
     extern __shared__ float qsm[];   // [words] word sums, [words] dead-value sums, [ngroups] scales of the row
     __shared__ uint8_t ctab[64];     // 5-bit code by (zero position, negative bits)
     __shared__ float4 tpat[32];      // the block's ternary values by 5-bit code
-    if (threadIdx.x < 64) ctab[threadIdx.x] = (uint8_t)code_of(threadIdx.x >> 4, threadIdx.x & 15u);
+    for (int i = threadIdx.x; i < 64; i += kQThreads) ctab[i] = (uint8_t)code_of(i >> 4, i & 15u);
     if (threadIdx.x < 32) {
         // inverse of code_of: the kept signs in position order, the zero slot reinserted
         const uint32_t nib = threadIdx.x & 15u, g = threadIdx.x >> 4;
