@@ -197,8 +197,8 @@ size_t sherry_quantize_pack_batched_workspace_bytes(const sherry_quantize_desc* 
  *            fully overwritten
  *   workspace  sherry_workspace_bytes(SHERRY_OP_LINEAR, M, N, K, g, group) bytes
  * fp32 accumulation; alpha applied once per group (or row).  Kernels:
- * M <= 2 with K % 512 == 0 (group 128 or 256, per-channel or per-tensor) a
- * warp-specialised lookup-table decode kernel; other 2 <= M <= 8 with
+ * M <= 3 with K % 512 == 0, or M == 4 with K % 256 == 0 (group 128 or 256,
+ * per-channel or per-tensor) a warp-specialised lookup-table decode kernel; other 2 <= M <= 8 with
  * K % 128 == 0 a warp-level tensor-core (mma.sync) kernel; 9 <= M <= 32 with K % 256 == 0 and
  * (per-group) group % 64 == 0 a tensor-core (tcgen05) kernel for few tokens;
  * M >= 17 with K % 64 == 0 and group % 64 == 0 the tcgen05 prefill kernel;
@@ -264,8 +264,8 @@ float sherry_arenas_lambda(int64_t step, int64_t total, float lambda0);
  * phase's Y as its X (bf16 Y, y_dtype SHERRY_BF16, read in place).  Each Y is
  * computed as by sherry_linear (fp32 accumulation, alpha once per group), within
  * the fp32 summation-order bound of it.
- *   One and two tokens with every K % 256 == 0 and group 128 or 256 (or row
- *   scales): one cooperative launch (one CTA per SM, all resident) in which a
+ *   One to three tokens with every K % 512 == 0, or four tokens with every
+ *   K % 256 == 0, and group 128 or 256 (or row scales): one cooperative launch (one CTA per SM, all resident) in which a
  *   grid-wide bounded barrier separates the phases and the packed weights of the
  *   next phase stream in while it resolves ("Sherry: ..." digest: inference
  *   streams the packed weights through lookup tables; the pages' layer is

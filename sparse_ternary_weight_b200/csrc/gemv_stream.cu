@@ -6,9 +6,9 @@
 // Y = X T alpha).
 //
 // Work unit: 512 output rows x 32 W weights (W packed words) of one linear, W =
-// 16 for independent linears of one to three tokens (one batched launch per decode
-// step), W = 8 for four tokens (whose tables take more shared memory) and
-// for chained phases, whose layers are small enough that finer units balance better.
+// 16 for one to three tokens, W = 8 for four tokens (whose tables take more
+// shared memory); the same for independent linears (one batched launch per
+// decode step) and for chained phases.
 // All units of a phase (one or many independent linears) are split into equal
 // contiguous ranges, one per CTA (stream-K): every CTA streams the same number
 // of bytes.  A row block whose units straddle CTAs is finished by the CTA that
@@ -800,7 +800,9 @@ static bool stream_eligible_w(const ProbShape& s, int64_t M) {
 bool stream_eligible(const ProbShape& s, int64_t M) {
     return M <= 3 ? stream_eligible_w<16>(s, M) : stream_eligible_w<8>(s, M);
 }
-bool chain_eligible(const ProbShape& s, int64_t M) { return stream_eligible_w<8>(s, M); }
+bool chain_eligible(const ProbShape& s, int64_t M) {
+    return M <= 3 ? stream_eligible_w<16>(s, M) : stream_eligible_w<8>(s, M);
+}
 
 int64_t stream_tiles(const ProbShape& s) { return (s.N + kSRows - 1) / kSRows; }
 
@@ -870,7 +872,7 @@ size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int
 
 size_t chain_workspace_bytes(const ProbShape* shapes, int count, const int* phase_begin, int n_phases, int64_t M,
                              int sms) {
-    return make_splan(shapes, count, phase_begin, n_phases, M, sms, 8).ws_bytes;
+    return make_splan(shapes, count, phase_begin, n_phases, M, sms, M <= 3 ? 16 : 8).ws_bytes;
 }
 
 template <int MAXP, int MT, int W>
@@ -963,14 +965,14 @@ bool chain_launch_ok(const ProbShape* shapes, int count, int n_phases, int64_t M
 int chain_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, const int* phase_begin,
                         int n_phases, int64_t M, int y_bf16, void* workspace, int sms, cudaStream_t stream) {
     if (!chain_launch_ok(shapes, count, n_phases, M)) return SHERRY_ERR_UNSUPPORTED;
-    SPlan pl = make_splan(shapes, count, phase_begin, n_phases, M, sms, 8);
+    SPlan pl = make_splan(shapes, count, phase_begin, n_phases, M, sms, M <= 3 ? 16 : 8);
     attach(pl, descs, count);
     // the kernel's phase table has one slot per problem slot of its instantiation
     const int slots = std::max(count, n_phases);
     switch (M) {
-        case 1: return stream_launch_mt<1, 8>(pl, slots, y_bf16, workspace, true, stream);
-        case 2: return stream_launch_mt<2, 8>(pl, slots, y_bf16, workspace, true, stream);
-        case 3: return stream_launch_mt<3, 8>(pl, slots, y_bf16, workspace, true, stream);
+        case 1: return stream_launch_mt<1, 16>(pl, slots, y_bf16, workspace, true, stream);
+        case 2: return stream_launch_mt<2, 16>(pl, slots, y_bf16, workspace, true, stream);
+        case 3: return stream_launch_mt<3, 16>(pl, slots, y_bf16, workspace, true, stream);
         default: return stream_launch_mt<4, 8>(pl, slots, y_bf16, workspace, true, stream);
     }
 }

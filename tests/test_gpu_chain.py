@@ -122,7 +122,7 @@ def test_chain_single_phase_matches_oracle_fp32(sw, orc):
     gate and the fp32 accumulation bound of every element."""
     import torch
     from tests.gpu_common import check_linear
-    shapes = [(1000, 3072, "group", 128), (513, 2048, "channel", 0), (77, 1024, "group", 256), (2048, 256, "tensor", 0)]
+    shapes = [(1000, 3072, "group", 128), (513, 2048, "channel", 0), (77, 1024, "group", 256), (2048, 512, "tensor", 0)]
     ph, refs = [], []
     for i, (N, K, gname, group) in enumerate(shapes):
         g = GRAN[gname]
