@@ -31,6 +31,37 @@ static int device_sms() {
 
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Side streams for the prefill launches of one batched call, per device.  The
+// problems are independent linears, each a persistent grid over its own tiles; a
+// small one leaves SMs idle that the next one's CTAs can take if the launches
+// run on different streams.  They are forked from the caller's stream and joined
+// back into it with events, so stream order and graph capture hold.
+constexpr int kForkStreams = 4;
+struct ForkPool {
+    cudaStream_t s[kForkStreams];
+    cudaEvent_t fork, join[kForkStreams];
+    bool ready = false;
+};
+static std::mutex g_fork_mu;  // held for a whole fork/join (host-side enqueue only)
+static std::vector<ForkPool> g_fork;
+
+static int fork_pool(ForkPool** out) {
+    int dev = 0;
+    SHERRY_CUDA_CHECK(cudaGetDevice(&dev));
+    if ((int)g_fork.size() <= dev) g_fork.resize(dev + 1);
+    ForkPool& fp = g_fork[dev];
+    if (!fp.ready) {
+        for (int k = 0; k < kForkStreams; ++k) {
+            SHERRY_CUDA_CHECK(cudaStreamCreateWithFlags(&fp.s[k], cudaStreamNonBlocking));
+            SHERRY_CUDA_CHECK(cudaEventCreateWithFlags(&fp.join[k], cudaEventDisableTiming));
+        }
+        SHERRY_CUDA_CHECK(cudaEventCreateWithFlags(&fp.fork, cudaEventDisableTiming));
+        fp.ready = true;
+    }
+    *out = &fp;
+    return SHERRY_OK;
+}
+
 static int check_shape(int64_t N, int64_t K) {
     if (N < 0 || K < 32 || K > SHERRY_MAX_K || (K % 32) != 0) return SHERRY_ERR_SHAPE;
     if (N > (int64_t)0x7fffffff) return SHERRY_ERR_SHAPE;
@@ -50,7 +81,7 @@ static int check_planes(const uint32_t* idx, const uint8_t* sgn, const float* sc
     return SHERRY_OK;
 }
 
-// Which kernel computes each problem of a call.  Problems with one or two tokens
+// Which kernel computes each problem of a call.  Problems with one to four tokens
 // that fit the streaming lookup-table kernel share one launch of it (unless their
 // row blocks would outnumber its tickets); 2 <= M <= 8 problems with K % 128 == 0
 // share one launch of the warp-MMA kernel; other problems with up to 32 tokens
@@ -110,8 +141,26 @@ static int linear_launch(const ProbShape* shapes, const sherry_linear_desc* desc
         (st = skinny_linear_launch(r.skinny_s.data(), r.skinny_d.data(), (int)r.skinny_s.size(), M, y_bf16, sms,
                                    stream)))
         return st;
-    for (int i : r.prefill)
-        if ((st = prefill_launch(shapes[i], descs[i], M, y_bf16, stream))) return st;
+    if (r.prefill.size() == 1) {
+        if ((st = prefill_launch(shapes[r.prefill[0]], descs[r.prefill[0]], M, y_bf16, stream))) return st;
+    } else if (!r.prefill.empty()) {
+        std::lock_guard<std::mutex> lk(g_fork_mu);
+        ForkPool* fp = nullptr;
+        if ((st = fork_pool(&fp))) return st;
+        const int ns = std::min(kForkStreams, (int)r.prefill.size());
+        SHERRY_CUDA_CHECK(cudaEventRecord(fp->fork, stream));
+        for (int k = 0; k < ns; ++k) SHERRY_CUDA_CHECK(cudaStreamWaitEvent(fp->s[k], fp->fork, 0));
+        for (size_t j = 0; j < r.prefill.size() && st == SHERRY_OK; ++j) {
+            const int i = r.prefill[j];
+            st = prefill_launch(shapes[i], descs[i], M, y_bf16, fp->s[j % ns]);
+        }
+        // joined even after a failed launch, so the caller's stream stays ordered
+        for (int k = 0; k < ns; ++k) {
+            SHERRY_CUDA_CHECK(cudaEventRecord(fp->join[k], fp->s[k]));
+            SHERRY_CUDA_CHECK(cudaStreamWaitEvent(stream, fp->join[k], 0));
+        }
+        if (st) return st;
+    }
     if (!r.stream_s.empty() &&
         (st = stream_linear_launch(r.stream_s.data(), r.stream_d.data(), (int)r.stream_s.size(), M, y_bf16, workspace,
                                    sms, stream)))
