@@ -474,3 +474,33 @@ def test_linear_at_max_k(sw, orc, case):
     y = sw.linear(X, P, torch.float32)
     assert _abi.lib().sherry_device_status(None) == 0
     check_linear(y.cpu().numpy(), y_ref, Xb, orc.unpack_f32(*ref, N, K, gran, group))
+
+
+def test_batched_prefill_side_streams_and_graph_capture(sw, orc):
+    """A batched call with several prefill problems forks them over the library's
+    side streams and joins them into the caller's stream: results equal the single
+    calls bit for bit, eagerly and when the call is captured in a CUDA graph."""
+    import torch
+    shapes = [(384, 512, "group", 128), (130, 1024, "channel", 0), (256, 256, "group", 64),
+              (1000, 512, "tensor", 0), (64, 768, "group", 256)]
+    M = 300
+    pairs = []
+    for i, (N, K, gname, group) in enumerate(shapes):
+        W = _weights("t4", N, K, seed=52000 + i)
+        Xb = synth.activations_bf16(M, K, seed=52500 + i)
+        pairs.append((to_dev(Xb.view(np.int16)).view(torch.bfloat16), sw.quantize_pack(to_dev(W), GRAN[gname], group)))
+    singles = [sw.linear(X, P) for X, P in pairs]
+    outs = sw.linear_batched(pairs, torch.float32)
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(singles, outs))
+    outs_g = [torch.full_like(o, float("nan")) for o in outs]
+    sw.linear_batched(pairs, torch.float32, outs=outs_g)  # warm-up outside the capture
+    for o in outs_g:
+        o.fill_(float("nan"))
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        sw.linear_batched(pairs, torch.float32, outs=outs_g)
+    g.replay()
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(singles, outs_g))
