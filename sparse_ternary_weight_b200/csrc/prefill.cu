@@ -317,14 +317,17 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t t_row = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kPBN + half * kCols);
-                // 16 columns at a time keeps the 64 running sums in registers
+                // 32 columns per wait (two TMEM loads in flight); the running sums stay in registers
 #pragma unroll
-                for (int c = 0; c < kCols / 16; ++c) {
-                    uint32_t v[16];
-                    SHERRY_TMEM_LD16(t_row + 16 * c, v);
+                for (int c = 0; c < kCols / 32; ++c) {
+                    uint32_t v[16], w[16];
+                    SHERRY_TMEM_LD16(t_row + 32 * c, v);
+                    SHERRY_TMEM_LD16(t_row + 32 * c + 16, w);
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) acc[16 * c + j] = fmaf(a, __uint_as_float(v[j]), acc[16 * c + j]);
+                    for (int j = 0; j < 16; ++j) acc[32 * c + j] = fmaf(a, __uint_as_float(v[j]), acc[32 * c + j]);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) acc[32 * c + 16 + j] = fmaf(a, __uint_as_float(w[j]), acc[32 * c + 16 + j]);
                 }
                 tc_fence_before();
                 mbar_arrive(acc_empty(b));
