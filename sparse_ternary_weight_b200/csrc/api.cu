@@ -82,27 +82,31 @@ static int check_planes(const uint32_t* idx, const uint8_t* sgn, const float* sc
 }
 
 // Which kernel computes each problem of a call.  Problems with one to four tokens
-// that fit the streaming lookup-table kernel share one launch of it (unless their
-// row blocks would outnumber its tickets); 2 <= M <= 8 problems with K % 128 == 0
+// that fit the streaming lookup-table kernel share one launch of it, problems with
+// five to sixteen tokens of the same shapes one launch of its tensor-core form
+// (unless their row blocks would outnumber its tickets); 2 <= M <= 8 problems with K % 128 == 0
 // share one launch of the warp-MMA kernel; other problems with up to 32 tokens
 // that fit the tcgen05 few-token kernel share one launch of it; each problem with
 // M >= 17 that fits the prefill kernel gets a launch of its own; what remains
 // shares one launch of the general lookup-table kernel.
 struct Routes {
-    std::vector<ProbShape> stream_s, hmma_s, skinny_s, rest_s;
-    std::vector<sherry_linear_desc> stream_d, hmma_d, skinny_d, rest_d;
+    std::vector<ProbShape> stream_s, mstream_s, hmma_s, skinny_s, rest_s;
+    std::vector<sherry_linear_desc> stream_d, mstream_d, hmma_d, skinny_d, rest_d;
     std::vector<int> prefill;  // indices into the call's problems
 };
 
 static void route(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, Routes& r) {
     int64_t tiles = 0;
     for (int i = 0; i < count; ++i)
-        if (stream_eligible(shapes[i], M)) tiles += stream_tiles(shapes[i]);
+        if (stream_eligible(shapes[i], M) || mstream_eligible(shapes[i], M)) tiles += stream_tiles(shapes[i]);
     const bool stream_ok = tiles > 0 && tiles <= kMaxTickets;
     for (int i = 0; i < count; ++i) {
         if (stream_ok && stream_eligible(shapes[i], M)) {
             r.stream_s.push_back(shapes[i]);
             if (descs) r.stream_d.push_back(descs[i]);
+        } else if (stream_ok && mstream_eligible(shapes[i], M)) {
+            r.mstream_s.push_back(shapes[i]);
+            if (descs) r.mstream_d.push_back(descs[i]);
         } else if (hmma_eligible(shapes[i], M)) {
             r.hmma_s.push_back(shapes[i]);
             if (descs) r.hmma_d.push_back(descs[i]);
@@ -125,6 +129,8 @@ static size_t linear_ws_bytes(const ProbShape* shapes, int count, int64_t M, int
     route(shapes, nullptr, count, M, r);
     size_t ws = 0;
     if (!r.stream_s.empty()) ws = stream_workspace_bytes(r.stream_s.data(), (int)r.stream_s.size(), M, sms);
+    if (!r.mstream_s.empty())
+        ws = std::max(ws, stream_workspace_bytes(r.mstream_s.data(), (int)r.mstream_s.size(), M, sms));
     if (!r.rest_s.empty()) ws = std::max(ws, lut_workspace_bytes(r.rest_s.data(), (int)r.rest_s.size(), M, sms));
     return ws;
 }
@@ -164,6 +170,10 @@ static int linear_launch(const ProbShape* shapes, const sherry_linear_desc* desc
     if (!r.stream_s.empty() &&
         (st = stream_linear_launch(r.stream_s.data(), r.stream_d.data(), (int)r.stream_s.size(), M, y_bf16, workspace,
                                    sms, stream)))
+        return st;
+    if (!r.mstream_s.empty() &&
+        (st = mstream_linear_launch(r.mstream_s.data(), r.mstream_d.data(), (int)r.mstream_s.size(), M, y_bf16,
+                                    workspace, sms, stream)))
         return st;
     if (r.rest_s.empty()) return SHERRY_OK;
     return lut_linear_launch(r.rest_s.data(), r.rest_d.data(), (int)r.rest_s.size(), M, y_bf16, workspace, sms, stream);

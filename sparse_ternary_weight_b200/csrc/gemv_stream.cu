@@ -781,13 +781,330 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     }
 }
 
+// ---- tensor-core consumers for 5 to 16 tokens ------------------------------------
+//
+// The same streaming pipeline (units of 512 rows x 512 weights, stream-K ranges,
+// helper warps copying the packed planes into a cp.async ring, split tiles
+// finished through tickets), with a different consumer: instead of one table
+// lookup per block and token, each 4-weight block is expanded once to bf16
+// {-1, 0, +1} (two 4-byte lookups in a 32-entry pattern table) straight into the
+// A fragment of mma.sync m16n8k16 and multiplied with all tokens at once.  The
+// helpers stage the unit's activations (NT token rows of 512 bf16, zero rows for
+// tokens >= M) in the stage instead of tables.  K is permuted inside each 32-weight
+// word identically for both operands: in slice h of a word the lane with c =
+// lane % 4 holds the fragment positions k = 2c, 2c+1, 2c+8, 2c+9, taken to be the 4
+// weights of block 2c + h, so its two blocks per word are byte c of the packed
+// word and its activation fragments for both slices are the 8 consecutive
+// activations 8c .. 8c+7 of the word, one 16-byte load.  Each consumer warp owns
+// 32 rows (two m16 tiles); alpha is applied once per scale group (or at the end
+// for row scales) in fp32 registers.
+
+constexpr int kMXRow = 16 * 32 * 2 + 64;  // bytes per staged token row (padded: conflict-free 16-byte reads)
+constexpr int kMPat = 256;                // pattern table: 32 low words (weights 0, 1), then 32 high words
+
+template <int NT>
+struct MCfg {
+    using G = SGeo<16>;
+    static constexpr int kStages = 3;
+    static constexpr int kX = NT * kMXRow;  // staged activations per stage
+    static constexpr int kStage = G::kStage + kX;
+    static constexpr int kSmem = 256 + kMPat + kStages * kStage + kSBars;
+    static_assert(kSmem <= 232448, "shared memory per CTA");
+    static_assert(kStage % 16 == 0, "16-byte aligned stages");
+};
+
+__device__ __forceinline__ void m_mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                      uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Table offsets (4 * code, code = nibble + 16 G) of blocks 2c and 2c+1 of a packed
+// word w with sign byte s, for the lane's c (shifts precomputed: sh = 8c, ss = 2c).
+__device__ __forceinline__ void m_codes(uint32_t w, uint32_t s, uint32_t sh, uint32_t ss, uint32_t& oa,
+                                        uint32_t& ob) {
+    const uint32_t x = w >> sh, sb = s >> ss;
+    oa = ((x << 2) & 0x3cu) | ((sb << 6) & 0x40u);
+    ob = ((x >> 2) & 0x3cu) | ((sb << 5) & 0x40u);
+}
+
+template <int MAXP, int NT>
+__global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_constant__ SParams<MAXP> P, int M) {
+    using C = MCfg<NT>;
+    using G = SGeo<16>;
+    constexpr int S = C::kStages;
+    constexpr int NB = NT / 8;  // n8 token tiles
+    __shared__ int s_last;
+    __shared__ int s_abort;
+    const uint32_t base = (smem_u32(g_smem) + 255u) & ~255u;
+    const uint32_t pat = base;                     // [32] low words, [32] high words
+    const uint32_t stages = base + kMPat;          // stage s: planes, then NT staged token rows
+    const uint32_t bars = stages + S * C::kStage;
+    auto ready = [&](int s) { return bars + 8u * (uint32_t)s; };
+    auto empty = [&](int s) { return bars + 48u + 8u * (uint32_t)s; };
+    const uint32_t bar_part = bars + 96u;
+    const uint32_t bar_last = bars + 104u;
+
+    const int t = threadIdx.x;
+    const int lane = t & 31, warp = t >> 5;
+    if (t == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(ready(s), kSHelperThreads + kSHelperThreads);  // a cp.async and a staging arrival per helper
+            mbar_init(empty(s), kSRows);
+        }
+        mbar_init(bar_part, kSRows);
+        mbar_init(bar_last, 1);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (t < 32) {
+        const uint2 e = decode_block_bf16(t & 15u, t >> 4);
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(pat + 4u * t), "r"(e.x) : "memory");
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(pat + 128u + 4u * t), "r"(e.y) : "memory");
+    }
+    // token rows >= M read zeros: written once, never copied over
+    for (int i = t; i < S * (NT - M) * (kMXRow / 16); i += kSThreads) {
+        const int per = (NT - M) * (kMXRow / 16);
+        const int s = i / per, r = i % per;
+        const int m = M + r / (kMXRow / 16), ch = r % (kMXRow / 16);
+        sts128(stages + s * C::kStage + G::kStage + m * kMXRow + 16 * ch, make_uint4(0u, 0u, 0u, 0u));
+    }
+    __syncthreads();
+    volatile int* abort_flag = &s_abort;
+    int u_begin, u_end;
+    phase_range(P, 0, u_begin, u_end);
+    const int nu = max(0, u_end - u_begin);
+
+    if (warp >= kSConsumers) {
+        // ---- helpers: copies and activation staging of unit j into stage j % S
+        const int h = warp - kSConsumers;
+        const int ht = t - 32 * kSConsumers;
+        UnitPos cu = locate(P, u_begin);
+        CopyRows<16> cr;
+        int cr_p = -1, cr_rb = -1;
+        for (int j = 0; j < nu; ++j) {
+            const int s = j % S;
+            if (j >= S && !mbar_wait(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag, P.wait_cycles)) break;
+            const SProb& pr = P.p[cu.p];
+            if (cu.p != cr_p || cu.rb != cr_rb) {
+                copy_rows<16>(pr, cu.rb, h, lane, cr);
+                cr_p = cu.p;
+                cr_rb = cu.rb;
+            }
+            const uint32_t st = stages + s * C::kStage;
+            copy_unit<16>(pr, cr, cu.sub, st, h, lane);
+            cp_async_arrive(ready(s));
+            // the unit's 512 activations of each token (64 chunks of 16 bytes per token)
+            const uint4* xs = reinterpret_cast<const uint4*>(pr.X) + (int64_t)cu.sub * 64;
+            for (int i = ht; i < M * 64; i += kSHelperThreads) {
+                const int m = i >> 6, ch = i & 63;
+                sts128(st + G::kStage + m * kMXRow + 16 * ch, __ldg(xs + (int64_t)m * pr.words * 4 + ch));
+            }
+            mbar_arrive(ready(s));
+            advance(P.p, cu);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        return;
+    }
+
+    // ---- consumers: warp w owns unit rows 32w .. 32w+31 as two m16 tiles
+    const int g = lane >> 2, c = lane & 3;
+    const uint32_t sh = 8u * c, ss = 2u * c;
+    int rows[4];  // unit rows of the lane: tile 0 rows g, g+8; tile 1 rows g, g+8
+#pragma unroll
+    for (int i = 0; i < 4; ++i) rows[i] = 32 * warp + 16 * (i >> 1) + g + 8 * (i & 1);
+    float acc[2][NB][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[a][b][i] = 0.0f;
+    UnitPos cur = locate(P, u_begin);
+    bool tile_from_start = (P.p[cur.p].unit_begin + cur.rb * P.p[cur.p].n_sub == u_begin);
+    const int pb = P.ph_unit[0], upc = P.ph_upc[0];
+    int events = 0;
+    for (int k = 0; k < nu; ++k) {
+        const int s = k % S;
+        if (!mbar_wait(ready(s), (uint32_t)((k / S) & 1), abort_flag, P.wait_cycles)) break;
+        const SProb& pr = P.p[cur.p];
+        const uint32_t st = stages + s * C::kStage;
+        const uint32_t xs = st + G::kStage + (uint32_t)(g * kMXRow + 16 * c);
+        const int mode = pr.mode;
+        float cs[2][NB][4];  // group partial sums: row tile, token tile
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+            if (q == 0 || mode == kSG128 || (mode == kSG256 && q == 2)) {
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) cs[a][b][i] = 0.0f;
+            }
+            uint4 wv[4];
+            uint32_t sv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = rows[i];
+                wv[i] = lds128(st + r * G::kRowB + (((uint32_t)q ^ (uint32_t)((r / G::kSwz) % G::kLanesPerRow)) << 4));
+                sv[i] = lds32(st + G::kIdx + r * 16 + 4 * q);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint4 xb[NB];
+#pragma unroll
+                for (int b = 0; b < NB; ++b) xb[b] = lds128(xs + (uint32_t)(b * 8 * kMXRow + (4 * q + j) * 64));
+                uint32_t A[4][2][2];  // row, slice, (low, high)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w = j == 0 ? wv[i].x : j == 1 ? wv[i].y : j == 2 ? wv[i].z : wv[i].w;
+                    uint32_t oa, ob;
+                    m_codes(w, sv[i] >> (8 * j), sh, ss, oa, ob);
+                    A[i][0][0] = lds32(pat + oa);
+                    A[i][0][1] = lds32(pat + 128u + oa);
+                    A[i][1][0] = lds32(pat + ob);
+                    A[i][1][1] = lds32(pat + 128u + ob);
+                }
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                        for (int b = 0; b < NB; ++b) {
+                            const uint32_t b0 = hh ? xb[b].z : xb[b].x, b1 = hh ? xb[b].w : xb[b].y;
+                            m_mma(cs[a][b], A[2 * a][hh][0], A[2 * a + 1][hh][0], A[2 * a][hh][1], A[2 * a + 1][hh][1],
+                                  b0, b1);
+                        }
+            }
+            // end of a scale group (group 128: every 4 words; 256: every 8; row scales: the unit)
+            if (mode == kSG128 || (mode == kSG256 && (q & 1)) || (mode == kSRow && q == 3)) {
+                float al[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+                if (mode != kSRow) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t sc_a = st + G::kIdx + G::kSgn + rows[i] * 16;
+                        al[i] = __uint_as_float(lds32(mode == kSG128 ? sc_a + 4 * q : sc_a + 4 * (q >> 1)));
+                    }
+                }
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float v = cs[a][b][i];
+                            acc[a][b][i] = mode == kSRow ? acc[a][b][i] + v : fmaf(al[2 * a + (i >> 1)], v, acc[a][b][i]);
+                        }
+            }
+        }
+        mbar_arrive(empty(s));
+
+        const bool tile_end = (cur.sub == pr.n_sub - 1);
+        if (tile_end || k == nu - 1) {
+            // lane values: acc[a][b][i] = row rows[2a + (i >> 1)], token 8b + 2c + (i & 1)
+            float v[2][NB][4];
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int n = cur.rb * kSRows + rows[2 * a + (i >> 1)];
+                    const float rs = (pr.mode == kSRow && n < pr.N) ? __ldg(pr.scales + (pr.per_tensor ? 0 : n)) : 1.0f;
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) v[a][b][i] = pr.mode == kSRow ? acc[a][b][i] * rs : acc[a][b][i];
+                }
+            auto store = [&](int a, int b, int i, float val) {
+                const int n = cur.rb * kSRows + rows[2 * a + (i >> 1)];
+                const int m = 8 * b + 2 * c + (i & 1);
+                if (n < pr.N && m < M) {
+                    if (P.y_bf16)
+                        reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)m * pr.N + n] = __float2bfloat16_rn(val);
+                    else
+                        reinterpret_cast<float*>(pr.Y)[(int64_t)m * pr.N + n] = val;
+                }
+            };
+            if (tile_from_start && tile_end) {
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) store(a, b, i, v[a][b][i]);
+            } else {
+                // split tile: partials [cta][slot][token][row], then the ticket
+                const int tile = pr.tile_begin + cur.rb;
+                const int tile_u0 = pr.unit_begin + cur.rb * pr.n_sub;
+                const int c_a = (tile_u0 - pb) / upc;
+                const int c_b = (tile_u0 + pr.n_sub - 1 - pb) / upc;
+                const int slot = (u_begin >= tile_u0) ? 0 : 1;
+                auto part = [&](int cta, int sl, int a, int b, int i) {
+                    const int m = 8 * b + 2 * c + (i & 1);
+                    return P.part + (((int64_t)cta * 2 + sl) * M + m) * kSRows + rows[2 * a + (i >> 1)];
+                };
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            if (8 * b + 2 * c + (i & 1) < M) __stcg(part((int)blockIdx.x, slot, a, b, i), v[a][b][i]);
+                __threadfence();
+                mbar_arrive(bar_part);
+                const uint32_t ph2 = (uint32_t)(events & 1);
+                ++events;
+                const bool stored = mbar_wait(bar_part, ph2, abort_flag, P.wait_cycles);
+                if (stored && t == 0) {
+                    s_last = (atomicAdd(P.ticket + tile, 1) == c_b - c_a);
+                    mbar_arrive(bar_last);
+                }
+                __syncwarp();
+                if (!stored || !mbar_wait(bar_last, ph2, abort_flag, P.wait_cycles)) break;
+                if (s_last) {
+                    __threadfence();
+#pragma unroll
+                    for (int a = 0; a < 2; ++a)
+#pragma unroll
+                        for (int b = 0; b < NB; ++b)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                if (8 * b + 2 * c + (i & 1) >= M) continue;
+                                float sum = 0.0f;
+                                for (int cc = c_a; cc <= c_b; ++cc) {
+                                    const int sl = (pb + cc * upc >= tile_u0) ? 0 : 1;
+                                    const float pv = __ldcg(part(cc, sl, a, b, i));
+                                    sum = (cc == c_a) ? pv : sum + pv;
+                                }
+                                store(a, b, i, sum);
+                            }
+                    if (t == 0) P.ticket[tile] = 0;  // leave the ticket zeroed
+                }
+            }
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[a][b][i] = 0.0f;
+            tile_from_start = true;
+        }
+        advance(P.p, cur);
+    }
+}
+
 // ---- host side -------------------------------------------------------------------
 
 // Units of W words: K a multiple of 32 W; group scales of 128 or 256 weights
 // (whole groups per unit), or row scales.
 template <int W>
-static bool stream_eligible_w(const ProbShape& s, int64_t M) {
-    if (M < 1 || M > (W == 16 ? 3 : 4) || s.N == 0) return false;
+static bool stream_shape_ok(const ProbShape& s) {
+    if (s.N == 0) return false;
     if ((s.N + kSRows - 1) / kSRows > kMaxTickets - kChainCtrs) return false;
     if (s.K % (32 * W) != 0) return false;
     if (s.N * (s.K / 8) >= (int64_t(1) << 32) - 64) return false;  // 32-bit byte offsets into the planes
@@ -795,11 +1112,21 @@ static bool stream_eligible_w(const ProbShape& s, int64_t M) {
     if (s.granularity != SHERRY_PER_GROUP) return false;
     return s.group == 128 || s.group == 256;
 }
+template <int W>
+static bool stream_eligible_w(const ProbShape& s, int64_t M) {
+    return M >= 1 && M <= (W == 16 ? 3 : 4) && stream_shape_ok<W>(s);
+}
+
+// unit width of the streaming plans: 8 words for four tokens (lookup tables of four
+// tokens), 16 otherwise (lookups for up to three tokens, tensor cores from five)
+static int stream_w(int64_t M) { return M == 4 ? 8 : 16; }
 
 // one to three tokens: 16-word units; four: 8-word units
 bool stream_eligible(const ProbShape& s, int64_t M) {
     return M <= 3 ? stream_eligible_w<16>(s, M) : stream_eligible_w<8>(s, M);
 }
+// five to sixteen tokens: the tensor-core consumers on 16-word units
+bool mstream_eligible(const ProbShape& s, int64_t M) { return M >= 5 && M <= 16 && stream_shape_ok<16>(s); }
 bool chain_eligible(const ProbShape& s, int64_t M) {
     return M <= 3 ? stream_eligible_w<16>(s, M) : stream_eligible_w<8>(s, M);
 }
@@ -867,7 +1194,7 @@ static SPlan make_splan(const ProbShape* shapes, int count, const int* phase_beg
 }
 
 size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
-    return make_splan(shapes, count, nullptr, 1, M, sms, M <= 3 ? 16 : 8).ws_bytes;
+    return make_splan(shapes, count, nullptr, 1, M, sms, stream_w(M)).ws_bytes;
 }
 
 size_t chain_workspace_bytes(const ProbShape* shapes, int count, const int* phase_begin, int n_phases, int64_t M,
@@ -940,7 +1267,7 @@ static void attach(SPlan& pl, const sherry_linear_desc* descs, int count) {
 int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream) {
     if (M < 1 || M > 4) return SHERRY_ERR_UNSUPPORTED;
-    SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, M <= 3 ? 16 : 8);
+    SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, stream_w(M));
     attach(pl, descs, count);
     if (pl.total_units == 0) return SHERRY_OK;
     switch (M) {
@@ -949,6 +1276,53 @@ int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* desc
         case 3: return stream_launch_mt<3, 16>(pl, count, y_bf16, workspace, false, stream);
         default: return stream_launch_mt<4, 8>(pl, count, y_bf16, workspace, false, stream);
     }
+}
+
+template <int MAXP, int NT>
+static int mstream_launch_t(SPlan& pl, int64_t M, int y_bf16, void* workspace, cudaStream_t stream) {
+    static SParams<MAXP> P;
+    static std::mutex mu;
+    static PerDevice attr;
+    std::lock_guard<std::mutex> lk(mu);
+    P.wait_cycles = g_stream_wait.load();
+    P.count = (int)pl.probs.size();
+    P.y_bf16 = y_bf16;
+    P.n_phases = 1;
+    P.ticket = static_cast<int*>(workspace);
+    P.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.part_off);
+    P.phase_cnt = nullptr;
+    for (int i = 0; i < P.count; ++i) P.p[i] = pl.probs[i];
+    P.ph_unit[0] = pl.ph_unit[0];
+    P.ph_unit[1] = pl.ph_unit[1];
+    P.ph_upc[0] = pl.ph_upc[0];
+    int done = 0;
+    const int st = per_device(attr, &done, [](int& v) {
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_mma_stream<MAXP, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               MCfg<NT>::kSmem));
+        v = 1;
+        return SHERRY_OK;
+    });
+    if (st) return st;
+    k_mma_stream<MAXP, NT><<<pl.grid, kSThreads, MCfg<NT>::kSmem, stream>>>(P, (int)M);
+    SHERRY_LAUNCH_CHECK();
+    return SHERRY_OK;
+}
+
+template <int NT>
+static int mstream_launch_nt(SPlan& pl, int count, int64_t M, int y_bf16, void* workspace, cudaStream_t stream) {
+    if (count <= 1) return mstream_launch_t<1, NT>(pl, M, y_bf16, workspace, stream);
+    if (count <= 16) return mstream_launch_t<16, NT>(pl, M, y_bf16, workspace, stream);
+    return mstream_launch_t<SHERRY_MAX_BATCH, NT>(pl, M, y_bf16, workspace, stream);
+}
+
+int mstream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
+                          void* workspace, int sms, cudaStream_t stream) {
+    if (M < 5 || M > 16) return SHERRY_ERR_UNSUPPORTED;
+    SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, 16);
+    attach(pl, descs, count);
+    if (pl.total_units == 0) return SHERRY_OK;
+    return M <= 8 ? mstream_launch_nt<8>(pl, count, M, y_bf16, workspace, stream)
+                  : mstream_launch_nt<16>(pl, count, M, y_bf16, workspace, stream);
 }
 
 bool chain_launch_ok(const ProbShape* shapes, int count, int n_phases, int64_t M) {

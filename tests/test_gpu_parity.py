@@ -235,11 +235,11 @@ STREAM_SHAPES = [(1024, 3072, "group", 128), (300, 3072, "channel", 0), (3072, 8
                  (1, 512, "group", 128), (257, 3072, "group", 256), (96, 1536, "group", 256)]
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 12, 16])
 def test_stream_batch_many_problems_vs_oracle(sw, orc, M):
-    """Batches of one to four tokens over many eligible linears (the streaming
-    kernel: units split evenly over CTAs, tiles straddling CTAs finished through
-    the ticket)."""
+    """Batches of 1 to 16 tokens over many eligible linears (the streaming kernel,
+    lookup tables up to four tokens, tensor-core consumers from five: units split
+    evenly over CTAs, tiles straddling CTAs finished through the ticket)."""
     import torch
     pairs, refs = [], []
     for i in range(24):
@@ -379,7 +379,8 @@ def test_batched_mixed_routes_vs_oracle(sw, orc, M):
     for y, (y_ref, Wq, Xb) in zip(outs, refs):
         check_linear(y.cpu().numpy(), y_ref, Xb, Wq)
     for (X, P), y, (N, K, gname, group) in zip(pairs, outs, MIXED_SHAPES):
-        tc = (SKINNY_MIN_M <= M <= 32 and K % 256 == 0 and (gname != "group" or group % 64 == 0)) or \
+        mstream = 5 <= M <= 16 and K % 512 == 0 and (gname != "group" or group in (128, 256))
+        tc = (not mstream and SKINNY_MIN_M <= M <= 32 and K % 256 == 0 and (gname != "group" or group % 64 == 0)) or \
              (M >= 17 and K % 64 == 0 and (gname != "group" or group % 64 == 0))
         if tc:
             assert torch.equal(sw.linear(X, P), y)
@@ -449,8 +450,10 @@ MAXK_CASES = [
     (3, 5, "channel", 0),   # three-token streaming kernel
     (4, 5, "group", 256),   # four-token streaming kernel (8-word units)
     (1, 3, "group", 32),    # general lookup-table kernel
-    (5, 5, "group", 128),   # warp-MMA kernel
-    (16, 3, "channel", 0),  # tcgen05 few-token kernel
+    (5, 5, "group", 128),   # streaming kernel, tensor-core consumers (8 token columns)
+    (16, 5, "channel", 0),  # streaming kernel, tensor-core consumers (16 token columns)
+    (6, 5, "group", 32),    # warp-MMA kernel
+    (16, 3, "group", 64),   # tcgen05 few-token kernel (group 64: not a streaming shape)
     (64, 3, "group", 256),  # tcgen05 prefill kernel
 ]
 
