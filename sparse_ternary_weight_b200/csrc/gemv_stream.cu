@@ -1117,16 +1117,12 @@ static bool stream_eligible_w(const ProbShape& s, int64_t M) {
     return M >= 1 && M <= (W == 16 ? 3 : 4) && stream_shape_ok<W>(s);
 }
 
-// unit width of the streaming plans: 8 words for four tokens (lookup tables of four
-// tokens), 16 otherwise (lookups for up to three tokens, tensor cores from five)
-static int stream_w(int64_t M) { return M == 4 ? 8 : 16; }
-
-// one to three tokens: 16-word units; four: 8-word units
-bool stream_eligible(const ProbShape& s, int64_t M) {
-    return M <= 3 ? stream_eligible_w<16>(s, M) : stream_eligible_w<8>(s, M);
-}
-// five to sixteen tokens: the tensor-core consumers on 16-word units
-bool mstream_eligible(const ProbShape& s, int64_t M) { return M >= 5 && M <= 16 && stream_shape_ok<16>(s); }
+// one to three tokens: lookup tables on 16-word units (the four-token lookup form,
+// on 8-word units, serves the chained launches; independent linears of four or
+// more tokens go to the tensor-core consumers)
+bool stream_eligible(const ProbShape& s, int64_t M) { return M <= 3 && stream_eligible_w<16>(s, M); }
+// four to sixteen tokens: the tensor-core consumers on 16-word units
+bool mstream_eligible(const ProbShape& s, int64_t M) { return M >= 4 && M <= 16 && stream_shape_ok<16>(s); }
 bool chain_eligible(const ProbShape& s, int64_t M) {
     return M <= 3 ? stream_eligible_w<16>(s, M) : stream_eligible_w<8>(s, M);
 }
@@ -1194,7 +1190,7 @@ static SPlan make_splan(const ProbShape* shapes, int count, const int* phase_beg
 }
 
 size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int sms) {
-    return make_splan(shapes, count, nullptr, 1, M, sms, stream_w(M)).ws_bytes;
+    return make_splan(shapes, count, nullptr, 1, M, sms, 16).ws_bytes;
 }
 
 size_t chain_workspace_bytes(const ProbShape* shapes, int count, const int* phase_begin, int n_phases, int64_t M,
@@ -1266,15 +1262,14 @@ static void attach(SPlan& pl, const sherry_linear_desc* descs, int count) {
 
 int stream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                          void* workspace, int sms, cudaStream_t stream) {
-    if (M < 1 || M > 4) return SHERRY_ERR_UNSUPPORTED;
-    SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, stream_w(M));
+    if (M < 1 || M > 3) return SHERRY_ERR_UNSUPPORTED;
+    SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, 16);
     attach(pl, descs, count);
     if (pl.total_units == 0) return SHERRY_OK;
     switch (M) {
         case 1: return stream_launch_mt<1, 16>(pl, count, y_bf16, workspace, false, stream);
         case 2: return stream_launch_mt<2, 16>(pl, count, y_bf16, workspace, false, stream);
-        case 3: return stream_launch_mt<3, 16>(pl, count, y_bf16, workspace, false, stream);
-        default: return stream_launch_mt<4, 8>(pl, count, y_bf16, workspace, false, stream);
+        default: return stream_launch_mt<3, 16>(pl, count, y_bf16, workspace, false, stream);
     }
 }
 
@@ -1317,7 +1312,7 @@ static int mstream_launch_nt(SPlan& pl, int count, int64_t M, int y_bf16, void* 
 
 int mstream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                           void* workspace, int sms, cudaStream_t stream) {
-    if (M < 5 || M > 16) return SHERRY_ERR_UNSUPPORTED;
+    if (M < 4 || M > 16) return SHERRY_ERR_UNSUPPORTED;
     SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, 16);
     attach(pl, descs, count);
     if (pl.total_units == 0) return SHERRY_OK;

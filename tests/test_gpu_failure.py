@@ -87,7 +87,7 @@ LIN_CANARY = [
     (1, 1000, 3072, "group", 128),   # one-token streaming
     (2, 513, 1024, "channel", 0),    # two-token streaming
     (3, 700, 2048, "group", 256),    # three-token streaming
-    (4, 1000, 3072, "group", 128),   # four-token streaming (8-word units)
+    (4, 1000, 3072, "group", 128),   # streaming, tensor-core consumers
     (1, 77, 96, "group", 32),        # general lookup-table
     (5, 300, 1024, "tensor", 0),     # warp MMA
     (13, 129, 3072, "group", 128),   # tcgen05 few-token

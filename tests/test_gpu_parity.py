@@ -134,7 +134,7 @@ LIN_CASES = [
     (2, 513, 1024, "channel", 0),
     (2, 77, 1536, "group", 256),
     (2, 1000, 8192, "tensor", 0),
-    (3, 64, 3072, "channel", 0),    # three and four tokens: streaming kernel (four: 8-word units)
+    (3, 64, 3072, "channel", 0),    # three tokens: streaming lookup kernel; four: its tensor-core consumers
     (3, 1000, 2048, "group", 256),
     (4, 500, 1024, "group", 128),
     (4, 77, 768, "tensor", 0),
@@ -238,7 +238,7 @@ STREAM_SHAPES = [(1024, 3072, "group", 128), (300, 3072, "channel", 0), (3072, 8
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 12, 16])
 def test_stream_batch_many_problems_vs_oracle(sw, orc, M):
     """Batches of 1 to 16 tokens over many eligible linears (the streaming kernel,
-    lookup tables up to four tokens, tensor-core consumers from five: units split
+    lookup tables up to three tokens, tensor-core consumers from four: units split
     evenly over CTAs, tiles straddling CTAs finished through the ticket)."""
     import torch
     pairs, refs = [], []
@@ -448,7 +448,7 @@ MAXK_CASES = [
     (1, 5, "group", 128),   # one-token streaming kernel
     (2, 5, "group", 128),   # two-token streaming kernel
     (3, 5, "channel", 0),   # three-token streaming kernel
-    (4, 5, "group", 256),   # four-token streaming kernel (8-word units)
+    (4, 5, "group", 256),   # streaming kernel, tensor-core consumers
     (1, 3, "group", 32),    # general lookup-table kernel
     (5, 5, "group", 128),   # streaming kernel, tensor-core consumers (8 token columns)
     (16, 5, "channel", 0),  # streaming kernel, tensor-core consumers (16 token columns)
