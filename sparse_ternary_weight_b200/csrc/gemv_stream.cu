@@ -939,7 +939,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
         const uint32_t xs = st + G::kStage + (uint32_t)(g * kMXRow + 16 * c);
         const int mode = pr.mode;
         float cs[2][NB][4];  // group partial sums: row tile, token tile
-#pragma unroll 1
+#pragma unroll
         for (int q = 0; q < 4; ++q) {
             if (q == 0 || mode == kSG128 || (mode == kSG256 && q == 2)) {
 #pragma unroll
@@ -962,27 +962,28 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
                 uint4 xb[NB];
 #pragma unroll
                 for (int b = 0; b < NB; ++b) xb[b] = lds128(xs + (uint32_t)(b * 8 * kMXRow + (4 * q + j) * 64));
-                uint32_t A[4][2][2];  // row, slice, (low, high)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w = j == 0 ? wv[i].x : j == 1 ? wv[i].y : j == 2 ? wv[i].z : wv[i].w;
-                    uint32_t oa, ob;
-                    m_codes(w, sv[i] >> (8 * j), sh, ss, oa, ob);
-                    A[i][0][0] = lds32(pat + oa);
-                    A[i][0][1] = lds32(pat + 128u + oa);
-                    A[i][1][0] = lds32(pat + ob);
-                    A[i][1][1] = lds32(pat + 128u + ob);
-                }
+                for (int a = 0; a < 2; ++a) {
+                    uint32_t A[2][2][2];  // row of the tile, slice, (low, high)
 #pragma unroll
-                for (int a = 0; a < 2; ++a)
+                    for (int ii = 0; ii < 2; ++ii) {
+                        const int i = 2 * a + ii;
+                        const uint32_t w = j == 0 ? wv[i].x : j == 1 ? wv[i].y : j == 2 ? wv[i].z : wv[i].w;
+                        uint32_t oa, ob;
+                        m_codes(w, sv[i] >> (8 * j), sh, ss, oa, ob);
+                        A[ii][0][0] = lds32(pat + oa);
+                        A[ii][0][1] = lds32(pat + 128u + oa);
+                        A[ii][1][0] = lds32(pat + ob);
+                        A[ii][1][1] = lds32(pat + 128u + ob);
+                    }
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
                         for (int b = 0; b < NB; ++b) {
                             const uint32_t b0 = hh ? xb[b].z : xb[b].x, b1 = hh ? xb[b].w : xb[b].y;
-                            m_mma(cs[a][b], A[2 * a][hh][0], A[2 * a + 1][hh][0], A[2 * a][hh][1], A[2 * a + 1][hh][1],
-                                  b0, b1);
+                            m_mma(cs[a][b], A[0][hh][0], A[1][hh][0], A[0][hh][1], A[1][hh][1], b0, b1);
                         }
+                }
             }
             // end of a scale group (group 128: every 4 words; 256: every 8; row scales: the unit)
             if (mode == kSG128 || (mode == kSG256 && (q & 1)) || (mode == kSRow && q == 3)) {
