@@ -295,7 +295,7 @@ size_t sherry_linear_chain_workspace_bytes(const sherry_linear_desc* descs, int 
  * what the previous call left; all calls share the one array, so calls that
  * overlap on the GPU (other streams, other host threads) race -- keep them
  * ordered.  Nothing is allocated or freed. */
-#define SHERRY_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)  /* one problem's largest plan on up to 224 SMs
+#define SHERRY_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)  /* one problem's largest plan on up to 224 SMs
                                                            (checked at compile time for each plan) */
 int sherry_linear_noalloc(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                           const uint32_t* idx, const uint8_t* sgn, const float* scales,

@@ -16,7 +16,7 @@ F32, BF16 = 0, 1
 OP_QUANTIZE_PACK, OP_LINEAR, OP_UNPACK = 0, 1, 2
 MAX_K = 262144
 MAX_BATCH = 256
-NOALLOC_SCRATCH_BYTES = 4 << 20
+NOALLOC_SCRATCH_BYTES = 16 << 20
 TEQUILA_ONES, TEQUILA_SIGN = 0, 1
 
 vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t

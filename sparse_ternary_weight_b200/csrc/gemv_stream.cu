@@ -802,6 +802,11 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
 constexpr int kMXRow = 16 * 32 * 2 + 64;  // bytes per staged token row (padded: conflict-free 16-byte reads)
 constexpr int kMPat = 256;                // pattern table: 32 low words (weights 0, 1), then 32 high words
 
+// The no-workspace entry point's fixed scratch holds the largest tensor-core plan
+// (sixteen tokens, one CTA per SM, two partial slots per CTA) on up to 224 SMs.
+static_assert(kTicketBytes + (size_t)224 * 2 * 16 * kSRows * sizeof(float) <= SHERRY_NOALLOC_SCRATCH_BYTES,
+              "no-workspace scratch too small for the tensor-core streaming plan");
+
 template <int NT>
 struct MCfg {
     using G = SGeo<16>;

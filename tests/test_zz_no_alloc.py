@@ -14,9 +14,11 @@ pytestmark = pytest.mark.gpu
 
 CASES = [
     # (M, N, K, granularity, group): the streaming kernel (one and two tokens)
-    # with tiles split over CTAs, the same over a wide linear, the general kernel
+    # with tiles split over CTAs, the same over a wide linear, its tensor-core form
+    # at 16 tokens on a full grid (the largest scratch plan), the general kernel
     # with split K, and the tensor-core kernel (which needs no scratch)
     (1, 64, 8192, _abi.PER_GROUP, 128),
+    (16, 4096, 8192, _abi.PER_GROUP, 128),
     (1, 3072, 3072, _abi.PER_GROUP, 128),
     (2, 3072, 3072, _abi.PER_GROUP, 128),
     (3, 300, 3072, _abi.PER_CHANNEL, 0),
