@@ -110,10 +110,6 @@ struct SProb {
     int mode, per_tensor;
     int n_rb, n_sub;    // row blocks, sub-slices (units) per row block
     int unit_begin, tile_begin;
-    // chained launches: the earlier problem whose bf16 Y holds this X (-1: none), and
-    // X's element offset in that Y
-    int dep;
-    long long dep_off;
 };
 
 template <int MAXP>
@@ -123,11 +119,8 @@ struct SParams {
     float* part;            // [grid][2][MT][kSRows] split-tile partials
     int* ticket;            // [total tiles]
     int* phase_cnt;         // chained launches: [n_phases] arrivals + exit counter; else null
-    int* flags;             // chained launches with dataflow: [total tiles] Y-complete flags; else null
-    int total_tiles;
     int ph_unit[MAXP + 1];  // first unit of each phase; ph_unit[n_phases] = all units
     int ph_upc[MAXP];       // units per CTA of each phase
-    int ph_mode[MAXP];      // chained: bit 0 = grid barrier before the phase, bit 1 = arrivals after it
     SProb p[MAXP];
 };
 
@@ -195,9 +188,6 @@ __device__ __forceinline__ bool gate_wait(const int* gate, int target, volatile 
         }
     }
 }
-__device__ __forceinline__ void st_release(int* p, int v) {
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 // arrival at a phase counter: a release at GPU scope (the Y this CTA wrote, seen by
 // this thread through the CTA's mbarrier, is visible before the count), no reply
 __device__ __forceinline__ void red_release_add(int* p, int v) {
@@ -224,52 +214,6 @@ __device__ __forceinline__ int grid_poll(const int* cnt, int target, volatile in
             if (*abort_flag) {
                 quit = 1;
             } else if (clock64() - t0 > budget) {
-                *abort_flag = 1;
-                atomicExch(&g_stream_status, SHERRY_ERR_TIMEOUT);
-                quit = 1;
-            }
-        }
-        if (__shfl_sync(kFull, quit, 0)) return -1;
-    }
-}
-// Completion flags of the producer tiles of one unit of a chained launch: the unit
-// reads activations [k0, k0 + span) of each of its MT token rows from problem
-// pi's X, which is a bf16 view into the Y of problem dep at element offset
-// dep_off; lane m < MT checks the tiles (512 rows each) that hold its token row's
-// range, which may wrap into the next row of Y.  One warp, converged: 1 = every
-// flag set, 0 = not yet (when block is false), -1 = timeout or abort.
-template <int MAXP>
-__device__ __forceinline__ int flags_poll(const SParams<MAXP>& P, int pi, int k0, int MT, volatile int* abort_flag,
-                                          long long budget, bool block, int lane, int span) {
-    const SProb& pr = P.p[pi];
-    const SProb& pj = P.p[pr.dep];
-    int t0 = 0, t1 = -1, t2 = 0, t3 = -1;  // tile ranges [t0, t1] and [t2, t3] of this lane
-    if (lane < MT) {
-        const long long e0 = pr.dep_off + (long long)lane * pr.words * 32 + k0;
-        const int n0 = (int)(e0 % pj.N), n1 = (int)((e0 + span - 1) % pj.N);
-        if (n0 <= n1) {
-            t0 = n0 / kSRows;
-            t1 = n1 / kSRows;
-        } else {
-            t0 = n0 / kSRows;
-            t1 = (pj.N - 1) / kSRows;
-            t2 = 0;
-            t3 = n1 / kSRows;
-        }
-    }
-    const int* fl = P.flags + pj.tile_begin;
-    const long long c0 = clock64();
-    while (true) {
-        bool done = true;
-        for (int t = t0; t <= t1; ++t) done = done && ld_acquire(fl + t) != 0;
-        for (int t = t2; t <= t3; ++t) done = done && ld_acquire(fl + t) != 0;
-        if (__all_sync(kFull, done)) return 1;
-        if (!block) return 0;
-        int quit = 0;
-        if (lane == 0) {
-            if (*abort_flag) {
-                quit = 1;
-            } else if (clock64() - c0 > budget) {
                 *abort_flag = 1;
                 atomicExch(&g_stream_status, SHERRY_ERR_TIMEOUT);
                 quit = 1;
@@ -541,9 +485,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     constexpr int S = C::kStages;
     __shared__ int s_last;
     __shared__ int s_abort;
-    __shared__ int s_gate;  // phases known complete on every CTA (written by helper warp 0)
-    __shared__ int s_ok;    // units of this CTA whose producer tiles are known complete (helper warp 0)
-    __shared__ int s_exit;  // this CTA is the last to leave a chained launch
+    __shared__ int s_gate;  // phases known complete on every CTA (written by helper thread 0)
     // Shared addresses: the buffer is rounded up to 256 bytes, so every table
     // base is a multiple of 256 (a lookup's address replaces its low byte); the
     // XOR swizzles need only 16-byte alignment, since writer and reader apply them.
@@ -556,7 +498,6 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     const uint32_t bar_part = bars + 96u;    // every consumer stored its split-tile partial
     const uint32_t bar_last = bars + 104u;   // the ticket's outcome is in s_last
     const uint32_t bar_phase = bars + 112u;  // every consumer finished the CTA's units of a phase
-    const uint32_t bar_tile = bars + 120u;   // every consumer stored its rows of a finished tile
 
     const int t = threadIdx.x;
     const int lane = t & 31, warp = t >> 5;
@@ -569,10 +510,8 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         mbar_init(bar_part, kSRows);
         mbar_init(bar_last, 1);
         mbar_init(bar_phase, kSRows);
-        mbar_init(bar_tile, kSRows);
         s_abort = 0;
         s_gate = 0;
-        s_ok = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -619,30 +558,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                 ++jt;
                 return true;
             }
-            if (chain && P.flags && P.p[tc.pos.p].dep >= 0) {
-                // the unit reads tiles of an earlier problem's Y: helper warp 0 (as a whole
-                // warp) checks their completion flags and publishes the unit in a shared
-                // counter that the other helper warps read (monotonic, like s_gate)
-                if (h == 0) {
-                    const int st = flags_poll(P, tc.pos.p, tc.pos.sub * G::kTabs * 4, MT, abort_flag, P.wait_cycles,
-                                              block, lane, G::kTabs * 4);
-                    if (st != 1) {
-                        fail = st < 0;
-                        return false;
-                    }
-                    __threadfence();
-                    if (lane == 0) *reinterpret_cast<volatile int*>(&s_ok) = jt + 1;
-                } else if (block) {
-                    if (!gate_wait(&s_ok, jt + 1, abort_flag, P.wait_cycles)) {
-                        fail = true;
-                        return false;
-                    }
-                } else if (*reinterpret_cast<volatile int*>(&s_ok) < jt + 1) {
-                    return false;
-                }
-                __threadfence();
-                have_x = false;
-            } else if (chain && (P.ph_mode[tc.ph] & 1) && tc.ph > passed) {
+            if (chain && tc.ph > passed) {
                 // helper warp 0 (as a whole warp) reads the arrivals of every CTA and
                 // publishes the phase in a shared counter that the other helper warps read
                 // (a monotonic count, so a warp that looks late still sees it)
@@ -676,8 +592,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
             ++jt;
             // the next unit's activations are fetched now unless it opens a phase that is
             // still being written
-            have_x = jt < nu && (!chain || (((P.ph_mode[tc.ph] & 1) == 0 || tc.ph <= passed) &&
-                                             !(P.flags && P.p[tc.pos.p].dep >= 0)));
+            have_x = jt < nu && (!chain || tc.ph <= passed);
             if (have_x) load_x(P.p[tc.pos.p], tc.pos.sub);
             return true;
         };
@@ -711,22 +626,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
         int k = 0;       // units consumed so far (all phases): stage k % S
         int events = 0;  // split tiles handled so far (phase of bar_part / bar_last)
         int phases = 0;  // phases this CTA's consumers completed with units (phase of bar_phase)
-        int tdone = 0;   // tiles this CTA finished with flags (phase of bar_tile)
         bool ok = true;
-        // a tile whose Y this CTA finished: once every consumer's rows are stored, warp
-        // 0 (as a whole warp) waits for them and lane 0 sets the tile's flag (release)
-        auto tile_done = [&](int tile) -> bool {
-            __threadfence();
-            mbar_arrive(bar_tile);
-            bool done = true;
-            if (warp == 0) {
-                done = mbar_wait(bar_tile, (uint32_t)(tdone & 1), abort_flag, P.wait_cycles);
-                if (done && lane == 0) st_release(P.flags + tile, 1);
-                __syncwarp();
-            }
-            ++tdone;
-            return done;
-        };
         for (int ph = 0; ph < P.n_phases && ok; ++ph) {
             int u_begin, u_end;
             phase_range(P, ph, u_begin, u_end);
@@ -775,10 +675,6 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                                     else
                                         reinterpret_cast<float*>(pr.Y)[(int64_t)m * pr.N + n] = v[m];
                                 }
-                            }
-                            if (P.flags && !tile_done(pr.tile_begin + cur.rb)) {
-                                ok = false;
-                                break;
                             }
                         } else {
                             // split tile: partials into this CTA's slot, then the ticket
@@ -843,10 +739,6 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                                     }
                                 }
                                 if (r == 0) P.ticket[tile] = 0;  // leave the ticket zeroed
-                                if (P.flags && !tile_done(tile)) {
-                                    ok = false;
-                                    break;
-                                }
                             }
                         }
 #pragma unroll
@@ -856,10 +748,9 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                     advance(P.p, cur);
                 }
                 if (!ok) break;
-                if (chain && (P.ph_mode[ph] & 2)) {
-                    // (only before a phase that starts at a grid barrier) every consumer's Y
-                    // of this phase is written before the CTA's arrival; warp 0 waits for all
-                    // of them (as a whole warp) and lane 0 arrives
+                if (chain) {
+                    // every consumer's Y of this phase is written before the CTA's arrival;
+                    // warp 0 waits for all of them (as a whole warp) and lane 0 arrives
                     __threadfence();
                     mbar_arrive(bar_phase);
                     if (warp == 0) {
@@ -873,28 +764,19 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
                     }
                     ++phases;
                 }
-            } else if (chain && (P.ph_mode[ph] & 2) && r == 0) {
+            } else if (chain && r == 0) {
                 red_release_add(P.phase_cnt + ph, 1);  // nothing of this phase here
             }
         }
     }
 
     __syncthreads();
-    if (chain) {
-        // the last CTA to leave zeroes the phase counters and the tile flags for the next launch
-        if (t == 0) {
-            s_exit = 0;
-            if (!*abort_flag) {
-                __threadfence();
-                s_exit = atomicAdd(P.phase_cnt + P.n_phases, 1) == (int)gridDim.x - 1;
-            }
-        }
-        __syncthreads();
-        if (s_exit) {
+    if (chain && t == 0 && !*abort_flag) {
+        // the last CTA to leave zeroes the phase counters for the next launch
+        __threadfence();
+        if (atomicAdd(P.phase_cnt + P.n_phases, 1) == (int)gridDim.x - 1) {
+            for (int ph = 0; ph <= P.n_phases; ++ph) P.phase_cnt[ph] = 0;
             __threadfence();
-            for (int i = t; i <= P.n_phases; i += kSThreads) P.phase_cnt[i] = 0;
-            if (P.flags)
-                for (int i = t; i < P.total_tiles; i += kSThreads) P.flags[i] = 0;
         }
     }
 }
@@ -1262,8 +1144,7 @@ long long stream_set_wait_cycles(long long cycles) {
 
 struct SPlan {
     std::vector<SProb> probs;
-    std::vector<int> ph_unit, ph_upc, ph_mode;
-    bool dataflow = false;  // chained: tile flags replace the grid barriers
+    std::vector<int> ph_unit, ph_upc;
     int total_units = 0, total_tiles = 0, grid = 0;
     size_t ws_bytes = 0, part_off = 0;
 };
@@ -1287,8 +1168,6 @@ static SPlan make_splan(const ProbShape* shapes, int count, const int* phase_beg
         p.n_sub = (p.words + W - 1) / W;
         p.unit_begin = ub;
         p.tile_begin = tb;
-        p.dep = -1;
-        p.dep_off = 0;
         ub += p.n_rb * p.n_sub;
         tb += p.n_rb;
         pl.probs.push_back(p);
@@ -1338,14 +1217,9 @@ static int stream_launch_t(SPlan& pl, int y_bf16, void* workspace, bool chain, c
     P.ticket = static_cast<int*>(workspace);
     P.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.part_off);
     P.phase_cnt = chain ? static_cast<int*>(workspace) + (kMaxTickets - kChainCtrs) : nullptr;
-    P.total_tiles = pl.total_tiles;
-    P.flags = (chain && pl.dataflow) ? static_cast<int*>(workspace) + pl.total_tiles : nullptr;
     for (int i = 0; i < P.count; ++i) P.p[i] = pl.probs[i];
     for (int i = 0; i <= P.n_phases; ++i) P.ph_unit[i] = pl.ph_unit[i];
-    for (int i = 0; i < P.n_phases; ++i) {
-        P.ph_upc[i] = pl.ph_upc[i];
-        P.ph_mode[i] = chain ? pl.ph_mode[i] : 0;
-    }
+    for (int i = 0; i < P.n_phases; ++i) P.ph_upc[i] = pl.ph_upc[i];
     int done = 0;
     const int st = per_device(attr, &done, [](int& v) {
         SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_lut_stream<MAXP, MT, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1418,9 +1292,6 @@ static int mstream_launch_t(SPlan& pl, int64_t M, int y_bf16, void* workspace, c
     P.ticket = static_cast<int*>(workspace);
     P.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.part_off);
     P.phase_cnt = nullptr;
-    P.flags = nullptr;
-    P.total_tiles = pl.total_tiles;
-    P.ph_mode[0] = 0;
     for (int i = 0; i < P.count; ++i) P.p[i] = pl.probs[i];
     P.ph_unit[0] = pl.ph_unit[0];
     P.ph_unit[1] = pl.ph_unit[1];
@@ -1455,63 +1326,6 @@ int mstream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* des
                   : mstream_launch_nt<16>(pl, count, M, y_bf16, workspace, stream);
 }
 
-// Producers of a chained launch.  A problem's X that lies inside one earlier
-// problem's bf16 Y (at an element offset) is read as that problem's output: its
-// units wait only for the Y tiles that hold their K slice (flags set when a tile's
-// Y is complete).  A phase starts at a grid barrier instead (after every CTA has
-// arrived at the previous phase, hence finished every earlier phase) when one of
-// its X overlaps an earlier Y any other way, when its Y overlaps an earlier X or
-// Y (an earlier phase may still read or write it), or for a chain with fp32 Y or
-// too many tiles for the flag region.
-static void plan_dataflow(SPlan& pl, const sherry_linear_desc* descs, int count, const int* phase_begin,
-                          int n_phases, int64_t M, int y_bf16) {
-    (void)count;
-    pl.ph_mode.assign(n_phases, 0);
-    pl.dataflow = y_bf16 && 2 * (int64_t)pl.total_tiles <= kMaxTickets - kChainCtrs;
-    const int ysz = y_bf16 ? 2 : 4;
-    auto xr = [&](int i, uintptr_t& a, uintptr_t& b) {
-        a = reinterpret_cast<uintptr_t>(descs[i].X);
-        b = a + (uintptr_t)(M * descs[i].K) * 2;
-    };
-    auto yr = [&](int i, uintptr_t& a, uintptr_t& b) {
-        a = reinterpret_cast<uintptr_t>(descs[i].Y);
-        b = a + (uintptr_t)(M * descs[i].N) * ysz;
-    };
-    auto overlap = [](uintptr_t a0, uintptr_t a1, uintptr_t b0, uintptr_t b1) { return a0 < b1 && b0 < a1; };
-    for (int ph = 1; ph < n_phases; ++ph) {
-        bool barrier = !pl.dataflow;
-        for (int i = phase_begin[ph]; i < phase_begin[ph + 1] && !barrier; ++i) {
-            uintptr_t xa, xb, wa, wb;
-            xr(i, xa, xb);
-            yr(i, wa, wb);
-            int dep = -1;
-            for (int j = 0; j < phase_begin[ph] && !barrier; ++j) {
-                uintptr_t ya, yb, ra, rb;
-                yr(j, ya, yb);
-                xr(j, ra, rb);
-                if (overlap(wa, wb, ra, rb) || overlap(wa, wb, ya, yb)) {
-                    barrier = true;  // this Y is an earlier X or Y
-                    break;
-                }
-                if (!overlap(xa, xb, ya, yb)) continue;
-                if (dep < 0 && xa >= ya && xb <= yb && (xa - ya) % 2 == 0)
-                    dep = j;
-                else
-                    barrier = true;  // partial, misaligned or a second overlap
-            }
-            if (!barrier) {
-                pl.probs[i].dep = dep;
-                pl.probs[i].dep_off = dep < 0 ? 0 : (long long)((xa - reinterpret_cast<uintptr_t>(descs[dep].Y)) / 2);
-            }
-        }
-        if (barrier) {
-            pl.ph_mode[ph] |= 1;
-            pl.ph_mode[ph - 1] |= 2;
-            for (int i = phase_begin[ph]; i < phase_begin[ph + 1]; ++i) pl.probs[i].dep = -1;
-        }
-    }
-}
-
 bool chain_launch_ok(const ProbShape* shapes, int count, int n_phases, int64_t M) {
     if (M < 1 || M > 4 || n_phases > kSMaxPhases || n_phases > SHERRY_MAX_BATCH || count > SHERRY_MAX_BATCH)
         return false;
@@ -1528,7 +1342,6 @@ int chain_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs
     if (!chain_launch_ok(shapes, count, n_phases, M)) return SHERRY_ERR_UNSUPPORTED;
     SPlan pl = make_splan(shapes, count, phase_begin, n_phases, M, sms, M <= 3 ? 16 : 8);
     attach(pl, descs, count);
-    plan_dataflow(pl, descs, count, phase_begin, n_phases, M, y_bf16);
     // the kernel's phase table has one slot per problem slot of its instantiation
     const int slots = std::max(count, n_phases);
     switch (M) {
