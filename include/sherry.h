@@ -229,9 +229,11 @@ typedef struct sherry_linear_desc {
  * (except that the streaming kernel's problems go to the others when the whole
  * batch has more row blocks than its tickets): the problems that share a kernel
  * share one launch of it (each prefill problem, M >= 17, gets a launch of its
- * own).  Y agrees with sherry_linear's within the fp32 summation-order bound;
- * the streaming kernel (one or two tokens) splits K where the batch as a whole
- * balances best, so it is not bit-identical to a single call.  A call
+ * own; several such launches run on four library-owned side streams per device,
+ * forked from `stream` and joined back into it with events, so `stream`'s order
+ * and graph capture hold).  Y agrees with sherry_linear's within the fp32
+ * summation-order bound; the streaming kernels (1 to 16 tokens) split K where the
+ * batch as a whole balances best, so they are not bit-identical to a single call.  A call
  * repeated with the same arguments gives bit-identical Y.  `descs` is a HOST
  * array, read during the call only.  count <= SHERRY_MAX_BATCH.
  *   workspace  sherry_linear_batched_workspace_bytes(descs, count, M) bytes. */
@@ -344,13 +346,14 @@ int sherry_device_status(void* stream);
  * wait gave up since, and the cached ticket regions must be zeroed again. */
 int64_t sherry_timeout_count(void);
 /* Budget, in SM clock cycles, of every bounded wait of the streaming decode
- * kernel (one or two tokens), for launches made after this call; cycles <= 0
+ * kernels (1 to 16 tokens, and chained launches), for launches made after this call; cycles <= 0
  * restores the default (4e9, about 2 s at the boost clock).  Returns the previous
  * budget.  Meant for exercising the failure path: with a budget of a few cycles
  * the waits give up, the call's outputs are invalid, and sherry_device_status
- * reports SHERRY_ERR_TIMEOUT.  That kernel holds no tensor memory and issues
- * only cp.async copies, which it completes before exiting, so the context stays
- * usable.  The tensor-core kernels keep the default budget. */
+ * reports SHERRY_ERR_TIMEOUT.  These kernels hold no tensor memory (their
+ * tensor-core form multiplies with mma.sync in registers) and issue only
+ * cp.async copies, which they complete before exiting, so the context stays
+ * usable.  The tcgen05 kernels keep the default budget. */
 int64_t sherry_set_wait_budget(int64_t cycles);
 /* library version, e.g. 0x000100 = 0.1.0 */
 int sherry_version(void);

@@ -1,14 +1,16 @@
-// gemv_stream.cu -- packed 3:4 ternary linear for one to four tokens (M <= 4),
-// HBM-streaming version of the lookup-table decode (the method's inference
+// gemv_stream.cu -- packed 3:4 ternary linear for 1 to 16 tokens, streamed from
+// HBM: the lookup-table decode for up to three tokens (the method's inference
 // scheme: tables built from the activations, looked up by the packed weights,
 // accumulated, then scaled; "Sherry: Hardware-Efficient 1.25-Bit Ternary
 // Quantization via Fine-grained Sparsification", digest paragraph on inference;
 // Y = X T alpha).
 //
-// Work unit: 512 output rows x 32 W weights (W packed words) of one linear, W =
-// 16 for one to three tokens, W = 8 for four tokens (whose tables take more
-// shared memory); the same for independent linears (one batched launch per
-// decode step) and for chained phases.
+// Work unit: 512 output rows x 32 W weights (W packed words) of one linear: W =
+// 16 for independent linears (one batched launch per decode step) and for
+// chained phases of up to three tokens, W = 8 for a four-token chain (whose
+// tables take more shared memory).  From four tokens on, independent linears
+// take the tensor-core consumers (k_mma_stream, further below) on the same
+// pipeline.
 // All units of a phase (one or many independent linears) are split into equal
 // contiguous ranges, one per CTA (stream-K): every CTA streams the same number
 // of bytes.  A row block whose units straddle CTAs is finished by the CTA that
@@ -19,10 +21,11 @@
 // of a decoder layer stack for one token): a later phase may read an earlier
 // phase's Y as its X.  The launch is cooperative (one CTA per SM, all resident);
 // after its last unit of a phase a CTA adds one arrival to the phase's counter,
-// and before building the first tables of a phase a CTA waits (bounded) until
+// and before building the first tables of a phase a CTA checks (bounded) that
 // every CTA has arrived at the previous phase.  Packed weights do not depend on
-// X, so the copies of the next units run ahead of that wait and stream from HBM
-// while the barrier resolves.
+// X, so the copies of the next units go on while the barrier resolves; a helper
+// blocks on it only when the stage it would refill still waits for the blocked
+// tables.
 //
 // Roles (20 warps).  16 consumer warps: each thread owns one row of the unit
 // and only looks up and accumulates (per packed word it spreads the 8 nibbles
@@ -485,7 +488,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     constexpr int S = C::kStages;
     __shared__ int s_last;
     __shared__ int s_abort;
-    __shared__ int s_gate;  // phases known complete on every CTA (written by helper thread 0)
+    __shared__ int s_gate;  // phases known complete on every CTA (written by helper warp 0)
     // Shared addresses: the buffer is rounded up to 256 bytes, so every table
     // base is a multiple of 256 (a lookup's address replaces its low byte); the
     // XOR swizzles need only 16-byte alignment, since writer and reader apply them.
