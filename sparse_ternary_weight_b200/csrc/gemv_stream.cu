@@ -925,6 +925,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
     // ---- consumers: warp w owns unit rows 32w .. 32w+31 as two m16 tiles
     const int g = lane >> 2, c = lane & 3;
     const uint32_t sh = 8u * c, ss = 2u * c;
+    const uint32_t psel = 0x7650u | (uint32_t)c;  // byte c of an offset vector, bytes 1-3 of the table base
     int rows[4];  // unit rows of the lane: tile 0 rows g, g+8; tile 1 rows g, g+8
 #pragma unroll
     for (int i = 0; i < 4; ++i) rows[i] = 32 * warp + 16 * (i >> 1) + g + 8 * (i & 1);
@@ -957,13 +958,25 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
 #pragma unroll
                         for (int i = 0; i < 4; ++i) cs[a][b][i] = 0.0f;
             }
+            // rows' packed words: with one token tile each lane reads its rows' 4-word
+            // chunk and decodes its own bytes; with two, lane (g, c) spreads word 4q + c of
+            // each of its rows into table offsets (byte i of ev: 4 * code of block 2i, of
+            // od: block 2i + 1) and the four lanes of a row share them through shuffles,
+            // which saves registers and instructions there
             uint4 wv[4];
-            uint32_t sv[4];
+            uint32_t sv[4], evr[4], odr[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = rows[i];
-                wv[i] = lds128(st + r * G::kRowB + (((uint32_t)q ^ (uint32_t)((r / G::kSwz) % G::kLanesPerRow)) << 4));
-                sv[i] = lds32(st + G::kIdx + r * 16 + 4 * q);
+                const uint32_t chunk = st + r * G::kRowB + (((uint32_t)q ^ (uint32_t)((r / G::kSwz) % G::kLanesPerRow)) << 4);
+                if constexpr (NB == 1) {
+                    wv[i] = lds128(chunk);
+                    sv[i] = lds32(st + G::kIdx + r * 16 + 4 * q);
+                } else {
+                    const uint32_t w = lds32(chunk + 4u * c);
+                    const uint32_t sb = (lds32(st + G::kIdx + r * 16 + 4 * q) >> (8u * c)) & 0xffu;
+                    spread_word(w, sb, evr[i], odr[i]);
+                }
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -976,13 +989,21 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
 #pragma unroll
                     for (int ii = 0; ii < 2; ++ii) {
                         const int i = 2 * a + ii;
-                        const uint32_t w = j == 0 ? wv[i].x : j == 1 ? wv[i].y : j == 2 ? wv[i].z : wv[i].w;
-                        uint32_t oa, ob;
-                        m_codes(w, sv[i] >> (8 * j), sh, ss, oa, ob);
-                        A[ii][0][0] = lds32(pat + oa);
-                        A[ii][0][1] = lds32(pat + 128u + oa);
-                        A[ii][1][0] = lds32(pat + ob);
-                        A[ii][1][1] = lds32(pat + 128u + ob);
+                        uint32_t aa, ab;  // table addresses of blocks 2c and 2c + 1
+                        if constexpr (NB == 1) {
+                            const uint32_t w = j == 0 ? wv[i].x : j == 1 ? wv[i].y : j == 2 ? wv[i].z : wv[i].w;
+                            m_codes(w, sv[i] >> (8 * j), sh, ss, aa, ab);
+                            aa += pat;
+                            ab += pat;
+                        } else {
+                            const int src = (lane & ~3) | j;
+                            aa = __byte_perm(__shfl_sync(kFull, evr[i], src), pat, psel);
+                            ab = __byte_perm(__shfl_sync(kFull, odr[i], src), pat, psel);
+                        }
+                        A[ii][0][0] = lds32(aa);
+                        A[ii][0][1] = lds32(aa + 128u);
+                        A[ii][1][0] = lds32(ab);
+                        A[ii][1][1] = lds32(ab + 128u);
                     }
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh)
