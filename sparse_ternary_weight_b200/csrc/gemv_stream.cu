@@ -784,7 +784,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
     }
 }
 
-// ---- tensor-core consumers for 5 to 16 tokens ------------------------------------
+// ---- tensor-core consumers for 4 to 16 tokens ------------------------------------
 //
 // The same streaming pipeline (units of 512 rows x 512 weights, stream-K ranges,
 // helper warps copying the packed planes into a cp.async ring, split tiles
@@ -798,7 +798,10 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_stream(const __grid_consta
 // lane % 4 holds the fragment positions k = 2c, 2c+1, 2c+8, 2c+9, taken to be the 4
 // weights of block 2c + h, so its two blocks per word are byte c of the packed
 // word and its activation fragments for both slices are the 8 consecutive
-// activations 8c .. 8c+7 of the word, one 16-byte load.  Each consumer warp owns
+// activations 8c .. 8c+7 of the word, one 16-byte load.  A lane gathers byte c of
+// the four words of a row's 16-byte chunk into one register and spreads all eight
+// blocks into table offsets at once; each block then costs one byte permute (its
+// table address) and the two lookups.  Each consumer warp owns
 // 32 rows (two m16 tiles); alpha is applied once per scale group (or at the end
 // for row scales) in fp32 registers.
 
@@ -834,13 +837,17 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
                  : "memory");
 }
 
-// Table offsets (4 * code, code = nibble + 16 G) of blocks 2c and 2c+1 of a packed
-// word w with sign byte s, for the lane's c (shifts precomputed: sh = 8c, ss = 2c).
-__device__ __forceinline__ void m_codes(uint32_t w, uint32_t s, uint32_t sh, uint32_t ss, uint32_t& oa,
-                                        uint32_t& ob) {
-    const uint32_t x = w >> sh, sb = s >> ss;
-    oa = ((x << 2) & 0x3cu) | ((sb << 6) & 0x40u);
-    ob = ((x >> 2) & 0x3cu) | ((sb << 5) & 0x40u);
+// Table offsets of the lane's blocks in the four words of a 16-byte chunk: byte j of
+// ev is 4 * code of block 2c of word j, of od of block 2c + 1 (code = nibble + 16 G;
+// s holds the four words' sign bytes).  Byte c of every word is gathered first
+// (gsel = c | (c + 4) << 4), so one spread serves the four words; the sign bits 2c
+// and 2c + 1 of each sign byte move to bit 6 with one shift (gsh = 6 - 2c).
+__device__ __forceinline__ void m_offsets(uint4 w, uint32_t s, uint32_t gsel, uint32_t gsh, uint32_t& ev,
+                                          uint32_t& od) {
+    const uint32_t b = __byte_perm(__byte_perm(w.x, w.y, gsel), __byte_perm(w.z, w.w, gsel), 0x5410u);
+    const uint32_t v = s << gsh;
+    ev = ((b << 2) & 0x3c3c3c3cu) | (v & 0x40404040u);
+    od = ((b >> 2) & 0x3c3c3c3cu) | ((v >> 1) & 0x40404040u);
 }
 
 template <int MAXP, int NT>
@@ -924,8 +931,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
 
     // ---- consumers: warp w owns unit rows 32w .. 32w+31 as two m16 tiles
     const int g = lane >> 2, c = lane & 3;
-    const uint32_t sh = 8u * c, ss = 2u * c;
-    const uint32_t psel = 0x7650u | (uint32_t)c;  // byte c of an offset vector, bytes 1-3 of the table base
+    const uint32_t gsel = (uint32_t)c | ((uint32_t)(c + 4) << 4), gsh = 6u - 2u * (uint32_t)c;
     int rows[4];  // unit rows of the lane: tile 0 rows g, g+8; tile 1 rows g, g+8
 #pragma unroll
     for (int i = 0; i < 4; ++i) rows[i] = 32 * warp + 16 * (i >> 1) + g + 8 * (i & 1);
@@ -958,25 +964,14 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
 #pragma unroll
                         for (int i = 0; i < 4; ++i) cs[a][b][i] = 0.0f;
             }
-            // rows' packed words: with one token tile each lane reads its rows' 4-word
-            // chunk and decodes its own bytes; with two, lane (g, c) spreads word 4q + c of
-            // each of its rows into table offsets (byte i of ev: 4 * code of block 2i, of
-            // od: block 2i + 1) and the four lanes of a row share them through shuffles,
-            // which saves registers and instructions there
-            uint4 wv[4];
-            uint32_t sv[4], evr[4], odr[4];
+            // rows' packed words: each lane reads its rows' 4-word chunk and spreads its
+            // blocks of all four words into table offsets at once (m_offsets)
+            uint32_t evr[4], odr[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = rows[i];
                 const uint32_t chunk = st + r * G::kRowB + (((uint32_t)q ^ (uint32_t)((r / G::kSwz) % G::kLanesPerRow)) << 4);
-                if constexpr (NB == 1) {
-                    wv[i] = lds128(chunk);
-                    sv[i] = lds32(st + G::kIdx + r * 16 + 4 * q);
-                } else {
-                    const uint32_t w = lds32(chunk + 4u * c);
-                    const uint32_t sb = (lds32(st + G::kIdx + r * 16 + 4 * q) >> (8u * c)) & 0xffu;
-                    spread_word(w, sb, evr[i], odr[i]);
-                }
+                m_offsets(lds128(chunk), lds32(st + G::kIdx + r * 16 + 4 * q), gsel, gsh, evr[i], odr[i]);
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -989,17 +984,10 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
 #pragma unroll
                     for (int ii = 0; ii < 2; ++ii) {
                         const int i = 2 * a + ii;
-                        uint32_t aa, ab;  // table addresses of blocks 2c and 2c + 1
-                        if constexpr (NB == 1) {
-                            const uint32_t w = j == 0 ? wv[i].x : j == 1 ? wv[i].y : j == 2 ? wv[i].z : wv[i].w;
-                            m_codes(w, sv[i] >> (8 * j), sh, ss, aa, ab);
-                            aa += pat;
-                            ab += pat;
-                        } else {
-                            const int src = (lane & ~3) | j;
-                            aa = __byte_perm(__shfl_sync(kFull, evr[i], src), pat, psel);
-                            ab = __byte_perm(__shfl_sync(kFull, odr[i], src), pat, psel);
-                        }
+                        // table addresses of blocks 2c and 2c + 1 of word j (the table base
+                        // is 256-byte aligned: its low byte is the offset)
+                        const uint32_t aa = __byte_perm(evr[i], pat, 0x7650u | (uint32_t)j);
+                        const uint32_t ab = __byte_perm(odr[i], pat, 0x7650u | (uint32_t)j);
                         A[ii][0][0] = lds32(aa);
                         A[ii][0][1] = lds32(aa + 128u);
                         A[ii][1][0] = lds32(ab);
