@@ -1116,6 +1116,306 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
     }
 }
 
+// ---- chained decode on whole-K row blocks (one and two tokens) ---------------------
+//
+// A chained phase of one decode step holds 4.5-19 MB of packed weights; split into
+// the streaming kernel's 512 x 512 units, every row block of a phase is shared by
+// 6-16 CTAs and each phase pays the split-tile handshake (partials, ticket, the last
+// CTA's sum) on top of the grid barrier.  This kernel gives every row block to one
+// CTA instead.  Item = 32 rows of one linear over all of K: lane = row, and the 16
+// consumer warps split K into 128-weight slices (one packed 16-byte chunk, one
+// group-128 scale), so the K reduction stays inside the CTA (a fixed-order sum
+// over the warps in shared memory).  K runs in chunks of 2048 weights (16 slices):
+// per chunk the consumers build the chunk's 512 tables per token (one per thread)
+// and then look up every item of the CTA's current segment (up to kCSeg items of
+// one linear), so the tables are built once per segment, not per item.  Four
+// helper warps copy the items' packed words (row-major, XOR-swizzled 16-byte
+// chunks), sign words and scales (both transposed to [slice][row], 4-byte copies)
+// into a ring of stages; they run ahead across phases, since weights do not
+// depend on X.  Each phase's items are split into contiguous, balanced ranges over
+// the CTAs; a CTA arrives at the phase counter after its Y stores (release) and
+// waits for the previous phase's count before reading its X (acquire).
+constexpr int kCRows = 32;                      // rows per item: one per lane
+constexpr int kCSl = kSConsumers;               // 128-weight slices per chunk: one per consumer warp
+constexpr int kCChunk = 128 * kCSl;             // weights per chunk
+constexpr int kCBlocks = kCChunk / 4;           // tables per chunk and token: one per consumer thread
+constexpr int kCIdx = kCRows * kCSl * 16;       // packed words of a stage: [row][slice] 16-byte chunks
+constexpr int kCSgn = kCSl * kCRows * 4;        // sign words (4 per slice): [slice][row]
+constexpr int kCSc = kCSl * kCRows * 4;         // scales: [slot][row], slot = slice (group 128) or slice / 2
+constexpr int kCStage = kCIdx + kCSgn + kCSc;   // 12 KB
+constexpr int kCTok = kCBlocks * kTab;          // one token's tables of a chunk
+constexpr int kCSeg = 4;                        // items of one linear sharing the tables
+constexpr int kCStages = 4;
+static_assert(kCBlocks == 32 * kSConsumers, "one table per consumer thread");
+static_assert(kCTok % 256 == 0 && (32 * kTab) % 256 == 0 && kCStage % 256 == 0, "256-aligned table bases");
+
+template <int MT>
+struct CCfg {
+    static constexpr int kStages = MT * kCTok;                      // after the tables
+    static constexpr int kRed = kStages + kCStages * kCStage;       // [warp][item][token][row] partials
+    static constexpr int kBars = kRed + kSConsumers * kCSeg * MT * kCRows * 4;
+    static constexpr int kSmem = 256 + kBars + 8 * (2 * kCStages + 1);
+    static_assert(kSmem <= 232448, "shared memory per CTA");
+};
+
+struct CProb {
+    const uint16_t* X;
+    const uint32_t* idx;
+    const uint8_t* sgn;
+    const float* scales;
+    void* Y;
+    int N, K, spr;      // spr: scales per row (group scales)
+    int mode, per_tensor;
+    int n_items, item_begin;  // 32-row items; the first one's index in the launch
+};
+
+template <int MAXP>
+struct CParams {
+    long long wait_cycles;
+    int count, y_bf16, n_phases;
+    int* phase_cnt;          // [n_phases] arrivals + the exit counter
+    int ph_prob[MAXP + 1];   // first problem of each phase
+    int ph_item[MAXP + 1];   // first item of each phase; ph_item[n_phases] = all items
+    CProb p[MAXP];
+};
+
+struct CSeg {
+    int p, it, n;  // problem, its first item of the segment, items
+};
+
+// the segment of this CTA's range [g, e) of a phase that starts at launch item g
+template <int MAXP>
+__device__ __forceinline__ CSeg seg_at(const CParams<MAXP>& P, int ph, int g, int e) {
+    int lo = P.ph_prob[ph], hi = P.ph_prob[ph + 1] - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.p[mid].item_begin <= g)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    const CProb& pr = P.p[lo];
+    return CSeg{lo, g - pr.item_begin, min(kCSeg, min(e, pr.item_begin + pr.n_items) - g)};
+}
+
+template <int MAXP>
+__device__ __forceinline__ void cta_items(const CParams<MAXP>& P, int ph, int& b, int& e) {
+    const int b0 = P.ph_item[ph];
+    const long long n = P.ph_item[ph + 1] - b0;
+    b = b0 + (int)(n * blockIdx.x / gridDim.x);
+    e = b0 + (int)(n * (blockIdx.x + 1) / gridDim.x);
+}
+
+__device__ __forceinline__ int chunk_slices(const CProb& pr, int c) { return min(kCSl, (pr.K - c * kCChunk) >> 7); }
+
+// Copy item `it`, chunk c of problem pr into the stage at st (128 helper threads,
+// ht = 0..127); rows past N are not copied (their results are never stored).
+__device__ __forceinline__ void copy_item(const CProb& pr, int it, int c, uint32_t st, int ht) {
+    const int row0 = it * kCRows;
+    const int rows = min(kCRows, pr.N - row0);
+    const int nsl = chunk_slices(pr, c);
+    const char* ib = reinterpret_cast<const char*>(pr.idx) + (int64_t)row0 * (pr.K >> 3) + (c * kCChunk >> 3);
+    for (int i = ht; i < rows * nsl; i += kSHelperThreads) {
+        const int r = i / nsl, q = i - r * nsl;
+        cp_async16(st + r * (16 * kCSl) + ((q ^ (r & 7)) << 4), ib + (int64_t)r * (pr.K >> 3) + 16 * q);
+    }
+    const uint8_t* sb = pr.sgn + (int64_t)row0 * (pr.K >> 5) + (c * kCChunk >> 5);
+    for (int i = ht; i < rows * nsl; i += kSHelperThreads) {
+        const int r = i / nsl, q = i - r * nsl;
+        cp_async4(st + kCIdx + 4 * (q * kCRows + r), sb + (int64_t)r * (pr.K >> 5) + 4 * q);
+    }
+    if (pr.mode != kSRow) {
+        const int ns = pr.mode == kSG128 ? nsl : nsl >> 1;
+        const float* cb = pr.scales + (int64_t)row0 * pr.spr + (pr.mode == kSG128 ? c * kCSl : c * kCSl / 2);
+        for (int i = ht; i < rows * ns; i += kSHelperThreads) {
+            const int r = i / ns, q = i - r * ns;
+            cp_async4(st + kCIdx + kCSgn + 4 * (q * kCRows + r), cb + (int64_t)r * pr.spr + q);
+        }
+    }
+}
+
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+
+template <int MAXP, int MT>
+__global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant__ CParams<MAXP> P) {
+    using C = CCfg<MT>;
+    constexpr int S = kCStages;
+    __shared__ int s_abort;
+    const uint32_t tabs = (smem_u32(g_smem) + 255u) & ~255u;  // [token][kCBlocks tables]
+    const uint32_t stages = tabs + C::kStages;
+    const uint32_t red = tabs + C::kRed;
+    const uint32_t bars = tabs + C::kBars;
+    auto ready = [&](int s) { return bars + 8u * (uint32_t)s; };
+    auto empty = [&](int s) { return bars + 8u * (uint32_t)(S + s); };
+    const uint32_t cb = bars + 8u * (uint32_t)(2 * S);  // the consumer warps' own barrier
+
+    const int t = threadIdx.x;
+    const int lane = t & 31, warp = t >> 5;
+    if (t == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(ready(s), kSHelperThreads);  // one cp.async arrival per helper thread
+            mbar_init(empty(s), kSRows);
+        }
+        mbar_init(cb, kSRows);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    volatile int* abort_flag = &s_abort;
+
+    if (warp >= kSConsumers) {
+        // ---- helpers: the CTA's stages (segment, chunk, item) in the consumers' order
+        const int ht = t - 32 * kSConsumers;
+        int j = 0;
+        bool ok = true;
+        for (int ph = 0; ph < P.n_phases && ok; ++ph) {
+            int b, e;
+            cta_items(P, ph, b, e);
+            for (int g = b; g < e && ok;) {
+                const CSeg sg = seg_at(P, ph, g, e);
+                const CProb& pr = P.p[sg.p];
+                const int nc = (pr.K + kCChunk - 1) / kCChunk;
+                for (int c = 0; c < nc && ok; ++c)
+                    for (int i = 0; i < sg.n; ++i, ++j) {
+                        const int s = j % S;
+                        if (j >= S && !mbar_wait(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag, P.wait_cycles)) {
+                            ok = false;
+                            break;
+                        }
+                        copy_item(pr, sg.it + i, c, stages + s * kCStage, ht);
+                        cp_async_arrive(ready(s));
+                    }
+                g += sg.n;
+            }
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    } else {
+        // ---- consumers: lane = row of the item, warp = 128-weight slice of the chunk
+        const int w = warp, r = lane;
+        int k = 0;   // stages consumed
+        int nb = 0;  // consumer barriers passed
+        bool ok = true;
+        auto csync = [&]() -> bool {
+            mbar_arrive(cb);
+            const bool fine = mbar_wait(cb, (uint32_t)(nb & 1), abort_flag, P.wait_cycles);
+            ++nb;
+            return fine;
+        };
+        float acc[kCSeg][MT];
+        for (int ph = 0; ph < P.n_phases && ok; ++ph) {
+            int b, e;
+            cta_items(P, ph, b, e);
+            bool gated = ph == 0;
+            for (int g = b; g < e && ok;) {
+                const CSeg sg = seg_at(P, ph, g, e);
+                const CProb& pr = P.p[sg.p];
+                const int nc = (pr.K + kCChunk - 1) / kCChunk;
+#pragma unroll
+                for (int i = 0; i < kCSeg; ++i)
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) acc[i][m] = 0.0f;
+                for (int c = 0; c < nc && ok; ++c) {
+                    if (!gated) {
+                        // every CTA is past the previous phase: this phase's X is complete
+                        if (w == 0) {
+                            if (grid_poll(P.phase_cnt + ph - 1, (int)gridDim.x, abort_flag, P.wait_cycles, true,
+                                          lane) != 1) {
+                                ok = false;
+                                break;
+                            }
+                            __threadfence();
+                        }
+                        gated = true;
+                    }
+                    // nobody reads the previous chunk's tables any more
+                    if (!(ok = csync())) break;
+                    const int nsl = chunk_slices(pr, c);
+                    if (t < 32 * nsl) {
+                        // table of block t of the chunk, per token (X read through L2: an
+                        // earlier phase of this launch wrote it)
+                        const uint2* xs = reinterpret_cast<const uint2*>(pr.X) + (c * kCChunk >> 2) + t;
+#pragma unroll
+                        for (int m = 0; m < MT; ++m)
+                            build_table(tabs + m * kCTok + t * kTab, __ldcg(xs + (int64_t)m * (pr.K >> 2)));
+                    }
+                    if (!(ok = csync())) break;
+#pragma unroll
+                    for (int i = 0; i < kCSeg; ++i) {
+                        if (i < sg.n) {
+                            const int s = k % S;
+                            if (!(ok = mbar_wait(ready(s), (uint32_t)((k / S) & 1), abort_flag, P.wait_cycles))) break;
+                            if (w < nsl) {
+                                const uint32_t st = stages + s * kCStage;
+                                const uint4 wq = lds128(st + r * (16 * kCSl) + (((uint32_t)w ^ (uint32_t)(r & 7)) << 4));
+                                const uint32_t sq = lds32(st + kCIdx + 4 * (w * kCRows + r));
+                                const uint32_t tb = tabs + (uint32_t)(w * 32 * kTab);
+                                float p0[MT], p1[MT], q0[MT], q1[MT], r0[MT], r1[MT], u0[MT], u1[MT];
+                                word_sums<0, MT, kCTok>(wq.x, sq & 0xffu, tb, p0, p1);
+                                word_sums<8, MT, kCTok>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
+                                word_sums<16, MT, kCTok>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
+                                word_sums<24, MT, kCTok>(wq.w, sq >> 24, tb, u0, u1);
+                                float al = 1.0f;
+                                if (pr.mode == kSG128) al = __uint_as_float(lds32(st + kCIdx + kCSgn + 4 * (w * kCRows + r)));
+                                if (pr.mode == kSG256)
+                                    al = __uint_as_float(lds32(st + kCIdx + kCSgn + 4 * ((w >> 1) * kCRows + r)));
+#pragma unroll
+                                for (int m = 0; m < MT; ++m) {
+                                    const float v =
+                                        ((p0[m] + p1[m]) + (q0[m] + q1[m])) + ((r0[m] + r1[m]) + (u0[m] + u1[m]));
+                                    acc[i][m] = pr.mode == kSRow ? acc[i][m] + v : fmaf(al, v, acc[i][m]);
+                                }
+                            }
+                            mbar_arrive(empty(s));
+                            ++k;
+                        }
+                    }
+                }
+                if (!ok) break;
+                // the K reduction: every warp's partials, summed over the warps in order
+#pragma unroll
+                for (int i = 0; i < kCSeg; ++i)
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        if (i < sg.n) sts_f32(red + 4 * (((w * kCSeg + i) * MT + m) * kCRows + r), acc[i][m]);
+                if (!(ok = csync())) break;
+                if (w < sg.n * MT) {
+                    const int i = w / MT, m = w - i * MT;
+                    float sum = 0.0f;
+#pragma unroll
+                    for (int v = 0; v < kSConsumers; ++v) sum += lds_f32(red + 4 * (((v * kCSeg + i) * MT + m) * kCRows + r));
+                    const int n = (sg.it + i) * kCRows + r;
+                    if (n < pr.N) {
+                        if (pr.mode == kSRow) sum *= __ldg(pr.scales + (pr.per_tensor ? 0 : n));
+                        if (P.y_bf16)
+                            reinterpret_cast<__nv_bfloat16*>(pr.Y)[(int64_t)m * pr.N + n] = __float2bfloat16_rn(sum);
+                        else
+                            reinterpret_cast<float*>(pr.Y)[(int64_t)m * pr.N + n] = sum;
+                    }
+                }
+                g += sg.n;
+            }
+            if (!ok) break;
+            // arrival: the CTA's Y of this phase is stored (seen through the barrier)
+            if (!(ok = csync())) break;
+            if (t == 0) {
+                __threadfence();
+                red_release_add(P.phase_cnt + ph, 1);
+            }
+        }
+    }
+    __syncthreads();
+    if (t == 0 && !*abort_flag) {
+        // the last CTA to leave zeroes the phase counters for the next launch
+        __threadfence();
+        if (atomicAdd(P.phase_cnt + P.n_phases, 1) == (int)gridDim.x - 1) {
+            for (int ph = 0; ph <= P.n_phases; ++ph) P.phase_cnt[ph] = 0;
+            __threadfence();
+        }
+    }
+}
+
 // ---- host side -------------------------------------------------------------------
 
 // Units of W words: K a multiple of 32 W; group scales of 128 or 256 weights
@@ -1213,6 +1513,7 @@ size_t stream_workspace_bytes(const ProbShape* shapes, int count, int64_t M, int
 
 size_t chain_workspace_bytes(const ProbShape* shapes, int count, const int* phase_begin, int n_phases, int64_t M,
                              int sms) {
+    if (M <= 2) return kTicketBytes;  // the row-block kernel keeps only its phase counters there
     return make_splan(shapes, count, phase_begin, n_phases, M, sms, M <= 3 ? 16 : 8).ws_bytes;
 }
 
@@ -1349,9 +1650,85 @@ bool chain_launch_ok(const ProbShape* shapes, int count, int n_phases, int64_t M
     return tiles <= kMaxTickets - kChainCtrs;
 }
 
+// Chains of one or two tokens run on the row-block kernel (k_lut_rows): every linear's
+// items are 32 rows over all of K, so no row block is split over CTAs.  Shapes are
+// those of the streaming kernel (K a multiple of 512: whole 16-byte slices per row
+// and 16-byte aligned row starts in every plane).
+template <int MAXP, int MT>
+static int rows_launch_t(const ProbShape* shapes, const sherry_linear_desc* descs, int count, const int* phase_begin,
+                         int n_phases, int y_bf16, void* workspace, int sms, cudaStream_t stream) {
+    static CParams<MAXP> P;
+    static std::mutex mu;
+    static PerDevice attr;
+    std::lock_guard<std::mutex> lk(mu);
+    P.wait_cycles = g_stream_wait.load();
+    P.count = count;
+    P.y_bf16 = y_bf16;
+    P.n_phases = n_phases;
+    P.phase_cnt = static_cast<int*>(workspace) + (kMaxTickets - kChainCtrs);
+    int items = 0;
+    for (int i = 0; i < count; ++i) {
+        const ProbShape& sh = shapes[i];
+        CProb c{};
+        c.X = descs[i].X;
+        c.idx = descs[i].idx;
+        c.sgn = descs[i].sgn;
+        c.scales = descs[i].scales;
+        c.Y = descs[i].Y;
+        c.N = (int)sh.N;
+        c.K = (int)sh.K;
+        c.spr = sh.granularity == SHERRY_PER_GROUP ? (int)(sh.K / sh.group) : 0;
+        c.mode = sh.granularity != SHERRY_PER_GROUP ? kSRow : (sh.group == 128 ? kSG128 : kSG256);
+        c.per_tensor = sh.granularity == SHERRY_PER_TENSOR;
+        c.n_items = (int)((sh.N + kCRows - 1) / kCRows);
+        c.item_begin = items;
+        items += c.n_items;
+        P.p[i] = c;
+    }
+    for (int ph = 0; ph <= n_phases; ++ph) {
+        P.ph_prob[ph] = phase_begin[ph];
+        P.ph_item[ph] = phase_begin[ph] < count ? P.p[phase_begin[ph]].item_begin : items;
+    }
+    int done = 0;
+    const int st = per_device(attr, &done, [](int& v) {
+        SHERRY_CUDA_CHECK(cudaFuncSetAttribute(k_lut_rows<MAXP, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               CCfg<MT>::kSmem));
+        v = 1;
+        return SHERRY_OK;
+    });
+    if (st) return st;
+    // every CTA must be resident: the phase barrier waits for all of them
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::max(1, sms));
+    cfg.blockDim = dim3(kSThreads);
+    cfg.dynamicSmemBytes = CCfg<MT>::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    SHERRY_CUDA_CHECK(cudaLaunchKernelEx(&cfg, k_lut_rows<MAXP, MT>, P));
+    SHERRY_LAUNCH_CHECK();
+    return SHERRY_OK;
+}
+
+template <int MT>
+static int rows_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, const int* phase_begin,
+                       int n_phases, int y_bf16, void* workspace, int sms, cudaStream_t stream) {
+    const int slots = std::max(count, n_phases);
+    if (slots <= 1) return rows_launch_t<1, MT>(shapes, descs, count, phase_begin, n_phases, y_bf16, workspace, sms, stream);
+    if (slots <= 16)
+        return rows_launch_t<16, MT>(shapes, descs, count, phase_begin, n_phases, y_bf16, workspace, sms, stream);
+    return rows_launch_t<SHERRY_MAX_BATCH, MT>(shapes, descs, count, phase_begin, n_phases, y_bf16, workspace, sms,
+                                               stream);
+}
+
 int chain_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, const int* phase_begin,
                         int n_phases, int64_t M, int y_bf16, void* workspace, int sms, cudaStream_t stream) {
     if (!chain_launch_ok(shapes, count, n_phases, M)) return SHERRY_ERR_UNSUPPORTED;
+    if (M == 1) return rows_launch<1>(shapes, descs, count, phase_begin, n_phases, y_bf16, workspace, sms, stream);
+    if (M == 2) return rows_launch<2>(shapes, descs, count, phase_begin, n_phases, y_bf16, workspace, sms, stream);
     SPlan pl = make_splan(shapes, count, phase_begin, n_phases, M, sms, M <= 3 ? 16 : 8);
     attach(pl, descs, count);
     // the kernel's phase table has one slot per problem slot of its instantiation
