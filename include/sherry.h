@@ -42,8 +42,8 @@
  *     unspecified (but memory-safe) results.
  *   - Shapes: N >= 0, M >= 0 (0 = nothing to do), 32 <= K <= SHERRY_MAX_K,
  *     K % 32 == 0; per-group needs group > 0, group % 32 == 0, K % group == 0.
- *   - Alignment: W, X, Y, W_out, scales and sgn 4-byte aligned, idx 16-byte
- *     aligned (else SHERRY_ERR_ALIGN).
+ *   - Alignment: W, X, Y, W_out, idx, sgn and scales 16-byte aligned (else
+ *     SHERRY_ERR_ALIGN): the kernels copy them in 16-byte pieces.
  *   - Results are deterministic: the same call on the same inputs gives the
  *     same bits (no float atomics; every reduction has a fixed order).
  */

@@ -1130,7 +1130,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
 // and then look up every item of the CTA's current segment (up to kCSeg items of
 // one linear), so the tables are built once per segment, not per item.  Four
 // helper warps copy the items' packed words (row-major, XOR-swizzled 16-byte
-// chunks), sign words and scales (both transposed to [slice][row], 4-byte copies)
+// chunks), sign words and scales (rows padded to 80 bytes) with 16-byte copies
 // into a ring of stages; they run ahead across phases, since weights do not
 // depend on X.  Each phase's items are split into contiguous, balanced ranges over
 // the CTAs; a CTA arrives at the phase counter after its Y stores (release) and
@@ -1140,18 +1140,21 @@ constexpr int kCSl = kSConsumers;               // 128-weight slices per chunk: 
 constexpr int kCChunk = 128 * kCSl;             // weights per chunk
 constexpr int kCBlocks = kCChunk / 4;           // tables per chunk and token: one per consumer thread
 constexpr int kCIdx = kCRows * kCSl * 16;       // packed words of a stage: [row][slice] 16-byte chunks
-constexpr int kCSgn = kCSl * kCRows * 4;        // sign words (4 per slice): [slice][row]
-constexpr int kCSc = kCSl * kCRows * 4;         // scales: [slot][row], slot = slice (group 128) or slice / 2
-constexpr int kCStage = kCIdx + kCSgn + kCSc;   // 12 KB
+constexpr int kCPad = 4 * kCSl + 16;            // bytes per row of sign words or scales (one per slice, padded)
+constexpr int kCSgn = kCRows * kCPad;           // sign words: 4 sign bytes per slice
+constexpr int kCSc = kCRows * kCPad;            // scales: one per slice (group 128) or per two (group 256)
+constexpr int kCStage = kCIdx + kCSgn + kCSc;   // 13 KB
 constexpr int kCTok = kCBlocks * kTab;          // one token's tables of a chunk
 constexpr int kCSeg = 4;                        // items of one linear sharing the tables
 constexpr int kCStages = 4;
 static_assert(kCBlocks == 32 * kSConsumers, "one table per consumer thread");
-static_assert(kCTok % 256 == 0 && (32 * kTab) % 256 == 0 && kCStage % 256 == 0, "256-aligned table bases");
+static_assert(kCTok % 256 == 0 && (32 * kTab) % 256 == 0, "256-aligned table bases");
+static_assert(kCStage % 16 == 0 && kCIdx % 16 == 0 && kCPad % 16 == 0, "16-byte aligned copies");
 
 template <int MT>
 struct CCfg {
-    static constexpr int kStages = MT * kCTok;                      // after the tables
+    static constexpr int kTB = MT == 1 ? 2 : 1;                     // table buffers (two fit for one token)
+    static constexpr int kStages = kTB * MT * kCTok;                // after the tables
     static constexpr int kRed = kStages + kCStages * kCStage;       // [warp][item][token][row] partials
     static constexpr int kBars = kRed + kSConsumers * kCSeg * MT * kCRows * 4;
     static constexpr int kSmem = 256 + kBars + 8 * (2 * kCStages + 1);
@@ -1219,17 +1222,31 @@ __device__ __forceinline__ void copy_item(const CProb& pr, int it, int c, uint32
         const int r = i / nsl, q = i - r * nsl;
         cp_async16(st + r * (16 * kCSl) + ((q ^ (r & 7)) << 4), ib + (int64_t)r * (pr.K >> 3) + 16 * q);
     }
-    const uint8_t* sb = pr.sgn + (int64_t)row0 * (pr.K >> 5) + (c * kCChunk >> 5);
-    for (int i = ht; i < rows * nsl; i += kSHelperThreads) {
-        const int r = i / nsl, q = i - r * nsl;
-        cp_async4(st + kCIdx + 4 * (q * kCRows + r), sb + (int64_t)r * (pr.K >> 5) + 4 * q);
+    // sign words: 4 * nsl bytes per row, whole 16-byte pieces (nsl is a multiple of 4)
+    const char* sb = reinterpret_cast<const char*>(pr.sgn) + (int64_t)row0 * (pr.K >> 5) + (c * kCChunk >> 5);
+    const int sp = nsl >> 2;
+    for (int i = ht; i < rows * sp; i += kSHelperThreads) {
+        const int r = i / sp, q = i - r * sp;
+        cp_async16(st + kCIdx + r * kCPad + 16 * q, sb + (int64_t)r * (pr.K >> 5) + 16 * q);
     }
     if (pr.mode != kSRow) {
-        const int ns = pr.mode == kSG128 ? nsl : nsl >> 1;
-        const float* cb = pr.scales + (int64_t)row0 * pr.spr + (pr.mode == kSG128 ? c * kCSl : c * kCSl / 2);
-        for (int i = ht; i < rows * ns; i += kSHelperThreads) {
-            const int r = i / ns, q = i - r * ns;
-            cp_async4(st + kCIdx + kCSgn + 4 * (q * kCRows + r), cb + (int64_t)r * pr.spr + q);
+        // group 128: nsl scales per row (16-byte pieces); group 256: nsl / 2 (8-byte pieces)
+        const int bytes = pr.mode == kSG128 ? 4 * nsl : 2 * nsl;
+        const char* cb = reinterpret_cast<const char*>(pr.scales + (int64_t)row0 * pr.spr) +
+                         (pr.mode == kSG128 ? 4 * c * kCSl : 2 * c * kCSl);
+        const uint32_t sc = st + kCIdx + kCSgn;
+        if (pr.mode == kSG128) {
+            const int np = bytes >> 4;
+            for (int i = ht; i < rows * np; i += kSHelperThreads) {
+                const int r = i / np, q = i - r * np;
+                cp_async16(sc + r * kCPad + 16 * q, cb + (int64_t)r * 4 * pr.spr + 16 * q);
+            }
+        } else {
+            const int np = bytes >> 3;
+            for (int i = ht; i < rows * np; i += kSHelperThreads) {
+                const int r = i / np, q = i - r * np;
+                cp_async8(sc + r * kCPad + 8 * q, cb + (int64_t)r * 4 * pr.spr + 8 * q);
+            }
         }
     }
 }
@@ -1243,7 +1260,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
     using C = CCfg<MT>;
     constexpr int S = kCStages;
     __shared__ int s_abort;
-    const uint32_t tabs = (smem_u32(g_smem) + 255u) & ~255u;  // [token][kCBlocks tables]
+    const uint32_t tabs = (smem_u32(g_smem) + 255u) & ~255u;  // [buffer][token][kCBlocks tables]
     const uint32_t stages = tabs + C::kStages;
     const uint32_t red = tabs + C::kRed;
     const uint32_t bars = tabs + C::kBars;
@@ -1256,9 +1273,9 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
     if (t == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(ready(s), kSHelperThreads);  // one cp.async arrival per helper thread
-            mbar_init(empty(s), kSRows);
+            mbar_init(empty(s), kSConsumers);      // one arrival per consumer warp
         }
-        mbar_init(cb, kSRows);
+        mbar_init(cb, kSConsumers);
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -1296,18 +1313,33 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
         const int w = warp, r = lane;
         int k = 0;   // stages consumed
         int nb = 0;  // consumer barriers passed
+        int nt = 0;  // chunks whose tables were built
         bool ok = true;
+        // a barrier of the 16 consumer warps: each warp's lanes meet first, then lane 0
+        // arrives for the warp (its release covers the lanes' shared-memory writes)
         auto csync = [&]() -> bool {
-            mbar_arrive(cb);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(cb);
             const bool fine = mbar_wait(cb, (uint32_t)(nb & 1), abort_flag, P.wait_cycles);
             ++nb;
             return fine;
         };
         float acc[kCSeg][MT];
+        uint2 xn[MT];  // this thread's block of the next chunk's activations, per token
+        // activations of block t of chunk c (read through L2: an earlier phase of this
+        // launch wrote them)
+        auto load_x = [&](const CProb& px, int c) {
+            const uint2* xs = reinterpret_cast<const uint2*>(px.X) + (c * kCChunk >> 2) + t;
+            if (t < 32 * chunk_slices(px, c)) {
+#pragma unroll
+                for (int m = 0; m < MT; ++m) xn[m] = __ldcg(xs + (int64_t)m * (px.K >> 2));
+            }
+        };
         for (int ph = 0; ph < P.n_phases && ok; ++ph) {
             int b, e;
             cta_items(P, ph, b, e);
             bool gated = ph == 0;
+            bool have_x = false;  // xn holds the next chunk's activations
             for (int g = b; g < e && ok;) {
                 const CSeg sg = seg_at(P, ph, g, e);
                 const CProb& pr = P.p[sg.p];
@@ -1317,6 +1349,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
 #pragma unroll
                     for (int m = 0; m < MT; ++m) acc[i][m] = 0.0f;
                 for (int c = 0; c < nc && ok; ++c) {
+                    bool fresh = false;  // this chunk opens a phase behind the grid barrier
                     if (!gated) {
                         // every CTA is past the previous phase: this phase's X is complete
                         if (w == 0) {
@@ -1328,18 +1361,29 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
                             __threadfence();
                         }
                         gated = true;
+                        fresh = true;
                     }
-                    // nobody reads the previous chunk's tables any more
-                    if (!(ok = csync())) break;
+                    // nobody reads this table buffer any more (with two buffers the barrier
+                    // after the previous chunk's build already ensures it) and, after a
+                    // grid barrier, every warp may read the new X
+                    if ((C::kTB == 1 || fresh) && !(ok = csync())) break;
+                    const uint32_t tb0 = tabs + (uint32_t)((nt++ % C::kTB) * MT * kCTok);
                     const int nsl = chunk_slices(pr, c);
+                    if (!have_x) load_x(pr, c);
                     if (t < 32 * nsl) {
-                        // table of block t of the chunk, per token (X read through L2: an
-                        // earlier phase of this launch wrote it)
-                        const uint2* xs = reinterpret_cast<const uint2*>(pr.X) + (c * kCChunk >> 2) + t;
 #pragma unroll
-                        for (int m = 0; m < MT; ++m)
-                            build_table(tabs + m * kCTok + t * kTab, __ldcg(xs + (int64_t)m * (pr.K >> 2)));
+                        for (int m = 0; m < MT; ++m) build_table(tb0 + m * kCTok + t * kTab, xn[m]);
                     }
+                    // the next chunk's activations load while this one is looked up: the next
+                    // chunk of this linear, or the first of the CTA's next segment in this phase
+                    // (its X is complete too)
+                    have_x = true;
+                    if (c + 1 < nc)
+                        load_x(pr, c + 1);
+                    else if (g + sg.n < e)
+                        load_x(P.p[seg_at(P, ph, g + sg.n, e).p], 0);
+                    else
+                        have_x = false;
                     if (!(ok = csync())) break;
 #pragma unroll
                     for (int i = 0; i < kCSeg; ++i) {
@@ -1349,17 +1393,17 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
                             if (w < nsl) {
                                 const uint32_t st = stages + s * kCStage;
                                 const uint4 wq = lds128(st + r * (16 * kCSl) + (((uint32_t)w ^ (uint32_t)(r & 7)) << 4));
-                                const uint32_t sq = lds32(st + kCIdx + 4 * (w * kCRows + r));
-                                const uint32_t tb = tabs + (uint32_t)(w * 32 * kTab);
+                                const uint32_t sq = lds32(st + kCIdx + r * kCPad + 4 * w);
+                                const uint32_t tb = tb0 + (uint32_t)(w * 32 * kTab);
                                 float p0[MT], p1[MT], q0[MT], q1[MT], r0[MT], r1[MT], u0[MT], u1[MT];
                                 word_sums<0, MT, kCTok>(wq.x, sq & 0xffu, tb, p0, p1);
                                 word_sums<8, MT, kCTok>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
                                 word_sums<16, MT, kCTok>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
                                 word_sums<24, MT, kCTok>(wq.w, sq >> 24, tb, u0, u1);
                                 float al = 1.0f;
-                                if (pr.mode == kSG128) al = __uint_as_float(lds32(st + kCIdx + kCSgn + 4 * (w * kCRows + r)));
+                                if (pr.mode == kSG128) al = __uint_as_float(lds32(st + kCIdx + kCSgn + r * kCPad + 4 * w));
                                 if (pr.mode == kSG256)
-                                    al = __uint_as_float(lds32(st + kCIdx + kCSgn + 4 * ((w >> 1) * kCRows + r)));
+                                    al = __uint_as_float(lds32(st + kCIdx + kCSgn + r * kCPad + 4 * (w >> 1)));
 #pragma unroll
                                 for (int m = 0; m < MT; ++m) {
                                     const float v =
@@ -1367,7 +1411,8 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
                                     acc[i][m] = pr.mode == kSRow ? acc[i][m] + v : fmaf(al, v, acc[i][m]);
                                 }
                             }
-                            mbar_arrive(empty(s));
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(empty(s));
                             ++k;
                         }
                     }
