@@ -268,12 +268,15 @@ float sherry_arenas_lambda(int64_t step, int64_t total, float lambda0);
  * computed as by sherry_linear (fp32 accumulation, alpha once per group), within
  * the fp32 summation-order bound of it.
  *   One to three tokens with every K % 512 == 0, or four tokens with every
- *   K % 256 == 0, and group 128 or 256 (or row scales): one cooperative launch (one CTA per SM, all resident) in which a
- *   grid-wide bounded barrier separates the phases and the packed weights of the
- *   next phase stream in while it resolves ("Sherry: ..." digest: inference
- *   streams the packed weights through lookup tables; the pages' layer is
- *   F.linear).  Otherwise: one sherry_linear_batched-style launch set per phase,
- *   ordered by the stream.
+ *   K % 256 == 0, and group 128 or 256 (or row scales): one cooperative launch
+ *   (one CTA per SM, all resident) in which a grid-wide bounded barrier
+ *   separates the phases and the packed weights of the next phase stream in
+ *   while it resolves ("Sherry: ..." digest: inference streams the packed
+ *   weights through lookup tables; the pages' layer is F.linear).  One and two
+ *   tokens give each CTA whole 32-row blocks over all of K (the K sum stays in
+ *   the CTA, in a fixed order); three and four tokens split row blocks over CTAs
+ *   as the batched launch does.  Otherwise: one sherry_linear_batched-style
+ *   launch set per phase, ordered by the stream.
  *   workspace  sherry_linear_chain_workspace_bytes(...) bytes; the same ticket
  *            contract as a linear workspace (first 256 KiB zero before the first
  *            use; every successful call leaves it zero). */

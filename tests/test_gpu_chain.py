@@ -117,25 +117,69 @@ def test_chain_vs_oracle_chain(sw, orc_omp, M, gran, group):
     assert int(ws[: 256 * 1024].view(torch.int32).abs().sum()) == 0   # tickets and phase counters left zero
 
 
-def test_chain_single_phase_matches_oracle_fp32(sw, orc):
+@pytest.mark.parametrize("M", [1, 2])
+def test_chain_single_phase_matches_oracle_fp32(sw, orc, M):
     """One phase of independent linears through the chained kernel: fp32 Y within the
-    gate and the fp32 accumulation bound of every element."""
+    gate and the fp32 accumulation bound of every element.  Ragged row counts (N not
+    a multiple of the 32-row blocks), K of one to several 2048-weight chunks with a
+    partial last chunk, every scale granularity; guard bytes around every Y stay
+    untouched."""
     import torch
-    from tests.gpu_common import check_linear
-    shapes = [(1000, 3072, "group", 128), (513, 2048, "channel", 0), (77, 1024, "group", 256), (2048, 512, "tensor", 0)]
-    ph, refs = [], []
+    from tests.gpu_common import canaried, canaries_intact, check_linear
+    shapes = [(1000, 3072, "group", 128), (513, 2048, "channel", 0), (77, 1024, "group", 256), (2048, 512, "tensor", 0),
+              (40, 5120, "group", 256)]
+    ph, refs, fulls = [], [], []
     for i, (N, K, gname, group) in enumerate(shapes):
         g = GRAN[gname]
         W = synth.weights_normal(N, K, 32000 + i)
-        Xb = synth.activations_bf16(1, K, 32500 + i)
+        Xb = synth.activations_bf16(M, K, 32500 + i)
         P = sw.quantize_pack(to_dev(W), g, group)
         idx, sgn, sc = packed_to_host(P)
         refs.append((orc.linear(Xb, idx, sgn, sc, N, K, g, group), orc.unpack_f32(idx, sgn, sc, N, K, g, group), Xb))
-        ph.append((to_dev(Xb.view(np.int16)).view(torch.bfloat16), P, torch.empty((1, N), device="cuda")))
+        full, Y = canaried((M, N), torch.float32)
+        fulls.append(full)
+        ph.append((to_dev(Xb.view(np.int16)).view(torch.bfloat16), P, Y))
     sw.linear_chain([ph], torch.float32)
     torch.cuda.synchronize()
-    for (X, P, Y), (y_ref, Wq, Xb) in zip(ph, refs):
+    assert sw.device_status() == 0
+    for (X, P, Y), (y_ref, Wq, Xb), full in zip(ph, refs, fulls):
         check_linear(Y.cpu().numpy(), y_ref, Xb, Wq)
+        assert canaries_intact(full)
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_chain_many_row_blocks_per_cta(sw, orc, M):
+    """Phases with more 32-row blocks than four per CTA (so a CTA walks several
+    segments of one linear, rebuilding its tables) and a linear boundary inside CTA
+    ranges; the second phase reads the first one's bf16 output.  Every output row
+    is compared (fp32 output of the last phase against the oracle's chain)."""
+    import torch
+    g = oracle.PER_GROUP
+    N1, K1 = 24576, 512            # 768 row blocks over the CTAs
+    N2a, N2b = 9000, 700           # the second phase: two linears reading Y1 (K = N1)
+    W1 = synth.weights_student_t(N1, K1, 35000)
+    W2a = synth.weights_student_t(N2a, N1 // 2, 35001)
+    W2b = synth.weights_student_t(N2b, N1 // 2, 35002)
+    P1 = sw.quantize_pack(to_dev(W1), g, 128)
+    P2a = sw.quantize_pack(to_dev(W2a), g, 128)
+    P2b = sw.quantize_pack(to_dev(W2b), g, 128)
+    Xb = synth.activations_bf16(M, K1, 35003)
+    X = to_dev(Xb.view(np.int16)).view(torch.bfloat16)
+    Y1 = torch.empty((M, N1), dtype=torch.bfloat16, device="cuda")
+    Y2a = torch.empty((M, N2a), dtype=torch.float32, device="cuda")
+    Y2b = torch.empty((M, N2b), dtype=torch.float32, device="cuda")
+    x2 = Y1.view(-1)[: M * (N1 // 2)].view(M, N1 // 2)
+    # one chain call needs one output dtype: bf16 for the first phase, fp32 written by a second call
+    sw.linear_chain([[(X, P1, Y1)]], torch.bfloat16)
+    sw.linear_chain([[(x2, P2a, Y2a), (x2, P2b, Y2b)]], torch.float32)
+    torch.cuda.synchronize()
+    assert sw.device_status() == 0
+    r1 = orc.linear(Xb, *packed_to_host(P1), N1, K1, g, 128)
+    assert gate(Y1.float().cpu().numpy(), r1) <= 1e-3 + 2.0 ** -8
+    x2b = _bits(Y1).reshape(-1)[: M * (N1 // 2)].reshape(M, N1 // 2)
+    for P, Y, N in ((P2a, Y2a, N2a), (P2b, Y2b, N2b)):
+        r = orc.linear(x2b, *packed_to_host(P), N, N1 // 2, g, 128)
+        assert gate(Y.cpu().numpy(), r) <= 1e-3
 
 
 def test_chain_fallback_routes(sw, orc):
