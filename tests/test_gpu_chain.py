@@ -218,3 +218,33 @@ def test_fused_layout_is_the_concatenation(sw, gran):
     for i in range(3):
         assert np.array_equal(got[i].reshape(-1).view(np.uint8),
                               np.concatenate([s[i].reshape(-1) for s in singles]).view(np.uint8))
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_chain_wait_timeout_reports_and_recovers(sw, orc_omp, M):
+    """A chained launch whose bounded waits (stage copies, the consumers' barriers,
+    the grid barrier between phases) are given a budget of a few clock cycles gives
+    up instead of hanging: the status is OK or SHERRY_ERR_TIMEOUT, the context stays
+    usable, and once the budget is back the same chain is correct again (the
+    binding drops the workspace whose phase counters an aborted launch left)."""
+    import torch
+    from sparse_ternary_weight_b200 import _abi
+    L = _abi.lib()
+    layers, d, f, nkv = 2, 1024, 2560, 256
+    packs, X0, phases = _build(sw, layers, d, f, nkv, "group", 128, M)
+    assert sw.device_status() == 0
+    prev = L.sherry_set_wait_budget(2)
+    try:
+        for _ in range(3):
+            sw.linear_chain(phases, torch.bfloat16)
+        torch.cuda.synchronize()
+        st = sw.device_status()
+    finally:
+        L.sherry_set_wait_budget(prev)
+    assert st in (_abi.OK, _abi.ERR_TIMEOUT)
+    sw.linear_chain(phases, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert sw.device_status() == 0
+    refs = _oracle_chain(orc_omp, packs, X0, M, d, f, "group", 128)
+    for i, (ph, y_ref) in enumerate(zip(phases, refs)):
+        assert gate(ph[0][2].float().cpu().numpy(), y_ref) <= 1e-3 + 2.0 ** -8, i
