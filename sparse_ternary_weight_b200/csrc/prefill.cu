@@ -51,18 +51,24 @@ constexpr int kPBN = 128;     // tokens per tile
 constexpr int kPBK = 64;      // K per MMA step
 constexpr int kPChunkSteps = 4;                  // steps per chunk
 constexpr int kPStepB = kPBN * kPBK * 2;         // 16 KB of X per step
-constexpr int kPChunkB = kPChunkSteps * kPStepB; // 64 KB of X per chunk
 constexpr int kPXSlots = 3;                      // X chunks in flight
-constexpr int kPTable = 256;                     // 32 weight patterns: low words (128 B), then high words
+constexpr int kPABuf = 2;                        // A buffers (chunks) in TMEM
 constexpr int kPRing = 2;                        // chunks of packed words in flight per decode thread
-constexpr int kPSmem = kPXSlots * kPChunkB + kPTable + 1024;
+constexpr int kPArnSteps = 2, kPArnSlots = 3;    // Arenas: steps per chunk, slots (X and W tiles)
+constexpr int kPXBytes = kPXSlots * kPChunkSteps * kPStepB > kPArnSlots * 2 * kPArnSteps * kPStepB
+                             ? kPXSlots * kPChunkSteps * kPStepB
+                             : kPArnSlots * 2 * kPArnSteps * kPStepB;  // the slots of either form
+constexpr int kPTable = 256;                     // 32 weight patterns: low words (128 B), then high words
+constexpr int kPSmem = kPXBytes + kPTable + 1024;
 constexpr int kPAcc = 2;                         // group accumulators in flight
-constexpr int kPTmemCols = 512;                  // 2 x 128 accumulator columns + 2 x 4 x 32 A columns
+constexpr int kPTmemCols = 512;                  // 2 x 128 accumulator columns + the A buffers
 constexpr int kPAcol = kPAcc * kPBN;             // first TMEM column of the A stages (256)
 constexpr int kPAcols = kPBK / 2;                // 32 columns (64 bf16) per A stage
 constexpr long long kPWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
-static_assert(kPAcol + 2 * kPChunkSteps * kPAcols <= kPTmemCols, "TMEM plan");
-static_assert(kPXSlots >= 3, "the decode's A-buffer wait reads the slot barrier of chunk cc - 2");
+constexpr int kPMaxSlots = kPXSlots > kPArnSlots ? kPXSlots : kPArnSlots;
+constexpr int kPMaxABuf = kPABuf > 2 ? kPABuf : 2;
+static_assert(kPAcol + kPABuf * kPChunkSteps * kPAcols <= kPTmemCols, "TMEM plan");
+static_assert(kPXSlots >= kPABuf + 1, "the decode's A-buffer wait reads the slot barrier of chunk cc - kPABuf");
 
 __device__ int g_device_status = 0;
 
@@ -221,27 +227,31 @@ __global__ void __launch_bounds__(PRoles<EPI>::kThreads, 1)
 k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
           const __grid_constant__ PParams P) {
     constexpr int kPTmaWarp = PRoles<EPI>::kTmaWarp, kPMmaWarp = PRoles<EPI>::kMmaWarp;
-    constexpr int CS = ARN ? 2 : kPChunkSteps;      // K-steps per chunk
+    constexpr int CS = ARN ? kPArnSteps : kPChunkSteps;   // K-steps per chunk
+    constexpr int XS = ARN ? kPArnSlots : kPXSlots;       // chunk slots
+    constexpr int AB = ARN ? 2 : kPABuf;                  // A buffers
+    constexpr int SLOTB = (ARN ? 2 : 1) * CS * kPStepB;   // bytes per slot (ARN: X, then W tiles)
     constexpr int SPG = CS / kPDecGroups;           // steps each decode group expands per chunk
     constexpr int kWOff = CS * kPStepB;             // W tiles after the X tiles of a slot (ARN)
-    constexpr int kDenseCol = kPAcol + 2 * CS * kPAcols;  // dense accumulator (ARN)
-    static_assert(!ARN || (kWOff + CS * kPStepB <= kPChunkB && kDenseCol + kPBN <= kPTmemCols), "Arenas plan");
+    constexpr int kDenseCol = kPAcol + AB * CS * kPAcols;  // dense accumulator (ARN)
+    static_assert(!ARN || kDenseCol + kPBN <= kPTmemCols, "Arenas plan");
+    static_assert(XS * SLOTB <= kPXBytes && XS >= AB + 1 && SLOTB % 1024 == 0, "slot plan");
     extern __shared__ __align__(1024) unsigned char psmem[];
-    __shared__ uint64_t bars[2 * kPXSlots + 2 + 2 * kPAcc + 3];
+    __shared__ uint64_t bars[2 * kPMaxSlots + kPMaxABuf + 2 * kPAcc + 3];
     __shared__ uint32_t tmem_base_s;
     __shared__ volatile int abort_s;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t base = (smem_u32(psmem) + 1023u) & ~1023u;
-    const uint32_t stX = base;                               // kPXSlots x 64 KB, 1024-aligned
-    const uint32_t table = base + kPXSlots * kPChunkB;       // 256-aligned
+    const uint32_t stX = base;                               // XS slots of SLOTB bytes, 1024-aligned
+    const uint32_t table = base + kPXBytes;                  // 256-aligned
     const uint32_t bar0 = smem_u32(&bars[0]);
     auto full_x = [&](int c) { return bar0 + 8u * c; };                    // X (and W) chunk in slot c landed
-    auto chunk_empty = [&](int c) { return bar0 + 8u * (kPXSlots + c); };  // MMAs of slot c's chunk done
-    auto full_a = [&](int h) { return bar0 + 8u * (2 * kPXSlots + h); };   // A buffer h written
-    auto acc_full = [&](int b) { return bar0 + 8u * (2 * kPXSlots + 2 + b); };
-    auto acc_empty = [&](int b) { return bar0 + 8u * (2 * kPXSlots + 2 + kPAcc + b); };
-    const uint32_t drain = bar0 + 8u * (2 * kPXSlots + 2 + 2 * kPAcc);  // the MMA thread's last commit
+    auto chunk_empty = [&](int c) { return bar0 + 8u * (XS + c); };  // MMAs of slot c's chunk done
+    auto full_a = [&](int h) { return bar0 + 8u * (2 * XS + h); };   // A buffer h written
+    auto acc_full = [&](int b) { return bar0 + 8u * (2 * XS + AB + b); };
+    auto acc_empty = [&](int b) { return bar0 + 8u * (2 * XS + AB + kPAcc + b); };
+    const uint32_t drain = bar0 + 8u * (2 * XS + AB + 2 * kPAcc);  // the MMA thread's last commit
     const uint32_t dense_full = drain + 8u;    // ARN: a tile's dense product is complete
     const uint32_t dense_empty = drain + 16u;  // ARN: the epilogue has read it
 
@@ -256,11 +266,11 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
 
     if (threadIdx.x == 0) {
         abort_s = 0;
-        for (int c = 0; c < kPXSlots; ++c) {
+        for (int c = 0; c < XS; ++c) {
             mbar_init(full_x(c), 1);
             mbar_init(chunk_empty(c), 1);
         }
-        for (int h = 0; h < 2; ++h) mbar_init(full_a(h), 128 * kPDecGroups);
+        for (int h = 0; h < AB; ++h) mbar_init(full_a(h), 128 * kPDecGroups);
         for (int b = 0; b < kPAcc; ++b) {
             mbar_init(acc_full(b), 1);
             mbar_init(acc_empty(b), 32 * EPI);
@@ -372,7 +382,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
         }
     } else if (warp < kPTmaWarp) {
         // ---------------- decode: TMEM lane (= tile row) i per thread; group g expands
-        // steps SPG*g .. SPG*g + SPG-1 of every chunk into A buffer (cc & 1) ----------------
+        // steps SPG*g .. SPG*g + SPG-1 of every chunk into A buffer (cc % AB) ----------------
         const int g = (warp - EPI) >> 2, q = warp & 3;
         const int i = q * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)kPAcol;
@@ -408,7 +418,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
                     uint2 w[2] = {rw[r][0], rw[r][1]};
                     uint32_t sb[2] = {rs[r][0], rs[r][1]};
                     fetch(ch + kPRing, rw[r], rs[r]);
-                    const int hbuf = cc & 1;
+                    const int hbuf = cc % AB;
 #pragma unroll
                     for (int e = 0; e < SPG; ++e) {
                         const int st = SPG * g + e;
@@ -427,10 +437,10 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
                                 asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(v[16 * h + 2 * j + 1]) : "r"(a));
                             }
                         }
-                        // A buffer hbuf was last read by the MMAs of chunk cc - 2, whose
+                        // A buffer hbuf was last read by the MMAs of chunk cc - AB, whose
                         // completion the MMA thread commits to that chunk's slot barrier
-                        if (e == 0 && cc >= 2) {
-                            if (!mbar_wait(chunk_empty((cc - 2) % kPXSlots), (uint32_t)(((cc - 2) / kPXSlots) & 1),
+                        if (e == 0 && cc >= AB) {
+                            if (!mbar_wait(chunk_empty((cc - AB) % XS), (uint32_t)(((cc - AB) / XS) & 1),
                                            &abort_s)) {
                                 ok = false;
                                 break;
@@ -452,7 +462,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
         if (lane == 0) {
             int c = 0;
             uint32_t cph = 0;  // phase parity of slot c's use
-            int issued[kPXSlots] = {};  // chunks loaded into each slot (phases of full_x)
+            int issued[XS] = {};  // chunks loaded into each slot (phases of full_x)
             bool ok = true;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const int m0 = (t / ntn) * kPBN;
@@ -465,18 +475,18 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
                     const int steps = min(CS, nk - ch * CS);
                     mbar_expect_tx(full_x(c), (uint32_t)(steps * kPStepB * (ARN ? 2 : 1)));
                     for (int st = 0; st < steps; ++st) {
-                        tma_load_2d(stX + c * kPChunkB + st * kPStepB, &xmap, (ch * CS + st) * kPBK, m0, full_x(c));
+                        tma_load_2d(stX + c * SLOTB + st * kPStepB, &xmap, (ch * CS + st) * kPBK, m0, full_x(c));
                         if constexpr (ARN)
-                            tma_load_2d(stX + c * kPChunkB + kWOff + st * kPStepB, &wmap, (ch * CS + st) * kPBK, n0,
+                            tma_load_2d(stX + c * SLOTB + kWOff + st * kPStepB, &wmap, (ch * CS + st) * kPBK, n0,
                                         full_x(c));
                     }
                     ++issued[c];
-                    if (++c == kPXSlots) { c = 0; cph ^= 1u; }
+                    if (++c == XS) { c = 0; cph ^= 1u; }
                 }
             }
             // every load issued must land before the CTA's shared memory goes away
             // (after an abort the MMA thread may not have waited for the last ones)
-            for (int s = 0; s < kPXSlots; ++s)
+            for (int s = 0; s < XS; ++s)
                 if (issued[s] > 0) mbar_drain(full_x(s), (uint32_t)((issued[s] - 1) & 1));
         }
     } else {
@@ -527,12 +537,12 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 int gleft = gs;  // steps left in the current group
                 for (int ch = 0; ch < nchunks; ++ch, ++cc) {
-                    const int hbuf = cc & 1;
-                    if (!mbar_wait(full_a(hbuf), (uint32_t)((cc >> 1) & 1), &abort_s)) { ok = false; break; }
+                    const int hbuf = cc % AB;
+                    if (!mbar_wait(full_a(hbuf), (uint32_t)((cc / AB) & 1), &abort_s)) { ok = false; break; }
                     if (!mbar_wait(full_x(c), cph, &abort_s)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t db0 = smem_desc(stX + c * kPChunkB);
-                    const uint64_t dw0 = smem_desc(stX + c * kPChunkB + kWOff);
+                    const uint64_t db0 = smem_desc(stX + c * SLOTB);
+                    const uint64_t dw0 = smem_desc(stX + c * SLOTB + kWOff);
                     const uint32_t ta0 = tmem + (uint32_t)(kPAcol + hbuf * CS * kPAcols);
                     const int steps = min(CS, nk - ch * CS);
                     if (steps == CS) {
@@ -553,7 +563,7 @@ k_prefill(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
                     }
                     if (!ok) break;
                     mma_commit(chunk_empty(c));
-                    if (++c == kPXSlots) { c = 0; cph ^= 1u; }
+                    if (++c == XS) { c = 0; cph ^= 1u; }
                 }
             }
             // all MMAs this thread issued complete before TMEM is freed (after an abort
