@@ -198,8 +198,8 @@ size_t sherry_quantize_pack_batched_workspace_bytes(const sherry_quantize_desc* 
  *   workspace  sherry_workspace_bytes(SHERRY_OP_LINEAR, M, N, K, g, group) bytes
  * fp32 accumulation; alpha applied once per group (or row).  Kernels:
  * M <= 16 with K % 512 == 0 (group 128 or 256, per-channel or per-tensor) a
- * warp-specialised streaming kernel (lookup tables for M <= 3, tensor-core
- * consumers from M = 4); other 2 <= M <= 8 with
+ * warp-specialised streaming kernel (lookup tables for M <= 2, tensor-core
+ * consumers from M = 3); other 2 <= M <= 8 with
  * K % 128 == 0 a warp-level tensor-core (mma.sync) kernel; 9 <= M <= 32 with K % 256 == 0 and
  * (per-group) group % 64 == 0 a tensor-core (tcgen05) kernel for few tokens;
  * M >= 17 with K % 64 == 0 and group % 64 == 0 the tcgen05 prefill kernel;

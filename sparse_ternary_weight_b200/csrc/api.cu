@@ -81,9 +81,9 @@ static int check_planes(const uint32_t* idx, const uint8_t* sgn, const float* sc
     return SHERRY_OK;
 }
 
-// Which kernel computes each problem of a call.  Problems with one to four tokens
+// Which kernel computes each problem of a call.  Problems with one or two tokens
 // that fit the streaming lookup-table kernel share one launch of it, problems with
-// five to sixteen tokens of the same shapes one launch of its tensor-core form
+// three to sixteen tokens of the same shapes one launch of its tensor-core form
 // (unless their row blocks would outnumber its tickets); 2 <= M <= 8 problems with K % 128 == 0
 // share one launch of the warp-MMA kernel; other problems with up to 32 tokens
 // that fit the tcgen05 few-token kernel share one launch of it; each problem with

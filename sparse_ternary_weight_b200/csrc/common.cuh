@@ -193,7 +193,7 @@ int skinny_linear_launch(const ProbShape* shapes, const sherry_linear_desc* desc
                          int sms, cudaStream_t stream);
 // one- and two-token streaming kernel (gemv_stream.cu)
 bool stream_eligible(const ProbShape& s, int64_t M);
-bool mstream_eligible(const ProbShape& s, int64_t M);  // 5..16 tokens, tensor-core consumers
+bool mstream_eligible(const ProbShape& s, int64_t M);  // 3..16 tokens, tensor-core consumers
 int mstream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                           void* workspace, int sms, cudaStream_t stream);
 int64_t stream_tiles(const ProbShape& s);  // row blocks (tickets) of one problem

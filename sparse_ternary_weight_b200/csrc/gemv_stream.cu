@@ -1,5 +1,5 @@
 // gemv_stream.cu -- packed 3:4 ternary linear for 1 to 16 tokens, streamed from
-// HBM: the lookup-table decode for up to three tokens (the method's inference
+// HBM: the lookup-table decode for one and two tokens (the method's inference
 // scheme: tables built from the activations, looked up by the packed weights,
 // accumulated, then scaled; "Sherry: Hardware-Efficient 1.25-Bit Ternary
 // Quantization via Fine-grained Sparsification", digest paragraph on inference;
@@ -7,10 +7,10 @@
 //
 // Work unit: 512 output rows x 32 W weights (W packed words) of one linear: W =
 // 16 for independent linears (one batched launch per decode step) and for
-// chained phases of up to three tokens, W = 8 for a four-token chain (whose
-// tables take more shared memory).  From four tokens on, independent linears
-// take the tensor-core consumers (k_mma_stream, further below) on the same
-// pipeline.
+// chained phases of three tokens, W = 8 for a four-token chain (whose tables
+// take more shared memory; one- and two-token chains run on whole-K row blocks,
+// k_lut_rows, further below).  From three tokens on, independent linears take
+// the tensor-core consumers (k_mma_stream, further below) on the same pipeline.
 // All units of a phase (one or many independent linears) are split into equal
 // contiguous ranges, one per CTA (stream-K): every CTA streams the same number
 // of bytes.  A row block whose units straddle CTAs is finished by the CTA that
@@ -1480,12 +1480,12 @@ static bool stream_eligible_w(const ProbShape& s, int64_t M) {
     return M >= 1 && M <= (W == 16 ? 3 : 4) && stream_shape_ok<W>(s);
 }
 
-// one to three tokens: lookup tables on 16-word units (the four-token lookup form,
-// on 8-word units, serves the chained launches; independent linears of four or
-// more tokens go to the tensor-core consumers)
-bool stream_eligible(const ProbShape& s, int64_t M) { return M <= 3 && stream_eligible_w<16>(s, M); }
-// four to sixteen tokens: the tensor-core consumers on 16-word units
-bool mstream_eligible(const ProbShape& s, int64_t M) { return M >= 4 && M <= 16 && stream_shape_ok<16>(s); }
+// one and two tokens: lookup tables on 16-word units (the three- and four-token
+// lookup forms serve the chained launches; independent linears of three or more
+// tokens go to the tensor-core consumers, which expand each block once)
+bool stream_eligible(const ProbShape& s, int64_t M) { return M <= 2 && stream_eligible_w<16>(s, M); }
+// three to sixteen tokens: the tensor-core consumers on 16-word units
+bool mstream_eligible(const ProbShape& s, int64_t M) { return M >= 3 && M <= 16 && stream_shape_ok<16>(s); }
 bool chain_eligible(const ProbShape& s, int64_t M) {
     return M <= 3 ? stream_eligible_w<16>(s, M) : stream_eligible_w<8>(s, M);
 }
@@ -1676,7 +1676,7 @@ static int mstream_launch_nt(SPlan& pl, int count, int64_t M, int y_bf16, void* 
 
 int mstream_linear_launch(const ProbShape* shapes, const sherry_linear_desc* descs, int count, int64_t M, int y_bf16,
                           void* workspace, int sms, cudaStream_t stream) {
-    if (M < 4 || M > 16) return SHERRY_ERR_UNSUPPORTED;
+    if (M < 1 || M > 16) return SHERRY_ERR_UNSUPPORTED;
     SPlan pl = make_splan(shapes, count, nullptr, 1, M, sms, 16);
     attach(pl, descs, count);
     if (pl.total_units == 0) return SHERRY_OK;
