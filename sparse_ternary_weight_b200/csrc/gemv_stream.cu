@@ -176,6 +176,32 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         }
     }
 }
+// As mbar_wait, but each check may suspend the thread in hardware (up to ~10 us)
+// until the phase completes instead of returning at once: a waiting warp then
+// takes no issue slots from the warps that still work.
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(10000u)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                long long budget) {
+    if (mbar_try_sleep(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_sleep(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > budget) {
+            *abort_flag = 1;
+            atomicExch(&g_stream_status, SHERRY_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
 // wait until the shared phase counter reaches `target`; false on timeout or abort
 __device__ __forceinline__ bool gate_wait(const int* gate, int target, volatile int* abort_flag, long long budget) {
     const volatile int* g = gate;
@@ -1297,7 +1323,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
                 for (int c = 0; c < nc && ok; ++c)
                     for (int i = 0; i < sg.n; ++i, ++j) {
                         const int s = j % S;
-                        if (j >= S && !mbar_wait(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag, P.wait_cycles)) {
+                        if (j >= S && !mbar_wait_sleep(empty(s), (uint32_t)(((j / S) & 1) ^ 1), abort_flag, P.wait_cycles)) {
                             ok = false;
                             break;
                         }
@@ -1320,7 +1346,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
         auto csync = [&]() -> bool {
             __syncwarp();
             if (lane == 0) mbar_arrive(cb);
-            const bool fine = mbar_wait(cb, (uint32_t)(nb & 1), abort_flag, P.wait_cycles);
+            const bool fine = mbar_wait_sleep(cb, (uint32_t)(nb & 1), abort_flag, P.wait_cycles);
             ++nb;
             return fine;
         };
@@ -1389,7 +1415,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
                     for (int i = 0; i < kCSeg; ++i) {
                         if (i < sg.n) {
                             const int s = k % S;
-                            if (!(ok = mbar_wait(ready(s), (uint32_t)((k / S) & 1), abort_flag, P.wait_cycles))) break;
+                            if (!(ok = mbar_wait_sleep(ready(s), (uint32_t)((k / S) & 1), abort_flag, P.wait_cycles))) break;
                             if (w < nsl) {
                                 const uint32_t st = stages + s * kCStage;
                                 const uint4 wq = lds128(st + r * (16 * kCSl) + (((uint32_t)w ^ (uint32_t)(r & 7)) << 4));
