@@ -594,7 +594,8 @@ def dependent_rows(args, ws, dev, pk, steps, warm):
         assert sw.device_status(dev) == 0
         out[f"M{M}"] = {"GB/s": round(ws * b / (ms * 1e-3) / 1e9, 1), "tok_per_s": round(ws * M / (ms * 1e-3), 1),
                         "ms_per_step": round(ms, 4), "frac_hbm": round(b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-                        "bytes": b, "phases": len(phases), "launches": 1,
+                        "bytes": b, "phases": len(phases), "us_per_phase": round(ms * 1e3 / len(phases), 2),
+                        "launches": 1,
                         "call": "sherry_linear_chain: 28 layers x (fused q/k/v, o, fused gate/up, down), "
                                 "each phase reading the previous one's bf16 output"}
         del phases, flat, descs
