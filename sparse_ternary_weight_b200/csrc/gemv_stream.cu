@@ -1160,7 +1160,10 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
 // into a ring of stages; they run ahead across phases, since weights do not
 // depend on X.  Each phase's items are split into contiguous, balanced ranges over
 // the CTAs; a CTA arrives at the phase counter after its Y stores (release) and
-// waits for the previous phase's count before reading its X (acquire).
+// waits for the previous phase's count before reading its X (acquire).  One-token
+// tables are double-buffered (no barrier before a build), the next chunk's X is
+// loaded during the current chunk's lookups, and waiting warps suspend on their
+// mbarrier instead of polling, so they leave the issue slots to the working ones.
 constexpr int kCRows = 32;                      // rows per item: one per lane
 constexpr int kCSl = kSConsumers;               // 128-weight slices per chunk: one per consumer warp
 constexpr int kCChunk = 128 * kCSl;             // weights per chunk
