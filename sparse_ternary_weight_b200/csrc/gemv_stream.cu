@@ -1151,43 +1151,46 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
 // CTA instead.  Item = 32 rows of one linear over all of K: lane = row, and the 16
 // consumer warps split K into 128-weight slices (one packed 16-byte chunk, one
 // group-128 scale), so the K reduction stays inside the CTA (a fixed-order sum
-// over the warps in shared memory).  K runs in chunks of 2048 weights (16 slices):
-// per chunk the consumers build the chunk's 512 tables per token (one per thread)
-// and then look up every item of the CTA's current segment (up to kCSeg items of
-// one linear), so the tables are built once per segment, not per item.  Four
+// over the warps in shared memory).  K runs in chunks of 24 slices (3072 weights)
+// for one token and 16 slices for two (their tables take twice the space): per
+// chunk the consumers build the chunk's tables (one or two per thread and token;
+// a warp takes slices w and w + 16) and then look up every item of the CTA's
+// current segment (up to kCSeg items of one linear), so the tables are built once
+// per segment, not per item, and a K of 3072 is one chunk.  Four
 // helper warps copy the items' packed words (row-major, XOR-swizzled 16-byte
 // chunks), sign words and scales (rows padded to 80 bytes) with 16-byte copies
 // into a ring of stages; they run ahead across phases, since weights do not
 // depend on X.  Each phase's items are split into contiguous, balanced ranges over
 // the CTAs; a CTA arrives at the phase counter after its Y stores (release) and
-// waits for the previous phase's count before reading its X (acquire).  One-token
-// tables are double-buffered (no barrier before a build), the next chunk's X is
-// loaded during the current chunk's lookups, and waiting warps suspend on their
-// mbarrier instead of polling, so they leave the issue slots to the working ones.
+// waits for the previous phase's count before reading its X (acquire).  The next
+// chunk's X is loaded during the current chunk's lookups, and waiting warps suspend
+// on their mbarrier instead of polling, so they leave the issue slots to the
+// working ones.
 constexpr int kCRows = 32;                      // rows per item: one per lane
-constexpr int kCSl = kSConsumers;               // 128-weight slices per chunk: one per consumer warp
-constexpr int kCChunk = 128 * kCSl;             // weights per chunk
-constexpr int kCBlocks = kCChunk / 4;           // tables per chunk and token: one per consumer thread
-constexpr int kCIdx = kCRows * kCSl * 16;       // packed words of a stage: [row][slice] 16-byte chunks
-constexpr int kCPad = 4 * kCSl + 16;            // bytes per row of sign words or scales (one per slice, padded)
-constexpr int kCSgn = kCRows * kCPad;           // sign words: 4 sign bytes per slice
-constexpr int kCSc = kCRows * kCPad;            // scales: one per slice (group 128) or per two (group 256)
-constexpr int kCStage = kCIdx + kCSgn + kCSc;   // 13 KB
-constexpr int kCTok = kCBlocks * kTab;          // one token's tables of a chunk
 constexpr int kCSeg = 4;                        // items of one linear sharing the tables
 constexpr int kCStages = 4;
-static_assert(kCBlocks == 32 * kSConsumers, "one table per consumer thread");
-static_assert(kCTok % 256 == 0 && (32 * kTab) % 256 == 0, "256-aligned table bases");
-static_assert(kCStage % 16 == 0 && kCIdx % 16 == 0 && kCPad % 16 == 0, "16-byte aligned copies");
 
+// Chunk geometry and shared memory for MT tokens.
 template <int MT>
 struct CCfg {
-    static constexpr int kTB = MT == 1 ? 2 : 1;                     // table buffers (two fit for one token)
-    static constexpr int kStages = kTB * MT * kCTok;                // after the tables
-    static constexpr int kRed = kStages + kCStages * kCStage;       // [warp][item][token][row] partials
+    static constexpr int kSl = MT == 1 ? 24 : 16;        // 128-weight slices per chunk (warp w: w, w + 16)
+    static constexpr int kChunk = 128 * kSl;              // weights per chunk
+    static constexpr int kBlocks = kChunk / 4;            // tables per chunk and token
+    static constexpr int kTPT = (kBlocks + kSRows - 1) / kSRows;  // tables per consumer thread
+    static constexpr int kIdx = kCRows * kSl * 16;        // packed words of a stage: [row][slice] 16-byte chunks
+    static constexpr int kPad = 4 * kSl + 16;             // bytes per row of sign words or scales (padded)
+    static constexpr int kSgn = kCRows * kPad;            // sign words: 4 sign bytes per slice
+    static constexpr int kSc = kCRows * kPad;             // scales: one per slice (group 128) or per two (256)
+    static constexpr int kStage = kIdx + kSgn + kSc;
+    static constexpr int kTok = kBlocks * kTab;           // one token's tables of a chunk
+    static constexpr int kStages = MT * kTok;             // after the tables
+    static constexpr int kRed = kStages + kCStages * kStage;  // [warp][item][token][row] partials
     static constexpr int kBars = kRed + kSConsumers * kCSeg * MT * kCRows * 4;
     static constexpr int kSmem = 256 + kBars + 8 * (2 * kCStages + 1);
     static_assert(kSmem <= 232448, "shared memory per CTA");
+    static_assert(kSl % 8 == 0 && kSl <= 2 * kSConsumers, "whole swizzle groups; at most two slices per warp");
+    static_assert(kTok % 256 == 0 && (32 * kTab) % 256 == 0, "256-aligned table bases");
+    static_assert(kStage % 16 == 0 && kIdx % 16 == 0 && kPad % 16 == 0, "16-byte aligned copies");
 };
 
 struct CProb {
@@ -1238,43 +1241,48 @@ __device__ __forceinline__ void cta_items(const CParams<MAXP>& P, int ph, int& b
     e = b0 + (int)(n * (blockIdx.x + 1) / gridDim.x);
 }
 
-__device__ __forceinline__ int chunk_slices(const CProb& pr, int c) { return min(kCSl, (pr.K - c * kCChunk) >> 7); }
+template <int MT>
+__device__ __forceinline__ int chunk_slices(const CProb& pr, int c) {
+    return min(CCfg<MT>::kSl, (pr.K - c * CCfg<MT>::kChunk) >> 7);
+}
 
 // Copy item `it`, chunk c of problem pr into the stage at st (128 helper threads,
 // ht = 0..127); rows past N are not copied (their results are never stored).
+template <int MT>
 __device__ __forceinline__ void copy_item(const CProb& pr, int it, int c, uint32_t st, int ht) {
+    using C = CCfg<MT>;
     const int row0 = it * kCRows;
     const int rows = min(kCRows, pr.N - row0);
-    const int nsl = chunk_slices(pr, c);
-    const char* ib = reinterpret_cast<const char*>(pr.idx) + (int64_t)row0 * (pr.K >> 3) + (c * kCChunk >> 3);
+    const int nsl = chunk_slices<MT>(pr, c);
+    const char* ib = reinterpret_cast<const char*>(pr.idx) + (int64_t)row0 * (pr.K >> 3) + (c * C::kChunk >> 3);
     for (int i = ht; i < rows * nsl; i += kSHelperThreads) {
         const int r = i / nsl, q = i - r * nsl;
-        cp_async16(st + r * (16 * kCSl) + ((q ^ (r & 7)) << 4), ib + (int64_t)r * (pr.K >> 3) + 16 * q);
+        cp_async16(st + r * (16 * C::kSl) + ((q ^ (r & 7)) << 4), ib + (int64_t)r * (pr.K >> 3) + 16 * q);
     }
     // sign words: 4 * nsl bytes per row, whole 16-byte pieces (nsl is a multiple of 4)
-    const char* sb = reinterpret_cast<const char*>(pr.sgn) + (int64_t)row0 * (pr.K >> 5) + (c * kCChunk >> 5);
+    const char* sb = reinterpret_cast<const char*>(pr.sgn) + (int64_t)row0 * (pr.K >> 5) + (c * C::kChunk >> 5);
     const int sp = nsl >> 2;
     for (int i = ht; i < rows * sp; i += kSHelperThreads) {
         const int r = i / sp, q = i - r * sp;
-        cp_async16(st + kCIdx + r * kCPad + 16 * q, sb + (int64_t)r * (pr.K >> 5) + 16 * q);
+        cp_async16(st + C::kIdx + r * C::kPad + 16 * q, sb + (int64_t)r * (pr.K >> 5) + 16 * q);
     }
     if (pr.mode != kSRow) {
         // group 128: nsl scales per row (16-byte pieces); group 256: nsl / 2 (8-byte pieces)
         const int bytes = pr.mode == kSG128 ? 4 * nsl : 2 * nsl;
         const char* cb = reinterpret_cast<const char*>(pr.scales + (int64_t)row0 * pr.spr) +
-                         (pr.mode == kSG128 ? 4 * c * kCSl : 2 * c * kCSl);
-        const uint32_t sc = st + kCIdx + kCSgn;
+                         (pr.mode == kSG128 ? 4 * c * C::kSl : 2 * c * C::kSl);
+        const uint32_t sc = st + C::kIdx + C::kSgn;
         if (pr.mode == kSG128) {
             const int np = bytes >> 4;
             for (int i = ht; i < rows * np; i += kSHelperThreads) {
                 const int r = i / np, q = i - r * np;
-                cp_async16(sc + r * kCPad + 16 * q, cb + (int64_t)r * 4 * pr.spr + 16 * q);
+                cp_async16(sc + r * C::kPad + 16 * q, cb + (int64_t)r * 4 * pr.spr + 16 * q);
             }
         } else {
             const int np = bytes >> 3;
             for (int i = ht; i < rows * np; i += kSHelperThreads) {
                 const int r = i / np, q = i - r * np;
-                cp_async8(sc + r * kCPad + 8 * q, cb + (int64_t)r * 4 * pr.spr + 8 * q);
+                cp_async8(sc + r * C::kPad + 8 * q, cb + (int64_t)r * 4 * pr.spr + 8 * q);
             }
         }
     }
@@ -1289,7 +1297,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
     using C = CCfg<MT>;
     constexpr int S = kCStages;
     __shared__ int s_abort;
-    const uint32_t tabs = (smem_u32(g_smem) + 255u) & ~255u;  // [buffer][token][kCBlocks tables]
+    const uint32_t tabs = (smem_u32(g_smem) + 255u) & ~255u;  // [token][C::kBlocks tables]
     const uint32_t stages = tabs + C::kStages;
     const uint32_t red = tabs + C::kRed;
     const uint32_t bars = tabs + C::kBars;
@@ -1322,7 +1330,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
             for (int g = b; g < e && ok;) {
                 const CSeg sg = seg_at(P, ph, g, e);
                 const CProb& pr = P.p[sg.p];
-                const int nc = (pr.K + kCChunk - 1) / kCChunk;
+                const int nc = (pr.K + C::kChunk - 1) / C::kChunk;
                 for (int c = 0; c < nc && ok; ++c)
                     for (int i = 0; i < sg.n; ++i, ++j) {
                         const int s = j % S;
@@ -1330,7 +1338,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
                             ok = false;
                             break;
                         }
-                        copy_item(pr, sg.it + i, c, stages + s * kCStage, ht);
+                        copy_item<MT>(pr, sg.it + i, c, stages + s * C::kStage, ht);
                         cp_async_arrive(ready(s));
                     }
                 g += sg.n;
@@ -1338,11 +1346,11 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else {
-        // ---- consumers: lane = row of the item, warp = 128-weight slice of the chunk
+        // ---- consumers: lane = row of the item, warp w = 128-weight slices w and w + 16
+        // of the chunk
         const int w = warp, r = lane;
         int k = 0;   // stages consumed
         int nb = 0;  // consumer barriers passed
-        int nt = 0;  // chunks whose tables were built
         bool ok = true;
         // a barrier of the 16 consumer warps: each warp's lanes meet first, then lane 0
         // arrives for the warp (its release covers the lanes' shared-memory writes)
@@ -1354,15 +1362,18 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
             return fine;
         };
         float acc[kCSeg][MT];
-        uint2 xn[MT];  // this thread's block of the next chunk's activations, per token
-        // activations of block t of chunk c (read through L2: an earlier phase of this
-        // launch wrote them)
+        uint2 xn[C::kTPT][MT];  // this thread's blocks of the next chunk's activations, per token
+        // activations of blocks t and t + 512 of chunk c (read through L2: an earlier
+        // phase of this launch wrote them)
         auto load_x = [&](const CProb& px, int c) {
-            const uint2* xs = reinterpret_cast<const uint2*>(px.X) + (c * kCChunk >> 2) + t;
-            if (t < 32 * chunk_slices(px, c)) {
+            const uint2* xs = reinterpret_cast<const uint2*>(px.X) + (c * C::kChunk >> 2) + t;
+            const int nb4 = 32 * chunk_slices<MT>(px, c);
 #pragma unroll
-                for (int m = 0; m < MT; ++m) xn[m] = __ldcg(xs + (int64_t)m * (px.K >> 2));
-            }
+            for (int u = 0; u < C::kTPT; ++u)
+                if (t + kSRows * u < nb4) {
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) xn[u][m] = __ldcg(xs + kSRows * u + (int64_t)m * (px.K >> 2));
+                }
         };
         for (int ph = 0; ph < P.n_phases && ok; ++ph) {
             int b, e;
@@ -1372,13 +1383,12 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
             for (int g = b; g < e && ok;) {
                 const CSeg sg = seg_at(P, ph, g, e);
                 const CProb& pr = P.p[sg.p];
-                const int nc = (pr.K + kCChunk - 1) / kCChunk;
+                const int nc = (pr.K + C::kChunk - 1) / C::kChunk;
 #pragma unroll
                 for (int i = 0; i < kCSeg; ++i)
 #pragma unroll
                     for (int m = 0; m < MT; ++m) acc[i][m] = 0.0f;
                 for (int c = 0; c < nc && ok; ++c) {
-                    bool fresh = false;  // this chunk opens a phase behind the grid barrier
                     if (!gated) {
                         // every CTA is past the previous phase: this phase's X is complete
                         if (w == 0) {
@@ -1390,19 +1400,20 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
                             __threadfence();
                         }
                         gated = true;
-                        fresh = true;
                     }
-                    // nobody reads this table buffer any more (with two buffers the barrier
-                    // after the previous chunk's build already ensures it) and, after a
-                    // grid barrier, every warp may read the new X
-                    if ((C::kTB == 1 || fresh) && !(ok = csync())) break;
-                    const uint32_t tb0 = tabs + (uint32_t)((nt++ % C::kTB) * MT * kCTok);
-                    const int nsl = chunk_slices(pr, c);
+                    // nobody reads the tables any more and, after a grid barrier, every warp
+                    // may read the new X
+                    if (!(ok = csync())) break;
+                    const uint32_t tb0 = tabs;
+                    const int nsl = chunk_slices<MT>(pr, c);
                     if (!have_x) load_x(pr, c);
-                    if (t < 32 * nsl) {
 #pragma unroll
-                        for (int m = 0; m < MT; ++m) build_table(tb0 + m * kCTok + t * kTab, xn[m]);
-                    }
+                    for (int u = 0; u < C::kTPT; ++u)
+                        if (t + kSRows * u < 32 * nsl) {
+#pragma unroll
+                            for (int m = 0; m < MT; ++m)
+                                build_table(tb0 + m * C::kTok + (t + kSRows * u) * kTab, xn[u][m]);
+                        }
                     // the next chunk's activations load while this one is looked up: the next
                     // chunk of this linear, or the first of the CTA's next segment in this phase
                     // (its X is complete too)
@@ -1419,25 +1430,31 @@ __global__ void __launch_bounds__(kSThreads, 1) k_lut_rows(const __grid_constant
                         if (i < sg.n) {
                             const int s = k % S;
                             if (!(ok = mbar_wait_sleep(ready(s), (uint32_t)((k / S) & 1), abort_flag, P.wait_cycles))) break;
-                            if (w < nsl) {
-                                const uint32_t st = stages + s * kCStage;
-                                const uint4 wq = lds128(st + r * (16 * kCSl) + (((uint32_t)w ^ (uint32_t)(r & 7)) << 4));
-                                const uint32_t sq = lds32(st + kCIdx + r * kCPad + 4 * w);
-                                const uint32_t tb = tb0 + (uint32_t)(w * 32 * kTab);
-                                float p0[MT], p1[MT], q0[MT], q1[MT], r0[MT], r1[MT], u0[MT], u1[MT];
-                                word_sums<0, MT, kCTok>(wq.x, sq & 0xffu, tb, p0, p1);
-                                word_sums<8, MT, kCTok>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
-                                word_sums<16, MT, kCTok>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
-                                word_sums<24, MT, kCTok>(wq.w, sq >> 24, tb, u0, u1);
-                                float al = 1.0f;
-                                if (pr.mode == kSG128) al = __uint_as_float(lds32(st + kCIdx + kCSgn + r * kCPad + 4 * w));
-                                if (pr.mode == kSG256)
-                                    al = __uint_as_float(lds32(st + kCIdx + kCSgn + r * kCPad + 4 * (w >> 1)));
+                            const uint32_t st = stages + s * C::kStage;
 #pragma unroll
-                                for (int m = 0; m < MT; ++m) {
-                                    const float v =
-                                        ((p0[m] + p1[m]) + (q0[m] + q1[m])) + ((r0[m] + r1[m]) + (u0[m] + u1[m]));
-                                    acc[i][m] = pr.mode == kSRow ? acc[i][m] + v : fmaf(al, v, acc[i][m]);
+                            for (int h = 0; h < C::kSl; h += kSConsumers) {
+                                const int sl = w + h;  // this warp's slice
+                                if (sl < nsl) {
+                                    const uint4 wq = lds128(st + r * (16 * C::kSl) +
+                                                            (((uint32_t)sl ^ (uint32_t)(r & 7)) << 4));
+                                    const uint32_t sq = lds32(st + C::kIdx + r * C::kPad + 4 * sl);
+                                    const uint32_t tb = tb0 + (uint32_t)(sl * 32 * kTab);
+                                    float p0[MT], p1[MT], q0[MT], q1[MT], r0[MT], r1[MT], u0[MT], u1[MT];
+                                    word_sums<0, MT, C::kTok>(wq.x, sq & 0xffu, tb, p0, p1);
+                                    word_sums<8, MT, C::kTok>(wq.y, (sq >> 8) & 0xffu, tb, q0, q1);
+                                    word_sums<16, MT, C::kTok>(wq.z, (sq >> 16) & 0xffu, tb, r0, r1);
+                                    word_sums<24, MT, C::kTok>(wq.w, sq >> 24, tb, u0, u1);
+                                    float al = 1.0f;
+                                    if (pr.mode == kSG128)
+                                        al = __uint_as_float(lds32(st + C::kIdx + C::kSgn + r * C::kPad + 4 * sl));
+                                    if (pr.mode == kSG256)
+                                        al = __uint_as_float(lds32(st + C::kIdx + C::kSgn + r * C::kPad + 4 * (sl >> 1)));
+#pragma unroll
+                                    for (int m = 0; m < MT; ++m) {
+                                        const float v =
+                                            ((p0[m] + p1[m]) + (q0[m] + q1[m])) + ((r0[m] + r1[m]) + (u0[m] + u1[m]));
+                                        acc[i][m] = pr.mode == kSRow ? acc[i][m] + v : fmaf(al, v, acc[i][m]);
+                                    }
                                 }
                             }
                             __syncwarp();
