@@ -1158,7 +1158,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_mma_stream(const __grid_consta
 // current segment (up to kCSeg items of one linear), so the tables are built once
 // per segment, not per item, and a K of 3072 is one chunk.  Four
 // helper warps copy the items' packed words (row-major, XOR-swizzled 16-byte
-// chunks), sign words and scales (rows padded to 80 bytes) with 16-byte copies
+// chunks), sign words and scales (rows padded by 16 bytes) with 16-byte copies
 // into a ring of stages; they run ahead across phases, since weights do not
 // depend on X.  Each phase's items are split into contiguous, balanced ranges over
 // the CTAs; a CTA arrives at the phase counter after its Y stores (release) and
